@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark of the Bloom-filtered int8 IVF top-k search on B200.
+
+One step = one st_search call (probe -> plan -> scan -> final top-k) over one
+batch of queries, inputs resident in HBM. Default workload: 80M items, d=64,
+16384 Zipf(0.8)-skewed lists, 128-bit signatures, B=64 queries, nprobe=64,
+k=2048. The timed steps cycle through a pool of distinct query batches; the
+index (6.4 GB) is far larger than L2.
+
+Prints one JSON line (rank 0). `--impl reference` times the CPU oracle instead
+(the reference arm; host cores only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, generate  # noqa: E402
+
+METRIC = "queries/s & item-scores/s (80M int8 IVF, nprobe64, top-2048); % HBM roofline"
+KERNELS_PER_SEARCH = 5   # probe, plan, expand, scan, select
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="ivf_80m", choices=sorted(WORKLOADS))
+    p.add_argument("--batch", type=int, default=None, help="queries per step (default: workload B)")
+    p.add_argument("--pool", type=int, default=8, help="distinct query batches cycled by the steps")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allreduce_max(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_sum(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def make_data(args, world, rank):
+    wl = WORKLOADS[args.workload]
+    B = args.batch or wl.B
+    pool = max(1, args.pool)
+    # every rank builds the same index; each draws its own query batches
+    total_q = B * pool * world
+    data = generate(wl.with_(B=total_q), device="cuda")
+    q = data.queries[rank * B * pool:(rank + 1) * B * pool].reshape(pool, B, -1).contiguous()
+    m = data.masks[rank * B * pool:(rank + 1) * B * pool].reshape(pool, B, -1).contiguous()
+    return wl.with_(B=B), data, q, m
+
+
+def byte_model(data, probe, qmasks, W, d):
+    """Algorithmic bytes of one search's list scan: 8W bytes of signature for
+    every row of every distinct probed list, plus d bytes for every row that is
+    eligible for at least one query probing its list. Also the full-scan bytes
+    (every row of every distinct probed list)."""
+    off = data.offsets
+    sizes = (off[1:] - off[:-1])
+    lists = torch.unique(probe.flatten())
+    scanned = int(sizes[lists].sum())
+    surv = torch.zeros(data.items.shape[0], dtype=torch.bool, device=off.device)
+    for b in range(probe.shape[0]):
+        ls = probe[b].long()
+        starts, lens = off[ls], sizes[ls]
+        idx = torch.repeat_interleave(starts - torch.cumsum(lens, 0) + lens, lens) + torch.arange(
+            int(lens.sum()), device=off.device)
+        s = data.sigs[idx]
+        mk = qmasks[b].view(1, -1)
+        ok = torch.all((s & mk) == mk, dim=1)
+        surv[idx[ok]] = True
+    n_surv = int(surv.sum())
+    method = 8 * W * scanned + d * n_surv
+    full = (8 * W + d) * scanned
+    return method, full, scanned, n_surv, int(lists.numel())
+
+
+def cpu_baseline(data, q, m, wl, budget_s):
+    import oracle
+    from workloads import to_numpy
+    a = to_numpy(data)
+    qs = q.reshape(-1, q.shape[-1]).cpu().numpy()
+    ms = m.reshape(-1, m.shape[-1]).cpu().numpy().view(np.uint64)
+    cores = oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.search(a["items"], a["sigs"], a["offsets"], a["centroids"], qs, ms, wl.nprobe, wl.k,
+                  b0=0, b1=min(cores, qs.shape[0]), nthreads=cores)
+    t1 = time.perf_counter()
+    per_round = max(t1 - t0, 1e-3)
+    rounds = max(1, min(int(budget_s / per_round), qs.shape[0] // cores))
+    nq = min(qs.shape[0], rounds * cores)
+    t0 = time.perf_counter()
+    oracle.search(a["items"], a["sigs"], a["offsets"], a["centroids"], qs, ms, wl.nprobe, wl.k,
+                  b0=0, b1=nq, nthreads=cores)
+    dt = time.perf_counter() - t0
+    return {"value": nq / dt, "unit": "queries/s", "cores": cores, "kind": "oracle",
+            "sample": f"{nq} queries of the timed workload, OpenMP over queries on {cores} host threads, {dt:.2f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from workloads import to_numpy
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    wl, data, q, m = make_data(args, 1, 0)
+    a = to_numpy(data)
+    del data
+    torch.cuda.empty_cache()
+    qs = q.reshape(-1, q.shape[-1]).cpu().numpy()
+    ms = m.reshape(-1, m.shape[-1]).cpu().numpy().view(np.uint64)
+    cores = oracle.max_threads()
+    nq_total = qs.shape[0]
+
+    def step(i):
+        b0 = (i * cores) % nq_total
+        b1 = min(nq_total, b0 + cores)
+        oracle.search(a["items"], a["sigs"], a["offsets"], a["centroids"], qs, ms, wl.nprobe, wl.k,
+                      b0=b0, b1=b1, nthreads=cores)
+        return b1 - b0
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    done = 0
+    for i in range(args.steps):
+        done += step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    v = done / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/int32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "n": wl.n, "d": wl.d, "nlist": wl.nlist, "B": wl.B,
+                   "nprobe": wl.nprobe, "k": wl.k, "sig_bits": wl.sig_bits,
+                   "note": "CPU oracle, each step one query per host thread"},
+        "cpu_baseline": {"value": v, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{done} queries over {args.steps} steps of {cores} queries"},
+        "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    world, rank, local = dist_setup(args)
+    import filtered_int8_ann_b200 as st
+
+    wl, data, q, m = make_data(args, world, rank)
+    B, P, k, d, W = wl.B, wl.nprobe, wl.k, wl.d, wl.W
+    pool = q.shape[0]
+    idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
+    dev = torch.device("cuda", local)
+    ids = torch.empty((B, k), dtype=torch.int64, device=dev)
+    scores = torch.empty((B, k), dtype=torch.int32, device=dev)
+
+    # per-batch eligible counts and byte model (untimed)
+    elig = torch.empty((pool, B), dtype=torch.int64, device=dev)
+    probe = torch.empty((pool, B, P), dtype=torch.int32, device=dev)
+    for b in range(pool):
+        idx.search(q[b], m[b], P, k, out_ids=ids, out_scores=scores, eligible=elig[b], probe=probe[b])
+    assert idx.check() == st.ST_OK
+    models = [byte_model(data, probe[b], m[b], W, d) for b in range(pool)]
+    elig_per_batch = elig.sum(1).double().cpu().numpy()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(data, q, m, wl, args.cpu_seconds)
+    del data
+    torch.cuda.empty_cache()
+
+    # warm-up
+    for i in range(args.warmup):
+        idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(K):
+        idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores, stage_events=evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    assert idx.check() == st.ST_OK
+    ms_local = start.elapsed_time(end)
+    ms = allreduce_max(ms_local, world)
+
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(K)])
+    stage_mean = stage_ms.mean(0)
+    scan_ms = stage_mean[2]
+    method_bytes = np.array([models[i % pool][0] for i in range(K)], dtype=np.float64)
+    full_bytes = np.array([models[i % pool][1] for i in range(K)], dtype=np.float64)
+    scan_gbs = float(method_bytes.sum() / (stage_ms[:, 2].sum() * 1e-3) / 1e9)
+    peak, peak_kind = peaks()
+
+    total_q = allreduce_sum(float(B * K), world)
+    elig_total = allreduce_sum(float(sum(elig_per_batch[i % pool] for i in range(K))), world)
+    value = total_q / (ms * 1e-3)
+
+    # end to end through the host-buffer entry point (pinned memory)
+    Ke = min(K, 200)
+    hq = [q[b].cpu().pin_memory() for b in range(pool)]
+    hm = [m[b].cpu().pin_memory() for b in range(pool)]
+    hids = torch.empty((B, k), dtype=torch.int64).pin_memory()
+    hsc = torch.empty((B, k), dtype=torch.int32).pin_memory()
+    for i in range(3):
+        idx.search_host(hq[i % pool], hm[i % pool], P, k, out_ids=hids, out_scores=hsc)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(Ke):
+        idx.search_host(hq[i % pool], hm[i % pool], P, k, out_ids=hids, out_scores=hsc)
+    e1.record()
+    torch.cuda.synchronize()
+    ems = allreduce_max(e0.elapsed_time(e1), world)
+    e2e = allreduce_sum(float(B * Ke), world) / (ems * 1e-3)
+    idx.close()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8/int32", "data": "synthetic",
+            "config": {"workload": wl.name, "n": wl.n, "d": d, "nlist": wl.nlist, "B": B, "nprobe": P,
+                       "k": k, "sig_bits": wl.sig_bits, "mask_mode": "head",
+                       "l2": f"inputs larger than L2 (index {wl.n * (d + 8 * W) / 1e9:.1f} GB); steps cycle {pool} distinct query batches",
+                       "parallelism": f"replicas x{world} (independent query batches)"},
+            "item_scores_per_s": elig_total / (ms * 1e-3),
+            "stage_ms": {"probe": stage_mean[0], "plan": stage_mean[1], "scan": stage_mean[2],
+                         "select": stage_mean[3]},
+            "roofline": {"bound": "hbm", "kernel": "scan_kernel", "achieved": scan_gbs, "peak": peak,
+                         "unit": "GB/s", "frac": scan_gbs / peak, "traffic": None,
+                         "peak_kind": peak_kind,
+                         "bytes_per_launch": float(method_bytes.mean()),
+                         "full_scan_bytes_per_launch": float(full_bytes.mean()),
+                         "step_frac": float(method_bytes.mean() / (ms / K * 1e-3) / 1e9 / peak)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e, "unit": "queries/s", "h2d_bytes_per_step": B * (d + 8 * W),
+                    "d2h_bytes_per_step": B * k * 12},
+            "gpu_launches": KERNELS_PER_SEARCH * K,
+            "clocks": clk,
+            "workload_stats": {"scanned_items": float(np.mean([x[2] for x in models])),
+                               "survivor_rows": float(np.mean([x[3] for x in models])),
+                               "distinct_lists": float(np.mean([x[4] for x in models])),
+                               "eligible_per_query": float(elig_per_batch.mean() / B)},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

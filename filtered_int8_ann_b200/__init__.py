@@ -1,0 +1,205 @@
+"""Python binding of libst.so, the Bloom-filtered int8 IVF top-k search library.
+
+Argument marshalling only: every step of a search runs in the library's CUDA
+kernels. The functions keep the C names of include/st.h; torch tensors supply
+device memory and torch streams supply the CUDA stream. Loading fails loudly
+when libst.so has not been built (python -m filtered_int8_ann_b200.build):
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libst.so")
+
+ST_OK, ST_ERR_INVALID_ARG, ST_ERR_UNSUPPORTED, ST_ERR_OOM, ST_ERR_CUDA, ST_ERR_DEVICE = range(6)
+ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY = 1, 2
+ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE = 512, 4096, 4096
+
+# Every symbol include/st.h declares.
+EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
+           "st_index_set_option", "st_index_destroy", "st_status_string")
+
+
+class StError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class _Extras(ctypes.Structure):
+    _fields_ = [("eligible", ctypes.c_void_p), ("probe", ctypes.c_void_p),
+                ("stage_events", ctypes.c_void_p * 5)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m filtered_int8_ann_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    L.st_index_create.argtypes = [P, P, P, P, i64, i32, i32, i32, P, ctypes.POINTER(P)]
+    L.st_search.argtypes = [P, P, P, i32, i32, i32, P, P, P]
+    L.st_search_ex.argtypes = [P, P, P, i32, i32, i32, P, P, ctypes.POINTER(_Extras), P]
+    L.st_search_host.argtypes = [P, P, P, i32, i32, i32, P, P, P]
+    L.st_index_check.argtypes = [P, P]
+    L.st_index_set_option.argtypes = [P, ctypes.c_int, i64]
+    for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
+              "st_index_set_option"):
+        getattr(L, f).restype = ctypes.c_int
+    L.st_index_destroy.argtypes = [P]
+    L.st_index_destroy.restype = None
+    L.st_status_string.argtypes = [ctypes.c_int]
+    L.st_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().st_status_string(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != ST_OK:
+        raise StError(status, what)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return t.data_ptr()
+    return int(t)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _as_words(t: torch.Tensor) -> torch.Tensor:
+    """Signatures / masks as int64 words [rows, W] (bit patterns of uint64)."""
+    if t.dtype == torch.uint64:
+        t = t.view(torch.int64)
+    assert t.dtype == torch.int64, "signatures and masks are 64-bit words"
+    return t if t.dim() == 2 else t.reshape(-1, 1)
+
+
+def st_index_create(items: torch.Tensor, sigs: torch.Tensor, list_offsets: torch.Tensor,
+                    centroids: torch.Tensor, stream=None) -> int:
+    """Build an index from int8 items [n,d], signature words [n,W], int64 offsets
+    [nlist+1] and int8 centroids [nlist,d]; returns the opaque handle."""
+    sigs = _as_words(sigs).contiguous()
+    items, list_offsets, centroids = items.contiguous(), list_offsets.contiguous(), centroids.contiguous()
+    assert items.dtype == torch.int8 and centroids.dtype == torch.int8 and list_offsets.dtype == torch.int64
+    n, d = items.shape
+    h = ctypes.c_void_p()
+    _check(lib().st_index_create(_ptr(items), _ptr(sigs), _ptr(list_offsets), _ptr(centroids), n, d,
+                                 centroids.shape[0], sigs.shape[1], _stream(stream), ctypes.byref(h)),
+           "st_index_create")
+    return h.value
+
+
+def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: int, k: int,
+              out_ids: Optional[torch.Tensor] = None, out_scores: Optional[torch.Tensor] = None,
+              stream=None, eligible: Optional[torch.Tensor] = None,
+              probe: Optional[torch.Tensor] = None, stage_events=None):
+    """Asynchronous search of device-resident queries; returns (ids int64 [B,k],
+    scores int32 [B,k]). `eligible` [B] int64 and `probe` [B,nprobe] int32 are
+    optional extra outputs; `stage_events` is a list of up to five recorded
+    torch.cuda.Event objects marking the stage boundaries (st_search_ex)."""
+    qmasks = _as_words(qmasks)
+    B = queries.shape[0]
+    dev = queries.device
+    if out_ids is None:
+        out_ids = torch.empty((B, k), dtype=torch.int64, device=dev)
+    if out_scores is None:
+        out_scores = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if eligible is None and probe is None and not stage_events:
+        st = lib().st_search(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
+                             _ptr(out_scores), _stream(stream))
+        _check(st, "st_search")
+    else:
+        ex = _Extras(_ptr(eligible), _ptr(probe))
+        for i, ev in enumerate(stage_events or ()):
+            ex.stage_events[i] = ev.cuda_event if ev is not None else None
+        st = lib().st_search_ex(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
+                                _ptr(out_scores), ctypes.byref(ex), _stream(stream))
+        _check(st, "st_search_ex")
+    return out_ids, out_scores
+
+
+def st_search_host(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: int, k: int,
+                   out_ids: Optional[torch.Tensor] = None, out_scores: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Search host-resident (ideally pinned) queries; results land in host
+    tensors and are ready when the call returns."""
+    qmasks = _as_words(qmasks)
+    assert queries.device.type == "cpu" and qmasks.device.type == "cpu"
+    B = queries.shape[0]
+    if out_ids is None:
+        out_ids = torch.empty((B, k), dtype=torch.int64)
+    if out_scores is None:
+        out_scores = torch.empty((B, k), dtype=torch.int32)
+    _check(lib().st_search_host(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
+                                _ptr(out_scores), _stream(stream)), "st_search_host")
+    return out_ids, out_scores
+
+
+def st_index_check(index: int, stream=None) -> int:
+    """Synchronize and return the device-side status (ST_OK or ST_ERR_DEVICE)."""
+    return lib().st_index_check(index, _stream(stream))
+
+
+def st_index_set_option(index: int, option: int, value: int):
+    _check(lib().st_index_set_option(index, option, value), "st_index_set_option")
+
+
+def st_index_destroy(index: Optional[int]):
+    if index:
+        lib().st_index_destroy(index)
+
+
+class Index:
+    """Owning wrapper: builds on construction, frees on close()/GC."""
+
+    def __init__(self, items, sigs, list_offsets, centroids, stream=None):
+        self.handle = st_index_create(items, sigs, list_offsets, centroids, stream)
+        self.d = items.shape[1]
+        self.nlist = centroids.shape[0]
+
+    def search(self, queries, qmasks, nprobe, k, **kw):
+        return st_search(self.handle, queries, qmasks, nprobe, k, **kw)
+
+    def search_host(self, queries, qmasks, nprobe, k, **kw):
+        return st_search_host(self.handle, queries, qmasks, nprobe, k, **kw)
+
+    def check(self, stream=None) -> int:
+        return st_index_check(self.handle, stream)
+
+    def set_option(self, option, value):
+        st_index_set_option(self.handle, option, value)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            st_index_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,431 @@
+// Host side of the C ABI declared in include/st.h: argument validation, the
+// library-owned index copy, stream-ordered scratch, and the kernel sequence
+// probe -> plan -> expand -> scan -> select of one search.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "st_internal.cuh"
+
+struct st_index {
+    int device = 0;
+    int num_sms = 0;
+    int64_t n = 0;
+    int32_t d = 0, nlist = 0, W = 0;
+    int8_t* items = nullptr;
+    uint64_t* sigs = nullptr;
+    int64_t* offsets = nullptr;
+    int8_t* centroids = nullptr;
+    uint32_t* err = nullptr;
+    std::vector<int64_t> top_prefix;  // [p] = rows in the p largest lists
+    cudaMemPool_t pool = nullptr;
+    int64_t cand_bytes = int64_t(2) << 30;
+    int64_t cand_cap_override = 0;
+};
+
+namespace st {
+
+cudaError_t ensure_smem_attr(const void* func, int slot)
+{
+    static unsigned done[64] = {0};  // bit `slot` set once per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && slot < 32 && (done[dev] >> slot) & 1u) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess && dev < 64 && slot < 32) __atomic_fetch_or(&done[dev], 1u << slot, __ATOMIC_RELAXED);
+    return e;
+}
+
+}  // namespace st
+
+namespace {
+
+using st::SearchArgs;
+
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev)
+    {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard()
+    {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+bool is_device_ptr(const void* p, int device)
+{
+    if (p == nullptr) return false;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (attr.type == cudaMemoryTypeManaged) return true;
+    return attr.type == cudaMemoryTypeDevice && attr.device == device;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+st_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return ST_OK;
+    if (e == cudaErrorMemoryAllocation) return ST_ERR_OOM;
+    return ST_ERR_CUDA;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Carves one scratch allocation into the per-search arrays.
+struct ScratchLayout {
+    size_t total = 0;
+    size_t off_probe, off_probe_keys, off_list_cnt, off_list_qstart, off_list_fill, off_qlist,
+        off_dl_list, off_dl_qstart, off_dl_qcnt, off_dl_ustart, off_units, off_ctl, off_cand_cnt,
+        off_elig, off_cand;
+    size_t add(size_t bytes)
+    {
+        const size_t o = total;
+        total = align_up(total + bytes, 256);
+        return o;
+    }
+};
+
+int64_t candidate_capacity(const st_index* idx, int32_t B, int32_t P, int32_t k)
+{
+    int64_t cap = idx->top_prefix[std::min<int64_t>(P, idx->nlist)];
+    const int64_t budget = idx->cand_bytes / 8 / B;
+    if (cap > budget) cap = budget;
+    if (idx->cand_cap_override > 0) cap = idx->cand_cap_override;
+    const int64_t floor_cap = int64_t(k) + st::kSelectBlock;
+    if (cap < floor_cap) cap = floor_cap;
+    return cap;
+}
+
+int64_t max_units_bound(const st_index* idx, int32_t B, int32_t P)
+{
+    const int64_t W = st::kWarpItems;
+    const int64_t groups = (B + st::kQMax - 1) / st::kQMax;
+    const int64_t lists = std::min<int64_t>(idx->nlist, int64_t(B) * P);
+    const int64_t b1 = ((idx->n + W - 1) / W + lists) * groups;
+    const int64_t topP = idx->top_prefix[std::min<int64_t>(P, idx->nlist)];
+    const int64_t b2 = int64_t(B) * ((topP + W - 1) / W + P);
+    return std::min(b1, b2);
+}
+
+st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
+                      int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                      const st_search_extras* extras, cudaStream_t stream)
+{
+    const int64_t cap = candidate_capacity(idx, B, nprobe, k);
+    const int64_t max_units = max_units_bound(idx, B, nprobe);
+    if (max_units >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
+    const int64_t ndl = std::min<int64_t>(idx->nlist, int64_t(B) * nprobe);
+    const bool probe_in_smem = idx->nlist <= st::kProbeSmemKeys;
+
+    ScratchLayout L;
+    L.off_probe = L.add(size_t(B) * nprobe * 4);
+    L.off_probe_keys = probe_in_smem ? 0 : L.add(size_t(B) * idx->nlist * 8);
+    L.off_list_cnt = L.add(size_t(idx->nlist) * 4);
+    L.off_list_qstart = L.add(size_t(idx->nlist) * 4);
+    L.off_list_fill = L.add(size_t(idx->nlist) * 4);
+    L.off_qlist = L.add(size_t(B) * nprobe * 4);
+    L.off_dl_list = L.add(size_t(ndl) * 4);
+    L.off_dl_qstart = L.add(size_t(ndl) * 4);
+    L.off_dl_qcnt = L.add(size_t(ndl) * 4);
+    L.off_dl_ustart = L.add(size_t(ndl + 1) * 4);
+    L.off_units = L.add(size_t(max_units) * 16);
+    L.off_ctl = L.add(sizeof(st::PlanCtl));
+    L.off_cand_cnt = L.add(size_t(B) * 4);
+    L.off_elig = L.add(size_t(B) * 8);
+    L.off_cand = L.add(size_t(B) * size_t(cap) * 8);
+
+    unsigned char* base = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&base), L.total, idx->pool, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e == cudaErrorMemoryAllocation ? ST_ERR_OOM : ST_ERR_CUDA;
+    }
+
+    SearchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.items = idx->items;
+    a.sigs = idx->sigs;
+    a.offsets = idx->offsets;
+    a.centroids = idx->centroids;
+    a.d = idx->d;
+    a.nlist = idx->nlist;
+    a.W = idx->W;
+    a.queries = queries;
+    a.qmasks = qmasks;
+    a.B = B;
+    a.P = nprobe;
+    a.k = k;
+    a.out_ids = out_ids;
+    a.out_scores = out_scores;
+    a.out_eligible = extras ? extras->eligible : nullptr;
+    a.probe = reinterpret_cast<int32_t*>(base + L.off_probe);
+    a.probe_keys = probe_in_smem ? nullptr : reinterpret_cast<uint64_t*>(base + L.off_probe_keys);
+    a.list_cnt = reinterpret_cast<int32_t*>(base + L.off_list_cnt);
+    a.list_qstart = reinterpret_cast<int32_t*>(base + L.off_list_qstart);
+    a.list_fill = reinterpret_cast<int32_t*>(base + L.off_list_fill);
+    a.qlist = reinterpret_cast<int32_t*>(base + L.off_qlist);
+    a.dl_list = reinterpret_cast<int32_t*>(base + L.off_dl_list);
+    a.dl_qstart = reinterpret_cast<int32_t*>(base + L.off_dl_qstart);
+    a.dl_qcnt = reinterpret_cast<int32_t*>(base + L.off_dl_qcnt);
+    a.dl_ustart = reinterpret_cast<int32_t*>(base + L.off_dl_ustart);
+    a.units = reinterpret_cast<int4*>(base + L.off_units);
+    a.max_units = int32_t(max_units);
+    a.ctl = reinterpret_cast<st::PlanCtl*>(base + L.off_ctl);
+    a.cand_cnt = reinterpret_cast<uint32_t*>(base + L.off_cand_cnt);
+    a.eligible_cnt = reinterpret_cast<unsigned long long*>(base + L.off_elig);
+    a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
+    a.cap = cap;
+    a.err = idx->err;
+
+    auto mark = [&](int i) {
+        if (e == cudaSuccess && extras && extras->stage_events[i]) e = cudaEventRecord(extras->stage_events[i], stream);
+    };
+    e = cudaSuccess;
+    mark(0);
+    if (e == cudaSuccess) e = st::launch_probe(a, stream);
+    mark(1);
+    if (e == cudaSuccess) e = st::launch_plan(a, idx->num_sms, stream);
+    mark(2);
+    if (e == cudaSuccess) e = st::launch_scan(a, idx->num_sms, stream);
+    mark(3);
+    if (e == cudaSuccess) e = st::launch_select(a, stream);
+    mark(4);
+    if (e == cudaSuccess && extras && extras->probe)
+        e = cudaMemcpyAsync(extras->probe, a.probe, size_t(B) * nprobe * 4, cudaMemcpyDeviceToDevice, stream);
+    cudaError_t ef = cudaFreeAsync(base, stream);
+    if (e == cudaSuccess) e = ef;
+    return cuda_status(e);
+}
+
+st_status check_search_args(const st_index* idx, int32_t B, int32_t nprobe, int32_t k)
+{
+    if (idx == nullptr) return ST_ERR_INVALID_ARG;
+    if (B < 1 || k < 1 || nprobe < 1 || nprobe > idx->nlist) return ST_ERR_INVALID_ARG;
+    if (k > ST_MAX_K || nprobe > ST_MAX_NPROBE) return ST_ERR_UNSUPPORTED;
+    if (int64_t(B) * nprobe >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
+    return ST_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* st_status_string(st_status s)
+{
+    switch (s) {
+    case ST_OK: return "ok";
+    case ST_ERR_INVALID_ARG: return "invalid argument";
+    case ST_ERR_UNSUPPORTED: return "unsupported size";
+    case ST_ERR_OOM: return "out of device memory";
+    case ST_ERR_CUDA: return "CUDA error";
+    case ST_ERR_DEVICE: return "device-side error recorded by a kernel";
+    }
+    return "unknown status";
+}
+
+st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64_t* list_offsets,
+                          const int8_t* centroids, int64_t n, int32_t d, int32_t nlist,
+                          int32_t sig_words, cudaStream_t stream, st_index** out)
+{
+    if (out == nullptr) return ST_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!items || !sigs || !list_offsets || !centroids) return ST_ERR_INVALID_ARG;
+    if (n < 1 || nlist < 1 || d < 1) return ST_ERR_INVALID_ARG;
+    if (d % 16 != 0 || d > ST_MAX_D || (sig_words != 1 && sig_words != 2)) return ST_ERR_UNSUPPORTED;
+    if (n >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
+
+    st_index* idx = new (std::nothrow) st_index();
+    if (!idx) return ST_ERR_OOM;
+    auto fail = [&](st_status s) {
+        st_index_destroy(idx);
+        return s;
+    };
+    cudaError_t e = cudaGetDevice(&idx->device);
+    if (e != cudaSuccess) return fail(ST_ERR_CUDA);
+    e = cudaDeviceGetAttribute(&idx->num_sms, cudaDevAttrMultiProcessorCount, idx->device);
+    if (e != cudaSuccess) return fail(ST_ERR_CUDA);
+    idx->n = n;
+    idx->d = d;
+    idx->nlist = nlist;
+    idx->W = sig_words;
+
+    // offsets: validate on the host
+    std::vector<int64_t> off(size_t(nlist) + 1);
+    e = cudaMemcpyAsync(off.data(), list_offsets, off.size() * 8, cudaMemcpyDefault, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(ST_ERR_INVALID_ARG);
+    }
+    if (off[0] != 0 || off[nlist] != n) return fail(ST_ERR_INVALID_ARG);
+    std::vector<int64_t> sizes(nlist);
+    for (int32_t c = 0; c < nlist; ++c) {
+        if (off[c + 1] < off[c]) return fail(ST_ERR_INVALID_ARG);
+        sizes[c] = off[c + 1] - off[c];
+    }
+    std::sort(sizes.begin(), sizes.end(), std::greater<int64_t>());
+    idx->top_prefix.assign(size_t(nlist) + 1, 0);
+    for (int32_t c = 0; c < nlist; ++c) idx->top_prefix[c + 1] = idx->top_prefix[c] + sizes[c];
+
+    // library-owned copies (a little slack past the end of the row arrays)
+    const size_t items_bytes = size_t(n) * d, sig_bytes = size_t(n) * sig_words * 8;
+    if (cudaMalloc(&idx->items, items_bytes + 256) != cudaSuccess ||
+        cudaMalloc(&idx->sigs, sig_bytes + 256) != cudaSuccess ||
+        cudaMalloc(&idx->offsets, off.size() * 8) != cudaSuccess ||
+        cudaMalloc(&idx->centroids, size_t(nlist) * d + 256) != cudaSuccess ||
+        cudaMalloc(&idx->err, 256) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(ST_ERR_OOM);
+    }
+    e = cudaMemcpyAsync(idx->items, items, items_bytes, cudaMemcpyDefault, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(idx->sigs, sigs, sig_bytes, cudaMemcpyDefault, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(idx->offsets, off.data(), off.size() * 8, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(idx->centroids, centroids, size_t(nlist) * d, cudaMemcpyDefault, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(idx->err, 0, 256, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(e == cudaErrorInvalidValue ? ST_ERR_INVALID_ARG : ST_ERR_CUDA);
+    }
+
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = idx->device;
+    if (cudaMemPoolCreate(&idx->pool, &props) != cudaSuccess) {
+        cudaGetLastError();
+        idx->pool = nullptr;
+        return fail(ST_ERR_CUDA);
+    }
+    uint64_t keep = ~uint64_t(0);
+    cudaMemPoolSetAttribute(idx->pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    *out = idx;
+    return ST_OK;
+}
+
+st_status st_search_ex(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
+                       int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                       const st_search_extras* extras, cudaStream_t stream)
+{
+    st_status s = check_search_args(idx, B, nprobe, k);
+    if (s != ST_OK) return s;
+    DeviceGuard g(idx->device);
+    if (!is_device_ptr(queries, idx->device) || !is_device_ptr(qmasks, idx->device) ||
+        !is_device_ptr(out_ids, idx->device) || !is_device_ptr(out_scores, idx->device))
+        return ST_ERR_INVALID_ARG;
+    if (!aligned(queries, 16) || !aligned(qmasks, 8) || !aligned(out_ids, 8) || !aligned(out_scores, 4))
+        return ST_ERR_INVALID_ARG;
+    if (extras) {
+        if (extras->eligible && (!is_device_ptr(extras->eligible, idx->device) || !aligned(extras->eligible, 8)))
+            return ST_ERR_INVALID_ARG;
+        if (extras->probe && (!is_device_ptr(extras->probe, idx->device) || !aligned(extras->probe, 4)))
+            return ST_ERR_INVALID_ARG;
+    }
+    return search_impl(idx, queries, qmasks, B, nprobe, k, out_ids, out_scores, extras, stream);
+}
+
+st_status st_search(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
+                    int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores, cudaStream_t stream)
+{
+    return st_search_ex(idx, queries, qmasks, B, nprobe, k, out_ids, out_scores, nullptr, stream);
+}
+
+st_status st_search_host(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
+                         int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                         cudaStream_t stream)
+{
+    st_status s = check_search_args(idx, B, nprobe, k);
+    if (s != ST_OK) return s;
+    if (!queries || !qmasks || !out_ids || !out_scores) return ST_ERR_INVALID_ARG;
+    DeviceGuard g(idx->device);
+    const size_t qb = align_up(size_t(B) * idx->d, 256), mb = align_up(size_t(B) * idx->W * 8, 256);
+    const size_t ib = align_up(size_t(B) * k * 8, 256), sb = align_up(size_t(B) * k * 4, 256);
+    unsigned char* buf = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&buf), qb + mb + ib + sb, idx->pool, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e == cudaErrorMemoryAllocation ? ST_ERR_OOM : ST_ERR_CUDA;
+    }
+    int8_t* dq = reinterpret_cast<int8_t*>(buf);
+    uint64_t* dm = reinterpret_cast<uint64_t*>(buf + qb);
+    int64_t* dids = reinterpret_cast<int64_t*>(buf + qb + mb);
+    int32_t* dsc = reinterpret_cast<int32_t*>(buf + qb + mb + ib);
+    e = cudaMemcpyAsync(dq, queries, size_t(B) * idx->d, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dm, qmasks, size_t(B) * idx->W * 8, cudaMemcpyHostToDevice, stream);
+    st_status rs = ST_OK;
+    if (e == cudaSuccess) {
+        rs = search_impl(idx, dq, dm, B, nprobe, k, dids, dsc, nullptr, stream);
+        if (rs == ST_OK) {
+            e = cudaMemcpyAsync(out_ids, dids, size_t(B) * k * 8, cudaMemcpyDeviceToHost, stream);
+            if (e == cudaSuccess) e = cudaMemcpyAsync(out_scores, dsc, size_t(B) * k * 4, cudaMemcpyDeviceToHost, stream);
+        }
+    }
+    cudaError_t ef = cudaFreeAsync(buf, stream);
+    cudaError_t es = cudaStreamSynchronize(stream);
+    if (rs != ST_OK) return rs;
+    if (e == cudaSuccess) e = ef;
+    if (e == cudaSuccess) e = es;
+    return cuda_status(e);
+}
+
+st_status st_index_check(const st_index* idx, cudaStream_t stream)
+{
+    if (idx == nullptr) return ST_ERR_INVALID_ARG;
+    DeviceGuard g(idx->device);
+    uint32_t word = 0;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess) e = cudaMemcpy(&word, idx->err, 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return ST_ERR_CUDA;
+    if (word != 0) {
+        cudaMemset(idx->err, 0, 4);
+        return ST_ERR_DEVICE;
+    }
+    return ST_OK;
+}
+
+st_status st_index_set_option(st_index* idx, st_option opt, int64_t value)
+{
+    if (idx == nullptr || value < 0) return ST_ERR_INVALID_ARG;
+    switch (opt) {
+    case ST_OPT_CANDIDATE_BYTES:
+        idx->cand_bytes = value > 0 ? value : (int64_t(2) << 30);
+        return ST_OK;
+    case ST_OPT_CANDIDATE_CAPACITY:
+        idx->cand_cap_override = value;
+        return ST_OK;
+    }
+    return ST_ERR_INVALID_ARG;
+}
+
+void st_index_destroy(st_index* idx)
+{
+    if (idx == nullptr) return;
+    {
+        DeviceGuard g(idx->device);
+        cudaDeviceSynchronize();
+        cudaFree(idx->items);
+        cudaFree(idx->sigs);
+        cudaFree(idx->offsets);
+        cudaFree(idx->centroids);
+        cudaFree(idx->err);
+        if (idx->pool) cudaMemPoolDestroy(idx->pool);
+        cudaGetLastError();
+    }
+    delete idx;
+}
+
+}  // extern "C"

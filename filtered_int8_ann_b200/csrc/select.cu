@@ -1,0 +1,142 @@
+// Final top-k: one CTA per query picks the k best candidate keys and writes
+// them ordered by score descending, then item id ascending, padded with
+// (id -1, score INT32_MIN) when fewer than k items were eligible.
+//
+// "Top-2048 with 64 probes and no recall loss" / a large candidate pool --
+// SilverTorch: Index as Model, section on redesigning each stage as a pure
+// PyTorch module, fused Int8 ANN paragraph; maximum top-k row of the cost
+// efficiency table in the Spanish translation.
+//
+// The candidate keys of a query (written by the scan) are copied into shared
+// memory when they fit, an MSB-first radix select finds the k-th largest key,
+// the keys at or above it are gathered (exactly k: keys are unique) and a
+// bitonic network sorts them.
+//
+// Exact overflow path: when the scan emitted more candidates for a query than
+// its buffer holds (the count kept running past the capacity), this CTA
+// rescans that query's probed lists itself with a bounded buffer: whenever the
+// buffer fills it keeps only the k best keys and from then on drops any key
+// below the k-th, which can no longer enter the top-k. Exact for any input,
+// with memory bounded by the capacity; slow, and used only on overflow.
+#include "st_internal.cuh"
+
+namespace st {
+
+template <int BLOCK>
+__device__ int32_t select_into(const uint64_t* keys, int64_t n, int k, uint64_t* sortbuf, int pwk,
+                               SelectSmem& ss, uint32_t* err)
+{
+    int32_t got;
+    if (n > k) {
+        const uint64_t kth = block_kth_largest<BLOCK>(keys, n, k, ss);
+        got = block_collect_ge<BLOCK>(keys, n, kth, sortbuf, pwk, ss);
+        if (threadIdx.x == 0 && got != k) set_error(err, kErrSelectCount);
+    } else {
+        got = block_collect_ge<BLOCK>(keys, n, 1ull, sortbuf, pwk, ss);
+    }
+    if (got > pwk) got = pwk;
+    for (int i = got + threadIdx.x; i < pwk; i += BLOCK) sortbuf[i] = 0;
+    __syncthreads();
+    block_bitonic_desc<BLOCK>(sortbuf, pwk);
+    return got;
+}
+
+template <int BLOCK>
+__device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, int pwk, int4* s_qv,
+                              SelectSmem& ss)
+{
+    __shared__ int32_t s_count;
+    __shared__ uint64_t s_thr;
+    const int d = a.d, np = d >> 4, W = a.W, k = a.k;
+    uint64_t* buf = a.cand + int64_t(q) * a.cap;
+    const int64_t cap = a.cap;  // host guarantees cap >= k + BLOCK
+    for (int p = threadIdx.x; p < np; p += BLOCK)
+        s_qv[p] = reinterpret_cast<const int4*>(a.queries + int64_t(q) * d)[p];
+    const uint64_t m0 = a.qmasks[int64_t(q) * W];
+    const uint64_t m1 = W > 1 ? a.qmasks[int64_t(q) * W + 1] : 0ull;
+    if (threadIdx.x == 0) {
+        s_count = 0;
+        s_thr = 0;
+    }
+    __syncthreads();
+    for (int p = 0; p < a.P; ++p) {
+        const int L = a.probe[int64_t(q) * a.P + p];
+        if (L < 0 || L >= a.nlist) {
+            if (threadIdx.x == 0) set_error(a.err, kErrOverflowPath);
+            continue;
+        }
+        const int64_t o0 = a.offsets[L], o1 = a.offsets[L + 1];
+        for (int64_t base = o0; base < o1; base += BLOCK) {
+            if (int64_t(s_count) + BLOCK > cap) {
+                // keep the k best, raise the threshold to the k-th
+                const uint64_t kth = block_kth_largest<BLOCK>(buf, s_count, k, ss);
+                const int32_t got = block_collect_ge<BLOCK>(buf, s_count, kth, sortbuf, pwk, ss);
+                if (threadIdx.x == 0 && got != k) set_error(a.err, kErrOverflowPath);
+                for (int i = threadIdx.x; i < k; i += BLOCK) buf[i] = sortbuf[i];
+                if (threadIdx.x == 0) {
+                    s_count = k;
+                    s_thr = kth;
+                }
+                __syncthreads();
+            }
+            const int64_t i = base + threadIdx.x;
+            const uint64_t thr = s_thr;
+            if (i < o1) {
+                const uint64_t* sg = a.sigs + i * W;
+                bool pass = (sg[0] & m0) == m0;
+                if (W > 1) pass = pass && ((sg[1] & m1) == m1);
+                if (pass) {
+                    const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);
+                    int32_t acc = 0;
+                    for (int t = 0; t < np; ++t) acc = dot16(__ldg(rp + t), s_qv[t], acc);
+                    const uint64_t key = pack_key(acc, uint32_t(i));
+                    if (key > thr) buf[atomicAdd(&s_count, 1)] = key;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    return s_count;
+}
+
+template <int BLOCK>
+__global__ void __launch_bounds__(BLOCK)
+select_kernel(SearchArgs a)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ SelectSmem ss;
+    const int q = blockIdx.x;
+    const int k = a.k;
+    const int pwk = next_pow2(k);
+    uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* local = sortbuf + (pwk < 2 ? 2 : pwk);  // 16-byte aligned
+
+    const uint32_t cnt = a.cand_cnt[q];
+    const uint64_t* keys = a.cand + int64_t(q) * a.cap;
+    int64_t n = cnt;
+    if (n > a.cap) n = overflow_path<BLOCK>(a, q, sortbuf, pwk, reinterpret_cast<int4*>(local), ss);
+    if (n <= kSelectSmemKeys) {
+        for (int64_t i = threadIdx.x; i < n; i += BLOCK) local[i] = keys[i];
+        __syncthreads();
+        keys = local;
+    }
+    select_into<BLOCK>(keys, n, k, sortbuf, pwk, ss, a.err);
+    for (int r = threadIdx.x; r < k; r += BLOCK) {
+        const uint64_t key = sortbuf[r];
+        a.out_ids[int64_t(q) * k + r] = key_id(key);
+        a.out_scores[int64_t(q) * k + r] = key_score(key);
+    }
+    if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[q]);
+}
+
+cudaError_t launch_select(const SearchArgs& a, cudaStream_t s)
+{
+    const int pwk = next_pow2(a.k);
+    const size_t smem = size_t(pwk < 2 ? 2 : pwk) * 8 + size_t(kSelectSmemKeys) * 8;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8);
+    if (e != cudaSuccess) return e;
+    select_kernel<kSelectBlock><<<a.B, kSelectBlock, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace st

@@ -1,0 +1,165 @@
+/*
+ * st.h -- C ABI of the Bloom-filtered int8 IVF top-k search library (libst.so)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What it computes. For each query b (an int8 vector q_b and a Bloom mask m_b):
+ *   1. probe: score every IVF list c by the int32 inner product <q_b, cent_c>
+ *      and keep the nprobe best lists ("pick the most promising clusters
+ *      first" -- SilverTorch: Index as Model, section on how each component
+ *      worked before);
+ *   2. filter: inside the probed lists only, an item i is eligible when
+ *      (sig_i[w] & m_b[w]) == m_b[w] for every signature word w (same page,
+ *      section on redesigning each stage as a pure PyTorch module, Bloom index
+ *      filter paragraph);
+ *   3. score: eligible items only, by the int32 inner product <q_b, x_i> of
+ *      int8 vectors (same section, fused Int8 ANN paragraph);
+ *   4. top-k: the k best eligible items, ordered by score descending, then by
+ *      item id ascending (large top-k: "no recall loss at 64 probes and
+ *      top-2048", same paragraph; SilverTorch: Index as Model, Spanish
+ *      translation, table of compute cost efficiency, row on maximum top-k).
+ *   Probe ties go to the lower list id. The item id is the row index in the
+ *   arrays given to st_index_create. When fewer than k items are eligible, the
+ *   remaining slots hold id -1 and score INT32_MIN. The Bloom test alone
+ *   decides eligibility (a false-positive match is a legitimate result).
+ *   The result is unique, so every call returns exactly the same bytes.
+ *
+ * Conventions. Arrays are dense and row-major. "Device" pointers are CUDA
+ * device (or managed) memory on the index's device; "host" pointers may be
+ * pageable or pinned. All calls return an st_status and never throw. Invalid
+ * arguments are rejected on the host before any work is enqueued. There is no
+ * CPU fallback: every step runs in the library's own CUDA kernels.
+ */
+#ifndef ST_H_
+#define ST_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct st_index st_index; /* opaque */
+
+typedef enum {
+    ST_OK = 0,
+    ST_ERR_INVALID_ARG = 1,  /* null / non-device pointer, bad size, malformed offsets */
+    ST_ERR_UNSUPPORTED = 2,  /* a size outside the supported limits below */
+    ST_ERR_OOM = 3,          /* a device allocation failed */
+    ST_ERR_CUDA = 4,         /* a CUDA runtime or launch error */
+    ST_ERR_DEVICE = 5        /* a kernel recorded an internal error (see st_index_check) */
+} st_status;
+
+/* Supported limits (ST_ERR_UNSUPPORTED outside them). */
+#define ST_MAX_D 512         /* d must be a multiple of 16 in [16, 512] */
+#define ST_MAX_K 4096        /* 1 <= k <= 4096 */
+#define ST_MAX_NPROBE 4096   /* 1 <= nprobe <= min(nlist, 4096) */
+/* n < 2^31 items; sig_words is 1 (64-bit signatures) or 2 (128-bit). */
+
+/*
+ * Build an index. Copies every input into library-owned device memory, so the
+ * caller may free or reuse its arrays as soon as the call returns (the call
+ * waits for its copies on `stream`). Inputs may be device or host memory.
+ *
+ *   items        int8   [n][d]          item embeddings, rows grouped by list:
+ *                                       list c owns rows off[c] .. off[c+1]-1
+ *   sigs         uint64 [n][sig_words]  Bloom signatures; word 0 holds bits
+ *                                       0-63, word 1 bits 64-127
+ *   list_offsets int64  [nlist+1]       CSR offsets: off[0] = 0, off[nlist] = n,
+ *                                       nondecreasing (empty lists allowed)
+ *   centroids    int8   [nlist][d]      IVF list centroids
+ *   out          receives the index; *out is NULL on failure
+ *
+ * Errors: INVALID_ARG (null pointer, n < 1, nlist < 1, malformed offsets),
+ * UNSUPPORTED (d or sig_words outside the limits, n >= 2^31), OOM, CUDA.
+ * The index lives on the device that is current during this call.
+ */
+st_status st_index_create(const int8_t* items, const uint64_t* sigs,
+                          const int64_t* list_offsets, const int8_t* centroids,
+                          int64_t n, int32_t d, int32_t nlist, int32_t sig_words,
+                          cudaStream_t stream, st_index** out);
+
+/*
+ * Search B queries. Asynchronous on `stream`: it enqueues the kernels and
+ * returns without waiting for them; results are valid once `stream` reaches
+ * this point. Never synchronizes the host.
+ *
+ *   queries    device int8   [B][d]
+ *   qmasks     device uint64 [B][sig_words]
+ *   out_ids    device int64  [B][k]   caller-owned
+ *   out_scores device int32  [B][k]   caller-owned
+ *
+ * Scratch memory comes from a stream-ordered pool owned by the index and is
+ * returned to it when the search completes, so concurrent calls on different
+ * streams may share one index. The index itself is never modified.
+ *
+ * Errors: INVALID_ARG (null or non-device pointer, B < 1, k < 1, nprobe < 1 or
+ * nprobe > nlist), UNSUPPORTED (k or nprobe above the limits), OOM, CUDA.
+ * A kernel-side internal error is reported by st_index_check.
+ */
+st_status st_search(const st_index* idx, const int8_t* queries, const uint64_t* qmasks,
+                    int32_t B, int32_t nprobe, int32_t k,
+                    int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
+
+/* Optional extra outputs of st_search_ex; any member may be NULL. */
+typedef struct {
+    int64_t* eligible; /* device int64 [B]: eligible items in each query's probed
+                          lists (the number of (query, item) scores computed) */
+    int32_t* probe;    /* device int32 [B][nprobe]: the probed lists, best first */
+    /* Timing hooks: each non-NULL event is recorded on `stream` at a stage
+       boundary -- [0] before the probe kernel, [1] after it, [2] after the plan
+       kernels, [3] after the list scan, [4] after the final top-k. */
+    cudaEvent_t stage_events[5];
+} st_search_extras;
+
+/* st_search with optional extra outputs (extras may be NULL). */
+st_status st_search_ex(const st_index* idx, const int8_t* queries, const uint64_t* qmasks,
+                       int32_t B, int32_t nprobe, int32_t k,
+                       int64_t* out_ids, int32_t* out_scores,
+                       const st_search_extras* extras, cudaStream_t stream);
+
+/*
+ * st_search for host-resident queries and results: copies queries and masks to
+ * the device, searches, copies ids and scores back, and waits for `stream`
+ * before returning, so the outputs are ready on return. Pinned host memory
+ * makes the copies asynchronous DMA; pageable memory also works.
+ * Same arguments and errors as st_search, with every array in host memory.
+ */
+st_status st_search_host(const st_index* idx, const int8_t* queries, const uint64_t* qmasks,
+                         int32_t B, int32_t nprobe, int32_t k,
+                         int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
+
+/*
+ * Wait for `stream`, then report and clear the index's device-side error word.
+ * Returns ST_OK, ST_ERR_DEVICE when a kernel recorded an internal error since
+ * the last check (no result produced meanwhile should be trusted), or
+ * ST_ERR_CUDA when the stream itself failed.
+ */
+st_status st_index_check(const st_index* idx, cudaStream_t stream);
+
+/* Tuning options (all have working defaults). */
+typedef enum {
+    /* Device memory (bytes) that one search may use for candidate keys
+       (default 2 GiB). Searches whose candidates exceed it stay exact: the
+       affected queries take a slower exact path. */
+    ST_OPT_CANDIDATE_BYTES = 1,
+    /* Force the per-query candidate capacity (keys) instead of deriving it;
+       0 restores the default. Values below k + 1024 are raised to that. */
+    ST_OPT_CANDIDATE_CAPACITY = 2
+} st_option;
+
+/* Set an option; INVALID_ARG for an unknown option or a negative value.
+   Not safe to call while a search on the same index is being enqueued. */
+st_status st_index_set_option(st_index* idx, st_option opt, int64_t value);
+
+/* Free the index (NULL-safe). Waits for the device to finish work that may
+   still use it. */
+void st_index_destroy(st_index* idx);
+
+/* Static text for a status code. */
+const char* st_status_string(st_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ST_H_ */
