@@ -1,6 +1,6 @@
 // Host side of the C ABI declared in include/st.h: argument validation, the
 // library-owned index copy, stream-ordered scratch, and the kernel sequence
-// probe -> plan -> expand -> scan -> select of one search.
+// memset -> probe -> plan -> scan -> select of one search.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -17,6 +17,7 @@ struct st_index {
     int8_t* items = nullptr;
     uint64_t* sigs = nullptr;
     int64_t* offsets = nullptr;
+    int32_t* nchunks = nullptr;   // [nlist] ceil(list rows / warp unit rows)
     int8_t* centroids = nullptr;
     uint32_t* err = nullptr;
     std::vector<int64_t> top_prefix;  // [p] = rows in the p largest lists
@@ -27,14 +28,14 @@ struct st_index {
 
 namespace st {
 
-cudaError_t ensure_smem_attr(const void* func, int slot)
+cudaError_t ensure_smem_attr(const void* func, int slot, int bytes)
 {
     static unsigned done[64] = {0};  // bit `slot` set once per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && slot < 32 && (done[dev] >> slot) & 1u) return cudaSuccess;
-    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess && dev < 64 && slot < 32) __atomic_fetch_or(&done[dev], 1u << slot, __ATOMIC_RELAXED);
     return e;
 }
@@ -82,12 +83,12 @@ st_status cuda_status(cudaError_t e)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Carves one scratch allocation into the per-search arrays.
+// Carves one scratch allocation into the per-search arrays. The arrays that
+// must start at zero come first, so one memset clears them.
 struct ScratchLayout {
     size_t total = 0;
-    size_t off_probe, off_probe_keys, off_list_cnt, off_list_qstart, off_list_fill, off_qlist,
-        off_dl_list, off_dl_qstart, off_dl_qcnt, off_dl_ustart, off_units, off_ctl, off_cand_cnt,
-        off_elig, off_cand;
+    size_t off_list_cnt, off_list_fill, off_cand_cnt, off_elig, off_ctl, zero_bytes;
+    size_t off_probe, off_probe_keys, off_list_qstart, off_qlist, off_qmask, off_units, off_cand;
     size_t add(size_t bytes)
     {
         const size_t o = total;
@@ -104,7 +105,7 @@ int64_t candidate_capacity(const st_index* idx, int32_t B, int32_t P, int32_t k)
     if (idx->cand_cap_override > 0) cap = idx->cand_cap_override;
     const int64_t floor_cap = int64_t(k) + st::kSelectBlock;
     if (cap < floor_cap) cap = floor_cap;
-    return cap;
+    return (cap + 31) / 32 * 32;  // keeps every query's buffer 256-byte aligned
 }
 
 int64_t max_units_bound(const st_index* idx, int32_t B, int32_t P)
@@ -125,24 +126,22 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     const int64_t cap = candidate_capacity(idx, B, nprobe, k);
     const int64_t max_units = max_units_bound(idx, B, nprobe);
     if (max_units >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
-    const int64_t ndl = std::min<int64_t>(idx->nlist, int64_t(B) * nprobe);
     const bool probe_in_smem = idx->nlist <= st::kProbeSmemKeys;
+    const size_t nl4 = size_t(idx->nlist + 3) / 4 * 4;
 
     ScratchLayout L;
-    L.off_probe = L.add(size_t(B) * nprobe * 4);
-    L.off_probe_keys = probe_in_smem ? 0 : L.add(size_t(B) * idx->nlist * 8);
-    L.off_list_cnt = L.add(size_t(idx->nlist) * 4);
-    L.off_list_qstart = L.add(size_t(idx->nlist) * 4);
-    L.off_list_fill = L.add(size_t(idx->nlist) * 4);
-    L.off_qlist = L.add(size_t(B) * nprobe * 4);
-    L.off_dl_list = L.add(size_t(ndl) * 4);
-    L.off_dl_qstart = L.add(size_t(ndl) * 4);
-    L.off_dl_qcnt = L.add(size_t(ndl) * 4);
-    L.off_dl_ustart = L.add(size_t(ndl + 1) * 4);
-    L.off_units = L.add(size_t(max_units) * 16);
-    L.off_ctl = L.add(sizeof(st::PlanCtl));
+    L.off_list_cnt = L.add(nl4 * 4);
+    L.off_list_fill = L.add(nl4 * 4);
     L.off_cand_cnt = L.add(size_t(B) * 4);
     L.off_elig = L.add(size_t(B) * 8);
+    L.off_ctl = L.add(sizeof(st::PlanCtl));
+    L.zero_bytes = L.total;
+    L.off_probe = L.add(size_t(B) * nprobe * 4);
+    L.off_probe_keys = probe_in_smem ? 0 : L.add(size_t(B) * idx->nlist * 8);
+    L.off_list_qstart = L.add(nl4 * 4);
+    L.off_qlist = L.add(size_t(B) * nprobe * 4);
+    L.off_qmask = L.add(size_t(B) * nprobe * 16);
+    L.off_units = L.add(size_t(max_units) * 16);
     L.off_cand = L.add(size_t(B) * size_t(cap) * 8);
 
     unsigned char* base = nullptr;
@@ -157,6 +156,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.items = idx->items;
     a.sigs = idx->sigs;
     a.offsets = idx->offsets;
+    a.nchunks = idx->nchunks;
     a.centroids = idx->centroids;
     a.d = idx->d;
     a.nlist = idx->nlist;
@@ -169,21 +169,18 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.out_ids = out_ids;
     a.out_scores = out_scores;
     a.out_eligible = extras ? extras->eligible : nullptr;
-    a.probe = reinterpret_cast<int32_t*>(base + L.off_probe);
-    a.probe_keys = probe_in_smem ? nullptr : reinterpret_cast<uint64_t*>(base + L.off_probe_keys);
     a.list_cnt = reinterpret_cast<int32_t*>(base + L.off_list_cnt);
-    a.list_qstart = reinterpret_cast<int32_t*>(base + L.off_list_qstart);
     a.list_fill = reinterpret_cast<int32_t*>(base + L.off_list_fill);
-    a.qlist = reinterpret_cast<int32_t*>(base + L.off_qlist);
-    a.dl_list = reinterpret_cast<int32_t*>(base + L.off_dl_list);
-    a.dl_qstart = reinterpret_cast<int32_t*>(base + L.off_dl_qstart);
-    a.dl_qcnt = reinterpret_cast<int32_t*>(base + L.off_dl_qcnt);
-    a.dl_ustart = reinterpret_cast<int32_t*>(base + L.off_dl_ustart);
-    a.units = reinterpret_cast<int4*>(base + L.off_units);
-    a.max_units = int32_t(max_units);
-    a.ctl = reinterpret_cast<st::PlanCtl*>(base + L.off_ctl);
     a.cand_cnt = reinterpret_cast<uint32_t*>(base + L.off_cand_cnt);
     a.eligible_cnt = reinterpret_cast<unsigned long long*>(base + L.off_elig);
+    a.ctl = reinterpret_cast<st::PlanCtl*>(base + L.off_ctl);
+    a.probe = reinterpret_cast<int32_t*>(base + L.off_probe);
+    a.probe_keys = probe_in_smem ? nullptr : reinterpret_cast<uint64_t*>(base + L.off_probe_keys);
+    a.list_qstart = reinterpret_cast<int32_t*>(base + L.off_list_qstart);
+    a.qlist = reinterpret_cast<int32_t*>(base + L.off_qlist);
+    a.qmask_slot = reinterpret_cast<uint64_t*>(base + L.off_qmask);
+    a.units = reinterpret_cast<int4*>(base + L.off_units);
+    a.max_units = int32_t(max_units);
     a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
     a.cap = cap;
     a.err = idx->err;
@@ -191,7 +188,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     auto mark = [&](int i) {
         if (e == cudaSuccess && extras && extras->stage_events[i]) e = cudaEventRecord(extras->stage_events[i], stream);
     };
-    e = cudaSuccess;
+    e = cudaMemsetAsync(base, 0, L.zero_bytes, stream);
     mark(0);
     if (e == cudaSuccess) e = st::launch_probe(a, stream);
     mark(1);
@@ -284,6 +281,7 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         cudaMalloc(&idx->sigs, sig_bytes + 256) != cudaSuccess ||
         cudaMalloc(&idx->offsets, off.size() * 8) != cudaSuccess ||
         cudaMalloc(&idx->centroids, size_t(nlist) * d + 256) != cudaSuccess ||
+        cudaMalloc(&idx->nchunks, size_t(nlist) * 4) != cudaSuccess ||
         cudaMalloc(&idx->err, 256) != cudaSuccess) {
         cudaGetLastError();
         return fail(ST_ERR_OOM);
@@ -294,6 +292,9 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         e = cudaMemcpyAsync(idx->offsets, off.data(), off.size() * 8, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(idx->centroids, centroids, size_t(nlist) * d, cudaMemcpyDefault, stream);
+    std::vector<int32_t> nch(nlist);
+    for (int32_t c = 0; c < nlist; ++c) nch[c] = int32_t((off[c + 1] - off[c] + st::kWarpItems - 1) / st::kWarpItems);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(idx->nchunks, nch.data(), nch.size() * 4, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(idx->err, 0, 256, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) {
@@ -421,6 +422,7 @@ void st_index_destroy(st_index* idx)
         cudaFree(idx->sigs);
         cudaFree(idx->offsets);
         cudaFree(idx->centroids);
+        cudaFree(idx->nchunks);
         cudaFree(idx->err);
         if (idx->pool) cudaMemPoolDestroy(idx->pool);
         cudaGetLastError();

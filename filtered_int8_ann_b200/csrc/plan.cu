@@ -1,166 +1,168 @@
-// Plan: invert the probe result (query -> lists) into list -> queries, so the
-// scan reads each probed list once per batch however many queries probe it,
-// and cut every distinct probed list into fixed-size work units
-// (chunk of kWarpItems items) x (group of up to kQMax queries).
+// Plan: invert the probe result (query -> lists) into list -> query slots, so
+// the scan reads each probed list once per batch however many queries probe
+// it, and cut every probed list into warp work units of kWarpItems rows x a
+// group of up to kQMax queries. One 16-byte unit entry {first row, rows, first
+// query slot, queries} is all a scan warp needs.
 //
-// One CTA. Steps: count the queries of every list; one block-wide exclusive
-// scan gives each list its slice of the grouped query array and its first work
-// unit; a second pass scatters the query ids into their list's slice. It also
-// clears the per-query counters that the scan accumulates into and resets the
-// scan's work counter, so a search needs no separate memset.
+// Multi-CTA without any grid-wide wait: CTA c owns the list range
+// [c*nlist/G, (c+1)*nlist/G). Every CTA first reduces the per-list counts over
+// all lists (vectorised, from L2) to get the slot and unit offsets at the start
+// of its range and the grand total; it then scans its own lists, writes their
+// slot starts and unit entries, and scatters the (query, list) pairs whose
+// list it owns into the slot arrays (query id and that query's mask words, so
+// the scan reads a slot with one load instead of two dependent ones). The
+// per-list query counts were accumulated by the probe kernel into a zeroed
+// array.
 #include "st_internal.cuh"
 
 namespace st {
 
 template <int BLOCK>
-__device__ void block_exclusive_scan3(int32_t v[3], int32_t out[3], int32_t total[3])
+__device__ __forceinline__ void block_sum3(long long v[3], long long* red /*[3][BLOCK/32]*/)
 {
-    __shared__ int32_t warp_tot[BLOCK / 32][3];
+    constexpr int NW = BLOCK / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int32_t incl[3] = {v[0], v[1], v[2]};
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-#pragma unroll
-        for (int c = 0; c < 3; ++c) {
-            const int32_t t = __shfl_up_sync(0xffffffffu, incl[c], off);
-            if (lane >= off) incl[c] += t;
-        }
-    }
-    if (lane == 31)
-        for (int c = 0; c < 3; ++c) warp_tot[warp][c] = incl[c];
-    __syncthreads();
-    if (warp == 0) {
-        constexpr int NW = BLOCK / 32;
-        int32_t w[3];
-        for (int c = 0; c < 3; ++c) w[c] = lane < NW ? warp_tot[lane][c] : 0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-#pragma unroll
-            for (int c = 0; c < 3; ++c) {
-                const int32_t t = __shfl_up_sync(0xffffffffu, w[c], off);
-                if (lane >= off) w[c] += t;
-            }
-        }
-        if (lane < NW)
-            for (int c = 0; c < 3; ++c) warp_tot[lane][c] = w[c];  // inclusive per warp
-    }
-    __syncthreads();
     for (int c = 0; c < 3; ++c) {
-        const int32_t before = warp > 0 ? warp_tot[warp - 1][c] : 0;
-        out[c] = before + incl[c] - v[c];
-        total[c] = warp_tot[BLOCK / 32 - 1][c];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v[c] += __shfl_xor_sync(0xffffffffu, v[c], off);
+        if (lane == 0) red[c * NW + warp] = v[c];
     }
     __syncthreads();
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+        long long t = 0;
+        for (int w = 0; w < NW; ++w) t += red[c * NW + w];
+        v[c] = t;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ long long units_of(int32_t cnt, int32_t nch)
+{
+    return cnt > 0 ? (long long)nch * ((cnt + kQMax - 1) / kQMax) : 0;
 }
 
 template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK)
 plan_kernel(SearchArgs a)
 {
-    const int nlist = a.nlist;
-    const int npairs = a.B * a.P;
+    __shared__ long long s_red[3 * (BLOCK / 32)];
+    __shared__ uint32_t s_part[32];
+    __shared__ int32_t s_uex[BLOCK + 1];
+    __shared__ int32_t s_qex[BLOCK];
+    __shared__ int32_t s_cnt[BLOCK];
+    __shared__ int32_t s_nch[BLOCK];
+    __shared__ long long s_off0[BLOCK];
+    __shared__ long long s_off1[BLOCK];
+
     const int tid = threadIdx.x;
+    const int nlist = a.nlist;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int L0 = int((long long)c * nlist / G), L1 = int((long long)(c + 1) * nlist / G);
 
-    for (int L = tid; L < nlist; L += BLOCK) {
-        a.list_cnt[L] = 0;
-        a.list_fill[L] = 0;
-    }
-    for (int b = tid; b < a.B; b += BLOCK) {
-        a.cand_cnt[b] = 0;
-        a.eligible_cnt[b] = 0;
-    }
-    __syncthreads();
-    for (int i = tid; i < npairs; i += BLOCK) {
-        const int L = a.probe[i];
-        if (L >= 0 && L < nlist) atomicAdd(&a.list_cnt[L], 1);
-        else set_error(a.err, kErrSelectCount);
-    }
-    __syncthreads();
-
-    // each thread owns a contiguous range of lists
-    const int seg = (nlist + BLOCK - 1) / BLOCK;
-    const int lo = min(nlist, tid * seg), hi = min(nlist, lo + seg);
-    int32_t v[3] = {0, 0, 0};  // distinct lists with items, query slots, work units
-    for (int L = lo; L < hi; ++L) {
-        const int32_t c = a.list_cnt[L];
-        const int64_t nL = a.offsets[L + 1] - a.offsets[L];
-        v[1] += c;
-        if (c > 0 && nL > 0) {
-            v[0] += 1;
-            v[2] += int32_t((nL + kWarpItems - 1) / kWarpItems) * ((c + kQMax - 1) / kQMax);
+    // pass A: slot / unit offsets before L0, and the unit total (list_cnt is
+    // padded with zeros to a multiple of 4 entries)
+    long long v[3] = {0, 0, 0};  // slots before L0, units before L0, units total
+    const int n4 = (nlist + 3) >> 2;
+    const int4* cnt4 = reinterpret_cast<const int4*>(a.list_cnt);
+#pragma unroll 4
+    for (int i = tid; i < n4; i += BLOCK) {
+        const int4 q = cnt4[i];
+        const int cs[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int L = 4 * i + j;
+            if (cs[j] == 0 || L >= nlist) continue;
+            const long long u = units_of(cs[j], a.nchunks[L]);
+            if (L < L0) {
+                v[0] += cs[j];
+                v[1] += u;
+            }
+            v[2] += u;
         }
     }
-    int32_t ex[3], tot[3];
-    block_exclusive_scan3<BLOCK>(v, ex, tot);
-    for (int L = lo; L < hi; ++L) {
-        const int32_t c = a.list_cnt[L];
-        const int64_t nL = a.offsets[L + 1] - a.offsets[L];
-        a.list_qstart[L] = ex[1];
-        if (c > 0 && nL > 0) {
-            const int j = ex[0];
-            a.dl_list[j] = L;
-            a.dl_qstart[j] = ex[1];
-            a.dl_qcnt[j] = c;
-            a.dl_ustart[j] = ex[2];
-            ex[0] += 1;
-            ex[2] += int32_t((nL + kWarpItems - 1) / kWarpItems) * ((c + kQMax - 1) / kQMax);
+    block_sum3<BLOCK>(v, s_red);
+    const long long total_units = v[2];
+    if (c == 0 && tid == 0) {
+        a.ctl->n_units = int(total_units < a.max_units ? total_units : a.max_units);
+        if (total_units > a.max_units) set_error(a.err, kErrUnitTable);
+    }
+
+    // pass B: scan the owned lists tile by tile, write slot starts and units
+    long long qbase = v[0], ubase = v[1];
+    for (int t0 = L0; t0 < L1; t0 += BLOCK) {
+        const int L = t0 + tid;
+        int32_t cnt = 0, nch = 0;
+        long long o0 = 0, o1 = 0;
+        if (L < L1) {
+            cnt = a.list_cnt[L];
+            if (cnt > 0) {
+                nch = a.nchunks[L];
+                o0 = a.offsets[L];
+                o1 = a.offsets[L + 1];
+            }
         }
-        ex[1] += c;
+        const uint32_t u = uint32_t(units_of(cnt, nch));
+        uint32_t qtot, utot;
+        const uint32_t qex = block_excl_scan<BLOCK>(uint32_t(cnt), s_part, qtot);
+        const uint32_t uex = block_excl_scan<BLOCK>(u, s_part, utot);
+        if (L < L1) a.list_qstart[L] = int32_t(qbase + qex);
+        s_uex[tid] = int32_t(uex);
+        s_qex[tid] = int32_t(qex);
+        s_cnt[tid] = cnt;
+        s_nch[tid] = nch;
+        s_off0[tid] = o0;
+        s_off1[tid] = o1;
+        if (tid == 0) s_uex[BLOCK] = int32_t(utot);
+        __syncthreads();
+        for (uint32_t w = tid; w < utot; w += BLOCK) {
+            // owner: the last list of the tile whose first unit is <= w
+            int lo = 0, hi = BLOCK - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (uint32_t(s_uex[mid]) <= w) lo = mid; else hi = mid - 1;
+            }
+            const int local = int(w) - s_uex[lo];
+            const int nc = s_nch[lo];
+            const int g = nc > 0 ? local / nc : 0, ch = local - g * nc;
+            const long long ib = s_off0[lo] + (long long)ch * kWarpItems;
+            const long long rem = s_off1[lo] - ib;
+            const int len = int(rem < kWarpItems ? rem : kWarpItems);
+            const int qn = min(kQMax, s_cnt[lo] - g * kQMax);
+            const long long u_idx = ubase + w;
+            if (nc <= 0 || qn <= 0 || len <= 0) {
+                set_error(a.err, kErrUnitDecode);
+                continue;
+            }
+            if (u_idx < a.max_units)
+                a.units[u_idx] = make_int4(int(ib), len, int(qbase + s_qex[lo] + g * kQMax), qn);
+        }
+        qbase += qtot;
+        ubase += utot;
+        __syncthreads();
     }
-    if (tid == 0) {
-        a.ctl->n_lists = tot[0];
-        a.ctl->n_units = min(tot[2], a.max_units);
-        if (tot[2] > a.max_units) set_error(a.err, kErrUnitTable);
-        a.ctl->next_unit = 0;
-        a.dl_ustart[tot[0]] = tot[2];
-    }
-    __syncthreads();
+
+    // pass C: scatter the pairs whose list this CTA owns into the slot arrays
+    const int npairs = a.B * a.P;
+    const int W = a.W;
     for (int i = tid; i < npairs; i += BLOCK) {
         const int L = a.probe[i];
-        if (L < 0 || L >= nlist) continue;
+        if (L < L0 || L >= L1) continue;
         const int pos = a.list_qstart[L] + atomicAdd(&a.list_fill[L], 1);
-        a.qlist[pos] = i / a.P;
-    }
-}
-
-// Expand: one self-contained 16-byte entry per work unit, so a scan warp needs
-// a single load to know its rows and queries. Unit u of distinct list j covers
-// chunk c = local % nchunks of the list and query group g = local / nchunks,
-// where local = u - first unit of j (consecutive units walk down one list).
-__global__ void __launch_bounds__(kExpandBlock)
-expand_kernel(SearchArgs a)
-{
-    const int n_units = a.ctl->n_units;
-    const int n_lists = a.ctl->n_lists;
-    for (int u = blockIdx.x * kExpandBlock + threadIdx.x; u < n_units; u += gridDim.x * kExpandBlock) {
-        int lo = 0, hi = n_lists - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(a.dl_ustart + mid) <= u) lo = mid; else hi = mid - 1;
-        }
-        const int L = a.dl_list[lo];
-        const int64_t o0 = a.offsets[L], o1 = a.offsets[L + 1];
-        const int nchunks = int((o1 - o0 + kWarpItems - 1) / kWarpItems);
-        const int local = u - a.dl_ustart[lo];
-        const int g = local / nchunks, c = local - g * nchunks;
-        const int qn = min(kQMax, a.dl_qcnt[lo] - g * kQMax);
-        const int64_t ib = o0 + int64_t(c) * kWarpItems;
-        const int len = int(min(o1 - ib, int64_t(kWarpItems)));
-        if (local < 0 || qn <= 0 || len <= 0) {
-            set_error(a.err, kErrUnitDecode);
-            a.units[u] = make_int4(0, 0, 0, 0);
-            continue;
-        }
-        a.units[u] = make_int4(int(ib), len, a.dl_qstart[lo] + g * kQMax, qn);
+        const int b = i / a.P;
+        a.qlist[pos] = b;
+        a.qmask_slot[2 * int64_t(pos)] = a.qmasks[int64_t(b) * W];
+        a.qmask_slot[2 * int64_t(pos) + 1] = W > 1 ? a.qmasks[int64_t(b) * W + 1] : 0ull;
     }
 }
 
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s)
 {
-    plan_kernel<kPlanBlock><<<1, kPlanBlock, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    expand_kernel<<<num_sms * 2, kExpandBlock, 0, s>>>(a);
+    int G = a.nlist / 64;
+    if (G > num_sms) G = num_sms;
+    if (G < 1) G = 1;
+    plan_kernel<kPlanBlock><<<G, kPlanBlock, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -13,7 +13,8 @@
 // with 16-byte read-only loads and accumulates with dp4a. The centroid table
 // (nlist * d bytes, 1 MiB for 16384 x 64) stays L2-resident across CTAs. Keys
 // stay in shared memory up to 16384 lists and spill to a global scratch row
-// beyond, then an in-CTA radix select picks the nprobe best keys.
+// beyond, then an in-CTA radix select picks the nprobe best keys. Each chosen
+// list bumps its query count, which the plan kernel consumes.
 #include "st_internal.cuh"
 
 namespace st {
@@ -27,11 +28,13 @@ probe_kernel(SearchArgs a)
     const int b = blockIdx.x;
     const int d = a.d;
     const int nlist = a.nlist;
-    const int pw = next_pow2(a.P);
+    const int P = a.P;
+    const int pw = next_pow2(P);
+    const int pws = pw < 2 ? 2 : pw;
 
-    // shared layout: [sort buffer pw keys, 16-byte padded][query d bytes][keys nlist (if local)]
+    // shared layout: [sort buffer pws keys][query d bytes][keys nlist (if local)]
     uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem_raw);
-    int4* qv = reinterpret_cast<int4*>(sortbuf + (pw < 2 ? 2 : pw));
+    int4* qv = reinterpret_cast<int4*>(sortbuf + pws);
     const bool local_keys = (a.probe_keys == nullptr);
     uint64_t* keys = local_keys ? reinterpret_cast<uint64_t*>(qv + d / 16)
                                 : a.probe_keys + int64_t(b) * nlist;
@@ -49,19 +52,21 @@ probe_kernel(SearchArgs a)
     }
     __syncthreads();
 
-    const int P = a.P;
-    uint64_t kth = 0;
-    if (P < nlist) kth = block_kth_largest<BLOCK>(keys, nlist, P, ss);
-    const int got = block_collect_ge<BLOCK>(keys, nlist, kth, sortbuf, pw, ss);
+    uint64_t thr = 0;
+    if (P < nlist) thr = block_select_threshold<BLOCK>(keys, nlist, P, ss, a.err);
+    const int got = block_collect_ge<BLOCK>(keys, nlist, thr, sortbuf, pw, ss);
     if (threadIdx.x == 0 && got != P) set_error(a.err, kErrSelectCount);
-    for (int i = got + threadIdx.x; i < pw; i += BLOCK) sortbuf[i] = 0;
+    for (int i = (got < pw ? got : pw) + threadIdx.x; i < pw; i += BLOCK) sortbuf[i] = 0;
     __syncthreads();
     block_bitonic_desc<BLOCK>(sortbuf, pw);
-    for (int p = threadIdx.x; p < P; p += BLOCK)
-        a.probe[int64_t(b) * P + p] = int32_t(key_id(sortbuf[p]));
+    for (int p = threadIdx.x; p < P; p += BLOCK) {
+        const int L = int(key_id(sortbuf[p]));
+        a.probe[int64_t(b) * P + p] = L;
+        if (L >= 0 && L < nlist) atomicAdd(&a.list_cnt[L], 1);
+    }
 }
 
-size_t probe_smem_bytes(const SearchArgs& a)
+static size_t probe_smem_bytes(const SearchArgs& a)
 {
     const int pw = next_pow2(a.P);
     size_t bytes = size_t(pw < 2 ? 2 : pw) * 8 + size_t(a.d);
@@ -72,7 +77,7 @@ size_t probe_smem_bytes(const SearchArgs& a)
 cudaError_t launch_probe(const SearchArgs& a, cudaStream_t s)
 {
     const size_t smem = probe_smem_bytes(a);
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock>), 0);
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock>), 0, 200 * 1024);
     if (e != cudaSuccess) return e;
     probe_kernel<kProbeBlock><<<a.B, kProbeBlock, smem, s>>>(a);
     return cudaGetLastError();

@@ -8,16 +8,16 @@
 // efficiency table in the Spanish translation.
 //
 // The candidate keys of a query (written by the scan) are copied into shared
-// memory when they fit, an MSB-first radix select finds the k-th largest key,
-// the keys at or above it are gathered (exactly k: keys are unique) and a
+// memory when they fit; a radix select over the bits where they differ finds a
+// threshold with exactly k keys at or above it; those keys are gathered and a
 // bitonic network sorts them.
 //
-// Exact overflow path: when the scan emitted more candidates for a query than
-// its buffer holds (the count kept running past the capacity), this CTA
-// rescans that query's probed lists itself with a bounded buffer: whenever the
-// buffer fills it keeps only the k best keys and from then on drops any key
-// below the k-th, which can no longer enter the top-k. Exact for any input,
-// with memory bounded by the capacity; slow, and used only on overflow.
+// Exact overflow path: when the scan reserved more candidates for a query than
+// its buffer holds, this CTA rescans that query's probed lists itself with the
+// bounded buffer: whenever the buffer fills it keeps only the k best keys and
+// from then on drops any key below the k-th, which can no longer enter the
+// top-k. Exact for any input, with memory bounded by the capacity; slow, and
+// used only on overflow.
 #include "st_internal.cuh"
 
 namespace st {
@@ -28,8 +28,8 @@ __device__ int32_t select_into(const uint64_t* keys, int64_t n, int k, uint64_t*
 {
     int32_t got;
     if (n > k) {
-        const uint64_t kth = block_kth_largest<BLOCK>(keys, n, k, ss);
-        got = block_collect_ge<BLOCK>(keys, n, kth, sortbuf, pwk, ss);
+        const uint64_t thr = block_select_threshold<BLOCK>(keys, n, k, ss, err);
+        got = block_collect_ge<BLOCK>(keys, n, thr, sortbuf, pwk, ss);
         if (threadIdx.x == 0 && got != k) set_error(err, kErrSelectCount);
     } else {
         got = block_collect_ge<BLOCK>(keys, n, 1ull, sortbuf, pwk, ss);
@@ -43,7 +43,7 @@ __device__ int32_t select_into(const uint64_t* keys, int64_t n, int k, uint64_t*
 
 template <int BLOCK>
 __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, int pwk, int4* s_qv,
-                              SelectSmem& ss)
+                                 SelectSmem& ss)
 {
     __shared__ int32_t s_count;
     __shared__ uint64_t s_thr;
@@ -68,19 +68,22 @@ __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, 
         const int64_t o0 = a.offsets[L], o1 = a.offsets[L + 1];
         for (int64_t base = o0; base < o1; base += BLOCK) {
             if (int64_t(s_count) + BLOCK > cap) {
-                // keep the k best, raise the threshold to the k-th
-                const uint64_t kth = block_kth_largest<BLOCK>(buf, s_count, k, ss);
-                const int32_t got = block_collect_ge<BLOCK>(buf, s_count, kth, sortbuf, pwk, ss);
+                // keep the k best, drop everything below them from now on
+                const int64_t cnt = s_count;
+                const uint64_t thr = block_select_threshold<BLOCK>(buf, cnt, k, ss, a.err);
+                const int32_t got = block_collect_ge<BLOCK>(buf, cnt, thr, sortbuf, pwk, ss);
                 if (threadIdx.x == 0 && got != k) set_error(a.err, kErrOverflowPath);
                 for (int i = threadIdx.x; i < k; i += BLOCK) buf[i] = sortbuf[i];
                 if (threadIdx.x == 0) {
                     s_count = k;
-                    s_thr = kth;
+                    s_thr = thr;
                 }
                 __syncthreads();
             }
             const int64_t i = base + threadIdx.x;
             const uint64_t thr = s_thr;
+            bool keep = false;
+            uint64_t key = 0;
             if (i < o1) {
                 const uint64_t* sg = a.sigs + i * W;
                 bool pass = (sg[0] & m0) == m0;
@@ -89,9 +92,16 @@ __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, 
                     const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);
                     int32_t acc = 0;
                     for (int t = 0; t < np; ++t) acc = dot16(__ldg(rp + t), s_qv[t], acc);
-                    const uint64_t key = pack_key(acc, uint32_t(i));
-                    if (key > thr) buf[atomicAdd(&s_count, 1)] = key;
+                    key = pack_key(acc, uint32_t(i));
+                    keep = key >= thr;
                 }
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+            if (bal) {
+                int32_t b0 = 0;
+                if ((threadIdx.x & 31) == 0) b0 = atomicAdd(&s_count, __popc(bal));
+                b0 = __shfl_sync(0xffffffffu, b0, 0);
+                if (keep) buf[b0 + __popc(bal & lanemask_lt())] = key;
             }
             __syncthreads();
         }
@@ -116,7 +126,11 @@ select_kernel(SearchArgs a)
     int64_t n = cnt;
     if (n > a.cap) n = overflow_path<BLOCK>(a, q, sortbuf, pwk, reinterpret_cast<int4*>(local), ss);
     if (n <= kSelectSmemKeys) {
-        for (int64_t i = threadIdx.x; i < n; i += BLOCK) local[i] = keys[i];
+        const int64_t n2 = n >> 1;
+        const ulonglong2* src2 = reinterpret_cast<const ulonglong2*>(keys);
+        ulonglong2* dst2 = reinterpret_cast<ulonglong2*>(local);
+        for (int64_t i = threadIdx.x; i < n2; i += BLOCK) dst2[i] = src2[i];
+        if ((n & 1) && threadIdx.x == 0) local[n - 1] = keys[n - 1];
         __syncthreads();
         keys = local;
     }
@@ -133,7 +147,8 @@ cudaError_t launch_select(const SearchArgs& a, cudaStream_t s)
 {
     const int pwk = next_pow2(a.k);
     const size_t smem = size_t(pwk < 2 ? 2 : pwk) * 8 + size_t(kSelectSmemKeys) * 8;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8);
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8,
+                                     int(size_t(ST_MAX_K) * 8 + size_t(kSelectSmemKeys) * 8));
     if (e != cudaSuccess) return e;
     select_kernel<kSelectBlock><<<a.B, kSelectBlock, smem, s>>>(a);
     return cudaGetLastError();
