@@ -17,7 +17,10 @@ struct st_index {
     int8_t* items = nullptr;
     uint64_t* sigs = nullptr;
     int64_t* offsets = nullptr;
-    int32_t* nchunks = nullptr;   // [nlist] ceil(list rows / warp unit rows)
+    int32_t* chunk_start = nullptr;  // [nlist+1] first warp-unit chunk of each list
+    int32_t* chunk_list = nullptr;   // [n_chunks] list of each chunk
+    int32_t n_chunks = 0;
+    uint32_t* planes = nullptr;      // [n_chunks][64W][16] signature bit-planes
     int8_t* centroids = nullptr;
     uint32_t* err = nullptr;
     std::vector<int64_t> top_prefix;  // [p] = rows in the p largest lists
@@ -87,8 +90,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // must start at zero come first, so one memset clears them.
 struct ScratchLayout {
     size_t total = 0;
-    size_t off_list_cnt, off_list_fill, off_cand_cnt, off_elig, off_ctl, zero_bytes;
-    size_t off_probe, off_probe_keys, off_list_qstart, off_qlist, off_qmask, off_units, off_cand;
+    size_t off_list_cnt, off_probe_done, off_cand_cnt, off_elig, off_hist, off_ctl, zero_bytes;
+    size_t off_probe, off_probe_keys, off_probe_part, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_units, off_cand;
     size_t add(size_t bytes)
     {
         const size_t o = total;
@@ -105,6 +108,7 @@ int64_t candidate_capacity(const st_index* idx, int32_t B, int32_t P, int32_t k)
     if (idx->cand_cap_override > 0) cap = idx->cand_cap_override;
     const int64_t floor_cap = int64_t(k) + st::kSelectBlock;
     if (cap < floor_cap) cap = floor_cap;
+    cap += 1;  // one spare key so a pairwise copy of an odd count stays inside the buffer
     return (cap + 31) / 32 * 32;  // keeps every query's buffer 256-byte aligned
 }
 
@@ -126,21 +130,33 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     const int64_t cap = candidate_capacity(idx, B, nprobe, k);
     const int64_t max_units = max_units_bound(idx, B, nprobe);
     if (max_units >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
-    const bool probe_in_smem = idx->nlist <= st::kProbeSmemKeys;
+    if (int64_t(idx->nlist) * B >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
+    SearchArgs probe_shape;
+    std::memset(&probe_shape, 0, sizeof(probe_shape));
+    probe_shape.B = B;
+    probe_shape.P = nprobe;
+    probe_shape.nlist = idx->nlist;
+    const int S = st::probe_slices(probe_shape, idx->num_sms);
+    const bool probe_in_smem = (idx->nlist + S - 1) / S + 1 <= st::kProbeSmemKeys;
     const size_t nl4 = size_t(idx->nlist + 3) / 4 * 4;
+    const size_t slots = size_t(idx->nlist) * size_t(B);
 
     ScratchLayout L;
     L.off_list_cnt = L.add(nl4 * 4);
-    L.off_list_fill = L.add(nl4 * 4);
+    L.off_probe_done = L.add(size_t(B) * 4);
     L.off_cand_cnt = L.add(size_t(B) * 4);
     L.off_elig = L.add(size_t(B) * 8);
+    L.off_hist = L.add(size_t(B) * st::kHistBins * 4);
     L.off_ctl = L.add(sizeof(st::PlanCtl));
     L.zero_bytes = L.total;
     L.off_probe = L.add(size_t(B) * nprobe * 4);
     L.off_probe_keys = probe_in_smem ? 0 : L.add(size_t(B) * idx->nlist * 8);
-    L.off_list_qstart = L.add(nl4 * 4);
-    L.off_qlist = L.add(size_t(B) * nprobe * 4);
-    L.off_qmask = L.add(size_t(B) * nprobe * 16);
+    L.off_probe_part = L.add(size_t(B) * S * nprobe * 8);
+    L.off_list_ustart = L.add(nl4 * 4);
+    L.off_qbits = L.add(size_t(B) * st::kMaskBitsMax);
+    L.off_qnbits = L.add(size_t(B) * 4);
+    L.off_qlist = L.add(slots * 4);
+    L.off_qmask = L.add(slots * 16);
     L.off_units = L.add(size_t(max_units) * 16);
     L.off_cand = L.add(size_t(B) * size_t(cap) * 8);
 
@@ -155,8 +171,11 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     std::memset(&a, 0, sizeof(a));
     a.items = idx->items;
     a.sigs = idx->sigs;
+    a.planes = idx->planes;
     a.offsets = idx->offsets;
-    a.nchunks = idx->nchunks;
+    a.chunk_start = idx->chunk_start;
+    a.chunk_list = idx->chunk_list;
+    a.n_chunks = idx->n_chunks;
     a.centroids = idx->centroids;
     a.d = idx->d;
     a.nlist = idx->nlist;
@@ -170,13 +189,23 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.out_scores = out_scores;
     a.out_eligible = extras ? extras->eligible : nullptr;
     a.list_cnt = reinterpret_cast<int32_t*>(base + L.off_list_cnt);
-    a.list_fill = reinterpret_cast<int32_t*>(base + L.off_list_fill);
+    a.probe_done = reinterpret_cast<int32_t*>(base + L.off_probe_done);
     a.cand_cnt = reinterpret_cast<uint32_t*>(base + L.off_cand_cnt);
     a.eligible_cnt = reinterpret_cast<unsigned long long*>(base + L.off_elig);
+    a.hist = reinterpret_cast<uint32_t*>(base + L.off_hist);
+    a.smax = idx->d * 128 * 128;
+    {
+        int bits = 0;
+        while ((int64_t(1) << bits) < 2 * int64_t(a.smax)) ++bits;
+        a.hshift = bits > st::kSelBits ? bits - st::kSelBits : 0;
+    }
     a.ctl = reinterpret_cast<st::PlanCtl*>(base + L.off_ctl);
     a.probe = reinterpret_cast<int32_t*>(base + L.off_probe);
     a.probe_keys = probe_in_smem ? nullptr : reinterpret_cast<uint64_t*>(base + L.off_probe_keys);
-    a.list_qstart = reinterpret_cast<int32_t*>(base + L.off_list_qstart);
+    a.probe_part = reinterpret_cast<uint64_t*>(base + L.off_probe_part);
+    a.list_ustart = reinterpret_cast<int32_t*>(base + L.off_list_ustart);
+    a.qbits = reinterpret_cast<uint8_t*>(base + L.off_qbits);
+    a.qnbits = reinterpret_cast<int32_t*>(base + L.off_qnbits);
     a.qlist = reinterpret_cast<int32_t*>(base + L.off_qlist);
     a.qmask_slot = reinterpret_cast<uint64_t*>(base + L.off_qmask);
     a.units = reinterpret_cast<int4*>(base + L.off_units);
@@ -190,7 +219,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     };
     e = cudaMemsetAsync(base, 0, L.zero_bytes, stream);
     mark(0);
-    if (e == cudaSuccess) e = st::launch_probe(a, stream);
+    if (e == cudaSuccess) e = st::launch_probe(a, S, stream);
     mark(1);
     if (e == cudaSuccess) e = st::launch_plan(a, idx->num_sms, stream);
     mark(2);
@@ -281,7 +310,7 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         cudaMalloc(&idx->sigs, sig_bytes + 256) != cudaSuccess ||
         cudaMalloc(&idx->offsets, off.size() * 8) != cudaSuccess ||
         cudaMalloc(&idx->centroids, size_t(nlist) * d + 256) != cudaSuccess ||
-        cudaMalloc(&idx->nchunks, size_t(nlist) * 4) != cudaSuccess ||
+        cudaMalloc(&idx->chunk_start, size_t(nlist + 1) * 4) != cudaSuccess ||
         cudaMalloc(&idx->err, 256) != cudaSuccess) {
         cudaGetLastError();
         return fail(ST_ERR_OOM);
@@ -292,9 +321,29 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         e = cudaMemcpyAsync(idx->offsets, off.data(), off.size() * 8, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(idx->centroids, centroids, size_t(nlist) * d, cudaMemcpyDefault, stream);
-    std::vector<int32_t> nch(nlist);
-    for (int32_t c = 0; c < nlist; ++c) nch[c] = int32_t((off[c + 1] - off[c] + st::kWarpItems - 1) / st::kWarpItems);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(idx->nchunks, nch.data(), nch.size() * 4, cudaMemcpyHostToDevice, stream);
+    // static chunk table: list c owns chunks chunk_start[c] .. chunk_start[c+1]-1
+    std::vector<int32_t> cstart(size_t(nlist) + 1, 0);
+    for (int32_t c = 0; c < nlist; ++c)
+        cstart[c + 1] = cstart[c] + int32_t((off[c + 1] - off[c] + st::kWarpItems - 1) / st::kWarpItems);
+    idx->n_chunks = cstart[nlist];
+    std::vector<int32_t> clist(size_t(idx->n_chunks > 0 ? idx->n_chunks : 1), 0);
+    for (int32_t c = 0; c < nlist; ++c)
+        for (int32_t t = cstart[c]; t < cstart[c + 1]; ++t) clist[t] = c;
+    if (cudaMalloc(&idx->chunk_list, clist.size() * 4) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(ST_ERR_OOM);
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(idx->chunk_start, cstart.data(), cstart.size() * 4, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(idx->chunk_list, clist.data(), clist.size() * 4, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) {
+        const size_t pbytes = size_t(idx->n_chunks > 0 ? idx->n_chunks : 1) * 64 * sig_words * 16 * 4;
+        if (cudaMalloc(&idx->planes, pbytes) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(ST_ERR_OOM);
+        }
+        e = st::launch_build_planes(idx->sigs, idx->offsets, idx->chunk_start, idx->chunk_list, idx->n_chunks,
+                                    sig_words, idx->planes, stream);
+    }
     if (e == cudaSuccess) e = cudaMemsetAsync(idx->err, 0, 256, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) {
@@ -422,7 +471,9 @@ void st_index_destroy(st_index* idx)
         cudaFree(idx->sigs);
         cudaFree(idx->offsets);
         cudaFree(idx->centroids);
-        cudaFree(idx->nchunks);
+        cudaFree(idx->chunk_start);
+        cudaFree(idx->chunk_list);
+        cudaFree(idx->planes);
         cudaFree(idx->err);
         if (idx->pool) cudaMemPoolDestroy(idx->pool);
         cudaGetLastError();

@@ -11,63 +11,89 @@
 // gives the fusion principle kept here: intermediates stay in registers and
 // shared memory and never round-trip through HBM.
 //
-// B200 design. The plan kernel cut the probed lists into warp units (up to
-// kWarpItems consecutive rows x up to kQMax queries probing that list), so each
-// probed list is streamed once per batch whatever the number of queries
-// probing it. Warps are independent and take units round-robin; each warp runs
-// a two-stage software pipeline:
-//   * signatures: the unit's contiguous signature block (16 B per row for
-//     128-bit signatures) arrives by one bulk asynchronous copy (TMA engine,
-//     cp.async.bulk + mbarrier) into one of two per-warp shared buffers; the
-//     copy for the next unit is always in flight while this one is processed,
-//     so the signature stream never waits on the rest of the pipeline;
-//   * test: every signature against every query of the unit (masks by warp
-//     shuffle) gives a per-row query bitmask; the per-query survivor counts
-//     reserve candidate slots with one atomic per (unit, query), issued before
-//     the row loads so both round trips overlap;
-//   * filter-before-load: only survivors' rows are read (16-byte read-only
-//     loads into registers) -- rows of ineligible items never leave HBM -- and
-//     dotted with dp4a against the query vectors (staged in shared memory by
-//     cp.async); keys go straight to the reserved slots.
+// B200 design. The plan cut the probed lists into warp units: one list chunk
+// (kWarpItems rows) x up to kQMax queries probing that list, so each probed
+// list is streamed once per batch whatever the number of queries probing it.
+// Warps are independent (one-warp CTAs, many per SM) and take units
+// round-robin, with a two-deep pipeline:
+//   * signature planes: the index stores each chunk's signatures as bit-planes
+//     (layout.cu). A unit needs only the planes of the bits in the union of its
+//     queries' masks; its lanes issue one 64-byte bulk asynchronous copy (TMA
+//     engine, cp.async.bulk + mbarrier) per such plane into the next free slot
+//     of a small per-warp buffer (kPlaneSlots planes), and the next unit's
+//     planes are always in flight while this unit is processed. A unit whose
+//     union is wider than the buffer reads its planes from global memory
+//     instead (slower, same result);
+//   * test: for each query, the two half-warps AND the planes of the two
+//     halves of the query's mask bits (a list precomputed once per search) for
+//     the 32 rows of the lane's block; one shuffle joins the halves, so 32 rows
+//     cost one AND per mask bit;
+//   * filter-before-load: per-query survivor counts reserve candidate slots
+//     (one atomic per unit and query, overlapped with the row loads); only
+//     survivors' rows are read (16-byte read-only loads) and dotted with dp4a
+//     against the query vectors (staged in shared memory by cp.async); a key's
+//     slot is its ballot rank among the unit's survivors of that query; each
+//     key also counts into the query's score histogram, which the final top-k
+//     uses to find its cut without sorting every candidate.
 // Every wait on a copy is bounded: on expiry the warp records kErrCopyTimeout,
 // waits (bounded) for its copies in flight and stops.
 #include "st_internal.cuh"
 
 namespace st {
 
-template <int W>
-struct SigBuf {
-    // bytes of one signature buffer: a unit's signatures plus 16 bytes so that
-    // a 64-bit-signature copy can start at the 16-byte boundary below its row
-    static constexpr int kBytes = ((kWarpItems * 8 * W + 16) + 127) / 128 * 128;
-};
+constexpr int kPlaneSlots = 32;                         // planes one buffer holds
+constexpr int kPlaneBytes = kWarpItems / 8;             // 64 bytes per plane
+constexpr int kPlaneBufBytes = kPlaneSlots * kPlaneBytes;
 
+// Per-warp shared memory: 2 plane buffers | survivor offsets [kWarpItems] u16 |
+// pass words [kQMax][16] | query vectors [kQMax][d] | bit -> slot tables [2][128] |
+// query ids [kQMax] | 2 mbarriers
 __host__ __device__ inline size_t scan_warp_bytes(int d, int W)
 {
-    const size_t sig = W == 2 ? SigBuf<2>::kBytes : SigBuf<1>::kBytes;
-    // 2 signature buffers | query vectors [kQMax][d] | masks [kQMax][2] | qid [kQMax] | 2 mbarriers
-    return (2 * sig + size_t(kQMax) * d + kQMax * 16 + kQMax * 4 + 16 + 127) / 128 * 128;
+    (void)W;
+    return (2 * kPlaneBufBytes + kWarpItems * 2 + kQMax * 16 * 4 + size_t(kQMax) * d + 2 * kMaskBitsMax +
+            kQMax * 4 + 16 + 127) / 128 * 128;
 }
 
 size_t scan_smem_bytes(int d, int W) { return size_t(kScanBlock / 32) * scan_warp_bytes(d, W); }
 
+// Start the copies of the planes a unit needs (the union u0/u1 of its queries'
+// mask bits) into consecutive slots of `buf`, and record bit -> slot in `tab`.
+// Returns false (and copies nothing) when the union has more bits than a
+// buffer holds; the barrier phase completes either way.
 template <int W>
-__device__ __forceinline__ void issue_sig_copy(const SearchArgs& a, int4 e, unsigned char* buf, uint64_t* bar)
+__device__ __forceinline__ bool issue_planes(const SearchArgs& a, int chunk, uint64_t u0, uint64_t u1,
+                                             uint32_t* buf, uint8_t* tab, uint64_t* bar, int lane)
 {
-    const int64_t ib = e.x;
-    const int len = e.y;
-    const char* src;
-    uint32_t bytes;
-    if (W == 2) {
-        src = reinterpret_cast<const char*>(a.sigs + ib * 2);
-        bytes = uint32_t(len) * 16u;
-    } else {
-        const int64_t a0 = ib & ~int64_t(1);
-        src = reinterpret_cast<const char*>(a.sigs + a0);
-        bytes = uint32_t(((ib + len - a0) * 8 + 15) & ~int64_t(15));
+    constexpr int NPL = 64 * W;
+    const int n0 = __popcll(u0);
+    const int nb = n0 + (W > 1 ? __popcll(u1) : 0);
+    const bool fits = nb <= kPlaneSlots;
+    if (lane == 0) mbar_expect_tx(bar, fits ? uint32_t(nb) * kPlaneBytes : 0u);
+    __syncwarp();
+    if (!fits) return false;
+    const uint32_t* src = a.planes + int64_t(chunk) * NPL * 16;
+#pragma unroll
+    for (int r = 0; r < 2 * W; ++r) {
+        const int b = lane + 32 * r;
+        const uint64_t word = b < 64 ? u0 : u1;
+        const uint64_t below = (b & 63) ? (word & ((1ull << (b & 63)) - 1ull)) : 0ull;
+        const int slot = (b < 64 ? 0 : n0) + __popcll(below);
+        const bool on = (word >> (b & 63)) & 1ull;
+        tab[b] = on ? uint8_t(slot) : uint8_t(0);
+        if (on) bulk_g2s(buf + slot * 16, src + b * 16, kPlaneBytes, bar);
     }
-    mbar_expect_tx(bar, bytes);
-    bulk_g2s(buf, src, bytes, bar);
+    return true;
+}
+
+// OR of the masks held by lanes < qn (other lanes hold zeros).
+__device__ __forceinline__ void warp_or2(uint64_t& x, uint64_t& y)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        x |= __shfl_xor_sync(0xffffffffu, x, off);
+        y |= __shfl_xor_sync(0xffffffffu, y, off);
+    }
 }
 
 // NP = d/16 when the row is held in registers (d = 64 or 128), 0 for any other
@@ -77,20 +103,23 @@ __global__ void __launch_bounds__(kScanBlock)
 scan_kernel(SearchArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    constexpr int IPL = kWarpItems / 32;  // rows per lane
-    constexpr int SB = SigBuf<W>::kBytes;
+    constexpr int NPL = 64 * W;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int d = a.d;
     const int np = NP ? NP : (d >> 4);
+    const int blk = lane & 15;   // 32-row block of the chunk this lane tests
+    const int half = lane >> 4;  // which half of the mask bits it ANDs
 
     unsigned char* wb = smem_raw + size_t(warp) * scan_warp_bytes(d, W);
-    unsigned char* sbuf0 = wb;
-    unsigned char* sbuf1 = wb + SB;
-    int4* s_q = reinterpret_cast<int4*>(wb + 2 * SB);                                // [kQMax][np]
-    ulonglong2* s_m = reinterpret_cast<ulonglong2*>(wb + 2 * SB + size_t(kQMax) * d); // [kQMax]
-    int32_t* s_qid = reinterpret_cast<int32_t*>(s_m + kQMax);                         // [kQMax]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s_qid + kQMax);                      // [2]
+    uint32_t* const pbuf0 = reinterpret_cast<uint32_t*>(wb);
+    uint32_t* const pbuf1 = reinterpret_cast<uint32_t*>(wb + kPlaneBufBytes);
+    uint16_t* surv = reinterpret_cast<uint16_t*>(wb + 2 * kPlaneBufBytes);              // [kWarpItems]
+    uint32_t* s_pass = reinterpret_cast<uint32_t*>(surv + kWarpItems);                   // [kQMax][16]
+    int4* s_q = reinterpret_cast<int4*>(s_pass + kQMax * 16);                            // [kQMax][np]
+    uint8_t* s_tab = reinterpret_cast<uint8_t*>(s_q) + size_t(kQMax) * d;                // [2][128]
+    int32_t* s_qid = reinterpret_cast<int32_t*>(s_tab + 2 * kMaskBitsMax);               // [kQMax]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s_qid + kQMax);                         // [2]
 
     if (lane == 0) {
         mbar_init(&bars[0], 1);
@@ -99,55 +128,71 @@ scan_kernel(SearchArgs a)
     }
     __syncwarp();
 
-    const int n_units = a.ctl->n_units;
+    const int n_units = a.ctl->n_units < a.max_units ? a.ctl->n_units : a.max_units;
     const int stride = gridDim.x * (kScanBlock / 32);
     int u = blockIdx.x * (kScanBlock / 32) + warp;
     if (u >= n_units) return;
 
-    // prologue: copies for the first two units, slots of the first
+    // unit entry: {first row, chunk, first query slot, rows << 16 | queries}
+    auto load_slots = [&](const int4& e, int& qid, uint64_t& m0, uint64_t& m1) {
+        qid = 0;
+        m0 = 0;
+        m1 = 0;
+        if (lane < (e.w & 0xFFFF)) {
+            qid = a.qlist[e.z + lane];
+            const ulonglong2 m = reinterpret_cast<const ulonglong2*>(a.qmask_slot)[e.z + lane];
+            m0 = m.x;
+            m1 = m.y;
+        }
+    };
+
+    // prologue: entries of the first three units, slots of the first two,
+    // planes of the first two
     int4 e_cur = a.units[u];
-    int4 e_nxt = make_int4(0, 0, 0, 0);
+    int4 e_nxt = make_int4(0, 0, 0, 0), e_n2 = make_int4(0, 0, 0, 0);
     const bool has_nxt0 = u + stride < n_units;
     if (has_nxt0) e_nxt = a.units[u + stride];
-    if (lane == 0) {
-        issue_sig_copy<W>(a, e_cur, sbuf0, &bars[0]);
-        if (has_nxt0) issue_sig_copy<W>(a, e_nxt, sbuf1, &bars[1]);
+    if (u + 2 * stride < n_units) e_n2 = a.units[u + 2 * stride];
+    int qid_c, qid_n = 0;
+    uint64_t m0_c, m1_c, m0_n = 0, m1_n = 0;
+    load_slots(e_cur, qid_c, m0_c, m1_c);
+    if (has_nxt0) load_slots(e_nxt, qid_n, m0_n, m1_n);
+    uint32_t fits = 0;  // bit b: buffer b holds its unit's planes (else read them from global)
+    {
+        uint64_t x = m0_c, y = m1_c;
+        warp_or2(x, y);
+        if (issue_planes<W>(a, e_cur.y, x, y, pbuf0, s_tab, &bars[0], lane)) fits |= 1u;
     }
-    int qid_c = 0;
-    uint64_t m0_c = 0, m1_c = 0;
-    if (lane < e_cur.w) {
-        qid_c = a.qlist[e_cur.z + lane];
-        m0_c = a.qmask_slot[2 * int64_t(e_cur.z + lane)];
-        m1_c = a.qmask_slot[2 * int64_t(e_cur.z + lane) + 1];
+    if (has_nxt0) {
+        uint64_t x = m0_n, y = m1_n;
+        warp_or2(x, y);
+        if (issue_planes<W>(a, e_nxt.y, x, y, pbuf1, s_tab + kMaskBitsMax, &bars[1], lane)) fits |= 2u;
     }
-    uint32_t phase = 0;   // bit b: parity to wait for on buffer b
-    uint32_t pending = has_nxt0 ? 3u : 1u;  // bit b: a copy into buffer b is in flight
+    uint32_t phase = 0;                      // bit b: parity to wait for on buffer b
+    uint32_t pending = has_nxt0 ? 3u : 1u;   // bit b: a copy into buffer b is in flight
     int b = 0;
 
     for (; u < n_units; u += stride) {
         const int64_t ib = e_cur.x;
-        const int len = e_cur.y;
-        const int qn = e_cur.w;
-        unsigned char* sb = b ? sbuf1 : sbuf0;
-        const bool has_nxt = u + stride < n_units;
+        const int chunk = e_cur.y;
+        const int len = e_cur.w >> 16;
+        const int qn = e_cur.w & 0xFFFF;
+        uint32_t* pb = b ? pbuf1 : pbuf0;
+        const uint8_t* tab = s_tab + b * kMaskBitsMax;
+        const bool in_smem = (fits >> b) & 1u;
         const bool has_n2 = u + 2 * stride < n_units;
+        const bool has_n3 = u + 3 * stride < n_units;
 
-        // background loads for later units: entry two ahead, slots one ahead
-        int4 e_n2 = make_int4(0, 0, 0, 0);
-        if (has_n2) e_n2 = a.units[u + 2 * stride];
-        int qid_n = 0;
-        uint64_t m0_n = 0, m1_n = 0;
-        if (has_nxt && lane < e_nxt.w) {
-            qid_n = a.qlist[e_nxt.z + lane];
-            m0_n = a.qmask_slot[2 * int64_t(e_nxt.z + lane)];
-            m1_n = a.qmask_slot[2 * int64_t(e_nxt.z + lane) + 1];
-        }
+        // background loads: the entry three units ahead, the slots of the unit
+        // two ahead (whose entry arrived during the previous unit)
+        int4 e_n3 = make_int4(0, 0, 0, 0);
+        if (has_n3) e_n3 = a.units[u + 3 * stride];
+        int qid_2 = 0;
+        uint64_t m0_2 = 0, m1_2 = 0;
+        if (has_n2) load_slots(e_n2, qid_2, m0_2, m1_2);
 
-        // query ids and masks of this unit -> shared memory; vectors by cp.async
-        if (lane < qn) {
-            s_qid[lane] = qid_c;
-            s_m[lane] = make_ulonglong2(m0_c, m1_c);
-        }
+        // query ids of this unit -> shared memory; vectors by cp.async
+        if (lane < qn) s_qid[lane] = qid_c;
         __syncwarp();
         for (int idx = lane; idx < qn * np; idx += 32) {
             const int s = idx / np, p = idx - s * np;
@@ -155,7 +200,7 @@ scan_kernel(SearchArgs a)
         }
         cp_async_commit();
 
-        // wait for this unit's signatures
+        // wait for this unit's planes
         const bool ok = mbar_wait_bounded(&bars[b], (phase >> b) & 1u);
         if (!__all_sync(0xffffffffu, ok)) {
             if (lane == 0) set_error(a.err, kErrCopyTimeout);
@@ -164,87 +209,92 @@ scan_kernel(SearchArgs a)
         phase ^= 1u << b;
         pending &= ~(1u << b);
 
-        // test every row against every query of the unit: bit s of em[j] is set
-        // when row lane+32j carries every bit of query s's mask
-        uint32_t em[IPL];
-        const int off1 = (W == 1) ? int(ib & 1) : 0;
-#pragma unroll
-        for (int j = 0; j < IPL; ++j) {
-            const int t = lane + 32 * j;
-            uint32_t e = 0;
-            if (t < len) {
-                if (W == 2) {
-                    const ulonglong2 v = reinterpret_cast<const ulonglong2*>(sb)[t];
-                    for (int s = 0; s < qn; ++s) {
-                        const ulonglong2 m = s_m[s];
-                        const uint64_t miss = (~v.x & m.x) | (~v.y & m.y);
-                        e |= uint32_t(miss == 0ull) << s;
-                    }
-                } else {
-                    const uint64_t v = reinterpret_cast<const uint64_t*>(sb)[off1 + t];
-                    for (int s = 0; s < qn; ++s) {
-                        const uint64_t m = s_m[s].x;
-                        e |= uint32_t((~v & m) == 0ull) << s;
-                    }
-                }
+        // test: pass word of query s for block `blk` = AND of its mask planes;
+        // the two half-warps take halves of the query's precomputed bit list
+        const uint32_t valid = len >= 32 * (blk + 1) ? 0xFFFFFFFFu
+                             : (len <= 32 * blk ? 0u : ((1u << (len - 32 * blk)) - 1u));
+        const uint32_t* gpl = a.planes + int64_t(chunk) * NPL * 16 + blk;
+        uint32_t any = 0;
+        uint32_t mycnt = 0;  // lane s: survivors of query s
+        for (int s = 0; s < qn; ++s) {
+            const int qg = s_qid[s];
+            const int nb = __ldg(a.qnbits + qg);
+            const int h0 = (nb + 1) >> 1;
+            const uint8_t* bits = a.qbits + int64_t(qg) * kMaskBitsMax;
+            const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
+            uint32_t acc = 0xFFFFFFFFu;
+            if (in_smem) {
+                for (int j = j0; j < j1; ++j) acc &= pb[tab[__ldg(bits + j)] * 16 + blk];
+            } else {
+                for (int j = j0; j < j1; ++j) acc &= __ldg(gpl + __ldg(bits + j) * 16);
             }
-            em[j] = e;
+            acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
+            acc &= valid;
+            if (half == 0) s_pass[s * 16 + blk] = acc;
+            any |= acc;
+            // survivors of query s: half 0 holds the 16 pass words; the full
+            // 32-lane reduction leaves the total in every lane
+            uint32_t c = half == 0 ? uint32_t(__popc(acc)) : 0u;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+            if (lane == s) mycnt = c;
         }
 
-        // compact the survivors into this unit's (now consumed) signature buffer
-        __syncwarp();
-        uint64_t* surv = reinterpret_cast<uint64_t*>(sb);
-        int nsurv = 0;
-#pragma unroll
-        for (int j = 0; j < IPL; ++j) {
-            const unsigned bal = __ballot_sync(0xffffffffu, em[j] != 0u);
-            if (em[j]) surv[nsurv + __popc(bal & lanemask_lt())] = (uint64_t(lane + 32 * j) << 32) | em[j];
-            nsurv += __popc(bal);
-        }
-        cp_async_wait_all();
-        __syncwarp();
-
-        // survivors per query (lane s counts query s) -> one reservation each
-        uint32_t mycnt = 0;
-        for (int c0 = 0; c0 < nsurv; c0 += 32) {
-            const uint32_t e = (c0 + lane < nsurv) ? uint32_t(surv[c0 + lane]) : 0u;
-            for (int s = 0; s < qn; ++s) {
-                const uint32_t ns = __popc(__ballot_sync(0xffffffffu, (e >> s) & 1u));
-                if (lane == s) mycnt += ns;
-            }
-        }
+        // per-query survivor counts -> one reservation each (lane s)
         uint32_t base = 0;
         if (lane < qn && mycnt) {
             base = atomicAdd(&a.cand_cnt[qid_c], mycnt);
             atomicAdd(&a.eligible_cnt[qid_c], (unsigned long long)mycnt);
         }
 
+        // survivor row offsets, block by block
+        const uint32_t mine = half == 0 ? uint32_t(__popc(any)) : 0u;
+        uint32_t incl = mine;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += t;
+        }
+        const int nsurv = int(__shfl_sync(0xffffffffu, incl, 31));
+        if (half == 0) {
+            int pos = int(incl - mine);
+            uint32_t rest = any;
+            while (rest) {
+                const int i = __ffs(rest) - 1;
+                rest &= rest - 1u;
+                surv[pos++] = uint16_t(32 * blk + i);
+            }
+        }
+        cp_async_wait_all();
+        __syncwarp();
+
         // rows of the survivors (one load per survivor), dots, keys into the
-        // reserved slots; a key's slot is its rank among this unit's survivors
-        // of the same query (ballot prefix), so no shared atomics are needed
+        // reserved slots; a key's slot is its ballot rank among this unit's
+        // survivors of the same query
         uint32_t run = 0;  // lane s: keys of query s written so far
         for (int c0 = 0; c0 < nsurv; c0 += 32) {
             const int idx = c0 + lane;
-            uint32_t e = 0;
+            int off = -1;
             int64_t i = 0;
             int4 row[NP > 0 ? NP : 1];
             const int4* rp = nullptr;
             if (idx < nsurv) {
-                const uint64_t sv = surv[idx];
-                e = uint32_t(sv);
-                i = ib + int64_t(sv >> 32);
+                off = surv[idx];
+                i = ib + off;
                 rp = reinterpret_cast<const int4*>(a.items + i * d);
                 if (NP > 0) {
 #pragma unroll
                     for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
                 }
             }
+            const uint32_t* pw = s_pass + (off >= 0 ? (off >> 5) : 0);
+            const int bit = off & 31;
             for (int s = 0; s < qn; ++s) {
-                const bool mine = (e >> s) & 1u;
-                const unsigned bal = __ballot_sync(0xffffffffu, mine);
+                const bool on = off >= 0 && ((pw[s * 16] >> bit) & 1u);
+                const unsigned bal = __ballot_sync(0xffffffffu, on);
                 if (bal == 0u) continue;
                 const uint32_t slot0 = __shfl_sync(0xffffffffu, base, s) + __shfl_sync(0xffffffffu, run, s);
-                if (mine) {
+                if (on) {
                     const int4* qs = s_q + s * np;
                     int32_t acc0 = 0, acc1 = 0;
                     if (NP > 0) {
@@ -257,8 +307,10 @@ scan_kernel(SearchArgs a)
                         for (int p = 0; p < np; ++p) acc0 = dot16(__ldg(rp + p), qs[p], acc0);
                     }
                     const uint64_t pos = uint64_t(slot0) + __popc(bal & lanemask_lt());
-                    if (pos < uint64_t(a.cap))
-                        a.cand[int64_t(s_qid[s]) * a.cap + int64_t(pos)] = pack_key(acc0 + acc1, uint32_t(i));
+                    const int32_t score = acc0 + acc1;
+                    const int qg = s_qid[s];
+                    if (pos < uint64_t(a.cap)) a.cand[int64_t(qg) * a.cap + int64_t(pos)] = pack_key(score, uint32_t(i));
+                    atomicAdd(&a.hist[int64_t(qg) * kHistBins + score_bin(score, a.smax, a.hshift)], 1u);
                 }
                 if (lane == s) run += __popc(bal);
             }
@@ -266,14 +318,23 @@ scan_kernel(SearchArgs a)
         fence_proxy_async_smem();
         __syncwarp();
 
-        // buffer b is free: start the copy for the unit two ahead
-        if (has_n2 && lane == 0) issue_sig_copy<W>(a, e_n2, sb, &bars[b]);
-        if (has_n2) pending |= 1u << b;
+        // buffer b is free: start the planes of the unit two ahead
+        if (has_n2) {
+            uint64_t x = m0_2, y = m1_2;
+            warp_or2(x, y);
+            if (issue_planes<W>(a, e_n2.y, x, y, pb, s_tab + b * kMaskBitsMax, &bars[b], lane)) fits |= 1u << b;
+            else fits &= ~(1u << b);
+            pending |= 1u << b;
+        }
         e_cur = e_nxt;
         e_nxt = e_n2;
+        e_n2 = e_n3;
         qid_c = qid_n;
         m0_c = m0_n;
         m1_c = m1_n;
+        qid_n = qid_2;
+        m0_n = m0_2;
+        m1_n = m1_2;
         b ^= 1;
     }
 

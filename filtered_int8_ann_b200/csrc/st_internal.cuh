@@ -20,9 +20,12 @@ constexpr int kProbeSmemKeys = 16384;      // nlist up to this keeps probe keys 
 constexpr int kSelectBlock = 1024;
 constexpr int kSelectSmemKeys = 22528;     // candidates up to this are selected in smem
 constexpr int kPlanBlock = 512;
+constexpr int kHistBins = 2048;            // per-query score histogram bins
+constexpr int kMaskBitsMax = 128;          // signature bits
 constexpr int kSelBits = 11;               // radix digit of the selections
 constexpr int kSelBins = 1 << kSelBits;
-constexpr uint32_t kWaitLimit = 1u << 24;  // bounded mbarrier polls before giving up
+constexpr uint32_t kWaitLimit = 1u << 10;  // bounded mbarrier polls before giving up
+constexpr uint32_t kWaitHintNs = 10000000u; // each poll may sleep up to 10 ms waiting for the phase
 
 // Device error word bits (st_index_check reports any of them as ST_ERR_DEVICE).
 enum : uint32_t {
@@ -58,7 +61,7 @@ __host__ __device__ __forceinline__ int64_t key_id(uint64_t key)
 // Per-search state
 // ----------------------------------------------------------------------------
 struct PlanCtl {
-    int32_t n_units;       // work units of this search
+    int32_t n_units;       // work units allocated by the plan (clamped to the table by the scan)
     int32_t pad[3];
 };
 
@@ -66,8 +69,11 @@ struct SearchArgs {
     // index (read-only)
     const int8_t* items;
     const uint64_t* sigs;
+    const uint32_t* planes;      // [n_chunks][64W][16] signature bit-planes per list chunk
     const int64_t* offsets;
-    const int32_t* nchunks;  // [nlist] ceil(list rows / kWarpItems)
+    const int32_t* chunk_start;  // [nlist+1] first chunk of each list (chunks of kWarpItems rows)
+    const int32_t* chunk_list;   // [n_chunks] list of each chunk
+    int32_t n_chunks;
     const int8_t* centroids;
     int32_t d, nlist, W;
     // request
@@ -79,20 +85,26 @@ struct SearchArgs {
     int32_t* out_scores;
     int64_t* out_eligible;   // may be null
     // scratch (the zeroed block first: one memset clears it)
-    int32_t* list_cnt;       // [nlist] queries probing each list        (zeroed)
-    int32_t* list_fill;      // [nlist] scatter cursor                    (zeroed)
+    int32_t* list_cnt;       // [nlist] queries filed into each list      (zeroed)
+    int32_t* probe_done;     // [B] probe slices finished per query       (zeroed)
     uint32_t* cand_cnt;      // [B] candidates reserved per query         (zeroed)
     unsigned long long* eligible_cnt;  // [B]                             (zeroed)
-    PlanCtl* ctl;            //                                           (zeroed)
+    uint32_t* hist;          // [B][kHistBins] emitted-key score histogram (zeroed)
+    PlanCtl* ctl;            // unit allocation counter                   (zeroed)
     int32_t* probe;          // [B][P]
-    uint64_t* probe_keys;    // [B][nlist] when nlist > kProbeSmemKeys, else null
-    int32_t* list_qstart;    // [nlist] first query slot of each list
-    int32_t* qlist;          // [B*P] query id of each slot (slots grouped by list)
-    uint64_t* qmask_slot;    // [B*P][2] that query's mask words (word 1 = 0 when W = 1)
-    int4* units;             // [max_units] {first row, rows, first slot, queries}
+    uint64_t* probe_keys;    // [B][nlist] when a probe slice does not fit shared memory, else null
+    uint64_t* probe_part;    // [B][S][P] best keys of each probe slice
+    int32_t* list_ustart;    // [nlist] first unit of each probed list
+    int32_t* qlist;          // [nlist][B] slot row of each list: ids of the queries probing it
+    uint64_t* qmask_slot;    // [nlist][B][2] that query's mask words (word 1 = 0 when W = 1)
+    uint8_t* qbits;          // [B][kMaskBitsMax] each query's mask bits, in increasing order
+    int32_t* qnbits;         // [B] number of mask bits of each query
+    int4* units;             // [max_units] {first row, chunk, first slot, rows << 16 | queries}
     int32_t max_units;
     uint64_t* cand;          // [B][cap]
     int64_t cap;             // candidate keys per query
+    int32_t smax;            // largest possible |score|: d * 128 * 128
+    int32_t hshift;          // histogram bin = min(kHistBins-1, (score + smax) >> hshift)
     uint32_t* err;           // device error word
 };
 
@@ -109,6 +121,13 @@ __device__ __forceinline__ int32_t dot16(const int4 a, const int4 b, int32_t acc
 }
 
 __device__ __forceinline__ void set_error(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
+
+// Histogram bin of a score: monotone non-decreasing in the score.
+__device__ __forceinline__ uint32_t score_bin(int32_t score, int32_t smax, int32_t hshift)
+{
+    const uint32_t b = uint32_t(score + smax) >> hshift;
+    return b < uint32_t(kHistBins) ? b : uint32_t(kHistBins - 1);
+}
 
 __device__ __forceinline__ unsigned lanemask_lt()
 {
@@ -147,14 +166,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
         : "memory");
     return ok != 0;
 }
-// Poll the barrier phase at most kWaitLimit times; false if it never completed.
+// Poll the barrier phase at most kWaitLimit times (each poll suspends the
+// thread until the phase completes or the hint expires); false if it never
+// completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity)
 {
     for (uint32_t it = 0; it < kWaitLimit; ++it)
@@ -182,6 +203,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // ----------------------------------------------------------------------------
 struct SelectSmem {
     uint32_t hist[kSelBins];
+    uint32_t hist2[kSelBins];
     uint32_t part[32];
     unsigned long long red_lo[32], red_hi[32];
     uint64_t prefix;     // high bits of the threshold fixed so far
@@ -190,16 +212,8 @@ struct SelectSmem {
     int32_t done;
     int32_t found;
     int32_t count;
+    uint32_t lo32, hi32, maxcnt;
 };
-
-// Warp-aggregated shared histogram increment. Every lane of the warp calls it.
-__device__ __forceinline__ void hist_add(uint32_t* hist, bool active, uint32_t bin)
-{
-    const unsigned act = __ballot_sync(0xffffffffu, active);
-    if (!active) return;
-    const unsigned peers = __match_any_sync(act, bin);
-    if (int(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
-}
 
 // Block exclusive scan of one value per thread; `total` gets the block sum.
 template <int BLOCK>
@@ -233,9 +247,10 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* part, 
 
 // A threshold T such that exactly k of the n unique keys are >= T (1 <= k <= n).
 // MSB-first radix select restricted to the bits where the keys differ (the
-// score's high bits are shared by all candidates), 11-bit digits, warp-
-// aggregated histogram updates, and an early exit as soon as the bucket holding
-// the k-th key is taken whole. `keys` may be shared or global memory.
+// score's high bits are shared by all candidates), 11-bit digits (2048 shared
+// bins, so plain shared atomics rarely collide), and an early exit as soon as
+// the bucket holding the k-th key is taken whole. `keys` may be shared or
+// global memory.
 template <int BLOCK>
 __device__ uint64_t block_select_threshold(const uint64_t* keys, int64_t n, int64_t k, SelectSmem& s,
                                            uint32_t* err)
@@ -289,16 +304,10 @@ __device__ uint64_t block_select_threshold(const uint64_t* keys, int64_t n, int6
         const uint64_t prefix = s.prefix;
         for (int i = tid; i < nb; i += BLOCK) s.hist[i] = 0;
         __syncthreads();
-        for (int64_t base = 0; base < n; base += BLOCK) {
-            const int64_t i = base + tid;
-            bool act = false;
-            uint32_t bin = 0;
-            if (i < n) {
-                const uint64_t x = keys[i];
-                act = shift_hi >= 64 || (x >> shift_hi) == (prefix >> shift_hi);
-                bin = uint32_t(x >> shift) & uint32_t(nb - 1);
-            }
-            hist_add(s.hist, act, bin);
+        for (int64_t i = tid; i < n; i += BLOCK) {
+            const uint64_t x = keys[i];
+            if (shift_hi >= 64 || (x >> shift_hi) == (prefix >> shift_hi))
+                atomicAdd(&s.hist[uint32_t(x >> shift) & uint32_t(nb - 1)], 1u);
         }
         __syncthreads();
         // thread t owns `per` bins counted down from the top bin
@@ -340,6 +349,48 @@ __device__ uint64_t block_select_threshold(const uint64_t* keys, int64_t n, int6
     return s.prefix;
 }
 
+// block_collect_ge for a long 16-byte-aligned key array in global memory: each
+// thread keeps eight keys (four 16-byte loads) in flight per step.
+template <int BLOCK>
+__device__ int32_t block_collect_ge_wide(const uint64_t* keys, int64_t n, uint64_t thr, uint64_t* out,
+                                         int32_t out_cap, SelectSmem& s)
+{
+    if (threadIdx.x == 0) s.count = 0;
+    __syncthreads();
+    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
+    const int64_t n2 = n >> 1;
+    for (int64_t base = 0; base < n2; base += int64_t(BLOCK) * 4) {
+        ulonglong2 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t j = base + u * BLOCK + threadIdx.x;
+            v[u] = j < n2 ? __ldcg(k2 + j) : make_ulonglong2(0ull, 0ull);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint64_t key = (u & 1) ? v[u >> 1].y : v[u >> 1].x;
+            const bool take = key >= thr && key != 0ull;
+            const unsigned bal = __ballot_sync(0xffffffffu, take);
+            if (bal) {
+                int32_t b0 = 0;
+                if ((threadIdx.x & 31) == 0) b0 = atomicAdd(&s.count, __popc(bal));
+                b0 = __shfl_sync(0xffffffffu, b0, 0);
+                const int32_t pos = b0 + __popc(bal & lanemask_lt());
+                if (take && pos < out_cap) out[pos] = key;
+            }
+        }
+    }
+    if ((n & 1) && threadIdx.x == 0) {
+        const uint64_t key = keys[n - 1];
+        if (key >= thr && key != 0ull) {
+            const int32_t pos = atomicAdd(&s.count, 1);
+            if (pos < out_cap) out[pos] = key;
+        }
+    }
+    __syncthreads();
+    return s.count;
+}
+
 // Copy every key >= thr from keys[0..n) into out[] (at most out_cap); returns
 // how many keys were >= thr.
 template <int BLOCK>
@@ -369,13 +420,19 @@ __device__ int32_t block_collect_ge(const uint64_t* keys, int64_t n, uint64_t th
     return s.count;
 }
 
-// Sort m keys (m a power of two) in shared memory, descending.
+// Sort a[0..m) descending with a bitonic network in shared memory (the keys
+// are padded with zeros to a power of two; `a` needs room for next_pow2(m)
+// keys). Compact and slow; the counting sort below uses it only as a fallback.
 template <int BLOCK>
 __device__ void block_bitonic_desc(uint64_t* a, int m)
 {
-    for (int size = 2; size <= m; size <<= 1) {
+    int mm = 1;
+    while (mm < m) mm <<= 1;
+    for (int i = m + threadIdx.x; i < mm; i += BLOCK) a[i] = 0;
+    __syncthreads();
+    for (int size = 2; size <= mm; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = threadIdx.x; i < (m >> 1); i += BLOCK) {
+            for (int i = threadIdx.x; i < (mm >> 1); i += BLOCK) {
                 const int lo = 2 * i - (i & (stride - 1));
                 const int hi = lo + stride;
                 const bool desc = (lo & size) == 0;
@@ -388,6 +445,101 @@ __device__ void block_bitonic_desc(uint64_t* a, int m)
             __syncthreads();
         }
     }
+}
+
+// Sort a[0..m) descending, exactly, by counting: a histogram of the keys' high
+// words (the biased scores) over kSelBins bins spanning their range gives each
+// bin its output segment (keys of higher bins come first); keys are scattered
+// into their segments in `tmp`, and each key's place inside its segment is the
+// number of keys of the segment greater than it (keys are unique). The segments
+// of a top-k are short; when one holds more than 64 keys (for example many
+// equal scores) the bitonic network is used instead, which needs room for
+// next_pow2(m) keys in `a`. `tmp` needs m keys.
+template <int BLOCK>
+__device__ void block_sort_desc_counting(uint64_t* a, int m, uint64_t* tmp, SelectSmem& s)
+{
+    constexpr int NW = BLOCK / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (m <= 1) {
+        __syncthreads();
+        return;
+    }
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int i = tid; i < m; i += BLOCK) {
+        const uint32_t h = uint32_t(a[i] >> 32);
+        lo = h < lo ? h : lo;
+        hi = h > hi ? h : hi;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+        s.red_lo[warp] = lo;
+        s.red_hi[warp] = hi;
+    }
+    for (int i = tid; i < kSelBins; i += BLOCK) {
+        s.hist[i] = 0;
+        s.hist2[i] = 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t l = 0xFFFFFFFFu, h = 0u;
+        for (int w = 0; w < NW; ++w) {
+            l = min(l, uint32_t(s.red_lo[w]));
+            h = max(h, uint32_t(s.red_hi[w]));
+        }
+        s.lo32 = l;
+        s.hi32 = h;
+        s.maxcnt = 0;
+    }
+    __syncthreads();
+    const uint32_t base = s.lo32;
+    int shift = 0;
+    while (((s.hi32 - base) >> shift) >= uint32_t(kSelBins)) ++shift;
+    for (int i = tid; i < m; i += BLOCK) atomicAdd(&s.hist[(uint32_t(a[i] >> 32) - base) >> shift], 1u);
+    __syncthreads();
+    // descending exclusive scan: start of bin b = keys in bins above b
+    constexpr int PER = kSelBins / BLOCK > 0 ? kSelBins / BLOCK : 1;
+    const int owners = kSelBins / PER;
+    uint32_t local = 0, mx = 0;
+    if (tid < owners)
+        for (int j = 0; j < PER; ++j) {
+            const uint32_t c = s.hist[kSelBins - 1 - (tid * PER + j)];
+            local += c;
+            mx = c > mx ? c : mx;
+        }
+    uint32_t total;
+    uint32_t run = block_excl_scan<BLOCK>(local, s.part, total);
+    if (tid < owners)
+        for (int j = 0; j < PER; ++j) {
+            const int bin = kSelBins - 1 - (tid * PER + j);
+            s.hist2[bin] = run;
+            run += s.hist[bin];
+        }
+    if (mx > 64) atomicMax(&s.maxcnt, mx);
+    __syncthreads();
+    if (s.maxcnt > 64) {
+        block_bitonic_desc<BLOCK>(a, m);
+        return;
+    }
+    for (int i = tid; i < m; i += BLOCK) {
+        const uint64_t key = a[i];
+        const uint32_t bin = (uint32_t(key >> 32) - base) >> shift;
+        tmp[atomicAdd(&s.hist2[bin], 1u)] = key;
+    }
+    __syncthreads();
+    for (int p = tid; p < m; p += BLOCK) {
+        const uint64_t key = tmp[p];
+        const uint32_t bin = (uint32_t(key >> 32) - base) >> shift;
+        const int end = int(s.hist2[bin]);
+        const int beg = end - int(s.hist[bin]);
+        int r = 0;
+        for (int j = beg; j < end; ++j) r += tmp[j] > key ? 1 : 0;
+        a[beg + r] = key;
+    }
+    __syncthreads();
 }
 
 __host__ __device__ __forceinline__ int next_pow2(int v)
@@ -404,10 +556,14 @@ cudaError_t ensure_smem_attr(const void* func, int slot, int bytes);
 // ----------------------------------------------------------------------------
 // Kernel launchers (defined in the .cu files)
 // ----------------------------------------------------------------------------
-cudaError_t launch_probe(const SearchArgs& a, cudaStream_t s);
+int probe_slices(const SearchArgs& a, int num_sms);
+cudaError_t launch_probe(const SearchArgs& a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const SearchArgs& a, cudaStream_t s);
 size_t scan_smem_bytes(int d, int W);
+cudaError_t launch_build_planes(const uint64_t* sigs, const int64_t* offsets, const int32_t* chunk_start,
+                                const int32_t* chunk_list, int32_t n_chunks, int W, uint32_t* planes,
+                                cudaStream_t s);
 
 }  // namespace st
