@@ -153,29 +153,52 @@ def make_data(args, world, rank):
     return wl.with_(B=B), data, q, m
 
 
+CHUNK_ROWS = 512  # rows per signature bit-plane chunk in the index
+
+
 def byte_model(data, probe, qmasks, W, d):
-    """Algorithmic bytes of one search's list scan: 8W bytes of signature for
-    every row of every distinct probed list, plus d bytes for every row that is
-    eligible for at least one query probing its list. Also the full-scan bytes
-    (every row of every distinct probed list)."""
+    """Algorithmic bytes of one search's list scan, for the index layout the
+    library uses: every probed list is read once per batch; its signatures are
+    stored as bit-planes per 512-row chunk (64 bytes per plane), and the scan
+    needs, per chunk, the planes of the bits set in the union of the masks of
+    the queries probing the list; a row (d bytes) is read only when it is
+    eligible for at least one of those queries.
+    Also returned: the same model with row-major signatures (8W bytes for every
+    scanned row, the earlier layout) and the full-scan bytes (every row and
+    signature of every distinct probed list)."""
     off = data.offsets
     sizes = (off[1:] - off[:-1])
     lists = torch.unique(probe.flatten())
     scanned = int(sizes[lists].sum())
+    # union of the masks of the queries probing each list
+    pr = probe.long().cpu().numpy()
+    mk = qmasks.cpu().numpy().view(np.uint64).reshape(qmasks.shape[0], -1)
+    nl = int(sizes.numel())
+    union = np.zeros((nl, mk.shape[1]), dtype=np.uint64)
+    for w in range(mk.shape[1]):
+        np.bitwise_or.at(union[:, w], pr.reshape(-1), np.repeat(mk[:, w], pr.shape[1]))
+    ls = lists.cpu().numpy()
+    bits = np.zeros(ls.size, dtype=np.int64)
+    for w in range(mk.shape[1]):
+        u = union[ls, w]
+        bits += np.array([bin(int(x)).count("1") for x in u], dtype=np.int64)
+    chunks = (sizes[lists].cpu().numpy() + CHUNK_ROWS - 1) // CHUNK_ROWS
+    plane_bytes = int((chunks * bits * (CHUNK_ROWS // 8)).sum())
     surv = torch.zeros(data.items.shape[0], dtype=torch.bool, device=off.device)
     for b in range(probe.shape[0]):
-        ls = probe[b].long()
-        starts, lens = off[ls], sizes[ls]
+        lsb = probe[b].long()
+        starts, lens = off[lsb], sizes[lsb]
         idx = torch.repeat_interleave(starts - torch.cumsum(lens, 0) + lens, lens) + torch.arange(
             int(lens.sum()), device=off.device)
-        s = data.sigs[idx]
-        mk = qmasks[b].view(1, -1)
-        ok = torch.all((s & mk) == mk, dim=1)
+        sg = data.sigs[idx]
+        m = qmasks[b].view(1, -1)
+        ok = torch.all((sg & m) == m, dim=1)
         surv[idx[ok]] = True
     n_surv = int(surv.sum())
-    method = 8 * W * scanned + d * n_surv
+    method = plane_bytes + d * n_surv
+    rowmajor = 8 * W * scanned + d * n_surv
     full = (8 * W + d) * scanned
-    return method, full, scanned, n_surv, int(lists.numel())
+    return method, full, scanned, n_surv, int(lists.numel()), rowmajor, plane_bytes
 
 
 def cpu_baseline(data, q, m, wl, budget_s):
@@ -357,6 +380,8 @@ def main():
                          "unit": "GB/s", "frac": scan_gbs / peak, "traffic": None,
                          "peak_kind": peak_kind,
                          "bytes_per_launch": float(method_bytes.mean()),
+                         "signature_plane_bytes_per_launch": float(np.mean([x[6] for x in models])),
+                         "rowmajor_model_bytes_per_launch": float(np.mean([x[5] for x in models])),
                          "full_scan_bytes_per_launch": float(full_bytes.mean()),
                          "step_frac": float(method_bytes.mean() / (ms / K * 1e-3) / 1e9 / peak)},
             "cpu_baseline": cpu,

@@ -222,9 +222,17 @@ scan_kernel(SearchArgs a)
             const int h0 = (nb + 1) >> 1;
             const uint8_t* bits = a.qbits + int64_t(qg) * kMaskBitsMax;
             const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
+            // four independent bit -> slot -> plane chains per step
             uint32_t acc = 0xFFFFFFFFu;
             if (in_smem) {
-                for (int j = j0; j < j1; ++j) acc &= pb[tab[__ldg(bits + j)] * 16 + blk];
+                int j = j0;
+                for (; j + 4 <= j1; j += 4) {
+                    const int b0 = __ldg(bits + j), b1 = __ldg(bits + j + 1);
+                    const int b2 = __ldg(bits + j + 2), b3 = __ldg(bits + j + 3);
+                    const int s0 = tab[b0], s1 = tab[b1], s2 = tab[b2], s3 = tab[b3];
+                    acc &= pb[s0 * 16 + blk] & pb[s1 * 16 + blk] & pb[s2 * 16 + blk] & pb[s3 * 16 + blk];
+                }
+                for (; j < j1; ++j) acc &= pb[tab[__ldg(bits + j)] * 16 + blk];
             } else {
                 for (int j = j0; j < j1; ++j) acc &= __ldg(gpl + __ldg(bits + j) * 16);
             }

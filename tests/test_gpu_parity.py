@@ -31,6 +31,13 @@ CASES = [
     # flat uniform
     dict(n=30000, d=128, nlist=1, sig_bits=128, hash_bits=3, B=2, nprobe=1, k=2048, seed=12,
          uniform_items=True, mask_flags=2),
+    # item-mode masks (language and country vary per query) and many queries per
+    # list: a unit's mask union exceeds the 32-plane buffer, so the scan tests
+    # from the global planes
+    dict(n=8000, d=64, nlist=3, sig_bits=128, hash_bits=3, B=60, nprobe=3, k=150, seed=15,
+         mask_mode="item", mask_country=True, mask_flags=2),
+    dict(n=8000, d=128, nlist=2, sig_bits=64, hash_bits=2, B=40, nprobe=2, k=90, seed=16,
+         mask_mode="item", mask_country=True, mask_flags=3),
     # k = 1 and k = 4096
     dict(n=9000, d=64, nlist=10, sig_bits=64, B=3, nprobe=10, k=1, seed=13),
     dict(n=9000, d=64, nlist=10, sig_bits=128, B=3, nprobe=10, k=4096, seed=14, mask_flags=0,
@@ -64,6 +71,16 @@ def test_parity_mid_ivf():
     data = generate(WORKLOADS["mid_ivf"])
     wl = data.wl
     assert_parity(run_gpu(data, wl.nprobe, wl.k), run_oracle(data, wl.nprobe, wl.k), "mid_ivf")
+
+
+def test_wide_mask_union_uses_global_planes():
+    """The unit-level union of 60 item-mode masks has more than 32 bits."""
+    data = small(n=8000, d=64, nlist=3, sig_bits=128, hash_bits=3, B=60, nprobe=3, k=150, seed=15,
+                 mask_mode="item", mask_country=True, mask_flags=2)
+    m = data.masks.numpy().view(np.uint64)
+    union = np.bitwise_or.reduce(m[:32], axis=0)
+    assert sum(bin(int(w)).count("1") for w in union) > 32
+    assert_parity(run_gpu(data, 3, 150), run_oracle(data, 3, 150), "wide union")
 
 
 def test_padding_when_few_eligible():
