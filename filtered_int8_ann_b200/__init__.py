@@ -17,13 +17,15 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libst.so")
 
-ST_OK, ST_ERR_INVALID_ARG, ST_ERR_UNSUPPORTED, ST_ERR_OOM, ST_ERR_CUDA, ST_ERR_DEVICE = range(6)
+(ST_OK, ST_ERR_INVALID_ARG, ST_ERR_UNSUPPORTED, ST_ERR_OOM, ST_ERR_CUDA, ST_ERR_DEVICE,
+ ST_ERR_SCRATCH_LIMIT) = range(7)
+ST_PROBE_NOALLOC_SCRATCH_BYTES = 16 << 20
 ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY = 1, 2
 ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE = 512, 4096, 4096
 
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
-           "st_index_set_option", "st_index_destroy", "st_status_string")
+           "st_index_set_option", "st_probe_noalloc", "st_index_destroy", "st_status_string")
 
 
 class StError(RuntimeError):
@@ -54,8 +56,9 @@ def lib() -> ctypes.CDLL:
     L.st_search_host.argtypes = [P, P, P, i32, i32, i32, P, P, P]
     L.st_index_check.argtypes = [P, P]
     L.st_index_set_option.argtypes = [P, ctypes.c_int, i64]
+    L.st_probe_noalloc.argtypes = [P, P, i32, i32, P, P]
     for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
-              "st_index_set_option"):
+              "st_index_set_option", "st_probe_noalloc"):
         getattr(L, f).restype = ctypes.c_int
     L.st_index_destroy.argtypes = [P]
     L.st_index_destroy.restype = None
@@ -168,6 +171,17 @@ def st_index_set_option(index: int, option: int, value: int):
     _check(lib().st_index_set_option(index, option, value), "st_index_set_option")
 
 
+def st_probe_noalloc(index: int, queries: torch.Tensor, nprobe: int, out_probe: torch.Tensor,
+                     stream=None) -> torch.Tensor:
+    """Probe-only call that allocates no device memory (its scratch is a fixed
+    array inside the library); `out_probe` is the caller's int32 [B, nprobe]
+    device tensor. Calls on one device share that array: keep them ordered."""
+    B = queries.shape[0]
+    _check(lib().st_probe_noalloc(index, _ptr(queries), B, nprobe, _ptr(out_probe), _stream(stream)),
+           "st_probe_noalloc")
+    return out_probe
+
+
 def st_index_destroy(index: Optional[int]):
     if index:
         lib().st_index_destroy(index)
@@ -186,6 +200,9 @@ class Index:
 
     def search_host(self, queries, qmasks, nprobe, k, **kw):
         return st_search_host(self.handle, queries, qmasks, nprobe, k, **kw)
+
+    def probe_noalloc(self, queries, nprobe, out_probe, stream=None):
+        return st_probe_noalloc(self.handle, queries, nprobe, out_probe, stream)
 
     def check(self, stream=None) -> int:
         return st_index_check(self.handle, stream)

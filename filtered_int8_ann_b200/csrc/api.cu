@@ -256,6 +256,7 @@ const char* st_status_string(st_status s)
     case ST_ERR_OOM: return "out of device memory";
     case ST_ERR_CUDA: return "CUDA error";
     case ST_ERR_DEVICE: return "device-side error recorded by a kernel";
+    case ST_ERR_SCRATCH_LIMIT: return "request needs more than the fixed scratch of the allocation-free call";
     }
     return "unknown status";
 }
@@ -430,6 +431,36 @@ st_status st_search_host(const st_index* idx, const int8_t* queries, const uint6
     if (e == cudaSuccess) e = ef;
     if (e == cudaSuccess) e = es;
     return cuda_status(e);
+}
+
+st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B, int32_t nprobe,
+                           int32_t* out_probe, cudaStream_t stream)
+{
+    if (idx == nullptr) return ST_ERR_INVALID_ARG;
+    if (B < 1 || nprobe < 1 || nprobe > idx->nlist) return ST_ERR_INVALID_ARG;
+    if (nprobe > ST_MAX_NPROBE || int64_t(B) * nprobe >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
+    DeviceGuard g(idx->device);
+    if (!is_device_ptr(queries, idx->device) || !is_device_ptr(out_probe, idx->device)) return ST_ERR_INVALID_ARG;
+    if (!aligned(queries, 16) || !aligned(out_probe, 4)) return ST_ERR_INVALID_ARG;
+    SearchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.centroids = idx->centroids;
+    a.d = idx->d;
+    a.nlist = idx->nlist;
+    a.W = idx->W;
+    a.queries = queries;
+    a.B = B;
+    a.P = nprobe;
+    a.probe = out_probe;
+    a.err = idx->err;
+    const int S = st::probe_slices(a, idx->num_sms);
+    const bool keys_in_smem = (idx->nlist + S - 1) / S + 1 <= st::kProbeSmemKeys;
+    if (st::probe_noalloc_scratch_bytes(B, S, nprobe, idx->nlist, keys_in_smem) > ST_PROBE_NOALLOC_SCRATCH_BYTES)
+        return ST_ERR_SCRATCH_LIMIT;
+    // any non-null value asks for the keys in global scratch; the launcher
+    // points it into the fixed array
+    a.probe_keys = keys_in_smem ? nullptr : reinterpret_cast<uint64_t*>(uintptr_t(1));
+    return cuda_status(st::launch_probe_noalloc(a, S, stream));
 }
 
 st_status st_index_check(const st_index* idx, cudaStream_t stream)

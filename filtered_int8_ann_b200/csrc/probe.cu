@@ -17,11 +17,15 @@
 // the S partial lists, writes the probe result, and files the query into every
 // chosen list: it takes the next rank of the list's query counter and writes
 // its id and mask into the list's slot row, which the plan and the scan read.
+#include <mutex>
+
 #include "st_internal.cuh"
 
 namespace st {
 
-template <int BLOCK>
+// kFile: also file the query into its lists (the search); the allocation-free
+// probe-only call sets it false and writes the probe result alone.
+template <int BLOCK, bool kFile>
 __device__ void finish_query(const SearchArgs& a, int b, uint64_t* keys, int n, uint64_t* sortbuf,
                              int pw, SelectSmem& ss)
 {
@@ -33,6 +37,10 @@ __device__ void finish_query(const SearchArgs& a, int b, uint64_t* keys, int n, 
     for (int i = (got < pw ? got : pw) + threadIdx.x; i < pw; i += BLOCK) sortbuf[i] = 0;
     __syncthreads();
     block_sort_desc_counting<BLOCK>(sortbuf, got < pw ? got : pw, keys, ss);  // the score keys are done with
+    if (!kFile) {
+        for (int p = threadIdx.x; p < P; p += BLOCK) a.probe[int64_t(b) * P + p] = int(key_id(sortbuf[p]));
+        return;
+    }
     const int W = a.W;
     // the query's mask bits in increasing order
     if (threadIdx.x < 32) {
@@ -64,7 +72,7 @@ __device__ void finish_query(const SearchArgs& a, int b, uint64_t* keys, int n, 
     }
 }
 
-template <int BLOCK>
+template <int BLOCK, bool kFile>
 __global__ void __launch_bounds__(BLOCK)
 probe_kernel(SearchArgs a, int S)
 {
@@ -117,7 +125,7 @@ probe_kernel(SearchArgs a, int S)
     __syncthreads();
 
     if (S == 1) {
-        finish_query<BLOCK>(a, b, keys, nloc, sortbuf, pw, ss);
+        finish_query<BLOCK, kFile>(a, b, keys, nloc, sortbuf, pw, ss);
         return;
     }
 
@@ -143,7 +151,7 @@ probe_kernel(SearchArgs a, int S)
     const uint64_t* src = a.probe_part + int64_t(b) * S * P;
     for (int i = threadIdx.x; i < n; i += BLOCK) mk[i] = __ldcg(src + i);
     __syncthreads();
-    finish_query<BLOCK>(a, b, mk, n, sortbuf, pw, ss);
+    finish_query<BLOCK, kFile>(a, b, mk, n, sortbuf, pw, ss);
 }
 
 int probe_slices(const SearchArgs& a, int num_sms)
@@ -170,9 +178,59 @@ static size_t probe_smem_bytes(const SearchArgs& a, int S)
 cudaError_t launch_probe(const SearchArgs& a, int S, cudaStream_t s)
 {
     const size_t smem = probe_smem_bytes(a, S);
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock>), 0, 200 * 1024);
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock, true>), 0, 200 * 1024);
     if (e != cudaSuccess) return e;
-    probe_kernel<kProbeBlock><<<a.B * S, kProbeBlock, smem, s>>>(a, S);
+    probe_kernel<kProbeBlock, true><<<a.B * S, kProbeBlock, smem, s>>>(a, S);
+    return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// Allocation-free probe (st_probe_noalloc). Its scratch -- the per-query
+// completion counters, the slices' partial top-P rows and, for very large
+// nlist, the centroid score keys -- lives in this fixed device array instead
+// of memory allocated per call. Every call uses the same array.
+// ----------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_probe_scratch[ST_PROBE_NOALLOC_SCRATCH_BYTES];
+
+size_t probe_noalloc_scratch_bytes(int B, int S, int P, int nlist, bool keys_in_smem)
+{
+    size_t bytes = (size_t(B) * 4 + 255) / 256 * 256;  // completion counters
+    bytes += size_t(B) * S * P * 8;                       // partial rows
+    if (!keys_in_smem) bytes += size_t(B) * nlist * 8;    // score keys
+    return bytes;
+}
+
+cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s)
+{
+    // device address of the array, looked up once per device
+    static std::mutex mu;
+    static unsigned char* base_of[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64) return cudaErrorInvalidDevice;
+    unsigned char* base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (base_of[dev] == nullptr) {
+            void* ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_probe_scratch);
+            if (e != cudaSuccess) return e;
+            base_of[dev] = static_cast<unsigned char*>(ptr);
+        }
+        base = base_of[dev];
+    }
+    const size_t done_bytes = (size_t(a.B) * 4 + 255) / 256 * 256;
+    a.probe_done = reinterpret_cast<int32_t*>(base);
+    a.probe_part = reinterpret_cast<uint64_t*>(base + done_bytes);
+    if (a.probe_keys != nullptr)  // non-null marks "keys in global memory"
+        a.probe_keys = reinterpret_cast<uint64_t*>(base + done_bytes + size_t(a.B) * S * a.P * 8);
+    e = cudaMemsetAsync(a.probe_done, 0, size_t(a.B) * 4, s);
+    if (e != cudaSuccess) return e;
+    const size_t smem = probe_smem_bytes(a, S);
+    e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock, false>), 9, 200 * 1024);
+    if (e != cudaSuccess) return e;
+    probe_kernel<kProbeBlock, false><<<a.B * S, kProbeBlock, smem, s>>>(a, S);
     return cudaGetLastError();
 }
 

@@ -558,6 +558,8 @@ cudaError_t ensure_smem_attr(const void* func, int slot, int bytes);
 // ----------------------------------------------------------------------------
 int probe_slices(const SearchArgs& a, int num_sms);
 cudaError_t launch_probe(const SearchArgs& a, int S, cudaStream_t s);
+size_t probe_noalloc_scratch_bytes(int B, int S, int P, int nlist, bool keys_in_smem);
+cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const SearchArgs& a, cudaStream_t s);

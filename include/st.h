@@ -47,7 +47,9 @@ typedef enum {
     ST_ERR_UNSUPPORTED = 2,  /* a size outside the supported limits below */
     ST_ERR_OOM = 3,          /* a device allocation failed */
     ST_ERR_CUDA = 4,         /* a CUDA runtime or launch error */
-    ST_ERR_DEVICE = 5        /* a kernel recorded an internal error (see st_index_check) */
+    ST_ERR_DEVICE = 5,       /* a kernel recorded an internal error (see st_index_check) */
+    ST_ERR_SCRATCH_LIMIT = 6 /* st_probe_noalloc: the request needs more than its
+                                fixed scratch (ST_PROBE_NOALLOC_SCRATCH_BYTES) */
 } st_status;
 
 /* Supported limits (ST_ERR_UNSUPPORTED outside them). */
@@ -151,6 +153,50 @@ typedef enum {
 /* Set an option; INVALID_ARG for an unknown option or a negative value.
    Not safe to call while a search on the same index is being enqueued. */
 st_status st_index_set_option(st_index* idx, st_option opt, int64_t value);
+
+/*
+ * Allocation-free coarse probe: step 1 above alone (each query's nprobe best
+ * lists, best first, ties to the lower list id -- exactly the lists st_search
+ * probes and reports in st_search_extras.probe), without allocating any
+ * memory. The method has no such call: it is a library addition for callers
+ * that must not allocate device memory at query time, e.g. a request router
+ * that has handed the rest of the GPU's memory to a fixed-size cache or to
+ * another process, or that cannot accept the synchronisation and latency
+ * spikes that cudaMalloc/cudaFree and a memory pool's growth can cause, and
+ * only needs to know which lists (or the shards holding them) a query reaches.
+ *
+ *   queries    device int8  [B][d]
+ *   out_probe  device int32 [B][nprobe]   caller-owned
+ *
+ * Its scratch is one fixed array of ST_PROBE_NOALLOC_SCRATCH_BYTES in the
+ * library's device memory (one per device, created when the library is
+ * loaded), needing B*4 (rounded up to 256) + B*S*nprobe*8 bytes, S being the
+ * number of centroid slices per query the probe picks (S = 1 for B >= 296 on
+ * a 148-SM GPU, at most 32), plus B*nlist*8 bytes when nlist exceeds 16384*S.
+ * Requests that need more are rejected on the host with ST_ERR_SCRATCH_LIMIT
+ * before anything is enqueued; smaller B or nprobe fit. The part that must
+ * start at zero (the per-query completion counters) is cleared on `stream`
+ * by every call (cudaMemsetAsync, which allocates nothing).
+ *
+ * All calls on a device share the one array, so calls whose work may overlap
+ * on the GPU -- on different streams, or from different host threads without
+ * ordering -- race on it and give wrong results. Issue them on one stream, or
+ * order them with events.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, which may load the library's GPU code) and raises
+ * the kernel's shared-memory limit; make that first call, for example with a
+ * small warm-up request, before any stream capture begins.
+ *
+ * Asynchronous on `stream` like st_search; kernel-side errors are reported by
+ * st_index_check. Errors: INVALID_ARG (null index, null or non-device pointer,
+ * misaligned queries (16 bytes) or out_probe (4 bytes), B < 1, nprobe < 1 or
+ * nprobe > nlist), UNSUPPORTED (nprobe above ST_MAX_NPROBE, B*nprobe >= 2^31),
+ * SCRATCH_LIMIT, CUDA.
+ */
+#define ST_PROBE_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB */
+st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B, int32_t nprobe,
+                           int32_t* out_probe, cudaStream_t stream);
 
 /* Free the index (NULL-safe). Waits for the device to finish work that may
    still use it. */

@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for s in range(6):
+    for s in range(7):
         assert st.status_string(s)
     assert st.status_string(3) == "out of device memory"
 
@@ -63,5 +63,6 @@ def test_search_rejects_null_index(lib):
     assert lib.st_search(None, fake, fake, 1, 1, 1, fake, fake, None) == st.ST_ERR_INVALID_ARG
     assert lib.st_search_host(None, fake, fake, 1, 1, 1, fake, fake, None) == st.ST_ERR_INVALID_ARG
     assert lib.st_index_check(None, None) == st.ST_ERR_INVALID_ARG
+    assert lib.st_probe_noalloc(None, fake, 1, 1, fake, None) == st.ST_ERR_INVALID_ARG
     assert lib.st_index_set_option(None, 1, 5) == st.ST_ERR_INVALID_ARG
     lib.st_index_destroy(None)  # NULL-safe
