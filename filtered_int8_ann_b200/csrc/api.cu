@@ -144,8 +144,8 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     ScratchLayout L;
     L.off_list_cnt = L.add(nl4 * 4);
     L.off_probe_done = L.add(size_t(B) * 4);
-    L.off_cand_cnt = L.add(size_t(B) * 4);
-    L.off_elig = L.add(size_t(B) * 8);
+    L.off_cand_cnt = L.add(size_t(B) * st::kCntStride * 4);
+    L.off_elig = L.add(size_t(B) * st::kCntStride * 4);
     L.off_hist = L.add(size_t(B) * st::kHistBins * 4);
     L.off_ctl = L.add(sizeof(st::PlanCtl));
     L.zero_bytes = L.total;

@@ -15,28 +15,32 @@
 // (kWarpItems rows) x up to kQMax queries probing that list, so each probed
 // list is streamed once per batch whatever the number of queries probing it.
 // Warps are independent (one-warp CTAs, many per SM) and take units
-// round-robin, with a two-deep pipeline:
+// round-robin, software-pipelined over three units:
 //   * signature planes: the index stores each chunk's signatures as bit-planes
 //     (layout.cu). A unit needs only the planes of the bits in the union of its
-//     queries' masks; its lanes issue one 64-byte bulk asynchronous copy (TMA
-//     engine, cp.async.bulk + mbarrier) per such plane into the next free slot
-//     of a small per-warp buffer (kPlaneSlots planes), and the next unit's
-//     planes are always in flight while this unit is processed. A unit whose
-//     union is wider than the buffer reads its planes from global memory
-//     instead (slower, same result);
+//     queries' masks. Each of the warp's lanes copies 16 bytes of one such
+//     plane with cp.async (8 planes per warp instruction, L1 bypassed) into the
+//     next free slot of a small per-warp buffer (kPlaneSlots planes); the
+//     planes of the unit two ahead are requested as soon as this unit's test
+//     has released its buffer. A unit whose union is wider than the buffer
+//     reads its planes from global memory instead (slower, same result). Many
+//     tiny copies suit the load/store path better than the bulk-copy engine,
+//     whose per-request cost made 64-byte copies the bottleneck;
 //   * test: for each query, the two half-warps AND the planes of the two
 //     halves of the query's mask bits (a list precomputed once per search) for
 //     the 32 rows of the lane's block; one shuffle joins the halves, so 32 rows
 //     cost one AND per mask bit;
 //   * filter-before-load: per-query survivor counts reserve candidate slots
-//     (one atomic per unit and query, overlapped with the row loads); only
-//     survivors' rows are read (16-byte read-only loads) and dotted with dp4a
-//     against the query vectors (staged in shared memory by cp.async); a key's
+//     (one atomic per unit and query, whose reply is needed only after the
+//     survivors' rows and dots); only survivors' rows are read (16-byte
+//     read-only loads) and dotted with dp4a against the query vectors (staged
+//     in shared memory by cp.async while the previous unit finished); a key's
 //     slot is its ballot rank among the unit's survivors of that query; each
 //     key also counts into the query's score histogram, which the final top-k
 //     uses to find its cut without sorting every candidate.
-// Every wait on a copy is bounded: on expiry the warp records kErrCopyTimeout,
-// waits (bounded) for its copies in flight and stops.
+// cp.async groups complete in order; each unit commits exactly two groups
+// (the planes two ahead, then the next unit's query vectors), so fixed
+// wait_group depths find every copy: no spin loop, nothing to time out.
 #include "st_internal.cuh"
 
 namespace st {
@@ -47,32 +51,29 @@ constexpr int kPlaneBufBytes = kPlaneSlots * kPlaneBytes;
 
 // Per-warp shared memory: 2 plane buffers | survivor offsets [kWarpItems] u16 |
 // pass words [kQMax][16] | query vectors [kQMax][d] | bit -> slot tables [2][128] |
-// query ids [kQMax] | 2 mbarriers
+// slot -> bit [kPlaneSlots] | query ids [kQMax]
 __host__ __device__ inline size_t scan_warp_bytes(int d, int W)
 {
     (void)W;
     return (2 * kPlaneBufBytes + kWarpItems * 2 + kQMax * 16 * 4 + size_t(kQMax) * d + 2 * kMaskBitsMax +
-            kQMax * 4 + 16 + 127) / 128 * 128;
+            kPlaneSlots + kQMax * 4 + 127) / 128 * 128;
 }
 
 size_t scan_smem_bytes(int d, int W) { return size_t(kScanBlock / 32) * scan_warp_bytes(d, W); }
 
-// Start the copies of the planes a unit needs (the union u0/u1 of its queries'
-// mask bits) into consecutive slots of `buf`, and record bit -> slot in `tab`.
-// Returns false (and copies nothing) when the union has more bits than a
-// buffer holds; the barrier phase completes either way.
+// Request the planes a unit needs (the union u0/u1 of its queries' mask bits)
+// into consecutive slots of `buf`, recording bit -> slot in `tab`. Returns
+// false (and copies nothing) when the union has more bits than a buffer
+// holds. The caller commits the group.
 template <int W>
 __device__ __forceinline__ bool issue_planes(const SearchArgs& a, int chunk, uint64_t u0, uint64_t u1,
-                                             uint32_t* buf, uint8_t* tab, uint64_t* bar, int lane)
+                                             uint32_t* buf, uint8_t* tab, uint8_t* inv, int lane)
 {
     constexpr int NPL = 64 * W;
     const int n0 = __popcll(u0);
     const int nb = n0 + (W > 1 ? __popcll(u1) : 0);
-    const bool fits = nb <= kPlaneSlots;
-    if (lane == 0) mbar_expect_tx(bar, fits ? uint32_t(nb) * kPlaneBytes : 0u);
-    __syncwarp();
-    if (!fits) return false;
-    const uint32_t* src = a.planes + int64_t(chunk) * NPL * 16;
+    if (nb > kPlaneSlots) return false;  // warp-uniform
+    __syncwarp();  // earlier reads of tab / inv are done
 #pragma unroll
     for (int r = 0; r < 2 * W; ++r) {
         const int b = lane + 32 * r;
@@ -81,8 +82,12 @@ __device__ __forceinline__ bool issue_planes(const SearchArgs& a, int chunk, uin
         const int slot = (b < 64 ? 0 : n0) + __popcll(below);
         const bool on = (word >> (b & 63)) & 1ull;
         tab[b] = on ? uint8_t(slot) : uint8_t(0);
-        if (on) bulk_g2s(buf + slot * 16, src + b * 16, kPlaneBytes, bar);
+        if (on) inv[slot] = uint8_t(b);
     }
+    __syncwarp();
+    // lane = 4 * (plane of this round) + (16-byte quarter of the plane)
+    const uint32_t* src = a.planes + int64_t(chunk) * NPL * 16 + (lane & 3) * 4;
+    for (int j = lane >> 2; j < nb; j += 8) cp_async16_cg(buf + j * 16 + (lane & 3) * 4, src + inv[j] * 16);
     return true;
 }
 
@@ -98,8 +103,9 @@ __device__ __forceinline__ void warp_or2(uint64_t& x, uint64_t& y)
 
 // NP = d/16 when the row is held in registers (d = 64 or 128), 0 for any other
 // d (rows are then re-read from L1 for each eligible query).
+// (at most as many registers as keep the shared-memory-limited warp count resident)
 template <int NP, int W>
-__global__ void __launch_bounds__(kScanBlock)
+__global__ void __launch_bounds__(kScanBlock, NP == 8 ? 16 : 20)
 scan_kernel(SearchArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -118,15 +124,8 @@ scan_kernel(SearchArgs a)
     uint32_t* s_pass = reinterpret_cast<uint32_t*>(surv + kWarpItems);                   // [kQMax][16]
     int4* s_q = reinterpret_cast<int4*>(s_pass + kQMax * 16);                            // [kQMax][np]
     uint8_t* s_tab = reinterpret_cast<uint8_t*>(s_q) + size_t(kQMax) * d;                // [2][128]
-    int32_t* s_qid = reinterpret_cast<int32_t*>(s_tab + 2 * kMaskBitsMax);               // [kQMax]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s_qid + kQMax);                         // [2]
-
-    if (lane == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
+    uint8_t* s_inv = s_tab + 2 * kMaskBitsMax;                                           // [kPlaneSlots]
+    int32_t* s_qid = reinterpret_cast<int32_t*>(s_inv + kPlaneSlots);                    // [kQMax]
 
     const int n_units = a.ctl->n_units < a.max_units ? a.ctl->n_units : a.max_units;
     const int stride = gridDim.x * (kScanBlock / 32);
@@ -145,9 +144,42 @@ scan_kernel(SearchArgs a)
             m1 = m.y;
         }
     };
+    // query ids of a unit -> shared memory, its query vectors by cp.async
+    auto stage_queries = [&](int qn, int qid) {
+        __syncwarp();  // earlier reads of s_qid / s_q are done
+        if (lane < qn) s_qid[lane] = qid;
+        __syncwarp();
+        for (int idx = lane; idx < qn * np; idx += 32) {
+            const int s = idx / np, p = idx - s * np;
+            cp_async16(s_q + s * np + p, a.queries + int64_t(s_qid[s]) * d + 16 * p);
+        }
+    };
 
-    // prologue: entries of the first three units, slots of the first two,
-    // planes of the first two
+    // Request the planes of a unit whose entry is `e` and whose slots (lanes <
+    // its query count) hold masks m0/m1, into buffer `bb`; returns the number
+    // of planes the buffer then holds, or -1 when the test must read global
+    // planes. A single-query unit needs no union: its planes are the query's
+    // mask bits in increasing order, listed by the probe.
+    auto request_planes = [&](const int4& e, int qid, uint64_t m0, uint64_t m1, int bb) -> int {
+        uint32_t* buf = bb ? pbuf1 : pbuf0;
+        if ((e.w & 0xFFFF) == 1) {
+            const int q = __shfl_sync(0xffffffffu, qid, 0);
+            const int nb = __ldg(a.qnbits + q);
+            if (nb > kPlaneSlots) return -1;
+            const uint8_t* bits = a.qbits + int64_t(q) * kMaskBitsMax;
+            const uint32_t* src = a.planes + int64_t(e.y) * NPL * 16 + (lane & 3) * 4;
+            for (int j = lane >> 2; j < nb; j += 8)
+                cp_async16_cg(buf + j * 16 + (lane & 3) * 4, src + __ldg(bits + j) * 16);
+            return nb;
+        }
+        uint64_t x = m0, y = m1;
+        warp_or2(x, y);
+        if (!issue_planes<W>(a, e.y, x, y, buf, s_tab + bb * kMaskBitsMax, s_inv, lane)) return -1;
+        return __popcll(x) + (W > 1 ? __popcll(y) : 0);
+    };
+
+    // prologue: entries of the first three units, slots of the first two;
+    // groups: planes(0), queries(0), planes(1)
     int4 e_cur = a.units[u];
     int4 e_nxt = make_int4(0, 0, 0, 0), e_n2 = make_int4(0, 0, 0, 0);
     const bool has_nxt0 = u + stride < n_units;
@@ -157,19 +189,12 @@ scan_kernel(SearchArgs a)
     uint64_t m0_c, m1_c, m0_n = 0, m1_n = 0;
     load_slots(e_cur, qid_c, m0_c, m1_c);
     if (has_nxt0) load_slots(e_nxt, qid_n, m0_n, m1_n);
-    uint32_t fits = 0;  // bit b: buffer b holds its unit's planes (else read them from global)
-    {
-        uint64_t x = m0_c, y = m1_c;
-        warp_or2(x, y);
-        if (issue_planes<W>(a, e_cur.y, x, y, pbuf0, s_tab, &bars[0], lane)) fits |= 1u;
-    }
-    if (has_nxt0) {
-        uint64_t x = m0_n, y = m1_n;
-        warp_or2(x, y);
-        if (issue_planes<W>(a, e_nxt.y, x, y, pbuf1, s_tab + kMaskBitsMax, &bars[1], lane)) fits |= 2u;
-    }
-    uint32_t phase = 0;                      // bit b: parity to wait for on buffer b
-    uint32_t pending = has_nxt0 ? 3u : 1u;   // bit b: a copy into buffer b is in flight
+    int held0 = request_planes(e_cur, qid_c, m0_c, m1_c, 0);  // planes held by buffer 0 / 1 (-1: global)
+    cp_async_commit();
+    stage_queries(e_cur.w & 0xFFFF, qid_c);
+    cp_async_commit();
+    int held1 = has_nxt0 ? request_planes(e_nxt, qid_n, m0_n, m1_n, 1) : -1;
+    cp_async_commit();
     int b = 0;
 
     for (; u < n_units; u += stride) {
@@ -177,9 +202,11 @@ scan_kernel(SearchArgs a)
         const int chunk = e_cur.y;
         const int len = e_cur.w >> 16;
         const int qn = e_cur.w & 0xFFFF;
-        uint32_t* pb = b ? pbuf1 : pbuf0;
+        const uint32_t* pb = b ? pbuf1 : pbuf0;
         const uint8_t* tab = s_tab + b * kMaskBitsMax;
-        const bool in_smem = (fits >> b) & 1u;
+        const int held = b ? held1 : held0;
+        const bool in_smem = held >= 0;
+        const bool single = qn == 1 && in_smem;  // warp-uniform fast path
         const bool has_n2 = u + 2 * stride < n_units;
         const bool has_n3 = u + 3 * stride < n_units;
 
@@ -191,69 +218,70 @@ scan_kernel(SearchArgs a)
         uint64_t m0_2 = 0, m1_2 = 0;
         if (has_n2) load_slots(e_n2, qid_2, m0_2, m1_2);
 
-        // query ids of this unit -> shared memory; vectors by cp.async
-        if (lane < qn) s_qid[lane] = qid_c;
+        // this unit's planes: pending groups are at most [queries(u), planes(u+1)]
+        cp_async_wait_group<2>();
         __syncwarp();
-        for (int idx = lane; idx < qn * np; idx += 32) {
-            const int s = idx / np, p = idx - s * np;
-            cp_async16(s_q + s * np + p, a.queries + int64_t(s_qid[s]) * d + 16 * p);
-        }
-        cp_async_commit();
-
-        // wait for this unit's planes
-        const bool ok = mbar_wait_bounded(&bars[b], (phase >> b) & 1u);
-        if (!__all_sync(0xffffffffu, ok)) {
-            if (lane == 0) set_error(a.err, kErrCopyTimeout);
-            break;
-        }
-        phase ^= 1u << b;
-        pending &= ~(1u << b);
 
         // test: pass word of query s for block `blk` = AND of its mask planes;
-        // the two half-warps take halves of the query's precomputed bit list
+        // the two half-warps AND the two halves of the query's mask bits
         const uint32_t valid = len >= 32 * (blk + 1) ? 0xFFFFFFFFu
                              : (len <= 32 * blk ? 0u : ((1u << (len - 32 * blk)) - 1u));
-        const uint32_t* gpl = a.planes + int64_t(chunk) * NPL * 16 + blk;
         uint32_t any = 0;
         uint32_t mycnt = 0;  // lane s: survivors of query s
-        for (int s = 0; s < qn; ++s) {
-            const int qg = s_qid[s];
-            const int nb = __ldg(a.qnbits + qg);
-            const int h0 = (nb + 1) >> 1;
-            const uint8_t* bits = a.qbits + int64_t(qg) * kMaskBitsMax;
-            const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
-            // four independent bit -> slot -> plane chains per step
+        if (single) {
+            // the buffer holds exactly the query's planes, in bit order
+            const int h0 = (held + 1) >> 1;
+            const int j1 = half ? held : h0;
+            int j = half ? h0 : 0;
             uint32_t acc = 0xFFFFFFFFu;
-            if (in_smem) {
-                int j = j0;
-                for (; j + 4 <= j1; j += 4) {
-                    const int b0 = __ldg(bits + j), b1 = __ldg(bits + j + 1);
-                    const int b2 = __ldg(bits + j + 2), b3 = __ldg(bits + j + 3);
-                    const int s0 = tab[b0], s1 = tab[b1], s2 = tab[b2], s3 = tab[b3];
-                    acc &= pb[s0 * 16 + blk] & pb[s1 * 16 + blk] & pb[s2 * 16 + blk] & pb[s3 * 16 + blk];
-                }
-                for (; j < j1; ++j) acc &= pb[tab[__ldg(bits + j)] * 16 + blk];
-            } else {
-                for (int j = j0; j < j1; ++j) acc &= __ldg(gpl + __ldg(bits + j) * 16);
-            }
+            for (; j + 4 <= j1; j += 4)
+                acc &= pb[j * 16 + blk] & pb[(j + 1) * 16 + blk] & pb[(j + 2) * 16 + blk] & pb[(j + 3) * 16 + blk];
+            for (; j < j1; ++j) acc &= pb[j * 16 + blk];
             acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
-            acc &= valid;
-            if (half == 0) s_pass[s * 16 + blk] = acc;
-            any |= acc;
-            // survivors of query s: half 0 holds the 16 pass words; the full
-            // 32-lane reduction leaves the total in every lane
-            uint32_t c = half == 0 ? uint32_t(__popc(acc)) : 0u;
+            any = acc & valid;
+        } else {
+            const uint32_t* gpl = a.planes + int64_t(chunk) * NPL * 16 + blk;
+            for (int s = 0; s < qn; ++s) {
+                const int qg = s_qid[s];
+                const int nb = __ldg(a.qnbits + qg);
+                const int h0 = (nb + 1) >> 1;
+                const uint8_t* bits = a.qbits + int64_t(qg) * kMaskBitsMax;
+                const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
+                // four independent bit -> slot -> plane chains per step
+                uint32_t acc = 0xFFFFFFFFu;
+                if (in_smem) {
+                    int j = j0;
+                    for (; j + 4 <= j1; j += 4) {
+                        const int b0 = __ldg(bits + j), b1 = __ldg(bits + j + 1);
+                        const int b2 = __ldg(bits + j + 2), b3 = __ldg(bits + j + 3);
+                        const int s0 = tab[b0], s1 = tab[b1], s2 = tab[b2], s3 = tab[b3];
+                        acc &= pb[s0 * 16 + blk] & pb[s1 * 16 + blk] & pb[s2 * 16 + blk] & pb[s3 * 16 + blk];
+                    }
+                    for (; j < j1; ++j) acc &= pb[tab[__ldg(bits + j)] * 16 + blk];
+                } else {
+                    for (int j = j0; j < j1; ++j) acc &= __ldg(gpl + __ldg(bits + j) * 16);
+                }
+                acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
+                acc &= valid;
+                if (half == 0) s_pass[s * 16 + blk] = acc;
+                any |= acc;
+                // survivors of query s: half 0 holds the 16 pass words; the full
+                // 32-lane reduction leaves the total in every lane
+                uint32_t c = half == 0 ? uint32_t(__popc(acc)) : 0u;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-            if (lane == s) mycnt = c;
+                for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+                if (lane == s) mycnt = c;
+            }
         }
 
-        // per-query survivor counts -> one reservation each (lane s)
-        uint32_t base = 0;
-        if (lane < qn && mycnt) {
-            base = atomicAdd(&a.cand_cnt[qid_c], mycnt);
-            atomicAdd(&a.eligible_cnt[qid_c], (unsigned long long)mycnt);
+        // buffer b is free: request the planes of the unit two ahead
+        if (has_n2) {
+            __syncwarp();  // every lane is done reading buffer b
+            const int h2 = request_planes(e_n2, qid_2, m0_2, m1_2, b);
+            if (b) held1 = h2;
+            else held0 = h2;
         }
+        cp_async_commit();
 
         // survivor row offsets, block by block
         const uint32_t mine = half == 0 ? uint32_t(__popc(any)) : 0u;
@@ -273,67 +301,111 @@ scan_kernel(SearchArgs a)
                 surv[pos++] = uint16_t(32 * blk + i);
             }
         }
-        cp_async_wait_all();
+
+        // per-query survivor counts -> one reservation each (lane s); the
+        // reply is first needed when the keys are stored
+        if (single && lane == 0) mycnt = uint32_t(nsurv);
+        uint32_t base = 0;
+        if (lane < qn && mycnt) {
+            base = atomicAdd(&a.cand_cnt[int64_t(qid_c) * kCntStride], mycnt);
+            atomicAdd(&a.eligible_cnt[int64_t(qid_c) * (kCntStride / 2)], (unsigned long long)mycnt);
+        }
+
+        // this unit's query vectors: pending groups are at most [planes(u+2)]
+        cp_async_wait_group<1>();
         __syncwarp();
 
         // rows of the survivors (one load per survivor), dots, keys into the
-        // reserved slots; a key's slot is its ballot rank among this unit's
-        // survivors of the same query
-        uint32_t run = 0;  // lane s: keys of query s written so far
-        for (int c0 = 0; c0 < nsurv; c0 += 32) {
-            const int idx = c0 + lane;
-            int off = -1;
-            int64_t i = 0;
-            int4 row[NP > 0 ? NP : 1];
-            const int4* rp = nullptr;
-            if (idx < nsurv) {
-                off = surv[idx];
-                i = ib + off;
-                rp = reinterpret_cast<const int4*>(a.items + i * d);
-                if (NP > 0) {
+        // reserved slots
+        if (single) {
+            // every survivor is a key of the one query, in survivor order
+            const int qg = s_qid[0];
+            uint64_t* cand = a.cand + int64_t(qg) * a.cap;
+            uint32_t* hist = a.hist + int64_t(qg) * kHistBins;
+            for (int c0 = 0; c0 < nsurv; c0 += 32) {
+                const int idx = c0 + lane;
+                int4 row[NP > 0 ? NP : 1];
+                const int4* rp = nullptr;
+                int64_t i = 0;
+                if (idx < nsurv) {
+                    i = ib + surv[idx];
+                    rp = reinterpret_cast<const int4*>(a.items + i * d);
+                    if (NP > 0) {
 #pragma unroll
-                    for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
+                        for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
+                    }
                 }
-            }
-            const uint32_t* pw = s_pass + (off >= 0 ? (off >> 5) : 0);
-            const int bit = off & 31;
-            for (int s = 0; s < qn; ++s) {
-                const bool on = off >= 0 && ((pw[s * 16] >> bit) & 1u);
-                const unsigned bal = __ballot_sync(0xffffffffu, on);
-                if (bal == 0u) continue;
-                const uint32_t slot0 = __shfl_sync(0xffffffffu, base, s) + __shfl_sync(0xffffffffu, run, s);
-                if (on) {
-                    const int4* qs = s_q + s * np;
+                const uint32_t base0 = __shfl_sync(0xffffffffu, base, 0);
+                if (idx < nsurv) {
                     int32_t acc0 = 0, acc1 = 0;
                     if (NP > 0) {
 #pragma unroll
                         for (int p = 0; p < (NP > 0 ? NP : 1); p += 2) {
-                            acc0 = dot16(row[p], qs[p], acc0);
-                            if (p + 1 < NP) acc1 = dot16(row[p + 1], qs[p + 1], acc1);
+                            acc0 = dot16(row[p], s_q[p], acc0);
+                            if (p + 1 < NP) acc1 = dot16(row[p + 1], s_q[p + 1], acc1);
                         }
                     } else {
-                        for (int p = 0; p < np; ++p) acc0 = dot16(__ldg(rp + p), qs[p], acc0);
+                        for (int p = 0; p < np; ++p) acc0 = dot16(__ldg(rp + p), s_q[p], acc0);
                     }
-                    const uint64_t pos = uint64_t(slot0) + __popc(bal & lanemask_lt());
                     const int32_t score = acc0 + acc1;
-                    const int qg = s_qid[s];
-                    if (pos < uint64_t(a.cap)) a.cand[int64_t(qg) * a.cap + int64_t(pos)] = pack_key(score, uint32_t(i));
-                    atomicAdd(&a.hist[int64_t(qg) * kHistBins + score_bin(score, a.smax, a.hshift)], 1u);
+                    const uint64_t pos = uint64_t(base0) + uint32_t(idx);
+                    if (pos < uint64_t(a.cap)) cand[pos] = pack_key(score, uint32_t(i));
+                    atomicAdd(&hist[score_bin(score, a.smax, a.hshift)], 1u);
                 }
-                if (lane == s) run += __popc(bal);
+            }
+        } else {
+            // a key's slot is its ballot rank among this unit's survivors of
+            // the same query
+            uint32_t run = 0;  // lane s: keys of query s written so far
+            for (int c0 = 0; c0 < nsurv; c0 += 32) {
+                const int idx = c0 + lane;
+                int off = -1;
+                int64_t i = 0;
+                int4 row[NP > 0 ? NP : 1];
+                const int4* rp = nullptr;
+                if (idx < nsurv) {
+                    off = surv[idx];
+                    i = ib + off;
+                    rp = reinterpret_cast<const int4*>(a.items + i * d);
+                    if (NP > 0) {
+#pragma unroll
+                        for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
+                    }
+                }
+                const uint32_t* pw = s_pass + (off >= 0 ? (off >> 5) : 0);
+                const int bit = off & 31;
+                for (int s = 0; s < qn; ++s) {
+                    const bool on = off >= 0 && ((pw[s * 16] >> bit) & 1u);
+                    const unsigned bal = __ballot_sync(0xffffffffu, on);
+                    if (bal == 0u) continue;
+                    const uint32_t slot0 = __shfl_sync(0xffffffffu, base, s) + __shfl_sync(0xffffffffu, run, s);
+                    if (on) {
+                        const int4* qs = s_q + s * np;
+                        int32_t acc0 = 0, acc1 = 0;
+                        if (NP > 0) {
+#pragma unroll
+                            for (int p = 0; p < (NP > 0 ? NP : 1); p += 2) {
+                                acc0 = dot16(row[p], qs[p], acc0);
+                                if (p + 1 < NP) acc1 = dot16(row[p + 1], qs[p + 1], acc1);
+                            }
+                        } else {
+                            for (int p = 0; p < np; ++p) acc0 = dot16(__ldg(rp + p), qs[p], acc0);
+                        }
+                        const uint64_t pos = uint64_t(slot0) + __popc(bal & lanemask_lt());
+                        const int32_t score = acc0 + acc1;
+                        const int qg = s_qid[s];
+                        if (pos < uint64_t(a.cap)) a.cand[int64_t(qg) * a.cap + int64_t(pos)] = pack_key(score, uint32_t(i));
+                        atomicAdd(&a.hist[int64_t(qg) * kHistBins + score_bin(score, a.smax, a.hshift)], 1u);
+                    }
+                    if (lane == s) run += __popc(bal);
+                }
             }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
 
-        // buffer b is free: start the planes of the unit two ahead
-        if (has_n2) {
-            uint64_t x = m0_2, y = m1_2;
-            warp_or2(x, y);
-            if (issue_planes<W>(a, e_n2.y, x, y, pb, s_tab + b * kMaskBitsMax, &bars[b], lane)) fits |= 1u << b;
-            else fits &= ~(1u << b);
-            pending |= 1u << b;
-        }
+        // the next unit's query vectors (group queries(u+1))
+        stage_queries(e_nxt.w & 0xFFFF, qid_n);
+        cp_async_commit();
+
         e_cur = e_nxt;
         e_nxt = e_n2;
         e_n2 = e_n3;
@@ -345,12 +417,7 @@ scan_kernel(SearchArgs a)
         m1_n = m1_2;
         b ^= 1;
     }
-
-    // after an error exit: let copies still in flight land before the warp
-    // leaves (bounded)
-    for (int bb = 0; bb < 2; ++bb)
-        if ((pending >> bb) & 1u) mbar_wait_bounded(&bars[bb], (phase >> bb) & 1u);
-    cp_async_wait_all();
+    cp_async_wait_all();  // no copy may land after the warp has left
 }
 
 template <int NP, int W>

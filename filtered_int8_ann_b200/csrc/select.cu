@@ -174,7 +174,7 @@ select_kernel(SearchArgs a)
     uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem_raw);    // max(pwk, BLOCK) keys
     uint64_t* local = sortbuf + (pwk > BLOCK ? pwk : BLOCK);       // 16-byte aligned
 
-    const uint32_t cnt = a.cand_cnt[q];
+    const uint32_t cnt = a.cand_cnt[int64_t(q) * kCntStride];
     const uint64_t* keys = a.cand + int64_t(q) * a.cap;
     int64_t n = cnt;
     const bool overflow = n > a.cap;
@@ -205,7 +205,7 @@ select_kernel(SearchArgs a)
         a.out_ids[int64_t(q) * k + r] = key_id(key);
         a.out_scores[int64_t(q) * k + r] = key_score(key);
     }
-    if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[q]);
+    if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
 }
 
 cudaError_t launch_select(const SearchArgs& a, cudaStream_t s)

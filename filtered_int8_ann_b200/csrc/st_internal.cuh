@@ -21,6 +21,9 @@ constexpr int kSelectBlock = 1024;
 constexpr int kSelectSmemKeys = 22528;     // candidates up to this are selected in smem
 constexpr int kPlanBlock = 512;
 constexpr int kHistBins = 2048;            // per-query score histogram bins
+// Per-query counters sit one 128-byte line apart, so the reservation atomics
+// of different queries spread over the L2 slices instead of queueing on one.
+constexpr int kCntStride = 32;             // uint32 words (16 uint64) per query
 constexpr int kMaskBitsMax = 128;          // signature bits
 constexpr int kSelBits = 11;               // radix digit of the selections
 constexpr int kSelBins = 1 << kSelBits;
@@ -87,8 +90,8 @@ struct SearchArgs {
     // scratch (the zeroed block first: one memset clears it)
     int32_t* list_cnt;       // [nlist] queries filed into each list      (zeroed)
     int32_t* probe_done;     // [B] probe slices finished per query       (zeroed)
-    uint32_t* cand_cnt;      // [B] candidates reserved per query         (zeroed)
-    unsigned long long* eligible_cnt;  // [B]                             (zeroed)
+    uint32_t* cand_cnt;      // [B][kCntStride] candidates reserved per query, word 0 used (zeroed)
+    unsigned long long* eligible_cnt;  // [B][kCntStride / 2], word 0 used        (zeroed)
     uint32_t* hist;          // [B][kHistBins] emitted-key score histogram (zeroed)
     PlanCtl* ctl;            // unit allocation counter                   (zeroed)
     int32_t* probe;          // [B][P]
@@ -195,8 +198,19 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+// 16-byte asynchronous copy global -> shared that bypasses L1 (data read once)
+__device__ __forceinline__ void cp_async16_cg(void* dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Wait until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // ----------------------------------------------------------------------------
 // Block-wide selection (one CTA of BLOCK threads)
