@@ -90,8 +90,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // must start at zero come first, so one memset clears them.
 struct ScratchLayout {
     size_t total = 0;
-    size_t off_list_cnt, off_probe_done, off_cand_cnt, off_elig, off_hist, off_ctl, zero_bytes;
-    size_t off_probe, off_probe_keys, off_probe_part, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_units, off_cand;
+    size_t off_list_cnt, off_cand_cnt, off_elig, off_hist, off_ctl, zero_bytes;
+    size_t off_probe, off_probe_keys, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_units, off_cand;
     size_t add(size_t bytes)
     {
         const size_t o = total;
@@ -131,27 +131,18 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     const int64_t max_units = max_units_bound(idx, B, nprobe);
     if (max_units >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
     if (int64_t(idx->nlist) * B >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
-    SearchArgs probe_shape;
-    std::memset(&probe_shape, 0, sizeof(probe_shape));
-    probe_shape.B = B;
-    probe_shape.P = nprobe;
-    probe_shape.nlist = idx->nlist;
-    const int S = st::probe_slices(probe_shape, idx->num_sms);
-    const bool probe_in_smem = (idx->nlist + S - 1) / S + 1 <= st::kProbeSmemKeys;
     const size_t nl4 = size_t(idx->nlist + 3) / 4 * 4;
     const size_t slots = size_t(idx->nlist) * size_t(B);
 
     ScratchLayout L;
     L.off_list_cnt = L.add(nl4 * 4);
-    L.off_probe_done = L.add(size_t(B) * 4);
     L.off_cand_cnt = L.add(size_t(B) * st::kCntStride * 4);
     L.off_elig = L.add(size_t(B) * st::kCntStride * 4);
     L.off_hist = L.add(size_t(B) * st::kHistBins * 4);
     L.off_ctl = L.add(sizeof(st::PlanCtl));
     L.zero_bytes = L.total;
     L.off_probe = L.add(size_t(B) * nprobe * 4);
-    L.off_probe_keys = probe_in_smem ? 0 : L.add(size_t(B) * idx->nlist * 8);
-    L.off_probe_part = L.add(size_t(B) * S * nprobe * 8);
+    L.off_probe_keys = L.add(size_t(B) * idx->nlist * 8);
     L.off_list_ustart = L.add(nl4 * 4);
     L.off_qbits = L.add(size_t(B) * st::kMaskBitsMax);
     L.off_qnbits = L.add(size_t(B) * 4);
@@ -189,7 +180,6 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.out_scores = out_scores;
     a.out_eligible = extras ? extras->eligible : nullptr;
     a.list_cnt = reinterpret_cast<int32_t*>(base + L.off_list_cnt);
-    a.probe_done = reinterpret_cast<int32_t*>(base + L.off_probe_done);
     a.cand_cnt = reinterpret_cast<uint32_t*>(base + L.off_cand_cnt);
     a.eligible_cnt = reinterpret_cast<unsigned long long*>(base + L.off_elig);
     a.hist = reinterpret_cast<uint32_t*>(base + L.off_hist);
@@ -201,8 +191,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     }
     a.ctl = reinterpret_cast<st::PlanCtl*>(base + L.off_ctl);
     a.probe = reinterpret_cast<int32_t*>(base + L.off_probe);
-    a.probe_keys = probe_in_smem ? nullptr : reinterpret_cast<uint64_t*>(base + L.off_probe_keys);
-    a.probe_part = reinterpret_cast<uint64_t*>(base + L.off_probe_part);
+    a.probe_keys = reinterpret_cast<uint64_t*>(base + L.off_probe_keys);
     a.list_ustart = reinterpret_cast<int32_t*>(base + L.off_list_ustart);
     a.qbits = reinterpret_cast<uint8_t*>(base + L.off_qbits);
     a.qnbits = reinterpret_cast<int32_t*>(base + L.off_qnbits);
@@ -219,7 +208,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     };
     e = cudaMemsetAsync(base, 0, L.zero_bytes, stream);
     mark(0);
-    if (e == cudaSuccess) e = st::launch_probe(a, S, stream);
+    if (e == cudaSuccess) e = st::launch_probe_search(a, stream);
     mark(1);
     if (e == cudaSuccess) e = st::launch_plan(a, idx->num_sms, stream);
     mark(2);

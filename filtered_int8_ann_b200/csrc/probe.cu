@@ -8,15 +8,21 @@
 // but not the index type; this library reads it as an IVF with int8 centroids
 // and contiguous lists.
 //
-// Grid: B queries x S centroid slices (S chosen so the grid fills the GPU).
-// Each CTA scores its slice (16-byte read-only loads of centroid rows from L2,
-// dp4a against the query held in shared memory, unrolled for memory-level
-// parallelism), keeps its slice's nprobe best keys (exact: the global top-P is
-// a subset of the union of the slices' top-P) and publishes them. The last CTA
-// of a query to finish -- found with one atomic counter, no waiting -- merges
-// the S partial lists, writes the probe result, and files the query into every
-// chosen list: it takes the next rank of the list's query counter and writes
-// its id and mask into the list's slot row, which the plan and the scan read.
+// The search runs the probe as two kernels:
+//   * probe_score_kernel: one CTA per tile of 64 centroids x 64 queries; the
+//     tile's queries sit in shared memory and every centroid row is read once
+//     per tile (not once per query), dotted by dp4a against 16 queries per
+//     thread, and the (score, list id) keys go to a [B][nlist] array that
+//     stays in L2;
+//   * probe_select_kernel: one CTA per query. The keys' score range, a 2048-bin
+//     histogram over it, and the suffix counts give the bin holding the
+//     nprobe-th best score, so only the keys at or above that bin (a few more
+//     than nprobe) go through the exact selection and the sort. The CTA then
+//     writes the probe result and files the query into every chosen list: it
+//     takes the next rank of the list's query counter and writes its id and
+//     mask into the list's slot row, which the plan and the scan read.
+// The allocation-free probe-only call keeps an older single-kernel form (CTAs
+// over query x centroid slices, last CTA merges), whose scratch is bounded.
 #include <mutex>
 
 #include "st_internal.cuh"
@@ -154,6 +160,161 @@ probe_kernel(SearchArgs a, int S)
     finish_query<BLOCK, kFile>(a, b, mk, n, sortbuf, pw, ss);
 }
 
+// ----------------------------------------------------------------------------
+// Search probe: tile scoring + per-query histogram-guided selection
+// ----------------------------------------------------------------------------
+constexpr int kTileC = 64;   // centroids per scoring CTA (one per thread of a query group)
+constexpr int kTileQ = 64;   // queries per scoring CTA
+constexpr int kQPer = 16;    // queries per thread
+constexpr int kScoreBlock = kTileC * (kTileQ / kQPer);
+
+__global__ void __launch_bounds__(kScoreBlock)
+probe_score_kernel(SearchArgs a)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    int4* sq = reinterpret_cast<int4*>(smem_raw);  // [kTileQ][np]
+    const int d = a.d, np = d >> 4, nlist = a.nlist;
+    const int c0 = blockIdx.x * kTileC, q0 = blockIdx.y * kTileQ;
+    const int nq = a.B - q0 < kTileQ ? a.B - q0 : kTileQ;
+    const int4* qsrc = reinterpret_cast<const int4*>(a.queries + int64_t(q0) * d);
+    for (int i = threadIdx.x; i < nq * np; i += kScoreBlock) sq[i] = qsrc[i];
+    __syncthreads();
+    const int c = c0 + (threadIdx.x % kTileC);
+    const int g = threadIdx.x / kTileC;  // this thread's queries: g*kQPer ..
+    if (c >= nlist || g * kQPer >= nq) return;
+    const int4* crow = reinterpret_cast<const int4*>(a.centroids + int64_t(c) * d);
+    const int4* qg = sq + g * kQPer * np;
+    int32_t acc[kQPer];
+#pragma unroll
+    for (int j = 0; j < kQPer; ++j) acc[j] = 0;
+    for (int p = 0; p < np; ++p) {
+        const int4 cv = __ldg(crow + p);
+#pragma unroll
+        for (int j = 0; j < kQPer; ++j) acc[j] = dot16(cv, qg[j * np + p], acc[j]);  // (rows past nq unused)
+    }
+    uint64_t* out = a.probe_keys + int64_t(q0 + g * kQPer) * nlist + c;
+#pragma unroll
+    for (int j = 0; j < kQPer; ++j)
+        if (g * kQPer + j < nq) out[int64_t(j) * nlist] = pack_key(acc[j], uint32_t(c));
+}
+
+template <int BLOCK>
+__global__ void __launch_bounds__(BLOCK)
+probe_select_kernel(SearchArgs a, int cap)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ SelectSmem ss;
+    __shared__ int32_t s_lo, s_hi, s_cut;
+    const int b = blockIdx.x;
+    const int nlist = a.nlist, P = a.P;
+    const int pw = next_pow2(P);
+    uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem_raw);   // max(pw, BLOCK) keys
+    uint64_t* cbuf = sortbuf + (pw > BLOCK ? pw : BLOCK);         // cap keys
+    uint64_t* keys = a.probe_keys + int64_t(b) * nlist;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = BLOCK / 32;
+
+    // score range
+    int32_t lo = INT32_MAX, hi = INT32_MIN;
+    for (int i = tid; i < nlist; i += BLOCK) {
+        const int32_t sc = key_score(keys[i]);
+        lo = sc < lo ? sc : lo;
+        hi = sc > hi ? sc : hi;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+        ss.part[warp] = uint32_t(lo);
+        ss.hist2[warp] = uint32_t(hi);
+    }
+    for (int i = tid; i < kSelBins; i += BLOCK) ss.hist[i] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        lo = lane < NW ? int32_t(ss.part[lane]) : INT32_MAX;
+        hi = lane < NW ? int32_t(ss.hist2[lane]) : INT32_MIN;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        if (lane == 0) {
+            s_lo = lo;
+            s_hi = hi;
+        }
+    }
+    __syncthreads();
+    lo = s_lo;
+    hi = s_hi;
+    int sh = 0;
+    while (((int64_t(hi) - lo) >> sh) >= kSelBins) ++sh;
+
+    // histogram of (score - lo) >> sh
+    for (int i = tid; i < nlist; i += BLOCK)
+        atomicAdd(&ss.hist[uint32_t((int64_t(key_score(keys[i])) - lo) >> sh)], 1u);
+    __syncthreads();
+
+    // the bin holding the P-th best score: thread t owns bins counted down from the top
+    if (tid == 0) s_cut = 0;
+    constexpr int PER = kSelBins / BLOCK;
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) local += ss.hist[kSelBins - 1 - (tid * PER + j)];
+    uint32_t total;
+    const uint32_t excl = block_excl_scan<BLOCK>(local, ss.part, total);
+    if (excl < uint32_t(P) && uint32_t(P) <= excl + local) {
+        uint32_t acc = excl;
+        for (int j = 0; j < PER; ++j) {
+            const int bin = kSelBins - 1 - (tid * PER + j);
+            acc += ss.hist[bin];
+            if (acc >= uint32_t(P)) {
+                s_cut = bin;
+                break;
+            }
+        }
+    }
+    __syncthreads();
+    // every key scoring at least the cut bin's lowest score
+    const int32_t cut_score = int32_t(int64_t(lo) + (int64_t(s_cut) << sh));
+    const uint64_t thr = pack_key(cut_score, 0xFFFFFFFFu);
+    const int m = block_collect_ge<BLOCK>(keys, nlist, thr, cbuf, cap, ss);
+    if (m <= cap)
+        finish_query<BLOCK, true>(a, b, cbuf, m, sortbuf, pw, ss);
+    else  // a crowded cut bin (many equal scores): select among all keys
+        finish_query<BLOCK, true>(a, b, keys, nlist, sortbuf, pw, ss);
+}
+
+constexpr int kProbeSelBlock = 1024;
+
+size_t probe_select_smem(int P, int* cap_out)
+{
+    const int pw = next_pow2(P);
+    const size_t sort_keys = size_t(pw > kProbeSelBlock ? pw : kProbeSelBlock);
+    int cap = 4 * pw > 4096 ? 4 * pw : 4096;
+    if ((sort_keys + cap) * 8 > 190 * 1024) cap = int(190 * 1024 / 8 - sort_keys);
+    if (cap_out) *cap_out = cap;
+    return (sort_keys + size_t(cap)) * 8;
+}
+
+cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s)
+{
+    const dim3 grid((a.nlist + kTileC - 1) / kTileC, (a.B + kTileQ - 1) / kTileQ);
+    const size_t qbytes = size_t(kTileQ) * a.d;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_score_kernel), 10, int(kTileQ * ST_MAX_D));
+    if (e != cudaSuccess) return e;
+    probe_score_kernel<<<grid, kScoreBlock, qbytes, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    int cap = 0;
+    const size_t smem = probe_select_smem(a.P, &cap);
+    e = ensure_smem_attr(reinterpret_cast<const void*>(probe_select_kernel<kProbeSelBlock>), 11, 200 * 1024);
+    if (e != cudaSuccess) return e;
+    probe_select_kernel<kProbeSelBlock><<<a.B, kProbeSelBlock, smem, s>>>(a, cap);
+    return cudaGetLastError();
+}
+
 int probe_slices(const SearchArgs& a, int num_sms)
 {
     // enough CTAs to cover the GPU twice, slices of at least 1024 centroids,
@@ -173,15 +334,6 @@ static size_t probe_smem_bytes(const SearchArgs& a, int S)
     size_t bytes = size_t(pw > kProbeBlock ? pw : kProbeBlock) * 8 + size_t(a.d);
     if (a.probe_keys == nullptr) bytes += size_t((a.nlist + S - 1) / S + 1) * 8;
     return bytes;
-}
-
-cudaError_t launch_probe(const SearchArgs& a, int S, cudaStream_t s)
-{
-    const size_t smem = probe_smem_bytes(a, S);
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock, true>), 0, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    probe_kernel<kProbeBlock, true><<<a.B * S, kProbeBlock, smem, s>>>(a, S);
-    return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------------------

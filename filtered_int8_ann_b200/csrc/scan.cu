@@ -15,32 +15,31 @@
 // (kWarpItems rows) x up to kQMax queries probing that list, so each probed
 // list is streamed once per batch whatever the number of queries probing it.
 // Warps are independent (one-warp CTAs, many per SM) and take units
-// round-robin, software-pipelined over three units:
+// round-robin. A warp tests one unit ahead of the one it scores, so every
+// memory round trip of a unit overlaps the previous unit's work:
 //   * signature planes: the index stores each chunk's signatures as bit-planes
 //     (layout.cu). A unit needs only the planes of the bits in the union of its
-//     queries' masks. Each of the warp's lanes copies 16 bytes of one such
-//     plane with cp.async (8 planes per warp instruction, L1 bypassed) into the
-//     next free slot of a small per-warp buffer (kPlaneSlots planes); the
-//     planes of the unit two ahead are requested as soon as this unit's test
-//     has released its buffer. A unit whose union is wider than the buffer
-//     reads its planes from global memory instead (slower, same result). Many
-//     tiny copies suit the load/store path better than the bulk-copy engine,
-//     whose per-request cost made 64-byte copies the bottleneck;
+//     queries' masks (for a single-query unit: the query's own mask bits, in
+//     order). Each lane copies 16 bytes of one such plane with cp.async (8
+//     planes per warp instruction, L1 bypassed) into the next slot of the
+//     warp's plane buffer (kPlaneSlots planes); the next unit's planes are
+//     requested as soon as this unit's test has released the buffer. A unit
+//     whose union is wider than the buffer reads its planes from global
+//     memory instead (slower, same result);
 //   * test: for each query, the two half-warps AND the planes of the two
-//     halves of the query's mask bits (a list precomputed once per search) for
-//     the 32 rows of the lane's block; one shuffle joins the halves, so 32 rows
-//     cost one AND per mask bit;
+//     halves of the query's mask bits for the 32 rows of the lane's block; one
+//     shuffle joins the halves, so 32 rows cost one AND per mask bit;
 //   * filter-before-load: per-query survivor counts reserve candidate slots
-//     (one atomic per unit and query, whose reply is needed only after the
-//     survivors' rows and dots); only survivors' rows are read (16-byte
-//     read-only loads) and dotted with dp4a against the query vectors (staged
-//     in shared memory by cp.async while the previous unit finished); a key's
-//     slot is its ballot rank among the unit's survivors of that query; each
+//     (one atomic per unit and query, answered while the previous unit is
+//     scored) and the survivors' rows are prefetched into L2; one iteration
+//     later only those rows are read (16-byte read-only loads) and dotted with
+//     dp4a against the query vectors (staged in shared memory by cp.async); a
+//     key's slot is its rank among the unit's survivors of that query; each
 //     key also counts into the query's score histogram, which the final top-k
 //     uses to find its cut without sorting every candidate.
-// cp.async groups complete in order; each unit commits exactly two groups
-// (the planes two ahead, then the next unit's query vectors), so fixed
-// wait_group depths find every copy: no spin loop, nothing to time out.
+// Every unit commits exactly two cp.async groups (planes of the unit two
+// ahead, then query vectors of the next unit), so fixed wait_group depths find
+// every copy: there is no spin loop and nothing to time out.
 #include "st_internal.cuh"
 
 namespace st {
@@ -49,14 +48,14 @@ constexpr int kPlaneSlots = 32;                         // planes one buffer hol
 constexpr int kPlaneBytes = kWarpItems / 8;             // 64 bytes per plane
 constexpr int kPlaneBufBytes = kPlaneSlots * kPlaneBytes;
 
-// Per-warp shared memory: 2 plane buffers | survivor offsets [kWarpItems] u16 |
-// pass words [kQMax][16] | query vectors [kQMax][d] | bit -> slot tables [2][128] |
-// slot -> bit [kPlaneSlots] | query ids [kQMax]
+// Per-warp shared memory: plane buffer | survivor offsets [2][kWarpItems] u16 |
+// pass words [2][kQMax][16] | query vectors [kQMax][d] | bit -> slot table [128] |
+// slot -> bit [kPlaneSlots]
 __host__ __device__ inline size_t scan_warp_bytes(int d, int W)
 {
     (void)W;
-    return (2 * kPlaneBufBytes + kWarpItems * 2 + kQMax * 16 * 4 + size_t(kQMax) * d + 2 * kMaskBitsMax +
-            kPlaneSlots + kQMax * 4 + 127) / 128 * 128;
+    return (kPlaneBufBytes + 2 * kWarpItems * 2 + 2 * kQMax * 16 * 4 + size_t(kQMax) * d + kMaskBitsMax +
+            kPlaneSlots + 127) / 128 * 128;
 }
 
 size_t scan_smem_bytes(int d, int W) { return size_t(kScanBlock / 32) * scan_warp_bytes(d, W); }
@@ -101,6 +100,12 @@ __device__ __forceinline__ void warp_or2(uint64_t& x, uint64_t& y)
     }
 }
 
+// L2 prefetch of a row (one per 32-byte sector)
+__device__ __forceinline__ void prefetch_l2(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // NP = d/16 when the row is held in registers (d = 64 or 128), 0 for any other
 // d (rows are then re-read from L1 for each eligible query).
 // (at most as many registers as keep the shared-memory-limited warp count resident)
@@ -118,21 +123,20 @@ scan_kernel(SearchArgs a)
     const int half = lane >> 4;  // which half of the mask bits it ANDs
 
     unsigned char* wb = smem_raw + size_t(warp) * scan_warp_bytes(d, W);
-    uint32_t* const pbuf0 = reinterpret_cast<uint32_t*>(wb);
-    uint32_t* const pbuf1 = reinterpret_cast<uint32_t*>(wb + kPlaneBufBytes);
-    uint16_t* surv = reinterpret_cast<uint16_t*>(wb + 2 * kPlaneBufBytes);              // [kWarpItems]
-    uint32_t* s_pass = reinterpret_cast<uint32_t*>(surv + kWarpItems);                   // [kQMax][16]
-    int4* s_q = reinterpret_cast<int4*>(s_pass + kQMax * 16);                            // [kQMax][np]
-    uint8_t* s_tab = reinterpret_cast<uint8_t*>(s_q) + size_t(kQMax) * d;                // [2][128]
-    uint8_t* s_inv = s_tab + 2 * kMaskBitsMax;                                           // [kPlaneSlots]
-    int32_t* s_qid = reinterpret_cast<int32_t*>(s_inv + kPlaneSlots);                    // [kQMax]
+    uint32_t* const pbuf = reinterpret_cast<uint32_t*>(wb);
+    uint16_t* const surv2 = reinterpret_cast<uint16_t*>(wb + kPlaneBufBytes);            // [2][kWarpItems]
+    uint32_t* const pass2 = reinterpret_cast<uint32_t*>(surv2 + 2 * kWarpItems);         // [2][kQMax][16]
+    int4* const s_q = reinterpret_cast<int4*>(pass2 + 2 * kQMax * 16);                  // [kQMax][np]
+    uint8_t* const s_tab = reinterpret_cast<uint8_t*>(s_q) + size_t(kQMax) * d;          // [128]
+    uint8_t* const s_inv = s_tab + kMaskBitsMax;                                         // [kPlaneSlots]
 
     const int n_units = a.ctl->n_units < a.max_units ? a.ctl->n_units : a.max_units;
     const int stride = gridDim.x * (kScanBlock / 32);
     int u = blockIdx.x * (kScanBlock / 32) + warp;
     if (u >= n_units) return;
 
-    // unit entry: {first row, chunk, first query slot, rows << 16 | queries}
+    // unit entry: {first row, chunk, first query slot, rows << 16 | queries};
+    // lane s < queries holds query s's id and mask
     auto load_slots = [&](const int4& e, int& qid, uint64_t& m0, uint64_t& m1) {
         qid = 0;
         m0 = 0;
@@ -144,24 +148,12 @@ scan_kernel(SearchArgs a)
             m1 = m.y;
         }
     };
-    // query ids of a unit -> shared memory, its query vectors by cp.async
-    auto stage_queries = [&](int qn, int qid) {
-        __syncwarp();  // earlier reads of s_qid / s_q are done
-        if (lane < qn) s_qid[lane] = qid;
-        __syncwarp();
-        for (int idx = lane; idx < qn * np; idx += 32) {
-            const int s = idx / np, p = idx - s * np;
-            cp_async16(s_q + s * np + p, a.queries + int64_t(s_qid[s]) * d + 16 * p);
-        }
-    };
 
-    // Request the planes of a unit whose entry is `e` and whose slots (lanes <
-    // its query count) hold masks m0/m1, into buffer `bb`; returns the number
-    // of planes the buffer then holds, or -1 when the test must read global
-    // planes. A single-query unit needs no union: its planes are the query's
-    // mask bits in increasing order, listed by the probe.
-    auto request_planes = [&](const int4& e, int qid, uint64_t m0, uint64_t m1, int bb) -> int {
-        uint32_t* buf = bb ? pbuf1 : pbuf0;
+    // Request a unit's planes into the buffer; returns the number of planes it
+    // then holds, or -1 when the test must read global planes. A single-query
+    // unit needs no union: its planes are the query's mask bits in increasing
+    // order, listed by the probe.
+    auto request_planes = [&](const int4& e, int qid, uint64_t m0, uint64_t m1) -> int {
         if ((e.w & 0xFFFF) == 1) {
             const int q = __shfl_sync(0xffffffffu, qid, 0);
             const int nb = __ldg(a.qnbits + q);
@@ -169,121 +161,88 @@ scan_kernel(SearchArgs a)
             const uint8_t* bits = a.qbits + int64_t(q) * kMaskBitsMax;
             const uint32_t* src = a.planes + int64_t(e.y) * NPL * 16 + (lane & 3) * 4;
             for (int j = lane >> 2; j < nb; j += 8)
-                cp_async16_cg(buf + j * 16 + (lane & 3) * 4, src + __ldg(bits + j) * 16);
+                cp_async16_cg(pbuf + j * 16 + (lane & 3) * 4, src + __ldg(bits + j) * 16);
             return nb;
         }
         uint64_t x = m0, y = m1;
         warp_or2(x, y);
-        if (!issue_planes<W>(a, e.y, x, y, buf, s_tab + bb * kMaskBitsMax, s_inv, lane)) return -1;
+        if (!issue_planes<W>(a, e.y, x, y, pbuf, s_tab, s_inv, lane)) return -1;
         return __popcll(x) + (W > 1 ? __popcll(y) : 0);
     };
 
-    // prologue: entries of the first three units, slots of the first two;
-    // groups: planes(0), queries(0), planes(1)
-    int4 e_cur = a.units[u];
-    int4 e_nxt = make_int4(0, 0, 0, 0), e_n2 = make_int4(0, 0, 0, 0);
-    const bool has_nxt0 = u + stride < n_units;
-    if (has_nxt0) e_nxt = a.units[u + stride];
-    if (u + 2 * stride < n_units) e_n2 = a.units[u + 2 * stride];
-    int qid_c, qid_n = 0;
-    uint64_t m0_c, m1_c, m0_n = 0, m1_n = 0;
-    load_slots(e_cur, qid_c, m0_c, m1_c);
-    if (has_nxt0) load_slots(e_nxt, qid_n, m0_n, m1_n);
-    int held0 = request_planes(e_cur, qid_c, m0_c, m1_c, 0);  // planes held by buffer 0 / 1 (-1: global)
-    cp_async_commit();
-    stage_queries(e_cur.w & 0xFFFF, qid_c);
-    cp_async_commit();
-    int held1 = has_nxt0 ? request_planes(e_nxt, qid_n, m0_n, m1_n, 1) : -1;
-    cp_async_commit();
-    int b = 0;
+    // query vectors of a unit -> shared memory by cp.async
+    auto stage_queries = [&](int qn, int qid) {
+        for (int i0 = 0; i0 < qn * np; i0 += 32) {
+            const int idx = i0 + lane;
+            const int sq = idx / np;
+            const int qg = __shfl_sync(0xffffffffu, qid, sq < qn ? sq : qn - 1);
+            if (idx < qn * np) cp_async16(s_q + idx, a.queries + int64_t(qg) * d + 16 * (idx - sq * np));
+        }
+    };
 
-    for (; u < n_units; u += stride) {
-        const int64_t ib = e_cur.x;
-        const int chunk = e_cur.y;
-        const int len = e_cur.w >> 16;
-        const int qn = e_cur.w & 0xFFFF;
-        const uint32_t* pb = b ? pbuf1 : pbuf0;
-        const uint8_t* tab = s_tab + b * kMaskBitsMax;
-        const int held = b ? held1 : held0;
-        const bool in_smem = held >= 0;
-        const bool single = qn == 1 && in_smem;  // warp-uniform fast path
-        const bool has_n2 = u + 2 * stride < n_units;
-        const bool has_n3 = u + 3 * stride < n_units;
-
-        // background loads: the entry three units ahead, the slots of the unit
-        // two ahead (whose entry arrived during the previous unit)
-        int4 e_n3 = make_int4(0, 0, 0, 0);
-        if (has_n3) e_n3 = a.units[u + 3 * stride];
-        int qid_2 = 0;
-        uint64_t m0_2 = 0, m1_2 = 0;
-        if (has_n2) load_slots(e_n2, qid_2, m0_2, m1_2);
-
-        // this unit's planes: pending groups are at most [queries(u), planes(u+1)]
-        cp_async_wait_group<2>();
-        __syncwarp();
-
-        // test: pass word of query s for block `blk` = AND of its mask planes;
-        // the two half-warps AND the two halves of the query's mask bits
+    // Test a unit whose planes are in the buffer (held >= 0) or in global
+    // memory: pass words -> pass[s][blk]; returns the OR over queries in `any`
+    // and, in lane s, query s's survivor count (general path only).
+    auto test_unit = [&](const int4& e, int qid, int held, uint32_t* pass, uint32_t& any, uint32_t& mycnt) {
+        const int len = e.w >> 16;
+        const int qn = e.w & 0xFFFF;
         const uint32_t valid = len >= 32 * (blk + 1) ? 0xFFFFFFFFu
                              : (len <= 32 * blk ? 0u : ((1u << (len - 32 * blk)) - 1u));
-        uint32_t any = 0;
-        uint32_t mycnt = 0;  // lane s: survivors of query s
-        if (single) {
+        any = 0;
+        mycnt = 0;
+        if (qn == 1 && held >= 0) {
             // the buffer holds exactly the query's planes, in bit order
             const int h0 = (held + 1) >> 1;
             const int j1 = half ? held : h0;
             int j = half ? h0 : 0;
             uint32_t acc = 0xFFFFFFFFu;
             for (; j + 4 <= j1; j += 4)
-                acc &= pb[j * 16 + blk] & pb[(j + 1) * 16 + blk] & pb[(j + 2) * 16 + blk] & pb[(j + 3) * 16 + blk];
-            for (; j < j1; ++j) acc &= pb[j * 16 + blk];
+                acc &= pbuf[j * 16 + blk] & pbuf[(j + 1) * 16 + blk] & pbuf[(j + 2) * 16 + blk] &
+                       pbuf[(j + 3) * 16 + blk];
+            for (; j < j1; ++j) acc &= pbuf[j * 16 + blk];
             acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
             any = acc & valid;
-        } else {
-            const uint32_t* gpl = a.planes + int64_t(chunk) * NPL * 16 + blk;
-            for (int s = 0; s < qn; ++s) {
-                const int qg = s_qid[s];
-                const int nb = __ldg(a.qnbits + qg);
-                const int h0 = (nb + 1) >> 1;
-                const uint8_t* bits = a.qbits + int64_t(qg) * kMaskBitsMax;
-                const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
-                // four independent bit -> slot -> plane chains per step
-                uint32_t acc = 0xFFFFFFFFu;
-                if (in_smem) {
-                    int j = j0;
-                    for (; j + 4 <= j1; j += 4) {
-                        const int b0 = __ldg(bits + j), b1 = __ldg(bits + j + 1);
-                        const int b2 = __ldg(bits + j + 2), b3 = __ldg(bits + j + 3);
-                        const int s0 = tab[b0], s1 = tab[b1], s2 = tab[b2], s3 = tab[b3];
-                        acc &= pb[s0 * 16 + blk] & pb[s1 * 16 + blk] & pb[s2 * 16 + blk] & pb[s3 * 16 + blk];
-                    }
-                    for (; j < j1; ++j) acc &= pb[tab[__ldg(bits + j)] * 16 + blk];
-                } else {
-                    for (int j = j0; j < j1; ++j) acc &= __ldg(gpl + __ldg(bits + j) * 16);
+            return;
+        }
+        const uint32_t* gpl = a.planes + int64_t(e.y) * NPL * 16 + blk;
+        for (int s = 0; s < qn; ++s) {
+            const int qg = __shfl_sync(0xffffffffu, qid, s);
+            const int nb = __ldg(a.qnbits + qg);
+            const int h0 = (nb + 1) >> 1;
+            const uint8_t* bits = a.qbits + int64_t(qg) * kMaskBitsMax;
+            const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
+            // four independent bit -> slot -> plane chains per step
+            uint32_t acc = 0xFFFFFFFFu;
+            if (held >= 0) {
+                int j = j0;
+                for (; j + 4 <= j1; j += 4) {
+                    const int b0 = __ldg(bits + j), b1 = __ldg(bits + j + 1);
+                    const int b2 = __ldg(bits + j + 2), b3 = __ldg(bits + j + 3);
+                    const int s0 = s_tab[b0], s1 = s_tab[b1], s2 = s_tab[b2], s3 = s_tab[b3];
+                    acc &= pbuf[s0 * 16 + blk] & pbuf[s1 * 16 + blk] & pbuf[s2 * 16 + blk] & pbuf[s3 * 16 + blk];
                 }
-                acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
-                acc &= valid;
-                if (half == 0) s_pass[s * 16 + blk] = acc;
-                any |= acc;
-                // survivors of query s: half 0 holds the 16 pass words; the full
-                // 32-lane reduction leaves the total in every lane
-                uint32_t c = half == 0 ? uint32_t(__popc(acc)) : 0u;
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-                if (lane == s) mycnt = c;
+                for (; j < j1; ++j) acc &= pbuf[s_tab[__ldg(bits + j)] * 16 + blk];
+            } else {
+                for (int j = j0; j < j1; ++j) acc &= __ldg(gpl + __ldg(bits + j) * 16);
             }
+            acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
+            acc &= valid;
+            if (half == 0) pass[s * 16 + blk] = acc;
+            any |= acc;
+            // survivors of query s: half 0 holds the 16 pass words; the full
+            // 32-lane reduction leaves the total in every lane
+            uint32_t c = half == 0 ? uint32_t(__popc(acc)) : 0u;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+            if (lane == s) mycnt = c;
         }
+    };
 
-        // buffer b is free: request the planes of the unit two ahead
-        if (has_n2) {
-            __syncwarp();  // every lane is done reading buffer b
-            const int h2 = request_planes(e_n2, qid_2, m0_2, m1_2, b);
-            if (b) held1 = h2;
-            else held0 = h2;
-        }
-        cp_async_commit();
-
-        // survivor row offsets, block by block
+    // After a unit's test: survivor row offsets -> sv, one reservation per
+    // query (lane s, the reply lands in `base`), L2 prefetch of the first
+    // survivors' rows. Returns the number of survivors.
+    auto settle_unit = [&](const int4& e, int qid, bool single, uint32_t any, uint32_t mycnt, uint16_t* sv,
+                           uint32_t& base) -> int {
         const uint32_t mine = half == 0 ? uint32_t(__popc(any)) : 0u;
         uint32_t incl = mine;
 #pragma unroll
@@ -298,47 +257,110 @@ scan_kernel(SearchArgs a)
             while (rest) {
                 const int i = __ffs(rest) - 1;
                 rest &= rest - 1u;
-                surv[pos++] = uint16_t(32 * blk + i);
+                sv[pos++] = uint16_t(32 * blk + i);
             }
         }
-
-        // per-query survivor counts -> one reservation each (lane s); the
-        // reply is first needed when the keys are stored
         if (single && lane == 0) mycnt = uint32_t(nsurv);
-        uint32_t base = 0;
-        if (lane < qn && mycnt) {
-            base = atomicAdd(&a.cand_cnt[int64_t(qid_c) * kCntStride], mycnt);
-            atomicAdd(&a.eligible_cnt[int64_t(qid_c) * (kCntStride / 2)], (unsigned long long)mycnt);
+        base = 0;
+        if (lane < (e.w & 0xFFFF) && mycnt) {
+            base = atomicAdd(&a.cand_cnt[int64_t(qid) * kCntStride], mycnt);
+            atomicAdd(&a.eligible_cnt[int64_t(qid) * (kCntStride / 2)], (unsigned long long)mycnt);
+        }
+        __syncwarp();
+        const int npf = nsurv < 64 ? nsurv : 64;
+        for (int idx = lane; idx < npf; idx += 32) {
+            const int8_t* row = a.items + (int64_t(e.x) + sv[idx]) * d;
+            for (int o = 0; o < d; o += 32) prefetch_l2(row + o);
+        }
+        return nsurv;
+    };
+
+    // prologue: test unit 0; groups planes(0) [waited], planes(1), queries(0)
+    int4 e_cur = a.units[u];
+    int4 e_nxt = make_int4(0, 0, 0, 0), e_n2 = make_int4(0, 0, 0, 0);
+    if (u + stride < n_units) e_nxt = a.units[u + stride];
+    if (u + 2 * stride < n_units) e_n2 = a.units[u + 2 * stride];
+    int qid_c, qid_n = 0;
+    uint64_t m0_n = 0, m1_n = 0;
+    int held;          // planes the buffer holds for the next unit to test (-1: global)
+    uint32_t base_c;   // lane s: reservation of query s of the unit being scored
+    int nsurv_c;       // survivors of the unit being scored
+    bool single_c;     // it took the single-query path
+    {
+        uint64_t m0_c, m1_c;
+        load_slots(e_cur, qid_c, m0_c, m1_c);
+        if (u + stride < n_units) load_slots(e_nxt, qid_n, m0_n, m1_n);
+        const int held0 = request_planes(e_cur, qid_c, m0_c, m1_c);
+        cp_async_commit();
+        cp_async_wait_group<0>();
+        __syncwarp();
+        uint32_t any, mycnt;
+        test_unit(e_cur, qid_c, held0, pass2, any, mycnt);
+        single_c = (e_cur.w & 0xFFFF) == 1 && held0 >= 0;
+        __syncwarp();
+        held = u + stride < n_units ? request_planes(e_nxt, qid_n, m0_n, m1_n) : -1;
+        cp_async_commit();
+        nsurv_c = settle_unit(e_cur, qid_c, single_c, any, mycnt, surv2, base_c);
+    }
+    stage_queries(e_cur.w & 0xFFFF, qid_c);
+    cp_async_commit();
+    int cb = 0;
+
+    for (; u < n_units; u += stride) {
+        const bool has_n1 = u + stride < n_units;
+        const bool has_n2 = u + 2 * stride < n_units;
+        const bool has_n3 = u + 3 * stride < n_units;
+
+        // background loads: the entry three units ahead, the slots of the unit
+        // two ahead (whose entry arrived during the previous unit)
+        int4 e_n3 = make_int4(0, 0, 0, 0);
+        if (has_n3) e_n3 = a.units[u + 3 * stride];
+        int qid_2 = 0;
+        uint64_t m0_2 = 0, m1_2 = 0;
+        if (has_n2) load_slots(e_n2, qid_2, m0_2, m1_2);
+
+        // test the next unit: its planes are the older of the (at most two)
+        // pending groups [planes(u+1), queries(u)]
+        int nsurv_n = 0;
+        uint32_t base_n = 0;
+        bool single_n = false;
+        if (has_n1) {
+            cp_async_wait_group<1>();
+            __syncwarp();
+            uint32_t any, mycnt;
+            test_unit(e_nxt, qid_n, held, pass2 + (cb ^ 1) * kQMax * 16, any, mycnt);
+            single_n = (e_nxt.w & 0xFFFF) == 1 && held >= 0;
+            __syncwarp();
+            held = has_n2 ? request_planes(e_n2, qid_2, m0_2, m1_2) : -1;
+            cp_async_commit();
+            nsurv_n = settle_unit(e_nxt, qid_n, single_n, any, mycnt, surv2 + (cb ^ 1) * kWarpItems, base_n);
+        } else {
+            cp_async_commit();  // two groups per unit, always
         }
 
-        // this unit's query vectors: pending groups are at most [planes(u+2)]
+        // score this unit: its query vectors are pending at most behind [planes(u+2)]
         cp_async_wait_group<1>();
         __syncwarp();
-
-        // rows of the survivors (one load per survivor), dots, keys into the
-        // reserved slots
-        if (single) {
+        const int64_t ib = e_cur.x;
+        const int qn = e_cur.w & 0xFFFF;
+        const uint16_t* surv = surv2 + cb * kWarpItems;
+        const uint32_t* s_pass = pass2 + cb * kQMax * 16;
+        if (single_c) {
             // every survivor is a key of the one query, in survivor order
-            const int qg = s_qid[0];
+            const int qg = __shfl_sync(0xffffffffu, qid_c, 0);
+            const uint32_t base0 = __shfl_sync(0xffffffffu, base_c, 0);
             uint64_t* cand = a.cand + int64_t(qg) * a.cap;
             uint32_t* hist = a.hist + int64_t(qg) * kHistBins;
-            for (int c0 = 0; c0 < nsurv; c0 += 32) {
+            for (int c0 = 0; c0 < nsurv_c; c0 += 32) {
                 const int idx = c0 + lane;
-                int4 row[NP > 0 ? NP : 1];
-                const int4* rp = nullptr;
-                int64_t i = 0;
-                if (idx < nsurv) {
-                    i = ib + surv[idx];
-                    rp = reinterpret_cast<const int4*>(a.items + i * d);
-                    if (NP > 0) {
-#pragma unroll
-                        for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
-                    }
-                }
-                const uint32_t base0 = __shfl_sync(0xffffffffu, base, 0);
-                if (idx < nsurv) {
+                if (idx < nsurv_c) {
+                    const int64_t i = ib + surv[idx];
+                    const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);
                     int32_t acc0 = 0, acc1 = 0;
                     if (NP > 0) {
+                        int4 row[NP > 0 ? NP : 1];
+#pragma unroll
+                        for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
 #pragma unroll
                         for (int p = 0; p < (NP > 0 ? NP : 1); p += 2) {
                             acc0 = dot16(row[p], s_q[p], acc0);
@@ -357,13 +379,13 @@ scan_kernel(SearchArgs a)
             // a key's slot is its ballot rank among this unit's survivors of
             // the same query
             uint32_t run = 0;  // lane s: keys of query s written so far
-            for (int c0 = 0; c0 < nsurv; c0 += 32) {
+            for (int c0 = 0; c0 < nsurv_c; c0 += 32) {
                 const int idx = c0 + lane;
                 int off = -1;
                 int64_t i = 0;
                 int4 row[NP > 0 ? NP : 1];
                 const int4* rp = nullptr;
-                if (idx < nsurv) {
+                if (idx < nsurv_c) {
                     off = surv[idx];
                     i = ib + off;
                     rp = reinterpret_cast<const int4*>(a.items + i * d);
@@ -378,7 +400,8 @@ scan_kernel(SearchArgs a)
                     const bool on = off >= 0 && ((pw[s * 16] >> bit) & 1u);
                     const unsigned bal = __ballot_sync(0xffffffffu, on);
                     if (bal == 0u) continue;
-                    const uint32_t slot0 = __shfl_sync(0xffffffffu, base, s) + __shfl_sync(0xffffffffu, run, s);
+                    const uint32_t slot0 = __shfl_sync(0xffffffffu, base_c, s) + __shfl_sync(0xffffffffu, run, s);
+                    const int qg = __shfl_sync(0xffffffffu, qid_c, s);
                     if (on) {
                         const int4* qs = s_q + s * np;
                         int32_t acc0 = 0, acc1 = 0;
@@ -393,7 +416,6 @@ scan_kernel(SearchArgs a)
                         }
                         const uint64_t pos = uint64_t(slot0) + __popc(bal & lanemask_lt());
                         const int32_t score = acc0 + acc1;
-                        const int qg = s_qid[s];
                         if (pos < uint64_t(a.cap)) a.cand[int64_t(qg) * a.cap + int64_t(pos)] = pack_key(score, uint32_t(i));
                         atomicAdd(&a.hist[int64_t(qg) * kHistBins + score_bin(score, a.smax, a.hshift)], 1u);
                     }
@@ -403,19 +425,21 @@ scan_kernel(SearchArgs a)
         }
 
         // the next unit's query vectors (group queries(u+1))
-        stage_queries(e_nxt.w & 0xFFFF, qid_n);
+        __syncwarp();
+        if (has_n1) stage_queries(e_nxt.w & 0xFFFF, qid_n);
         cp_async_commit();
 
         e_cur = e_nxt;
         e_nxt = e_n2;
         e_n2 = e_n3;
         qid_c = qid_n;
-        m0_c = m0_n;
-        m1_c = m1_n;
         qid_n = qid_2;
         m0_n = m0_2;
         m1_n = m1_2;
-        b ^= 1;
+        base_c = base_n;
+        nsurv_c = nsurv_n;
+        single_c = single_n;
+        cb ^= 1;
     }
     cp_async_wait_all();  // no copy may land after the warp has left
 }

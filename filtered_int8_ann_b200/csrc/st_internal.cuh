@@ -13,7 +13,7 @@ namespace st {
 // ----------------------------------------------------------------------------
 constexpr int kScanBlock = 32;             // threads per scan CTA (one independent warp)
 constexpr int kWarpItems = 512;            // list rows per work unit (one warp)
-constexpr int kQMax = 32;                  // queries per work unit (one bit each)
+constexpr int kQMax = 16;                  // queries per work unit
 
 constexpr int kProbeBlock = 512;
 constexpr int kProbeSmemKeys = 16384;      // nlist up to this keeps probe keys in smem
@@ -402,7 +402,9 @@ __device__ int32_t block_collect_ge_wide(const uint64_t* keys, int64_t n, uint64
         }
     }
     __syncthreads();
-    return s.count;
+    const int32_t count = s.count;
+    __syncthreads();  // a following collect may reset the counter at once
+    return count;
 }
 
 // Copy every key >= thr from keys[0..n) into out[] (at most out_cap); returns
@@ -431,7 +433,9 @@ __device__ int32_t block_collect_ge(const uint64_t* keys, int64_t n, uint64_t th
         }
     }
     __syncthreads();
-    return s.count;
+    const int32_t count = s.count;
+    __syncthreads();  // a following collect may reset the counter at once
+    return count;
 }
 
 // Sort a[0..m) descending with a bitonic network in shared memory (the keys
@@ -571,7 +575,7 @@ cudaError_t ensure_smem_attr(const void* func, int slot, int bytes);
 // Kernel launchers (defined in the .cu files)
 // ----------------------------------------------------------------------------
 int probe_slices(const SearchArgs& a, int num_sms);
-cudaError_t launch_probe(const SearchArgs& a, int S, cudaStream_t s);
+cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s);
 size_t probe_noalloc_scratch_bytes(int B, int S, int P, int nlist, bool keys_in_smem);
 cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
