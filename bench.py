@@ -27,7 +27,7 @@ sys.path.insert(0, ROOT)
 from workloads import WORKLOADS, generate  # noqa: E402
 
 METRIC = "queries/s & item-scores/s (80M int8 IVF, nprobe64, top-2048); % HBM roofline"
-KERNELS_PER_SEARCH = 4   # probe, plan, scan, select (plus one memset node)
+KERNELS_PER_SEARCH = 8  # probe score + probe select, units alloc + write, scan, select hist + scatter + finish
 
 
 def parse():

@@ -39,6 +39,10 @@ cudaError_t ensure_smem_attr(const void* func, int slot, int bytes)
     if (e != cudaSuccess) return e;
     if (dev < 64 && slot < 32 && (done[dev] >> slot) & 1u) return cudaSuccess;
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // every large-shared-memory kernel asks for the same (largest) carveout, so
+    // an SM need not reconfigure its L1 / shared split between them
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess && dev < 64 && slot < 32) __atomic_fetch_or(&done[dev], 1u << slot, __ATOMIC_RELAXED);
     return e;
 }
@@ -90,7 +94,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // must start at zero come first, so one memset clears them.
 struct ScratchLayout {
     size_t total = 0;
-    size_t off_list_cnt, off_cand_cnt, off_elig, off_hist, off_ctl, zero_bytes;
+    size_t off_list_cnt, off_cand_cnt, off_elig, off_rng, off_sel_hist, off_sel_cursor, off_ctl, zero_bytes;
+    size_t off_sel_out, off_sel_tie;
     size_t off_probe, off_probe_keys, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_units, off_cand;
     size_t add(size_t bytes)
     {
@@ -138,11 +143,13 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_list_cnt = L.add(nl4 * 4);
     L.off_cand_cnt = L.add(size_t(B) * st::kCntStride * 4);
     L.off_elig = L.add(size_t(B) * st::kCntStride * 4);
-    L.off_hist = L.add(size_t(B) * st::kHistBins * 4);
+    L.off_rng = L.add(size_t(B) * st::kCntStride * 4);
+    L.off_sel_hist = L.add(size_t(B) * st::kSelBins * 4);
+    L.off_sel_cursor = L.add(size_t(B) * st::kSelBins * 4);
     L.off_ctl = L.add(sizeof(st::PlanCtl));
     L.zero_bytes = L.total;
     L.off_probe = L.add(size_t(B) * nprobe * 4);
-    L.off_probe_keys = L.add(size_t(B) * idx->nlist * 8);
+    L.off_probe_keys = L.add(size_t(B) * size_t(st::probe_keys_ld(idx->nlist)) * 8);
     L.off_list_ustart = L.add(nl4 * 4);
     L.off_qbits = L.add(size_t(B) * st::kMaskBitsMax);
     L.off_qnbits = L.add(size_t(B) * 4);
@@ -150,6 +157,8 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_qmask = L.add(slots * 16);
     L.off_units = L.add(size_t(max_units) * 16);
     L.off_cand = L.add(size_t(B) * size_t(cap) * 8);
+    L.off_sel_out = L.add(size_t(B) * size_t(k) * 8);
+    L.off_sel_tie = L.add(size_t(B) * st::kSelTieCap * 8);
 
     unsigned char* base = nullptr;
     cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&base), L.total, idx->pool, stream);
@@ -182,13 +191,9 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.list_cnt = reinterpret_cast<int32_t*>(base + L.off_list_cnt);
     a.cand_cnt = reinterpret_cast<uint32_t*>(base + L.off_cand_cnt);
     a.eligible_cnt = reinterpret_cast<unsigned long long*>(base + L.off_elig);
-    a.hist = reinterpret_cast<uint32_t*>(base + L.off_hist);
-    a.smax = idx->d * 128 * 128;
-    {
-        int bits = 0;
-        while ((int64_t(1) << bits) < 2 * int64_t(a.smax)) ++bits;
-        a.hshift = bits > st::kSelBits ? bits - st::kSelBits : 0;
-    }
+    a.score_rng = reinterpret_cast<uint32_t*>(base + L.off_rng);
+    a.sel_hist = reinterpret_cast<uint32_t*>(base + L.off_sel_hist);
+    a.sel_cursor = reinterpret_cast<uint32_t*>(base + L.off_sel_cursor);
     a.ctl = reinterpret_cast<st::PlanCtl*>(base + L.off_ctl);
     a.probe = reinterpret_cast<int32_t*>(base + L.off_probe);
     a.probe_keys = reinterpret_cast<uint64_t*>(base + L.off_probe_keys);
@@ -201,6 +206,8 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.max_units = int32_t(max_units);
     a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
     a.cap = cap;
+    a.sel_out = reinterpret_cast<uint64_t*>(base + L.off_sel_out);
+    a.sel_tie = reinterpret_cast<uint64_t*>(base + L.off_sel_tie);
     a.err = idx->err;
 
     auto mark = [&](int i) {
@@ -214,7 +221,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     mark(2);
     if (e == cudaSuccess) e = st::launch_scan(a, idx->num_sms, stream);
     mark(3);
-    if (e == cudaSuccess) e = st::launch_select(a, stream);
+    if (e == cudaSuccess) e = st::launch_select(a, idx->num_sms, stream);
     mark(4);
     if (e == cudaSuccess && extras && extras->probe)
         e = cudaMemcpyAsync(extras->probe, a.probe, size_t(B) * nprobe * 4, cudaMemcpyDeviceToDevice, stream);

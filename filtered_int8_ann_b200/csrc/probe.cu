@@ -29,26 +29,20 @@
 
 namespace st {
 
-// kFile: also file the query into its lists (the search); the allocation-free
-// probe-only call sets it false and writes the probe result alone.
+// Write the probe result of query b from its P best keys, sorted (sorted[p],
+// p < P). kFile: also file the query into its lists (the search): the query's
+// mask bits in increasing order, then for each chosen list the next rank of
+// the list's query counter and the query's id and mask in that slot of the
+// list's slot row. The allocation-free probe-only call writes the result alone.
 template <int BLOCK, bool kFile>
-__device__ void finish_query(const SearchArgs& a, int b, uint64_t* keys, int n, uint64_t* sortbuf,
-                             int pw, SelectSmem& ss)
+__device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
 {
     const int P = a.P;
-    uint64_t thr = 1;  // key 0 marks an empty partial slot and is never a real key
-    if (P < n) thr = block_select_threshold<BLOCK>(keys, n, P, ss, a.err);
-    const int got = block_collect_ge<BLOCK>(keys, n, thr < 1 ? 1 : thr, sortbuf, pw, ss);
-    if (threadIdx.x == 0 && got != P) set_error(a.err, kErrSelectCount);
-    for (int i = (got < pw ? got : pw) + threadIdx.x; i < pw; i += BLOCK) sortbuf[i] = 0;
-    __syncthreads();
-    block_sort_desc_counting<BLOCK>(sortbuf, got < pw ? got : pw, keys, ss);  // the score keys are done with
     if (!kFile) {
-        for (int p = threadIdx.x; p < P; p += BLOCK) a.probe[int64_t(b) * P + p] = int(key_id(sortbuf[p]));
+        for (int p = threadIdx.x; p < P; p += BLOCK) a.probe[int64_t(b) * P + p] = int(key_id(sorted[p]));
         return;
     }
     const int W = a.W;
-    // the query's mask bits in increasing order
     if (threadIdx.x < 32) {
         const uint64_t m0 = a.qmasks[int64_t(b) * W];
         const uint64_t m1 = W > 1 ? a.qmasks[int64_t(b) * W + 1] : 0ull;
@@ -65,7 +59,7 @@ __device__ void finish_query(const SearchArgs& a, int b, uint64_t* keys, int n, 
         if (lane == 0) a.qnbits[b] = n_before;
     }
     for (int p = threadIdx.x; p < P; p += BLOCK) {
-        const int L = int(key_id(sortbuf[p]));
+        const int L = int(key_id(sorted[p]));
         a.probe[int64_t(b) * P + p] = L;
         if (L >= 0 && L < a.nlist) {
             const int r = atomicAdd(&a.list_cnt[L], 1);
@@ -76,6 +70,23 @@ __device__ void finish_query(const SearchArgs& a, int b, uint64_t* keys, int n, 
             reinterpret_cast<ulonglong2*>(a.qmask_slot)[slot] = make_ulonglong2(m0, m1);
         }
     }
+}
+
+// Select query b's P best of the n keys (radix threshold), sort them, and
+// write its probe result (file_query).
+template <int BLOCK, bool kFile>
+__device__ void finish_query(const SearchArgs& a, int b, uint64_t* keys, int n, uint64_t* sortbuf,
+                             int pw, SelectSmem& ss)
+{
+    const int P = a.P;
+    uint64_t thr = 1;  // key 0 marks an empty partial slot and is never a real key
+    if (P < n) thr = block_select_threshold<BLOCK>(keys, n, P, ss, a.err);
+    const int got = block_collect_ge<BLOCK>(keys, n, thr < 1 ? 1 : thr, sortbuf, pw, ss);
+    if (threadIdx.x == 0 && got != P) set_error(a.err, kErrSelectCount);
+    for (int i = (got < pw ? got : pw) + threadIdx.x; i < pw; i += BLOCK) sortbuf[i] = 0;
+    __syncthreads();
+    block_sort_desc_counting<BLOCK>(sortbuf, got < pw ? got : pw, keys, ss);  // the score keys are done with
+    file_query<BLOCK, kFile>(a, b, sortbuf);
 }
 
 template <int BLOCK, bool kFile>
@@ -192,110 +203,59 @@ probe_score_kernel(SearchArgs a)
 #pragma unroll
         for (int j = 0; j < kQPer; ++j) acc[j] = dot16(cv, qg[j * np + p], acc[j]);  // (rows past nq unused)
     }
-    uint64_t* out = a.probe_keys + int64_t(q0 + g * kQPer) * nlist + c;
+    const int64_t ld = probe_keys_ld(nlist);
+    uint64_t* out = a.probe_keys + int64_t(q0 + g * kQPer) * ld + c;
 #pragma unroll
     for (int j = 0; j < kQPer; ++j)
-        if (g * kQPer + j < nq) out[int64_t(j) * nlist] = pack_key(acc[j], uint32_t(c));
+        if (g * kQPer + j < nq) out[int64_t(j) * ld] = pack_key(acc[j], uint32_t(c));
 }
 
 template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK)
-probe_select_kernel(SearchArgs a, int cap)
+probe_select_kernel(SearchArgs a, int stage_cap, int tie_cap)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ SelectSmem ss;
-    __shared__ int32_t s_lo, s_hi, s_cut;
     const int b = blockIdx.x;
     const int nlist = a.nlist, P = a.P;
-    const int pw = next_pow2(P);
-    uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem_raw);   // max(pw, BLOCK) keys
-    uint64_t* cbuf = sortbuf + (pw > BLOCK ? pw : BLOCK);         // cap keys
-    uint64_t* keys = a.probe_keys + int64_t(b) * nlist;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int NW = BLOCK / 32;
-
-    // score range
-    int32_t lo = INT32_MAX, hi = INT32_MIN;
-    for (int i = tid; i < nlist; i += BLOCK) {
-        const int32_t sc = key_score(keys[i]);
-        lo = sc < lo ? sc : lo;
-        hi = sc > hi ? sc : hi;
+    // shared layout: [tmp P keys, rounded up to even][tie tie_cap keys][staged keys
+    // stage_cap (>= next_pow2(P)), reused as the output]
+    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* tie = tmp + ((P + 1) & ~1);
+    uint64_t* stage = tie + tie_cap;
+    uint64_t* const row = a.probe_keys + int64_t(b) * probe_keys_ld(nlist);  // 16-byte aligned
+    const uint64_t* keys = row;
+    if (nlist <= stage_cap) {
+        // every key of the row in flight at once
+        const ulonglong2* src2 = reinterpret_cast<const ulonglong2*>(keys);
+        ulonglong2* dst2 = reinterpret_cast<ulonglong2*>(stage);
+        for (int i = threadIdx.x; i < (nlist >> 1); i += BLOCK) cp_async16(dst2 + i, src2 + i);
+        if ((nlist & 1) && threadIdx.x == 0) stage[nlist - 1] = keys[nlist - 1];
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncthreads();
+        keys = stage;  // the output below overwrites it only after the last read
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-    }
-    if (lane == 0) {
-        ss.part[warp] = uint32_t(lo);
-        ss.hist2[warp] = uint32_t(hi);
-    }
-    for (int i = tid; i < kSelBins; i += BLOCK) ss.hist[i] = 0;
-    __syncthreads();
-    if (warp == 0) {
-        lo = lane < NW ? int32_t(ss.part[lane]) : INT32_MAX;
-        hi = lane < NW ? int32_t(ss.hist2[lane]) : INT32_MIN;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-        }
-        if (lane == 0) {
-            s_lo = lo;
-            s_hi = hi;
-        }
-    }
-    __syncthreads();
-    lo = s_lo;
-    hi = s_hi;
-    int sh = 0;
-    while (((int64_t(hi) - lo) >> sh) >= kSelBins) ++sh;
-
-    // histogram of (score - lo) >> sh
-    for (int i = tid; i < nlist; i += BLOCK)
-        atomicAdd(&ss.hist[uint32_t((int64_t(key_score(keys[i])) - lo) >> sh)], 1u);
-    __syncthreads();
-
-    // the bin holding the P-th best score: thread t owns bins counted down from the top
-    if (tid == 0) s_cut = 0;
-    constexpr int PER = kSelBins / BLOCK;
-    uint32_t local = 0;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) local += ss.hist[kSelBins - 1 - (tid * PER + j)];
-    uint32_t total;
-    const uint32_t excl = block_excl_scan<BLOCK>(local, ss.part, total);
-    if (excl < uint32_t(P) && uint32_t(P) <= excl + local) {
-        uint32_t acc = excl;
-        for (int j = 0; j < PER; ++j) {
-            const int bin = kSelBins - 1 - (tid * PER + j);
-            acc += ss.hist[bin];
-            if (acc >= uint32_t(P)) {
-                s_cut = bin;
-                break;
-            }
-        }
-    }
-    __syncthreads();
-    // every key scoring at least the cut bin's lowest score
-    const int32_t cut_score = int32_t(int64_t(lo) + (int64_t(s_cut) << sh));
-    const uint64_t thr = pack_key(cut_score, 0xFFFFFFFFu);
-    const int m = block_collect_ge<BLOCK>(keys, nlist, thr, cbuf, cap, ss);
-    if (m <= cap)
-        finish_query<BLOCK, true>(a, b, cbuf, m, sortbuf, pw, ss);
-    else  // a crowded cut bin (many equal scores): select among all keys
-        finish_query<BLOCK, true>(a, b, keys, nlist, sortbuf, pw, ss);
+    uint64_t* out = nlist <= stage_cap ? stage : row;
+    const int m = block_topk_sorted<BLOCK>(keys, nlist, P, out, tmp, tie, tie_cap, false, 0, 0, ss, a.err);
+    if (threadIdx.x == 0 && m != P) set_error(a.err, kErrSelectCount);
+    file_query<BLOCK, true>(a, b, out);
 }
 
 constexpr int kProbeSelBlock = 1024;
 
-size_t probe_select_smem(int P, int* cap_out)
+constexpr int kProbeTieCap = 1024;
+
+// Shared memory of probe_select_kernel; *stage_cap = keys that can be staged.
+size_t probe_select_smem(int P, int nlist, int* stage_cap)
 {
-    const int pw = next_pow2(P);
-    const size_t sort_keys = size_t(pw > kProbeSelBlock ? pw : kProbeSelBlock);
-    int cap = 4 * pw > 4096 ? 4 * pw : 4096;
-    if ((sort_keys + cap) * 8 > 190 * 1024) cap = int(190 * 1024 / 8 - sort_keys);
-    if (cap_out) *cap_out = cap;
-    return (sort_keys + size_t(cap)) * 8;
+    const size_t budget = 200 * 1024;
+    const size_t fixed = (size_t((P + 1) & ~1) + kProbeTieCap) * 8;
+    const int want = nlist > next_pow2(P) ? nlist : next_pow2(P);
+    size_t cap = (budget - fixed) / 8;
+    if (cap > size_t(want)) cap = size_t(want);
+    *stage_cap = int(cap);
+    return fixed + cap * 8;
 }
 
 cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s)
@@ -307,11 +267,11 @@ cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s)
     probe_score_kernel<<<grid, kScoreBlock, qbytes, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    int cap = 0;
-    const size_t smem = probe_select_smem(a.P, &cap);
+    int stage_cap = 0;
+    const size_t smem = probe_select_smem(a.P, a.nlist, &stage_cap);
     e = ensure_smem_attr(reinterpret_cast<const void*>(probe_select_kernel<kProbeSelBlock>), 11, 200 * 1024);
     if (e != cudaSuccess) return e;
-    probe_select_kernel<kProbeSelBlock><<<a.B, kProbeSelBlock, smem, s>>>(a, cap);
+    probe_select_kernel<kProbeSelBlock><<<a.B, kProbeSelBlock, smem, s>>>(a, stage_cap, kProbeTieCap);
     return cudaGetLastError();
 }
 

@@ -7,11 +7,20 @@
 // PyTorch module, fused Int8 ANN paragraph; maximum top-k row of the cost
 // efficiency table in the Spanish translation.
 //
-// The candidate keys of a query (written by the scan) are copied into shared
-// memory when they fit; a radix select over the bits where they differ finds a
-// threshold with exactly k keys at or above it; those keys are gathered and a
-// bitonic network sorts them.
-//
+// Three kernels, so that a query with a hundred thousand candidates is spread
+// over many SMs instead of holding one: the candidates of every query are cut
+// into chunks of kChunk keys, and
+//   * select_hist_kernel: each chunk's keys go into a 2048-bin histogram of
+//     their scores over the query's score range (recorded by the scan),
+//     added into the query's histogram;
+//   * select_scatter_kernel: from that histogram every chunk finds the same
+//     cut bin (the one holding the k-th best score) and the output segment of
+//     each bin above it, and writes its keys of those bins into their segments;
+//     the cut bin's keys are gathered aside;
+//   * select_kernel: one CTA per query takes the cut bin's best, orders every
+//     segment (each key's rank among its segment's keys) and writes ids and
+//     scores. A query whose candidates overflowed the scan's buffer takes the
+//     exact overflow path instead, all in this kernel.
 // Exact overflow path: when the scan reserved more candidates for a query than
 // its buffer holds, this CTA rescans that query's probed lists itself with the
 // bounded buffer: whenever the buffer fills it keeps only the k best keys and
@@ -21,78 +30,6 @@
 #include "st_internal.cuh"
 
 namespace st {
-
-template <int BLOCK>
-__device__ int32_t select_into(const uint64_t* keys, int64_t n, int k, uint64_t* sortbuf, int pwk,
-                               SelectSmem& ss, uint32_t* err, uint64_t* tmp)
-{
-    int32_t got;
-    if (n > k) {
-        const uint64_t thr = block_select_threshold<BLOCK>(keys, n, k, ss, err);
-        got = block_collect_ge<BLOCK>(keys, n, thr, sortbuf, pwk, ss);
-        if (threadIdx.x == 0 && got != k) set_error(err, kErrSelectCount);
-    } else {
-        got = block_collect_ge<BLOCK>(keys, n, 1ull, sortbuf, pwk, ss);
-    }
-    if (got > pwk) got = pwk;
-    for (int i = got + threadIdx.x; i < pwk; i += BLOCK) sortbuf[i] = 0;
-    __syncthreads();
-    block_sort_desc_counting<BLOCK>(sortbuf, got, tmp, ss);
-    return got;
-}
-
-// Histogram-guided threshold: the bin holding the k-th best score is found from
-// the per-query histogram the scan built; every key of that bin or above is
-// collected (about k plus one bin), and the exact threshold is selected among
-// them only. Returns false (and leaves nothing) when the histogram does not
-// match the keys or the collected set does not fit, so the caller falls back.
-template <int BLOCK>
-__device__ bool hist_guided_select(const SearchArgs& a, int q, const uint64_t* keys, int64_t n, int k,
-                                   uint64_t* sortbuf, int pwk, uint64_t* buf, int buf_cap, SelectSmem& ss)
-{
-    __shared__ uint32_t s_cut_bin, s_cut_above;
-    const uint32_t* h = a.hist + int64_t(q) * kHistBins;
-    constexpr int PER = kHistBins / BLOCK > 0 ? kHistBins / BLOCK : 1;
-    uint32_t c[PER];
-    uint32_t local = 0;
-    // thread t owns bins counted down from the top: kHistBins-1-(t*PER+j)
-    for (int j = 0; j < PER; ++j) {
-        const int bin = kHistBins - 1 - (int(threadIdx.x) * PER + j);
-        c[j] = bin >= 0 ? h[bin] : 0u;
-        local += c[j];
-    }
-    if (threadIdx.x == 0) {
-        s_cut_bin = 0;
-        s_cut_above = 0xFFFFFFFFu;
-    }
-    uint32_t total;
-    const uint32_t excl = block_excl_scan<BLOCK>(local, ss.part, total);
-    if (excl < uint32_t(k) && uint32_t(k) <= excl + local) {
-        uint32_t acc = excl;
-        for (int j = 0; j < PER; ++j) {
-            if (acc + c[j] >= uint32_t(k)) {
-                s_cut_bin = uint32_t(kHistBins - 1 - (int(threadIdx.x) * PER + j));
-                s_cut_above = acc;
-                break;
-            }
-            acc += c[j];
-        }
-    }
-    __syncthreads();
-    if (int64_t(total) != n || s_cut_above == 0xFFFFFFFFu) return false;
-    // lowest score of the cut bin -> key threshold (every key of a score >= it)
-    const int32_t s_lo = s_cut_bin == 0 ? INT32_MIN + 1 : int32_t((int64_t(s_cut_bin) << a.hshift) - a.smax);
-    const uint64_t thr = pack_key(s_lo, 0xFFFFFFFFu);
-    const int32_t got = block_collect_ge_wide<BLOCK>(keys, n, thr, buf, buf_cap, ss);
-    if (got > buf_cap || got < k) return false;
-    const uint64_t t2 = block_select_threshold<BLOCK>(buf, got, k, ss, a.err);
-    const int32_t fin = block_collect_ge<BLOCK>(buf, got, t2, sortbuf, pwk, ss);
-    if (threadIdx.x == 0 && fin != k) set_error(a.err, kErrSelectCount);
-    for (int i = (fin < pwk ? fin : pwk) + threadIdx.x; i < pwk; i += BLOCK) sortbuf[i] = 0;
-    __syncthreads();
-    block_sort_desc_counting<BLOCK>(sortbuf, fin < pwk ? fin : pwk, buf, ss);  // buf's keys are no longer needed
-    return true;
-}
 
 template <int BLOCK>
 __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, int pwk, int4* s_qv,
@@ -162,60 +99,237 @@ __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, 
     return s_count;
 }
 
+constexpr int kChunk = 4096;      // candidates per histogram / scatter item
+constexpr int kChunkBlock = 512;
+constexpr int kSelectTieCapSmem = 1024;
+
+// The query's score range (a superset of its candidates' scores)
+__device__ __forceinline__ void query_range(const SearchArgs& a, int q, int32_t& lo, uint32_t& sh)
+{
+    const uint32_t* qr = a.score_rng + int64_t(q) * kCntStride;
+    const int32_t hi = int32_t(qr[0] ^ 0x80000000u);
+    lo = int32_t(~qr[1] ^ 0x80000000u);
+    sh = topk_shift(lo, hi);
+}
+
+// Candidates the chunked kernels handle for query q: all of them, unless the
+// scan overflowed the query's buffer (the final kernel rescans those).
+__device__ __forceinline__ int64_t chunked_count(const SearchArgs& a, int q)
+{
+    const int64_t n = a.cand_cnt[int64_t(q) * kCntStride];
+    return n <= a.cap ? n : 0;
+}
+
+// pre[q] = first item of query q (items: chunks of kChunk candidates), pre[B] = total
+template <int BLOCK>
+__device__ void chunk_prefix(const SearchArgs& a, int* pre, uint32_t* part)
+{
+    const int B = a.B;
+    const int per = (B + BLOCK - 1) / BLOCK;
+    const int q0 = threadIdx.x * per;
+    uint32_t local = 0;
+    for (int j = 0; j < per; ++j)
+        if (q0 + j < B) local += uint32_t((chunked_count(a, q0 + j) + kChunk - 1) / kChunk);
+    uint32_t total;
+    uint32_t run = block_excl_scan<BLOCK>(local, part, total);
+    for (int j = 0; j < per; ++j)
+        if (q0 + j < B) {
+            pre[q0 + j] = int(run);
+            run += uint32_t((chunked_count(a, q0 + j) + kChunk - 1) / kChunk);
+        }
+    if (threadIdx.x == 0) pre[B] = int(total);
+    __syncthreads();
+}
+
+__device__ __forceinline__ int item_query(const int* pre, int B, int item)
+{
+    int lo = 0, hi = B - 1;  // the last q with pre[q] <= item
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= item) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kChunkBlock)
+select_hist_kernel(SearchArgs a)
+{
+    extern __shared__ int pre[];  // [B + 1]
+    __shared__ uint32_t h[kSelBins];
+    __shared__ uint32_t part[32];
+    chunk_prefix<kChunkBlock>(a, pre, part);
+    const int total = pre[a.B];
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const int q = item_query(pre, a.B, item);
+        const int64_t c0 = int64_t(item - pre[q]) * kChunk;
+        const int64_t n = chunked_count(a, q);
+        const int cnt = int(n - c0 < kChunk ? n - c0 : kChunk);
+        int32_t lo;
+        uint32_t sh;
+        query_range(a, q, lo, sh);
+        for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock) h[i] = 0;
+        __syncthreads();
+        const uint64_t* keys = a.cand + int64_t(q) * a.cap + c0;
+        constexpr int U = kChunk / kChunkBlock;
+        uint64_t v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = u * kChunkBlock + threadIdx.x;
+            v[u] = i < cnt ? keys[i] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (u * kChunkBlock + int(threadIdx.x) < cnt) atomicAdd(&h[topk_bin(v[u], lo, sh)], 1u);
+        __syncthreads();
+        uint32_t* gh = a.sel_hist + int64_t(q) * kSelBins;
+        for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock)
+            if (h[i]) atomicAdd(&gh[i], h[i]);
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kChunkBlock)
+select_scatter_kernel(SearchArgs a)
+{
+    extern __shared__ int pre[];  // [B + 1]
+    __shared__ SelectSmem ss;
+    chunk_prefix<kChunkBlock>(a, pre, ss.part);
+    const int total = pre[a.B];
+    const int k = a.k;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const int q = item_query(pre, a.B, item);
+        const int64_t c0 = int64_t(item - pre[q]) * kChunk;
+        const int64_t n = chunked_count(a, q);
+        const int cnt = int(n - c0 < kChunk ? n - c0 : kChunk);
+        int32_t lo;
+        uint32_t sh;
+        query_range(a, q, lo, sh);
+        const uint32_t* gh = a.sel_hist + int64_t(q) * kSelBins;
+        for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock) ss.hist[i] = gh[i];
+        __syncthreads();
+        const TopkCut t = topk_cut_from_hist<kChunkBlock>(n, k, lo, sh, ss);
+        const uint64_t* keys = a.cand + int64_t(q) * a.cap + c0;
+        uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
+        uint64_t* out = a.sel_out + int64_t(q) * k;
+        uint64_t* tie = a.sel_tie + int64_t(q) * kSelTieCap;
+        uint32_t* tcnt = a.score_rng + int64_t(q) * kCntStride + 2;
+        constexpr int U = kChunk / kChunkBlock;
+        uint64_t v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = u * kChunkBlock + threadIdx.x;
+            v[u] = i < cnt ? keys[i] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (u * kChunkBlock + int(threadIdx.x) >= cnt) continue;
+            const int b = topk_bin(v[u], lo, sh);
+            if (b > t.cut) {
+                out[ss.hist2[b] + atomicAdd(&cur[b], 1u)] = v[u];
+            } else if (b == t.cut) {
+                const uint32_t tp = atomicAdd(tcnt, 1u);
+                if (tp < uint32_t(kSelTieCap)) tie[tp] = v[u];
+            }
+        }
+        __syncthreads();
+    }
+}
+
 template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK)
-select_kernel(SearchArgs a)
+select_kernel(SearchArgs a, int stage_cap)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ SelectSmem ss;
     const int q = blockIdx.x;
     const int k = a.k;
     const int pwk = next_pow2(k);
-    uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem_raw);    // max(pwk, BLOCK) keys
-    uint64_t* local = sortbuf + (pwk > BLOCK ? pwk : BLOCK);       // 16-byte aligned
+    // shared layout: [tmp k keys, rounded up to even][tie kSelectTieCapSmem keys]
+    // [stage_cap keys (>= next_pow2(k)): staged candidates / the output]
+    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* tie = tmp + ((k + 1) & ~1);
+    uint64_t* stage = tie + kSelectTieCapSmem;
 
     const uint32_t cnt = a.cand_cnt[int64_t(q) * kCntStride];
-    const uint64_t* keys = a.cand + int64_t(q) * a.cap;
     int64_t n = cnt;
-    const bool overflow = n > a.cap;
-    if (overflow) n = overflow_path<BLOCK>(a, q, sortbuf, pwk, reinterpret_cast<int4*>(local), ss);
-    bool done = false;
-    if (!overflow && n > k) {
-        // common case: the scan's histogram gives the cut; one pass over the
-        // candidates in global memory collects about k keys into shared memory
-        done = hist_guided_select<BLOCK>(a, q, keys, n, k, sortbuf, pwk, local, kSelectSmemKeys, ss);
-    }
-    if (!done && n <= kSelectSmemKeys) {
-        // all of this thread's 16-byte copies in flight at once (cp.async)
-        const int64_t n2 = (n + 1) >> 1;
-        const ulonglong2* src2 = reinterpret_cast<const ulonglong2*>(keys);
-        ulonglong2* dst2 = reinterpret_cast<ulonglong2*>(local);
-        for (int64_t i = threadIdx.x; i < n2; i += BLOCK) cp_async16(dst2 + i, src2 + i);
-        cp_async_commit();
-        cp_async_wait_all();
+    int m = 0;
+    uint64_t* out = stage;
+    if (n > a.cap) {
+        // the scan overflowed this query's buffer: rescan exactly, then select
+        // from the kept keys here
+        n = overflow_path<BLOCK>(a, q, stage, pwk, reinterpret_cast<int4*>(tie), ss);
+        const uint64_t* keys = a.cand + int64_t(q) * a.cap;
+        if (n <= stage_cap) {
+            for (int64_t i = threadIdx.x; i < n; i += BLOCK) stage[i] = keys[i];
+            __syncthreads();
+            keys = stage;
+        } else {
+            out = a.cand + int64_t(q) * a.cap;  // cap >= n > stage_cap >= next_pow2(k)
+        }
+        m = block_topk_sorted<BLOCK>(keys, n, k, out, tmp, tie, kSelectTieCapSmem, false, 0, 0, ss, a.err);
+    } else if (n > 0) {
+        // the chunked kernels grouped the keys above the cut bin by bin
+        int32_t lo;
+        uint32_t sh;
+        query_range(a, q, lo, sh);
+        const uint32_t* gh = a.sel_hist + int64_t(q) * kSelBins;
+        for (int i = threadIdx.x; i < kSelBins; i += BLOCK) ss.hist[i] = gh[i];
         __syncthreads();
-        if ((n & 1) && threadIdx.x == 0) local[n] = 0;  // the pair's second key was past the end
+        const TopkCut t = topk_cut_from_hist<BLOCK>(n, k, lo, sh, ss);
+        const uint64_t* gout = a.sel_out + int64_t(q) * k;
+        for (int i = threadIdx.x; i < t.above; i += BLOCK) tmp[i] = gout[i];
+        const uint64_t* gtie = a.sel_tie + int64_t(q) * kSelTieCap;
+        const uint64_t* tsrc = nullptr;  // the cut bin's keys, if they were all kept
+        if (t.tcount <= kSelectTieCapSmem) {
+            for (int i = threadIdx.x; i < t.tcount; i += BLOCK) tie[i] = gtie[i];
+            tsrc = tie;
+        } else if (t.tcount <= kSelTieCap) {
+            tsrc = gtie;
+        }
         __syncthreads();
-        keys = local;
+        topk_take_ties<BLOCK>(t, tsrc, a.cand + int64_t(q) * a.cap, n, tmp, ss, a.err);
+        topk_rank<BLOCK>(t, tmp, out, ss);
+        m = t.m;
     }
-    // the candidate area is free once the final keys are in sortbuf
-    if (!done) select_into<BLOCK>(keys, n, k, sortbuf, pwk, ss, a.err, local);
     for (int r = threadIdx.x; r < k; r += BLOCK) {
-        const uint64_t key = sortbuf[r];
+        const uint64_t key = r < m ? out[r] : 0ull;  // key 0 reads as (id -1, INT32_MIN)
         a.out_ids[int64_t(q) * k + r] = key_id(key);
         a.out_scores[int64_t(q) * k + r] = key_score(key);
     }
     if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
 }
 
-cudaError_t launch_select(const SearchArgs& a, cudaStream_t s)
+size_t select_smem(int k, int* stage_cap)
 {
-    const int pwk = next_pow2(a.k);
-    const size_t smem = size_t(pwk > kSelectBlock ? pwk : kSelectBlock) * 8 + size_t(kSelectSmemKeys) * 8;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8,
-                                     int(size_t(ST_MAX_K) * 8 + size_t(kSelectSmemKeys) * 8));
+    const size_t budget = 208 * 1024;
+    const size_t fixed = (size_t((k + 1) & ~1) + kSelectTieCapSmem) * 8;
+    *stage_cap = int((budget - fixed) / 8) & ~1;
+    return budget;
+}
+
+cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
+{
+    // the attribute is set once per device: give it the largest size any batch uses
+    constexpr int kPreSmemMax = 160 * 1024;
+    const size_t pre_bytes = size_t(a.B + 1) * 4;
+    if (pre_bytes > size_t(kPreSmemMax)) return cudaErrorInvalidValue;
+    const int grid = 2 * num_sms;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_hist_kernel), 12, kPreSmemMax);
     if (e != cudaSuccess) return e;
-    select_kernel<kSelectBlock><<<a.B, kSelectBlock, smem, s>>>(a);
+    select_hist_kernel<<<grid, kChunkBlock, pre_bytes, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = ensure_smem_attr(reinterpret_cast<const void*>(select_scatter_kernel), 13, kPreSmemMax);
+    if (e != cudaSuccess) return e;
+    select_scatter_kernel<<<grid, kChunkBlock, pre_bytes, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    int stage_cap = 0;
+    const size_t smem = select_smem(a.k, &stage_cap);
+    e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8, int(smem));
+    if (e != cudaSuccess) return e;
+    select_kernel<kSelectBlock><<<a.B, kSelectBlock, smem, s>>>(a, stage_cap);
     return cudaGetLastError();
 }
 

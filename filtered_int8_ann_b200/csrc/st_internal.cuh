@@ -20,13 +20,17 @@ constexpr int kProbeSmemKeys = 16384;      // nlist up to this keeps probe keys 
 constexpr int kSelectBlock = 1024;
 constexpr int kSelectSmemKeys = 22528;     // candidates up to this are selected in smem
 constexpr int kPlanBlock = 512;
-constexpr int kHistBins = 2048;            // per-query score histogram bins
 // Per-query counters sit one 128-byte line apart, so the reservation atomics
 // of different queries spread over the L2 slices instead of queueing on one.
 constexpr int kCntStride = 32;             // uint32 words (16 uint64) per query
+
+// Row stride (keys) of the search probe's [B][nlist] centroid keys: even, so
+// every row starts on a 16-byte boundary for vector copies.
+__host__ __device__ __forceinline__ int64_t probe_keys_ld(int nlist) { return (int64_t(nlist) + 1) & ~int64_t(1); }
 constexpr int kMaskBitsMax = 128;          // signature bits
 constexpr int kSelBits = 11;               // radix digit of the selections
 constexpr int kSelBins = 1 << kSelBits;
+constexpr int kSelTieCap = 4096;           // cut-bin keys the final top-k keeps per query
 constexpr uint32_t kWaitLimit = 1u << 10;  // bounded mbarrier polls before giving up
 constexpr uint32_t kWaitHintNs = 10000000u; // each poll may sleep up to 10 ms waiting for the phase
 
@@ -91,8 +95,14 @@ struct SearchArgs {
     int32_t* list_cnt;       // [nlist] queries filed into each list      (zeroed)
     int32_t* probe_done;     // [B] probe slices finished per query       (zeroed)
     uint32_t* cand_cnt;      // [B][kCntStride] candidates reserved per query, word 0 used (zeroed)
+    uint32_t* score_rng;     // [B][kCntStride] per query: [0] max of the biased scores (score ^ 2^31)
+                             // of its candidates, [1] max of their complements, [2] cut-bin keys
+                             // gathered by the final top-k (zeroed)
+    uint32_t* sel_hist;      // [B][kSelBins] final top-k: candidate score histogram (zeroed)
+    uint32_t* sel_cursor;    // [B][kSelBins] final top-k: keys placed per bin (zeroed)
+    uint64_t* sel_out;       // [B][k] final top-k: keys above the cut, grouped by bin
+    uint64_t* sel_tie;       // [B][kSelTieCap] final top-k: keys of the cut bin
     unsigned long long* eligible_cnt;  // [B][kCntStride / 2], word 0 used        (zeroed)
-    uint32_t* hist;          // [B][kHistBins] emitted-key score histogram (zeroed)
     PlanCtl* ctl;            // unit allocation counter                   (zeroed)
     int32_t* probe;          // [B][P]
     uint64_t* probe_keys;    // [B][nlist] when a probe slice does not fit shared memory, else null
@@ -106,8 +116,6 @@ struct SearchArgs {
     int32_t max_units;
     uint64_t* cand;          // [B][cap]
     int64_t cap;             // candidate keys per query
-    int32_t smax;            // largest possible |score|: d * 128 * 128
-    int32_t hshift;          // histogram bin = min(kHistBins-1, (score + smax) >> hshift)
     uint32_t* err;           // device error word
 };
 
@@ -124,13 +132,6 @@ __device__ __forceinline__ int32_t dot16(const int4 a, const int4 b, int32_t acc
 }
 
 __device__ __forceinline__ void set_error(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
-
-// Histogram bin of a score: monotone non-decreasing in the score.
-__device__ __forceinline__ uint32_t score_bin(int32_t score, int32_t smax, int32_t hshift)
-{
-    const uint32_t b = uint32_t(score + smax) >> hshift;
-    return b < uint32_t(kHistBins) ? b : uint32_t(kHistBins - 1);
-}
 
 __device__ __forceinline__ unsigned lanemask_lt()
 {
@@ -560,6 +561,256 @@ __device__ void block_sort_desc_counting(uint64_t* a, int m, uint64_t* tmp, Sele
     __syncthreads();
 }
 
+// ----------------------------------------------------------------------------
+// Histogram top-k. The keys' scores are binned over kSelBins bins spanning a
+// range [lo, hi] that contains them all: bin = (score - lo) >> sh, sh the
+// smallest shift that fits the range. Suffix sums of the bin counts give the
+// bin holding the k-th key (the cut bin) and the output segment of every bin
+// above it, so the keys of those bins can be scattered straight to their
+// segments; only the cut bin's keys need an exact selection, and each key's
+// place inside its segment is the number of the segment's keys greater than
+// it (segments longer than 64 keys, i.e. many equal scores, use the bitonic
+// network instead).
+// ----------------------------------------------------------------------------
+struct TopkCut {
+    int32_t lo;     // range base
+    uint32_t sh;    // bin shift
+    int cut;        // cut bin (-1: n <= k, every key is taken)
+    int above;      // keys in the bins above the cut
+    int tcount;     // keys in the cut bin
+    int m;          // min(n, k)
+    int maxseg;     // longest output segment
+};
+
+__host__ __device__ __forceinline__ uint32_t topk_shift(int32_t lo, int32_t hi)
+{
+    uint32_t sh = 0;
+    while (((int64_t(hi) - lo) >> sh) >= kSelBins) ++sh;
+    return sh;
+}
+
+__device__ __forceinline__ int topk_bin(uint64_t key, int32_t lo, uint32_t sh)
+{
+    return int((int64_t(key_score(key)) - lo) >> sh);
+}
+
+// From the bin counts in s.hist: s.hist2[b] = start of bin b's segment (a
+// segment ends where the next lower bin's starts), s.hist[b] = the same start
+// (a write cursor for the scatter), and the cut. All threads get the result.
+template <int BLOCK>
+__device__ TopkCut topk_cut_from_hist(int64_t n, int k, int32_t lo, uint32_t sh, SelectSmem& s)
+{
+    __shared__ int32_t c_cut, c_above, c_tcount, c_maxseg;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        c_cut = -1;
+        c_above = int32_t(n < k ? n : k);
+        c_tcount = 0;
+        c_maxseg = 0;
+    }
+    constexpr int PER = kSelBins / BLOCK > 0 ? kSelBins / BLOCK : 1;
+    const int owners = kSelBins / PER;
+    uint32_t local = 0;
+    if (tid < owners)
+        for (int j = 0; j < PER; ++j) local += s.hist[kSelBins - 1 - (tid * PER + j)];
+    uint32_t total;
+    uint32_t run = block_excl_scan<BLOCK>(local, s.part, total);
+    int mseg = 0;
+    if (tid < owners)
+        for (int j = 0; j < PER; ++j) {
+            const int bin = kSelBins - 1 - (tid * PER + j);
+            const uint32_t c = s.hist[bin];
+            s.hist2[bin] = run;
+            s.hist[bin] = run;
+            if (n > k && run < uint32_t(k) && uint32_t(k) <= run + c) {
+                c_cut = bin;
+                c_above = int32_t(run);
+                c_tcount = int32_t(c);
+            }
+            if (run + c <= uint32_t(k) && int(c) > mseg) mseg = int(c);
+            run += c;
+        }
+    if (mseg > 0) atomicMax(&c_maxseg, mseg);
+    __syncthreads();
+    TopkCut t;
+    t.lo = lo;
+    t.sh = sh;
+    t.cut = c_cut;
+    t.above = c_above;
+    t.tcount = c_tcount;
+    t.m = n < k ? int(n) : k;
+    t.maxseg = c_maxseg;
+    __syncthreads();  // the shared fields may be rewritten by a later call
+    return t;
+}
+
+// Choose the cut bin's best (m - above) keys into tmp[above, m). `tie` holds
+// the cut bin's tcount keys (shared or global; nullptr when they were not
+// kept); without them the threshold is selected over all n `keys`.
+template <int BLOCK>
+__device__ void topk_take_ties(const TopkCut& t, const uint64_t* tie, const uint64_t* keys, int64_t n, uint64_t* tmp,
+                               SelectSmem& s, uint32_t* err)
+{
+    __shared__ int32_t r_pos;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int need = t.m - t.above;
+    if (need <= 0) return;
+    if (tie != nullptr && t.tcount <= 64) {
+        // one warp: a tie key's rank among the tie keys is its place
+        if (warp == 0) {
+            const uint64_t k1 = lane < t.tcount ? tie[lane] : 0ull;
+            const uint64_t k2 = lane + 32 < t.tcount ? tie[lane + 32] : 0ull;
+            int r1 = 0, r2 = 0;
+            for (int j = 0; j < 32; ++j) {
+                const uint64_t o1 = __shfl_sync(0xffffffffu, k1, j), o2 = __shfl_sync(0xffffffffu, k2, j);
+                r1 += int(o1 > k1) + int(o2 > k1);
+                r2 += int(o1 > k2) + int(o2 > k2);
+            }
+            if (k1 != 0ull && r1 < need) tmp[t.above + r1] = k1;
+            if (k2 != 0ull && r2 < need) tmp[t.above + r2] = k2;
+        }
+        __syncthreads();
+        return;
+    }
+    const uint64_t* src = tie != nullptr ? tie : keys;
+    const int64_t ns = tie != nullptr ? int64_t(t.tcount) : n;
+    const int64_t want = tie != nullptr ? int64_t(need) : int64_t(t.m);
+    uint64_t thr = 1;
+    if (want < ns) thr = block_select_threshold<BLOCK>(src, ns, want, s, err);
+    if (tid == 0) r_pos = 0;
+    __syncthreads();
+    for (int64_t i = tid; i < ns; i += BLOCK) {
+        const uint64_t key = src[i];
+        if (key >= thr && key != 0ull && topk_bin(key, t.lo, t.sh) == t.cut) {
+            const int pos = atomicAdd(&r_pos, 1);
+            if (pos < need) tmp[t.above + pos] = key;
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && r_pos != need) set_error(err, kErrSelectCount);
+    __syncthreads();
+}
+
+// Order tmp[0, m) (bins above the cut in their segments, then the cut bin's
+// keys) into out[0, m), descending. s.hist2 holds the segment starts.
+template <int BLOCK>
+__device__ void topk_rank(const TopkCut& t, const uint64_t* tmp, uint64_t* out, SelectSmem& s)
+{
+    const int tid = threadIdx.x;
+    const int m = t.m, above = t.above;
+    if (t.maxseg > 64 || m - above > 64) {
+        for (int i = tid; i < m; i += BLOCK) out[i] = tmp[i];
+        __syncthreads();
+        block_bitonic_desc<BLOCK>(out, m);
+        return;
+    }
+    for (int p = tid; p < m; p += BLOCK) {
+        const uint64_t key = tmp[p];
+        int beg, end;
+        if (p >= above) {
+            beg = above;
+            end = m;
+        } else {
+            const int b = topk_bin(key, t.lo, t.sh);  // b > cut >= -1
+            beg = int(s.hist2[b]);
+            end = b > 0 ? int(s.hist2[b - 1]) : m;
+        }
+        int r = 0;
+        for (int j = beg; j < end; ++j) r += tmp[j] > key ? 1 : 0;
+        out[beg + r] = key;
+    }
+    __syncthreads();
+}
+
+// Top-k of n unique keys, sorted descending (score desc, then id asc), in one
+// CTA: range (unless `range_known`, when [lo, hi] must contain every score),
+// histogram, cut, one scatter pass, ties, ranks. Writes min(n, k) keys to
+// out[] and returns that count. `keys` may be shared or global memory (each
+// pass keeps eight loads per thread in flight). out[] needs next_pow2(k) keys,
+// tmp[] k keys, tie[] tie_cap keys.
+template <int BLOCK>
+__device__ int block_topk_sorted(const uint64_t* keys, int64_t n, int k, uint64_t* out, uint64_t* tmp,
+                                 uint64_t* tie, int tie_cap, bool range_known, int32_t lo, int32_t hi,
+                                 SelectSmem& s, uint32_t* err)
+{
+    constexpr int NW = BLOCK / 32;
+    constexpr int U = 8;  // loads in flight per thread and pass
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int32_t t_lo, t_tpos;
+    __shared__ uint32_t t_sh;
+    if (n <= 0) {
+        __syncthreads();
+        return 0;
+    }
+    auto for_keys = [&](auto&& fn) {
+        for (int64_t base = 0; base < n; base += int64_t(BLOCK) * U) {
+            uint64_t v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t i = base + int64_t(u) * BLOCK + tid;
+                v[u] = i < n ? keys[i] : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (base + int64_t(u) * BLOCK + tid < n) fn(v[u]);
+        }
+    };
+    if (!range_known) {
+        lo = INT32_MAX;
+        hi = INT32_MIN;
+        for_keys([&](uint64_t key) {
+            const int32_t sc = key_score(key);
+            lo = sc < lo ? sc : lo;
+            hi = sc > hi ? sc : hi;
+        });
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        if (lane == 0) {
+            s.red_lo[warp] = (unsigned long long)(uint32_t(lo));
+            s.red_hi[warp] = (unsigned long long)(uint32_t(hi));
+        }
+    }
+    for (int i = tid; i < kSelBins; i += BLOCK) s.hist[i] = 0;
+    __syncthreads();
+    if (tid == 0) {
+        int32_t l = lo, h = hi;
+        if (!range_known) {
+            l = INT32_MAX;
+            h = INT32_MIN;
+            for (int w = 0; w < NW; ++w) {
+                l = min(l, int32_t(uint32_t(s.red_lo[w])));
+                h = max(h, int32_t(uint32_t(s.red_hi[w])));
+            }
+        }
+        t_lo = l;
+        t_sh = topk_shift(l, h);
+        t_tpos = 0;
+    }
+    __syncthreads();
+    const int32_t base = t_lo;
+    const uint32_t sh = t_sh;
+    for_keys([&](uint64_t key) { atomicAdd(&s.hist[topk_bin(key, base, sh)], 1u); });
+    __syncthreads();
+    const TopkCut t = topk_cut_from_hist<BLOCK>(n, k, base, sh, s);
+    const bool tie_fits = t.tcount <= tie_cap;
+    // scatter the bins above the cut to their segments; gather the cut bin
+    for_keys([&](uint64_t key) {
+        const int b = topk_bin(key, base, sh);
+        if (b > t.cut) {
+            tmp[atomicAdd(&s.hist[b], 1u)] = key;
+        } else if (b == t.cut && tie_fits) {
+            tie[atomicAdd(&t_tpos, 1)] = key;
+        }
+    });
+    __syncthreads();
+    topk_take_ties<BLOCK>(t, tie_fits ? tie : nullptr, keys, n, tmp, s, err);
+    topk_rank<BLOCK>(t, tmp, out, s);
+    return t.m;
+}
+
 __host__ __device__ __forceinline__ int next_pow2(int v)
 {
     int p = 1;
@@ -580,7 +831,7 @@ size_t probe_noalloc_scratch_bytes(int B, int S, int P, int nlist, bool keys_in_
 cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
-cudaError_t launch_select(const SearchArgs& a, cudaStream_t s);
+cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s);
 size_t scan_smem_bytes(int d, int W);
 cudaError_t launch_build_planes(const uint64_t* sigs, const int64_t* offsets, const int32_t* chunk_start,
                                 const int32_t* chunk_list, int32_t n_chunks, int W, uint32_t* planes,
