@@ -119,25 +119,33 @@ def barrier(world):
         dist.barrier()
 
 
-def allreduce_max(x, world):
+def allreduce_max(x, world, device="cuda"):
+    """Max over ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def allreduce_sum(x, world):
+def allreduce_sum(x, world, device="cuda"):
+    """Sum over ranks (whole-job work)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
 
-def make_data(args, world, rank):
+def rank_query_rows(rank, B, pool):
+    """Rows of the generated query set that rank `rank` searches: its own
+    `pool` batches of B queries, disjoint from every other rank's."""
+    return rank * B * pool, (rank + 1) * B * pool
+
+
+def make_data(args, world, rank, device="cuda"):
     wl = WORKLOADS[args.workload]
     if args.n or args.nlist:
         n = args.n or wl.n
@@ -147,9 +155,10 @@ def make_data(args, world, rank):
     pool = max(1, args.pool)
     # every rank builds the same index; each draws its own query batches
     total_q = B * pool * world
-    data = generate(wl.with_(B=total_q), device="cuda")
-    q = data.queries[rank * B * pool:(rank + 1) * B * pool].reshape(pool, B, -1).contiguous()
-    m = data.masks[rank * B * pool:(rank + 1) * B * pool].reshape(pool, B, -1).contiguous()
+    data = generate(wl.with_(B=total_q), device=device)
+    r0, r1 = rank_query_rows(rank, B, pool)
+    q = data.queries[r0:r1].reshape(pool, B, -1).contiguous()
+    m = data.masks[r0:r1].reshape(pool, B, -1).contiguous()
     return wl.with_(B=B), data, q, m
 
 
