@@ -14,8 +14,8 @@
 // B200 design. The plan cut the probed lists into warp units: one list chunk
 // (kWarpItems rows) x up to kQMax queries probing that list, so each probed
 // list is streamed once per batch whatever the number of queries probing it.
-// Warps are independent (one-warp CTAs, many per SM) and take units
-// round-robin. A warp tests one unit ahead of the one it scores, so every
+// Warps work independently (four per CTA, sharing only a unit counter) and
+// take units in turn. A warp tests one unit ahead of the one it scores, so every
 // memory round trip of a unit overlaps the previous unit's work:
 //   * signature planes: the index stores each chunk's signatures as bit-planes
 //     (layout.cu). A unit needs only the planes of the bits in the union of its
@@ -108,7 +108,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p)
 // d (rows are then re-read from L1 for each eligible query).
 // (at most as many registers as keep the shared-memory-limited warp count resident)
 template <int NP, int W>
-__global__ void __launch_bounds__(kScanBlock, NP == 8 ? 16 : 20)
+__global__ void __launch_bounds__(kScanBlock, NP == 8 ? 4 : 5)
 scan_kernel(SearchArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -129,9 +129,21 @@ scan_kernel(SearchArgs a)
     uint8_t* const s_tab = reinterpret_cast<uint8_t*>(s_rng + 2 * kQMax);                 // [128]
     uint8_t* const s_inv = s_tab + kMaskBitsMax;                                         // [kPlaneSlots]
 
+    // units: CTA c owns units c, c + ncta, c + 2 ncta, ... (an even mix of the
+    // table); its warps take them in turn from a shared counter, three units
+    // ahead, so a warp that drew cheap units takes more of them
+    __shared__ int s_next;
+    if (threadIdx.x == 0) s_next = 0;
+    __syncthreads();
     const int n_units = a.ctl->n_units < a.max_units ? a.ctl->n_units : a.max_units;
-    const int stride = gridDim.x * (kScanBlock / 32);
-    int u = blockIdx.x * (kScanBlock / 32) + warp;
+    auto draw = [&]() -> int {
+        int j = 0;
+        if (lane == 0) j = atomicAdd(&s_next, 1);
+        j = __shfl_sync(0xffffffffu, j, 0);
+        const int64_t v = int64_t(blockIdx.x) + int64_t(j) * gridDim.x;
+        return v < n_units ? int(v) : n_units;
+    };
+    int u = draw();
     if (u >= n_units) return;
 
     // unit entry: {first row, chunk, first query slot, rows << 16 | queries};
@@ -277,8 +289,9 @@ scan_kernel(SearchArgs a)
     // prologue: test unit 0; groups planes(0) [waited], planes(1), queries(0)
     int4 e_cur = a.units[u];
     int4 e_nxt = make_int4(0, 0, 0, 0), e_n2 = make_int4(0, 0, 0, 0);
-    if (u + stride < n_units) e_nxt = a.units[u + stride];
-    if (u + 2 * stride < n_units) e_n2 = a.units[u + 2 * stride];
+    int u_n1 = draw(), u_n2 = draw();
+    if (u_n1 < n_units) e_nxt = a.units[u_n1];
+    if (u_n2 < n_units) e_n2 = a.units[u_n2];
     int qid_c, qid_n = 0;
     uint64_t m0_n = 0, m1_n = 0;
     int held;          // planes the buffer holds for the next unit to test (-1: global)
@@ -288,7 +301,7 @@ scan_kernel(SearchArgs a)
     {
         uint64_t m0_c, m1_c;
         load_slots(e_cur, qid_c, m0_c, m1_c);
-        if (u + stride < n_units) load_slots(e_nxt, qid_n, m0_n, m1_n);
+        if (u_n1 < n_units) load_slots(e_nxt, qid_n, m0_n, m1_n);
         const int held0 = request_planes(e_cur, qid_c, m0_c, m1_c);
         cp_async_commit();
         cp_async_wait_group<0>();
@@ -297,7 +310,7 @@ scan_kernel(SearchArgs a)
         test_unit(e_cur, qid_c, held0, pass2, any, mycnt);
         single_c = (e_cur.w & 0xFFFF) == 1 && held0 >= 0;
         __syncwarp();
-        held = u + stride < n_units ? request_planes(e_nxt, qid_n, m0_n, m1_n) : -1;
+        held = u_n1 < n_units ? request_planes(e_nxt, qid_n, m0_n, m1_n) : -1;
         cp_async_commit();
         nsurv_c = settle_unit(e_cur, qid_c, single_c, any, mycnt, surv2, base_c);
     }
@@ -305,15 +318,16 @@ scan_kernel(SearchArgs a)
     cp_async_commit();
     int cb = 0;
 
-    for (; u < n_units; u += stride) {
-        const bool has_n1 = u + stride < n_units;
-        const bool has_n2 = u + 2 * stride < n_units;
-        const bool has_n3 = u + 3 * stride < n_units;
+    while (u < n_units) {
+        const int u_n3 = draw();
+        const bool has_n1 = u_n1 < n_units;
+        const bool has_n2 = u_n2 < n_units;
+        const bool has_n3 = u_n3 < n_units;
 
         // background loads: the entry three units ahead, the slots of the unit
         // two ahead (whose entry arrived during the previous unit)
         int4 e_n3 = make_int4(0, 0, 0, 0);
-        if (has_n3) e_n3 = a.units[u + 3 * stride];
+        if (has_n3) e_n3 = a.units[u_n3];
         int qid_2 = 0;
         uint64_t m0_2 = 0, m1_2 = 0;
         if (has_n2) load_slots(e_n2, qid_2, m0_2, m1_2);
@@ -462,6 +476,9 @@ scan_kernel(SearchArgs a)
         nsurv_c = nsurv_n;
         single_c = single_n;
         cb ^= 1;
+        u = u_n1;
+        u_n1 = u_n2;
+        u_n2 = u_n3;
     }
     cp_async_wait_all();  // no copy may land after the warp has left
 }

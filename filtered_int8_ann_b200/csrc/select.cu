@@ -152,14 +152,20 @@ __device__ __forceinline__ int item_query(const int* pre, int B, int item)
     return lo;
 }
 
+// Per-query words of score_rng used by the final top-k, after the scan's range:
+// [2] cut-bin keys gathered, [3] chunks histogrammed, [4] cut bin, [5] keys
+// above it, [6] keys in it, [7] longest output segment.
+constexpr int kRngTie = 2, kRngDone = 3, kRngCut = 4, kRngAbove = 5, kRngTcount = 6, kRngMaxseg = 7;
+
 __global__ void __launch_bounds__(kChunkBlock)
 select_hist_kernel(SearchArgs a)
 {
     extern __shared__ int pre[];  // [B + 1]
-    __shared__ uint32_t h[kSelBins];
-    __shared__ uint32_t part[32];
-    chunk_prefix<kChunkBlock>(a, pre, part);
+    __shared__ SelectSmem ss;
+    __shared__ int s_last;
+    chunk_prefix<kChunkBlock>(a, pre, ss.part);
     const int total = pre[a.B];
+    uint32_t* h = ss.hist2;  // this chunk's histogram
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
         const int q = item_query(pre, a.B, item);
         const int64_t c0 = int64_t(item - pre[q]) * kChunk;
@@ -185,6 +191,27 @@ select_hist_kernel(SearchArgs a)
         uint32_t* gh = a.sel_hist + int64_t(q) * kSelBins;
         for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock)
             if (h[i]) atomicAdd(&gh[i], h[i]);
+        // the query's last chunk to finish (one counter, no waiting) finds the
+        // cut and writes each bin's segment start as the scatter's cursor
+        __threadfence();
+        __syncthreads();
+        uint32_t* rng = a.score_rng + int64_t(q) * kCntStride;
+        if (threadIdx.x == 0) s_last = atomicAdd(&rng[kRngDone], 1u) == uint32_t((n + kChunk - 1) / kChunk - 1);
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock) ss.hist[i] = __ldcg(gh + i);
+            __syncthreads();
+            const TopkCut t = topk_cut_from_hist<kChunkBlock>(n, a.k, lo, sh, ss);
+            uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
+            for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock) cur[i] = ss.hist2[i];
+            if (threadIdx.x == 0) {
+                rng[kRngCut] = uint32_t(t.cut);
+                rng[kRngAbove] = uint32_t(t.above);
+                rng[kRngTcount] = uint32_t(t.tcount);
+                rng[kRngMaxseg] = uint32_t(t.maxseg);
+            }
+        }
         __syncthreads();
     }
 }
@@ -193,8 +220,8 @@ __global__ void __launch_bounds__(kChunkBlock)
 select_scatter_kernel(SearchArgs a)
 {
     extern __shared__ int pre[];  // [B + 1]
-    __shared__ SelectSmem ss;
-    chunk_prefix<kChunkBlock>(a, pre, ss.part);
+    __shared__ uint32_t part[32];
+    chunk_prefix<kChunkBlock>(a, pre, part);
     const int total = pre[a.B];
     const int k = a.k;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
@@ -205,10 +232,7 @@ select_scatter_kernel(SearchArgs a)
         int32_t lo;
         uint32_t sh;
         query_range(a, q, lo, sh);
-        const uint32_t* gh = a.sel_hist + int64_t(q) * kSelBins;
-        for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock) ss.hist[i] = gh[i];
-        __syncthreads();
-        const TopkCut t = topk_cut_from_hist<kChunkBlock>(n, k, lo, sh, ss);
+        const int cut = int(a.score_rng[int64_t(q) * kCntStride + kRngCut]);
         const uint64_t* keys = a.cand + int64_t(q) * a.cap + c0;
         uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
         uint64_t* out = a.sel_out + int64_t(q) * k;
@@ -225,9 +249,9 @@ select_scatter_kernel(SearchArgs a)
         for (int u = 0; u < U; ++u) {
             if (u * kChunkBlock + int(threadIdx.x) >= cnt) continue;
             const int b = topk_bin(v[u], lo, sh);
-            if (b > t.cut) {
-                out[ss.hist2[b] + atomicAdd(&cur[b], 1u)] = v[u];
-            } else if (b == t.cut) {
+            if (b > cut) {
+                out[atomicAdd(&cur[b], 1u)] = v[u];
+            } else if (b == cut) {
                 const uint32_t tp = atomicAdd(tcnt, 1u);
                 if (tp < uint32_t(kSelTieCap)) tie[tp] = v[u];
             }
@@ -273,10 +297,20 @@ select_kernel(SearchArgs a, int stage_cap)
         int32_t lo;
         uint32_t sh;
         query_range(a, q, lo, sh);
-        const uint32_t* gh = a.sel_hist + int64_t(q) * kSelBins;
-        for (int i = threadIdx.x; i < kSelBins; i += BLOCK) ss.hist[i] = gh[i];
-        __syncthreads();
-        const TopkCut t = topk_cut_from_hist<BLOCK>(n, k, lo, sh, ss);
+        // the histogram kernel's cut; after the scatter the cursor of bin b + 1
+        // (the next higher bin) stands at the end of its segment, which is
+        // where bin b's segment starts
+        const uint32_t* rng = a.score_rng + int64_t(q) * kCntStride;
+        TopkCut t;
+        t.lo = lo;
+        t.sh = sh;
+        t.cut = int(rng[kRngCut]);
+        t.above = int(rng[kRngAbove]);
+        t.tcount = int(rng[kRngTcount]);
+        t.maxseg = int(rng[kRngMaxseg]);
+        t.m = n < k ? int(n) : k;
+        const uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
+        for (int i = threadIdx.x; i < kSelBins; i += BLOCK) ss.hist2[i] = i + 1 < kSelBins ? cur[i + 1] : 0u;
         const uint64_t* gout = a.sel_out + int64_t(q) * k;
         for (int i = threadIdx.x; i < t.above; i += BLOCK) tmp[i] = gout[i];
         const uint64_t* gtie = a.sel_tie + int64_t(q) * kSelTieCap;
@@ -314,7 +348,7 @@ cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
     constexpr int kPreSmemMax = 160 * 1024;
     const size_t pre_bytes = size_t(a.B + 1) * 4;
     if (pre_bytes > size_t(kPreSmemMax)) return cudaErrorInvalidValue;
-    const int grid = 2 * num_sms;
+    const int grid = 3 * num_sms;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_hist_kernel), 12, kPreSmemMax);
     if (e != cudaSuccess) return e;
     select_hist_kernel<<<grid, kChunkBlock, pre_bytes, s>>>(a);

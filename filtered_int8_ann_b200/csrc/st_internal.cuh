@@ -11,7 +11,7 @@ namespace st {
 // ----------------------------------------------------------------------------
 // Tunables
 // ----------------------------------------------------------------------------
-constexpr int kScanBlock = 32;             // threads per scan CTA (one independent warp)
+constexpr int kScanBlock = 128;            // threads per scan CTA (four warps sharing a unit counter)
 constexpr int kWarpItems = 512;            // list rows per work unit (one warp)
 constexpr int kQMax = 16;                  // queries per work unit
 
@@ -569,7 +569,7 @@ __device__ void block_sort_desc_counting(uint64_t* a, int m, uint64_t* tmp, Sele
 // above it, so the keys of those bins can be scattered straight to their
 // segments; only the cut bin's keys need an exact selection, and each key's
 // place inside its segment is the number of the segment's keys greater than
-// it (segments longer than 64 keys, i.e. many equal scores, use the bitonic
+// it (very long segments, i.e. many equal or close scores, use the bitonic
 // network instead).
 // ----------------------------------------------------------------------------
 struct TopkCut {
@@ -692,13 +692,17 @@ __device__ void topk_take_ties(const TopkCut& t, const uint64_t* tie, const uint
 }
 
 // Order tmp[0, m) (bins above the cut in their segments, then the cut bin's
-// keys) into out[0, m), descending. s.hist2 holds the segment starts.
+// keys) into out[0, m), descending. s.hist2 holds the segment starts. A key's
+// place is its rank in its segment (one pass over the segment per key), up to
+// kRankSegMax keys per segment; longer segments (many equal or close scores)
+// sort everything with the bitonic network instead.
+constexpr int kRankSegMax = 256;
 template <int BLOCK>
 __device__ void topk_rank(const TopkCut& t, const uint64_t* tmp, uint64_t* out, SelectSmem& s)
 {
     const int tid = threadIdx.x;
     const int m = t.m, above = t.above;
-    if (t.maxseg > 64 || m - above > 64) {
+    if (t.maxseg > kRankSegMax || m - above > kRankSegMax) {
         for (int i = tid; i < m; i += BLOCK) out[i] = tmp[i];
         __syncthreads();
         block_bitonic_desc<BLOCK>(out, m);
