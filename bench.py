@@ -44,6 +44,9 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--n", type=int, default=None, help="override the item count (profiling cases)")
     p.add_argument("--nlist", type=int, default=None, help="override the list count (profiling cases)")
+    p.add_argument("--mode", default="replica", choices=["replica", "shard"],
+                   help="N>1: replicas search their own batches (default), or document shards search the "
+                        "same batch, all-gather their top-k over NCCL and merge it exactly")
     return p.parse_args()
 
 
@@ -290,11 +293,26 @@ def main():
     world, rank, local = dist_setup(args)
     import filtered_int8_ann_b200 as st
 
-    wl, data, q, m = make_data(args, world, rank)
+    shard = args.mode == "shard"
+    # shards all search rank 0's batches; replicas search their own
+    wl, data, q, m = make_data(args, 1 if shard else world, 0 if shard else rank)
     B, P, k, d, W = wl.B, wl.nprobe, wl.k, wl.d, wl.W
     pool = q.shape[0]
-    idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
     dev = torch.device("cuda", local)
+    if shard:
+        from types import SimpleNamespace
+        from filtered_int8_ann_b200.shard import shard_arrays
+        it, sg, off, base = shard_arrays(data.items, data.sigs, data.offsets, world, rank)
+        data = SimpleNamespace(items=it.contiguous(), sigs=sg.contiguous(), offsets=off, centroids=data.centroids,
+                               queries=data.queries, masks=data.masks)
+        idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
+        idx.set_option(st.ST_OPT_ID_OFFSET, base)
+        g_ids = torch.empty((world, B, k), dtype=torch.int64, device=dev)
+        g_sc = torch.empty((world, B, k), dtype=torch.int32, device=dev)
+        m_ids = torch.empty((B, k), dtype=torch.int64, device=dev)
+        m_sc = torch.empty((B, k), dtype=torch.int32, device=dev)
+    else:
+        idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
     ids = torch.empty((B, k), dtype=torch.int64, device=dev)
     scores = torch.empty((B, k), dtype=torch.int32, device=dev)
 
@@ -313,9 +331,25 @@ def main():
     del data
     torch.cuda.empty_cache()
 
+    def step(i, stage_events=None):
+        if stage_events is None:
+            idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores)
+        else:
+            idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores, stage_events=stage_events)
+        if shard:
+            # every shard's top-k to every rank, then the exact merge
+            if world > 1:
+                import torch.distributed as dist
+                dist.all_gather_into_tensor(g_ids, ids)
+                dist.all_gather_into_tensor(g_sc, scores)
+            else:
+                g_ids[0].copy_(ids)
+                g_sc[0].copy_(scores)
+            st.st_merge_topk(g_ids, g_sc, out_ids=m_ids, out_scores=m_sc)
+
     # warm-up
     for i in range(args.warmup):
-        idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores)
+        step(i)
     torch.cuda.synchronize()
 
     K = args.steps
@@ -331,7 +365,7 @@ def main():
     torch.cuda.synchronize()
     start.record()
     for i in range(K):
-        idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores, stage_events=evs[i])
+        step(i, evs[i])
     end.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -348,12 +382,13 @@ def main():
     scan_gbs = float(method_bytes.sum() / (stage_ms[:, 2].sum() * 1e-3) / 1e9)
     peak, peak_kind = peaks()
 
-    total_q = allreduce_sum(float(B * K), world)
+    # shards share one batch per step (their eligible counts add up); replicas each run their own
+    total_q = float(B * K) if shard else allreduce_sum(float(B * K), world)
     elig_total = allreduce_sum(float(sum(elig_per_batch[i % pool] for i in range(K))), world)
     value = total_q / (ms * 1e-3)
 
     # end to end through the host-buffer entry point (pinned memory)
-    Ke = 0 if args.no_e2e else min(K, 200)
+    Ke = 0 if (args.no_e2e or shard) else min(K, 200)
     hq = [q[b].cpu().pin_memory() for b in range(pool)]
     hm = [m[b].cpu().pin_memory() for b in range(pool)]
     hids = torch.empty((B, k), dtype=torch.int64).pin_memory()
@@ -376,12 +411,14 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "strong" if shard else "weak",
             "vs_baseline": None, "dtype": "int8/int32", "data": "synthetic",
             "config": {"workload": wl.name, "n": wl.n, "d": d, "nlist": wl.nlist, "B": B, "nprobe": P,
                        "k": k, "sig_bits": wl.sig_bits, "mask_mode": "head",
                        "l2": f"inputs larger than L2 (index {wl.n * (d + 8 * W) / 1e9:.1f} GB); steps cycle {pool} distinct query batches",
-                       "parallelism": f"replicas x{world} (independent query batches)"},
+                       "parallelism": (f"document shards x{world} (NCCL all-gather of the shards' top-k, exact merge)"
+                                       if shard else f"replicas x{world} (independent query batches)")},
             "item_scores_per_s": elig_total / (ms * 1e-3),
             "stage_ms": {"probe": stage_mean[0], "plan": stage_mean[1], "scan": stage_mean[2],
                          "select": stage_mean[3]},
@@ -396,7 +433,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": e2e, "unit": "queries/s", "h2d_bytes_per_step": B * (d + 8 * W),
                     "d2h_bytes_per_step": B * k * 12},
-            "gpu_launches": KERNELS_PER_SEARCH * K,  # memset node not counted
+            "gpu_launches": (KERNELS_PER_SEARCH + (1 if shard else 0)) * K,  # memset node not counted
             "clocks": clk,
             "workload_stats": {"scanned_items": float(np.mean([x[2] for x in models])),
                                "survivor_rows": float(np.mean([x[3] for x in models])),

@@ -20,12 +20,14 @@ LIB_PATH = os.path.join(_HERE, "libst.so")
 (ST_OK, ST_ERR_INVALID_ARG, ST_ERR_UNSUPPORTED, ST_ERR_OOM, ST_ERR_CUDA, ST_ERR_DEVICE,
  ST_ERR_SCRATCH_LIMIT) = range(7)
 ST_PROBE_NOALLOC_SCRATCH_BYTES = 16 << 20
-ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY = 1, 2
+ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY, ST_OPT_ID_OFFSET = 1, 2, 3
+ST_MERGE_MAX_KEYS = 16384
 ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE = 512, 4096, 4096
 
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
-           "st_index_set_option", "st_probe_noalloc", "st_index_destroy", "st_status_string")
+           "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_destroy",
+           "st_status_string")
 
 
 class StError(RuntimeError):
@@ -57,8 +59,10 @@ def lib() -> ctypes.CDLL:
     L.st_index_check.argtypes = [P, P]
     L.st_index_set_option.argtypes = [P, ctypes.c_int, i64]
     L.st_probe_noalloc.argtypes = [P, P, i32, i32, P, P]
+    L.st_merge_topk.argtypes = [P, P, i32, i32, i32, P, P, P]
+    L.st_merge_check.argtypes = [P]
     for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
-              "st_index_set_option", "st_probe_noalloc"):
+              "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check"):
         getattr(L, f).restype = ctypes.c_int
     L.st_index_destroy.argtypes = [P]
     L.st_index_destroy.restype = None
@@ -182,6 +186,25 @@ def st_probe_noalloc(index: int, queries: torch.Tensor, nprobe: int, out_probe: 
     return out_probe
 
 
+def st_merge_topk(ids: torch.Tensor, scores: torch.Tensor, out_ids: Optional[torch.Tensor] = None,
+                  out_scores: Optional[torch.Tensor] = None, stream=None):
+    """Exact merge of G document shards' results: ids int64 [G, B, k] and
+    scores int32 [G, B, k] (device, contiguous) -> (ids [B, k], scores [B, k])."""
+    G, B, k = ids.shape
+    if out_ids is None:
+        out_ids = torch.empty((B, k), dtype=torch.int64, device=ids.device)
+    if out_scores is None:
+        out_scores = torch.empty((B, k), dtype=torch.int32, device=ids.device)
+    _check(lib().st_merge_topk(_ptr(ids), _ptr(scores), G, B, k, _ptr(out_ids), _ptr(out_scores),
+                               _stream(stream)), "st_merge_topk")
+    return out_ids, out_scores
+
+
+def st_merge_check(stream=None) -> int:
+    """Synchronize and return the merge's device-side status (ST_OK or ST_ERR_DEVICE)."""
+    return lib().st_merge_check(_stream(stream))
+
+
 def st_index_destroy(index: Optional[int]):
     if index:
         lib().st_index_destroy(index)
@@ -206,6 +229,16 @@ class Index:
 
     def check(self, stream=None) -> int:
         return st_index_check(self.handle, stream)
+
+    @classmethod
+    def shard(cls, items, sigs, list_offsets, centroids, shards, g, stream=None):
+        """Index of document shard g of `shards` (rows split by contiguous ranges,
+        global ids returned)."""
+        from .shard import shard_arrays
+        it, sg, off, base = shard_arrays(items, sigs, list_offsets, shards, g)
+        idx = cls(it.contiguous(), sg.contiguous(), off, centroids, stream)
+        idx.set_option(ST_OPT_ID_OFFSET, base)
+        return idx
 
     def set_option(self, option, value):
         st_index_set_option(self.handle, option, value)

@@ -27,6 +27,7 @@ struct st_index {
     cudaMemPool_t pool = nullptr;
     int64_t cand_bytes = int64_t(2) << 30;
     int64_t cand_cap_override = 0;
+    int64_t id_offset = 0;
 };
 
 namespace st {
@@ -206,6 +207,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.max_units = int32_t(max_units);
     a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
     a.cap = cap;
+    a.id_offset = idx->id_offset;
     a.sel_out = reinterpret_cast<uint64_t*>(base + L.off_sel_out);
     a.sel_tie = reinterpret_cast<uint64_t*>(base + L.off_sel_tie);
     a.err = idx->err;
@@ -459,6 +461,29 @@ st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B
     return cuda_status(st::launch_probe_noalloc(a, S, stream));
 }
 
+st_status st_merge_topk(const int64_t* ids, const int32_t* scores, int32_t G, int32_t B, int32_t k,
+                        int64_t* out_ids, int32_t* out_scores, cudaStream_t stream)
+{
+    if (G < 1 || B < 1 || k < 1) return ST_ERR_INVALID_ARG;
+    if (k > ST_MAX_K || int64_t(G) * k > ST_MERGE_MAX_KEYS) return ST_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ST_ERR_CUDA;
+    if (!is_device_ptr(ids, dev) || !is_device_ptr(scores, dev) || !is_device_ptr(out_ids, dev) ||
+        !is_device_ptr(out_scores, dev))
+        return ST_ERR_INVALID_ARG;
+    if (!aligned(ids, 8) || !aligned(scores, 4) || !aligned(out_ids, 8) || !aligned(out_scores, 4))
+        return ST_ERR_INVALID_ARG;
+    return cuda_status(st::launch_merge(ids, scores, G, B, k, out_ids, out_scores, stream));
+}
+
+st_status st_merge_check(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return ST_ERR_CUDA;
+    uint32_t word = 0;
+    if (st::merge_error_word(&word, true) != cudaSuccess) return ST_ERR_CUDA;
+    return word ? ST_ERR_DEVICE : ST_OK;
+}
+
 st_status st_index_check(const st_index* idx, cudaStream_t stream)
 {
     if (idx == nullptr) return ST_ERR_INVALID_ARG;
@@ -483,6 +508,10 @@ st_status st_index_set_option(st_index* idx, st_option opt, int64_t value)
         return ST_OK;
     case ST_OPT_CANDIDATE_CAPACITY:
         idx->cand_cap_override = value;
+        return ST_OK;
+    case ST_OPT_ID_OFFSET:
+        if (value + idx->n >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
+        idx->id_offset = value;
         return ST_OK;
     }
     return ST_ERR_INVALID_ARG;

@@ -328,7 +328,7 @@ select_kernel(SearchArgs a, int stage_cap)
     }
     for (int r = threadIdx.x; r < k; r += BLOCK) {
         const uint64_t key = r < m ? out[r] : 0ull;  // key 0 reads as (id -1, INT32_MIN)
-        a.out_ids[int64_t(q) * k + r] = key_id(key);
+        a.out_ids[int64_t(q) * k + r] = key == 0ull ? -1 : key_id(key) + a.id_offset;
         a.out_scores[int64_t(q) * k + r] = key_score(key);
     }
     if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);

@@ -102,6 +102,7 @@ struct SearchArgs {
     uint32_t* sel_cursor;    // [B][kSelBins] final top-k: keys placed per bin (zeroed)
     uint64_t* sel_out;       // [B][k] final top-k: keys above the cut, grouped by bin
     uint64_t* sel_tie;       // [B][kSelTieCap] final top-k: keys of the cut bin
+    int64_t id_offset;       // added to every returned item id
     unsigned long long* eligible_cnt;  // [B][kCntStride / 2], word 0 used        (zeroed)
     PlanCtl* ctl;            // unit allocation counter                   (zeroed)
     int32_t* probe;          // [B][P]
@@ -836,6 +837,9 @@ cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
+                         int32_t* out_scores, cudaStream_t s);
+cudaError_t merge_error_word(uint32_t* word, bool clear);
 size_t scan_smem_bytes(int d, int W);
 cudaError_t launch_build_planes(const uint64_t* sigs, const int64_t* offsets, const int32_t* chunk_start,
                                 const int32_t* chunk_list, int32_t n_chunks, int W, uint32_t* planes,

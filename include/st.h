@@ -147,7 +147,12 @@ typedef enum {
     ST_OPT_CANDIDATE_BYTES = 1,
     /* Force the per-query candidate capacity (keys) instead of deriving it;
        0 restores the default. Values below k + 1024 are raised to that. */
-    ST_OPT_CANDIDATE_CAPACITY = 2
+    ST_OPT_CANDIDATE_CAPACITY = 2,
+    /* Added to every item id the index returns (default 0): an index built
+       from rows [r0, r1) of a larger collection, with this option set to r0,
+       returns ids of that collection -- one document shard of it (see
+       st_merge_topk). Rejected with UNSUPPORTED unless offset + n < 2^31. */
+    ST_OPT_ID_OFFSET = 3
 } st_option;
 
 /* Set an option; INVALID_ARG for an unknown option or a negative value.
@@ -197,6 +202,37 @@ st_status st_index_set_option(st_index* idx, st_option opt, int64_t value);
 #define ST_PROBE_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB */
 st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B, int32_t nprobe,
                            int32_t* out_probe, cudaStream_t stream);
+
+/*
+ * Exact merge of document-shard results. Splitting the items into disjoint
+ * shards (each searched as its own index with the same centroids, nprobe and
+ * the shard's ST_OPT_ID_OFFSET) and keeping the k best of the union of the
+ * shards' top-k lists gives exactly the unsharded top-k: every item of the
+ * global top-k is in the top-k of its own shard. The pages name document
+ * sharding across GPUs as the way to scale the index out (SilverTorch: Index
+ * as Model, section on scaling); this call is its merge step, after the
+ * caller has gathered the shards' results (for example with an NCCL
+ * all-gather) into one device buffer.
+ *
+ *   ids        device int64 [G][B][k]   shard g's ids for query b (id -1 = padding)
+ *   scores     device int32 [G][B][k]
+ *   out_ids    device int64 [B][k]      merged, ordered like st_search, padded
+ *   out_scores device int32 [B][k]
+ *
+ * Ids must be distinct across shards (disjoint shards) and below 2^31.
+ * Asynchronous on `stream`; allocates nothing. Errors: INVALID_ARG (null or
+ * non-device pointer, G < 1, B < 1, k < 1), UNSUPPORTED (k above ST_MAX_K, or
+ * G * k above ST_MERGE_MAX_KEYS), CUDA. A kernel-side error (an id out of
+ * range) sets the calling device's merge error word, read by st_merge_check.
+ */
+#define ST_MERGE_MAX_KEYS 16384
+st_status st_merge_topk(const int64_t* ids, const int32_t* scores, int32_t G, int32_t B, int32_t k,
+                        int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
+
+/* Wait for `stream`, then report and clear the merge error word of the
+   current device: ST_OK, ST_ERR_DEVICE (an input id was out of range), or
+   ST_ERR_CUDA. */
+st_status st_merge_check(cudaStream_t stream);
 
 /* Free the index (NULL-safe). Waits for the device to finish work that may
    still use it. */

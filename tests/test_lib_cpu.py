@@ -64,5 +64,8 @@ def test_search_rejects_null_index(lib):
     assert lib.st_search_host(None, fake, fake, 1, 1, 1, fake, fake, None) == st.ST_ERR_INVALID_ARG
     assert lib.st_index_check(None, None) == st.ST_ERR_INVALID_ARG
     assert lib.st_probe_noalloc(None, fake, 1, 1, fake, None) == st.ST_ERR_INVALID_ARG
+    assert lib.st_merge_topk(fake, fake, 0, 1, 1, fake, fake, None) == st.ST_ERR_INVALID_ARG
+    assert lib.st_merge_topk(fake, fake, 1, 1, 0, fake, fake, None) == st.ST_ERR_INVALID_ARG
+    assert lib.st_merge_topk(fake, fake, 2, 1, 8192, fake, fake, None) == st.ST_ERR_UNSUPPORTED
     assert lib.st_index_set_option(None, 1, 5) == st.ST_ERR_INVALID_ARG
     lib.st_index_destroy(None)  # NULL-safe
