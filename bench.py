@@ -50,6 +50,24 @@ def parse():
     return p.parse_args()
 
 
+def scan_traffic():
+    """DRAM bytes per scan launch from the committed ncu summary, if it was
+    measured on the scan source as it is now (else None)."""
+    import hashlib
+    try:
+        text = open(os.path.join(ROOT, "profiles", "scan_kernel_traffic_ivf_80m.md")).read()
+        fields = dict(l.split(": ", 1) for l in text.splitlines() if l.startswith(("source_sha256", "dram_bytes")))
+        h = hashlib.sha256()
+        for f in ("scan.cu", "st_internal.cuh"):
+            with open(os.path.join(ROOT, "filtered_int8_ann_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest() != fields["source_sha256"].strip():
+            return None
+        return float(fields["dram_bytes_per_launch_mean"])
+    except Exception:
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -423,7 +441,8 @@ def main():
             "stage_ms": {"probe": stage_mean[0], "plan": stage_mean[1], "scan": stage_mean[2],
                          "select": stage_mean[3]},
             "roofline": {"bound": "hbm", "kernel": "scan_kernel", "achieved": scan_gbs, "peak": peak,
-                         "unit": "GB/s", "frac": scan_gbs / peak, "traffic": None,
+                         "unit": "GB/s", "frac": scan_gbs / peak,
+                         "traffic": scan_traffic() if wl.name == "ivf_80m" else None,
                          "peak_kind": peak_kind,
                          "bytes_per_launch": float(method_bytes.mean()),
                          "signature_plane_bytes_per_launch": float(np.mean([x[6] for x in models])),
