@@ -1,8 +1,10 @@
 // Exact merge of document-shard top-k lists: for each query, the k best keys
 // (score descending, then id ascending) of the union of the shards' lists.
 // With disjoint shards every item of the global top-k is in its own shard's
-// top-k, so the merge reproduces the unsharded search (SilverTorch: Index as
-// Model, section on scaling the index out across GPUs by sharding documents).
+// top-k, so the merge reproduces the unsharded search. Document sharding is how
+// the pages scale out once one GPU is used up (SilverTorch: Index as Model,
+// section on engineering for scale and freshness, vertical and horizontal
+// scaling paragraph).
 //
 // One CTA per query: the G*k (id, score) pairs become 64-bit keys in shared
 // memory (padding entries, id -1, are dropped), and block_topk_sorted picks

@@ -209,8 +209,9 @@ st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B
  * the shard's ST_OPT_ID_OFFSET) and keeping the k best of the union of the
  * shards' top-k lists gives exactly the unsharded top-k: every item of the
  * global top-k is in the top-k of its own shard. The pages name document
- * sharding across GPUs as the way to scale the index out (SilverTorch: Index
- * as Model, section on scaling); this call is its merge step, after the
+ * sharding as the way to scale out once one GPU is used up (SilverTorch:
+ * Index as Model, section on engineering for scale and freshness, vertical and
+ * horizontal scaling paragraph); this call is its merge step, after the
  * caller has gathered the shards' results (for example with an NCCL
  * all-gather) into one device buffer.
  *
