@@ -237,7 +237,7 @@ select_scatter_kernel(SearchArgs a)
         uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
         uint64_t* out = a.sel_out + int64_t(q) * k;
         uint64_t* tie = a.sel_tie + int64_t(q) * kSelTieCap;
-        uint32_t* tcnt = a.score_rng + int64_t(q) * kCntStride + 2;
+        uint32_t* tcnt = a.score_rng + int64_t(q) * kCntStride + kRngTie;
         constexpr int U = kChunk / kChunkBlock;
         uint64_t v[U];
 #pragma unroll
