@@ -26,8 +26,8 @@ ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE = 512, 4096, 4096
 
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
-           "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_destroy",
-           "st_status_string")
+           "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
+           "st_index_destroy", "st_status_string")
 
 
 class StError(RuntimeError):
@@ -61,8 +61,9 @@ def lib() -> ctypes.CDLL:
     L.st_probe_noalloc.argtypes = [P, P, i32, i32, P, P]
     L.st_merge_topk.argtypes = [P, P, i32, i32, i32, P, P, P]
     L.st_merge_check.argtypes = [P]
+    L.st_index_update.argtypes = [P, P, P, P, i64, P]
     for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
-              "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check"):
+              "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update"):
         getattr(L, f).restype = ctypes.c_int
     L.st_index_destroy.argtypes = [P]
     L.st_index_destroy.restype = None
@@ -223,6 +224,13 @@ class Index:
 
     def search_host(self, queries, qmasks, nprobe, k, **kw):
         return st_search_host(self.handle, queries, qmasks, nprobe, k, **kw)
+
+    def update(self, ids, items=None, sigs=None, stream=None):
+        """Replace the rows and/or signatures of existing items in place (device tensors)."""
+        if sigs is not None:
+            sigs = _as_words(sigs)
+        _check(lib().st_index_update(self.handle, _ptr(ids), _ptr(items), _ptr(sigs), int(ids.numel()),
+                                     _stream(stream)), "st_index_update")
 
     def probe_noalloc(self, queries, nprobe, out_probe, stream=None):
         return st_probe_noalloc(self.handle, queries, nprobe, out_probe, stream)

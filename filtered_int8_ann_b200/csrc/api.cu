@@ -484,6 +484,20 @@ st_status st_merge_check(cudaStream_t stream)
     return word ? ST_ERR_DEVICE : ST_OK;
 }
 
+st_status st_index_update(st_index* idx, const int64_t* ids, const int8_t* items, const uint64_t* sigs,
+                          int64_t m, cudaStream_t stream)
+{
+    if (idx == nullptr || m < 0 || (items == nullptr && sigs == nullptr)) return ST_ERR_INVALID_ARG;
+    if (m == 0) return ST_OK;
+    DeviceGuard g(idx->device);
+    if (!is_device_ptr(ids, idx->device) || !aligned(ids, 8)) return ST_ERR_INVALID_ARG;
+    if (items && (!is_device_ptr(items, idx->device) || !aligned(items, 16))) return ST_ERR_INVALID_ARG;
+    if (sigs && (!is_device_ptr(sigs, idx->device) || !aligned(sigs, 8))) return ST_ERR_INVALID_ARG;
+    return cuda_status(st::launch_update(idx->items, idx->sigs, idx->planes, idx->offsets, idx->chunk_start,
+                                         idx->nlist, idx->n, idx->d, idx->W, ids, items, sigs, m, idx->err,
+                                         stream));
+}
+
 st_status st_index_check(const st_index* idx, cudaStream_t stream)
 {
     if (idx == nullptr) return ST_ERR_INVALID_ARG;

@@ -49,6 +49,67 @@ build_planes_kernel(const uint64_t* __restrict__ sigs, const int64_t* __restrict
     }
 }
 
+// In-place update of m rows: one warp per updated row copies the new row
+// and signature and rewrites the row's bit in each of its chunk's planes
+// (atomically: other rows of the same plane words may change at the same time).
+template <int W>
+__global__ void __launch_bounds__(256)
+update_kernel(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets, const int32_t* chunk_start,
+              int32_t nlist, int64_t n, int d, const int64_t* ids, const int8_t* new_items,
+              const uint64_t* new_sigs, int64_t m, uint32_t* err)
+{
+    constexpr int NPL = 64 * W;
+    const int lane = threadIdx.x & 31;
+    const int64_t j = (int64_t(blockIdx.x) * 256 + threadIdx.x) >> 5;
+    if (j >= m) return;
+    const int64_t id = ids[j];
+    if (id < 0 || id >= n) {
+        if (lane == 0) atomicOr(err, kErrUpdateId);
+        return;
+    }
+    if (new_items)
+        for (int p = lane; p < d / 16; p += 32)
+            reinterpret_cast<int4*>(items + id * d)[p] = reinterpret_cast<const int4*>(new_items + j * d)[p];
+    if (!new_sigs) return;
+    // the row's list: the last c with offsets[c] <= id (empty lists share offsets)
+    int lo = 0, hi = nlist - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= id) lo = mid;
+        else hi = mid - 1;
+    }
+    const int64_t r = id - offsets[lo];
+    const int64_t t = chunk_start[lo] + r / kWarpItems;
+    const int w = int((r % kWarpItems) >> 5);
+    const uint32_t bit = 1u << (r & 31);
+    uint64_t s0 = new_sigs[j * W], s1 = W > 1 ? new_sigs[j * W + 1] : 0ull;
+    if (lane == 0) {
+        sigs[id * W] = s0;
+        if (W > 1) sigs[id * W + 1] = s1;
+    }
+    uint32_t* pl = planes + t * NPL * 16 + w;
+    for (int b = lane; b < NPL; b += 32) {
+        const bool on = ((b < 64 ? s0 : s1) >> (b & 63)) & 1ull;
+        if (on) atomicOr(pl + b * 16, bit);
+        else atomicAnd(pl + b * 16, ~bit);
+    }
+}
+
+cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets,
+                          const int32_t* chunk_start, int32_t nlist, int64_t n, int d, int W, const int64_t* ids,
+                          const int8_t* new_items, const uint64_t* new_sigs, int64_t m, uint32_t* err, cudaStream_t s)
+{
+    if (m <= 0) return cudaSuccess;
+    const int64_t blocks = (m * 32 + 255) / 256;
+    if (W == 2)
+        update_kernel<2><<<unsigned(blocks), 256, 0, s>>>(items, sigs, planes, offsets, chunk_start, nlist, n, d, ids,
+                                                          new_items, new_sigs, m, err);
+    else
+        update_kernel<1><<<unsigned(blocks), 256, 0, s>>>(items, sigs, planes, offsets, chunk_start, nlist, n, d, ids,
+                                                          new_items, new_sigs, m, err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_build_planes(const uint64_t* sigs, const int64_t* offsets, const int32_t* chunk_start,
                                 const int32_t* chunk_list, int32_t n_chunks, int W, uint32_t* planes,
                                 cudaStream_t s)

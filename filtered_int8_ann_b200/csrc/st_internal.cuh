@@ -42,6 +42,7 @@ enum : uint32_t {
     kErrOverflowPath = 1u << 3, // the exact overflow path met an impossible state
     kErrUnitTable = 1u << 4,    // more work units than the host-sized table holds
     kErrCopyTimeout = 1u << 5,  // a bulk copy did not complete within the wait bound
+    kErrUpdateId = 1u << 6,     // an in-place update named a row outside the index
 };
 
 // ----------------------------------------------------------------------------
@@ -841,6 +842,9 @@ cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B
                          int32_t* out_scores, cudaStream_t s);
 cudaError_t merge_error_word(uint32_t* word, bool clear);
 size_t scan_smem_bytes(int d, int W);
+cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets,
+                          const int32_t* chunk_start, int32_t nlist, int64_t n, int d, int W, const int64_t* ids,
+                          const int8_t* new_items, const uint64_t* new_sigs, int64_t m, uint32_t* err, cudaStream_t s);
 cudaError_t launch_build_planes(const uint64_t* sigs, const int64_t* offsets, const int32_t* chunk_start,
                                 const int32_t* chunk_list, int32_t n_chunks, int W, uint32_t* planes,
                                 cudaStream_t s);

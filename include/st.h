@@ -235,6 +235,31 @@ st_status st_merge_topk(const int64_t* ids, const int32_t* scores, int32_t G, in
    ST_ERR_CUDA. */
 st_status st_merge_check(cudaStream_t stream);
 
+/*
+ * Streaming in-place update: replace the embedding rows and/or the Bloom
+ * signatures of m existing items, without a rebuild. The pages keep the
+ * index fresh between full snapshots by streaming new signals into the
+ * in-memory model (SilverTorch: Index as Model, section on engineering for
+ * scale and freshness, index freshness paragraph); this call is that step for
+ * items whose row stays in its list. Inserting new items and deleting items
+ * are not provided.
+ *
+ *   ids    device int64 [m]             row indices of the index (without any
+ *                                       ST_OPT_ID_OFFSET); distinct within a call
+ *   items  device int8  [m][d] or NULL  new rows (NULL: rows unchanged)
+ *   sigs   device uint64 [m][sig_words] or NULL  new signatures (NULL: unchanged)
+ *
+ * The signature bit-planes the search reads are rewritten with the
+ * signatures. Asynchronous on `stream`: searches enqueued later on the same
+ * stream see the new values; searches on other streams must be ordered after
+ * it by the caller (they read the same memory), and two updates must not
+ * overlap. An id outside [0, n) is skipped and recorded in the index's error
+ * word (st_index_check). Errors: INVALID_ARG (null index, m < 0, null or
+ * non-device ids when m > 0, non-device items / sigs, both NULL), CUDA.
+ */
+st_status st_index_update(st_index* idx, const int64_t* ids, const int8_t* items, const uint64_t* sigs,
+                          int64_t m, cudaStream_t stream);
+
 /* Free the index (NULL-safe). Waits for the device to finish work that may
    still use it. */
 void st_index_destroy(st_index* idx);
