@@ -108,6 +108,13 @@ struct ScratchLayout {
 
 int64_t candidate_capacity(const st_index* idx, int32_t B, int32_t P, int32_t k)
 {
+    if (k > ST_SMALL_K) {
+        // the global-memory final top-k has no overflow path: room for the key
+        // of every row of the nprobe largest lists, so the scan cannot overflow
+        int64_t cap = std::max<int64_t>(idx->top_prefix[std::min<int64_t>(P, idx->nlist)], int64_t(k) + st::kSelectBlock);
+        cap += 1;
+        return (cap + 31) / 32 * 32;
+    }
     int64_t cap = idx->top_prefix[std::min<int64_t>(P, idx->nlist)];
     const int64_t budget = idx->cand_bytes / 8 / B;
     if (cap > budget) cap = budget;
@@ -465,7 +472,7 @@ st_status st_merge_topk(const int64_t* ids, const int32_t* scores, int32_t G, in
                         int64_t* out_ids, int32_t* out_scores, cudaStream_t stream)
 {
     if (G < 1 || B < 1 || k < 1) return ST_ERR_INVALID_ARG;
-    if (k > ST_MAX_K || int64_t(G) * k > ST_MERGE_MAX_KEYS) return ST_ERR_UNSUPPORTED;
+    if (k > ST_SMALL_K || int64_t(G) * k > ST_MERGE_MAX_KEYS) return ST_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ST_ERR_CUDA;
     if (!is_device_ptr(ids, dev) || !is_device_ptr(scores, dev) || !is_device_ptr(out_ids, dev) ||

@@ -75,7 +75,7 @@ cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B
     const int nkeys = G * k > pw ? G * k : pw;
     const size_t smem = (size_t((k + 1) & ~1) + kMergeTieCap + size_t(nkeys)) * 8;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_kernel), 14,
-                                     int((size_t(ST_MAX_K) + kMergeTieCap + ST_MERGE_MAX_KEYS) * 8));
+                                     int((size_t(ST_SMALL_K) + kMergeTieCap + ST_MERGE_MAX_KEYS) * 8));
     if (e != cudaSuccess) return e;
     merge_kernel<<<B, kMergeBlock, smem, s>>>(ids, scores, G, B, k, out_ids, out_scores);
     return cudaGetLastError();

@@ -334,6 +334,76 @@ select_kernel(SearchArgs a, int stage_cap)
     if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
 }
 
+// ----------------------------------------------------------------------------
+// k above ST_SMALL_K: the same histogram and scatter, then the cut bin's best
+// per query and every key's rank in its segment, all in global memory.
+// ----------------------------------------------------------------------------
+template <int BLOCK>
+__global__ void __launch_bounds__(BLOCK)
+select_ties_kernel(SearchArgs a)
+{
+    __shared__ SelectSmem ss;
+    const int q = blockIdx.x;
+    const int k = a.k;
+    const int64_t n = a.cand_cnt[int64_t(q) * kCntStride];
+    if (n <= 0) return;
+    int32_t lo;
+    uint32_t sh;
+    query_range(a, q, lo, sh);
+    const uint32_t* rng = a.score_rng + int64_t(q) * kCntStride;
+    TopkCut t;
+    t.lo = lo;
+    t.sh = sh;
+    t.cut = int(rng[kRngCut]);
+    t.above = int(rng[kRngAbove]);
+    t.tcount = int(rng[kRngTcount]);
+    t.maxseg = int(rng[kRngMaxseg]);
+    t.m = n < k ? int(n) : k;
+    const uint64_t* gtie = t.tcount <= kSelTieCap ? a.sel_tie + int64_t(q) * kSelTieCap : nullptr;
+    topk_take_ties<BLOCK>(t, gtie, a.cand + int64_t(q) * a.cap, n, a.sel_out + int64_t(q) * k, ss, a.err);
+}
+
+// One thread per output position: the key at position p of the query's
+// bin-grouped keys goes to its segment start + its rank in the segment.
+__global__ void __launch_bounds__(256)
+select_rank_kernel(SearchArgs a)
+{
+    const int k = a.k;
+    const int64_t idx = int64_t(blockIdx.x) * 256 + threadIdx.x;
+    if (idx >= int64_t(a.B) * k) return;
+    const int q = int(idx / k);
+    const int p = int(idx - int64_t(q) * k);
+    const int64_t n = a.cand_cnt[int64_t(q) * kCntStride];
+    const int m = n < k ? int(n) : k;
+    if (p == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
+    if (p >= m) {
+        a.out_ids[idx] = -1;
+        a.out_scores[idx] = INT32_MIN;
+        return;
+    }
+    const uint64_t* keys = a.sel_out + int64_t(q) * k;
+    const uint64_t key = keys[p];
+    const int above = int(a.score_rng[int64_t(q) * kCntStride + kRngAbove]);
+    int beg, end;
+    if (p >= above) {
+        beg = above;
+        end = m;
+    } else {
+        int32_t lo;
+        uint32_t sh;
+        query_range(a, q, lo, sh);
+        const int b = topk_bin(key, lo, sh);
+        const uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;  // after the scatter: bin ends
+        beg = b + 1 < kSelBins ? int(cur[b + 1]) : 0;
+        end = int(cur[b]);
+    }
+    int r = 0;
+    for (int j = beg; j < end; ++j) r += keys[j] > key ? 1 : 0;
+    const int64_t o = int64_t(q) * k + beg + r;
+    a.out_ids[o] = key_id(key) + a.id_offset;
+    a.out_scores[o] = key_score(key);
+}
+
 size_t select_smem(int k, int* stage_cap)
 {
     const size_t budget = 208 * 1024;
@@ -359,6 +429,14 @@ cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
     select_scatter_kernel<<<grid, kChunkBlock, pre_bytes, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (a.k > ST_SMALL_K) {
+        select_ties_kernel<kSelectBlock><<<a.B, kSelectBlock, 0, s>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        const int64_t threads = int64_t(a.B) * a.k;
+        select_rank_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(a);
+        return cudaGetLastError();
+    }
     int stage_cap = 0;
     const size_t smem = select_smem(a.k, &stage_cap);
     e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8, int(smem));

@@ -54,7 +54,10 @@ typedef enum {
 
 /* Supported limits (ST_ERR_UNSUPPORTED outside them). */
 #define ST_MAX_D 512         /* d must be a multiple of 16 in [16, 512] */
-#define ST_MAX_K 4096        /* 1 <= k <= 4096 */
+#define ST_MAX_K 262144      /* 1 <= k <= 262144 */
+#define ST_SMALL_K 4096      /* k above this takes a global-memory final top-k and
+                                needs device memory for the key of every row of the
+                                probed lists (ST_ERR_OOM when it does not fit) */
 #define ST_MAX_NPROBE 4096   /* 1 <= nprobe <= min(nlist, 4096) */
 /* n < 2^31 items; sig_words is 1 (64-bit signatures) or 2 (128-bit). */
 
@@ -222,7 +225,7 @@ st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B
  *
  * Ids must be distinct across shards (disjoint shards) and below 2^31.
  * Asynchronous on `stream`; allocates nothing. Errors: INVALID_ARG (null or
- * non-device pointer, G < 1, B < 1, k < 1), UNSUPPORTED (k above ST_MAX_K, or
+ * non-device pointer, G < 1, B < 1, k < 1), UNSUPPORTED (k above ST_SMALL_K, or
  * G * k above ST_MERGE_MAX_KEYS), CUDA. A kernel-side error (an id out of
  * range) sets the calling device's merge error word, read by st_merge_check.
  */
