@@ -18,8 +18,6 @@ constexpr int kQMax = 16;                  // queries per work unit
 constexpr int kProbeBlock = 512;
 constexpr int kProbeSmemKeys = 16384;      // nlist up to this keeps probe keys in smem
 constexpr int kSelectBlock = 1024;
-constexpr int kSelectSmemKeys = 22528;     // candidates up to this are selected in smem
-constexpr int kPlanBlock = 512;
 // Per-query counters sit one 128-byte line apart, so the reservation atomics
 // of different queries spread over the L2 slices instead of queueing on one.
 constexpr int kCntStride = 32;             // uint32 words (16 uint64) per query
@@ -31,17 +29,13 @@ constexpr int kMaskBitsMax = 128;          // signature bits
 constexpr int kSelBits = 11;               // radix digit of the selections
 constexpr int kSelBins = 1 << kSelBits;
 constexpr int kSelTieCap = 4096;           // cut-bin keys the final top-k keeps per query
-constexpr uint32_t kWaitLimit = 1u << 10;  // bounded mbarrier polls before giving up
-constexpr uint32_t kWaitHintNs = 10000000u; // each poll may sleep up to 10 ms waiting for the phase
 
 // Device error word bits (st_index_check reports any of them as ST_ERR_DEVICE).
 enum : uint32_t {
     kErrUnitDecode = 1u << 0,   // a work unit did not map to a list
-    kErrQueryGroup = 1u << 1,   // a query group exceeded kQMax
     kErrSelectCount = 1u << 2,  // a selection collected the wrong number of keys
     kErrOverflowPath = 1u << 3, // the exact overflow path met an impossible state
     kErrUnitTable = 1u << 4,    // more work units than the host-sized table holds
-    kErrCopyTimeout = 1u << 5,  // a bulk copy did not complete within the wait bound
     kErrUpdateId = 1u << 6,     // an in-place update named a row outside the index
 };
 
@@ -145,55 +139,6 @@ __device__ __forceinline__ unsigned lanemask_lt()
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// mbarrier + bulk async copy (global -> this CTA's shared memory; never multicast)
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init()
-{
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
-        : "memory");
-    return ok != 0;
-}
-// Poll the barrier phase at most kWaitLimit times (each poll suspends the
-// thread until the phase completes or the hint expires); false if it never
-// completed.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity)
-{
-    for (uint32_t it = 0; it < kWaitLimit; ++it)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
-}
-
-// Order this thread's generic-proxy shared-memory accesses before later
-// async-proxy (bulk copy) accesses to the same memory.
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 16-byte asynchronous copy global -> shared (cp.async, L1-allocating)
@@ -364,50 +309,6 @@ __device__ uint64_t block_select_threshold(const uint64_t* keys, int64_t n, int6
         }
     }
     return s.prefix;
-}
-
-// block_collect_ge for a long 16-byte-aligned key array in global memory: each
-// thread keeps eight keys (four 16-byte loads) in flight per step.
-template <int BLOCK>
-__device__ int32_t block_collect_ge_wide(const uint64_t* keys, int64_t n, uint64_t thr, uint64_t* out,
-                                         int32_t out_cap, SelectSmem& s)
-{
-    if (threadIdx.x == 0) s.count = 0;
-    __syncthreads();
-    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
-    const int64_t n2 = n >> 1;
-    for (int64_t base = 0; base < n2; base += int64_t(BLOCK) * 4) {
-        ulonglong2 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int64_t j = base + u * BLOCK + threadIdx.x;
-            v[u] = j < n2 ? __ldcg(k2 + j) : make_ulonglong2(0ull, 0ull);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const uint64_t key = (u & 1) ? v[u >> 1].y : v[u >> 1].x;
-            const bool take = key >= thr && key != 0ull;
-            const unsigned bal = __ballot_sync(0xffffffffu, take);
-            if (bal) {
-                int32_t b0 = 0;
-                if ((threadIdx.x & 31) == 0) b0 = atomicAdd(&s.count, __popc(bal));
-                b0 = __shfl_sync(0xffffffffu, b0, 0);
-                const int32_t pos = b0 + __popc(bal & lanemask_lt());
-                if (take && pos < out_cap) out[pos] = key;
-            }
-        }
-    }
-    if ((n & 1) && threadIdx.x == 0) {
-        const uint64_t key = keys[n - 1];
-        if (key >= thr && key != 0ull) {
-            const int32_t pos = atomicAdd(&s.count, 1);
-            if (pos < out_cap) out[pos] = key;
-        }
-    }
-    __syncthreads();
-    const int32_t count = s.count;
-    __syncthreads();  // a following collect may reset the counter at once
-    return count;
 }
 
 // Copy every key >= thr from keys[0..n) into out[] (at most out_cap); returns
