@@ -27,7 +27,7 @@ ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K = 512, 262144, 4096, 4096
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
            "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
-           "st_index_destroy", "st_status_string")
+           "st_index_delete", "st_index_destroy", "st_status_string")
 
 
 class StError(RuntimeError):
@@ -38,7 +38,7 @@ class StError(RuntimeError):
 
 class _Extras(ctypes.Structure):
     _fields_ = [("eligible", ctypes.c_void_p), ("probe", ctypes.c_void_p),
-                ("stage_events", ctypes.c_void_p * 5)]
+                ("stage_events", ctypes.c_void_p * 5), ("exclude_masks", ctypes.c_void_p)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -62,8 +62,10 @@ def lib() -> ctypes.CDLL:
     L.st_merge_topk.argtypes = [P, P, i32, i32, i32, P, P, P]
     L.st_merge_check.argtypes = [P]
     L.st_index_update.argtypes = [P, P, P, P, i64, P]
+    L.st_index_delete.argtypes = [P, P, i64, P]
     for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
-              "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update"):
+              "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
+              "st_index_delete"):
         getattr(L, f).restype = ctypes.c_int
     L.st_index_destroy.argtypes = [P]
     L.st_index_destroy.restype = None
@@ -124,11 +126,13 @@ def st_index_create(items: torch.Tensor, sigs: torch.Tensor, list_offsets: torch
 def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: int, k: int,
               out_ids: Optional[torch.Tensor] = None, out_scores: Optional[torch.Tensor] = None,
               stream=None, eligible: Optional[torch.Tensor] = None,
-              probe: Optional[torch.Tensor] = None, stage_events=None):
+              probe: Optional[torch.Tensor] = None, stage_events=None,
+              exclude: Optional[torch.Tensor] = None):
     """Asynchronous search of device-resident queries; returns (ids int64 [B,k],
     scores int32 [B,k]). `eligible` [B] int64 and `probe` [B,nprobe] int32 are
     optional extra outputs; `stage_events` is a list of up to five recorded
-    torch.cuda.Event objects marking the stage boundaries (st_search_ex)."""
+    torch.cuda.Event objects marking the stage boundaries; `exclude` [B,W]
+    holds per-query exclude masks (st_search_ex)."""
     qmasks = _as_words(qmasks)
     B = queries.shape[0]
     dev = queries.device
@@ -136,12 +140,15 @@ def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: i
         out_ids = torch.empty((B, k), dtype=torch.int64, device=dev)
     if out_scores is None:
         out_scores = torch.empty((B, k), dtype=torch.int32, device=dev)
-    if eligible is None and probe is None and not stage_events:
+    if exclude is not None:
+        exclude = _as_words(exclude)
+    if eligible is None and probe is None and not stage_events and exclude is None:
         st = lib().st_search(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
                              _ptr(out_scores), _stream(stream))
         _check(st, "st_search")
     else:
         ex = _Extras(_ptr(eligible), _ptr(probe))
+        ex.exclude_masks = _ptr(exclude)
         for i, ev in enumerate(stage_events or ()):
             ex.stage_events[i] = ev.cuda_event if ev is not None else None
         st = lib().st_search_ex(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
@@ -231,6 +238,10 @@ class Index:
             sigs = _as_words(sigs)
         _check(lib().st_index_update(self.handle, _ptr(ids), _ptr(items), _ptr(sigs), int(ids.numel()),
                                      _stream(stream)), "st_index_update")
+
+    def delete(self, ids, stream=None):
+        """Delete items in place (device int64 row indices)."""
+        _check(lib().st_index_delete(self.handle, _ptr(ids), int(ids.numel()), _stream(stream)), "st_index_delete")
 
     def probe_noalloc(self, queries, nprobe, out_probe, stream=None):
         return st_probe_noalloc(self.handle, queries, nprobe, out_probe, stream)

@@ -28,6 +28,7 @@ struct st_index {
     int64_t cand_bytes = int64_t(2) << 30;
     int64_t cand_cap_override = 0;
     int64_t id_offset = 0;
+    uint32_t* dead = nullptr;        // [ceil(n / 32)] deletion bitmap, allocated at the first deletion
 };
 
 namespace st {
@@ -215,6 +216,8 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
     a.cap = cap;
     a.id_offset = idx->id_offset;
+    a.dead = idx->dead;
+    a.qexclude = extras ? extras->exclude_masks : nullptr;
     a.sel_out = reinterpret_cast<uint64_t*>(base + L.off_sel_out);
     a.sel_tie = reinterpret_cast<uint64_t*>(base + L.off_sel_tie);
     a.err = idx->err;
@@ -390,6 +393,9 @@ st_status st_search_ex(const st_index* idx, const int8_t* queries, const uint64_
             return ST_ERR_INVALID_ARG;
         if (extras->probe && (!is_device_ptr(extras->probe, idx->device) || !aligned(extras->probe, 4)))
             return ST_ERR_INVALID_ARG;
+        if (extras->exclude_masks &&
+            (!is_device_ptr(extras->exclude_masks, idx->device) || !aligned(extras->exclude_masks, 8)))
+            return ST_ERR_INVALID_ARG;
     }
     return search_impl(idx, queries, qmasks, B, nprobe, k, out_ids, out_scores, extras, stream);
 }
@@ -505,6 +511,24 @@ st_status st_index_update(st_index* idx, const int64_t* ids, const int8_t* items
                                          stream));
 }
 
+st_status st_index_delete(st_index* idx, const int64_t* ids, int64_t m, cudaStream_t stream)
+{
+    if (idx == nullptr || m < 0) return ST_ERR_INVALID_ARG;
+    if (m == 0) return ST_OK;
+    DeviceGuard g(idx->device);
+    if (!is_device_ptr(ids, idx->device) || !aligned(ids, 8)) return ST_ERR_INVALID_ARG;
+    if (idx->dead == nullptr) {
+        const size_t bytes = size_t((idx->n + 31) / 32) * 4;
+        if (cudaMalloc(&idx->dead, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            idx->dead = nullptr;
+            return ST_ERR_OOM;
+        }
+        if (cudaMemsetAsync(idx->dead, 0, bytes, stream) != cudaSuccess) return ST_ERR_CUDA;
+    }
+    return cuda_status(st::launch_delete(idx->dead, idx->n, ids, m, idx->err, stream));
+}
+
 st_status st_index_check(const st_index* idx, cudaStream_t stream)
 {
     if (idx == nullptr) return ST_ERR_INVALID_ARG;
@@ -552,6 +576,7 @@ void st_index_destroy(st_index* idx)
         cudaFree(idx->chunk_list);
         cudaFree(idx->planes);
         cudaFree(idx->err);
+        cudaFree(idx->dead);
         if (idx->pool) cudaMemPoolDestroy(idx->pool);
         cudaGetLastError();
     }

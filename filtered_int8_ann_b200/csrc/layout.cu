@@ -95,6 +95,27 @@ update_kernel(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* of
     }
 }
 
+// Deletion: one thread per id sets the item's bit in the deletion bitmap.
+__global__ void __launch_bounds__(256)
+delete_kernel(uint32_t* dead, int64_t n, const int64_t* ids, int64_t m, uint32_t* err)
+{
+    const int64_t j = int64_t(blockIdx.x) * 256 + threadIdx.x;
+    if (j >= m) return;
+    const int64_t id = ids[j];
+    if (id < 0 || id >= n) {
+        atomicOr(err, kErrUpdateId);
+        return;
+    }
+    atomicOr(dead + (id >> 5), 1u << (id & 31));
+}
+
+cudaError_t launch_delete(uint32_t* dead, int64_t n, const int64_t* ids, int64_t m, uint32_t* err, cudaStream_t s)
+{
+    if (m <= 0) return cudaSuccess;
+    delete_kernel<<<unsigned((m + 255) / 256), 256, 0, s>>>(dead, n, ids, m, err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets,
                           const int32_t* chunk_start, int32_t nlist, int64_t n, int d, int W, const int64_t* ids,
                           const int8_t* new_items, const uint64_t* new_sigs, int64_t m, uint32_t* err, cudaStream_t s)

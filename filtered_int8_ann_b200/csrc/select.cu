@@ -78,6 +78,7 @@ __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, 
                 const uint64_t* sg = a.sigs + i * W;
                 bool pass = (sg[0] & m0) == m0;
                 if (W > 1) pass = pass && ((sg[1] & m1) == m1);
+                pass = pass && keep_item(a, q, i);
                 if (pass) {
                     const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);
                     int32_t acc = 0;
@@ -156,6 +157,40 @@ __device__ __forceinline__ int item_query(const int* pre, int B, int item)
 // [2] cut-bin keys gathered, [3] chunks histogrammed, [4] cut bin, [5] keys
 // above it, [6] keys in it, [7] longest output segment.
 constexpr int kRngTie = 2, kRngDone = 3, kRngCut = 4, kRngAbove = 5, kRngTcount = 6, kRngMaxseg = 7;
+constexpr int kRngKept = 9;  // candidates left after the post-filter
+
+// The query's candidates that pass the post-filter (all of them without one).
+__device__ __forceinline__ int64_t kept_count(const SearchArgs& a, int q)
+{
+    return (a.dead || a.qexclude) ? int64_t(__ldcg(a.score_rng + int64_t(q) * kCntStride + kRngKept))
+                                  : chunked_count(a, q);
+}
+
+// Compact query q's candidates of the cut bin that pass the post-filter to
+// the front of its candidate buffer (no longer read by anyone else) and
+// return their count: one CTA, every thread's writes land only on positions
+// already read.
+template <int BLOCK>
+__device__ int compact_cut_bin(const SearchArgs& a, int q, int64_t n, const TopkCut& t)
+{
+    __shared__ int c_cnt;
+    uint64_t* keys = a.cand + int64_t(q) * a.cap;
+    if (threadIdx.x == 0) c_cnt = 0;
+    __syncthreads();
+    for (int64_t base = 0; base < n; base += BLOCK) {
+        const int64_t i = base + threadIdx.x;
+        uint64_t key = 0;
+        bool take = false;
+        if (i < n) {
+            key = keys[i];
+            take = topk_bin(key, t.lo, t.sh) == t.cut && keep_item(a, q, key_id(key));
+        }
+        __syncthreads();  // this round's reads are done before any write
+        if (take) keys[atomicAdd(&c_cnt, 1)] = key;
+        __syncthreads();
+    }
+    return c_cnt;
+}
 
 __global__ void __launch_bounds__(kChunkBlock)
 select_hist_kernel(SearchArgs a)
@@ -184,9 +219,18 @@ select_hist_kernel(SearchArgs a)
             const int i = u * kChunkBlock + threadIdx.x;
             v[u] = i < cnt ? keys[i] : 0ull;
         }
+        const bool filt = a.dead || a.qexclude;
+        int kept = 0;
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            if (u * kChunkBlock + int(threadIdx.x) < cnt) atomicAdd(&h[topk_bin(v[u], lo, sh)], 1u);
+            if (u * kChunkBlock + int(threadIdx.x) < cnt && (!filt || keep_item(a, q, key_id(v[u])))) {
+                atomicAdd(&h[topk_bin(v[u], lo, sh)], 1u);
+                ++kept;
+            }
+        if (filt) {
+            kept = __reduce_add_sync(0xffffffffu, kept);
+            if ((threadIdx.x & 31) == 0 && kept) atomicAdd(a.score_rng + int64_t(q) * kCntStride + kRngKept, uint32_t(kept));
+        }
         __syncthreads();
         uint32_t* gh = a.sel_hist + int64_t(q) * kSelBins;
         for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock)
@@ -202,7 +246,7 @@ select_hist_kernel(SearchArgs a)
             __threadfence();
             for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock) ss.hist[i] = __ldcg(gh + i);
             __syncthreads();
-            const TopkCut t = topk_cut_from_hist<kChunkBlock>(n, a.k, lo, sh, ss);
+            const TopkCut t = topk_cut_from_hist<kChunkBlock>(kept_count(a, q), a.k, lo, sh, ss);
             uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
             for (int i = threadIdx.x; i < kSelBins; i += kChunkBlock) cur[i] = ss.hist2[i];
             if (threadIdx.x == 0) {
@@ -248,6 +292,7 @@ select_scatter_kernel(SearchArgs a)
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (u * kChunkBlock + int(threadIdx.x) >= cnt) continue;
+            if ((a.dead || a.qexclude) && !keep_item(a, q, key_id(v[u]))) continue;
             const int b = topk_bin(v[u], lo, sh);
             if (b > cut) {
                 out[atomicAdd(&cur[b], 1u)] = v[u];
@@ -308,7 +353,8 @@ select_kernel(SearchArgs a, int stage_cap)
         t.above = int(rng[kRngAbove]);
         t.tcount = int(rng[kRngTcount]);
         t.maxseg = int(rng[kRngMaxseg]);
-        t.m = n < k ? int(n) : k;
+        const int64_t nk = kept_count(a, q);
+        t.m = nk < k ? int(nk) : k;
         const uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
         for (int i = threadIdx.x; i < kSelBins; i += BLOCK) ss.hist2[i] = i + 1 < kSelBins ? cur[i + 1] : 0u;
         const uint64_t* gout = a.sel_out + int64_t(q) * k;
@@ -322,6 +368,12 @@ select_kernel(SearchArgs a, int stage_cap)
             tsrc = gtie;
         }
         __syncthreads();
+        if (tsrc == nullptr && (a.dead || a.qexclude) && t.m > t.above) {
+            // the cut bin was too large to keep aside: its filtered keys, compacted
+            const int nt = compact_cut_bin<BLOCK>(a, q, n, t);
+            t.tcount = nt;
+            tsrc = a.cand + int64_t(q) * a.cap;
+        }
         topk_take_ties<BLOCK>(t, tsrc, a.cand + int64_t(q) * a.cap, n, tmp, ss, a.err);
         topk_rank<BLOCK>(t, tmp, out, ss);
         m = t.m;
@@ -358,8 +410,13 @@ select_ties_kernel(SearchArgs a)
     t.above = int(rng[kRngAbove]);
     t.tcount = int(rng[kRngTcount]);
     t.maxseg = int(rng[kRngMaxseg]);
-    t.m = n < k ? int(n) : k;
+    const int64_t nk = kept_count(a, q);
+    t.m = nk < k ? int(nk) : k;
     const uint64_t* gtie = t.tcount <= kSelTieCap ? a.sel_tie + int64_t(q) * kSelTieCap : nullptr;
+    if (gtie == nullptr && (a.dead || a.qexclude) && t.m > t.above) {
+        t.tcount = compact_cut_bin<BLOCK>(a, q, n, t);  // the cut bin's filtered keys
+        gtie = a.cand + int64_t(q) * a.cap;
+    }
     topk_take_ties<BLOCK>(t, gtie, a.cand + int64_t(q) * a.cap, n, a.sel_out + int64_t(q) * k, ss, a.err);
 }
 
@@ -373,7 +430,7 @@ select_rank_kernel(SearchArgs a)
     if (idx >= int64_t(a.B) * k) return;
     const int q = int(idx / k);
     const int p = int(idx - int64_t(q) * k);
-    const int64_t n = a.cand_cnt[int64_t(q) * kCntStride];
+    const int64_t n = a.cand_cnt[int64_t(q) * kCntStride] > 0 ? kept_count(a, q) : 0;
     const int m = n < k ? int(n) : k;
     if (p == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
     if (p >= m) {

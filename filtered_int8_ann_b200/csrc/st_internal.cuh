@@ -98,6 +98,8 @@ struct SearchArgs {
     uint64_t* sel_out;       // [B][k] final top-k: keys above the cut, grouped by bin
     uint64_t* sel_tie;       // [B][kSelTieCap] final top-k: keys of the cut bin
     int64_t id_offset;       // added to every returned item id
+    const uint32_t* dead;    // [ceil(n / 32)] deleted items, or null (none deleted)
+    const uint64_t* qexclude;  // [B][W] exclude masks, or null
     unsigned long long* eligible_cnt;  // [B][kCntStride / 2], word 0 used        (zeroed)
     PlanCtl* ctl;            // unit allocation counter                   (zeroed)
     int32_t* probe;          // [B][P]
@@ -475,6 +477,22 @@ __device__ void block_sort_desc_counting(uint64_t* a, int m, uint64_t* tmp, Sele
 // it (very long segments, i.e. many equal or close scores, use the bitonic
 // network instead).
 // ----------------------------------------------------------------------------
+// Candidate post-filter of query q: false for an item that was deleted or
+// whose signature holds every bit of q's (non-zero) exclude mask. Local id.
+__device__ __forceinline__ bool keep_item(const SearchArgs& a, int q, int64_t id)
+{
+    if (a.dead && ((a.dead[id >> 5] >> (id & 31)) & 1u)) return false;
+    if (a.qexclude) {
+        const int W = a.W;
+        const uint64_t x0 = a.qexclude[int64_t(q) * W], x1 = W > 1 ? a.qexclude[int64_t(q) * W + 1] : 0ull;
+        if (x0 | x1) {
+            const uint64_t* sg = a.sigs + id * W;
+            if ((sg[0] & x0) == x0 && (W < 2 || (sg[1] & x1) == x1)) return false;
+        }
+    }
+    return true;
+}
+
 struct TopkCut {
     int32_t lo;     // range base
     uint32_t sh;    // bin shift
@@ -743,6 +761,7 @@ cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B
                          int32_t* out_scores, cudaStream_t s);
 cudaError_t merge_error_word(uint32_t* word, bool clear);
 size_t scan_smem_bytes(int d, int W);
+cudaError_t launch_delete(uint32_t* dead, int64_t n, const int64_t* ids, int64_t m, uint32_t* err, cudaStream_t s);
 cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets,
                           const int32_t* chunk_start, int32_t nlist, int64_t n, int d, int W, const int64_t* ids,
                           const int8_t* new_items, const uint64_t* new_sigs, int64_t m, uint32_t* err, cudaStream_t s);

@@ -106,15 +106,23 @@ st_status st_search(const st_index* idx, const int8_t* queries, const uint64_t* 
                     int32_t B, int32_t nprobe, int32_t k,
                     int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
 
-/* Optional extra outputs of st_search_ex; any member may be NULL. */
+/* Optional extra inputs and outputs of st_search_ex; any member may be NULL. */
 typedef struct {
-    int64_t* eligible; /* device int64 [B]: eligible items in each query's probed
-                          lists (the number of (query, item) scores computed) */
+    int64_t* eligible; /* device int64 [B]: items of each query's probed lists
+                          that pass its mask (the number of (query, item) scores
+                          computed; items later dropped by exclusion or deletion
+                          are included) */
     int32_t* probe;    /* device int32 [B][nprobe]: the probed lists, best first */
     /* Timing hooks: each non-NULL event is recorded on `stream` at a stage
        boundary -- [0] before the probe kernel, [1] after it, [2] after the plan
        kernels, [3] after the list scan, [4] after the final top-k. */
     cudaEvent_t stage_events[5];
+    /* device uint64 [B][sig_words]: negative rules. An item whose signature
+       holds every bit of query b's exclude mask is not a result of query b
+       (an all-zero exclude mask excludes nothing). A negative targeting rule
+       of the pages' advertiser-defined targeting, tested like the mask itself
+       (so a Bloom false positive excludes too). */
+    const uint64_t* exclude_masks;
 } st_search_extras;
 
 /* st_search with optional extra outputs (extras may be NULL). */
@@ -262,6 +270,19 @@ st_status st_merge_check(cudaStream_t stream);
  */
 st_status st_index_update(st_index* idx, const int64_t* ids, const int8_t* items, const uint64_t* sigs,
                           int64_t m, cudaStream_t stream);
+
+/*
+ * Delete m items in place (tombstones): a deleted item is never returned
+ * again, by any later search on `stream` (other streams: order them after it).
+ * ids are row indices of the index (without any ST_OPT_ID_OFFSET); deleting
+ * twice is harmless; st_index_update does not revive an item. Deleted rows
+ * still take part in the scan (their scores are dropped before the final
+ * top-k) and in st_search_extras.eligible. The first deletion allocates a
+ * bitmap of n bits. An id outside [0, n) is skipped and recorded in the
+ * index's error word. Errors: INVALID_ARG (null index, m < 0, null or
+ * non-device ids when m > 0), OOM, CUDA.
+ */
+st_status st_index_delete(st_index* idx, const int64_t* ids, int64_t m, cudaStream_t stream);
 
 /* Free the index (NULL-safe). Waits for the device to finish work that may
    still use it. */
