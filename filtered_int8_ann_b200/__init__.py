@@ -27,7 +27,7 @@ ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K = 512, 262144, 4096, 4096
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
            "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
-           "st_index_delete", "st_index_destroy", "st_status_string")
+           "st_index_delete", "st_merge_topk_union", "st_index_destroy", "st_status_string")
 
 
 class StError(RuntimeError):
@@ -63,9 +63,10 @@ def lib() -> ctypes.CDLL:
     L.st_merge_check.argtypes = [P]
     L.st_index_update.argtypes = [P, P, P, P, i64, P]
     L.st_index_delete.argtypes = [P, P, i64, P]
+    L.st_merge_topk_union.argtypes = [P, P, i32, i32, i32, P, P, P]
     for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
               "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
-              "st_index_delete"):
+              "st_index_delete", "st_merge_topk_union"):
         getattr(L, f).restype = ctypes.c_int
     L.st_index_destroy.argtypes = [P]
     L.st_index_destroy.restype = None
@@ -208,6 +209,19 @@ def st_merge_topk(ids: torch.Tensor, scores: torch.Tensor, out_ids: Optional[tor
     return out_ids, out_scores
 
 
+def st_merge_topk_union(ids: torch.Tensor, scores: torch.Tensor, out_ids: Optional[torch.Tensor] = None,
+                        out_scores: Optional[torch.Tensor] = None, stream=None):
+    """Exact top-k of the union of G result lists [G, B, k] that may share items."""
+    G, B, k = ids.shape
+    if out_ids is None:
+        out_ids = torch.empty((B, k), dtype=torch.int64, device=ids.device)
+    if out_scores is None:
+        out_scores = torch.empty((B, k), dtype=torch.int32, device=ids.device)
+    _check(lib().st_merge_topk_union(_ptr(ids), _ptr(scores), G, B, k, _ptr(out_ids), _ptr(out_scores),
+                                     _stream(stream)), "st_merge_topk_union")
+    return out_ids, out_scores
+
+
 def st_merge_check(stream=None) -> int:
     """Synchronize and return the merge's device-side status (ST_OK or ST_ERR_DEVICE)."""
     return lib().st_merge_check(_stream(stream))
@@ -238,6 +252,18 @@ class Index:
             sigs = _as_words(sigs)
         _check(lib().st_index_update(self.handle, _ptr(ids), _ptr(items), _ptr(sigs), int(ids.numel()),
                                      _stream(stream)), "st_index_update")
+
+    def search_any(self, queries, mask_sets, nprobe, k, stream=None, **kw):
+        """OR of several masks per query: an item is eligible if any of the masks
+        passes. mask_sets [M, B, W] (M alternatives); one search per alternative,
+        then the exact union merge (k <= 4096, M * k <= ST_MERGE_MAX_KEYS)."""
+        M, B = mask_sets.shape[0], queries.shape[0]
+        ids = torch.empty((M, B, k), dtype=torch.int64, device=queries.device)
+        sc = torch.empty((M, B, k), dtype=torch.int32, device=queries.device)
+        for j in range(M):
+            self.search(queries, mask_sets[j].contiguous(), nprobe, k, out_ids=ids[j], out_scores=sc[j],
+                        stream=stream, **kw)
+        return st_merge_topk_union(ids, sc, stream=stream)
 
     def delete(self, ids, stream=None):
         """Delete items in place (device int64 row indices)."""

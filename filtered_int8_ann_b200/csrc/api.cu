@@ -9,6 +9,13 @@
 
 #include "st_internal.cuh"
 
+namespace st {
+// the union merge (merge.cu)
+cudaError_t launch_merge_union(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
+                               int32_t* out_scores, cudaStream_t s);
+}  // namespace st
+
+
 struct st_index {
     int device = 0;
     int num_sms = 0;
@@ -487,6 +494,21 @@ st_status st_merge_topk(const int64_t* ids, const int32_t* scores, int32_t G, in
     if (!aligned(ids, 8) || !aligned(scores, 4) || !aligned(out_ids, 8) || !aligned(out_scores, 4))
         return ST_ERR_INVALID_ARG;
     return cuda_status(st::launch_merge(ids, scores, G, B, k, out_ids, out_scores, stream));
+}
+
+st_status st_merge_topk_union(const int64_t* ids, const int32_t* scores, int32_t G, int32_t B, int32_t k,
+                              int64_t* out_ids, int32_t* out_scores, cudaStream_t stream)
+{
+    if (G < 1 || B < 1 || k < 1) return ST_ERR_INVALID_ARG;
+    if (k > ST_SMALL_K || int64_t(G) * k > ST_MERGE_MAX_KEYS) return ST_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ST_ERR_CUDA;
+    if (!is_device_ptr(ids, dev) || !is_device_ptr(scores, dev) || !is_device_ptr(out_ids, dev) ||
+        !is_device_ptr(out_scores, dev))
+        return ST_ERR_INVALID_ARG;
+    if (!aligned(ids, 8) || !aligned(scores, 4) || !aligned(out_ids, 8) || !aligned(out_scores, 4))
+        return ST_ERR_INVALID_ARG;
+    return cuda_status(st::launch_merge_union(ids, scores, G, B, k, out_ids, out_scores, stream));
 }
 
 st_status st_merge_check(cudaStream_t stream)

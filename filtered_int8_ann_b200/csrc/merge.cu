@@ -20,6 +20,25 @@ static __device__ uint32_t g_merge_err;
 constexpr int kMergeBlock = 1024;
 constexpr int kMergeTieCap = 1024;
 
+// Is `key` in list g' (ordered like st_search: keys descending, padding last)?
+__device__ __forceinline__ bool in_sorted_list(const int64_t* ids, const int32_t* scores, int64_t row, int k,
+                                               uint64_t key)
+{
+    int lo = 0, hi = k - 1;  // the first position whose key is <= `key`
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int64_t id = ids[row + mid];
+        const uint64_t km = id >= 0 ? pack_key(scores[row + mid], uint32_t(id)) : 0ull;
+        if (km > key) lo = mid + 1;
+        else hi = mid;
+    }
+    const int64_t id = ids[row + lo];
+    return id >= 0 && pack_key(scores[row + lo], uint32_t(id)) == key;
+}
+
+// UNION: drop a key that an earlier list already holds (one binary search per
+// earlier list), so an item found by several lists is merged once.
+template <bool UNION>
 __global__ void __launch_bounds__(kMergeBlock)
 merge_kernel(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
              int32_t* out_scores)
@@ -47,6 +66,9 @@ merge_kernel(const int64_t* ids, const int32_t* scores, int G, int B, int k, int
             if (id >= 0 && id < (int64_t(1) << 31)) {
                 key = pack_key(scores[src], uint32_t(id));
                 take = true;
+                if (UNION)
+                    for (int h = 0; h < g && take; ++h)
+                        take = !in_sorted_list(ids, scores, (int64_t(h) * B + b) * k, k, key);
             } else if (id != -1) {
                 atomicOr(&g_merge_err, kErrUnitDecode);
             }
@@ -68,17 +90,30 @@ merge_kernel(const int64_t* ids, const int32_t* scores, int G, int B, int k, int
     }
 }
 
-cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
-                         int32_t* out_scores, cudaStream_t s)
+template <bool UNION>
+static cudaError_t launch_merge_impl(const int64_t* ids, const int32_t* scores, int G, int B, int k,
+                                     int64_t* out_ids, int32_t* out_scores, cudaStream_t s)
 {
     const int pw = next_pow2(k);
     const int nkeys = G * k > pw ? G * k : pw;
     const size_t smem = (size_t((k + 1) & ~1) + kMergeTieCap + size_t(nkeys)) * 8;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_kernel), 14,
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_kernel<UNION>), UNION ? 15 : 14,
                                      int((size_t(ST_SMALL_K) + kMergeTieCap + ST_MERGE_MAX_KEYS) * 8));
     if (e != cudaSuccess) return e;
-    merge_kernel<<<B, kMergeBlock, smem, s>>>(ids, scores, G, B, k, out_ids, out_scores);
+    merge_kernel<UNION><<<B, kMergeBlock, smem, s>>>(ids, scores, G, B, k, out_ids, out_scores);
     return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
+                         int32_t* out_scores, cudaStream_t s)
+{
+    return launch_merge_impl<false>(ids, scores, G, B, k, out_ids, out_scores, s);
+}
+
+cudaError_t launch_merge_union(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
+                               int32_t* out_scores, cudaStream_t s)
+{
+    return launch_merge_impl<true>(ids, scores, G, B, k, out_ids, out_scores, s);
 }
 
 cudaError_t merge_error_word(uint32_t* word, bool clear)

@@ -241,6 +241,19 @@ st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B
 st_status st_merge_topk(const int64_t* ids, const int32_t* scores, int32_t G, int32_t B, int32_t k,
                         int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
 
+/*
+ * Exact top-k of the union of G result lists that may share items (the same
+ * item, with the same score, in several lists): like st_merge_topk, except
+ * that an item is kept once. Each list must be ordered as st_search orders
+ * its results (score descending, then id ascending, padding last) -- every
+ * st_search result is. This is the merge step of an OR of several masks per
+ * query (pass if any mask passes; a targeting rule allowing several values
+ * of a field): search once per mask, then take the union. Same arguments,
+ * limits and errors as st_merge_topk.
+ */
+st_status st_merge_topk_union(const int64_t* ids, const int32_t* scores, int32_t G, int32_t B, int32_t k,
+                              int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
+
 /* Wait for `stream`, then report and clear the merge error word of the
    current device: ST_OK, ST_ERR_DEVICE (an input id was out of range), or
    ST_ERR_CUDA. */
