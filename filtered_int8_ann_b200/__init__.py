@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libst.so")
 ST_PROBE_NOALLOC_SCRATCH_BYTES = 16 << 20
 ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY, ST_OPT_ID_OFFSET = 1, 2, 3
 ST_MERGE_MAX_KEYS = 16384
-ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K = 512, 262144, 4096, 4096
+ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K, ST_MAX_B = 512, 262144, 4096, 4096, 32768
 
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",

@@ -253,7 +253,7 @@ st_status check_search_args(const st_index* idx, int32_t B, int32_t nprobe, int3
 {
     if (idx == nullptr) return ST_ERR_INVALID_ARG;
     if (B < 1 || k < 1 || nprobe < 1 || nprobe > idx->nlist) return ST_ERR_INVALID_ARG;
-    if (k > ST_MAX_K || nprobe > ST_MAX_NPROBE) return ST_ERR_UNSUPPORTED;
+    if (k > ST_MAX_K || nprobe > ST_MAX_NPROBE || B > ST_MAX_B) return ST_ERR_UNSUPPORTED;
     if (int64_t(B) * nprobe >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
     return ST_OK;
 }

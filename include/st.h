@@ -59,6 +59,7 @@ typedef enum {
                                 needs device memory for the key of every row of the
                                 probed lists (ST_ERR_OOM when it does not fit) */
 #define ST_MAX_NPROBE 4096   /* 1 <= nprobe <= min(nlist, 4096) */
+#define ST_MAX_B 32768       /* 1 <= B <= 32768 queries per call */
 /* n < 2^31 items; sig_words is 1 (64-bit signatures) or 2 (128-bit). */
 
 /*
@@ -99,7 +100,7 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs,
  * streams may share one index. The index itself is never modified.
  *
  * Errors: INVALID_ARG (null or non-device pointer, B < 1, k < 1, nprobe < 1 or
- * nprobe > nlist), UNSUPPORTED (k or nprobe above the limits), OOM, CUDA.
+ * nprobe > nlist), UNSUPPORTED (B, k or nprobe above the limits), OOM, CUDA.
  * A kernel-side internal error is reported by st_index_check.
  */
 st_status st_search(const st_index* idx, const int8_t* queries, const uint64_t* qmasks,

@@ -198,6 +198,7 @@ def test_host_side_errors_with_device_buffers():
         assert call(P=0) == st.ST_ERR_INVALID_ARG
         assert call(P=9) == st.ST_ERR_INVALID_ARG          # nprobe > nlist
         assert call(k=st.ST_MAX_K + 1) == st.ST_ERR_UNSUPPORTED
+        assert call(B=st.ST_MAX_B + 1) == st.ST_ERR_UNSUPPORTED   # checked before any buffer is read
         host = torch.empty((4, 64), dtype=torch.int8)
         assert call(qp=host.data_ptr()) == st.ST_ERR_INVALID_ARG   # host pointer
         assert call(qp=q.data_ptr() + 1) == st.ST_ERR_INVALID_ARG  # misaligned
