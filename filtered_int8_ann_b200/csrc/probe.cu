@@ -2,9 +2,9 @@
 // accumulation and keep the query's nprobe best lists, best first (score
 // descending, lower list id first among equal scores).
 //
-// "Pick the most promising clusters first, filter only inside them, then score
-// only the survivors" -- SilverTorch: Index as Model, section on how each
-// component worked before. The pages name probes (64 of them with top-2048)
+// The most promising clusters are chosen first, the filter runs only inside
+// them, and only the items that pass are scored -- SilverTorch: Index as Model,
+// section on how each component worked before. The pages name probes (64 of them with top-2048)
 // but not the index type; this library reads it as an IVF with int8 centroids
 // and contiguous lists.
 //

@@ -2,7 +2,8 @@
 // them ordered by score descending, then item id ascending, padded with
 // (id -1, score INT32_MIN) when fewer than k items were eligible.
 //
-// "Top-2048 with 64 probes and no recall loss" / a large candidate pool --
+// A large result (2048 per query from 64 probes, with recall kept) drawn from a
+// large candidate pool --
 // SilverTorch: Index as Model, section on redesigning each stage as a pure
 // PyTorch module, fused Int8 ANN paragraph; maximum top-k row of the cost
 // efficiency table in the Spanish translation.

@@ -4,8 +4,8 @@
  *
  * What it computes. For each query b (an int8 vector q_b and a Bloom mask m_b):
  *   1. probe: score every IVF list c by the int32 inner product <q_b, cent_c>
- *      and keep the nprobe best lists ("pick the most promising clusters
- *      first" -- SilverTorch: Index as Model, section on how each component
+ *      and keep the nprobe best lists (the clusters judged best are chosen
+ *      first -- SilverTorch: Index as Model, section on how each component
  *      worked before);
  *   2. filter: inside the probed lists only, an item i is eligible when
  *      (sig_i[w] & m_b[w]) == m_b[w] for every signature word w (same page,
@@ -14,8 +14,8 @@
  *   3. score: eligible items only, by the int32 inner product <q_b, x_i> of
  *      int8 vectors (same section, fused Int8 ANN paragraph);
  *   4. top-k: the k best eligible items, ordered by score descending, then by
- *      item id ascending (large top-k: "no recall loss at 64 probes and
- *      top-2048", same paragraph; SilverTorch: Index as Model, Spanish
+ *      item id ascending (large top-k: 2048 results from 64 probes with
+ *      recall kept, same paragraph; SilverTorch: Index as Model, Spanish
  *      translation, table of compute cost efficiency, row on maximum top-k).
  *   Probe ties go to the lower list id. The item id is the row index in the
  *   arrays given to st_index_create. When fewer than k items are eligible, the

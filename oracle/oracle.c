@@ -10,20 +10,21 @@
  *
  *   For each query b, independently:
  *   1. cs[c] = sum_j q[b][j] * cent[c][j] in int32, for every list c.
- *      (Probe: "pick the most promising clusters first" -- SilverTorch: Index
- *      as Model, section on how each component worked before.)
+ *      (Probe: the most promising clusters are chosen first -- SilverTorch:
+ *      Index as Model, section on how each component worked before.)
  *   2. Order the pairs (cs[c], c) by score descending, then list id ascending;
  *      the first P list ids are the probed lists.
  *   3. For every item i of every probed list (rows off[c] .. off[c+1]-1), the
  *      item is eligible when (sig[i][w] & m[b][w]) == m[b][w] for all words w
- *      ("each item gets a compact signature when published; at serving time a
- *      simple bit operation checks it against the request" -- same page, Bloom
- *      index filter paragraph). Only eligible items are scored ("filter only
- *      inside those clusters, then score only the survivors").
+ *      (every item carries a compact signature written at publication time,
+ *      and one bit operation tests it against the request at serving time --
+ *      same page, Bloom index filter paragraph). Only eligible items are
+ *      scored: the filter runs inside the chosen clusters and only the items
+ *      that pass it are scored.
  *   4. Score = sum_j q[b][j] * x[i][j] in int32 (int8 storage, fused Int8 ANN
  *      paragraph). Order the candidates by score descending, then item id
  *      ascending, and output the first min(k, count); the remaining slots get
- *      id -1 and score INT32_MIN (large top-k: "top-2048 with 64 probes",
+ *      id -1 and score INT32_MIN (large top-k: 2048 results from 64 probes,
  *      same paragraph).
  *
  * Readings where the pages are silent: inner product for both the probe and
