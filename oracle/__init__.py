@@ -38,6 +38,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_search.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i32, i32, i32, i32,
                                   P, P, P, P, i32]
     lib.oracle_search.restype = i32
+    lib.oracle_search_ids.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, i32, i32, i32, i32,
+                                      P, P, P, P, i32]
+    lib.oracle_search_ids.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     return lib
@@ -72,9 +75,10 @@ def probe(q: np.ndarray, cent: np.ndarray, P: int, lib=None) -> np.ndarray:
 
 
 def search(items, sigs, offsets, centroids, queries, masks, nprobe, k, b0=0, b1=None,
-           nthreads=1, lib=None):
+           nthreads=1, lib=None, row_ids=None):
     """Search queries [b0, b1). Returns (ids int64 [nb,k], scores int32 [nb,k],
-    probe int32 [nb,P], eligible int64 [nb])."""
+    probe int32 [nb,P], eligible int64 [nb]). row_ids (int64 [n], optional)
+    gives the item id of each row; by default it is the row index."""
     lib = lib or load()
     items = np.ascontiguousarray(items, dtype=np.int8)
     sigs = np.ascontiguousarray(sigs).view(np.uint64)
@@ -96,9 +100,16 @@ def search(items, sigs, offsets, centroids, queries, masks, nprobe, k, b0=0, b1=
     scores = np.empty((nb, k), dtype=np.int32)
     probe_out = np.empty((nb, nprobe), dtype=np.int32)
     elig = np.empty(nb, dtype=np.int64)
-    rc = lib.oracle_search(_ptr(items), _ptr(sigs), _ptr(offsets), _ptr(centroids), n, d, nlist,
-                           W, _ptr(queries), _ptr(masks), b0, b1, nprobe, k, _ptr(ids),
-                           _ptr(scores), _ptr(probe_out), _ptr(elig), nthreads)
+    if row_ids is None:
+        rc = lib.oracle_search(_ptr(items), _ptr(sigs), _ptr(offsets), _ptr(centroids), n, d, nlist,
+                               W, _ptr(queries), _ptr(masks), b0, b1, nprobe, k, _ptr(ids),
+                               _ptr(scores), _ptr(probe_out), _ptr(elig), nthreads)
+    else:
+        row_ids = np.ascontiguousarray(row_ids, dtype=np.int64)
+        assert row_ids.shape == (n,)
+        rc = lib.oracle_search_ids(_ptr(items), _ptr(sigs), _ptr(offsets), _ptr(row_ids), _ptr(centroids), n,
+                                   d, nlist, W, _ptr(queries), _ptr(masks), b0, b1, nprobe, k, _ptr(ids),
+                                   _ptr(scores), _ptr(probe_out), _ptr(elig), nthreads)
     assert rc == 0, "oracle allocation failed"
     return ids, scores, probe_out, elig
 

@@ -29,7 +29,9 @@
  *
  * Readings where the pages are silent: inner product for both the probe and
  * the score; lower list id wins a probe tie; lower item id wins a score tie;
- * the item id is its row index; the Bloom test alone decides eligibility (no
+ * the item id is its row index unless the caller gives an id per row (an index
+ * that has taken insertions keeps each list's rows together here, and the ids
+ * say which items they are); the Bloom test alone decides eligibility (no
  * exact attribute re-check); short results are padded as above.
  *
  * Build: gcc -O2 -fopenmp -shared -fPIC oracle.c -o liboracle.so
@@ -88,9 +90,10 @@ int32_t oracle_probe(const int8_t* q, const int8_t* cent, int32_t nlist, int32_t
     return 0;
 }
 
-/* Steps 3-4 for one query over a given set of lists. */
+/* Steps 3-4 for one query over a given set of lists. Row i is item row_ids[i]
+ * (item i when row_ids is NULL). */
 static int32_t search_lists(const int8_t* items, const uint64_t* sigs, const int64_t* off,
-                            int32_t d, int32_t W, const int8_t* q, const uint64_t* m,
+                            const int64_t* row_ids, int32_t d, int32_t W, const int8_t* q, const uint64_t* m,
                             const int32_t* lists, int32_t P, int32_t k,
                             int64_t* out_ids, int32_t* out_scores, int64_t* out_count)
 {
@@ -104,7 +107,7 @@ static int32_t search_lists(const int8_t* items, const uint64_t* sigs, const int
         for (int64_t i = off[c]; i < off[c + 1]; ++i) {
             if (!oracle_bloom_pass(sigs + i * W, m, W)) continue;
             cand[n].score = oracle_dot(q, items + i * d, d);
-            cand[n].id = i;
+            cand[n].id = row_ids ? row_ids[i] : i;
             ++n;
         }
     }
@@ -125,17 +128,18 @@ static int32_t search_lists(const int8_t* items, const uint64_t* sigs, const int
 
 /*
  * The whole search for queries [b0, b1). Arrays are row-major:
- * items int8 [n][d], sigs uint64 [n][W], off int64 [nlist+1], cent int8
+ * items int8 [n][d], sigs uint64 [n][W], off int64 [nlist+1], row_ids int64
+ * [n] or NULL (item id of each row; NULL: the row index), cent int8
  * [nlist][d], queries int8 [B][d], masks uint64 [B][W]; outputs int64/int32
  * [B][k]; out_probe int32 [B][P] and out_eligible int64 [B] may be NULL.
  * nthreads > 1 runs queries in parallel (the result does not depend on it).
  * Returns 0, or -1 when an allocation failed.
  */
-int32_t oracle_search(const int8_t* items, const uint64_t* sigs, const int64_t* off,
-                      const int8_t* cent, int64_t n, int32_t d, int32_t nlist, int32_t W,
-                      const int8_t* queries, const uint64_t* masks, int32_t b0, int32_t b1,
-                      int32_t P, int32_t k, int64_t* out_ids, int32_t* out_scores,
-                      int32_t* out_probe, int64_t* out_eligible, int32_t nthreads)
+int32_t oracle_search_ids(const int8_t* items, const uint64_t* sigs, const int64_t* off,
+                          const int64_t* row_ids, const int8_t* cent, int64_t n, int32_t d, int32_t nlist,
+                          int32_t W, const int8_t* queries, const uint64_t* masks, int32_t b0, int32_t b1,
+                          int32_t P, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                          int32_t* out_probe, int64_t* out_eligible, int32_t nthreads)
 {
     (void)n;
     int32_t err = 0;
@@ -149,7 +153,7 @@ int32_t oracle_search(const int8_t* items, const uint64_t* sigs, const int64_t* 
         if (oracle_probe(q, cent, nlist, d, P, lists) != 0) { err |= 1; free(lists); continue; }
         if (out_probe) memcpy(out_probe + (int64_t)(b - b0) * P, lists, sizeof(int32_t) * (size_t)P);
         int64_t cnt = 0;
-        if (search_lists(items, sigs, off, d, W, q, m, lists, P, k,
+        if (search_lists(items, sigs, off, row_ids, d, W, q, m, lists, P, k,
                          out_ids + (int64_t)(b - b0) * k, out_scores + (int64_t)(b - b0) * k,
                          &cnt) != 0)
             err |= 1;
@@ -157,6 +161,17 @@ int32_t oracle_search(const int8_t* items, const uint64_t* sigs, const int64_t* 
         free(lists);
     }
     return err ? -1 : 0;
+}
+
+/* oracle_search_ids with every item id equal to its row index */
+int32_t oracle_search(const int8_t* items, const uint64_t* sigs, const int64_t* off,
+                      const int8_t* cent, int64_t n, int32_t d, int32_t nlist, int32_t W,
+                      const int8_t* queries, const uint64_t* masks, int32_t b0, int32_t b1,
+                      int32_t P, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                      int32_t* out_probe, int64_t* out_eligible, int32_t nthreads)
+{
+    return oracle_search_ids(items, sigs, off, NULL, cent, n, d, nlist, W, queries, masks, b0, b1, P, k,
+                             out_ids, out_scores, out_probe, out_eligible, nthreads);
 }
 
 int32_t oracle_max_threads(void)

@@ -35,7 +35,8 @@ def probe(q, cent, P):
     return o[:P].astype(np.int32)
 
 
-def search(items, sigs, offsets, centroids, queries, masks, nprobe, k):
+def search(items, sigs, offsets, centroids, queries, masks, nprobe, k, row_ids=None):
+    """row_ids (optional): the item id of each row; by default the row index."""
     B = queries.shape[0]
     ids = np.full((B, k), -1, dtype=np.int64)
     out = np.full((B, k), INT32_MIN, dtype=np.int32)
@@ -51,7 +52,8 @@ def search(items, sigs, offsets, centroids, queries, masks, nprobe, k):
         if rows.size == 0:
             continue
         s = scores(queries[b][None, :], items[rows])[0]
-        o = order_desc(s, rows)[:k]
-        ids[b, :o.size] = rows[o]
+        item = rows if row_ids is None else np.asarray(row_ids, dtype=np.int64)[rows]
+        o = order_desc(s, item)[:k]
+        ids[b, :o.size] = item[o]
         out[b, :o.size] = s[o]
     return ids, out, probes, elig

@@ -216,4 +216,55 @@ def pin_sub_batch(lib):
         assert np.array_equal(x[4:7], y)
 
 
+# --- explicit item ids per row (an index whose lists took insertions) -------------------
+def _permute_within_lists(a, rng):
+    """Rows of each list in a random order, with the original row index as the id."""
+    off = a["offsets"]
+    perm = np.concatenate([off[c] + rng.permutation(off[c + 1] - off[c]) for c in range(len(off) - 1)])
+    return a["items"][perm], a["sigs"][perm], perm.astype(np.int64)
+
+
+def pin_row_ids_permutation(lib):
+    """Reordering the rows inside each list, each keeping its item id, leaves
+    the result unchanged; repeated rows make every score tie, so only the ids
+    order them."""
+    rng = np.random.default_rng(61)
+    for c in (dict(n=1500, d=32, nlist=10, sig_bits=128, B=6, nprobe=4, k=120, seed=62),
+              dict(n=800, d=16, nlist=3, sig_bits=64, B=4, nprobe=2, k=900, seed=63)):
+        a = _arrays(small(**c))
+        P, k = c["nprobe"], c["k"]
+        exp = oracle.search(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"], a["masks"], P, k,
+                            lib=lib)
+        items, sigs, ids = _permute_within_lists(a, rng)
+        got = oracle.search(items, sigs, a["offsets"], a["centroids"], a["queries"], a["masks"], P, k, lib=lib,
+                            row_ids=ids)
+        for g, e in zip(got, exp):
+            assert np.array_equal(g, e), c
+    # all scores equal: the order is the ids' order
+    n, d = 300, 16
+    x = np.tile(rng.integers(-128, 128, d, dtype=np.int8), (n, 1))
+    q = rng.integers(-128, 128, (1, d), dtype=np.int8)
+    off, cen = _one_list(n, d)
+    ids = rng.permutation(np.arange(1000, 1000 + 3 * n, 3)).astype(np.int64)
+    got_ids, got_sc, _, el = oracle.search(x, np.zeros((n, 1), np.uint64), off, cen, q, np.zeros((1, 1), np.uint64),
+                                           1, 50, lib=lib, row_ids=ids)
+    assert list(got_ids[0]) == list(range(1000, 1150, 3)) and el[0] == n
+
+
+def pin_row_ids_bruteforce(lib):
+    rng = np.random.default_rng(64)
+    for c in (dict(n=1200, d=32, nlist=8, sig_bits=128, hash_bits=3, B=5, nprobe=3, k=80, seed=65),
+              dict(n=600, d=16, nlist=1, sig_bits=64, B=4, nprobe=1, k=700, seed=66, uniform_items=True)):
+        a = _arrays(small(**c))
+        n = a["items"].shape[0]
+        ids = rng.choice(20 * n, n, replace=False).astype(np.int64)
+        P, k = c["nprobe"], c["k"]
+        got = oracle.search(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"], a["masks"], P, k,
+                            lib=lib, row_ids=ids)
+        exp = bruteforce.search(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"], a["masks"],
+                                P, k, row_ids=ids)
+        for g, e, what in zip(got, exp, ("ids", "scores", "probe", "eligible")):
+            assert np.array_equal(g, e), (c, what)
+
+
 PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

@@ -33,6 +33,7 @@ MUTANTS = {
     "pad_id_zero": ("out_ids[r] = -1;", "out_ids[r] = 0;"),
     "pad_score_zero": ("out_scores[r] = INT32_MIN;", "out_scores[r] = 0;"),
     "filter_after_topk": ("if (!oracle_bloom_pass(sigs + i * W, m, W)) continue;", ""),
+    "row_ids_ignored": ("cand[n].id = row_ids ? row_ids[i] : i;", "cand[n].id = i;"),
 }
 
 
