@@ -12,6 +12,7 @@ import ctypes
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -20,14 +21,15 @@ LIB_PATH = os.path.join(_HERE, "libst.so")
 (ST_OK, ST_ERR_INVALID_ARG, ST_ERR_UNSUPPORTED, ST_ERR_OOM, ST_ERR_CUDA, ST_ERR_DEVICE,
  ST_ERR_SCRATCH_LIMIT) = range(7)
 ST_PROBE_NOALLOC_SCRATCH_BYTES = 16 << 20
-ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY, ST_OPT_ID_OFFSET = 1, 2, 3
+ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY, ST_OPT_ID_OFFSET, ST_OPT_INSERT_RESERVE = 1, 2, 3, 4
+ST_INSERT_CHUNK = 512
 ST_MERGE_MAX_KEYS = 16384
 ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K, ST_MAX_B = 512, 262144, 4096, 4096, 32768
 
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
            "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
-           "st_index_delete", "st_merge_topk_union", "st_index_destroy", "st_status_string")
+           "st_index_delete", "st_merge_topk_union", "st_index_insert", "st_index_destroy", "st_status_string")
 
 
 class StError(RuntimeError):
@@ -64,9 +66,10 @@ def lib() -> ctypes.CDLL:
     L.st_index_update.argtypes = [P, P, P, P, i64, P]
     L.st_index_delete.argtypes = [P, P, i64, P]
     L.st_merge_topk_union.argtypes = [P, P, i32, i32, i32, P, P, P]
+    L.st_index_insert.argtypes = [P, P, P, P, i64, P, P]
     for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
               "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
-              "st_index_delete", "st_merge_topk_union"):
+              "st_index_delete", "st_merge_topk_union", "st_index_insert"):
         getattr(L, f).restype = ctypes.c_int
     L.st_index_destroy.argtypes = [P]
     L.st_index_destroy.restype = None
@@ -265,8 +268,26 @@ class Index:
                         stream=stream, **kw)
         return st_merge_topk_union(ids, sc, stream=stream)
 
+    def insert(self, lists, items, sigs, stream=None):
+        """Insert new items: lists (host, one list id per item), items int8 [m, d]
+        and sigs [m, W] (device tensors). Returns the ids given to them (numpy
+        int64 [m]); waits for the stream."""
+        lists = np.ascontiguousarray(np.asarray(lists, dtype=np.int32).reshape(-1))
+        m = lists.shape[0]
+        out = np.empty(m, dtype=np.int64)
+        if m:
+            items = items.contiguous()
+            sigs = _as_words(sigs).contiguous()
+            if items.shape[0] != m or sigs.shape[0] != m:
+                raise ValueError("lists, items and sigs must have the same number of rows")
+        _check(lib().st_index_insert(self.handle, lists.ctypes.data_as(ctypes.c_void_p) if m else None,
+                                     _ptr(items) if m else None, _ptr(sigs) if m else None, m,
+                                     out.ctypes.data_as(ctypes.c_void_p) if m else None, _stream(stream)),
+               "st_index_insert")
+        return out
+
     def delete(self, ids, stream=None):
-        """Delete items in place (device int64 row indices)."""
+        """Delete items in place (device int64 item ids)."""
         _check(lib().st_index_delete(self.handle, _ptr(ids), int(ids.numel()), _stream(stream)), "st_index_delete")
 
     def probe_noalloc(self, queries, nprobe, out_probe, stream=None):

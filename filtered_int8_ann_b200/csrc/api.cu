@@ -16,26 +16,40 @@ cudaError_t launch_merge_union(const int64_t* ids, const int32_t* scores, int G,
 }  // namespace st
 
 
+// Rows: [0, n) the creation lists (list c: offsets[c] .. offsets[c+1]-1), then
+// append chunks of kWarpItems rows, chunk a at rows n + kWarpItems * a, each
+// owned by one list and filled in order. An item's id is its row.
 struct st_index {
     int device = 0;
     int num_sms = 0;
-    int64_t n = 0;
+    int64_t n = 0;                   // creation rows
     int32_t d = 0, nlist = 0, W = 0;
-    int8_t* items = nullptr;
-    uint64_t* sigs = nullptr;
-    int64_t* offsets = nullptr;
-    int32_t* chunk_start = nullptr;  // [nlist+1] first warp-unit chunk of each list
-    int32_t* chunk_list = nullptr;   // [n_chunks] list of each chunk
-    int32_t n_chunks = 0;
-    uint32_t* planes = nullptr;      // [n_chunks][64W][16] signature bit-planes
+    int8_t* items = nullptr;         // [rows_alloc][d]
+    uint64_t* sigs = nullptr;        // [rows_alloc][W]
+    int64_t rows_alloc = 0;          // n + kWarpItems * app_cap
+    int64_t* offsets = nullptr;      // [nlist+1] creation lists
+    int32_t* base_chunk_start = nullptr;  // [nlist+1] first creation chunk (plane block) of each list
+    int32_t* chunk_list = nullptr;   // [n_base_chunks] list of each creation chunk
+    int32_t n_base_chunks = 0;
+    uint32_t* planes = nullptr;      // [n_base_chunks + app_cap][64W][16] signature bit-planes
+    int4* chunk_desc = nullptr;      // [desc_cap] chunk table, list by list: {first row, plane block, rows, list}
+    int32_t* chunk_start = nullptr;  // [nlist+1] first chunk table entry of each list
+    int32_t n_desc = 0, desc_cap = 0;
+    int32_t* app_len = nullptr;      // [app_cap] rows filled in each append chunk
+    int32_t app_used = 0, app_cap = 0;
+    std::vector<int64_t> off_host;                // creation offsets
+    std::vector<int32_t> base_cstart_host;        // creation chunk starts
+    std::vector<std::vector<int32_t>> list_app;   // append chunks of each list, in fill order
+    std::vector<int32_t> app_len_host;            // [app_used]
     int8_t* centroids = nullptr;
     uint32_t* err = nullptr;
     std::vector<int64_t> top_prefix;  // [p] = rows in the p largest lists
+    std::vector<int64_t> top_chunks;  // [p] = chunk table entries of the p lists with the most
     cudaMemPool_t pool = nullptr;
     int64_t cand_bytes = int64_t(2) << 30;
     int64_t cand_cap_override = 0;
     int64_t id_offset = 0;
-    uint32_t* dead = nullptr;        // [ceil(n / 32)] deletion bitmap, allocated at the first deletion
+    uint32_t* dead = nullptr;        // [ceil(rows_alloc / 32)] deletion bitmap, allocated at the first deletion
 };
 
 namespace st {
@@ -99,6 +113,158 @@ st_status cuda_status(cudaError_t e)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+constexpr int64_t kIdLimit = int64_t(1) << 31;  // ids (with the offset) stay below this
+
+size_t plane_block_bytes(int W) { return size_t(64) * W * 16 * 4; }
+
+st::RowMap row_map(const st_index* idx)
+{
+    st::RowMap m;
+    m.offsets = idx->offsets;
+    m.base_chunk_start = idx->base_chunk_start;
+    m.nlist = idx->nlist;
+    m.n = idx->n;
+    m.n_base_chunks = idx->n_base_chunks;
+    m.app_len = idx->app_len;
+    m.n_app = idx->app_used;
+    return m;
+}
+
+// The chunk table (list by list: creation chunks, then append chunks in fill
+// order), each list's first entry, and the two size prefixes the search sizes
+// its scratch with.
+struct Tables {
+    std::vector<int4> desc;
+    std::vector<int32_t> start;
+    std::vector<int64_t> top_prefix, top_chunks;
+};
+
+Tables build_tables(const st_index* idx, const std::vector<std::vector<int32_t>>& list_app,
+                    const std::vector<int32_t>& app_len)
+{
+    Tables t;
+    const int32_t nl = idx->nlist;
+    const int64_t Wi = st::kWarpItems;
+    t.start.assign(size_t(nl) + 1, 0);
+    std::vector<int64_t> rows(nl), chunks(nl);
+    for (int32_t c = 0; c < nl; ++c) {
+        t.start[c] = int32_t(t.desc.size());
+        const int64_t o0 = idx->off_host[c], nc = idx->off_host[c + 1] - o0;
+        int64_t r = nc;
+        for (int64_t j = 0; j * Wi < nc; ++j)
+            t.desc.push_back(make_int4(int(o0 + j * Wi), idx->base_cstart_host[c] + int(j), int(std::min(Wi, nc - j * Wi)), c));
+        for (int32_t a : list_app[c]) {
+            t.desc.push_back(make_int4(int(idx->n + Wi * a), idx->n_base_chunks + a, app_len[a], c));
+            r += app_len[a];
+        }
+        rows[c] = r;
+        chunks[c] = int64_t(t.desc.size()) - t.start[c];
+    }
+    t.start[nl] = int32_t(t.desc.size());
+    std::sort(rows.begin(), rows.end(), std::greater<int64_t>());
+    std::sort(chunks.begin(), chunks.end(), std::greater<int64_t>());
+    t.top_prefix.assign(size_t(nl) + 1, 0);
+    t.top_chunks.assign(size_t(nl) + 1, 0);
+    for (int32_t c = 0; c < nl; ++c) {
+        t.top_prefix[c + 1] = t.top_prefix[c] + rows[c];
+        t.top_chunks[c + 1] = t.top_chunks[c] + chunks[c];
+    }
+    return t;
+}
+
+// Copy the chunk table to the device (a larger array when it outgrew the old
+// one: the device is drained first, since earlier searches may still read it).
+cudaError_t upload_tables(st_index* idx, const Tables& t, cudaStream_t stream)
+{
+    const int32_t nd = int32_t(t.desc.size());
+    if (nd > idx->desc_cap || idx->chunk_desc == nullptr) {
+        const int32_t cap = std::max<int32_t>(std::max<int32_t>(nd, 1), idx->desc_cap + idx->desc_cap / 2);
+        int4* fresh = nullptr;
+        cudaError_t e = cudaMalloc(&fresh, size_t(cap) * sizeof(int4));
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) {
+            cudaFree(fresh);
+            return e;
+        }
+        cudaFree(idx->chunk_desc);
+        idx->chunk_desc = fresh;
+        idx->desc_cap = cap;
+    }
+    cudaError_t e = cudaSuccess;
+    if (nd > 0) e = cudaMemcpyAsync(idx->chunk_desc, t.desc.data(), size_t(nd) * sizeof(int4), cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(idx->chunk_start, t.start.data(), t.start.size() * 4, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // the host vectors may go after this
+    if (e == cudaSuccess) {
+        idx->n_desc = nd;
+        idx->top_prefix = t.top_prefix;
+        idx->top_chunks = t.top_chunks;
+    }
+    return e;
+}
+
+// Room for app_cap append chunks: new item, signature, plane, fill-count and
+// deletion arrays, the old contents copied in, the rest zeroed. All or nothing.
+st_status grow_rows(st_index* idx, int32_t app_cap, cudaStream_t stream)
+{
+    if (app_cap <= idx->app_cap) return ST_OK;
+    const int64_t rows = idx->n + int64_t(st::kWarpItems) * app_cap;
+    if (rows + idx->id_offset >= kIdLimit) return ST_ERR_UNSUPPORTED;
+    const int64_t old_rows = idx->rows_alloc;
+    const size_t pb = plane_block_bytes(idx->W);
+    const size_t old_planes = size_t(idx->n_base_chunks + idx->app_cap) * pb;
+    const size_t new_planes = size_t(idx->n_base_chunks + app_cap) * pb;
+    const size_t old_words = size_t((old_rows + 31) / 32), new_words = size_t((rows + 31) / 32);
+    int8_t* items = nullptr;
+    uint64_t* sigs = nullptr;
+    uint32_t* planes = nullptr;
+    int32_t* app_len = nullptr;
+    uint32_t* dead = nullptr;
+    auto release = [&]() {
+        cudaFree(items);
+        cudaFree(sigs);
+        cudaFree(planes);
+        cudaFree(app_len);
+        cudaFree(dead);
+        cudaGetLastError();
+    };
+    if (cudaMalloc(&items, size_t(rows) * idx->d + 256) != cudaSuccess ||
+        cudaMalloc(&sigs, size_t(rows) * idx->W * 8 + 256) != cudaSuccess ||
+        cudaMalloc(&planes, new_planes) != cudaSuccess ||
+        cudaMalloc(&app_len, size_t(app_cap) * 4) != cudaSuccess ||
+        (idx->dead && cudaMalloc(&dead, new_words * 4) != cudaSuccess)) {
+        release();
+        return ST_ERR_OOM;
+    }
+    cudaError_t e = cudaMemcpyAsync(items, idx->items, size_t(old_rows) * idx->d, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sigs, idx->sigs, size_t(old_rows) * idx->W * 8, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(planes, idx->planes, old_planes, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(reinterpret_cast<char*>(planes) + old_planes, 0, new_planes - old_planes, stream);
+    if (e == cudaSuccess && idx->app_cap > 0)
+        e = cudaMemcpyAsync(app_len, idx->app_len, size_t(idx->app_cap) * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(app_len + idx->app_cap, 0, size_t(app_cap - idx->app_cap) * 4, stream);
+    if (e == cudaSuccess && dead) {
+        e = cudaMemcpyAsync(dead, idx->dead, old_words * 4, cudaMemcpyDeviceToDevice, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dead + old_words, 0, (new_words - old_words) * 4, stream);
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();  // also drains searches on other streams
+    if (e != cudaSuccess) {
+        release();
+        return ST_ERR_CUDA;
+    }
+    std::swap(items, idx->items);
+    std::swap(sigs, idx->sigs);
+    std::swap(planes, idx->planes);
+    std::swap(app_len, idx->app_len);
+    if (dead) std::swap(dead, idx->dead);
+    release();  // the old arrays
+    idx->app_cap = app_cap;
+    idx->rows_alloc = rows;
+    return ST_OK;
+}
+
 // Carves one scratch allocation into the per-search arrays. The arrays that
 // must start at zero come first, so one memset clears them.
 struct ScratchLayout {
@@ -133,15 +299,15 @@ int64_t candidate_capacity(const st_index* idx, int32_t B, int32_t P, int32_t k)
     return (cap + 31) / 32 * 32;  // keeps every query's buffer 256-byte aligned
 }
 
+// Units = sum over probed lists of chunks(list) x query groups(list): at most
+// every chunk for every group, and at most each query's P lists with the most
+// chunks for each query.
 int64_t max_units_bound(const st_index* idx, int32_t B, int32_t P)
 {
-    const int64_t W = st::kWarpItems;
     const int64_t groups = (B + st::kQMax - 1) / st::kQMax;
-    const int64_t lists = std::min<int64_t>(idx->nlist, int64_t(B) * P);
-    const int64_t b1 = ((idx->n + W - 1) / W + lists) * groups;
-    const int64_t topP = idx->top_prefix[std::min<int64_t>(P, idx->nlist)];
-    const int64_t b2 = int64_t(B) * ((topP + W - 1) / W + P);
-    return std::min(b1, b2);
+    const int64_t b1 = int64_t(idx->n_desc) * groups;
+    const int64_t b2 = int64_t(B) * idx->top_chunks[std::min<int64_t>(P, idx->nlist)];
+    return std::max<int64_t>(1, std::min(b1, b2));
 }
 
 st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
@@ -188,10 +354,11 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.items = idx->items;
     a.sigs = idx->sigs;
     a.planes = idx->planes;
-    a.offsets = idx->offsets;
+    a.chunk_desc = idx->chunk_desc;
     a.chunk_start = idx->chunk_start;
-    a.chunk_list = idx->chunk_list;
-    a.n_chunks = idx->n_chunks;
+    a.n_chunks = idx->n_desc;
+    a.n_plane_chunks = idx->n_base_chunks + idx->app_cap;
+    a.n_rows = idx->rows_alloc;
     a.centroids = idx->centroids;
     a.d = idx->d;
     a.nlist = idx->nlist;
@@ -311,14 +478,9 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         return fail(ST_ERR_INVALID_ARG);
     }
     if (off[0] != 0 || off[nlist] != n) return fail(ST_ERR_INVALID_ARG);
-    std::vector<int64_t> sizes(nlist);
-    for (int32_t c = 0; c < nlist; ++c) {
+    for (int32_t c = 0; c < nlist; ++c)
         if (off[c + 1] < off[c]) return fail(ST_ERR_INVALID_ARG);
-        sizes[c] = off[c + 1] - off[c];
-    }
-    std::sort(sizes.begin(), sizes.end(), std::greater<int64_t>());
-    idx->top_prefix.assign(size_t(nlist) + 1, 0);
-    for (int32_t c = 0; c < nlist; ++c) idx->top_prefix[c + 1] = idx->top_prefix[c] + sizes[c];
+    idx->rows_alloc = n;
 
     // library-owned copies (a little slack past the end of the row arrays)
     const size_t items_bytes = size_t(n) * d, sig_bytes = size_t(n) * sig_words * 8;
@@ -326,6 +488,7 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         cudaMalloc(&idx->sigs, sig_bytes + 256) != cudaSuccess ||
         cudaMalloc(&idx->offsets, off.size() * 8) != cudaSuccess ||
         cudaMalloc(&idx->centroids, size_t(nlist) * d + 256) != cudaSuccess ||
+        cudaMalloc(&idx->base_chunk_start, size_t(nlist + 1) * 4) != cudaSuccess ||
         cudaMalloc(&idx->chunk_start, size_t(nlist + 1) * 4) != cudaSuccess ||
         cudaMalloc(&idx->err, 256) != cudaSuccess) {
         cudaGetLastError();
@@ -337,34 +500,41 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         e = cudaMemcpyAsync(idx->offsets, off.data(), off.size() * 8, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(idx->centroids, centroids, size_t(nlist) * d, cudaMemcpyDefault, stream);
-    // static chunk table: list c owns chunks chunk_start[c] .. chunk_start[c+1]-1
+    // creation chunks: list c owns plane blocks cstart[c] .. cstart[c+1]-1
     std::vector<int32_t> cstart(size_t(nlist) + 1, 0);
     for (int32_t c = 0; c < nlist; ++c)
         cstart[c + 1] = cstart[c] + int32_t((off[c + 1] - off[c] + st::kWarpItems - 1) / st::kWarpItems);
-    idx->n_chunks = cstart[nlist];
-    std::vector<int32_t> clist(size_t(idx->n_chunks > 0 ? idx->n_chunks : 1), 0);
+    idx->n_base_chunks = cstart[nlist];
+    std::vector<int32_t> clist(size_t(idx->n_base_chunks > 0 ? idx->n_base_chunks : 1), 0);
     for (int32_t c = 0; c < nlist; ++c)
         for (int32_t t = cstart[c]; t < cstart[c + 1]; ++t) clist[t] = c;
     if (cudaMalloc(&idx->chunk_list, clist.size() * 4) != cudaSuccess) {
         cudaGetLastError();
         return fail(ST_ERR_OOM);
     }
-    if (e == cudaSuccess) e = cudaMemcpyAsync(idx->chunk_start, cstart.data(), cstart.size() * 4, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(idx->base_chunk_start, cstart.data(), cstart.size() * 4, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) e = cudaMemcpyAsync(idx->chunk_list, clist.data(), clist.size() * 4, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) {
-        const size_t pbytes = size_t(idx->n_chunks > 0 ? idx->n_chunks : 1) * 64 * sig_words * 16 * 4;
+        const size_t pbytes = size_t(idx->n_base_chunks > 0 ? idx->n_base_chunks : 1) * plane_block_bytes(sig_words);
         if (cudaMalloc(&idx->planes, pbytes) != cudaSuccess) {
             cudaGetLastError();
             return fail(ST_ERR_OOM);
         }
-        e = st::launch_build_planes(idx->sigs, idx->offsets, idx->chunk_start, idx->chunk_list, idx->n_chunks,
-                                    sig_words, idx->planes, stream);
+        e = st::launch_build_planes(idx->sigs, idx->offsets, idx->base_chunk_start, idx->chunk_list,
+                                    idx->n_base_chunks, sig_words, idx->planes, stream);
     }
+    idx->off_host = off;
+    idx->base_cstart_host = cstart;
+    idx->list_app.assign(size_t(nlist), std::vector<int32_t>());
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess) e = upload_tables(idx, build_tables(idx, idx->list_app, idx->app_len_host), stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(idx->err, 0, 256, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) {
         cudaGetLastError();
-        return fail(e == cudaErrorInvalidValue ? ST_ERR_INVALID_ARG : ST_ERR_CUDA);
+        return fail(e == cudaErrorInvalidValue ? ST_ERR_INVALID_ARG
+                    : e == cudaErrorMemoryAllocation ? ST_ERR_OOM : ST_ERR_CUDA);
     }
 
     cudaMemPoolProps props;
@@ -528,9 +698,8 @@ st_status st_index_update(st_index* idx, const int64_t* ids, const int8_t* items
     if (!is_device_ptr(ids, idx->device) || !aligned(ids, 8)) return ST_ERR_INVALID_ARG;
     if (items && (!is_device_ptr(items, idx->device) || !aligned(items, 16))) return ST_ERR_INVALID_ARG;
     if (sigs && (!is_device_ptr(sigs, idx->device) || !aligned(sigs, 8))) return ST_ERR_INVALID_ARG;
-    return cuda_status(st::launch_update(idx->items, idx->sigs, idx->planes, idx->offsets, idx->chunk_start,
-                                         idx->nlist, idx->n, idx->d, idx->W, ids, items, sigs, m, idx->err,
-                                         stream));
+    return cuda_status(st::launch_update(idx->items, idx->sigs, idx->planes, row_map(idx), idx->d, idx->W, ids,
+                                         items, sigs, m, idx->err, stream));
 }
 
 st_status st_index_delete(st_index* idx, const int64_t* ids, int64_t m, cudaStream_t stream)
@@ -540,7 +709,7 @@ st_status st_index_delete(st_index* idx, const int64_t* ids, int64_t m, cudaStre
     DeviceGuard g(idx->device);
     if (!is_device_ptr(ids, idx->device) || !aligned(ids, 8)) return ST_ERR_INVALID_ARG;
     if (idx->dead == nullptr) {
-        const size_t bytes = size_t((idx->n + 31) / 32) * 4;
+        const size_t bytes = size_t((idx->rows_alloc + 31) / 32) * 4;
         if (cudaMalloc(&idx->dead, bytes) != cudaSuccess) {
             cudaGetLastError();
             idx->dead = nullptr;
@@ -548,7 +717,7 @@ st_status st_index_delete(st_index* idx, const int64_t* ids, int64_t m, cudaStre
         }
         if (cudaMemsetAsync(idx->dead, 0, bytes, stream) != cudaSuccess) return ST_ERR_CUDA;
     }
-    return cuda_status(st::launch_delete(idx->dead, idx->n, ids, m, idx->err, stream));
+    return cuda_status(st::launch_delete(idx->dead, row_map(idx), ids, m, idx->err, stream));
 }
 
 st_status st_index_check(const st_index* idx, cudaStream_t stream)
@@ -577,11 +746,92 @@ st_status st_index_set_option(st_index* idx, st_option opt, int64_t value)
         idx->cand_cap_override = value;
         return ST_OK;
     case ST_OPT_ID_OFFSET:
-        if (value + idx->n >= (int64_t(1) << 31)) return ST_ERR_UNSUPPORTED;
+        if (value >= kIdLimit || value + idx->rows_alloc >= kIdLimit) return ST_ERR_UNSUPPORTED;
         idx->id_offset = value;
         return ST_OK;
+    case ST_OPT_INSERT_RESERVE: {
+        if (value == 0) return ST_OK;
+        const int64_t chunks = (value + st::kWarpItems - 1) / st::kWarpItems;
+        if (idx->n + (idx->app_used + chunks) * st::kWarpItems + idx->id_offset >= kIdLimit) return ST_ERR_UNSUPPORTED;
+        DeviceGuard g(idx->device);
+        return grow_rows(idx, int32_t(idx->app_used + chunks), nullptr);
+    }
     }
     return ST_ERR_INVALID_ARG;
+}
+
+st_status st_index_insert(st_index* idx, const int32_t* lists, const int8_t* items, const uint64_t* sigs,
+                          int64_t m, int64_t* out_ids, cudaStream_t stream)
+{
+    if (idx == nullptr || m < 0) return ST_ERR_INVALID_ARG;
+    if (m == 0) return ST_OK;
+    if (lists == nullptr || out_ids == nullptr) return ST_ERR_INVALID_ARG;
+    DeviceGuard g(idx->device);
+    if (!is_device_ptr(items, idx->device) || !aligned(items, 16) || !is_device_ptr(sigs, idx->device) ||
+        !aligned(sigs, 8))
+        return ST_ERR_INVALID_ARG;
+    for (int64_t j = 0; j < m; ++j)
+        if (lists[j] < 0 || lists[j] >= idx->nlist) return ST_ERR_INVALID_ARG;
+    if (m >= kIdLimit) return ST_ERR_UNSUPPORTED;
+
+    // place the items on the host: each fills its list's last append chunk,
+    // then a fresh chunk
+    std::vector<std::vector<int32_t>> list_app = idx->list_app;
+    std::vector<int32_t> app_len = idx->app_len_host;
+    std::vector<int64_t> ids(static_cast<size_t>(m));
+    int64_t used = idx->app_used;
+    for (int64_t j = 0; j < m; ++j) {
+        std::vector<int32_t>& own = list_app[lists[j]];
+        if (own.empty() || app_len[own.back()] == st::kWarpItems) {
+            if (idx->n + (used + 1) * st::kWarpItems + idx->id_offset >= kIdLimit) return ST_ERR_UNSUPPORTED;
+            own.push_back(int32_t(used));
+            app_len.push_back(0);
+            ++used;
+        }
+        const int32_t a = own.back();
+        ids[j] = idx->n + int64_t(st::kWarpItems) * a + app_len[a];
+        ++app_len[a];
+    }
+    if (used > idx->app_cap) {
+        // at least double the append room, within the id limit
+        int64_t cap = std::max<int64_t>(used, 2 * int64_t(idx->app_cap));
+        const int64_t cap_max = (kIdLimit - 1 - idx->id_offset - idx->n) / st::kWarpItems;
+        cap = std::min(cap, cap_max);
+        const st_status gs = grow_rows(idx, int32_t(cap), stream);
+        if (gs != ST_OK) return gs;
+    }
+    const Tables t = build_tables(idx, list_app, app_len);
+
+    int64_t* dids = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&dids), size_t(m) * 8, idx->pool, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e == cudaErrorMemoryAllocation ? ST_ERR_OOM : ST_ERR_CUDA;
+    }
+    e = cudaMemcpyAsync(dids, ids.data(), size_t(m) * 8, cudaMemcpyHostToDevice, stream);
+    // the fill counts cover the new rows before the rows are written
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(idx->app_len, app_len.data(), app_len.size() * 4, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) {
+        st::RowMap map = row_map(idx);
+        map.n_app = int32_t(used);
+        e = st::launch_update(idx->items, idx->sigs, idx->planes, map, idx->d, idx->W, dids, items, sigs, m, idx->err,
+                              stream);
+    }
+    // the chunk table last: searches enqueued after this call see the new rows
+    if (e == cudaSuccess) e = upload_tables(idx, t, stream);
+    cudaError_t ef = cudaFreeAsync(dids, stream);
+    if (e == cudaSuccess) e = ef;
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e == cudaErrorMemoryAllocation ? ST_ERR_OOM : ST_ERR_CUDA;
+    }
+    idx->list_app = std::move(list_app);
+    idx->app_len_host = std::move(app_len);
+    idx->app_used = int32_t(used);
+    std::memcpy(out_ids, ids.data(), size_t(m) * 8);
+    return ST_OK;
 }
 
 void st_index_destroy(st_index* idx)
@@ -595,6 +845,9 @@ void st_index_destroy(st_index* idx)
         cudaFree(idx->offsets);
         cudaFree(idx->centroids);
         cudaFree(idx->chunk_start);
+        cudaFree(idx->base_chunk_start);
+        cudaFree(idx->chunk_desc);
+        cudaFree(idx->app_len);
         cudaFree(idx->chunk_list);
         cudaFree(idx->planes);
         cudaFree(idx->err);

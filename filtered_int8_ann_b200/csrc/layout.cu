@@ -13,6 +13,12 @@
 // chunk (rows past the end of the list are zero). A scan unit then fetches only
 // the planes of the bits its queries' masks use, and tests 32 items with one
 // 32-bit AND per mask bit.
+//
+// Inserted items go to append chunks: blocks of kWarpItems rows after all the
+// creation rows, each owned by one list and filled in order; their planes
+// follow the creation chunks' planes. The search walks a list chunk by chunk
+// through a descriptor table, so a list's creation rows and append chunks need
+// not be adjacent.
 #include "st_internal.cuh"
 
 namespace st {
@@ -49,21 +55,48 @@ build_planes_kernel(const uint64_t* __restrict__ sigs, const int64_t* __restrict
     }
 }
 
-// In-place update of m rows: one warp per updated row copies the new row
-// and signature and rewrites the row's bit in each of its chunk's planes
+// The plane block of item `id` and its row within the block; false for an id
+// the index never handed out.
+__device__ __forceinline__ bool locate_row(const RowMap& map, int64_t id, int64_t& block, int& r)
+{
+    if (id < 0) return false;
+    if (id < map.n) {
+        // the row's list: the last c with offsets[c] <= id (empty lists share offsets)
+        int lo = 0, hi = map.nlist - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (map.offsets[mid] <= id) lo = mid;
+            else hi = mid - 1;
+        }
+        const int64_t rr = id - map.offsets[lo];
+        block = map.base_chunk_start[lo] + rr / kWarpItems;
+        r = int(rr % kWarpItems);
+        return true;
+    }
+    const int64_t a = (id - map.n) / kWarpItems;
+    if (a >= map.n_app) return false;
+    r = int((id - map.n) % kWarpItems);
+    if (r >= map.app_len[a]) return false;
+    block = map.n_base_chunks + a;
+    return true;
+}
+
+// In-place update (and insertion) of m rows: one warp per row copies the new
+// row and signature and rewrites the row's bit in each of its chunk's planes
 // (atomically: other rows of the same plane words may change at the same time).
 template <int W>
 __global__ void __launch_bounds__(256)
-update_kernel(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets, const int32_t* chunk_start,
-              int32_t nlist, int64_t n, int d, const int64_t* ids, const int8_t* new_items,
-              const uint64_t* new_sigs, int64_t m, uint32_t* err)
+update_kernel(int8_t* items, uint64_t* sigs, uint32_t* planes, RowMap map, int d, const int64_t* ids,
+              const int8_t* new_items, const uint64_t* new_sigs, int64_t m, uint32_t* err)
 {
     constexpr int NPL = 64 * W;
     const int lane = threadIdx.x & 31;
     const int64_t j = (int64_t(blockIdx.x) * 256 + threadIdx.x) >> 5;
     if (j >= m) return;
     const int64_t id = ids[j];
-    if (id < 0 || id >= n) {
+    int64_t t = 0;
+    int r = 0;
+    if (!locate_row(map, id, t, r)) {
         if (lane == 0) atomicOr(err, kErrUpdateId);
         return;
     }
@@ -71,16 +104,7 @@ update_kernel(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* of
         for (int p = lane; p < d / 16; p += 32)
             reinterpret_cast<int4*>(items + id * d)[p] = reinterpret_cast<const int4*>(new_items + j * d)[p];
     if (!new_sigs) return;
-    // the row's list: the last c with offsets[c] <= id (empty lists share offsets)
-    int lo = 0, hi = nlist - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (offsets[mid] <= id) lo = mid;
-        else hi = mid - 1;
-    }
-    const int64_t r = id - offsets[lo];
-    const int64_t t = chunk_start[lo] + r / kWarpItems;
-    const int w = int((r % kWarpItems) >> 5);
+    const int w = r >> 5;
     const uint32_t bit = 1u << (r & 31);
     uint64_t s0 = new_sigs[j * W], s1 = W > 1 ? new_sigs[j * W + 1] : 0ull;
     if (lane == 0) {
@@ -97,37 +121,40 @@ update_kernel(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* of
 
 // Deletion: one thread per id sets the item's bit in the deletion bitmap.
 __global__ void __launch_bounds__(256)
-delete_kernel(uint32_t* dead, int64_t n, const int64_t* ids, int64_t m, uint32_t* err)
+delete_kernel(uint32_t* dead, RowMap map, const int64_t* ids, int64_t m, uint32_t* err)
 {
     const int64_t j = int64_t(blockIdx.x) * 256 + threadIdx.x;
     if (j >= m) return;
     const int64_t id = ids[j];
-    if (id < 0 || id >= n) {
+    int64_t t = 0;
+    int r = 0;
+    if (!locate_row(map, id, t, r)) {
         atomicOr(err, kErrUpdateId);
         return;
     }
     atomicOr(dead + (id >> 5), 1u << (id & 31));
 }
 
-cudaError_t launch_delete(uint32_t* dead, int64_t n, const int64_t* ids, int64_t m, uint32_t* err, cudaStream_t s)
+cudaError_t launch_delete(uint32_t* dead, const RowMap& map, const int64_t* ids, int64_t m, uint32_t* err,
+                          cudaStream_t s)
 {
     if (m <= 0) return cudaSuccess;
-    delete_kernel<<<unsigned((m + 255) / 256), 256, 0, s>>>(dead, n, ids, m, err);
+    delete_kernel<<<unsigned((m + 255) / 256), 256, 0, s>>>(dead, map, ids, m, err);
     return cudaGetLastError();
 }
 
-cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets,
-                          const int32_t* chunk_start, int32_t nlist, int64_t n, int d, int W, const int64_t* ids,
-                          const int8_t* new_items, const uint64_t* new_sigs, int64_t m, uint32_t* err, cudaStream_t s)
+cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const RowMap& map, int d, int W,
+                          const int64_t* ids, const int8_t* new_items, const uint64_t* new_sigs, int64_t m,
+                          uint32_t* err, cudaStream_t s)
 {
     if (m <= 0) return cudaSuccess;
     const int64_t blocks = (m * 32 + 255) / 256;
     if (W == 2)
-        update_kernel<2><<<unsigned(blocks), 256, 0, s>>>(items, sigs, planes, offsets, chunk_start, nlist, n, d, ids,
-                                                          new_items, new_sigs, m, err);
+        update_kernel<2><<<unsigned(blocks), 256, 0, s>>>(items, sigs, planes, map, d, ids, new_items, new_sigs, m,
+                                                          err);
     else
-        update_kernel<1><<<unsigned(blocks), 256, 0, s>>>(items, sigs, planes, offsets, chunk_start, nlist, n, d, ids,
-                                                          new_items, new_sigs, m, err);
+        update_kernel<1><<<unsigned(blocks), 256, 0, s>>>(items, sigs, planes, map, d, ids, new_items, new_sigs, m,
+                                                          err);
     return cudaGetLastError();
 }
 

@@ -9,9 +9,10 @@
 //   * units_alloc: one thread per list; a warp-wide scan of the lists' unit
 //     counts and one atomic per warp give every probed list its block of the
 //     unit table (blocks land in completion order, which the scan ignores);
-//   * units_write: one thread per list chunk (the index's static chunk table),
-//     so a list of millions of rows is written by thousands of threads: the
-//     thread writes its chunk's entry for each query group of the list.
+//   * units_write: one thread per list chunk (the index's chunk table, list by
+//     list: a list's creation chunks, then its append chunks), so a list of
+//     millions of rows is written by thousands of threads: the thread writes
+//     its chunk's entry for each query group of the list.
 #include "st_internal.cuh"
 
 namespace st {
@@ -49,28 +50,37 @@ units_alloc_kernel(SearchArgs a)
 __global__ void __launch_bounds__(kUnitsBlock)
 units_write_kernel(SearchArgs a)
 {
-    const int t = blockIdx.x * kUnitsBlock + threadIdx.x;  // global chunk id
+    const int t = blockIdx.x * kUnitsBlock + threadIdx.x;  // chunk table entry
     if (t >= a.n_chunks) return;
-    const int L = a.chunk_list[t];
+    const int4 c = a.chunk_desc[t];  // {first row, plane block, rows, list}
+    const int L = c.w;
+    if (L < 0 || L >= a.nlist) {
+        set_error(a.err, kErrUnitDecode);
+        return;
+    }
     const int cnt = a.list_cnt[L];
     if (cnt <= 0) return;
     const int c0 = a.chunk_start[L];
     const int nch = a.chunk_start[L + 1] - c0;
-    const int c = t - c0;
-    const long long o0 = a.offsets[L], o1 = a.offsets[L + 1];
-    const long long ib = o0 + (long long)c * kWarpItems;
-    const long long rem = o1 - ib;
-    const int len = int(rem < kWarpItems ? rem : kWarpItems);
-    if (c < 0 || c >= nch || len <= 0) {
+    const int ci = t - c0;
+    if (ci < 0 || ci >= nch) {  // the list's block of units does not cover this entry
         set_error(a.err, kErrUnitDecode);
         return;
+    }
+    int4 unit = make_int4(c.x, c.y, 0, c.z);
+    if (c.z < 1 || c.z > kWarpItems || c.x < 0 || int64_t(c.x) + c.z > a.n_rows || c.y < 0 ||
+        c.y >= a.n_plane_chunks) {
+        // a unit the scan can run but that finds nothing
+        set_error(a.err, kErrUnitDecode);
+        unit = make_int4(0, 0, 0, 0);
     }
     const int64_t base = a.list_ustart[L];
     const int groups = (cnt + kQMax - 1) / kQMax;
     for (int g = 0; g < groups; ++g) {
-        const int64_t idx = base + int64_t(g) * nch + c;
+        const int64_t idx = base + int64_t(g) * nch + ci;
         if (idx < a.max_units)
-            a.units[idx] = make_int4(int(ib), t, L * a.B + g * kQMax, (len << 16) | min(kQMax, cnt - g * kQMax));
+            a.units[idx] = make_int4(unit.x, unit.y, L * a.B + g * kQMax,
+                                     (unit.w << 16) | min(kQMax, cnt - g * kQMax));
     }
 }
 

@@ -56,46 +56,55 @@ __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, 
             if (threadIdx.x == 0) set_error(a.err, kErrOverflowPath);
             continue;
         }
-        const int64_t o0 = a.offsets[L], o1 = a.offsets[L + 1];
-        for (int64_t base = o0; base < o1; base += BLOCK) {
-            if (int64_t(s_count) + BLOCK > cap) {
-                // keep the k best, drop everything below them from now on
-                const int64_t cnt = s_count;
-                const uint64_t thr = block_select_threshold<BLOCK>(buf, cnt, k, ss, a.err);
-                const int32_t got = block_collect_ge<BLOCK>(buf, cnt, thr, sortbuf, pwk, ss);  // unsorted is fine here
-                if (threadIdx.x == 0 && got != k) set_error(a.err, kErrOverflowPath);
-                for (int i = threadIdx.x; i < k; i += BLOCK) buf[i] = sortbuf[i];
-                if (threadIdx.x == 0) {
-                    s_count = k;
-                    s_thr = thr;
+        // the list's chunks: its creation rows, then its append chunks
+        const int t0 = a.chunk_start[L], t1 = a.chunk_start[L + 1];
+        for (int t = t0; t < t1; ++t) {
+            const int4 c = a.chunk_desc[t];  // {first row, plane block, rows, list}
+            if (c.w != L || c.z < 0 || c.z > kWarpItems || c.x < 0 || int64_t(c.x) + c.z > a.n_rows) {
+                if (threadIdx.x == 0) set_error(a.err, kErrOverflowPath);
+                continue;
+            }
+            const int64_t o0 = c.x, o1 = int64_t(c.x) + c.z;
+            for (int64_t base = o0; base < o1; base += BLOCK) {
+                if (int64_t(s_count) + BLOCK > cap) {
+                    // keep the k best, drop everything below them from now on
+                    const int64_t cnt = s_count;
+                    const uint64_t thr = block_select_threshold<BLOCK>(buf, cnt, k, ss, a.err);
+                    const int32_t got = block_collect_ge<BLOCK>(buf, cnt, thr, sortbuf, pwk, ss);  // unsorted is fine here
+                    if (threadIdx.x == 0 && got != k) set_error(a.err, kErrOverflowPath);
+                    for (int i = threadIdx.x; i < k; i += BLOCK) buf[i] = sortbuf[i];
+                    if (threadIdx.x == 0) {
+                        s_count = k;
+                        s_thr = thr;
+                    }
+                    __syncthreads();
+                }
+                const int64_t i = base + threadIdx.x;
+                const uint64_t thr = s_thr;
+                bool keep = false;
+                uint64_t key = 0;
+                if (i < o1) {
+                    const uint64_t* sg = a.sigs + i * W;
+                    bool pass = (sg[0] & m0) == m0;
+                    if (W > 1) pass = pass && ((sg[1] & m1) == m1);
+                    pass = pass && keep_item(a, q, i);
+                    if (pass) {
+                        const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);
+                        int32_t acc = 0;
+                        for (int j = 0; j < np; ++j) acc = dot16(__ldg(rp + j), s_qv[j], acc);
+                        key = pack_key(acc, uint32_t(i));
+                        keep = key >= thr;
+                    }
+                }
+                const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                if (bal) {
+                    int32_t b0 = 0;
+                    if ((threadIdx.x & 31) == 0) b0 = atomicAdd(&s_count, __popc(bal));
+                    b0 = __shfl_sync(0xffffffffu, b0, 0);
+                    if (keep) buf[b0 + __popc(bal & lanemask_lt())] = key;
                 }
                 __syncthreads();
             }
-            const int64_t i = base + threadIdx.x;
-            const uint64_t thr = s_thr;
-            bool keep = false;
-            uint64_t key = 0;
-            if (i < o1) {
-                const uint64_t* sg = a.sigs + i * W;
-                bool pass = (sg[0] & m0) == m0;
-                if (W > 1) pass = pass && ((sg[1] & m1) == m1);
-                pass = pass && keep_item(a, q, i);
-                if (pass) {
-                    const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);
-                    int32_t acc = 0;
-                    for (int t = 0; t < np; ++t) acc = dot16(__ldg(rp + t), s_qv[t], acc);
-                    key = pack_key(acc, uint32_t(i));
-                    keep = key >= thr;
-                }
-            }
-            const unsigned bal = __ballot_sync(0xffffffffu, keep);
-            if (bal) {
-                int32_t b0 = 0;
-                if ((threadIdx.x & 31) == 0) b0 = atomicAdd(&s_count, __popc(bal));
-                b0 = __shfl_sync(0xffffffffu, b0, 0);
-                if (keep) buf[b0 + __popc(bal & lanemask_lt())] = key;
-            }
-            __syncthreads();
         }
     }
     return s_count;

@@ -71,11 +71,13 @@ struct SearchArgs {
     // index (read-only)
     const int8_t* items;
     const uint64_t* sigs;
-    const uint32_t* planes;      // [n_chunks][64W][16] signature bit-planes per list chunk
-    const int64_t* offsets;
-    const int32_t* chunk_start;  // [nlist+1] first chunk of each list (chunks of kWarpItems rows)
-    const int32_t* chunk_list;   // [n_chunks] list of each chunk
+    const uint32_t* planes;      // [n_plane_chunks][64W][16] signature bit-planes, one block per chunk
+    const int4* chunk_desc;      // [n_chunks] the chunks (up to kWarpItems rows of one list), list by list:
+                                 // {first row, plane block, rows, list}
+    const int32_t* chunk_start;  // [nlist+1] first chunk_desc entry of each list
     int32_t n_chunks;
+    int32_t n_plane_chunks;      // plane blocks allocated
+    int64_t n_rows;              // rows the item and signature arrays hold
     const int8_t* centroids;
     int32_t d, nlist, W;
     // request
@@ -761,10 +763,24 @@ cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B
                          int32_t* out_scores, cudaStream_t s);
 cudaError_t merge_error_word(uint32_t* word, bool clear);
 size_t scan_smem_bytes(int d, int W);
-cudaError_t launch_delete(uint32_t* dead, int64_t n, const int64_t* ids, int64_t m, uint32_t* err, cudaStream_t s);
-cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const int64_t* offsets,
-                          const int32_t* chunk_start, int32_t nlist, int64_t n, int d, int W, const int64_t* ids,
-                          const int8_t* new_items, const uint64_t* new_sigs, int64_t m, uint32_t* err, cudaStream_t s);
+// Where the rows of an index live, for the update, insert and delete kernels:
+// rows [0, n) are the creation lists (list c: offsets[c] .. offsets[c+1]-1, plane
+// blocks from base_chunk_start[c]); rows n + kWarpItems * a + r (r < app_len[a])
+// are append chunk a, plane block n_base_chunks + a.
+struct RowMap {
+    const int64_t* offsets;
+    const int32_t* base_chunk_start;
+    int32_t nlist;
+    int64_t n;
+    int32_t n_base_chunks;
+    const int32_t* app_len;  // [n_app] rows filled in each append chunk
+    int32_t n_app;
+};
+cudaError_t launch_delete(uint32_t* dead, const RowMap& map, const int64_t* ids, int64_t m, uint32_t* err,
+                          cudaStream_t s);
+cudaError_t launch_update(int8_t* items, uint64_t* sigs, uint32_t* planes, const RowMap& map, int d, int W,
+                          const int64_t* ids, const int8_t* new_items, const uint64_t* new_sigs, int64_t m,
+                          uint32_t* err, cudaStream_t s);
 cudaError_t launch_build_planes(const uint64_t* sigs, const int64_t* offsets, const int32_t* chunk_start,
                                 const int32_t* chunk_list, int32_t n_chunks, int W, uint32_t* planes,
                                 cudaStream_t s);

@@ -163,12 +163,21 @@ typedef enum {
     /* Added to every item id the index returns (default 0): an index built
        from rows [r0, r1) of a larger collection, with this option set to r0,
        returns ids of that collection -- one document shard of it (see
-       st_merge_topk). Rejected with UNSUPPORTED unless offset + n < 2^31. */
-    ST_OPT_ID_OFFSET = 3
+       st_merge_topk). Rejected with UNSUPPORTED unless offset plus the rows
+       the index has room for stays below 2^31. */
+    ST_OPT_ID_OFFSET = 3,
+    /* Make room now for insertions (st_index_insert): at least
+       ceil(value / ST_INSERT_CHUNK) more append chunks, i.e. value rows added
+       to one list, without a reallocation later. Growing copies the index
+       once and needs the old and the new arrays at the same time. 0 is a
+       no-op; the room is never given back. OOM when it cannot be had,
+       UNSUPPORTED when the ids would reach 2^31 (with the id offset). */
+    ST_OPT_INSERT_RESERVE = 4
 } st_option;
 
 /* Set an option; INVALID_ARG for an unknown option or a negative value.
-   Not safe to call while a search on the same index is being enqueued. */
+   Not safe to call while a search on the same index is being enqueued, and
+   ST_OPT_INSERT_RESERVE waits for the device like st_index_insert does. */
 st_status st_index_set_option(st_index* idx, st_option opt, int64_t value);
 
 /*
@@ -266,11 +275,13 @@ st_status st_merge_check(cudaStream_t stream);
  * index fresh between full snapshots by streaming new signals into the
  * in-memory model (SilverTorch: Index as Model, section on engineering for
  * scale and freshness, index freshness paragraph); this call is that step for
- * items whose row stays in its list. Inserting new items and deleting items
- * are not provided.
+ * items whose row stays in its list (new items: st_index_insert; removal:
+ * st_index_delete).
  *
- *   ids    device int64 [m]             row indices of the index (without any
- *                                       ST_OPT_ID_OFFSET); distinct within a call
+ *   ids    device int64 [m]             item ids of the index (without any
+ *                                       ST_OPT_ID_OFFSET): rows given to
+ *                                       st_index_create or ids returned by
+ *                                       st_index_insert; distinct within a call
  *   items  device int8  [m][d] or NULL  new rows (NULL: rows unchanged)
  *   sigs   device uint64 [m][sig_words] or NULL  new signatures (NULL: unchanged)
  *
@@ -278,7 +289,8 @@ st_status st_merge_check(cudaStream_t stream);
  * signatures. Asynchronous on `stream`: searches enqueued later on the same
  * stream see the new values; searches on other streams must be ordered after
  * it by the caller (they read the same memory), and two updates must not
- * overlap. An id outside [0, n) is skipped and recorded in the index's error
+ * overlap. An id that the index never handed out (outside [0, n) and not
+ * returned by st_index_insert) is skipped and recorded in the index's error
  * word (st_index_check). Errors: INVALID_ARG (null index, m < 0, null or
  * non-device ids when m > 0, non-device items / sigs, both NULL), CUDA.
  */
@@ -288,15 +300,48 @@ st_status st_index_update(st_index* idx, const int64_t* ids, const int8_t* items
 /*
  * Delete m items in place (tombstones): a deleted item is never returned
  * again, by any later search on `stream` (other streams: order them after it).
- * ids are row indices of the index (without any ST_OPT_ID_OFFSET); deleting
- * twice is harmless; st_index_update does not revive an item. Deleted rows
- * still take part in the scan (their scores are dropped before the final
- * top-k) and in st_search_extras.eligible. The first deletion allocates a
- * bitmap of n bits. An id outside [0, n) is skipped and recorded in the
- * index's error word. Errors: INVALID_ARG (null index, m < 0, null or
+ * ids are item ids of the index, as for st_index_update; deleting twice is
+ * harmless; st_index_update does not revive an item. Deleted rows still take
+ * part in the scan (their scores are dropped before the final top-k) and in
+ * st_search_extras.eligible. The first deletion allocates a bitmap with one
+ * bit per row the index has room for. An id the index never handed out is
+ * skipped and recorded in the index's error word. Errors: INVALID_ARG (null index, m < 0, null or
  * non-device ids when m > 0), OOM, CUDA.
  */
 st_status st_index_delete(st_index* idx, const int64_t* ids, int64_t m, cudaStream_t stream);
+
+/*
+ * Insert m new items into existing IVF lists without a rebuild (the insertion
+ * half of index freshness: SilverTorch: Index as Model, section on engineering
+ * for scale and freshness, index freshness paragraph).
+ *
+ *   lists   HOST int32 [m]                 the list each new item joins, in [0, nlist)
+ *   items   device int8 [m][d]             the new rows (16-byte aligned)
+ *   sigs    device uint64 [m][sig_words]   their Bloom signatures
+ *   out_ids HOST int64 [m]                 receives the id given to each item
+ *
+ * Layout: each list owns, after its creation rows, zero or more append chunks
+ * of ST_INSERT_CHUNK rows placed after all creation rows; a list's new items
+ * fill its last append chunk in argument order, then a fresh one. An item's
+ * id is its row, so ids are >= n (the creation rows), unique, never reused and
+ * stable, but not consecutive: the unfilled rows of each list's last append
+ * chunk are ids no call returned yet. ST_OPT_ID_OFFSET is added to them in
+ * search results, like to every id. The item's Bloom bit-planes are written as
+ * by st_index_update, and later searches on `stream` see it (other streams:
+ * order them after this call). When the append chunks run out, the index
+ * grows (the item, signature and plane arrays are copied once into arrays
+ * with at least twice the append room; see ST_OPT_INSERT_RESERVE).
+ *
+ * The call waits for `stream` (and, when it grows the index or its chunk
+ * table, for the device) before it returns, so the host arrays may be reused
+ * at once. Errors, with the index unchanged: INVALID_ARG (null index, m < 0,
+ * null host arrays or non-device items / sigs when m > 0, a list id outside
+ * [0, nlist)), UNSUPPORTED (ids would reach 2^31 with the id offset), OOM;
+ * CUDA if a copy or kernel fails (the index should then be destroyed).
+ */
+#define ST_INSERT_CHUNK 512
+st_status st_index_insert(st_index* idx, const int32_t* lists, const int8_t* items, const uint64_t* sigs,
+                          int64_t m, int64_t* out_ids, cudaStream_t stream);
 
 /* Free the index (NULL-safe). Waits for the device to finish work that may
    still use it. */
