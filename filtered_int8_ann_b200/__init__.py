@@ -27,7 +27,8 @@ ST_MERGE_MAX_KEYS = 16384
 ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K, ST_MAX_B = 512, 262144, 4096, 4096, 32768
 
 # Every symbol include/st.h declares.
-EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
+EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_search_host_async",
+           "st_index_check",
            "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
            "st_index_delete", "st_merge_topk_union", "st_index_insert", "st_index_destroy", "st_status_string")
 
@@ -58,6 +59,7 @@ def lib() -> ctypes.CDLL:
     L.st_search.argtypes = [P, P, P, i32, i32, i32, P, P, P]
     L.st_search_ex.argtypes = [P, P, P, i32, i32, i32, P, P, ctypes.POINTER(_Extras), P]
     L.st_search_host.argtypes = [P, P, P, i32, i32, i32, P, P, P]
+    L.st_search_host_async.argtypes = [P, P, P, i32, i32, i32, P, P, P]
     L.st_index_check.argtypes = [P, P]
     L.st_index_set_option.argtypes = [P, ctypes.c_int, i64]
     L.st_probe_noalloc.argtypes = [P, P, i32, i32, P, P]
@@ -67,7 +69,8 @@ def lib() -> ctypes.CDLL:
     L.st_index_delete.argtypes = [P, P, i64, P]
     L.st_merge_topk_union.argtypes = [P, P, i32, i32, i32, P, P, P]
     L.st_index_insert.argtypes = [P, P, P, P, i64, P, P]
-    for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_index_check",
+    for f in ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_search_host_async",
+              "st_index_check",
               "st_index_set_option", "st_probe_noalloc", "st_merge_topk", "st_merge_check", "st_index_update",
               "st_index_delete", "st_merge_topk_union", "st_index_insert"):
         getattr(L, f).restype = ctypes.c_int
@@ -178,6 +181,17 @@ def st_search_host(index: int, queries: torch.Tensor, qmasks: torch.Tensor, npro
     return out_ids, out_scores
 
 
+def st_search_host_async(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: int, k: int,
+                         out_ids: torch.Tensor, out_scores: torch.Tensor, stream=None):
+    """Enqueue a search on page-locked host tensors and return at once; the
+    outputs are complete when the stream has finished it."""
+    qmasks = _as_words(qmasks)
+    B = queries.shape[0]
+    _check(lib().st_search_host_async(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
+                                      _ptr(out_scores), _stream(stream)), "st_search_host_async")
+    return out_ids, out_scores
+
+
 def st_index_check(index: int, stream=None) -> int:
     """Synchronize and return the device-side status (ST_OK or ST_ERR_DEVICE)."""
     return lib().st_index_check(index, _stream(stream))
@@ -248,6 +262,9 @@ class Index:
 
     def search_host(self, queries, qmasks, nprobe, k, **kw):
         return st_search_host(self.handle, queries, qmasks, nprobe, k, **kw)
+
+    def search_host_async(self, queries, qmasks, nprobe, k, out_ids, out_scores, stream=None):
+        return st_search_host_async(self.handle, queries, qmasks, nprobe, k, out_ids, out_scores, stream)
 
     def update(self, ids, items=None, sigs=None, stream=None):
         """Replace the rows and/or signatures of existing items in place (device tensors)."""

@@ -583,14 +583,27 @@ st_status st_search(const st_index* idx, const int8_t* queries, const uint64_t* 
     return st_search_ex(idx, queries, qmasks, B, nprobe, k, out_ids, out_scores, nullptr, stream);
 }
 
-st_status st_search_host(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
-                         int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores,
-                         cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+bool is_pinned_host(const void* p)
 {
-    st_status s = check_search_args(idx, B, nprobe, k);
-    if (s != ST_OK) return s;
-    if (!queries || !qmasks || !out_ids || !out_scores) return ST_ERR_INVALID_ARG;
-    DeviceGuard g(idx->device);
+    if (p == nullptr) return false;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeHost;
+}
+
+// Host-buffer search: stage the inputs in pool memory, search, copy the
+// outputs back; optionally wait for the stream.
+st_status search_host_impl(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
+                           int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores, cudaStream_t stream,
+                           bool wait)
+{
     const size_t qb = align_up(size_t(B) * idx->d, 256), mb = align_up(size_t(B) * idx->W * 8, 256);
     const size_t ib = align_up(size_t(B) * k * 8, 256), sb = align_up(size_t(B) * k * 4, 256);
     unsigned char* buf = nullptr;
@@ -614,11 +627,39 @@ st_status st_search_host(const st_index* idx, const int8_t* queries, const uint6
         }
     }
     cudaError_t ef = cudaFreeAsync(buf, stream);
-    cudaError_t es = cudaStreamSynchronize(stream);
+    cudaError_t es = wait ? cudaStreamSynchronize(stream) : cudaSuccess;
     if (rs != ST_OK) return rs;
     if (e == cudaSuccess) e = ef;
     if (e == cudaSuccess) e = es;
     return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+st_status st_search_host(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
+                         int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                         cudaStream_t stream)
+{
+    st_status s = check_search_args(idx, B, nprobe, k);
+    if (s != ST_OK) return s;
+    if (!queries || !qmasks || !out_ids || !out_scores) return ST_ERR_INVALID_ARG;
+    DeviceGuard g(idx->device);
+    return search_host_impl(idx, queries, qmasks, B, nprobe, k, out_ids, out_scores, stream, true);
+}
+
+st_status st_search_host_async(const st_index* idx, const int8_t* queries, const uint64_t* qmasks, int32_t B,
+                               int32_t nprobe, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                               cudaStream_t stream)
+{
+    st_status s = check_search_args(idx, B, nprobe, k);
+    if (s != ST_OK) return s;
+    DeviceGuard g(idx->device);
+    if (!is_pinned_host(queries) || !is_pinned_host(qmasks) || !is_pinned_host(out_ids) ||
+        !is_pinned_host(out_scores))
+        return ST_ERR_INVALID_ARG;
+    return search_host_impl(idx, queries, qmasks, B, nprobe, k, out_ids, out_scores, stream, false);
 }
 
 st_status st_probe_noalloc(const st_index* idx, const int8_t* queries, int32_t B, int32_t nprobe,

@@ -144,6 +144,20 @@ st_status st_search_host(const st_index* idx, const int8_t* queries, const uint6
                          int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
 
 /*
+ * st_search_host without the wait, for a serving loop that keeps several
+ * batches in flight (one stream each): enqueues the copy of queries and masks
+ * to the device, the search and the copy of ids and scores back, and returns.
+ * Every host array must be page-locked (cudaHostAlloc / cudaHostRegister) --
+ * pageable memory is refused with INVALID_ARG, since its copies would block.
+ * The outputs are complete once `stream` has finished this work (an event or
+ * a stream synchronize); until then the caller must neither read the outputs
+ * nor change the inputs. Same arguments and errors as st_search otherwise.
+ */
+st_status st_search_host_async(const st_index* idx, const int8_t* queries, const uint64_t* qmasks,
+                               int32_t B, int32_t nprobe, int32_t k,
+                               int64_t* out_ids, int32_t* out_scores, cudaStream_t stream);
+
+/*
  * Wait for `stream`, then report and clear the index's device-side error word.
  * Returns ST_OK, ST_ERR_DEVICE when a kernel recorded an internal error since
  * the last check (no result produced meanwhile should be trusted), or

@@ -165,6 +165,42 @@ def test_search_host_matches_device_path():
         idx.close()
 
 
+def test_search_host_async_pipelined_matches_oracle():
+    """Two batches in flight on two streams through the asynchronous host call,
+    each slot's outputs checked when its stream is done; pageable buffers are
+    refused before anything is enqueued."""
+    data = small(n=12000, d=64, nlist=24, sig_bits=128, hash_bits=3, B=24, nprobe=6, k=300, seed=31)
+    g = data.to("cuda")
+    exp = run_oracle(data, 6, 300)
+    idx = st.Index(g.items, g.sigs, g.offsets, g.centroids)
+    try:
+        halves = [(0, 12), (12, 24)]
+        qs = [data.queries[a:b].contiguous().pin_memory() for a, b in halves]
+        ms = [data.masks[a:b].contiguous().pin_memory() for a, b in halves]
+        streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+        outs = [(torch.full((12, 300), -7, dtype=torch.int64).pin_memory(),
+                 torch.full((12, 300), -7, dtype=torch.int32).pin_memory()) for _ in range(2)]
+        for rep in range(3):
+            for j in range(2):
+                idx.search_host_async(qs[j], ms[j], 6, 300, outs[j][0], outs[j][1], stream=streams[j])
+            for j, (a, b) in enumerate(halves):
+                streams[j].synchronize()
+                assert np.array_equal(outs[j][0].numpy(), exp[0][a:b])
+                assert np.array_equal(outs[j][1].numpy(), exp[1][a:b])
+                outs[j][0].fill_(-7)
+        assert idx.check() == st.ST_OK
+        pageable = torch.empty((12, 300), dtype=torch.int64)
+        with pytest.raises(st.StError) as ei:
+            idx.search_host_async(qs[0], ms[0], 6, 300, pageable, outs[0][1])
+        assert ei.value.status == st.ST_ERR_INVALID_ARG
+        with pytest.raises(st.StError) as ei:
+            idx.search_host_async(data.queries[:12].contiguous(), ms[0], 6, 300, outs[0][0], outs[0][1])
+        assert ei.value.status == st.ST_ERR_INVALID_ARG
+        assert bool((outs[0][0] == -7).all())
+    finally:
+        idx.close()
+
+
 def test_index_independent_of_caller_buffers():
     data = small(n=5000, d=64, nlist=8, B=4, nprobe=3, k=80, seed=29)
     g = data.to("cuda")
