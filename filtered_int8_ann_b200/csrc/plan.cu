@@ -22,6 +22,7 @@ constexpr int kUnitsBlock = 256;
 __global__ void __launch_bounds__(kUnitsBlock)
 units_alloc_kernel(SearchArgs a)
 {
+    dep_enter();
     const int lane = threadIdx.x & 31;
     const int L = blockIdx.x * kUnitsBlock + threadIdx.x;
     uint32_t u = 0;
@@ -50,6 +51,7 @@ units_alloc_kernel(SearchArgs a)
 __global__ void __launch_bounds__(kUnitsBlock)
 units_write_kernel(SearchArgs a)
 {
+    dep_enter();
     const int t = blockIdx.x * kUnitsBlock + threadIdx.x;  // chunk table entry
     if (t >= a.n_chunks) return;
     const int4 c = a.chunk_desc[t];  // {first row, plane block, rows, list}
@@ -87,11 +89,9 @@ units_write_kernel(SearchArgs a)
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s)
 {
     (void)num_sms;
-    units_alloc_kernel<<<(a.nlist + kUnitsBlock - 1) / kUnitsBlock, kUnitsBlock, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_dep(units_alloc_kernel, dim3((a.nlist + kUnitsBlock - 1) / kUnitsBlock), dim3(kUnitsBlock), 0, s, a);
     if (e != cudaSuccess) return e;
-    units_write_kernel<<<(a.n_chunks + kUnitsBlock - 1) / kUnitsBlock, kUnitsBlock, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_dep(units_write_kernel, dim3((a.n_chunks + kUnitsBlock - 1) / kUnitsBlock), dim3(kUnitsBlock), 0, s, a);
 }
 
 }  // namespace st

@@ -214,6 +214,7 @@ template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK)
 probe_select_kernel(SearchArgs a, int stage_cap, int tie_cap)
 {
+    dep_enter();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ SelectSmem ss;
     const int b = blockIdx.x;
@@ -271,8 +272,7 @@ cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s)
     const size_t smem = probe_select_smem(a.P, a.nlist, &stage_cap);
     e = ensure_smem_attr(reinterpret_cast<const void*>(probe_select_kernel<kProbeSelBlock>), 11, 200 * 1024);
     if (e != cudaSuccess) return e;
-    probe_select_kernel<kProbeSelBlock><<<a.B, kProbeSelBlock, smem, s>>>(a, stage_cap, kProbeTieCap);
-    return cudaGetLastError();
+    return launch_dep(probe_select_kernel<kProbeSelBlock>, dim3(a.B), dim3(kProbeSelBlock), smem, s, a, stage_cap, int(kProbeTieCap));
 }
 
 int probe_slices(const SearchArgs& a, int num_sms)

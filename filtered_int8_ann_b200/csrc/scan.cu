@@ -111,6 +111,7 @@ template <int NP, int W>
 __global__ void __launch_bounds__(kScanBlock, NP == 8 ? 4 : 5)
 scan_kernel(SearchArgs a)
 {
+    dep_enter();
     extern __shared__ __align__(128) unsigned char smem_raw[];
     constexpr int NPL = 64 * W;
     const int lane = threadIdx.x & 31;
@@ -503,8 +504,7 @@ static cudaError_t launch_variant(const SearchArgs& a, int num_sms, cudaStream_t
         if (occ < 1) occ = 1;
         if (NP > 0 && dev < 64) occ_cache[dev][slot - 1] = occ;
     }
-    scan_kernel<NP, W><<<num_sms * occ, kScanBlock, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_dep(scan_kernel<NP, W>, dim3(num_sms * occ), dim3(kScanBlock), smem, s, a);
 }
 
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s)

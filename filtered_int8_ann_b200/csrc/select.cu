@@ -205,6 +205,7 @@ __device__ int compact_cut_bin(const SearchArgs& a, int q, int64_t n, const Topk
 __global__ void __launch_bounds__(kChunkBlock)
 select_hist_kernel(SearchArgs a)
 {
+    dep_enter();
     extern __shared__ int pre[];  // [B + 1]
     __shared__ SelectSmem ss;
     __shared__ int s_last;
@@ -273,6 +274,7 @@ select_hist_kernel(SearchArgs a)
 __global__ void __launch_bounds__(kChunkBlock)
 select_scatter_kernel(SearchArgs a)
 {
+    dep_enter();
     extern __shared__ int pre[];  // [B + 1]
     __shared__ uint32_t part[32];
     chunk_prefix<kChunkBlock>(a, pre, part);
@@ -319,6 +321,7 @@ template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK)
 select_kernel(SearchArgs a, int stage_cap)
 {
+    dep_enter();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ SelectSmem ss;
     const int q = blockIdx.x;
@@ -404,6 +407,7 @@ template <int BLOCK>
 __global__ void __launch_bounds__(BLOCK)
 select_ties_kernel(SearchArgs a)
 {
+    dep_enter();
     __shared__ SelectSmem ss;
     const int q = blockIdx.x;
     const int k = a.k;
@@ -435,6 +439,7 @@ select_ties_kernel(SearchArgs a)
 __global__ void __launch_bounds__(256)
 select_rank_kernel(SearchArgs a)
 {
+    dep_enter();
     const int k = a.k;
     const int64_t idx = int64_t(blockIdx.x) * 256 + threadIdx.x;
     if (idx >= int64_t(a.B) * k) return;
@@ -488,28 +493,23 @@ cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
     const int grid = 3 * num_sms;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_hist_kernel), 12, kPreSmemMax);
     if (e != cudaSuccess) return e;
-    select_hist_kernel<<<grid, kChunkBlock, pre_bytes, s>>>(a);
-    e = cudaGetLastError();
+    e = launch_dep(select_hist_kernel, dim3(grid), dim3(kChunkBlock), pre_bytes, s, a);
     if (e != cudaSuccess) return e;
     e = ensure_smem_attr(reinterpret_cast<const void*>(select_scatter_kernel), 13, kPreSmemMax);
     if (e != cudaSuccess) return e;
-    select_scatter_kernel<<<grid, kChunkBlock, pre_bytes, s>>>(a);
-    e = cudaGetLastError();
+    e = launch_dep(select_scatter_kernel, dim3(grid), dim3(kChunkBlock), pre_bytes, s, a);
     if (e != cudaSuccess) return e;
     if (a.k > ST_SMALL_K) {
-        select_ties_kernel<kSelectBlock><<<a.B, kSelectBlock, 0, s>>>(a);
-        e = cudaGetLastError();
+        e = launch_dep(select_ties_kernel<kSelectBlock>, dim3(a.B), dim3(kSelectBlock), 0, s, a);
         if (e != cudaSuccess) return e;
         const int64_t threads = int64_t(a.B) * a.k;
-        select_rank_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(a);
-        return cudaGetLastError();
+        return launch_dep(select_rank_kernel, dim3(unsigned((threads + 255) / 256)), dim3(256), 0, s, a);
     }
     int stage_cap = 0;
     const size_t smem = select_smem(a.k, &stage_cap);
     e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8, int(smem));
     if (e != cudaSuccess) return e;
-    select_kernel<kSelectBlock><<<a.B, kSelectBlock, smem, s>>>(a, stage_cap);
-    return cudaGetLastError();
+    return launch_dep(select_kernel<kSelectBlock>, dim3(a.B), dim3(kSelectBlock), smem, s, a, stage_cap);
 }
 
 }  // namespace st

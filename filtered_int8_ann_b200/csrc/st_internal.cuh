@@ -1,5 +1,6 @@
 // Internal definitions shared by the libst kernels and the host API.
 #pragma once
+#include <utility>
 
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -118,6 +119,33 @@ struct SearchArgs {
     int64_t cap;             // candidate keys per query
     uint32_t* err;           // device error word
 };
+
+
+// Programmatic dependent launch: launch_dep() lets a kernel start while its
+// predecessor in the stream drains; every such kernel calls dep_enter() first
+// (wait for the predecessor's completion and memory, then let its own
+// successor launch).
+__device__ __forceinline__ void dep_enter()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dep(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ----------------------------------------------------------------------------
 // Small device helpers
