@@ -4,7 +4,7 @@
  *
  * What it computes. For each query b (an int8 vector q_b and a Bloom mask m_b):
  *   1. probe: score every IVF list c by the int32 inner product <q_b, cent_c>
- *      and keep the nprobe best lists (the clusters judged best are chosen
+ *      and keep the nprobe best lists (the best-scoring clusters are chosen
  *      first -- SilverTorch: Index as Model, section on how each component
  *      worked before);
  *   2. filter: inside the probed lists only, an item i is eligible when
