@@ -12,6 +12,7 @@ Prints one JSON line (rank 0). `--impl reference` times the CPU oracle instead
 """
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -372,8 +373,14 @@ def main():
     torch.cuda.synchronize()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    for row in evs:
+    # stage events on every `stride`-th timed step only: an event between two
+    # kernels ends the programmatic dependent launch across it, so the other
+    # steps run exactly as a caller's searches do. The stride is coprime with
+    # the batch pool, so the sampled steps cover every batch equally.
+    stride = next(s_ for s_ in range(3, 1000) if math.gcd(s_, pool) == 1)
+    sampled = list(range(0, K, stride))
+    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for i in sampled}
+    for row in evs.values():
         for e in row:
             e.record()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -384,7 +391,7 @@ def main():
     torch.cuda.synchronize()
     start.record()
     for i in range(K):
-        step(i, evs[i])
+        step(i, evs.get(i))
     end.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -393,11 +400,11 @@ def main():
     ms_local = start.elapsed_time(end)
     ms = allreduce_max(ms_local, world)
 
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(K)])
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in sampled])
     stage_mean = stage_ms.mean(0)
     scan_ms = stage_mean[2]
-    method_bytes = np.array([models[i % pool][0] for i in range(K)], dtype=np.float64)
-    full_bytes = np.array([models[i % pool][1] for i in range(K)], dtype=np.float64)
+    method_bytes = np.array([models[i % pool][0] for i in sampled], dtype=np.float64)
+    full_bytes = np.array([models[i % pool][1] for i in sampled], dtype=np.float64)
     scan_gbs = float(method_bytes.sum() / (stage_ms[:, 2].sum() * 1e-3) / 1e9)
     peak, peak_kind = peaks()
 
@@ -405,6 +412,37 @@ def main():
     total_q = float(B * K) if shard else allreduce_sum(float(B * K), world)
     elig_total = allreduce_sum(float(sum(elig_per_batch[i % pool] for i in range(K))), world)
     value = total_q / (ms * 1e-3)
+
+    # the same device-resident searches with E2E_INFLIGHT batches in flight on
+    # as many streams (no copies): how much of the end-to-end figure comes from
+    # running two searches at once rather than from the copies overlapping
+    Kc = 0 if (args.no_e2e or shard) else min(K, 500)
+    inflight = None
+    if Kc:
+        cstreams = [torch.cuda.Stream() for _ in range(E2E_INFLIGHT)]
+        couts = [(torch.empty((B, k), dtype=torch.int64, device=dev), torch.empty((B, k), dtype=torch.int32, device=dev))
+                 for _ in range(E2E_INFLIGHT)]
+
+        def conc_step(i):
+            j = i % E2E_INFLIGHT
+            idx.search(q[i % pool], m[i % pool], P, k, out_ids=couts[j][0], out_scores=couts[j][1], stream=cstreams[j])
+
+        for i in range(3 * E2E_INFLIGHT):
+            conc_step(i)
+        barrier(world)
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record()
+        for st_ in cstreams:
+            st_.wait_event(c0)
+        for i in range(Kc):
+            conc_step(i)
+        for st_ in cstreams:
+            torch.cuda.current_stream().wait_stream(st_)
+        c1.record()
+        torch.cuda.synchronize()
+        assert idx.check() == st.ST_OK
+        inflight = allreduce_sum(float(B * Kc), world) / (allreduce_max(c0.elapsed_time(c1), world) * 1e-3)
 
     # end to end through the host-buffer entry point (page-locked memory): a
     # serving loop with E2E_INFLIGHT batches in flight, one stream each, so one
@@ -470,6 +508,10 @@ def main():
             "e2e": {"value": e2e, "unit": "queries/s", "h2d_bytes_per_step": B * (d + 8 * W),
                     "d2h_bytes_per_step": B * k * 12,
                     "call": f"st_search_host_async, page-locked buffers, {E2E_INFLIGHT} batches in flight"},
+            "device_inflight": None if inflight is None else {
+                "value": inflight, "unit": "queries/s",
+                "note": f"device-resident searches, {E2E_INFLIGHT} batches in flight on {E2E_INFLIGHT} streams"},
+            "stage_sampling": f"stage events on one timed step in {stride} ({len(sampled)} of {K})",
             "gpu_launches": (KERNELS_PER_SEARCH + (1 if shard else 0)) * K,  # memset node not counted
             "clocks": clk,
             "workload_stats": {"scanned_items": float(np.mean([x[2] for x in models])),
