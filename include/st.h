@@ -340,7 +340,11 @@ st_status st_index_delete(st_index* idx, const int64_t* ids, int64_t m, cudaStre
  * id is its row, so ids are >= n (the creation rows), unique, never reused and
  * stable, but not consecutive: the unfilled rows of each list's last append
  * chunk are ids no call returned yet. ST_OPT_ID_OFFSET is added to them in
- * search results, like to every id. The item's Bloom bit-planes are written as
+ * search results, like to every id; on a document shard built from rows
+ * [r0, r1) of a collection, inserted ids land at r1 - r0 + offset and above,
+ * which may be ids of the next shard, so a sharded deployment needs its own
+ * id map for inserted items (or one shard that takes all insertions last in
+ * the id space). The item's Bloom bit-planes are written as
  * by st_index_update, and later searches on `stream` see it (other streams:
  * order them after this call). When the append chunks run out, the index
  * grows (the item, signature and plane arrays are copied once into arrays
