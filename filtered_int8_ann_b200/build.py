@@ -19,7 +19,7 @@ def sources():
 def up_to_date(out=OUT):
     if not os.path.exists(out):
         return False
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         [os.path.join(HERE, "..", "include", "st.h"), __file__]
     t = os.path.getmtime(out)
     return all(os.path.getmtime(p) <= t for p in deps)

@@ -7,6 +7,7 @@
 #include <new>
 #include <vector>
 
+#include "index_map.h"
 #include "st_internal.cuh"
 
 namespace st {
@@ -37,10 +38,7 @@ struct st_index {
     int32_t n_desc = 0, desc_cap = 0;
     int32_t* app_len = nullptr;      // [app_cap] rows filled in each append chunk
     int32_t app_used = 0, app_cap = 0;
-    std::vector<int64_t> off_host;                // creation offsets
-    std::vector<int32_t> base_cstart_host;        // creation chunk starts
-    std::vector<std::vector<int32_t>> list_app;   // append chunks of each list, in fill order
-    std::vector<int32_t> app_len_host;            // [app_used]
+    st::rowmap::Layout layout;       // host copy of where every row lives (creation lists, append chunks)
     int8_t* centroids = nullptr;
     uint32_t* err = nullptr;
     std::vector<int64_t> top_prefix;  // [p] = rows in the p largest lists
@@ -130,53 +128,14 @@ st::RowMap row_map(const st_index* idx)
     return m;
 }
 
-// The chunk table (list by list: creation chunks, then append chunks in fill
-// order), each list's first entry, and the two size prefixes the search sizes
-// its scratch with.
-struct Tables {
-    std::vector<int4> desc;
-    std::vector<int32_t> start;
-    std::vector<int64_t> top_prefix, top_chunks;
-};
-
-Tables build_tables(const st_index* idx, const std::vector<std::vector<int32_t>>& list_app,
-                    const std::vector<int32_t>& app_len)
-{
-    Tables t;
-    const int32_t nl = idx->nlist;
-    const int64_t Wi = st::kWarpItems;
-    t.start.assign(size_t(nl) + 1, 0);
-    std::vector<int64_t> rows(nl), chunks(nl);
-    for (int32_t c = 0; c < nl; ++c) {
-        t.start[c] = int32_t(t.desc.size());
-        const int64_t o0 = idx->off_host[c], nc = idx->off_host[c + 1] - o0;
-        int64_t r = nc;
-        for (int64_t j = 0; j * Wi < nc; ++j)
-            t.desc.push_back(make_int4(int(o0 + j * Wi), idx->base_cstart_host[c] + int(j), int(std::min(Wi, nc - j * Wi)), c));
-        for (int32_t a : list_app[c]) {
-            t.desc.push_back(make_int4(int(idx->n + Wi * a), idx->n_base_chunks + a, app_len[a], c));
-            r += app_len[a];
-        }
-        rows[c] = r;
-        chunks[c] = int64_t(t.desc.size()) - t.start[c];
-    }
-    t.start[nl] = int32_t(t.desc.size());
-    std::sort(rows.begin(), rows.end(), std::greater<int64_t>());
-    std::sort(chunks.begin(), chunks.end(), std::greater<int64_t>());
-    t.top_prefix.assign(size_t(nl) + 1, 0);
-    t.top_chunks.assign(size_t(nl) + 1, 0);
-    for (int32_t c = 0; c < nl; ++c) {
-        t.top_prefix[c + 1] = t.top_prefix[c] + rows[c];
-        t.top_chunks[c + 1] = t.top_chunks[c] + chunks[c];
-    }
-    return t;
-}
-
 // Copy the chunk table to the device (a larger array when it outgrew the old
 // one: the device is drained first, since earlier searches may still read it).
-cudaError_t upload_tables(st_index* idx, const Tables& t, cudaStream_t stream)
+cudaError_t upload_tables(st_index* idx, const st::rowmap::Tables& t, cudaStream_t stream)
 {
     const int32_t nd = int32_t(t.desc.size());
+    std::vector<int4> desc(t.desc.size());
+    for (size_t i = 0; i < desc.size(); ++i)
+        desc[i] = make_int4(t.desc[i].first_row, t.desc[i].plane_block, t.desc[i].rows, t.desc[i].list);
     if (nd > idx->desc_cap || idx->chunk_desc == nullptr) {
         const int32_t cap = std::max<int32_t>(std::max<int32_t>(nd, 1), idx->desc_cap + idx->desc_cap / 2);
         int4* fresh = nullptr;
@@ -192,13 +151,13 @@ cudaError_t upload_tables(st_index* idx, const Tables& t, cudaStream_t stream)
         idx->desc_cap = cap;
     }
     cudaError_t e = cudaSuccess;
-    if (nd > 0) e = cudaMemcpyAsync(idx->chunk_desc, t.desc.data(), size_t(nd) * sizeof(int4), cudaMemcpyHostToDevice, stream);
+    if (nd > 0) e = cudaMemcpyAsync(idx->chunk_desc, desc.data(), size_t(nd) * sizeof(int4), cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(idx->chunk_start, t.start.data(), t.start.size() * 4, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // the host vectors may go after this
     if (e == cudaSuccess) {
         idx->n_desc = nd;
-        idx->top_prefix = t.top_prefix;
+        idx->top_prefix = t.top_rows;
         idx->top_chunks = t.top_chunks;
     }
     return e;
@@ -501,10 +460,9 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(idx->centroids, centroids, size_t(nlist) * d, cudaMemcpyDefault, stream);
     // creation chunks: list c owns plane blocks cstart[c] .. cstart[c+1]-1
-    std::vector<int32_t> cstart(size_t(nlist) + 1, 0);
-    for (int32_t c = 0; c < nlist; ++c)
-        cstart[c + 1] = cstart[c] + int32_t((off[c + 1] - off[c] + st::kWarpItems - 1) / st::kWarpItems);
-    idx->n_base_chunks = cstart[nlist];
+    idx->layout = st::rowmap::make_layout(off, st::kWarpItems);
+    const std::vector<int32_t>& cstart = idx->layout.base_cstart;
+    idx->n_base_chunks = idx->layout.n_base_chunks;
     std::vector<int32_t> clist(size_t(idx->n_base_chunks > 0 ? idx->n_base_chunks : 1), 0);
     for (int32_t c = 0; c < nlist; ++c)
         for (int32_t t = cstart[c]; t < cstart[c + 1]; ++t) clist[t] = c;
@@ -524,11 +482,8 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         e = st::launch_build_planes(idx->sigs, idx->offsets, idx->base_chunk_start, idx->chunk_list,
                                     idx->n_base_chunks, sig_words, idx->planes, stream);
     }
-    idx->off_host = off;
-    idx->base_cstart_host = cstart;
-    idx->list_app.assign(size_t(nlist), std::vector<int32_t>());
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    if (e == cudaSuccess) e = upload_tables(idx, build_tables(idx, idx->list_app, idx->app_len_host), stream);
+    if (e == cudaSuccess) e = upload_tables(idx, st::rowmap::build_tables(idx->layout), stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(idx->err, 0, 256, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) {
@@ -816,23 +771,11 @@ st_status st_index_insert(st_index* idx, const int32_t* lists, const int8_t* ite
     if (m >= kIdLimit) return ST_ERR_UNSUPPORTED;
 
     // place the items on the host: each fills its list's last append chunk,
-    // then a fresh chunk
-    std::vector<std::vector<int32_t>> list_app = idx->list_app;
-    std::vector<int32_t> app_len = idx->app_len_host;
-    std::vector<int64_t> ids(static_cast<size_t>(m));
-    int64_t used = idx->app_used;
-    for (int64_t j = 0; j < m; ++j) {
-        std::vector<int32_t>& own = list_app[lists[j]];
-        if (own.empty() || app_len[own.back()] == st::kWarpItems) {
-            if (idx->n + (used + 1) * st::kWarpItems + idx->id_offset >= kIdLimit) return ST_ERR_UNSUPPORTED;
-            own.push_back(int32_t(used));
-            app_len.push_back(0);
-            ++used;
-        }
-        const int32_t a = own.back();
-        ids[j] = idx->n + int64_t(st::kWarpItems) * a + app_len[a];
-        ++app_len[a];
-    }
+    // then a fresh chunk (on a copy of the layout, kept only on success)
+    st::rowmap::Layout lay = idx->layout;
+    std::vector<int64_t> ids;
+    if (!st::rowmap::place(lay, lists, m, idx->id_offset, kIdLimit, ids)) return ST_ERR_UNSUPPORTED;
+    const int64_t used = lay.app_used();
     if (used > idx->app_cap) {
         // at least double the append room, within the id limit
         int64_t cap = std::max<int64_t>(used, 2 * int64_t(idx->app_cap));
@@ -841,7 +784,7 @@ st_status st_index_insert(st_index* idx, const int32_t* lists, const int8_t* ite
         const st_status gs = grow_rows(idx, int32_t(cap), stream);
         if (gs != ST_OK) return gs;
     }
-    const Tables t = build_tables(idx, list_app, app_len);
+    const st::rowmap::Tables t = st::rowmap::build_tables(lay);
 
     int64_t* dids = nullptr;
     cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&dids), size_t(m) * 8, idx->pool, stream);
@@ -852,7 +795,7 @@ st_status st_index_insert(st_index* idx, const int32_t* lists, const int8_t* ite
     e = cudaMemcpyAsync(dids, ids.data(), size_t(m) * 8, cudaMemcpyHostToDevice, stream);
     // the fill counts cover the new rows before the rows are written
     if (e == cudaSuccess)
-        e = cudaMemcpyAsync(idx->app_len, app_len.data(), app_len.size() * 4, cudaMemcpyHostToDevice, stream);
+        e = cudaMemcpyAsync(idx->app_len, lay.app_len.data(), lay.app_len.size() * 4, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) {
         st::RowMap map = row_map(idx);
         map.n_app = int32_t(used);
@@ -868,8 +811,7 @@ st_status st_index_insert(st_index* idx, const int32_t* lists, const int8_t* ite
         cudaGetLastError();
         return e == cudaErrorMemoryAllocation ? ST_ERR_OOM : ST_ERR_CUDA;
     }
-    idx->list_app = std::move(list_app);
-    idx->app_len_host = std::move(app_len);
+    idx->layout = std::move(lay);
     idx->app_used = int32_t(used);
     std::memcpy(out_ids, ids.data(), size_t(m) * 8);
     return ST_OK;
