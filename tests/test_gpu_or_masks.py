@@ -1,12 +1,16 @@
 """OR of several masks per query (Index.search_any: one search per alternative
-and st_merge_topk_union) against an independent numpy brute force that tests
-every alternative on every item of the probed lists."""
+and st_merge_topk_union) against two expected values that must agree: the
+oracle run once per alternative, its lists united by the plain definition
+(every item of the union's top-k is in the top-k of each alternative it
+passes), and an independent numpy brute force that tests every alternative on
+every item of the probed lists."""
 import numpy as np
 import pytest
 import torch
 
 import bruteforce as bf
 import filtered_int8_ann_b200 as st
+import oracle
 from workloads import small, to_numpy
 
 pytestmark = pytest.mark.gpu
@@ -28,6 +32,24 @@ def _bf_search_any(a, mask_sets, P, k):
         s = bf.scores(a["queries"][b][None, :], a["items"][rows])[0]
         o = bf.order_desc(s, rows)[:k]
         ids[b, :o.size], sc[b, :o.size] = rows[o], s[o]
+    return ids, sc
+
+
+def _oracle_search_any(a, mask_sets, P, k):
+    per = [oracle.search(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"], np.ascontiguousarray(ms),
+                         P, k, nthreads=oracle.max_threads()) for ms in mask_sets]
+    B = a["queries"].shape[0]
+    ids = np.full((B, k), -1, np.int64)
+    sc = np.full((B, k), np.iinfo(np.int32).min, np.int32)
+    for b in range(B):
+        pairs = {}
+        for r in per:
+            for i, s in zip(r[0][b], r[1][b]):
+                if i >= 0:
+                    pairs[int(i)] = int(s)
+        best = sorted(pairs.items(), key=lambda t: (-t[1], t[0]))[:k]
+        for j, (i, s) in enumerate(best):
+            ids[b, j], sc[b, j] = i, s
     return ids, sc
 
 
@@ -55,6 +77,8 @@ def test_or_of_masks_matches_brute_force(sig_bits):
         i1, s1 = idx.search(g.queries, g.masks, 6, 200)
     finally:
         idx.close()
-    exp = _bf_search_any(a, sets, 6, 200)
+    exp = _oracle_search_any(a, sets, 6, 200)
+    brute = _bf_search_any(a, sets, 6, 200)
+    assert np.array_equal(exp[0], brute[0]) and np.array_equal(exp[1], brute[1])
     assert np.array_equal(ids.cpu().numpy(), exp[0]) and np.array_equal(sc.cpu().numpy(), exp[1])
     assert np.array_equal(i2.cpu().numpy(), i1.cpu().numpy()) and np.array_equal(s2.cpu().numpy(), s1.cpu().numpy())
