@@ -233,6 +233,36 @@ def byte_model(data, probe, qmasks, W, d):
     return method, full, scanned, n_surv, int(lists.numel()), rowmajor, plane_bytes
 
 
+def bloom_fp(data, probe, q0):
+    """Bloom false positives of one batch: over every (query, item of a list
+    the query probes) pair, the items whose signature passes the query's mask
+    and the ones among them whose exact attributes do not match the query's
+    (language, country, required flags). Queries are rows q0 .. q0+B-1 of the
+    generated data. Returns (pairs passing the Bloom test, false positives,
+    exact matches that fail the Bloom test -- always 0: Bloom filters have no
+    false negatives)."""
+    off = data.offsets
+    sizes = off[1:] - off[:-1]
+    passed = fp = fn = 0
+    for b in range(probe.shape[0]):
+        lsb = probe[b].long()
+        starts, lens = off[lsb], sizes[lsb]
+        idx = torch.repeat_interleave(starts - torch.cumsum(lens, 0) + lens, lens) + torch.arange(
+            int(lens.sum()), device=off.device)
+        m = data.masks[q0 + b].view(1, -1)
+        ok = torch.all((data.sigs[idx] & m) == m, dim=1)
+        ql, qc, qf = int(data.q_lang[q0 + b]), int(data.q_country[q0 + b]), data.q_flags[q0 + b]
+        exact = torch.all(data.flags[idx] | ~qf.view(1, -1), dim=1)
+        if ql >= 0:
+            exact &= data.lang[idx] == ql
+        if qc >= 0:
+            exact &= data.country[idx] == qc
+        passed += int(ok.sum())
+        fp += int((ok & ~exact).sum())
+        fn += int((exact & ~ok).sum())
+    return passed, fp, fn
+
+
 def cpu_baseline(data, q, m, wl, budget_s):
     """The CPU oracle timed on the host cores over a bounded sample of the same
     workload: batches of one query per host thread, cycling through the query
@@ -343,6 +373,10 @@ def main():
         idx.search(q[b], m[b], P, k, out_ids=ids, out_scores=scores, eligible=elig[b], probe=probe[b])
     assert idx.check() == st.ST_OK
     models = [byte_model(data, probe[b], m[b], W, d) for b in range(pool)]
+    fp_stats = None
+    if hasattr(data, "lang"):  # the generator's exact attributes (not kept for a shard's arrays)
+        r0 = rank_query_rows(rank, B, pool)[0]
+        fp_stats = np.array([bloom_fp(data, probe[b], r0 + b * B) for b in range(pool)]).sum(0)
     elig_per_batch = elig.sum(1).double().cpu().numpy()
 
     cpu = None
@@ -517,7 +551,10 @@ def main():
             "workload_stats": {"scanned_items": float(np.mean([x[2] for x in models])),
                                "survivor_rows": float(np.mean([x[3] for x in models])),
                                "distinct_lists": float(np.mean([x[4] for x in models])),
-                               "eligible_per_query": float(elig_per_batch.mean() / B)},
+                               "eligible_per_query": float(elig_per_batch.mean() / B),
+                               "bloom_false_positive_rate": (None if fp_stats is None or fp_stats[0] == 0
+                                                             else float(fp_stats[1] / fp_stats[0])),
+                               "bloom_false_negatives": None if fp_stats is None else int(fp_stats[2])},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -1,0 +1,62 @@
+"""Host-side statistics of the benchmark on CPU tensors: the Bloom
+false-positive count it reports, against an independent numpy count over the
+same probed lists (the oracle's probe) and the generator's exact attributes."""
+import numpy as np
+import torch
+
+import bench
+import bruteforce as bf
+import oracle
+from workloads import small, to_numpy
+
+
+def _numpy_fp(data, a, lists_per_query):
+    lang, country, flags = data.lang.numpy(), data.country.numpy(), data.flags.numpy()
+    passed = fp = fn = 0
+    for b, lists in enumerate(lists_per_query):
+        rows = np.concatenate([np.arange(a["offsets"][c], a["offsets"][c + 1]) for c in lists])
+        ok = bf.bloom_pass(a["sigs"][rows], a["masks"][b])
+        exact = np.ones(rows.size, bool)
+        if int(data.q_lang[b]) >= 0:
+            exact &= lang[rows] == int(data.q_lang[b])
+        if int(data.q_country[b]) >= 0:
+            exact &= country[rows] == int(data.q_country[b])
+        for f in np.nonzero(data.q_flags[b].numpy())[0]:
+            exact &= flags[rows, f]
+        passed += int(ok.sum())
+        fp += int((ok & ~exact).sum())
+        fn += int((exact & ~ok).sum())
+    return passed, fp, fn
+
+
+def test_bloom_false_positive_count_matches_numpy():
+    for kw in (dict(n=6000, d=32, nlist=12, sig_bits=64, hash_bits=3, B=10, nprobe=4, k=50, seed=5,
+                    mask_country=True, mask_flags=2),
+               dict(n=5000, d=32, nlist=8, sig_bits=128, hash_bits=2, B=6, nprobe=3, k=50, seed=6,
+                    mask_mode="item", mask_country=True, mask_flags=1)):
+        data = small(**kw)
+        a = to_numpy(data)
+        lists = [oracle.probe(a["queries"][b], a["centroids"], kw["nprobe"]) for b in range(kw["B"])]
+        probe = torch.from_numpy(np.stack(lists))
+        got = bench.bloom_fp(data, probe, 0)
+        exp = _numpy_fp(data, a, lists)
+        assert got == exp
+        assert got[2] == 0  # no false negatives
+    # the 64-bit case has collisions: some false positives are expected
+    data = small(n=6000, d=32, nlist=12, sig_bits=64, hash_bits=3, B=10, nprobe=4, k=50, seed=5,
+                 mask_country=True, mask_flags=2)
+    a = to_numpy(data)
+    lists = [oracle.probe(a["queries"][b], a["centroids"], 4) for b in range(10)]
+    assert bench.bloom_fp(data, torch.from_numpy(np.stack(lists)), 0)[1] > 0
+
+
+def test_bloom_false_positive_count_uses_the_batch_rows():
+    """Batch b of the pool is rows q0 .. q0+B-1 of the generated queries."""
+    data = small(n=4000, d=32, nlist=8, sig_bits=64, hash_bits=3, B=12, nprobe=3, k=20, seed=7,
+                 mask_country=True, mask_flags=2)
+    a = to_numpy(data)
+    lists = [oracle.probe(a["queries"][b], a["centroids"], 3) for b in range(12)]
+    probe = torch.from_numpy(np.stack(lists))
+    whole = bench.bloom_fp(data, probe, 0)
+    halves = [bench.bloom_fp(data, probe[h * 6:(h + 1) * 6], h * 6) for h in range(2)]
+    assert tuple(x + y for x, y in zip(*halves)) == whole
