@@ -69,3 +69,17 @@ def test_search_rejects_null_index(lib):
     assert lib.st_merge_topk(fake, fake, 2, 1, 8192, fake, fake, None) == st.ST_ERR_UNSUPPORTED
     assert lib.st_index_set_option(None, 1, 5) == st.ST_ERR_INVALID_ARG
     lib.st_index_destroy(None)  # NULL-safe
+
+
+def test_freshness_and_host_calls_reject_null_index(lib):
+    fake = ctypes.c_void_p(16)
+    lists = (ctypes.c_int32 * 2)(0, 1)
+    ids = (ctypes.c_int64 * 2)()
+    L = lib  # argument types as the binding declares them
+    assert L.st_index_insert(None, ctypes.cast(lists, ctypes.c_void_p), fake, fake, 2,
+                             ctypes.cast(ids, ctypes.c_void_p), None) == st.ST_ERR_INVALID_ARG
+    assert L.st_index_update(None, fake, fake, fake, 2, None) == st.ST_ERR_INVALID_ARG
+    assert L.st_index_delete(None, fake, 2, None) == st.ST_ERR_INVALID_ARG
+    assert L.st_search_host_async(None, fake, fake, 1, 1, 1, fake, fake, None) == st.ST_ERR_INVALID_ARG
+    assert L.st_merge_topk_union(fake, fake, 0, 1, 1, fake, fake, None) == st.ST_ERR_INVALID_ARG
+    assert L.st_merge_topk_union(fake, fake, 4, 1, 8192, fake, fake, None) == st.ST_ERR_UNSUPPORTED
