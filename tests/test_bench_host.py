@@ -60,3 +60,15 @@ def test_bloom_false_positive_count_uses_the_batch_rows():
     whole = bench.bloom_fp(data, probe, 0)
     halves = [bench.bloom_fp(data, probe[h * 6:(h + 1) * 6], h * 6) for h in range(2)]
     assert tuple(x + y for x, y in zip(*halves)) == whole
+
+
+def test_cpu_baseline_reports_parallel_and_single_thread_rates():
+    data = small(n=3000, d=32, nlist=8, sig_bits=64, B=8, nprobe=3, k=20, seed=9)
+    q = data.queries.reshape(2, 4, -1)
+    m = data.masks.reshape(2, 4, -1)
+    wl = data.wl.with_(B=4)
+    cpu = bench.cpu_baseline(data, q, m, wl, 0.3)
+    assert cpu["kind"] == "oracle" and cpu["unit"] == "queries/s" and cpu["value"] > 0
+    assert cpu["cores"] == oracle.max_threads()
+    assert cpu["single_thread"]["value"] > 0 and cpu["single_thread"]["unit"] == "queries/s"
+    assert "cpu_model" in cpu
