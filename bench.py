@@ -7,10 +7,20 @@ batch of queries, inputs resident in HBM. Default workload: 80M items, d=64,
 k=2048. The timed steps cycle through a pool of distinct query batches; the
 index (6.4 GB) is far larger than L2.
 
+Besides the timed headline it reports, on the same GPU in the same run:
+  * the same search with the L2 flushed before every step (median of R);
+  * the roofline of the dominant kernel and of the whole step against HBM
+    bandwidth, the int8 tensor peak and the measured dp4a issue rate;
+  * recall@k of the IVF search against the flat filtered search;
+  * every other workload (tiny, mid, flat 10M, the 10M batch sweep at each B)
+    with the same figures (`per_config`);
+  * large k and streamed-update costs on the headline index.
+
 Prints one JSON line (rank 0). `--impl reference` times the CPU oracle instead
 (the reference arm; host cores only).
 """
 import argparse
+import ctypes
 import json
 import math
 import os
@@ -25,11 +35,19 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, generate  # noqa: E402
+from workloads import SWEEP_BATCHES, WORKLOADS, generate  # noqa: E402
 
 METRIC = "queries/s & item-scores/s (80M int8 IVF, nprobe64, top-2048); % HBM roofline"
-KERNELS_PER_SEARCH = 8  # probe score + probe select, units alloc + write, scan, select hist + scatter + finish
 E2E_INFLIGHT = 2  # query batches in flight in the end-to-end loop
+CHUNK_ROWS = 512  # rows per signature bit-plane chunk in the index
+FLUSH_BYTES = 512 << 20  # written between L2-flushed steps (L2 is 126 MB)
+
+
+def kernels_per_search(k):
+    """Kernels one search launches: probe score + select, units alloc + write,
+    scan, then select hist + scatter + finish (k <= 4096) or hist + scatter +
+    ties + rank (larger k). The memset node is not counted."""
+    return 8 if k <= 4096 else 9
 
 
 def parse():
@@ -44,6 +62,10 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip recall, large k, freshness and the other workloads")
+    p.add_argument("--config-steps", type=int, default=100, help="timed steps per other workload")
+    p.add_argument("--flush-reps", type=int, default=30, help="L2-flushed steps timed per workload")
     p.add_argument("--n", type=int, default=None, help="override the item count (profiling cases)")
     p.add_argument("--nlist", type=int, default=None, help="override the list count (profiling cases)")
     p.add_argument("--mode", default="replica", choices=["replica", "shard"],
@@ -52,31 +74,81 @@ def parse():
     return p.parse_args()
 
 
-def scan_traffic():
-    """DRAM bytes per scan launch from the committed ncu summary, if it was
+# ----------------------------------------------------------------------------
+# Peaks (roofline denominators)
+# ----------------------------------------------------------------------------
+class Peaks:
+    """HBM and bf16 tensor peaks measured on this machine's B200s (driver-written
+    MEASURED_PEAKS.json; else the pool's earlier measurement as a fallback);
+    the int8 tensor peak as 2x the measured bf16 dense peak (the nominal
+    int8 : bf16 ratio of the part, 4.5 : 2.25 PFLOP/s); the dp4a issue rate
+    measured here by the microbenchmark in filtered_int8_ann_b200/microbench."""
+
+    def __init__(self):
+        self.hbm_gbs, self.bf16_tflops, self.bf16_sustained, self.kind = 6650.0, 1590.0, 1400.0, "fallback"
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                j = json.load(f)
+            self.hbm_gbs = float(j["hbm_gbs"])
+            self.bf16_tflops = float(j.get("bf16_tflops", self.bf16_tflops))
+            self.bf16_sustained = float(j.get("bf16_tflops_sustained", self.bf16_sustained))
+            self.kind = "measured"
+        except Exception:
+            pass
+        self.int8_tensor_tops = 2.0 * self.bf16_tflops
+        self.dp4a_tops = self._dp4a()
+
+    @staticmethod
+    def _dp4a():
+        from filtered_int8_ann_b200 import build as libbuild
+        path = libbuild.PEAKS_OUT
+        if not os.path.exists(path):
+            return None
+        L = ctypes.CDLL(path)
+        L.st_peak_dp4a_tops.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+        L.st_peak_dp4a_tops.restype = ctypes.c_int
+        v = ctypes.c_double(0.0)
+        return float(v.value) if L.st_peak_dp4a_tops(5, ctypes.byref(v)) == 0 else None
+
+    def describe(self):
+        return {"hbm_gbs": self.hbm_gbs, "hbm_kind": self.kind,
+                "int8_tensor_tops": self.int8_tensor_tops,
+                "int8_tensor_kind": f"2 x bf16 dense {self.bf16_tflops:.0f} TFLOP/s ({self.kind}, burst)",
+                "dp4a_tops": self.dp4a_tops, "dp4a_kind": "measured (dp4a_peak.cu, 8 chains per thread)"}
+
+
+def roofline(bytes_, ops, ms, pk, compute="dp4a"):
+    """Bound times of one launch (or step) and the fraction of the slower bound
+    achieved. `compute` names the unit the int8 products ran on."""
+    t = ms * 1e-3
+    t_hbm = bytes_ / (pk.hbm_gbs * 1e9)
+    t_tensor = ops / (pk.int8_tensor_tops * 1e12)
+    t_dp4a = ops / (pk.dp4a_tops * 1e12) if pk.dp4a_tops else None
+    t_comp = t_dp4a if (compute == "dp4a" and t_dp4a is not None) else t_tensor
+    bound = "hbm" if t_hbm >= t_comp else ("alu" if compute == "dp4a" else "tensor")
+    return {"bound": bound, "frac": max(t_hbm, t_comp) / t if t > 0 else None,
+            "hbm_frac": t_hbm / t if t > 0 else None, "achieved_gbs": bytes_ / t / 1e9 if t > 0 else None,
+            "int8_tensor_frac": t_tensor / t if t > 0 else None,
+            "dp4a_frac": (t_dp4a / t) if (t_dp4a is not None and t > 0) else None,
+            "achieved_tops": ops / t / 1e12 if t > 0 else None}
+
+
+def scan_traffic(workload):
+    """DRAM bytes per scan launch from the committed ncu record, if it was
     measured on the scan source as it is now (else None)."""
     import hashlib
     try:
-        text = open(os.path.join(ROOT, "profiles", "scan_kernel_traffic_ivf_80m.md")).read()
-        fields = dict(l.split(": ", 1) for l in text.splitlines() if l.startswith(("source_sha256", "dram_bytes")))
+        with open(os.path.join(ROOT, "profiles", "scan_kernel_traffic.json")) as f:
+            rec = json.load(f)
         h = hashlib.sha256()
-        for f in ("scan.cu", "st_internal.cuh"):
-            with open(os.path.join(ROOT, "filtered_int8_ann_b200", "csrc", f), "rb") as fh:
+        for fn in rec["sources"]:
+            with open(os.path.join(ROOT, "filtered_int8_ann_b200", "csrc", fn), "rb") as fh:
                 h.update(fh.read())
-        if h.hexdigest() != fields["source_sha256"].strip():
+        if h.hexdigest() != rec["source_sha256"]:
             return None
-        return float(fields["dram_bytes_per_launch_mean"])
+        return float(rec["per_launch"][workload]["dram_bytes"])
     except Exception:
         return None
-
-
-def peaks():
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            j = json.load(f)
-        return float(j["hbm_gbs"]), "measured"
-    except Exception:
-        return 6650.0, "fallback"
 
 
 class Clocks:
@@ -121,6 +193,9 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------
+# Ranks
+# ----------------------------------------------------------------------------
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -168,14 +243,14 @@ def rank_query_rows(rank, B, pool):
     return rank * B * pool, (rank + 1) * B * pool
 
 
-def make_data(args, world, rank, device="cuda"):
-    wl = WORKLOADS[args.workload]
-    if args.n or args.nlist:
+def make_data(args, world, rank, device="cuda", name=None, B=None, pool=None):
+    wl = WORKLOADS[name or args.workload]
+    if name is None and (args.n or args.nlist):
         n = args.n or wl.n
         nl = args.nlist or wl.nlist
         wl = wl.with_(name=f"{wl.name}[n={n},nlist={nl}]", n=n, nlist=nl)
-    B = args.batch or wl.B
-    pool = max(1, args.pool)
+    B = B or args.batch or wl.B
+    pool = max(1, pool or args.pool)
     # every rank builds the same index; each draws its own query batches
     total_q = B * pool * world
     data = generate(wl.with_(B=total_q), device=device)
@@ -185,52 +260,69 @@ def make_data(args, world, rank, device="cuda"):
     return wl.with_(B=B), data, q, m
 
 
-CHUNK_ROWS = 512  # rows per signature bit-plane chunk in the index
+# ----------------------------------------------------------------------------
+# Byte and operation models
+# ----------------------------------------------------------------------------
+def _probed_rows(off, sizes, lists):
+    """Row indices of the lists `lists` (1-D), concatenated."""
+    starts, lens = off[lists], sizes[lists]
+    return torch.repeat_interleave(starts - torch.cumsum(lens, 0) + lens, lens) + torch.arange(
+        int(lens.sum()), device=off.device)
 
 
-def byte_model(data, probe, qmasks, W, d):
-    """Algorithmic bytes of one search's list scan, for the index layout the
-    library uses: every probed list is read once per batch; its signatures are
-    stored as bit-planes per 512-row chunk (64 bytes per plane), and the scan
-    needs, per chunk, the planes of the bits set in the union of the masks of
-    the queries probing the list; a row (d bytes) is read only when it is
-    eligible for at least one of those queries.
-    Also returned: the same model with row-major signatures (8W bytes for every
-    scanned row, the earlier layout) and the full-scan bytes (every row and
-    signature of every distinct probed list)."""
+def byte_model(data, probe, qmasks, W, d, k, nlist):
+    """Algorithmic bytes of one search (probe [B, P] of the batch).
+
+    Scan kernel, index layout of the library: every probed list is read once
+    per batch; its signatures are bit-planes per 512-row chunk (64 bytes per
+    plane) and a chunk needs the planes of the bits set in the union of the
+    masks of the queries probing the list; a row (d bytes) is read only when it
+    is eligible for at least one of those queries (`scan_planes`).
+    The same with row-major signatures (8W bytes for every scanned row), the
+    model the method's description implies (`scan_rowmajor`).
+    Whole step: the scan plus the centroids (nlist d), the queries and masks
+    (B (d + 8W)) and the outputs (B k 12) -- `step_planes`, `step_rowmajor`.
+    Full scan: every row and signature of every distinct probed list."""
     off = data.offsets
-    sizes = (off[1:] - off[:-1])
-    lists = torch.unique(probe.flatten())
+    sizes = off[1:] - off[:-1]
+    lists = torch.unique(probe.flatten().long())
     scanned = int(sizes[lists].sum())
-    # union of the masks of the queries probing each list
     pr = probe.long().cpu().numpy()
     mk = qmasks.cpu().numpy().view(np.uint64).reshape(qmasks.shape[0], -1)
-    nl = int(sizes.numel())
-    union = np.zeros((nl, mk.shape[1]), dtype=np.uint64)
+    union = np.zeros((sizes.numel(), mk.shape[1]), dtype=np.uint64)
     for w in range(mk.shape[1]):
         np.bitwise_or.at(union[:, w], pr.reshape(-1), np.repeat(mk[:, w], pr.shape[1]))
     ls = lists.cpu().numpy()
     bits = np.zeros(ls.size, dtype=np.int64)
     for w in range(mk.shape[1]):
-        u = union[ls, w]
-        bits += np.array([bin(int(x)).count("1") for x in u], dtype=np.int64)
+        bits += np.array([bin(int(x)).count("1") for x in union[ls, w]], dtype=np.int64)
     chunks = (sizes[lists].cpu().numpy() + CHUNK_ROWS - 1) // CHUNK_ROWS
     plane_bytes = int((chunks * bits * (CHUNK_ROWS // 8)).sum())
+    # rows eligible for at least one query probing their list, queries in
+    # groups of at most ~32M probed rows
     surv = torch.zeros(data.items.shape[0], dtype=torch.bool, device=off.device)
-    for b in range(probe.shape[0]):
-        lsb = probe[b].long()
-        starts, lens = off[lsb], sizes[lsb]
-        idx = torch.repeat_interleave(starts - torch.cumsum(lens, 0) + lens, lens) + torch.arange(
-            int(lens.sum()), device=off.device)
-        sg = data.sigs[idx]
-        m = qmasks[b].view(1, -1)
-        ok = torch.all((sg & m) == m, dim=1)
+    per_q = sizes[probe.long()].sum(1)
+    b0, B = 0, probe.shape[0]
+    while b0 < B:
+        b1, acc = b0, 0
+        while b1 < B and (b1 == b0 or acc + int(per_q[b1]) <= (32 << 20)):
+            acc += int(per_q[b1])
+            b1 += 1
+        pl = probe[b0:b1].long()
+        idx = _probed_rows(off, sizes, pl.reshape(-1))
+        owner = torch.repeat_interleave(torch.arange(b0, b1, device=off.device), sizes[pl].sum(1))
+        m = qmasks[owner]
+        ok = torch.all((data.sigs[idx] & m) == m, dim=1)
         surv[idx[ok]] = True
+        b0 = b1
     n_surv = int(surv.sum())
-    method = plane_bytes + d * n_surv
-    rowmajor = 8 * W * scanned + d * n_surv
-    full = (8 * W + d) * scanned
-    return method, full, scanned, n_surv, int(lists.numel()), rowmajor, plane_bytes
+    extra = nlist * d + B * (d + 8 * W) + B * k * 12
+    scan_planes = plane_bytes + d * n_surv
+    scan_rowmajor = 8 * W * scanned + d * n_surv
+    return {"scan_planes": scan_planes, "scan_rowmajor": scan_rowmajor,
+            "step_planes": scan_planes + extra, "step_rowmajor": scan_rowmajor + extra,
+            "full_scan": (8 * W + d) * scanned, "plane_bytes": plane_bytes,
+            "scanned_items": scanned, "survivor_rows": n_surv, "distinct_lists": int(lists.numel())}
 
 
 def bloom_fp(data, probe, q0):
@@ -245,10 +337,7 @@ def bloom_fp(data, probe, q0):
     sizes = off[1:] - off[:-1]
     passed = fp = fn = 0
     for b in range(probe.shape[0]):
-        lsb = probe[b].long()
-        starts, lens = off[lsb], sizes[lsb]
-        idx = torch.repeat_interleave(starts - torch.cumsum(lens, 0) + lens, lens) + torch.arange(
-            int(lens.sum()), device=off.device)
+        idx = _probed_rows(off, sizes, probe[b].long())
         m = data.masks[q0 + b].view(1, -1)
         ok = torch.all((data.sigs[idx] & m) == m, dim=1)
         ql, qc, qf = int(data.q_lang[q0 + b]), int(data.q_country[q0 + b]), data.q_flags[q0 + b]
@@ -360,6 +449,186 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# Timing helpers
+# ----------------------------------------------------------------------------
+def sampled_steps(K, pool):
+    """Steps that record stage events: one in `stride`, the stride coprime with
+    the batch pool so every batch is sampled equally. An event between two
+    kernels ends the programmatic dependent launch across it, so the other
+    steps run exactly as a caller's searches do."""
+    stride = next(s_ for s_ in range(3, 1000) if math.gcd(s_, pool) == 1)
+    return stride, list(range(0, K, stride))
+
+
+def stage_times(evs, sampled):
+    st_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in sampled])
+    return st_ms
+
+
+def flushed_steps(search, reps, flush):
+    """Median device time of one search with the L2 flushed before it: a
+    buffer larger than L2 is written between the timed searches, outside the
+    events."""
+    ts = []
+    pairs = []
+    for r in range(reps):
+        flush.fill_(r & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        search(r)
+        e1.record()
+        pairs.append((e0, e1))
+    torch.cuda.synchronize()
+    for e0, e1 in pairs:
+        ts.append(e0.elapsed_time(e1))
+    return float(statistics.median(ts))
+
+
+def recall(ivf_ids, flat_ids):
+    """Mean over queries of |IVF top-k ∩ flat top-k| / |flat top-k| (flat =
+    exact filtered search over every item)."""
+    r = []
+    for a, b in zip(ivf_ids, flat_ids):
+        fb = set(int(x) for x in b if x >= 0)
+        if fb:
+            r.append(len(fb & set(int(x) for x in a if x >= 0)) / len(fb))
+    return float(np.mean(r)) if r else None
+
+
+# ----------------------------------------------------------------------------
+# One workload measured the same way as the headline (used for per_config)
+# ----------------------------------------------------------------------------
+def measure_config(st, name, B, steps, warmup, flush_reps, flush, pk, pool=4, data=None, idx=None,
+                   recall_flat=False):
+    wl = WORKLOADS[name].with_(B=B)
+    own = data is None
+    if own:
+        data = generate(wl.with_(B=B * pool), device="cuda")
+        idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
+    q = data.queries[:B * pool].reshape(pool, B, -1).contiguous()
+    m = data.masks[:B * pool].reshape(pool, B, -1).contiguous()
+    P, k, d, W = wl.nprobe, wl.k, wl.d, wl.W
+    ids = torch.empty((B, k), dtype=torch.int64, device="cuda")
+    sc = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    elig = torch.empty((pool, B), dtype=torch.int64, device="cuda")
+    cands = torch.empty((pool, B), dtype=torch.int64, device="cuda")
+    probe = torch.empty((pool, B, P), dtype=torch.int32, device="cuda")
+    for b in range(pool):
+        idx.search(q[b], m[b], P, k, out_ids=ids, out_scores=sc, eligible=elig[b], probe=probe[b],
+                   candidates=cands[b])
+    assert idx.check() == st.ST_OK
+    models = [byte_model(data, probe[b], m[b], W, d, k, wl.nlist) for b in range(min(pool, 2))]
+    mdl = {key: float(np.mean([x[key] for x in models])) for key in models[0]}
+    for i in range(warmup):
+        idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=sc)
+    stride, sampled = sampled_steps(steps, pool)
+    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for i in sampled}
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s0.record()
+    for i in range(steps):
+        if i in evs:
+            idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=sc, stage_events=evs[i])
+        else:
+            idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=sc)
+    s1.record()
+    torch.cuda.synchronize()
+    assert idx.check() == st.ST_OK
+    ms = s0.elapsed_time(s1) / steps
+    stg = stage_times(evs, sampled).mean(0)
+    fl_ms = flushed_steps(lambda r: idx.search(q[r % pool], m[r % pool], P, k, out_ids=ids, out_scores=sc),
+                          flush_reps, flush)
+    el = float(elig.sum(1).double().mean())
+    ops_scan = 2.0 * d * el
+    ops_step = ops_scan + 2.0 * d * B * wl.nlist
+    out = {"workload": name, "B": B, "nprobe": P, "k": k, "n": wl.n, "d": d, "nlist": wl.nlist,
+           "queries_per_s": B / (ms * 1e-3), "item_scores_per_s": el / (ms * 1e-3), "ms_per_step": ms,
+           "l2_flushed": {"ms_per_step": fl_ms, "queries_per_s": B / (fl_ms * 1e-3)},
+           "stage_ms": {"probe": stg[0], "plan": stg[1], "scan": stg[2], "select": stg[3]},
+           "selectivity": el / max(1.0, float((data.offsets[1:] - data.offsets[:-1])[probe.long()]
+                                              .sum(2).double().mean()) * B),
+           "eligible_per_query": el / B,
+           "candidates_per_query": float(cands.double().mean()),
+           "candidate_bytes_per_step": float(cands.sum(1).double().mean()) * 8,
+           "bytes": mdl, "int8_ops": {"scan": ops_scan, "step": ops_step},
+           "scan_roofline": {"planes": roofline(mdl["scan_planes"], ops_scan, stg[2], pk),
+                             "rowmajor": roofline(mdl["scan_rowmajor"], ops_scan, stg[2], pk)},
+           "step_roofline": {"planes": roofline(mdl["step_planes"], ops_step, ms, pk),
+                             "rowmajor": roofline(mdl["step_rowmajor"], ops_step, ms, pk)},
+           "l2": f"steps cycle {pool} query batches; l2_flushed writes {FLUSH_BYTES >> 20} MB between steps"}
+    if recall_flat and P < wl.nlist <= 4096:
+        # flat filtered search = the same index probed with nprobe = nlist
+        idx.set_option(st.ST_OPT_CANDIDATE_BYTES, 12 << 30)
+        Bq = min(B, 64)
+        fids, _ = idx.search(q[0][:Bq].contiguous(), m[0][:Bq].contiguous(), wl.nlist, k)
+        vids, _ = idx.search(q[0][:Bq].contiguous(), m[0][:Bq].contiguous(), P, k)
+        idx.set_option(st.ST_OPT_CANDIDATE_BYTES, 2 << 30)
+        assert idx.check() == st.ST_OK
+        out["recall_at_k"] = {"value": recall(vids.cpu().numpy(), fids.cpu().numpy()), "queries": Bq,
+                              "flat": f"same index, nprobe = nlist = {wl.nlist}"}
+    if own:
+        idx.close()
+        del data
+        torch.cuda.empty_cache()
+    return out
+
+
+def freshness(st, idx, src_items, src_sigs, nlist, q, m, P, k, m_rows=100_000, batch=10_000):
+    """Streamed-update costs on a live index: rows/s of insertion (random
+    lists), in-place update and deletion of m_rows items, and the search time
+    before and after."""
+    ids = torch.empty((q.shape[1], k), dtype=torch.int64, device="cuda")
+    sc = torch.empty((q.shape[1], k), dtype=torch.int32, device="cuda")
+
+    def search_ms(reps=50):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(reps):
+            idx.search(q[i % q.shape[0]], m[i % m.shape[0]], P, k, out_ids=ids, out_scores=sc)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    before = search_ms()
+    rng = np.random.default_rng(7)
+    lists = rng.integers(0, nlist, m_rows).astype(np.int32)
+    # room for the insertions first (one copy of the index, untimed)
+    idx.set_option(st.ST_OPT_INSERT_RESERVE, int(min(nlist, m_rows)) * 512)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    new_ids = []
+    for b0 in range(0, m_rows, batch):
+        b1 = min(m_rows, b0 + batch)
+        new_ids.append(idx.insert(lists[b0:b1], src_items[b0:b1], src_sigs[b0:b1]))
+    t_ins = time.perf_counter() - t0
+    new_ids = torch.from_numpy(np.concatenate(new_ids)).cuda()
+    perm = torch.randperm(m_rows, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for b0 in range(0, m_rows, batch):
+        sel = perm[b0:b0 + batch]
+        idx.update(new_ids[sel], items=src_items[sel], sigs=src_sigs[sel])
+    torch.cuda.synchronize()
+    t_upd = time.perf_counter() - t0
+    after_insert = search_ms()
+    t0 = time.perf_counter()
+    for b0 in range(0, m_rows, batch):
+        idx.delete(new_ids[perm[b0:b0 + batch]])
+    torch.cuda.synchronize()
+    t_del = time.perf_counter() - t0
+    after_delete = search_ms()
+    assert idx.check() == st.ST_OK
+    return {"rows": m_rows, "batch": batch,
+            "insert_rows_per_s": m_rows / t_ins, "update_rows_per_s": m_rows / t_upd,
+            "delete_rows_per_s": m_rows / t_del,
+            "search_ms_before": before, "search_ms_after_insert": after_insert,
+            "search_ms_after_delete": after_delete,
+            "note": "host wall time per call sequence (insert waits for its stream); searches warm, cycling batches"}
+
+
+# ----------------------------------------------------------------------------
 def main():
     args = parse()
     if args.impl == "reference":
@@ -368,6 +637,8 @@ def main():
     import filtered_int8_ann_b200 as st
 
     shard = args.mode == "shard"
+    extras = (not args.no_extras) and world == 1 and not shard and args.n is None and args.nlist is None
+    pk = Peaks()
     # shards all search rank 0's batches; replicas search their own
     wl, data, q, m = make_data(args, 1 if shard else world, 0 if shard else rank)
     B, P, k, d, W = wl.B, wl.nprobe, wl.k, wl.d, wl.W
@@ -390,13 +661,15 @@ def main():
     ids = torch.empty((B, k), dtype=torch.int64, device=dev)
     scores = torch.empty((B, k), dtype=torch.int32, device=dev)
 
-    # per-batch eligible counts and byte model (untimed)
+    # per-batch eligible counts, candidates and byte model (untimed)
     elig = torch.empty((pool, B), dtype=torch.int64, device=dev)
+    cands = torch.empty((pool, B), dtype=torch.int64, device=dev)
     probe = torch.empty((pool, B, P), dtype=torch.int32, device=dev)
     for b in range(pool):
-        idx.search(q[b], m[b], P, k, out_ids=ids, out_scores=scores, eligible=elig[b], probe=probe[b])
+        idx.search(q[b], m[b], P, k, out_ids=ids, out_scores=scores, eligible=elig[b], probe=probe[b],
+                   candidates=cands[b])
     assert idx.check() == st.ST_OK
-    models = [byte_model(data, probe[b], m[b], W, d) for b in range(pool)]
+    models = [byte_model(data, probe[b], m[b], W, d, k, wl.nlist) for b in range(pool)]
     fp_stats = None
     if hasattr(data, "lang"):  # the generator's exact attributes (not kept for a shard's arrays)
         r0 = rank_query_rows(rank, B, pool)[0]
@@ -406,6 +679,15 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(data, q, m, wl, args.cpu_seconds)
+    # kept for the extras: the flat index (recall) and rows to insert
+    flat_src = None
+    if extras:
+        nsrc = 100_000
+        sel = torch.randint(0, data.items.shape[0], (nsrc,), device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+        flat_src = (data.items[sel].contiguous(), data.sigs[sel].contiguous())
+        flat_idx = st.Index(data.items, data.sigs,
+                            torch.tensor([0, data.items.shape[0]], dtype=torch.int64, device=dev),
+                            torch.zeros((1, d), dtype=torch.int8, device=dev))
     del data
     torch.cuda.empty_cache()
 
@@ -431,12 +713,7 @@ def main():
     torch.cuda.synchronize()
 
     K = args.steps
-    # stage events on every `stride`-th timed step only: an event between two
-    # kernels ends the programmatic dependent launch across it, so the other
-    # steps run exactly as a caller's searches do. The stride is coprime with
-    # the batch pool, so the sampled steps cover every batch equally.
-    stride = next(s_ for s_ in range(3, 1000) if math.gcd(s_, pool) == 1)
-    sampled = list(range(0, K, stride))
+    stride, sampled = sampled_steps(K, pool)
     evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for i in sampled}
     for row in evs.values():
         for e in row:
@@ -458,18 +735,24 @@ def main():
     ms_local = start.elapsed_time(end)
     ms = allreduce_max(ms_local, world)
 
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in sampled])
+    stage_ms = stage_times(evs, sampled)
     stage_mean = stage_ms.mean(0)
-    scan_ms = stage_mean[2]
-    method_bytes = np.array([models[i % pool][0] for i in sampled], dtype=np.float64)
-    full_bytes = np.array([models[i % pool][1] for i in sampled], dtype=np.float64)
-    scan_gbs = float(method_bytes.sum() / (stage_ms[:, 2].sum() * 1e-3) / 1e9)
-    peak, peak_kind = peaks()
+    scan_b = np.array([models[i % pool]["scan_planes"] for i in sampled], dtype=np.float64)
+    scan_gbs = float(scan_b.sum() / (stage_ms[:, 2].sum() * 1e-3) / 1e9)
+    scan_ms = float(stage_ms[:, 2].mean())
+    mean = {key: float(np.mean([x[key] for x in models])) for key in models[0]}
+    elig_mean = float(elig_per_batch.mean())
+    ops_scan = 2.0 * d * elig_mean
+    ops_step = ops_scan + 2.0 * d * B * wl.nlist
 
     # shards share one batch per step (their eligible counts add up); replicas each run their own
     total_q = float(B * K) if shard else allreduce_sum(float(B * K), world)
     elig_total = allreduce_sum(float(sum(elig_per_batch[i % pool] for i in range(K))), world)
     value = total_q / (ms * 1e-3)
+
+    # the same search with the L2 flushed before every step
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fl_ms = allreduce_max(flushed_steps(lambda r: step(r), args.flush_reps, flush), world)
 
     # the same device-resident searches with E2E_INFLIGHT batches in flight on
     # as many streams (no copies): how much of the end-to-end figure comes from
@@ -537,9 +820,68 @@ def main():
     torch.cuda.synchronize()
     ems = allreduce_max(e0.elapsed_time(e1), world)
     e2e = allreduce_sum(float(B * Ke), world) / (ems * 1e-3) if Ke else None
+
+    # ---- extras (1 GPU, replica mode, default workload sizes) --------------
+    ext = {}
+    if extras:
+        # recall of the IVF search (nprobe P) against the exact flat filtered search
+        flat_idx.set_option(st.ST_OPT_CANDIDATE_BYTES, 12 << 30)
+        fids, _ = flat_idx.search(q[0], m[0], 1, k)
+        assert flat_idx.check() == st.ST_OK
+        flat_idx.close()
+        idx.search(q[0], m[0], P, k, out_ids=ids, out_scores=scores)
+        ext["recall_at_k"] = {"value": recall(ids.cpu().numpy(), fids.cpu().numpy()), "queries": B,
+                              "flat": "index of one list holding every item, zero centroid, nprobe 1"}
+        del fids
+        # large k on the same index
+        lk = {}
+        for kk in (16384, 65536):
+            try:
+                li = torch.empty((B, kk), dtype=torch.int64, device=dev)
+                ls = torch.empty((B, kk), dtype=torch.int32, device=dev)
+                for i in range(3):
+                    idx.search(q[i % pool], m[i % pool], P, kk, out_ids=li, out_scores=ls)
+                torch.cuda.synchronize()
+                x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = 20
+                x0.record()
+                for i in range(reps):
+                    idx.search(q[i % pool], m[i % pool], P, kk, out_ids=li, out_scores=ls)
+                x1.record()
+                torch.cuda.synchronize()
+                assert idx.check() == st.ST_OK
+                t = x0.elapsed_time(x1) / reps
+                lk[str(kk)] = {"ms_per_step": t, "queries_per_s": B / (t * 1e-3)}
+                del li, ls
+            except st.StError as ex:
+                lk[str(kk)] = {"error": str(ex)}
+        ext["large_k"] = lk
+        # streamed updates, last: they change the headline index
+        ext["freshness"] = freshness(st, idx, flat_src[0], flat_src[1], wl.nlist, q, m, P, k)
+        del flat_src
     idx.close()
+    if extras:
+        torch.cuda.empty_cache()
+        # the other workloads
+        pc = []
+        for name in ("tiny_ivf", "mid_ivf", "flat_10m"):
+            wlx = WORKLOADS[name]
+            pc.append(measure_config(st, name, wlx.B, args.config_steps, 5, args.flush_reps, flush, pk))
+        sw = WORKLOADS["sweep_10m"]
+        pool_sw = 4
+        data_sw = generate(sw.with_(B=max(SWEEP_BATCHES) * pool_sw), device=dev)
+        idx_sw = st.Index(data_sw.items, data_sw.sigs, data_sw.offsets, data_sw.centroids)
+        for Bs in SWEEP_BATCHES:
+            pc.append(measure_config(st, "sweep_10m", Bs, args.config_steps if Bs < 1024 else max(20, args.config_steps // 4),
+                                     5, args.flush_reps, flush, pk, pool=pool_sw, data=data_sw, idx=idx_sw,
+                                     recall_flat=(Bs == 64)))
+        idx_sw.close()
+        del data_sw
+        ext["per_config"] = pc
 
     if rank == 0:
+        traffic = scan_traffic(wl.name)
+        scan_rf = roofline(mean["scan_planes"], ops_scan, scan_ms, pk)
         line = {
             "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
@@ -547,21 +889,30 @@ def main():
             "vs_baseline": None, "dtype": "int8/int32", "data": "synthetic",
             "config": {"workload": wl.name, "n": wl.n, "d": d, "nlist": wl.nlist, "B": B, "nprobe": P,
                        "k": k, "sig_bits": wl.sig_bits, "mask_mode": "head",
-                       "l2": f"inputs larger than L2 (index {wl.n * (d + 8 * W) / 1e9:.1f} GB); steps cycle {pool} distinct query batches",
+                       "l2": f"inputs larger than L2 (index {wl.n * (d + 8 * W) / 1e9:.1f} GB); steps cycle "
+                             f"{pool} distinct query batches; l2_flushed: {FLUSH_BYTES >> 20} MB written "
+                             f"before each of {args.flush_reps} steps",
                        "parallelism": (f"document shards x{world} (NCCL all-gather of the shards' top-k, exact merge)"
                                        if shard else f"replicas x{world} (independent query batches)")},
             "item_scores_per_s": elig_total / (ms * 1e-3),
+            "l2_flushed": {"ms_per_step": fl_ms, "queries_per_s": B / (fl_ms * 1e-3) * (1 if shard else world)},
             "stage_ms": {"probe": stage_mean[0], "plan": stage_mean[1], "scan": stage_mean[2],
                          "select": stage_mean[3]},
-            "roofline": {"bound": "hbm", "kernel": "scan_kernel", "achieved": scan_gbs, "peak": peak,
-                         "unit": "GB/s", "frac": scan_gbs / peak,
-                         "traffic": scan_traffic() if wl.name == "ivf_80m" else None,
-                         "peak_kind": peak_kind,
-                         "bytes_per_launch": float(method_bytes.mean()),
-                         "signature_plane_bytes_per_launch": float(np.mean([x[6] for x in models])),
-                         "rowmajor_model_bytes_per_launch": float(np.mean([x[5] for x in models])),
-                         "full_scan_bytes_per_launch": float(full_bytes.mean()),
-                         "step_frac": float(method_bytes.mean() / (ms / K * 1e-3) / 1e9 / peak)},
+            "roofline": {"bound": scan_rf["bound"], "kernel": "scan_kernel", "achieved": scan_gbs,
+                         "peak": pk.hbm_gbs, "unit": "GB/s", "frac": scan_gbs / pk.hbm_gbs,
+                         "traffic": traffic, "peak_kind": pk.kind,
+                         "bytes_per_launch": mean["scan_planes"],
+                         "int8_ops_per_launch": ops_scan,
+                         "int8_tensor_frac": scan_rf["int8_tensor_frac"], "dp4a_frac": scan_rf["dp4a_frac"],
+                         "signature_plane_bytes_per_launch": mean["plane_bytes"],
+                         "rowmajor_model_bytes_per_launch": mean["scan_rowmajor"],
+                         "rowmajor_model_frac": roofline(mean["scan_rowmajor"], ops_scan, scan_ms, pk)["hbm_frac"],
+                         "full_scan_bytes_per_launch": mean["full_scan"]},
+            "step_roofline": {"planes": roofline(mean["step_planes"], ops_step, ms / K, pk),
+                              "rowmajor": roofline(mean["step_rowmajor"], ops_step, ms / K, pk),
+                              "step_bytes_planes": mean["step_planes"], "step_bytes_rowmajor": mean["step_rowmajor"],
+                              "int8_ops_per_step": ops_step},
+            "peaks": pk.describe(),
             "cpu_baseline": cpu,
             "e2e": {"value": e2e, "unit": "queries/s", "h2d_bytes_per_step": B * (d + 8 * W),
                     "d2h_bytes_per_step": B * k * 12,
@@ -570,16 +921,21 @@ def main():
                 "value": inflight, "unit": "queries/s",
                 "note": f"device-resident searches, {E2E_INFLIGHT} batches in flight on {E2E_INFLIGHT} streams"},
             "stage_sampling": f"stage events on one timed step in {stride} ({len(sampled)} of {K})",
-            "gpu_launches": (KERNELS_PER_SEARCH + (1 if shard else 0)) * K,  # memset node not counted
+            "gpu_launches": (kernels_per_search(k) + (1 if shard else 0)) * K,
             "clocks": clk,
-            "workload_stats": {"scanned_items": float(np.mean([x[2] for x in models])),
-                               "survivor_rows": float(np.mean([x[3] for x in models])),
-                               "distinct_lists": float(np.mean([x[4] for x in models])),
-                               "eligible_per_query": float(elig_per_batch.mean() / B),
+            "workload_stats": {"scanned_items": mean["scanned_items"], "survivor_rows": mean["survivor_rows"],
+                               "distinct_lists": mean["distinct_lists"],
+                               "eligible_per_query": elig_mean / B,
+                               "candidates_per_query": float(cands.double().mean()),
+                               "candidate_bytes_per_step": float(cands.sum(1).double().mean()) * 8,
                                "bloom_false_positive_rate": (None if fp_stats is None or fp_stats[0] == 0
                                                              else float(fp_stats[1] / fp_stats[0])),
-                               "bloom_false_negatives": None if fp_stats is None else int(fp_stats[2])},
+                               "bloom_false_negatives": None if fp_stats is None else int(fp_stats[2]),
+                               **({"recall_at_k": ext["recall_at_k"]} if "recall_at_k" in ext else {})},
         }
+        for key in ("large_k", "freshness", "per_config"):
+            if key in ext:
+                line[key] = ext[key]
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

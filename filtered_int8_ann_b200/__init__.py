@@ -41,7 +41,8 @@ class StError(RuntimeError):
 
 class _Extras(ctypes.Structure):
     _fields_ = [("eligible", ctypes.c_void_p), ("probe", ctypes.c_void_p),
-                ("stage_events", ctypes.c_void_p * 5), ("exclude_masks", ctypes.c_void_p)]
+                ("stage_events", ctypes.c_void_p * 5), ("exclude_masks", ctypes.c_void_p),
+                ("candidates", ctypes.c_void_p)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -134,10 +135,11 @@ def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: i
               out_ids: Optional[torch.Tensor] = None, out_scores: Optional[torch.Tensor] = None,
               stream=None, eligible: Optional[torch.Tensor] = None,
               probe: Optional[torch.Tensor] = None, stage_events=None,
-              exclude: Optional[torch.Tensor] = None):
+              exclude: Optional[torch.Tensor] = None, candidates: Optional[torch.Tensor] = None):
     """Asynchronous search of device-resident queries; returns (ids int64 [B,k],
     scores int32 [B,k]). `eligible` [B] int64 and `probe` [B,nprobe] int32 are
-    optional extra outputs; `stage_events` is a list of up to five recorded
+    optional extra outputs, as is `candidates` [B] int64 (keys the scan wrote
+    for each query's final top-k); `stage_events` is a list of up to five recorded
     torch.cuda.Event objects marking the stage boundaries; `exclude` [B,W]
     holds per-query exclude masks (st_search_ex)."""
     qmasks = _as_words(qmasks)
@@ -149,13 +151,14 @@ def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: i
         out_scores = torch.empty((B, k), dtype=torch.int32, device=dev)
     if exclude is not None:
         exclude = _as_words(exclude)
-    if eligible is None and probe is None and not stage_events and exclude is None:
+    if eligible is None and probe is None and not stage_events and exclude is None and candidates is None:
         st = lib().st_search(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
                              _ptr(out_scores), _stream(stream))
         _check(st, "st_search")
     else:
         ex = _Extras(_ptr(eligible), _ptr(probe))
         ex.exclude_masks = _ptr(exclude)
+        ex.candidates = _ptr(candidates)
         for i, ev in enumerate(stage_events or ()):
             ex.stage_events[i] = ev.cuda_event if ev is not None else None
         st = lib().st_search_ex(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),

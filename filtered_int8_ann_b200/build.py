@@ -1,4 +1,5 @@
-"""Build libst.so (the C-ABI search library) in-tree for sm_100a with nvcc."""
+"""Build libst.so (the C-ABI search library) in-tree for sm_100a with nvcc, and
+libst_peaks.so (the dp4a peak microbenchmark the benchmark reports against)."""
 import glob
 import os
 import subprocess
@@ -7,6 +8,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libst.so")
+PEAKS_SRC = os.path.join(HERE, "microbench", "dp4a_peak.cu")
+PEAKS_OUT = os.path.join(HERE, "libst_peaks.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr"]
@@ -25,7 +28,15 @@ def up_to_date(out=OUT):
     return all(os.path.getmtime(p) <= t for p in deps)
 
 
+def build_peaks(force=False):
+    if force or not os.path.exists(PEAKS_OUT) or os.path.getmtime(PEAKS_SRC) > os.path.getmtime(PEAKS_OUT):
+        nvcc = os.environ.get("NVCC", "nvcc")
+        subprocess.run([nvcc, *ARCH, *FLAGS, PEAKS_SRC, "-o", PEAKS_OUT], check=True)
+    return PEAKS_OUT
+
+
 def build(force=False, verbose=False, out=OUT):
+    build_peaks(force)
     if not force and up_to_date(out):
         return out
     nvcc = os.environ.get("NVCC", "nvcc")

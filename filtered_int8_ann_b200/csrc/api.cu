@@ -330,6 +330,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.out_ids = out_ids;
     a.out_scores = out_scores;
     a.out_eligible = extras ? extras->eligible : nullptr;
+    a.out_cands = extras ? extras->candidates : nullptr;
     a.list_cnt = reinterpret_cast<int32_t*>(base + L.off_list_cnt);
     a.cand_cnt = reinterpret_cast<uint32_t*>(base + L.off_cand_cnt);
     a.eligible_cnt = reinterpret_cast<unsigned long long*>(base + L.off_elig);

@@ -397,6 +397,7 @@ select_kernel(SearchArgs a, int stage_cap)
         a.out_scores[int64_t(q) * k + r] = key_score(key);
     }
     if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
+    if (threadIdx.x == 0 && a.out_cands) a.out_cands[q] = int64_t(cnt);
 }
 
 // ----------------------------------------------------------------------------
@@ -448,6 +449,7 @@ select_rank_kernel(SearchArgs a)
     const int64_t n = a.cand_cnt[int64_t(q) * kCntStride] > 0 ? kept_count(a, q) : 0;
     const int m = n < k ? int(n) : k;
     if (p == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
+    if (p == 0 && a.out_cands) a.out_cands[q] = int64_t(a.cand_cnt[int64_t(q) * kCntStride]);
     if (p >= m) {
         a.out_ids[idx] = -1;
         a.out_scores[idx] = INT32_MIN;

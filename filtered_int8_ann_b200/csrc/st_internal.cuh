@@ -89,6 +89,7 @@ struct SearchArgs {
     int64_t* out_ids;
     int32_t* out_scores;
     int64_t* out_eligible;   // may be null
+    int64_t* out_cands;      // may be null: candidate keys written per query
     // scratch (the zeroed block first: one memset clears it)
     int32_t* list_cnt;       // [nlist] queries filed into each list      (zeroed)
     int32_t* probe_done;     // [B] probe slices finished per query       (zeroed)

@@ -124,6 +124,10 @@ typedef struct {
        of the pages' advertiser-defined targeting, tested like the mask itself
        (so a Bloom false positive excludes too). */
     const uint64_t* exclude_masks;
+    /* device int64 [B]: candidate keys the list scan wrote for each query's
+       final top-k (at most its eligible count; fewer when the scan dropped
+       keys that could no longer enter the top-k). */
+    int64_t* candidates;
 } st_search_extras;
 
 /* st_search with optional extra outputs (extras may be NULL). */

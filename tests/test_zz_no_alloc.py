@@ -100,3 +100,35 @@ def test_noalloc_probe_rejects_requests_beyond_its_scratch():
         assert np.array_equal(out_small.cpu().numpy(), _oracle_probe(a, range(40), 8))
     finally:
         idx.close()
+
+
+def test_noalloc_probe_leaves_free_device_memory_unchanged():
+    # Every index, input and output exists before the first reading; after one
+    # warm-up call per case (the first call on a device looks up the array's
+    # address and sets the kernel's shared-memory limit), repeated calls of
+    # every case -- the spill of centroid keys into the array included -- must
+    # not change the device's free memory as the driver reports it. The
+    # library does not allocate through torch, so torch's own counters would
+    # not show an allocation; cudaMemGetInfo does.
+    built = []
+    try:
+        for case in CASES:
+            g = small(**case).to(torch.device("cuda"))
+            idx = st.Index(g.items, g.sigs, g.offsets, g.centroids)
+            out = torch.empty((case["B"], case["nprobe"]), dtype=torch.int32, device="cuda")
+            built.append((idx, g, case["nprobe"], out))
+        for idx, g, P, out in built:
+            idx.probe_noalloc(g.queries, P, out)
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        for _ in range(5):
+            for idx, g, P, out in built:
+                idx.probe_noalloc(g.queries, P, out)
+        torch.cuda.synchronize()
+        free1 = torch.cuda.mem_get_info()[0]
+        for idx, _, _, _ in built:
+            assert idx.check() == st.ST_OK
+        assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
+    finally:
+        for idx, _, _, _ in built:
+            idx.close()
