@@ -43,11 +43,15 @@ CHUNK_ROWS = 512  # rows per signature bit-plane chunk in the index
 FLUSH_BYTES = 512 << 20  # written between L2-flushed steps (L2 is 126 MB)
 
 
-def kernels_per_search(k):
+def kernels_per_search(k, B, d):
     """Kernels one search launches: probe score + select, units alloc + write,
-    scan, then select hist + scatter + finish (k <= 4096) or hist + scatter +
-    ties + rank (larger k). The memset node is not counted."""
-    return 8 if k <= 4096 else 9
+    the warp scan, the tensor-core scan (when a list can have the dense-unit
+    threshold of queries: B >= that threshold, d = 64 or 128), then the
+    cluster final top-k (k <= 4096) or hist + scatter + ties + rank (larger
+    k). The memset node is not counted."""
+    dmq = 8 if DENSE_MIN_Q is None else DENSE_MIN_Q
+    tc = 1 if (d in (64, 128) and dmq > 0 and B >= dmq) else 0
+    return (6 if k <= 4096 else 9) + tc
 
 
 def parse():
@@ -68,6 +72,8 @@ def parse():
     p.add_argument("--flush-reps", type=int, default=30, help="L2-flushed steps timed per workload")
     p.add_argument("--n", type=int, default=None, help="override the item count (profiling cases)")
     p.add_argument("--nlist", type=int, default=None, help="override the list count (profiling cases)")
+    p.add_argument("--dense-min-queries", type=int, default=None,
+                   help="ST_OPT_DENSE_MIN_QUERIES for every index (default: the library's; 0 = no tensor-core scan)")
     p.add_argument("--mode", default="replica", choices=["replica", "shard"],
                    help="N>1: replicas search their own batches (default), or document shards search the "
                         "same batch, all-gather their top-k over NCCL and merge it exactly")
@@ -449,6 +455,16 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+DENSE_MIN_Q = None  # set from --dense-min-queries
+
+
+def open_index(st, items, sigs, offsets, centroids):
+    idx = st.Index(items, sigs, offsets, centroids)
+    if DENSE_MIN_Q is not None:
+        idx.set_option(st.ST_OPT_DENSE_MIN_QUERIES, DENSE_MIN_Q)
+    return idx
+
+
 # ----------------------------------------------------------------------------
 # Timing helpers
 # ----------------------------------------------------------------------------
@@ -505,7 +521,7 @@ def measure_config(st, name, B, steps, warmup, flush_reps, flush, pk, pool=4, da
     own = data is None
     if own:
         data = generate(wl.with_(B=B * pool), device="cuda")
-        idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
+        idx = open_index(st, data.items, data.sigs, data.offsets, data.centroids)
     q = data.queries[:B * pool].reshape(pool, B, -1).contiguous()
     m = data.masks[:B * pool].reshape(pool, B, -1).contiguous()
     P, k, d, W = wl.nprobe, wl.k, wl.d, wl.W
@@ -631,6 +647,8 @@ def freshness(st, idx, src_items, src_sigs, nlist, q, m, P, k, m_rows=100_000, b
 # ----------------------------------------------------------------------------
 def main():
     args = parse()
+    global DENSE_MIN_Q
+    DENSE_MIN_Q = args.dense_min_queries
     if args.impl == "reference":
         return run_reference(args)
     world, rank, local = dist_setup(args)
@@ -650,14 +668,14 @@ def main():
         it, sg, off, base = shard_arrays(data.items, data.sigs, data.offsets, world, rank)
         data = SimpleNamespace(items=it.contiguous(), sigs=sg.contiguous(), offsets=off, centroids=data.centroids,
                                queries=data.queries, masks=data.masks)
-        idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
+        idx = open_index(st, data.items, data.sigs, data.offsets, data.centroids)
         idx.set_option(st.ST_OPT_ID_OFFSET, base)
         g_ids = torch.empty((world, B, k), dtype=torch.int64, device=dev)
         g_sc = torch.empty((world, B, k), dtype=torch.int32, device=dev)
         m_ids = torch.empty((B, k), dtype=torch.int64, device=dev)
         m_sc = torch.empty((B, k), dtype=torch.int32, device=dev)
     else:
-        idx = st.Index(data.items, data.sigs, data.offsets, data.centroids)
+        idx = open_index(st, data.items, data.sigs, data.offsets, data.centroids)
     ids = torch.empty((B, k), dtype=torch.int64, device=dev)
     scores = torch.empty((B, k), dtype=torch.int32, device=dev)
 
@@ -685,7 +703,7 @@ def main():
         nsrc = 100_000
         sel = torch.randint(0, data.items.shape[0], (nsrc,), device=dev, generator=torch.Generator(device=dev).manual_seed(5))
         flat_src = (data.items[sel].contiguous(), data.sigs[sel].contiguous())
-        flat_idx = st.Index(data.items, data.sigs,
+        flat_idx = open_index(st, data.items, data.sigs,
                             torch.tensor([0, data.items.shape[0]], dtype=torch.int64, device=dev),
                             torch.zeros((1, d), dtype=torch.int8, device=dev))
     del data
@@ -870,7 +888,7 @@ def main():
         sw = WORKLOADS["sweep_10m"]
         pool_sw = 4
         data_sw = generate(sw.with_(B=max(SWEEP_BATCHES) * pool_sw), device=dev)
-        idx_sw = st.Index(data_sw.items, data_sw.sigs, data_sw.offsets, data_sw.centroids)
+        idx_sw = open_index(st, data_sw.items, data_sw.sigs, data_sw.offsets, data_sw.centroids)
         for Bs in SWEEP_BATCHES:
             pc.append(measure_config(st, "sweep_10m", Bs, args.config_steps if Bs < 1024 else max(20, args.config_steps // 4),
                                      5, args.flush_reps, flush, pk, pool=pool_sw, data=data_sw, idx=idx_sw,
@@ -921,7 +939,7 @@ def main():
                 "value": inflight, "unit": "queries/s",
                 "note": f"device-resident searches, {E2E_INFLIGHT} batches in flight on {E2E_INFLIGHT} streams"},
             "stage_sampling": f"stage events on one timed step in {stride} ({len(sampled)} of {K})",
-            "gpu_launches": (kernels_per_search(k) + (1 if shard else 0)) * K,
+            "gpu_launches": (kernels_per_search(k, B, d) + (1 if shard else 0)) * K,
             "clocks": clk,
             "workload_stats": {"scanned_items": mean["scanned_items"], "survivor_rows": mean["survivor_rows"],
                                "distinct_lists": mean["distinct_lists"],

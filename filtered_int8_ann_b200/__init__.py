@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libst.so")
 (ST_OK, ST_ERR_INVALID_ARG, ST_ERR_UNSUPPORTED, ST_ERR_OOM, ST_ERR_CUDA, ST_ERR_DEVICE,
  ST_ERR_SCRATCH_LIMIT) = range(7)
 ST_PROBE_NOALLOC_SCRATCH_BYTES = 16 << 20
-ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY, ST_OPT_ID_OFFSET, ST_OPT_INSERT_RESERVE = 1, 2, 3, 4
+(ST_OPT_CANDIDATE_BYTES, ST_OPT_CANDIDATE_CAPACITY, ST_OPT_ID_OFFSET, ST_OPT_INSERT_RESERVE,
+ ST_OPT_DENSE_MIN_QUERIES) = 1, 2, 3, 4, 5
 ST_INSERT_CHUNK = 512
 ST_MERGE_MAX_KEYS = 16384
 ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K, ST_MAX_B = 512, 262144, 4096, 4096, 32768

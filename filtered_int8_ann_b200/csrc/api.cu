@@ -2,6 +2,7 @@
 // library-owned index copy, stream-ordered scratch, and the kernel sequence
 // memset -> probe -> plan -> scan -> select of one search.
 #include <algorithm>
+#include <cuda.h>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -48,6 +49,9 @@ struct st_index {
     int64_t cand_cap_override = 0;
     int64_t id_offset = 0;
     uint32_t* dead = nullptr;        // [ceil(rows_alloc / 32)] deletion bitmap, allocated at the first deletion
+    CUtensorMap tmap;                // the item rows as a 2-D tensor (TMA tile loads of the dense scan)
+    bool tmap_ok = false;
+    int32_t tc_min_q = st::kTcMinQDefault;  // queries per list from which its units are dense
 };
 
 namespace st {
@@ -126,6 +130,40 @@ st::RowMap row_map(const st_index* idx)
     m.app_len = idx->app_len;
     m.n_app = idx->app_used;
     return m;
+}
+
+// The item rows [rows_alloc][d] as a 2-D uint8 tensor for TMA tile loads of
+// 32 rows x d bytes into the dense scan's swizzled layout (128-byte swizzle for
+// d = 128, 64-byte for d = 64). Other d have no dense scan.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_items_tmap(st_index* idx)
+{
+    idx->tmap_ok = false;
+    if (!st::scan_tc_supported(idx->d)) return false;
+    static EncodeTiledFn encode = nullptr;
+    if (encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr) {
+            cudaGetLastError();
+            return false;
+        }
+        encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    const cuuint64_t dims[2] = {cuuint64_t(idx->d), cuuint64_t(idx->rows_alloc)};
+    const cuuint64_t strides[1] = {cuuint64_t(idx->d)};
+    const cuuint32_t box[2] = {cuuint32_t(idx->d), 32};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(&idx->tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, idx->items, dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              idx->d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    idx->tmap_ok = (r == CUDA_SUCCESS);
+    return idx->tmap_ok;
 }
 
 // Copy the chunk table to the device (a larger array when it outgrew the old
@@ -221,6 +259,7 @@ st_status grow_rows(st_index* idx, int32_t app_cap, cudaStream_t stream)
     release();  // the old arrays
     idx->app_cap = app_cap;
     idx->rows_alloc = rows;
+    make_items_tmap(idx);  // the rows moved
     return ST_OK;
 }
 
@@ -228,7 +267,8 @@ st_status grow_rows(st_index* idx, int32_t app_cap, cudaStream_t stream)
 // must start at zero come first, so one memset clears them.
 struct ScratchLayout {
     size_t total = 0;
-    size_t off_list_cnt, off_cand_cnt, off_elig, off_rng, off_sel_hist, off_sel_cursor, off_ctl, zero_bytes;
+    size_t off_list_cnt, off_cand_cnt, off_elig, off_rng, off_sel_hist, off_sel_cursor, off_ctl, off_tc_hist, zero_bytes;
+    size_t off_units_tc, off_qscale;
     size_t off_sel_out, off_sel_tie;
     size_t off_probe, off_probe_keys, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_units, off_cand;
     size_t add(size_t bytes)
@@ -288,6 +328,8 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_sel_hist = L.add(size_t(B) * st::kSelBins * 4);
     L.off_sel_cursor = L.add(size_t(B) * st::kSelBins * 4);
     L.off_ctl = L.add(sizeof(st::PlanCtl));
+    const int tc_min_q = (idx->tmap_ok && idx->tc_min_q > 0 && B >= idx->tc_min_q) ? idx->tc_min_q : 0;
+    L.off_tc_hist = L.add(tc_min_q ? size_t(B) * st::kTcBins * 4 : 0);
     L.zero_bytes = L.total;
     L.off_probe = L.add(size_t(B) * nprobe * 4);
     L.off_probe_keys = L.add(size_t(B) * size_t(st::probe_keys_ld(idx->nlist)) * 8);
@@ -297,6 +339,8 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_qlist = L.add(slots * 4);
     L.off_qmask = L.add(slots * 16);
     L.off_units = L.add(size_t(max_units) * 16);
+    L.off_units_tc = L.add(tc_min_q ? size_t(max_units) * 16 : 0);
+    L.off_qscale = L.add(tc_min_q ? size_t(B) * 8 : 0);
     L.off_cand = L.add(size_t(B) * size_t(cap) * 8);
     L.off_sel_out = L.add(size_t(B) * size_t(k) * 8);
     L.off_sel_tie = L.add(size_t(B) * st::kSelTieCap * 8);
@@ -347,6 +391,12 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.qmask_slot = reinterpret_cast<uint64_t*>(base + L.off_qmask);
     a.units = reinterpret_cast<int4*>(base + L.off_units);
     a.max_units = int32_t(max_units);
+    a.tc_min_q = tc_min_q;
+    if (tc_min_q) {
+        a.units_tc = reinterpret_cast<int4*>(base + L.off_units_tc);
+        a.qscale = reinterpret_cast<int2*>(base + L.off_qscale);
+        a.tc_hist = reinterpret_cast<uint32_t*>(base + L.off_tc_hist);
+    }
     a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
     a.cap = cap;
     a.id_offset = idx->id_offset;
@@ -366,6 +416,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     if (e == cudaSuccess) e = st::launch_plan(a, idx->num_sms, stream);
     mark(2);
     if (e == cudaSuccess) e = st::launch_scan(a, idx->num_sms, stream);
+    if (e == cudaSuccess && tc_min_q) e = st::launch_scan_tc(a, &idx->tmap, idx->num_sms, stream);
     mark(3);
     if (e == cudaSuccess) e = st::launch_select(a, idx->num_sms, stream);
     mark(4);
@@ -484,6 +535,7 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
                                     idx->n_base_chunks, sig_words, idx->planes, stream);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess) make_items_tmap(idx);
     if (e == cudaSuccess) e = upload_tables(idx, st::rowmap::build_tables(idx->layout), stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(idx->err, 0, 256, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
@@ -745,6 +797,10 @@ st_status st_index_set_option(st_index* idx, st_option opt, int64_t value)
     case ST_OPT_ID_OFFSET:
         if (value >= kIdLimit || value + idx->rows_alloc >= kIdLimit) return ST_ERR_UNSUPPORTED;
         idx->id_offset = value;
+        return ST_OK;
+    case ST_OPT_DENSE_MIN_QUERIES:
+        if (value > ST_MAX_B) return ST_ERR_INVALID_ARG;
+        idx->tc_min_q = int32_t(value);
         return ST_OK;
     case ST_OPT_INSERT_RESERVE: {
         if (value == 0) return ST_OK;

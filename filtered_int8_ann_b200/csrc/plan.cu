@@ -1,7 +1,10 @@
-// Plan: cut every probed list into warp work units of kWarpItems rows x a
-// group of up to kQMax of the queries probing it, so the scan reads each probed
-// list once per batch however many queries probe it. One self-contained
-// 16-byte entry per unit: {first row, chunk, first query slot, rows << 16 | queries}.
+// Plan: cut every probed list into work units of kWarpItems rows x a group of
+// the queries probing it, so the scan reads each probed list once per batch
+// however many queries probe it. One self-contained 16-byte entry per unit:
+// {first row, chunk, first query slot, rows << 16 | queries}. Lists probed by
+// fewer than tc_min_q queries get groups of up to kQMax queries, scanned by
+// one warp each (scan.cu); lists probed by more get groups of up to kTcQMax
+// queries in a second table, scanned as dense tensor-core tiles (scan_tc.cu).
 //
 // The probe kernel already filed each query into the slot row of every list it
 // chose (slots L*B .. L*B + count-1), so no scan over lists or scatter of pairs
@@ -19,6 +22,12 @@ namespace st {
 
 constexpr int kUnitsBlock = 256;
 
+// A list's units go to the tensor-core scan when enough queries probe it.
+__device__ __forceinline__ bool dense_list(const SearchArgs& a, int cnt)
+{
+    return a.tc_min_q > 0 && cnt >= a.tc_min_q;
+}
+
 __global__ void __launch_bounds__(kUnitsBlock)
 units_alloc_kernel(SearchArgs a)
 {
@@ -26,26 +35,42 @@ units_alloc_kernel(SearchArgs a)
     const int lane = threadIdx.x & 31;
     const int L = blockIdx.x * kUnitsBlock + threadIdx.x;
     uint32_t u = 0;
+    bool dense = false;
     if (L < a.nlist) {
         const int cnt = a.list_cnt[L];
-        if (cnt > 0)
-            u = uint32_t(a.chunk_start[L + 1] - a.chunk_start[L]) * uint32_t((cnt + kQMax - 1) / kQMax);
+        if (cnt > 0) {
+            dense = dense_list(a, cnt);
+            const int qg = dense ? kTcQMax : kQMax;
+            u = uint32_t(a.chunk_start[L + 1] - a.chunk_start[L]) * uint32_t((cnt + qg - 1) / qg);
+        }
     }
-    uint32_t incl = u;
+    // one warp-wide scan per table (sparse, dense)
+    const uint32_t us = dense ? 0u : u, ud = dense ? u : 0u;
+    uint32_t is = us, id = ud;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
+        const uint32_t ts = __shfl_up_sync(0xffffffffu, is, off), td = __shfl_up_sync(0xffffffffu, id, off);
+        if (lane >= off) {
+            is += ts;
+            id += td;
+        }
     }
-    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
-    if (total == 0u) return;  // warp-uniform
-    uint32_t base = 0;
+    const uint32_t tot_s = __shfl_sync(0xffffffffu, is, 31), tot_d = __shfl_sync(0xffffffffu, id, 31);
+    if (tot_s + tot_d == 0u) return;  // warp-uniform
+    uint32_t bs = 0, bd = 0;
     if (lane == 31) {
-        base = atomicAdd(reinterpret_cast<unsigned int*>(&a.ctl->n_units), total);
-        if (uint64_t(base) + total > uint64_t(a.max_units)) set_error(a.err, kErrUnitTable);
+        if (tot_s) {
+            bs = atomicAdd(reinterpret_cast<unsigned int*>(&a.ctl->n_units), tot_s);
+            if (uint64_t(bs) + tot_s > uint64_t(a.max_units)) set_error(a.err, kErrUnitTable);
+        }
+        if (tot_d) {
+            bd = atomicAdd(reinterpret_cast<unsigned int*>(&a.ctl->n_dense), tot_d);
+            if (uint64_t(bd) + tot_d > uint64_t(a.max_units)) set_error(a.err, kErrUnitTable);
+        }
     }
-    base = __shfl_sync(0xffffffffu, base, 31);
-    if (u > 0) a.list_ustart[L] = int32_t(base + incl - u);
+    bs = __shfl_sync(0xffffffffu, bs, 31);
+    bd = __shfl_sync(0xffffffffu, bd, 31);
+    if (u > 0) a.list_ustart[L] = dense ? int32_t(bd + id - ud) : int32_t(bs + is - us);
 }
 
 __global__ void __launch_bounds__(kUnitsBlock)
@@ -77,12 +102,14 @@ units_write_kernel(SearchArgs a)
         unit = make_int4(0, 0, 0, 0);
     }
     const int64_t base = a.list_ustart[L];
-    const int groups = (cnt + kQMax - 1) / kQMax;
+    const bool dense = dense_list(a, cnt);
+    const int qg = dense ? kTcQMax : kQMax;
+    int4* table = dense ? a.units_tc : a.units;
+    const int groups = (cnt + qg - 1) / qg;
     for (int g = 0; g < groups; ++g) {
         const int64_t idx = base + int64_t(g) * nch + ci;
         if (idx < a.max_units)
-            a.units[idx] = make_int4(unit.x, unit.y, L * a.B + g * kQMax,
-                                     (unit.w << 16) | min(kQMax, cnt - g * kQMax));
+            table[idx] = make_int4(unit.x, unit.y, L * a.B + g * qg, (unit.w << 16) | min(qg, cnt - g * qg));
     }
 }
 

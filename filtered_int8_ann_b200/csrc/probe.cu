@@ -58,6 +58,21 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
         }
         if (lane == 0) a.qnbits[b] = n_before;
     }
+    if (a.qscale != nullptr && threadIdx.x >= 32 && threadIdx.x < 64) {
+        // bound of the query's scores for the dense scan's score bins:
+        // |<q, x>| <= S = 128 * sum_j |q_j| for any int8 row x
+        const int lane = threadIdx.x - 32;
+        const int8_t* qv = a.queries + int64_t(b) * a.d;
+        int32_t sum = 0;
+        for (int j = lane; j < a.d; j += 32) sum += abs(int32_t(qv[j]));
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) {
+            const int32_t S = 128 * sum;
+            int sh = 0;
+            while (((int64_t(2) * S) >> sh) >= kTcBins) ++sh;
+            a.qscale[b] = make_int2(-S, sh);
+        }
+    }
     for (int p = threadIdx.x; p < P; p += BLOCK) {
         const int L = int(key_id(sorted[p]));
         a.probe[int64_t(b) * P + p] = L;

@@ -1,135 +1,34 @@
-// Final top-k: one CTA per query picks the k best candidate keys and writes
-// them ordered by score descending, then item id ascending, padded with
-// (id -1, score INT32_MIN) when fewer than k items were eligible.
+// Final top-k for k above ST_SMALL_K (k <= ST_SMALL_K: select_cluster.cu):
+// the k best candidate keys of each query, ordered by score descending, then
+// item id ascending, padded with (id -1, score INT32_MIN) when fewer than k
+// items were eligible.
 //
-// A large result (2048 per query from 64 probes, with recall kept) drawn from a
-// large candidate pool --
-// SilverTorch: Index as Model, section on redesigning each stage as a pure
-// PyTorch module, fused Int8 ANN paragraph; maximum top-k row of the cost
-// efficiency table in the Spanish translation.
+// A large result drawn from a large candidate pool -- SilverTorch: Index as
+// Model, section on redesigning each stage as a pure PyTorch module, fused
+// Int8 ANN paragraph; maximum top-k row of the cost efficiency table in the
+// Spanish translation (a count in the hundreds of thousands).
 //
-// Three kernels, so that a query with a hundred thousand candidates is spread
-// over many SMs instead of holding one: the candidates of every query are cut
+// Four kernels, all in global memory, so that a query with a hundred thousand
+// candidates is spread over many SMs: the candidates of every query are cut
 // into chunks of kChunk keys, and
 //   * select_hist_kernel: each chunk's keys go into a 2048-bin histogram of
 //     their scores over the query's score range (recorded by the scan),
-//     added into the query's histogram;
-//   * select_scatter_kernel: from that histogram every chunk finds the same
-//     cut bin (the one holding the k-th best score) and the output segment of
-//     each bin above it, and writes its keys of those bins into their segments;
-//     the cut bin's keys are gathered aside;
-//   * select_kernel: one CTA per query takes the cut bin's best, orders every
-//     segment (each key's rank among its segment's keys) and writes ids and
-//     scores. A query whose candidates overflowed the scan's buffer takes the
-//     exact overflow path instead, all in this kernel.
-// Exact overflow path: when the scan reserved more candidates for a query than
-// its buffer holds, this CTA rescans that query's probed lists itself with the
-// bounded buffer: whenever the buffer fills it keeps only the k best keys and
-// from then on drops any key below the k-th, which can no longer enter the
-// top-k. Exact for any input, with memory bounded by the capacity; slow, and
-// used only on overflow.
-#include "st_internal.cuh"
+//     added into the query's histogram; the query's last chunk finds the cut
+//     bin (the one holding the k-th best score) and each higher bin's output
+//     segment;
+//   * select_scatter_kernel: every chunk writes its keys of the bins above the
+//     cut into their segments; the cut bin's keys are gathered aside;
+//   * select_ties_kernel: one CTA per query takes the cut bin's best;
+//   * select_rank_kernel: one thread per output position ranks its key in
+//     its segment and writes the id and score.
+// The scan reserves room for every row of the probed lists when k is this
+// large, so there is no overflow path here.
+#include "select_common.cuh"
 
 namespace st {
 
-template <int BLOCK>
-__device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, int pwk, int4* s_qv,
-                                 SelectSmem& ss)
-{
-    __shared__ int32_t s_count;
-    __shared__ uint64_t s_thr;
-    const int d = a.d, np = d >> 4, W = a.W, k = a.k;
-    uint64_t* buf = a.cand + int64_t(q) * a.cap;
-    const int64_t cap = a.cap;  // host guarantees cap >= k + BLOCK
-    for (int p = threadIdx.x; p < np; p += BLOCK)
-        s_qv[p] = reinterpret_cast<const int4*>(a.queries + int64_t(q) * d)[p];
-    const uint64_t m0 = a.qmasks[int64_t(q) * W];
-    const uint64_t m1 = W > 1 ? a.qmasks[int64_t(q) * W + 1] : 0ull;
-    if (threadIdx.x == 0) {
-        s_count = 0;
-        s_thr = 0;
-    }
-    __syncthreads();
-    for (int p = 0; p < a.P; ++p) {
-        const int L = a.probe[int64_t(q) * a.P + p];
-        if (L < 0 || L >= a.nlist) {
-            if (threadIdx.x == 0) set_error(a.err, kErrOverflowPath);
-            continue;
-        }
-        // the list's chunks: its creation rows, then its append chunks
-        const int t0 = a.chunk_start[L], t1 = a.chunk_start[L + 1];
-        for (int t = t0; t < t1; ++t) {
-            const int4 c = a.chunk_desc[t];  // {first row, plane block, rows, list}
-            if (c.w != L || c.z < 0 || c.z > kWarpItems || c.x < 0 || int64_t(c.x) + c.z > a.n_rows) {
-                if (threadIdx.x == 0) set_error(a.err, kErrOverflowPath);
-                continue;
-            }
-            const int64_t o0 = c.x, o1 = int64_t(c.x) + c.z;
-            for (int64_t base = o0; base < o1; base += BLOCK) {
-                if (int64_t(s_count) + BLOCK > cap) {
-                    // keep the k best, drop everything below them from now on
-                    const int64_t cnt = s_count;
-                    const uint64_t thr = block_select_threshold<BLOCK>(buf, cnt, k, ss, a.err);
-                    const int32_t got = block_collect_ge<BLOCK>(buf, cnt, thr, sortbuf, pwk, ss);  // unsorted is fine here
-                    if (threadIdx.x == 0 && got != k) set_error(a.err, kErrOverflowPath);
-                    for (int i = threadIdx.x; i < k; i += BLOCK) buf[i] = sortbuf[i];
-                    if (threadIdx.x == 0) {
-                        s_count = k;
-                        s_thr = thr;
-                    }
-                    __syncthreads();
-                }
-                const int64_t i = base + threadIdx.x;
-                const uint64_t thr = s_thr;
-                bool keep = false;
-                uint64_t key = 0;
-                if (i < o1) {
-                    const uint64_t* sg = a.sigs + i * W;
-                    bool pass = (sg[0] & m0) == m0;
-                    if (W > 1) pass = pass && ((sg[1] & m1) == m1);
-                    pass = pass && keep_item(a, q, i);
-                    if (pass) {
-                        const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);
-                        int32_t acc = 0;
-                        for (int j = 0; j < np; ++j) acc = dot16(__ldg(rp + j), s_qv[j], acc);
-                        key = pack_key(acc, uint32_t(i));
-                        keep = key >= thr;
-                    }
-                }
-                const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                if (bal) {
-                    int32_t b0 = 0;
-                    if ((threadIdx.x & 31) == 0) b0 = atomicAdd(&s_count, __popc(bal));
-                    b0 = __shfl_sync(0xffffffffu, b0, 0);
-                    if (keep) buf[b0 + __popc(bal & lanemask_lt())] = key;
-                }
-                __syncthreads();
-            }
-        }
-    }
-    return s_count;
-}
-
 constexpr int kChunk = 4096;      // candidates per histogram / scatter item
 constexpr int kChunkBlock = 512;
-constexpr int kSelectTieCapSmem = 1024;
-
-// The query's score range (a superset of its candidates' scores)
-__device__ __forceinline__ void query_range(const SearchArgs& a, int q, int32_t& lo, uint32_t& sh)
-{
-    const uint32_t* qr = a.score_rng + int64_t(q) * kCntStride;
-    const int32_t hi = int32_t(qr[0] ^ 0x80000000u);
-    lo = int32_t(~qr[1] ^ 0x80000000u);
-    sh = topk_shift(lo, hi);
-}
-
-// Candidates the chunked kernels handle for query q: all of them, unless the
-// scan overflowed the query's buffer (the final kernel rescans those).
-__device__ __forceinline__ int64_t chunked_count(const SearchArgs& a, int q)
-{
-    const int64_t n = a.cand_cnt[int64_t(q) * kCntStride];
-    return n <= a.cap ? n : 0;
-}
 
 // pre[q] = first item of query q (items: chunks of kChunk candidates), pre[B] = total
 template <int BLOCK>
@@ -161,45 +60,6 @@ __device__ __forceinline__ int item_query(const int* pre, int B, int item)
         else hi = mid - 1;
     }
     return lo;
-}
-
-// Per-query words of score_rng used by the final top-k, after the scan's range:
-// [2] cut-bin keys gathered, [3] chunks histogrammed, [4] cut bin, [5] keys
-// above it, [6] keys in it, [7] longest output segment.
-constexpr int kRngTie = 2, kRngDone = 3, kRngCut = 4, kRngAbove = 5, kRngTcount = 6, kRngMaxseg = 7;
-constexpr int kRngKept = 9;  // candidates left after the post-filter
-
-// The query's candidates that pass the post-filter (all of them without one).
-__device__ __forceinline__ int64_t kept_count(const SearchArgs& a, int q)
-{
-    return (a.dead || a.qexclude) ? int64_t(__ldcg(a.score_rng + int64_t(q) * kCntStride + kRngKept))
-                                  : chunked_count(a, q);
-}
-
-// Compact query q's candidates of the cut bin that pass the post-filter to
-// the front of its candidate buffer (no longer read by anyone else) and
-// return their count: one CTA, every thread's writes land only on positions
-// already read.
-template <int BLOCK>
-__device__ int compact_cut_bin(const SearchArgs& a, int q, int64_t n, const TopkCut& t)
-{
-    __shared__ int c_cnt;
-    uint64_t* keys = a.cand + int64_t(q) * a.cap;
-    if (threadIdx.x == 0) c_cnt = 0;
-    __syncthreads();
-    for (int64_t base = 0; base < n; base += BLOCK) {
-        const int64_t i = base + threadIdx.x;
-        uint64_t key = 0;
-        bool take = false;
-        if (i < n) {
-            key = keys[i];
-            take = topk_bin(key, t.lo, t.sh) == t.cut && keep_item(a, q, key_id(key));
-        }
-        __syncthreads();  // this round's reads are done before any write
-        if (take) keys[atomicAdd(&c_cnt, 1)] = key;
-        __syncthreads();
-    }
-    return c_cnt;
 }
 
 __global__ void __launch_bounds__(kChunkBlock)
@@ -317,89 +177,6 @@ select_scatter_kernel(SearchArgs a)
     }
 }
 
-template <int BLOCK>
-__global__ void __launch_bounds__(BLOCK)
-select_kernel(SearchArgs a, int stage_cap)
-{
-    dep_enter();
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ SelectSmem ss;
-    const int q = blockIdx.x;
-    const int k = a.k;
-    const int pwk = next_pow2(k);
-    // shared layout: [tmp k keys, rounded up to even][tie kSelectTieCapSmem keys]
-    // [stage_cap keys (>= next_pow2(k)): staged candidates / the output]
-    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
-    uint64_t* tie = tmp + ((k + 1) & ~1);
-    uint64_t* stage = tie + kSelectTieCapSmem;
-
-    const uint32_t cnt = a.cand_cnt[int64_t(q) * kCntStride];
-    int64_t n = cnt;
-    int m = 0;
-    uint64_t* out = stage;
-    if (n > a.cap) {
-        // the scan overflowed this query's buffer: rescan exactly, then select
-        // from the kept keys here
-        n = overflow_path<BLOCK>(a, q, stage, pwk, reinterpret_cast<int4*>(tie), ss);
-        const uint64_t* keys = a.cand + int64_t(q) * a.cap;
-        if (n <= stage_cap) {
-            for (int64_t i = threadIdx.x; i < n; i += BLOCK) stage[i] = keys[i];
-            __syncthreads();
-            keys = stage;
-        } else {
-            out = a.cand + int64_t(q) * a.cap;  // cap >= n > stage_cap >= next_pow2(k)
-        }
-        m = block_topk_sorted<BLOCK>(keys, n, k, out, tmp, tie, kSelectTieCapSmem, false, 0, 0, ss, a.err);
-    } else if (n > 0) {
-        // the chunked kernels grouped the keys above the cut bin by bin
-        int32_t lo;
-        uint32_t sh;
-        query_range(a, q, lo, sh);
-        // the histogram kernel's cut; after the scatter the cursor of bin b + 1
-        // (the next higher bin) stands at the end of its segment, which is
-        // where bin b's segment starts
-        const uint32_t* rng = a.score_rng + int64_t(q) * kCntStride;
-        TopkCut t;
-        t.lo = lo;
-        t.sh = sh;
-        t.cut = int(rng[kRngCut]);
-        t.above = int(rng[kRngAbove]);
-        t.tcount = int(rng[kRngTcount]);
-        t.maxseg = int(rng[kRngMaxseg]);
-        const int64_t nk = kept_count(a, q);
-        t.m = nk < k ? int(nk) : k;
-        const uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
-        for (int i = threadIdx.x; i < kSelBins; i += BLOCK) ss.hist2[i] = i + 1 < kSelBins ? cur[i + 1] : 0u;
-        const uint64_t* gout = a.sel_out + int64_t(q) * k;
-        for (int i = threadIdx.x; i < t.above; i += BLOCK) tmp[i] = gout[i];
-        const uint64_t* gtie = a.sel_tie + int64_t(q) * kSelTieCap;
-        const uint64_t* tsrc = nullptr;  // the cut bin's keys, if they were all kept
-        if (t.tcount <= kSelectTieCapSmem) {
-            for (int i = threadIdx.x; i < t.tcount; i += BLOCK) tie[i] = gtie[i];
-            tsrc = tie;
-        } else if (t.tcount <= kSelTieCap) {
-            tsrc = gtie;
-        }
-        __syncthreads();
-        if (tsrc == nullptr && (a.dead || a.qexclude) && t.m > t.above) {
-            // the cut bin was too large to keep aside: its filtered keys, compacted
-            const int nt = compact_cut_bin<BLOCK>(a, q, n, t);
-            t.tcount = nt;
-            tsrc = a.cand + int64_t(q) * a.cap;
-        }
-        topk_take_ties<BLOCK>(t, tsrc, a.cand + int64_t(q) * a.cap, n, tmp, ss, a.err);
-        topk_rank<BLOCK>(t, tmp, out, ss);
-        m = t.m;
-    }
-    for (int r = threadIdx.x; r < k; r += BLOCK) {
-        const uint64_t key = r < m ? out[r] : 0ull;  // key 0 reads as (id -1, INT32_MIN)
-        a.out_ids[int64_t(q) * k + r] = key == 0ull ? -1 : key_id(key) + a.id_offset;
-        a.out_scores[int64_t(q) * k + r] = key_score(key);
-    }
-    if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
-    if (threadIdx.x == 0 && a.out_cands) a.out_cands[q] = int64_t(cnt);
-}
-
 // ----------------------------------------------------------------------------
 // k above ST_SMALL_K: the same histogram and scatter, then the cut bin's best
 // per query and every key's rank in its segment, all in global memory.
@@ -478,16 +255,11 @@ select_rank_kernel(SearchArgs a)
     a.out_scores[o] = key_score(key);
 }
 
-size_t select_smem(int k, int* stage_cap)
-{
-    const size_t budget = 208 * 1024;
-    const size_t fixed = (size_t((k + 1) & ~1) + kSelectTieCapSmem) * 8;
-    *stage_cap = int((budget - fixed) / 8) & ~1;
-    return budget;
-}
+cudaError_t launch_select_cluster(const SearchArgs& a, int num_sms, cudaStream_t s);
 
 cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
 {
+    if (a.k <= ST_SMALL_K) return launch_select_cluster(a, num_sms, s);
     // the attribute is set once per device: give it the largest size any batch uses
     constexpr int kPreSmemMax = 160 * 1024;
     const size_t pre_bytes = size_t(a.B + 1) * 4;
@@ -501,17 +273,10 @@ cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
     if (e != cudaSuccess) return e;
     e = launch_dep(select_scatter_kernel, dim3(grid), dim3(kChunkBlock), pre_bytes, s, a);
     if (e != cudaSuccess) return e;
-    if (a.k > ST_SMALL_K) {
-        e = launch_dep(select_ties_kernel<kSelectBlock>, dim3(a.B), dim3(kSelectBlock), 0, s, a);
-        if (e != cudaSuccess) return e;
-        const int64_t threads = int64_t(a.B) * a.k;
-        return launch_dep(select_rank_kernel, dim3(unsigned((threads + 255) / 256)), dim3(256), 0, s, a);
-    }
-    int stage_cap = 0;
-    const size_t smem = select_smem(a.k, &stage_cap);
-    e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), 8, int(smem));
+    e = launch_dep(select_ties_kernel<kSelectBlock>, dim3(a.B), dim3(kSelectBlock), 0, s, a);
     if (e != cudaSuccess) return e;
-    return launch_dep(select_kernel<kSelectBlock>, dim3(a.B), dim3(kSelectBlock), smem, s, a, stage_cap);
+    const int64_t threads = int64_t(a.B) * a.k;
+    return launch_dep(select_rank_kernel, dim3(unsigned((threads + 255) / 256)), dim3(256), 0, s, a);
 }
 
 }  // namespace st

@@ -15,6 +15,12 @@ namespace st {
 constexpr int kScanBlock = 128;            // threads per scan CTA (four warps sharing a unit counter)
 constexpr int kWarpItems = 512;            // list rows per work unit (one warp)
 constexpr int kQMax = 16;                  // queries per work unit
+// Dense units: lists probed by at least tc_min_q queries go to the tensor-core
+// scan in units of up to kTcQMax queries (the MMA's N).
+constexpr int kTcQMax = 64;
+constexpr int kTcMinQDefault = 8;
+constexpr int kTcBins = 64;                // per-query score bins of the running top-k bound
+constexpr int kRngThr = 12;                // score_rng word: the query's running score bound (biased)
 
 constexpr int kProbeBlock = 512;
 constexpr int kProbeSmemKeys = 16384;      // nlist up to this keeps probe keys in smem
@@ -38,6 +44,7 @@ enum : uint32_t {
     kErrOverflowPath = 1u << 3, // the exact overflow path met an impossible state
     kErrUnitTable = 1u << 4,    // more work units than the host-sized table holds
     kErrUpdateId = 1u << 6,     // an in-place update named a row outside the index
+    kErrTcWait = 1u << 7,       // a wait of the tensor-core scan ran out (bounded wait expired)
 };
 
 // ----------------------------------------------------------------------------
@@ -65,7 +72,8 @@ __host__ __device__ __forceinline__ int64_t key_id(uint64_t key)
 // ----------------------------------------------------------------------------
 struct PlanCtl {
     int32_t n_units;       // work units allocated by the plan (clamped to the table by the scan)
-    int32_t pad[3];
+    int32_t n_dense;       // dense (tensor-core) units allocated by the plan
+    int32_t pad[2];
 };
 
 struct SearchArgs {
@@ -115,7 +123,11 @@ struct SearchArgs {
     uint8_t* qbits;          // [B][kMaskBitsMax] each query's mask bits, in increasing order
     int32_t* qnbits;         // [B] number of mask bits of each query
     int4* units;             // [max_units] {first row, chunk, first slot, rows << 16 | queries}
+    int4* units_tc;          // [max_units] dense units, same entries (up to kTcQMax queries)
     int32_t max_units;
+    int32_t tc_min_q;        // queries per list from which its units are dense (0: no dense units)
+    int2* qscale;            // [B] per query {lowest possible score -S, bin shift}: S = 128 sum |q_j|
+    uint32_t* tc_hist;       // [B][kTcBins] keys written by the dense scan per score bin (zeroed)
     uint64_t* cand;          // [B][cap]
     int64_t cap;             // candidate keys per query
     uint32_t* err;           // device error word
@@ -787,6 +799,9 @@ size_t probe_noalloc_scratch_bytes(int B, int S, int P, int nlist, bool keys_in_
 cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
+// tmap: the index's item rows as a 2-D tensor map (opaque CUtensorMap, 128 bytes)
+cudaError_t launch_scan_tc(const SearchArgs& a, const void* tmap, int num_sms, cudaStream_t s);
+bool scan_tc_supported(int d);
 cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
                          int32_t* out_scores, cudaStream_t s);

@@ -190,7 +190,13 @@ typedef enum {
        once and needs the old and the new arrays at the same time. 0 is a
        no-op; the room is never given back. OOM when it cannot be had,
        UNSUPPORTED when the ids would reach 2^31 (with the id offset). */
-    ST_OPT_INSERT_RESERVE = 4
+    ST_OPT_INSERT_RESERVE = 4,
+    /* Lists probed by at least this many queries of a batch are scanned as
+       dense tiles on the tensor cores (int8 x int8 -> int32, up to 64 queries
+       per tile) instead of per-pair dp4a; results are identical. Default 8;
+       1 sends every probed list there; 0 turns the tensor-core scan off. Only
+       d = 64 and d = 128 have the tensor-core scan. At most ST_MAX_B. */
+    ST_OPT_DENSE_MIN_QUERIES = 5
 } st_option;
 
 /* Set an option; INVALID_ARG for an unknown option or a negative value.
