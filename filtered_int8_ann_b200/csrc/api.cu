@@ -411,7 +411,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     };
     e = cudaMemsetAsync(base, 0, L.zero_bytes, stream);
     mark(0);
-    if (e == cudaSuccess) e = st::launch_probe_search(a, stream);
+    if (e == cudaSuccess) e = st::launch_probe_search(a, idx->num_sms, stream);
     mark(1);
     if (e == cudaSuccess) e = st::launch_plan(a, idx->num_sms, stream);
     mark(2);

@@ -14,18 +14,21 @@
 //     per tile (not once per query), dotted by dp4a against 16 queries per
 //     thread, and the (score, list id) keys go to a [B][nlist] array that
 //     stays in L2;
-//   * probe_select_kernel: one CTA per query. The keys' score range, a 2048-bin
-//     histogram over it, and the suffix counts give the bin holding the
-//     nprobe-th best score, so only the keys at or above that bin (a few more
-//     than nprobe) go through the exact selection and the sort. The CTA then
-//     writes the probe result and files the query into every chosen list: it
-//     takes the next rank of the list's query counter and writes its id and
-//     mask into the list's slot row, which the plan and the scan read.
+//   * probe_select_cluster_kernel: one thread-block cluster per query (up to
+//     8 CTAs at small batches, so the whole GPU works on the selections). The
+//     keys' score range, a 2048-bin histogram over it summed through
+//     distributed shared memory, and the suffix counts give the bin holding
+//     the nprobe-th best score, so only the keys at or above that bin (a few
+//     more than nprobe) reach the leader CTA for the exact selection and the
+//     sort. The leader then writes the probe result and files the query into
+//     every chosen list: it takes the next rank of the list's query counter
+//     and writes its id and mask into the list's slot row, which the plan and
+//     the scan read.
 // The allocation-free probe-only call keeps an older single-kernel form (CTAs
 // over query x centroid slices, last CTA merges), whose scratch is bounded.
 #include <mutex>
 
-#include "st_internal.cuh"
+#include "cluster_topk.cuh"
 
 namespace st {
 
@@ -225,56 +228,53 @@ probe_score_kernel(SearchArgs a)
         if (g * kQPer + j < nq) out[int64_t(j) * ld] = pack_key(acc[j], uint32_t(c));
 }
 
-template <int BLOCK>
-__global__ void __launch_bounds__(BLOCK)
-probe_select_kernel(SearchArgs a, int stage_cap, int tie_cap)
-{
-    dep_enter();
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ SelectSmem ss;
-    const int b = blockIdx.x;
-    const int nlist = a.nlist, P = a.P;
-    // shared layout: [tmp P keys, rounded up to even][tie tie_cap keys][staged keys
-    // stage_cap (>= next_pow2(P)), reused as the output]
-    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
-    uint64_t* tie = tmp + ((P + 1) & ~1);
-    uint64_t* stage = tie + tie_cap;
-    uint64_t* const row = a.probe_keys + int64_t(b) * probe_keys_ld(nlist);  // 16-byte aligned
-    const uint64_t* keys = row;
-    if (nlist <= stage_cap) {
-        // every key of the row in flight at once
-        const ulonglong2* src2 = reinterpret_cast<const ulonglong2*>(keys);
-        ulonglong2* dst2 = reinterpret_cast<ulonglong2*>(stage);
-        for (int i = threadIdx.x; i < (nlist >> 1); i += BLOCK) cp_async16(dst2 + i, src2 + i);
-        if ((nlist & 1) && threadIdx.x == 0) stage[nlist - 1] = keys[nlist - 1];
-        cp_async_commit();
-        cp_async_wait_all();
-        __syncthreads();
-        keys = stage;  // the output below overwrites it only after the last read
-    }
-    uint64_t* out = nlist <= stage_cap ? stage : row;
-    const int m = block_topk_sorted<BLOCK>(keys, nlist, P, out, tmp, tie, tie_cap, false, 0, 0, ss, a.err);
-    if (threadIdx.x == 0 && m != P) set_error(a.err, kErrSelectCount);
-    file_query<BLOCK, true>(a, b, out);
-}
-
-constexpr int kProbeSelBlock = 1024;
-
+// One cluster of CS CTAs per query: the nprobe best keys of the query's row
+// of centroid keys (cluster_topk.cuh), then its probe result and filing.
+constexpr int kProbeCBlock = 512;
 constexpr int kProbeTieCap = 1024;
 
-// Shared memory of probe_select_kernel; *stage_cap = keys that can be staged.
-size_t probe_select_smem(int P, int nlist, int* stage_cap)
+template <int CS>
+__global__ void __launch_bounds__(kProbeCBlock)
+probe_select_cluster_kernel(SearchArgs a)
 {
-    const size_t budget = 200 * 1024;
-    const size_t fixed = (size_t((P + 1) & ~1) + kProbeTieCap) * 8;
-    const int want = nlist > next_pow2(P) ? nlist : next_pow2(P);
-    size_t cap = (budget - fixed) / 8;
-    if (cap > size_t(want)) cap = size_t(want);
-    *stage_cap = int(cap);
-    return fixed + cap * 8;
+    dep_enter();
+    cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+    const int b = int(blockIdx.x) / CS;
+    const int P = a.P;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ SelectSmem ss;
+    __shared__ ClusterCut cc;
+    // shared layout: [tmp: P keys, rounded up to even][tie: kProbeTieCap keys][out: next_pow2(P) keys]
+    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* tie = tmp + ((P + 1) & ~1);
+    uint64_t* out = tie + kProbeTieCap;
+    const uint64_t* row = a.probe_keys + int64_t(b) * probe_keys_ld(a.nlist);
+    auto none = [](uint64_t) { return true; };
+    auto no_compact = []() { return 0; };
+    const int m = cluster_topk<CS, kProbeCBlock>(cluster, row, a.nlist, P, false, 0, 0, false, none, no_compact, tmp,
+                                                 tie, kProbeTieCap, out, ss, cc, a.err);
+    if (m < 0) return;  // not the leader
+    if (threadIdx.x == 0 && m != P) set_error(a.err, kErrSelectCount);
+    file_query<kProbeCBlock, true>(a, b, out);
 }
 
-cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s)
+static size_t probe_select_smem(int P)
+{
+    return (size_t((P + 1) & ~1) + kProbeTieCap + size_t(next_pow2(P))) * 8;
+}
+
+template <int CS>
+static cudaError_t launch_probe_select(const SearchArgs& a, cudaStream_t s)
+{
+    const void* fn = reinterpret_cast<const void*>(probe_select_cluster_kernel<CS>);
+    cudaError_t e = ensure_smem_attr(fn, 14 + (CS == 1 ? 0 : CS == 2 ? 1 : CS == 4 ? 2 : 3),
+                                     int(probe_select_smem(ST_MAX_NPROBE)));
+    if (e != cudaSuccess) return e;
+    return launch_dep_cluster(probe_select_cluster_kernel<CS>, dim3(unsigned(a.B) * CS), dim3(kProbeCBlock),
+                              probe_select_smem(a.P), CS, s, a);
+}
+
+cudaError_t launch_probe_search(const SearchArgs& a, int num_sms, cudaStream_t s)
 {
     const dim3 grid((a.nlist + kTileC - 1) / kTileC, (a.B + kTileQ - 1) / kTileQ);
     const size_t qbytes = size_t(kTileQ) * a.d;
@@ -283,11 +283,12 @@ cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s)
     probe_score_kernel<<<grid, kScoreBlock, qbytes, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    int stage_cap = 0;
-    const size_t smem = probe_select_smem(a.P, a.nlist, &stage_cap);
-    e = ensure_smem_attr(reinterpret_cast<const void*>(probe_select_kernel<kProbeSelBlock>), 11, 200 * 1024);
-    if (e != cudaSuccess) return e;
-    return launch_dep(probe_select_kernel<kProbeSelBlock>, dim3(a.B), dim3(kProbeSelBlock), smem, s, a, stage_cap, int(kProbeTieCap));
+    switch (cluster_size_for(a.B, num_sms)) {
+    case 8: return launch_probe_select<8>(a, s);
+    case 4: return launch_probe_select<4>(a, s);
+    case 2: return launch_probe_select<2>(a, s);
+    default: return launch_probe_select<1>(a, s);
+    }
 }
 
 int probe_slices(const SearchArgs& a, int num_sms)

@@ -794,7 +794,7 @@ cudaError_t ensure_smem_attr(const void* func, int slot, int bytes);
 // Kernel launchers (defined in the .cu files)
 // ----------------------------------------------------------------------------
 int probe_slices(const SearchArgs& a, int num_sms);
-cudaError_t launch_probe_search(const SearchArgs& a, cudaStream_t s);
+cudaError_t launch_probe_search(const SearchArgs& a, int num_sms, cudaStream_t s);
 size_t probe_noalloc_scratch_bytes(int B, int S, int P, int nlist, bool keys_in_smem);
 cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
