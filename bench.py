@@ -540,6 +540,9 @@ def measure_config(st, name, B, steps, warmup, flush_reps, flush, pk, pool=4, da
         idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=sc)
     stride, sampled = sampled_steps(steps, pool)
     evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for i in sampled}
+    for row in evs.values():  # torch creates the CUDA event at its first record
+        for e in row:
+            e.record()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     s0.record()
@@ -733,7 +736,7 @@ def main():
     K = args.steps
     stride, sampled = sampled_steps(K, pool)
     evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(5)] for i in sampled}
-    for row in evs.values():
+    for row in evs.values():  # torch creates the CUDA event at its first record
         for e in row:
             e.record()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
