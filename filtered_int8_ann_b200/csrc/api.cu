@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -56,19 +57,28 @@ struct st_index {
 
 namespace st {
 
-cudaError_t ensure_smem_attr(const void* func, int slot, int bytes)
+cudaError_t ensure_smem_attr(const void* func, int bytes)
 {
-    static unsigned done[64] = {0};  // bit `slot` set once per device
+    // kernels whose limit has been raised, per device, with the size set
+    struct Entry {
+        int dev;
+        const void* func;
+        int bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> done;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 64 && slot < 32 && (done[dev] >> slot) & 1u) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& x : done)
+        if (x.dev == dev && x.func == func && x.bytes >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     // every large-shared-memory kernel asks for the same (largest) carveout, so
     // an SM need not reconfigure its L1 / shared split between them
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-    if (e == cudaSuccess && dev < 64 && slot < 32) __atomic_fetch_or(&done[dev], 1u << slot, __ATOMIC_RELAXED);
+    if (e == cudaSuccess) done.push_back(Entry{dev, func, bytes});
     return e;
 }
 

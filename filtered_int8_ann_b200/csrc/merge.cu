@@ -97,7 +97,7 @@ static cudaError_t launch_merge_impl(const int64_t* ids, const int32_t* scores, 
     const int pw = next_pow2(k);
     const int nkeys = G * k > pw ? G * k : pw;
     const size_t smem = (size_t((k + 1) & ~1) + kMergeTieCap + size_t(nkeys)) * 8;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_kernel<UNION>), UNION ? 15 : 14,
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(merge_kernel<UNION>),
                                      int((size_t(ST_SMALL_K) + kMergeTieCap + ST_MERGE_MAX_KEYS) * 8));
     if (e != cudaSuccess) return e;
     merge_kernel<UNION><<<B, kMergeBlock, smem, s>>>(ids, scores, G, B, k, out_ids, out_scores);

@@ -267,8 +267,7 @@ template <int CS>
 static cudaError_t launch_probe_select(const SearchArgs& a, cudaStream_t s)
 {
     const void* fn = reinterpret_cast<const void*>(probe_select_cluster_kernel<CS>);
-    cudaError_t e = ensure_smem_attr(fn, 14 + (CS == 1 ? 0 : CS == 2 ? 1 : CS == 4 ? 2 : 3),
-                                     int(probe_select_smem(ST_MAX_NPROBE)));
+    cudaError_t e = ensure_smem_attr(fn, int(probe_select_smem(ST_MAX_NPROBE)));
     if (e != cudaSuccess) return e;
     return launch_dep_cluster(probe_select_cluster_kernel<CS>, dim3(unsigned(a.B) * CS), dim3(kProbeCBlock),
                               probe_select_smem(a.P), CS, s, a);
@@ -278,7 +277,7 @@ cudaError_t launch_probe_search(const SearchArgs& a, int num_sms, cudaStream_t s
 {
     const dim3 grid((a.nlist + kTileC - 1) / kTileC, (a.B + kTileQ - 1) / kTileQ);
     const size_t qbytes = size_t(kTileQ) * a.d;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_score_kernel), 10, int(kTileQ * ST_MAX_D));
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(probe_score_kernel), int(kTileQ * ST_MAX_D));
     if (e != cudaSuccess) return e;
     probe_score_kernel<<<grid, kScoreBlock, qbytes, s>>>(a);
     e = cudaGetLastError();
@@ -356,7 +355,7 @@ cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s)
     e = cudaMemsetAsync(a.probe_done, 0, size_t(a.B) * 4, s);
     if (e != cudaSuccess) return e;
     const size_t smem = probe_smem_bytes(a, S);
-    e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock, false>), 9, 200 * 1024);
+    e = ensure_smem_attr(reinterpret_cast<const void*>(probe_kernel<kProbeBlock, false>), 200 * 1024);
     if (e != cudaSuccess) return e;
     probe_kernel<kProbeBlock, false><<<a.B * S, kProbeBlock, smem, s>>>(a, S);
     return cudaGetLastError();

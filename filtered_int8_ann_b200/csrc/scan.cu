@@ -490,7 +490,7 @@ static cudaError_t launch_variant(const SearchArgs& a, int num_sms, cudaStream_t
     const size_t smem = scan_smem_bytes(a.d, W);
     const void* fn = reinterpret_cast<const void*>(scan_kernel<NP, W>);
     const int slot = 1 + (NP == 4 ? 0 : NP == 8 ? 1 : 2) + 3 * (W - 1);
-    cudaError_t e = ensure_smem_attr(fn, slot, int(scan_smem_bytes(ST_MAX_D, W)));
+    cudaError_t e = ensure_smem_attr(fn, int(scan_smem_bytes(ST_MAX_D, W)));
     if (e != cudaSuccess) return e;
     // occupancy depends on d only through the shared memory size: cache it for
     // the fixed-d variants

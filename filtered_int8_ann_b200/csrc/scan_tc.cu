@@ -483,8 +483,7 @@ static cudaError_t launch_tc(const SearchArgs& a, const void* tmap, int num_sms,
     size_t smem = tc_dyn_smem<D>();
     if (smem < kTcMinSmem) smem = kTcMinSmem;
     const void* fn = reinterpret_cast<const void*>(scan_tc_kernel<D, W>);
-    const int slot = 20 + (D == 128 ? 1 : 0) + 2 * (W - 1);
-    cudaError_t e = ensure_smem_attr(fn, slot, int(smem));
+    cudaError_t e = ensure_smem_attr(fn, int(smem));
     if (e != cudaSuccess) return e;
     CUtensorMap map;
     memcpy(&map, tmap, sizeof(map));

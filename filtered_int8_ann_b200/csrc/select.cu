@@ -265,11 +265,11 @@ cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
     const size_t pre_bytes = size_t(a.B + 1) * 4;
     if (pre_bytes > size_t(kPreSmemMax)) return cudaErrorInvalidValue;
     const int grid = 3 * num_sms;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_hist_kernel), 12, kPreSmemMax);
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(select_hist_kernel), kPreSmemMax);
     if (e != cudaSuccess) return e;
     e = launch_dep(select_hist_kernel, dim3(grid), dim3(kChunkBlock), pre_bytes, s, a);
     if (e != cudaSuccess) return e;
-    e = ensure_smem_attr(reinterpret_cast<const void*>(select_scatter_kernel), 13, kPreSmemMax);
+    e = ensure_smem_attr(reinterpret_cast<const void*>(select_scatter_kernel), kPreSmemMax);
     if (e != cudaSuccess) return e;
     e = launch_dep(select_scatter_kernel, dim3(grid), dim3(kChunkBlock), pre_bytes, s, a);
     if (e != cudaSuccess) return e;

@@ -97,7 +97,7 @@ static cudaError_t launch_cs(const SearchArgs& a, cudaStream_t s)
 {
     const size_t smem = select_cluster_smem(ST_SMALL_K);  // the attribute covers every k
     const void* fn = reinterpret_cast<const void*>(select_cluster_kernel<CS>);
-    cudaError_t e = ensure_smem_attr(fn, 24 + (CS == 1 ? 0 : CS == 2 ? 1 : CS == 4 ? 2 : 3), int(smem));
+    cudaError_t e = ensure_smem_attr(fn, int(smem));
     if (e != cudaSuccess) return e;
     return launch_dep_cluster(select_cluster_kernel<CS>, dim3(unsigned(a.B) * CS), dim3(kCBlock),
                               select_cluster_smem(a.k), CS, s, a);

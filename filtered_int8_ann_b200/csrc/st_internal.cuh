@@ -786,9 +786,9 @@ __host__ __device__ __forceinline__ int next_pow2(int v)
     return p;
 }
 
-// Raise a kernel's dynamic shared memory limit, once per device and kernel slot
-// (slot < 32). Setting it twice is harmless, so a race only repeats it.
-cudaError_t ensure_smem_attr(const void* func, int slot, int bytes);
+// Raise a kernel's dynamic shared memory limit to at least `bytes`, once per
+// device and kernel.
+cudaError_t ensure_smem_attr(const void* func, int bytes);
 
 // ----------------------------------------------------------------------------
 // Kernel launchers (defined in the .cu files)
