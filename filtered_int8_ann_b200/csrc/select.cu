@@ -1,4 +1,5 @@
-// Final top-k for k above ST_SMALL_K (k <= ST_SMALL_K: select_cluster.cu):
+// Final top-k in global memory, for k above ST_SMALL_K and for batches of at
+// most kChunkedMaxB queries (otherwise select_cluster.cu):
 // the k best candidate keys of each query, ordered by score descending, then
 // item id ascending, padded with (id -1, score INT32_MIN) when fewer than k
 // items were eligible.
@@ -8,9 +9,8 @@
 // Int8 ANN paragraph; maximum top-k row of the cost efficiency table in the
 // Spanish translation (a count in the hundreds of thousands).
 //
-// Four kernels, all in global memory, so that a query with a hundred thousand
-// candidates is spread over many SMs: the candidates of every query are cut
-// into chunks of kChunk keys, and
+// The candidates of every query are cut into chunks of kChunk keys, so that a
+// query with millions of candidates is spread over every SM:
 //   * select_hist_kernel: each chunk's keys go into a 2048-bin histogram of
 //     their scores over the query's score range (recorded by the scan),
 //     added into the query's histogram; the query's last chunk finds the cut
@@ -18,17 +18,21 @@
 //     segment;
 //   * select_scatter_kernel: every chunk writes its keys of the bins above the
 //     cut into their segments; the cut bin's keys are gathered aside;
-//   * select_ties_kernel: one CTA per query takes the cut bin's best;
-//   * select_rank_kernel: one thread per output position ranks its key in
-//     its segment and writes the id and score.
-// The scan reserves room for every row of the probed lists when k is this
-// large, so there is no overflow path here.
+//   * k <= ST_SMALL_K: select_kernel, one CTA per query, takes the cut bin's
+//     best, orders every segment in shared memory and writes ids and scores
+//     (or takes the exact overflow path when the scan's buffer overflowed);
+//   * larger k: select_ties_kernel (one CTA per query) takes the cut bin's
+//     best and select_rank_kernel (one thread per output position) ranks each
+//     key in its segment and writes the id and score. The scan reserves room
+//     for every row of the probed lists when k is this large, so there is no
+//     overflow path there.
 #include "select_common.cuh"
 
 namespace st {
 
 constexpr int kChunk = 4096;      // candidates per histogram / scatter item
 constexpr int kChunkBlock = 512;
+constexpr int kChunkedMaxB = 8;   // batches up to this size take the chunked kernels for any k
 
 // pre[q] = first item of query q (items: chunks of kChunk candidates), pre[B] = total
 template <int BLOCK>
@@ -177,6 +181,94 @@ select_scatter_kernel(SearchArgs a)
     }
 }
 
+// Finish of the chunked path for k <= ST_SMALL_K: one CTA per query takes
+// the cut bin's best, orders every segment and writes ids and scores; a query
+// whose candidates overflowed the scan's buffer takes the exact overflow path.
+constexpr int kSelectTieCapSmem = 1024;
+
+template <int BLOCK>
+__global__ void __launch_bounds__(BLOCK)
+select_kernel(SearchArgs a, int stage_cap)
+{
+    dep_enter();
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ SelectSmem ss;
+    const int q = blockIdx.x;
+    const int k = a.k;
+    const int pwk = next_pow2(k);
+    // shared layout: [tmp k keys, rounded up to even][tie kSelectTieCapSmem keys]
+    // [stage_cap keys (>= next_pow2(k)): staged candidates / the output]
+    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* tie = tmp + ((k + 1) & ~1);
+    uint64_t* stage = tie + kSelectTieCapSmem;
+
+    const uint32_t cnt = a.cand_cnt[int64_t(q) * kCntStride];
+    int64_t n = cnt;
+    int m = 0;
+    uint64_t* out = stage;
+    if (n > a.cap) {
+        // the scan overflowed this query's buffer: rescan exactly, then select
+        // from the kept keys here
+        n = overflow_path<BLOCK>(a, q, stage, pwk, reinterpret_cast<int4*>(tie), ss);
+        const uint64_t* keys = a.cand + int64_t(q) * a.cap;
+        if (n <= stage_cap) {
+            for (int64_t i = threadIdx.x; i < n; i += BLOCK) stage[i] = keys[i];
+            __syncthreads();
+            keys = stage;
+        } else {
+            out = a.cand + int64_t(q) * a.cap;  // cap >= n > stage_cap >= next_pow2(k)
+        }
+        m = block_topk_sorted<BLOCK>(keys, n, k, out, tmp, tie, kSelectTieCapSmem, false, 0, 0, ss, a.err);
+    } else if (n > 0) {
+        // the chunked kernels grouped the keys above the cut bin by bin
+        int32_t lo;
+        uint32_t sh;
+        query_range(a, q, lo, sh);
+        // the histogram kernel's cut; after the scatter the cursor of bin b + 1
+        // (the next higher bin) stands at the end of its segment, which is
+        // where bin b's segment starts
+        const uint32_t* rng = a.score_rng + int64_t(q) * kCntStride;
+        TopkCut t;
+        t.lo = lo;
+        t.sh = sh;
+        t.cut = int(rng[kRngCut]);
+        t.above = int(rng[kRngAbove]);
+        t.tcount = int(rng[kRngTcount]);
+        t.maxseg = int(rng[kRngMaxseg]);
+        const int64_t nk = kept_count(a, q);
+        t.m = nk < k ? int(nk) : k;
+        const uint32_t* cur = a.sel_cursor + int64_t(q) * kSelBins;
+        for (int i = threadIdx.x; i < kSelBins; i += BLOCK) ss.hist2[i] = i + 1 < kSelBins ? cur[i + 1] : 0u;
+        const uint64_t* gout = a.sel_out + int64_t(q) * k;
+        for (int i = threadIdx.x; i < t.above; i += BLOCK) tmp[i] = gout[i];
+        const uint64_t* gtie = a.sel_tie + int64_t(q) * kSelTieCap;
+        const uint64_t* tsrc = nullptr;  // the cut bin's keys, if they were all kept
+        if (t.tcount <= kSelectTieCapSmem) {
+            for (int i = threadIdx.x; i < t.tcount; i += BLOCK) tie[i] = gtie[i];
+            tsrc = tie;
+        } else if (t.tcount <= kSelTieCap) {
+            tsrc = gtie;
+        }
+        __syncthreads();
+        if (tsrc == nullptr && (a.dead || a.qexclude) && t.m > t.above) {
+            // the cut bin was too large to keep aside: its filtered keys, compacted
+            const int nt = compact_cut_bin<BLOCK>(a, q, n, t);
+            t.tcount = nt;
+            tsrc = a.cand + int64_t(q) * a.cap;
+        }
+        topk_take_ties<BLOCK>(t, tsrc, a.cand + int64_t(q) * a.cap, n, tmp, ss, a.err);
+        topk_rank<BLOCK>(t, tmp, out, ss);
+        m = t.m;
+    }
+    for (int r = threadIdx.x; r < k; r += BLOCK) {
+        const uint64_t key = r < m ? out[r] : 0ull;  // key 0 reads as (id -1, INT32_MIN)
+        a.out_ids[int64_t(q) * k + r] = key == 0ull ? -1 : key_id(key) + a.id_offset;
+        a.out_scores[int64_t(q) * k + r] = key_score(key);
+    }
+    if (threadIdx.x == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
+    if (threadIdx.x == 0 && a.out_cands) a.out_cands[q] = int64_t(cnt);
+}
+
 // ----------------------------------------------------------------------------
 // k above ST_SMALL_K: the same histogram and scatter, then the cut bin's best
 // per query and every key's rank in its segment, all in global memory.
@@ -255,11 +347,22 @@ select_rank_kernel(SearchArgs a)
     a.out_scores[o] = key_score(key);
 }
 
+size_t select_smem(int k, int* stage_cap)
+{
+    const size_t budget = 208 * 1024;
+    const size_t fixed = (size_t((k + 1) & ~1) + kSelectTieCapSmem) * 8;
+    *stage_cap = int((budget - fixed) / 8) & ~1;
+    return budget;
+}
+
 cudaError_t launch_select_cluster(const SearchArgs& a, int num_sms, cudaStream_t s);
 
 cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
 {
-    if (a.k <= ST_SMALL_K) return launch_select_cluster(a, num_sms, s);
+    // a batch of few queries may hold millions of candidates per query (a
+    // flat scan): spread them over the whole GPU with the chunked kernels;
+    // otherwise one cluster per query does it in one launch
+    if (a.k <= ST_SMALL_K && a.B > kChunkedMaxB) return launch_select_cluster(a, num_sms, s);
     // the attribute is set once per device: give it the largest size any batch uses
     constexpr int kPreSmemMax = 160 * 1024;
     const size_t pre_bytes = size_t(a.B + 1) * 4;
@@ -273,6 +376,13 @@ cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
     if (e != cudaSuccess) return e;
     e = launch_dep(select_scatter_kernel, dim3(grid), dim3(kChunkBlock), pre_bytes, s, a);
     if (e != cudaSuccess) return e;
+    if (a.k <= ST_SMALL_K) {
+        int stage_cap = 0;
+        const size_t smem = select_smem(a.k, &stage_cap);
+        e = ensure_smem_attr(reinterpret_cast<const void*>(select_kernel<kSelectBlock>), int(smem));
+        if (e != cudaSuccess) return e;
+        return launch_dep(select_kernel<kSelectBlock>, dim3(a.B), dim3(kSelectBlock), smem, s, a, stage_cap);
+    }
     e = launch_dep(select_ties_kernel<kSelectBlock>, dim3(a.B), dim3(kSelectBlock), 0, s, a);
     if (e != cudaSuccess) return e;
     const int64_t threads = int64_t(a.B) * a.k;

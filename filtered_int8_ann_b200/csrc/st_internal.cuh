@@ -17,7 +17,7 @@ constexpr int kWarpItems = 512;            // list rows per work unit (one warp)
 constexpr int kQMax = 16;                  // queries per work unit
 // Dense units: lists probed by at least tc_min_q queries go to the tensor-core
 // scan in units of up to kTcQMax queries (the MMA's N).
-constexpr int kTcQMax = 64;
+constexpr int kTcQMax = 32;
 constexpr int kTcMinQDefault = 8;
 constexpr int kTcBins = 64;                // per-query score bins of the running top-k bound
 constexpr int kRngThr = 12;                // score_rng word: the query's running score bound (biased)

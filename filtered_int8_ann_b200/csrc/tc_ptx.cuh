@@ -44,6 +44,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     return false;
 }
 
+// Plain arrival (release) on the barrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier among `count` threads (whole warps) of the CTA, id 1..15.
+__device__ __forceinline__ void named_barrier(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Make this thread's earlier generic-proxy writes to shared memory (plain
 // stores, cp.async) visible to the asynchronous proxy (tensor-core reads).
 __device__ __forceinline__ void fence_proxy_async_smem()
