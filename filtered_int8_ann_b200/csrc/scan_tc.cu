@@ -35,11 +35,13 @@
 // keys that can no longer enter a query's top-k are not written at all. Every
 // written key is a real candidate, so if at least k written keys have scores
 // >= T, the query's k-th best score is >= T and any key below T can be
-// dropped. Each query's written keys are counted in 64 bins over its possible
+// dropped. Each query's written keys are counted in 256 bins over its possible
 // score range [-S, S], S = 128 sum_j |q_j| (bin b holds scores in
-// [-S + b 2^sh, -S + (b+1) 2^sh)); after a unit, the bins' totals give the
-// highest bin edge with k written keys at or above it, published with
-// atomicMax. The bound only grows and the final top-k is unchanged (exact).
+// [-S + b 2^sh, -S + (b+1) 2^sh)). After a unit the counts are added to the
+// query's global bins; when the unit wrote at least kTcBoundMinKeys keys of a
+// query, the global bins from the query's bound upward give the highest bin
+// edge with k written keys at or above it, published with atomicMax. The
+// bound only grows and the final top-k is unchanged (exact).
 // With deletions or exclude masks the post-filter is applied before a key is
 // counted, so every counted key is still a result candidate.
 //
@@ -58,6 +60,7 @@ constexpr int kTcPlaneSlots = 48;        // planes one buffer holds
 constexpr int kTcDenseBlk = ST_TC_DENSE_BLK;  // survivors of a 32-row block from which the whole block is loaded
 constexpr uint32_t kTcWaitLimit = 1u << 22;
 constexpr int kTcMeta = 8;               // units whose data are held at once
+constexpr uint32_t kTcBoundMinKeys = 16; // keys of a query in one unit that make it re-read its bound
 constexpr int kTcEpiWarps = 8;           // two epilogue warpgroups
 constexpr int kTcThreads = 32 * (2 + kTcEpiWarps);
 constexpr int kTcAccCols = 4 * kTcQMax;  // TMEM columns of one unit's accumulators (4 row blocks)
@@ -102,7 +105,7 @@ template <int D>
 __host__ __device__ constexpr size_t tc_dyn_smem()
 {
     return size_t(tc_stages<D>()) * (size_t(kTcRows) * D + size_t(kTcQMax) * D) + size_t(2) * kTcPlaneSlots * 64 +
-           1024;
+           kTcMeta * sizeof(TcMeta) + 2 * sizeof(TcEpi) + 1024;
 }
 
 template <int D, int W>
@@ -117,8 +120,6 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
     constexpr int NPL = 64 * W;          // planes per chunk
     constexpr int CH = D / 16;           // 16-byte chunks per row
     extern __shared__ unsigned char smem_raw[];
-    __shared__ TcMeta meta[kTcMeta];
-    __shared__ TcEpi epi[2];
     __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], acc_full[2], acc_empty[2], meta_full[kTcMeta];
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
@@ -129,6 +130,8 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
     unsigned char* const Abuf = base;                                     // [S][kTcRows * D]
     unsigned char* const Bbuf = base + S * kTcRows * D;                   // [S][kTcQMax * D]
     uint32_t* const Pbuf = reinterpret_cast<uint32_t*>(Bbuf + S * kTcQMax * D);  // [2][kTcPlaneSlots][16]
+    TcMeta* const meta = reinterpret_cast<TcMeta*>(Pbuf + 2 * kTcPlaneSlots * 16);   // [kTcMeta]
+    TcEpi* const epi = reinterpret_cast<TcEpi*>(meta + kTcMeta);                       // [2]
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
@@ -236,42 +239,54 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
             for (int item = lane; item < 4 * nb; item += 32)
                 cp_async16_cg(dst + item * 4, src + mt.inv[item >> 2] * 16 + (item & 3) * 4);
         };
-        // Bloom test of meta[m] with plane buffer p
+        // Bloom test of meta[m] with plane buffer p: lane q takes query q and
+        // ANDs, for each of its mask bits, the 16 words (512 rows) of that
+        // bit's plane into its 16 pass words
         auto test_unit = [&](int m, int p) {
             TcMeta& mt = meta[m];
             const int4 e = mt.e;
             const int qn = e.w & 0xFFFF, len = e.w >> 16;
             const int held = mt.held;
-            const int w = lane & 15;
-            const uint32_t valid = len >= 32 * (w + 1) ? 0xFFFFFFFFu
-                                 : (len <= 32 * w ? 0u : ((1u << (len - 32 * w)) - 1u));
-            const uint32_t* pl = Pbuf + p * kTcPlaneSlots * 16 + w;
-            const uint32_t* gpl = a.planes + int64_t(e.y) * NPL * 16 + w;
-            uint32_t uacc = 0;
-            for (int i = 0; 2 * i < qn; ++i) {
-                const int q = 2 * i + (lane >> 4);
-                uint32_t acc = 0;
-                if (q < qn) {
-                    acc = valid;
-                    for (int word = 0; word < W; ++word) {
-                        unsigned long long mk = mt.qm[q][word];
-                        while (mk) {
-                            const int b = 64 * word + __ffsll(static_cast<long long>(mk)) - 1;
-                            mk &= mk - 1;
-                            acc &= held >= 0 ? pl[mt.tab[b] * 16] : __ldg(gpl + b * 16);
+            uint32_t acc[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w)
+                acc[w] = len >= 32 * (w + 1) ? 0xFFFFFFFFu : (len <= 32 * w ? 0u : ((1u << (len - 32 * w)) - 1u));
+            if (lane < qn) {
+                const uint4* pl = reinterpret_cast<const uint4*>(Pbuf + p * kTcPlaneSlots * 16);
+                const uint4* gpl = reinterpret_cast<const uint4*>(a.planes + int64_t(e.y) * NPL * 16);
+#pragma unroll
+                for (int word = 0; word < W; ++word) {
+                    unsigned long long mk = mt.qm[lane][word];
+                    while (mk) {
+                        const int b = 64 * word + __ffsll(static_cast<long long>(mk)) - 1;
+                        mk &= mk - 1;
+                        const uint4* src = held >= 0 ? pl + mt.tab[b] * 4 : gpl + b * 4;
+                        uint4 v[4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) v[c] = held >= 0 ? src[c] : __ldg(src + c);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            acc[4 * c] &= v[c].x;
+                            acc[4 * c + 1] &= v[c].y;
+                            acc[4 * c + 2] &= v[c].z;
+                            acc[4 * c + 3] &= v[c].w;
                         }
                     }
-                    mt.pass[w][q] = acc;
                 }
-                uacc |= acc;
-                uint32_t c = __popc(acc);
+            } else {
 #pragma unroll
-                for (int off = 8; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-                if (w == 0 && q < qn && c)
-                    atomicAdd(&a.eligible_cnt[int64_t(mt.qid[q]) * (kCntStride / 2)], (unsigned long long)c);
+                for (int w = 0; w < 16; ++w) acc[w] = 0;
             }
-            uacc |= __shfl_xor_sync(0xffffffffu, uacc, 16);
-            if (lane < 16) mt.uni[lane] = uacc;
+            uint32_t c = 0;
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                if (lane < qn) mt.pass[w][lane] = acc[w];
+                c += __popc(acc[w]);
+                const uint32_t u = __reduce_or_sync(0xffffffffu, acc[w]);
+                if (lane == 0) mt.uni[w] = u;
+            }
+            if (lane < qn && c)
+                atomicAdd(&a.eligible_cnt[int64_t(mt.qid[lane]) * (kCntStride / 2)], (unsigned long long)c);
             __syncwarp();
         };
         // rows and query vectors of meta[m] -> operand stage s
@@ -479,43 +494,50 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                         }
                     }
                 }
-                // publish the counts and raise each query's bound: the highest
-                // bin edge with at least k written keys at or above it (the
-                // warp takes queries wq, wq + 4, ...; all its loads first)
-                for (int q0 = 0; q0 < qn; q0 += 16) {
-                    uint32_t gv[4][2];
-                    int qq[4];
+                // publish the counts (fire and forget); for a query that wrote
+                // at least kTcBoundMinKeys keys, raise its bound: the highest
+                // bin edge with at least k written keys at or above it, from
+                // the global bins at or above its bound's bin (lane l takes bins
+                // 8 l .. 8 l + 7; the warp takes queries wq, wq + 4, ...)
+                for (int q = wq; q < qn; q += 4) {
+                    const uint32_t cq = E.cnt[q];
+                    if (cq == 0) continue;  // warp-uniform
+                    uint32_t* gh = a.tc_hist + int64_t(mt.qid[q]) * kTcBins;
+                    const int tb = mt.thr[q] ? ((int32_t(mt.thr[q] ^ 0x80000000u) - mt.qbase[q]) >> mt.qsh[q]) : 0;
+                    const uint4 lw = reinterpret_cast<const uint4*>(&E.hist[q][0])[lane];
+                    const uint32_t wv[4] = {lw.x, lw.y, lw.z, lw.w};
+                    if (cq < kTcBoundMinKeys) {
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        qq[t] = q0 + wq + 4 * t;
-                        gv[t][0] = gv[t][1] = 0;
-                        if (qq[t] < qn && E.cnt[qq[t]]) {
-                            uint32_t* gh = a.tc_hist + int64_t(mt.qid[qq[t]]) * kTcBins;
-                            const uint32_t word = E.hist[qq[t]][lane];
-                            const uint32_t c0 = word & 0xFFFFu, c1 = word >> 16;
-                            gv[t][0] = c0 ? atomicAdd(gh + 2 * lane, c0) + c0 : __ldcg(gh + 2 * lane);
-                            gv[t][1] = c1 ? atomicAdd(gh + 2 * lane + 1, c1) + c1 : __ldcg(gh + 2 * lane + 1);
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t c = (wv[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu;
+                            if (c) atomicAdd(gh + 8 * lane + i, c);
                         }
+                        continue;
                     }
+                    uint32_t gv[8], tot = 0;
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        if (qq[t] >= qn || !E.cnt[qq[t]]) continue;  // warp-uniform
-                        uint32_t incl = gv[t][0] + gv[t][1];  // suffix sum over lanes >= this one
+                    for (int i = 0; i < 8; ++i) {
+                        const int bin = 8 * lane + i;
+                        const uint32_t c = (wv[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu;
+                        gv[i] = bin < tb ? 0u : (c ? atomicAdd(gh + bin, c) + c : __ldcg(gh + bin));
+                        tot += gv[i];
+                    }
+                    uint32_t incl = tot;  // suffix sum over lanes >= this one
 #pragma unroll
-                        for (int off = 1; off < 32; off <<= 1) {
-                            const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
-                            if (lane + off < 32) incl += o;
-                        }
-                        const uint32_t kk = uint32_t(a.k);
-                        uint32_t best = 0;  // highest bin b with (keys in bins >= b) >= k
-                        if (incl - gv[t][0] >= kk) best = uint32_t(2 * lane + 1);
-                        else if (incl >= kk) best = uint32_t(2 * lane);
-                        best = __reduce_max_sync(0xffffffffu, best);
-                        if (lane == 0 && best > 0) {
-                            const int32_t T = mt.qbase[qq[t]] + int32_t(best << mt.qsh[qq[t]]);
-                            atomicMax(a.score_rng + int64_t(mt.qid[qq[t]]) * kCntStride + kRngThr,
-                                      uint32_t(T) ^ 0x80000000u);
-                        }
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+                        if (lane + off < 32) incl += o;
+                    }
+                    uint32_t run = incl - tot, best = 0;  // keys in bins above this lane's
+#pragma unroll
+                    for (int i = 7; i >= 0; --i) {
+                        run += gv[i];
+                        if (best == 0 && run >= uint32_t(a.k)) best = uint32_t(8 * lane + i);
+                    }
+                    best = __reduce_max_sync(0xffffffffu, best);
+                    if (lane == 0 && best > 0) {
+                        const int32_t T = mt.qbase[q] + int32_t(best << mt.qsh[q]);
+                        atomicMax(a.score_rng + int64_t(mt.qid[q]) * kCntStride + kRngThr, uint32_t(T) ^ 0x80000000u);
                     }
                 }
             }

@@ -19,7 +19,7 @@ constexpr int kQMax = 16;                  // queries per work unit
 // scan in units of up to kTcQMax queries (the MMA's N).
 constexpr int kTcQMax = 32;
 constexpr int kTcMinQDefault = 8;
-constexpr int kTcBins = 64;                // per-query score bins of the running top-k bound
+constexpr int kTcBins = 256;               // per-query score bins of the running top-k bound
 constexpr int kRngThr = 12;                // score_rng word: the query's running score bound (biased)
 
 constexpr int kProbeBlock = 512;
