@@ -339,7 +339,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_sel_cursor = L.add(size_t(B) * st::kSelBins * 4);
     L.off_ctl = L.add(sizeof(st::PlanCtl));
     const int tc_min_q = (idx->tmap_ok && idx->tc_min_q > 0 && B >= idx->tc_min_q) ? idx->tc_min_q : 0;
-    L.off_tc_hist = L.add(tc_min_q ? size_t(B) * st::kTcBins * 4 : 0);
+    L.off_tc_hist = L.add(size_t(B) * st::kTcBins * 4);
     L.zero_bytes = L.total;
     L.off_probe = L.add(size_t(B) * nprobe * 4);
     L.off_probe_keys = L.add(size_t(B) * size_t(st::probe_keys_ld(idx->nlist)) * 8);
@@ -350,7 +350,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_qmask = L.add(slots * 16);
     L.off_units = L.add(size_t(max_units) * 16);
     L.off_units_tc = L.add(tc_min_q ? size_t(max_units) * 16 : 0);
-    L.off_qscale = L.add(tc_min_q ? size_t(B) * 8 : 0);
+    L.off_qscale = L.add(size_t(B) * 8);
     L.off_cand = L.add(size_t(B) * size_t(cap) * 8);
     L.off_sel_out = L.add(size_t(B) * size_t(k) * 8);
     L.off_sel_tie = L.add(size_t(B) * st::kSelTieCap * 8);
@@ -402,11 +402,9 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.units = reinterpret_cast<int4*>(base + L.off_units);
     a.max_units = int32_t(max_units);
     a.tc_min_q = tc_min_q;
-    if (tc_min_q) {
-        a.units_tc = reinterpret_cast<int4*>(base + L.off_units_tc);
-        a.qscale = reinterpret_cast<int2*>(base + L.off_qscale);
-        a.tc_hist = reinterpret_cast<uint32_t*>(base + L.off_tc_hist);
-    }
+    if (tc_min_q) a.units_tc = reinterpret_cast<int4*>(base + L.off_units_tc);
+    a.qscale = reinterpret_cast<int2*>(base + L.off_qscale);
+    a.qhist = reinterpret_cast<uint32_t*>(base + L.off_tc_hist);
     a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
     a.cap = cap;
     a.id_offset = idx->id_offset;

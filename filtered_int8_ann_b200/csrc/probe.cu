@@ -62,8 +62,8 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
         if (lane == 0) a.qnbits[b] = n_before;
     }
     if (a.qscale != nullptr && threadIdx.x >= 32 && threadIdx.x < 64) {
-        // bound of the query's scores for the dense scan's score bins:
-        // |<q, x>| <= S = 128 * sum_j |q_j| for any int8 row x
+        // bound of the query's scores, for the score bins of the scans and
+        // the final top-k: |<q, x>| <= S = 128 * sum_j |q_j| for any int8 row x
         const int lane = threadIdx.x - 32;
         const int8_t* qv = a.queries + int64_t(b) * a.d;
         int32_t sum = 0;

@@ -34,7 +34,9 @@
 //     scored) and the survivors' rows are prefetched into L2; one iteration
 //     later only those rows are read (16-byte read-only loads) and dotted with
 //     dp4a against the query vectors (staged in shared memory by cp.async); a
-//     key's slot is its rank among the unit's survivors of that query.
+//     key's slot is its rank among the unit's survivors of that query, and
+//     the key is counted in the query's score bins (kTcBins bins over the
+//     query's possible range [-S, S]), which guide the final top-k.
 // Every unit commits exactly two cp.async groups (planes of the unit two
 // ahead, then query vectors of the next unit), so fixed wait_group depths find
 // every copy: there is no spin loop and nothing to time out.
@@ -47,13 +49,13 @@ constexpr int kPlaneBytes = kWarpItems / 8;             // 64 bytes per plane
 constexpr int kPlaneBufBytes = kPlaneSlots * kPlaneBytes;
 
 // Per-warp shared memory: plane buffer | survivor offsets [2][kWarpItems] u16 |
-// pass words [2][kQMax][16] | query vectors [kQMax][d] | per-query score range
-// [2][kQMax] | bit -> slot table [128] | slot -> bit [kPlaneSlots]
+// pass words [2][kQMax][16] | query vectors [kQMax][d] | bit -> slot table
+// [128] | slot -> bit [kPlaneSlots]
 __host__ __device__ inline size_t scan_warp_bytes(int d, int W)
 {
     (void)W;
-    return (kPlaneBufBytes + 2 * kWarpItems * 2 + 2 * kQMax * 16 * 4 + size_t(kQMax) * d + 2 * kQMax * 4 +
-            kMaskBitsMax + kPlaneSlots + 127) / 128 * 128;
+    return (kPlaneBufBytes + 2 * kWarpItems * 2 + 2 * kQMax * 16 * 4 + size_t(kQMax) * d + kMaskBitsMax +
+            kPlaneSlots + 127) / 128 * 128;
 }
 
 size_t scan_smem_bytes(int d, int W) { return size_t(kScanBlock / 32) * scan_warp_bytes(d, W); }
@@ -126,8 +128,7 @@ scan_kernel(SearchArgs a)
     uint16_t* const surv2 = reinterpret_cast<uint16_t*>(wb + kPlaneBufBytes);            // [2][kWarpItems]
     uint32_t* const pass2 = reinterpret_cast<uint32_t*>(surv2 + 2 * kWarpItems);         // [2][kQMax][16]
     int4* const s_q = reinterpret_cast<int4*>(pass2 + 2 * kQMax * 16);                  // [kQMax][np]
-    uint32_t* const s_rng = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(s_q) + size_t(kQMax) * d);  // [2][kQMax]
-    uint8_t* const s_tab = reinterpret_cast<uint8_t*>(s_rng + 2 * kQMax);                 // [128]
+    uint8_t* const s_tab = reinterpret_cast<uint8_t*>(s_q) + size_t(kQMax) * d;           // [128]
     uint8_t* const s_inv = s_tab + kMaskBitsMax;                                         // [kPlaneSlots]
 
     // units: CTA c owns units c, c + ncta, c + 2 ncta, ... (an even mix of the
@@ -364,7 +365,8 @@ scan_kernel(SearchArgs a)
             const int qg = __shfl_sync(0xffffffffu, qid_c, 0);
             const uint32_t base0 = __shfl_sync(0xffffffffu, base_c, 0);
             uint64_t* cand = a.cand + int64_t(qg) * a.cap;
-            uint32_t rmax = 0, rmin = 0;  // biased score range of this unit's keys (max of x, max of ~x)
+            const int2 sc = a.qscale[qg];
+            uint32_t* qh = a.qhist + int64_t(qg) * kTcBins;
             for (int c0 = 0; c0 < nsurv_c; c0 += 32) {
                 const int idx = c0 + lane;
                 if (idx < nsurv_c) {
@@ -386,29 +388,13 @@ scan_kernel(SearchArgs a)
                     const int32_t score = acc0 + acc1;
                     const uint64_t pos = uint64_t(base0) + uint32_t(idx);
                     if (pos < uint64_t(a.cap)) cand[pos] = pack_key(score, uint32_t(i));
-                    const uint32_t enc = uint32_t(score) ^ 0x80000000u;
-                    rmax = enc > rmax ? enc : rmax;
-                    rmin = ~enc > rmin ? ~enc : rmin;
+                    atomicAdd(qh + ((score - sc.x) >> sc.y), 1u);  // the key's score bin
                 }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                rmax = max(rmax, __shfl_xor_sync(0xffffffffu, rmax, off));
-                rmin = max(rmin, __shfl_xor_sync(0xffffffffu, rmin, off));
-            }
-            if (lane == 0 && nsurv_c > 0) {
-                atomicMax(&a.score_rng[int64_t(qg) * kCntStride], rmax);
-                atomicMax(&a.score_rng[int64_t(qg) * kCntStride + 1], rmin);
             }
         } else {
             // a key's slot is its ballot rank among this unit's survivors of
             // the same query
             uint32_t run = 0;  // lane s: keys of query s written so far
-            if (lane < kQMax) {
-                s_rng[lane] = 0;
-                s_rng[kQMax + lane] = 0;
-            }
-            __syncwarp();
             for (int c0 = 0; c0 < nsurv_c; c0 += 32) {
                 const int idx = c0 + lane;
                 int off = -1;
@@ -433,6 +419,7 @@ scan_kernel(SearchArgs a)
                     const uint32_t slot0 = __shfl_sync(0xffffffffu, base_c, s) + __shfl_sync(0xffffffffu, run, s);
                     const int qg = __shfl_sync(0xffffffffu, qid_c, s);
                     if (on) {
+                        const int2 sc = a.qscale[qg];
                         const int4* qs = s_q + s * np;
                         int32_t acc0 = 0, acc1 = 0;
                         if (NP > 0) {
@@ -447,17 +434,10 @@ scan_kernel(SearchArgs a)
                         const uint64_t pos = uint64_t(slot0) + __popc(bal & lanemask_lt());
                         const int32_t score = acc0 + acc1;
                         if (pos < uint64_t(a.cap)) a.cand[int64_t(qg) * a.cap + int64_t(pos)] = pack_key(score, uint32_t(i));
-                        const uint32_t enc = uint32_t(score) ^ 0x80000000u;
-                        atomicMax(&s_rng[s], enc);
-                        atomicMax(&s_rng[kQMax + s], ~enc);
+                        atomicAdd(a.qhist + int64_t(qg) * kTcBins + ((score - sc.x) >> sc.y), 1u);
                     }
                     if (lane == s) run += __popc(bal);
                 }
-            }
-            __syncwarp();
-            if (lane < qn && s_rng[lane] != 0u) {
-                atomicMax(&a.score_rng[int64_t(qid_c) * kCntStride], s_rng[lane]);
-                atomicMax(&a.score_rng[int64_t(qid_c) * kCntStride + 1], s_rng[kQMax + lane]);
             }
         }
 

@@ -35,13 +35,12 @@
 // keys that can no longer enter a query's top-k are not written at all. Every
 // written key is a real candidate, so if at least k written keys have scores
 // >= T, the query's k-th best score is >= T and any key below T can be
-// dropped. Each query's written keys are counted in 256 bins over its possible
-// score range [-S, S], S = 128 sum_j |q_j| (bin b holds scores in
-// [-S + b 2^sh, -S + (b+1) 2^sh)). After a unit the counts are added to the
-// query's global bins; when the unit wrote at least kTcBoundMinKeys keys of a
-// query, the global bins from the query's bound upward give the highest bin
-// edge with k written keys at or above it, published with atomicMax. The
-// bound only grows and the final top-k is unchanged (exact).
+// dropped. Every written key (of either scan) is counted in the query's 256
+// bins over its possible score range [-S, S], S = 128 sum_j |q_j| (bin b
+// holds scores in [-S + b 2^sh, -S + (b+1) 2^sh)); when a unit wrote at least
+// kTcBoundMinKeys keys of a query, the bins from the query's bound upward give
+// the highest bin edge with k written keys at or above it, published with
+// atomicMax. The bound only grows and the final top-k is unchanged (exact).
 // With deletions or exclude masks the post-filter is applied before a key is
 // counted, so every counted key is still a result candidate.
 //
@@ -87,9 +86,8 @@ struct TcMeta {                          // one unit, from its slots to its epil
     uint32_t mbmask;                     // 128-row blocks with survivors (MMAs issued for them)
 };
 
-struct TcEpi {                           // one epilogue warpgroup's scratch
-    uint32_t cnt[kTcQMax], cur[kTcQMax], gbase[kTcQMax], smax[kTcQMax], smin[kTcQMax];
-    uint32_t hist[kTcQMax][kTcBins / 2]; // two 16-bit bin counts per word
+struct TcEpi {                           // one epilogue warpgroup's per-query counters
+    uint32_t cnt[kTcQMax], cur[kTcQMax], gbase[kTcQMax];
 };
 
 template <int D>
@@ -423,16 +421,11 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                 if (gt < qn) {
                     E.cnt[gt] = 0;
                     E.cur[gt] = 0;
-                    E.smax[gt] = 0;
-                    E.smin[gt] = 0;
-                }
-                {
-                    uint4* h = reinterpret_cast<uint4*>(&E.hist[0][0]);
-                    for (int i = gt; i < qn * (kTcBins / 2) / 4; i += 128) h[i] = make_uint4(0, 0, 0, 0);
                 }
                 named_barrier(1 + g, 128);
                 const int nsl = (qn + 15) >> 4;
-                // pass 1: count the keys at or above the bound, per query and bin
+                // pass 1: count the keys at or above the bound, per query (one
+                // shared atomic per warp and query)
                 bool anyk = false;
                 for (int mb = 0; mb < 4; ++mb) {
                     if (!((mbm >> mb) & 1u)) continue;
@@ -445,29 +438,22 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
 #pragma unroll
                         for (int jj = 0; jj < 16; ++jj) {
                             const int q = sl * 16 + jj;
-                            if (q >= qn || !((mt.pass[wb][q] >> lane) & 1u)) continue;
-                            const int32_t score = int32_t(v[jj]);
-                            const uint32_t ub = uint32_t(score) ^ 0x80000000u;
-                            if (ub < mt.thr[q]) continue;
-                            if (filt && !keep_item(a, mt.qid[q], int64_t(e.x) + r)) continue;
-                            anyk = true;
-                            atomicAdd(&E.cnt[q], 1u);
-                            const int bin = (score - mt.qbase[q]) >> mt.qsh[q];
-                            atomicAdd(&E.hist[q][bin >> 1], 1u << ((bin & 1) * 16));
-                            atomicMax(&E.smax[q], ub);
-                            atomicMax(&E.smin[q], ~ub);
+                            if (q >= qn) break;  // warp-uniform
+                            bool keep = ((mt.pass[wb][q] >> lane) & 1u) &&
+                                        (uint32_t(int32_t(v[jj])) ^ 0x80000000u) >= mt.thr[q];
+                            if (filt && keep) keep = keep_item(a, mt.qid[q], int64_t(e.x) + r);
+                            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                            if (bal && lane == 0) atomicAdd(&E.cnt[q], uint32_t(__popc(bal)));
+                            anyk |= keep;
                         }
                     }
                 }
                 named_barrier(1 + g, 128);
-                if (gt < qn && E.cnt[gt]) {
-                    const int qid = mt.qid[gt];
-                    E.gbase[gt] = atomicAdd(&a.cand_cnt[int64_t(qid) * kCntStride], E.cnt[gt]);
-                    atomicMax(&a.score_rng[int64_t(qid) * kCntStride], E.smax[gt]);
-                    atomicMax(&a.score_rng[int64_t(qid) * kCntStride + 1], E.smin[gt]);
-                }
+                if (gt < qn && E.cnt[gt])
+                    E.gbase[gt] = atomicAdd(&a.cand_cnt[int64_t(mt.qid[gt]) * kCntStride], E.cnt[gt]);
                 named_barrier(1 + g, 128);
-                // pass 2: write the same keys into the reserved slots
+                // pass 2: write the same keys into the reserved slots (ranked
+                // within the warp by ballot) and count each in its score bin
                 if (__any_sync(0xffffffffu, anyk)) {
                     for (int mb = 0; mb < 4; ++mb) {
                         if (!((mbm >> mb) & 1u)) continue;
@@ -478,50 +464,50 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                             uint32_t v[16];
                             tmem_ld16(acc_base + uint32_t(mb * kTcQMax + sl * 16), v);
                             tmem_wait_ld();
-                            if (!anyk) continue;
 #pragma unroll
                             for (int jj = 0; jj < 16; ++jj) {
                                 const int q = sl * 16 + jj;
-                                if (q >= qn || !((mt.pass[wb][q] >> lane) & 1u)) continue;
+                                if (q >= qn) break;  // warp-uniform
                                 const int32_t score = int32_t(v[jj]);
-                                const uint32_t ub = uint32_t(score) ^ 0x80000000u;
-                                if (ub < mt.thr[q]) continue;
+                                bool keep = ((mt.pass[wb][q] >> lane) & 1u) &&
+                                            (uint32_t(score) ^ 0x80000000u) >= mt.thr[q];
                                 const int qid = mt.qid[q];
-                                if (filt && !keep_item(a, qid, int64_t(id))) continue;
-                                const uint32_t pos = E.gbase[q] + atomicAdd(&E.cur[q], 1u);
-                                if (int64_t(pos) < a.cap) a.cand[int64_t(qid) * a.cap + pos] = pack_key(score, id);
+                                if (filt && keep) keep = keep_item(a, qid, int64_t(id));
+                                const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                                if (!bal) continue;
+                                uint32_t b0 = 0;
+                                if (lane == 0) b0 = atomicAdd(&E.cur[q], uint32_t(__popc(bal)));
+                                b0 = __shfl_sync(0xffffffffu, b0, 0);
+                                if (keep) {
+                                    const uint32_t pos = E.gbase[q] + b0 + __popc(bal & lanemask_lt());
+                                    if (int64_t(pos) < a.cap) a.cand[int64_t(qid) * a.cap + pos] = pack_key(score, id);
+                                    atomicAdd(a.qhist + int64_t(qid) * kTcBins + ((score - mt.qbase[q]) >> mt.qsh[q]), 1u);
+                                }
                             }
                         }
                     }
                 }
-                // publish the counts (fire and forget); for a query that wrote
-                // at least kTcBoundMinKeys keys, raise its bound: the highest
-                // bin edge with at least k written keys at or above it, from
-                // the global bins at or above its bound's bin (lane l takes bins
-                // 8 l .. 8 l + 7; the warp takes queries wq, wq + 4, ...)
+                // raise the bound of each query that wrote at least
+                // kTcBoundMinKeys keys here: the highest bin edge with at least
+                // k written keys at or above it, from the query's bins at or
+                // above its bound's bin (lane l reads bins 8 l .. 8 l + 7; the
+                // warp takes queries wq, wq + 4, ...)
                 for (int q = wq; q < qn; q += 4) {
-                    const uint32_t cq = E.cnt[q];
-                    if (cq == 0) continue;  // warp-uniform
-                    uint32_t* gh = a.tc_hist + int64_t(mt.qid[q]) * kTcBins;
+                    if (E.cnt[q] < kTcBoundMinKeys) continue;  // warp-uniform
+                    const uint32_t* gh = a.qhist + int64_t(mt.qid[q]) * kTcBins;
                     const int tb = mt.thr[q] ? ((int32_t(mt.thr[q] ^ 0x80000000u) - mt.qbase[q]) >> mt.qsh[q]) : 0;
-                    const uint4 lw = reinterpret_cast<const uint4*>(&E.hist[q][0])[lane];
-                    const uint32_t wv[4] = {lw.x, lw.y, lw.z, lw.w};
-                    if (cq < kTcBoundMinKeys) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const uint32_t c = (wv[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu;
-                            if (c) atomicAdd(gh + 8 * lane + i, c);
-                        }
-                        continue;
-                    }
                     uint32_t gv[8], tot = 0;
+                    if (8 * lane + 7 >= tb) {
+                        const uint4 x0 = __ldcg(reinterpret_cast<const uint4*>(gh) + 2 * lane);
+                        const uint4 x1 = __ldcg(reinterpret_cast<const uint4*>(gh) + 2 * lane + 1);
+                        gv[0] = x0.x; gv[1] = x0.y; gv[2] = x0.z; gv[3] = x0.w;
+                        gv[4] = x1.x; gv[5] = x1.y; gv[6] = x1.z; gv[7] = x1.w;
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int bin = 8 * lane + i;
-                        const uint32_t c = (wv[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu;
-                        gv[i] = bin < tb ? 0u : (c ? atomicAdd(gh + bin, c) + c : __ldcg(gh + bin));
-                        tot += gv[i];
+                        for (int i = 0; i < 8; ++i) gv[i] = 0;
                     }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) tot += gv[i];
                     uint32_t incl = tot;  // suffix sum over lanes >= this one
 #pragma unroll
                     for (int off = 1; off < 32; off <<= 1) {

@@ -1,28 +1,29 @@
-// Final top-k for k <= ST_SMALL_K: one thread-block cluster per query
-// (cluster_topk.cuh).
+// Final top-k for batches of more than 8 queries and k <= ST_SMALL_K: one
+// thread-block cluster of CS CTAs per query -- the k best candidate keys of
+// each query, score descending then item id ascending, padded with id -1 /
+// INT32_MIN (SilverTorch: Index as Model, section on redesigning each stage
+// as a pure PyTorch module, fused Int8 ANN paragraph: a large result pool;
+// maximum top-k row of the compute cost efficiency table in the Spanish
+// translation).
 //
-// Same result as the chunked kernels of select.cu (the k best candidate keys
-// of each query, score descending then item id ascending, padded with id -1 /
-// INT32_MIN) -- SilverTorch: Index as Model, section on redesigning each
-// stage as a pure PyTorch module, fused Int8 ANN paragraph (a large result
-// pool); maximum top-k row of the compute cost efficiency table in the
-// Spanish translation -- in one launch and without global atomics: the CS
-// CTAs of a query's cluster split its candidates and talk through distributed
-// shared memory.
-//   1. each CTA histograms its share of the keys (2048 bins over the query's
-//      score range, which the scan recorded) in its own shared memory;
-//   2. the leader (rank 0) sums the CS histograms through DSMEM and finds the
-//      cut bin (the one holding the k-th best key) and every higher bin's
-//      output segment;
-//   3. every CTA reads its share again and sends each key above the cut
-//      straight to its segment in the leader's shared memory (DSMEM atomics
-//      on the segment cursors), and each key of the cut bin to the leader's
-//      tie buffer;
-//   4. the leader takes the cut bin's best, ranks every segment and writes the
-//      ids and scores.
-// A query whose candidates overflowed the scan's buffer takes the exact
-// overflow path in the leader alone (the other CTAs of its cluster return at
-// once, before any cluster barrier, so no barrier waits for them).
+// The scans counted every candidate key they wrote in the query's score bins
+// (kTcBins bins over its possible range [-S, S]), so the bin holding the k-th
+// best score -- the cut -- is known before any key is read, and so is the
+// number of keys at or above it (k plus at most the cut bin's keys):
+//   1. every CTA reads the bins and finds the cut (no communication);
+//   2. each CTA reads its share of the keys once and sends the keys at or
+//      above the cut straight into the leader's shared memory (distributed
+//      shared memory; one atomic per warp for their positions);
+//   3. the leader selects and orders the k best of those few keys in its own
+//      shared memory and writes the ids and scores.
+// Two cluster barriers in all. When the keys above the cut would not fit the
+// leader's buffer (many equal scores), the leader selects over all of the
+// query's keys in global memory instead. With deletions or exclude masks the
+// scans' counts include keys the post-filter drops, so those searches take
+// the general cluster selection (cluster_topk.cuh) with the post-filter
+// applied to every key; a query whose candidates overflowed the scan's buffer
+// takes the exact overflow path in the leader alone. Both exits happen before
+// any cluster barrier and are the same for every CTA of the cluster.
 #include "cluster_topk.cuh"
 #include "select_common.cuh"
 
@@ -31,7 +32,23 @@ namespace cg = cooperative_groups;
 namespace st {
 
 constexpr int kCBlock = 512;
-constexpr int kCTieCap = 4096;
+constexpr int kCTieCap = 4096;   // cut-bin keys of the general (post-filter) path
+constexpr int kCTieSmall = 1024; // cut-bin keys of the leader's final selection
+
+// Keys at or above the cut the leader can hold.
+__host__ __device__ __forceinline__ int cl_buf_cap(int k)
+{
+    const int c = 2 * next_pow2(k);
+    return c < 1024 ? 1024 : c;
+}
+
+__host__ __device__ __forceinline__ size_t select_cluster_smem(int k)
+{
+    const size_t ke = size_t((k + 1) & ~1), pw = size_t(next_pow2(k));
+    const size_t fast = size_t(cl_buf_cap(k)) + pw + ke + kCTieSmall;
+    const size_t general = ke + kCTieCap + pw;
+    return (fast > general ? fast : general) * 8;
+}
 
 template <int CS>
 __global__ void __launch_bounds__(kCBlock)
@@ -44,39 +61,128 @@ select_cluster_kernel(SearchArgs a)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ SelectSmem ss;
     __shared__ ClusterCut cc;
+    __shared__ int s_cut;
+    __shared__ uint32_t s_m, s_cnt;
     const int k = a.k;
     const int pwk = next_pow2(k);
-    // shared layout: [tmp: k keys, rounded up to even][tie: kCTieCap keys][out: next_pow2(k) keys]
-    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
-    uint64_t* tie = tmp + ((k + 1) & ~1);
-    uint64_t* out = tie + kCTieCap;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     const uint32_t cnt = a.cand_cnt[int64_t(q) * kCntStride];
     const int64_t n = cnt;
     uint64_t* keys = a.cand + int64_t(q) * a.cap;
     const bool filt = a.dead || a.qexclude;
+    const int2 sc = a.qscale[q];  // {-S, shift of the scans' bins}
     int m = 0;
+    uint64_t* out;
 
     if (n > a.cap || n == 0) {
-        // (cluster-uniform) the scan overflowed this query's buffer, or no
-        // candidate: the leader alone, and no cluster barrier
+        // the scan overflowed this query's buffer, or no candidate: the
+        // leader alone, and no cluster barrier
         if (rank != 0) return;
+        uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
+        uint64_t* tie = tmp + ((k + 1) & ~1);
+        out = tie + kCTieCap;
         if (n > 0) {
             const int64_t nk = overflow_path<kCBlock>(a, q, out, pwk, reinterpret_cast<int4*>(tie), ss);
             // the kept keys are at the front of the candidate buffer
             m = block_topk_sorted<kCBlock>(keys, nk, k, out, tmp, tie, kCTieCap, false, 0, 0, ss, a.err);
         }
-    } else {
-        // the scan recorded a range containing every candidate's score
-        const uint32_t* qr = a.score_rng + int64_t(q) * kCntStride;
-        const int32_t hi = int32_t(qr[0] ^ 0x80000000u);
-        const int32_t lo = int32_t(~qr[1] ^ 0x80000000u);
+    } else if (filt) {
+        // general path: every key through the post-filter
+        uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
+        uint64_t* tie = tmp + ((k + 1) & ~1);
+        out = tie + kCTieCap;
         auto keep = [&](uint64_t key) { return keep_item(a, q, key_id(key)); };
         auto compact = [&]() { return compact_cut_bin<kCBlock>(a, q, n, cc.t); };
-        m = cluster_topk<CS, kCBlock>(cluster, keys, n, k, true, lo, hi, filt, keep, compact, tmp, tie, kCTieCap,
-                                      out, ss, cc, a.err);
+        m = cluster_topk<CS, kCBlock>(cluster, keys, n, k, true, sc.x, -sc.x, filt, keep, compact, tmp, tie,
+                                      kCTieCap, out, ss, cc, a.err);
         if (m < 0) return;  // not the leader
+    } else {
+        const int cap = cl_buf_cap(k);
+        uint64_t* buf = reinterpret_cast<uint64_t*>(smem_raw);   // [cap] keys at or above the cut (leader)
+        out = buf + cap;                                         // [next_pow2(k)]
+        uint64_t* tmp = out + pwk;                               // [k, rounded up to even]
+        uint64_t* tie = tmp + ((k + 1) & ~1);                    // [kCTieSmall]
+        // 1. the cut: the highest bin with at least min(n, k) keys at or above it
+        if (warp == 0) {
+            const uint4* h = reinterpret_cast<const uint4*>(a.qhist + int64_t(q) * kTcBins);
+            const uint4 x0 = __ldcg(h + 2 * lane), x1 = __ldcg(h + 2 * lane + 1);
+            const uint32_t gv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            uint32_t tot = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tot += gv[i];
+            uint32_t incl = tot;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+                if (lane + off < 32) incl += o;
+            }
+            const uint32_t want = n < k ? uint32_t(n) : uint32_t(k);
+            uint32_t run = incl - tot;
+            int best = -1;
+            uint32_t at = 0;
+#pragma unroll
+            for (int i = 7; i >= 0; --i) {
+                run += gv[i];
+                if (best < 0 && run >= want) {
+                    best = 8 * lane + i;
+                    at = run;
+                }
+            }
+            const int top = __reduce_max_sync(0xffffffffu, best + 1) - 1;
+            if (best == top && top >= 0) {  // the lane holding the cut
+                s_cut = top;
+                s_m = at;
+            }
+            if (lane == 0 && top < 0) {  // cannot happen: the bins hold all n keys
+                s_cut = 0;
+                s_m = 0xFFFFFFFFu;
+            }
+        }
+        __syncthreads();
+        const int cut = s_cut;
+        const uint32_t mt = s_m;
+        const int32_t T = sc.x + (cut << sc.y);  // lowest score of the cut bin
+        if (mt > uint32_t(cap)) {
+            // too many keys at or above the cut (many equal or close scores):
+            // the leader selects over all of them in global memory
+            if (rank != 0) return;
+            m = block_topk_sorted<kCBlock>(keys, n, k, out, tmp, tie, kCTieSmall, true, sc.x, -sc.x, ss, a.err);
+        } else {
+            if (rank == 0 && tid == 0) s_cnt = 0;
+            cluster.sync();  // the leader's counter is zero
+            uint32_t* lcnt = cluster.map_shared_rank(&s_cnt, 0);
+            uint64_t* lbuf = cluster.map_shared_rank(buf, 0);
+            // 2. this CTA's share of the keys; those at or above the cut go to the leader
+            const int64_t s0 = n * rank / CS, s1 = n * (rank + 1) / CS;
+            constexpr int U = 8;
+            for (int64_t base = s0; base < s1; base += int64_t(kCBlock) * U) {
+                uint64_t v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int64_t i = base + int64_t(u) * kCBlock + tid;
+                    v[u] = i < s1 ? keys[i] : 0ull;
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const bool take = base + int64_t(u) * kCBlock + tid < s1 && key_score(v[u]) >= T;
+                    const unsigned bal = __ballot_sync(0xffffffffu, take);
+                    if (!bal) continue;
+                    uint32_t p0 = 0;
+                    if (lane == 0) p0 = atomicAdd(lcnt, uint32_t(__popc(bal)));
+                    p0 = __shfl_sync(0xffffffffu, p0, 0);
+                    const uint32_t pos = p0 + __popc(bal & lanemask_lt());
+                    if (take && pos < uint32_t(cap)) lbuf[pos] = v[u];
+                }
+            }
+            cluster.sync();  // every key at or above the cut is in the leader's memory
+            if (rank != 0) return;
+            // 3. the leader: the k best of them, sorted
+            const uint32_t got = s_cnt;
+            if (tid == 0 && got != mt) set_error(a.err, kErrSelectCount);
+            const int64_t nb = got < uint32_t(cap) ? int64_t(got) : int64_t(cap);
+            m = block_topk_sorted<kCBlock>(buf, nb, k, out, tmp, tie, kCTieSmall, true, T, -sc.x, ss, a.err);
+        }
     }
     for (int r = tid; r < k; r += kCBlock) {
         const uint64_t key = r < m ? out[r] : 0ull;  // key 0 reads as (id -1, INT32_MIN)
@@ -85,11 +191,6 @@ select_cluster_kernel(SearchArgs a)
     }
     if (tid == 0 && a.out_eligible) a.out_eligible[q] = int64_t(a.eligible_cnt[int64_t(q) * (kCntStride / 2)]);
     if (tid == 0 && a.out_cands) a.out_cands[q] = int64_t(cnt);
-}
-
-size_t select_cluster_smem(int k)
-{
-    return (size_t((k + 1) & ~1) + kCTieCap + size_t(next_pow2(k))) * 8;
 }
 
 template <int CS>

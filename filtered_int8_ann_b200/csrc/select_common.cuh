@@ -91,13 +91,12 @@ __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, 
     return s_count;
 }
 
-// The query's score range (a superset of its candidates' scores)
+// A range containing every score of query q: [-S, S], S = 128 sum_j |q_j|
+// (the probe records -S); sh fits it into kSelBins bins.
 __device__ __forceinline__ void query_range(const SearchArgs& a, int q, int32_t& lo, uint32_t& sh)
 {
-    const uint32_t* qr = a.score_rng + int64_t(q) * kCntStride;
-    const int32_t hi = int32_t(qr[0] ^ 0x80000000u);
-    lo = int32_t(~qr[1] ^ 0x80000000u);
-    sh = topk_shift(lo, hi);
+    lo = a.qscale[q].x;
+    sh = topk_shift(lo, -lo);
 }
 
 // Candidates the chunked kernels handle for query q: all of them, unless the

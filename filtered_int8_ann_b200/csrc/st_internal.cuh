@@ -19,7 +19,7 @@ constexpr int kQMax = 16;                  // queries per work unit
 // scan in units of up to kTcQMax queries (the MMA's N).
 constexpr int kTcQMax = 32;
 constexpr int kTcMinQDefault = 8;
-constexpr int kTcBins = 256;               // per-query score bins of the running top-k bound
+constexpr int kTcBins = 256;               // per-query score bins of the written candidate keys
 constexpr int kRngThr = 12;                // score_rng word: the query's running score bound (biased)
 
 constexpr int kProbeBlock = 512;
@@ -102,9 +102,8 @@ struct SearchArgs {
     int32_t* list_cnt;       // [nlist] queries filed into each list      (zeroed)
     int32_t* probe_done;     // [B] probe slices finished per query       (zeroed)
     uint32_t* cand_cnt;      // [B][kCntStride] candidates reserved per query, word 0 used (zeroed)
-    uint32_t* score_rng;     // [B][kCntStride] per query: [0] max of the biased scores (score ^ 2^31)
-                             // of its candidates, [1] max of their complements, [2] cut-bin keys
-                             // gathered by the final top-k (zeroed)
+    uint32_t* score_rng;     // [B][kCntStride] per-query words of the final top-k and the dense
+                             // scan's running bound (zeroed)
     uint32_t* sel_hist;      // [B][kSelBins] final top-k: candidate score histogram (zeroed)
     uint32_t* sel_cursor;    // [B][kSelBins] final top-k: keys placed per bin (zeroed)
     uint64_t* sel_out;       // [B][k] final top-k: keys above the cut, grouped by bin
@@ -126,8 +125,9 @@ struct SearchArgs {
     int4* units_tc;          // [max_units] dense units, same entries (up to kTcQMax queries)
     int32_t max_units;
     int32_t tc_min_q;        // queries per list from which its units are dense (0: no dense units)
-    int2* qscale;            // [B] per query {lowest possible score -S, bin shift}: S = 128 sum |q_j|
-    uint32_t* tc_hist;       // [B][kTcBins] keys written by the dense scan per score bin (zeroed)
+    int2* qscale;            // [B] per query {lowest possible score -S, shift of kTcBins bins over
+                             // [-S, S]}: S = 128 sum_j |q_j| bounds |<q, x>| for any int8 row x
+    uint32_t* qhist;         // [B][kTcBins] candidate keys written by the scans per score bin (zeroed)
     uint64_t* cand;          // [B][cap]
     int64_t cap;             // candidate keys per query
     uint32_t* err;           // device error word

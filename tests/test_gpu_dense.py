@@ -83,13 +83,14 @@ def test_dense_scan_parity(case):
 
 
 def test_dense_scan_prunes_candidates():
-    # 40 queries on 4 lists of 250k rows (about 2000 dense units, many per
-    # CTA), nearly all rows eligible, k = 10: once the first units have
-    # published a bound, later units must write only a fraction of their keys
-    data = small(n=1_000_000, d=128, nlist=4, sig_bits=128, hash_bits=3, B=40, nprobe=4, k=10, seed=120,
+    # 40 queries over 64 lists of about 16k rows, 16 probed per query (one of
+    # them the query's own cluster), nearly all rows eligible, k = 10, every
+    # list on the tensor cores: once the first units have published a bound,
+    # the keys of the other lists fall below it and are not written
+    data = small(n=1_000_000, d=128, nlist=64, sig_bits=128, hash_bits=3, B=40, nprobe=16, k=10, seed=120,
                  mask_flags=1, mask_lang=False)
-    exp = run_oracle(data, 4, 10)
-    got, cands = _run(data, 4, 10, 1)
+    exp = run_oracle(data, 16, 10)
+    got, cands = _run(data, 16, 10, 1)
     assert_parity(got, exp, "pruned")
     assert cands.sum() < 0.5 * got[3].sum(), (cands.sum(), got[3].sum())
 
