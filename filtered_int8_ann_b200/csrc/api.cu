@@ -405,6 +405,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     if (tc_min_q) a.units_tc = reinterpret_cast<int4*>(base + L.off_units_tc);
     a.qscale = reinterpret_cast<int2*>(base + L.off_qscale);
     a.qhist = reinterpret_cast<uint32_t*>(base + L.off_tc_hist);
+    a.count_bins = st::select_reads_bins(B, k) ? 1 : 0;
     a.cand = reinterpret_cast<uint64_t*>(base + L.off_cand);
     a.cap = cap;
     a.id_offset = idx->id_offset;

@@ -388,7 +388,7 @@ scan_kernel(SearchArgs a)
                     const int32_t score = acc0 + acc1;
                     const uint64_t pos = uint64_t(base0) + uint32_t(idx);
                     if (pos < uint64_t(a.cap)) cand[pos] = pack_key(score, uint32_t(i));
-                    atomicAdd(qh + ((score - sc.x) >> sc.y), 1u);  // the key's score bin
+                    if (a.count_bins) count_bin(qh, (score - sc.x) >> sc.y, __activemask());
                 }
             }
         } else {
@@ -434,7 +434,7 @@ scan_kernel(SearchArgs a)
                         const uint64_t pos = uint64_t(slot0) + __popc(bal & lanemask_lt());
                         const int32_t score = acc0 + acc1;
                         if (pos < uint64_t(a.cap)) a.cand[int64_t(qg) * a.cap + int64_t(pos)] = pack_key(score, uint32_t(i));
-                        atomicAdd(a.qhist + int64_t(qg) * kTcBins + ((score - sc.x) >> sc.y), 1u);
+                        if (a.count_bins) count_bin(a.qhist + int64_t(qg) * kTcBins, (score - sc.x) >> sc.y, bal);
                     }
                     if (lane == s) run += __popc(bal);
                 }

@@ -35,7 +35,7 @@
 // keys that can no longer enter a query's top-k are not written at all. Every
 // written key is a real candidate, so if at least k written keys have scores
 // >= T, the query's k-th best score is >= T and any key below T can be
-// dropped. Every written key (of either scan) is counted in the query's 256
+// dropped. Every written key (of either scan) is counted in the query's 1024
 // bins over its possible score range [-S, S], S = 128 sum_j |q_j| (bin b
 // holds scores in [-S + b 2^sh, -S + (b+1) 2^sh)); when a unit wrote at least
 // kTcBoundMinKeys keys of a query, the bins from the query's bound upward give
@@ -89,6 +89,16 @@ struct TcMeta {                          // one unit, from its slots to its epil
 struct TcEpi {                           // one epilogue warpgroup's per-query counters
     uint32_t cnt[kTcQMax], cur[kTcQMax], gbase[kTcQMax];
 };
+
+#ifdef ST_TC_PROF
+// Per-CTA cycle counters of the pipeline roles (a measuring build only).
+static __device__ unsigned long long g_tc_prof[1024][16];
+#define TC_T0(v) const long long v = clock64()
+#define TC_ACC(slot, v) atomicAdd(&g_tc_prof[blockIdx.x][slot], (unsigned long long)(clock64() - (v)))
+#else
+#define TC_T0(v)
+#define TC_ACC(slot, v)
+#endif
 
 template <int D>
 __device__ __forceinline__ uint32_t swz(int r, int c)
@@ -349,23 +359,33 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
         }
         for (int j = 0; j < n_iter; ++j) {
             const int s = j % S, m = j % kTcMeta, p = j & 1;
+            TC_T0(t0);
             cp_async_wait_group<2>();  // planes of unit j
             __syncwarp();
+            TC_T0(t1);
             test_unit(m, p);
+            TC_T0(t2);
             if (j >= S && !wait(&empty_bar[s], uint32_t(j / S - 1) & 1u)) break;
+            TC_T0(t3);
             issue_rows(m, s);
             cp_async_commit();
             __syncwarp();
             if (lane == 0) mbar_arrive(&meta_full[m]);  // slots, pass words and row blocks of unit j
+            TC_T0(t4);
             if (j >= 1) {
                 cp_async_wait_group<2>();  // rows of unit j - 1
                 gathers_done((j - 1) % S);
             }
+            TC_T0(t5);
             if (j + 2 < n_iter) store_and_request((j + 2) % kTcMeta, p, nxt);
             cp_async_commit();
+            TC_T0(t6);
             if (j + 3 < n_iter) {
                 nxt = load_slots(j + 3);
                 finish_slots(nxt);
+            }
+            if (lane == 0) {
+                TC_ACC(1, t0); TC_ACC(2, t1); TC_ACC(3, t2); TC_ACC(4, t3); TC_ACC(5, t4); TC_ACC(6, t5); TC_ACC(7, t6);
             }
         }
         cp_async_wait_all();
@@ -374,8 +394,11 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
         // ================================ MMA =================================
         for (int j = 0; j < n_iter; ++j) {
             const int s = j % S, g = j & 1, m = j % kTcMeta;
+            TC_T0(t0);
             if (!wait(&full_bar[s], uint32_t(j / S) & 1u)) break;
+            TC_T0(t1);
             if (j >= 2 && !wait(&acc_empty[g], uint32_t(j / 2 - 1) & 1u)) break;
+            if (lane == 0) { TC_ACC(8, t0); TC_ACC(9, t1); }
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t mbm = meta[m].mbmask;
@@ -410,8 +433,11 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
         const uint32_t acc_base = tmem + (uint32_t(wq * 32) << 16) + uint32_t(g * kTcAccCols);
         for (int j = g; j < n_iter; j += 2) {
             const int m = j % kTcMeta;
+            TC_T0(e0);
             if (!wait(&meta_full[m], uint32_t(j / kTcMeta) & 1u)) break;
             if (!wait(&acc_full[g], uint32_t(j / 2) & 1u)) break;
+            if (gt == 0) TC_ACC(10 + g, e0);
+            TC_T0(e1);
             tc_fence_after();
             const TcMeta& mt = meta[m];
             const uint32_t mbm = mt.mbmask;
@@ -481,7 +507,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                                 if (keep) {
                                     const uint32_t pos = E.gbase[q] + b0 + __popc(bal & lanemask_lt());
                                     if (int64_t(pos) < a.cap) a.cand[int64_t(qid) * a.cap + pos] = pack_key(score, id);
-                                    atomicAdd(a.qhist + int64_t(qid) * kTcBins + ((score - mt.qbase[q]) >> mt.qsh[q]), 1u);
+                                    count_bin(a.qhist + int64_t(qid) * kTcBins, (score - mt.qbase[q]) >> mt.qsh[q], bal);
                                 }
                             }
                         }
@@ -490,24 +516,25 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                 // raise the bound of each query that wrote at least
                 // kTcBoundMinKeys keys here: the highest bin edge with at least
                 // k written keys at or above it, from the query's bins at or
-                // above its bound's bin (lane l reads bins 8 l .. 8 l + 7; the
-                // warp takes queries wq, wq + 4, ...)
+                // above its bound's bin (lane l reads bins 32 l .. 32 l + 31;
+                // the warp takes queries wq, wq + 4, ...)
+                constexpr int kPer = kTcBins / 32;
                 for (int q = wq; q < qn; q += 4) {
                     if (E.cnt[q] < kTcBoundMinKeys) continue;  // warp-uniform
-                    const uint32_t* gh = a.qhist + int64_t(mt.qid[q]) * kTcBins;
+                    const uint4* gh = reinterpret_cast<const uint4*>(a.qhist + int64_t(mt.qid[q]) * kTcBins) + lane * (kPer / 4);
                     const int tb = mt.thr[q] ? ((int32_t(mt.thr[q] ^ 0x80000000u) - mt.qbase[q]) >> mt.qsh[q]) : 0;
-                    uint32_t gv[8], tot = 0;
-                    if (8 * lane + 7 >= tb) {
-                        const uint4 x0 = __ldcg(reinterpret_cast<const uint4*>(gh) + 2 * lane);
-                        const uint4 x1 = __ldcg(reinterpret_cast<const uint4*>(gh) + 2 * lane + 1);
-                        gv[0] = x0.x; gv[1] = x0.y; gv[2] = x0.z; gv[3] = x0.w;
-                        gv[4] = x1.x; gv[5] = x1.y; gv[6] = x1.z; gv[7] = x1.w;
-                    } else {
+                    uint32_t gv[kPer], tot = 0;
+                    const bool mine = kPer * lane + kPer - 1 >= tb;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) gv[i] = 0;
+                    for (int i = 0; i < kPer / 4; ++i) {
+                        const uint4 x = mine ? __ldcg(gh + i) : make_uint4(0, 0, 0, 0);
+                        gv[4 * i] = x.x;
+                        gv[4 * i + 1] = x.y;
+                        gv[4 * i + 2] = x.z;
+                        gv[4 * i + 3] = x.w;
                     }
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) tot += gv[i];
+                    for (int i = 0; i < kPer; ++i) tot += gv[i];
                     uint32_t incl = tot;  // suffix sum over lanes >= this one
 #pragma unroll
                     for (int off = 1; off < 32; off <<= 1) {
@@ -516,9 +543,9 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                     }
                     uint32_t run = incl - tot, best = 0;  // keys in bins above this lane's
 #pragma unroll
-                    for (int i = 7; i >= 0; --i) {
+                    for (int i = kPer - 1; i >= 0; --i) {
                         run += gv[i];
-                        if (best == 0 && run >= uint32_t(a.k)) best = uint32_t(8 * lane + i);
+                        if (best == 0 && run >= uint32_t(a.k)) best = uint32_t(kPer * lane + i);
                     }
                     best = __reduce_max_sync(0xffffffffu, best);
                     if (lane == 0 && best > 0) {
@@ -530,10 +557,14 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
             tc_fence_before();
             named_barrier(1 + g, 128);  // every read of TMEM and of meta[m] is done
             if (gt == 0) mbar_arrive(&acc_empty[g]);
+            if (gt == 0) TC_ACC(12 + g, e1);
         }
     }
 
     // teardown: nothing of this CTA may be in flight when its TMEM is freed
+#ifdef ST_TC_PROF
+    if (tid == 0) g_tc_prof[blockIdx.x][0] += (unsigned long long)n_iter;
+#endif
     __syncthreads();
     if (s_abort && tid == 0) {
         for (int i = 0; i < S; ++i) mbar_wait(&full_bar[i], 0, 1u << 12);
@@ -546,6 +577,20 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
 }
 
 bool scan_tc_supported(int d) { return d == 64 || d == 128; }
+
+#ifdef ST_TC_PROF
+}  // namespace st
+extern "C" int st_tc_prof_read(unsigned long long* host, int clear)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(host, st::g_tc_prof, sizeof(st::g_tc_prof));
+    if (e == cudaSuccess && clear) {
+        static unsigned long long zero[1024][16];
+        e = cudaMemcpyToSymbol(st::g_tc_prof, zero, sizeof(zero));
+    }
+    return int(e);
+}
+namespace st {
+#endif
 
 template <int D, int W>
 static cudaError_t launch_tc(const SearchArgs& a, const void* tmap, int num_sms, cudaStream_t s)

@@ -357,12 +357,14 @@ size_t select_smem(int k, int* stage_cap)
 
 cudaError_t launch_select_cluster(const SearchArgs& a, int num_sms, cudaStream_t s);
 
+bool select_reads_bins(int B, int k) { return k <= ST_SMALL_K && B > kChunkedMaxB; }
+
 cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s)
 {
     // a batch of few queries may hold millions of candidates per query (a
     // flat scan): spread them over the whole GPU with the chunked kernels;
     // otherwise one cluster per query does it in one launch
-    if (a.k <= ST_SMALL_K && a.B > kChunkedMaxB) return launch_select_cluster(a, num_sms, s);
+    if (select_reads_bins(a.B, a.k)) return launch_select_cluster(a, num_sms, s);
     // the attribute is set once per device: give it the largest size any batch uses
     constexpr int kPreSmemMax = 160 * 1024;
     const size_t pre_bytes = size_t(a.B + 1) * 4;

@@ -17,8 +17,8 @@
 //   3. the leader selects and orders the k best of those few keys in its own
 //      shared memory and writes the ids and scores.
 // Two cluster barriers in all. When the keys above the cut would not fit the
-// leader's buffer (many equal scores), the leader selects over all of the
-// query's keys in global memory instead. With deletions or exclude masks the
+// leader's buffer (many equal or close scores), the general cluster selection
+// (cluster_topk.cuh) runs over the query's keys at or above the cut instead. With deletions or exclude masks the
 // scans' counts include keys the post-filter drops, so those searches take
 // the general cluster selection (cluster_topk.cuh) with the post-filter
 // applied to every key; a query whose candidates overflowed the scan's buffer
@@ -50,9 +50,39 @@ __host__ __device__ __forceinline__ size_t select_cluster_smem(int k)
     return (fast > general ? fast : general) * 8;
 }
 
+// The rare paths, kept out of line so that they do not crowd the common one's
+// registers: the exact overflow path (the leader alone) ...
+__device__ __noinline__ int cl_overflow(const SearchArgs& a, int q, int k, uint64_t* keys, uint64_t* smem_keys,
+                                        SelectSmem& ss)
+{
+    uint64_t* tmp = smem_keys;
+    uint64_t* tie = tmp + ((k + 1) & ~1);
+    uint64_t* out = tie + kCTieCap;
+    const int64_t nk = overflow_path<kCBlock>(a, q, out, next_pow2(k), reinterpret_cast<int4*>(tie), ss);
+    // the kept keys are at the front of the candidate buffer
+    return block_topk_sorted<kCBlock>(keys, nk, k, out, tmp, tie, kCTieCap, false, 0, 0, ss, a.err);
+}
+
+// ... and the general cluster selection over the keys in [lo, S] (all of
+// them through the post-filter when filt), for the post-filter and for many
+// keys at or above the cut.
+template <int CS>
+__device__ __noinline__ int cl_general(const SearchArgs& a, int q, int k, int64_t n, uint64_t* keys, bool filt,
+                                       int32_t lo, int32_t hi, uint64_t* smem_keys, SelectSmem& ss, ClusterCut& cc)
+{
+    cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+    uint64_t* tmp = smem_keys;
+    uint64_t* tie = tmp + ((k + 1) & ~1);
+    uint64_t* out = tie + kCTieCap;
+    auto keep = [&](uint64_t key) { return key_score(key) >= lo && (!filt || keep_item(a, q, key_id(key))); };
+    auto compact = [&]() { return compact_cut_bin<kCBlock>(a, q, n, cc.t); };
+    return cluster_topk<CS, kCBlock>(cluster, keys, n, k, true, lo, hi, true, keep, compact, tmp, tie, kCTieCap, out,
+                                     ss, cc, a.err);
+}
+
 template <int CS>
 __global__ void __launch_bounds__(kCBlock)
-select_cluster_kernel(SearchArgs a)
+select_cluster_kernel(const __grid_constant__ SearchArgs a)
 {
     dep_enter();
     cg::cluster_group cluster = cg::this_cluster();
@@ -79,23 +109,12 @@ select_cluster_kernel(SearchArgs a)
         // the scan overflowed this query's buffer, or no candidate: the
         // leader alone, and no cluster barrier
         if (rank != 0) return;
-        uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
-        uint64_t* tie = tmp + ((k + 1) & ~1);
-        out = tie + kCTieCap;
-        if (n > 0) {
-            const int64_t nk = overflow_path<kCBlock>(a, q, out, pwk, reinterpret_cast<int4*>(tie), ss);
-            // the kept keys are at the front of the candidate buffer
-            m = block_topk_sorted<kCBlock>(keys, nk, k, out, tmp, tie, kCTieCap, false, 0, 0, ss, a.err);
-        }
+        out = reinterpret_cast<uint64_t*>(smem_raw) + ((k + 1) & ~1) + kCTieCap;
+        if (n > 0) m = cl_overflow(a, q, k, keys, reinterpret_cast<uint64_t*>(smem_raw), ss);
     } else if (filt) {
         // general path: every key through the post-filter
-        uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
-        uint64_t* tie = tmp + ((k + 1) & ~1);
-        out = tie + kCTieCap;
-        auto keep = [&](uint64_t key) { return keep_item(a, q, key_id(key)); };
-        auto compact = [&]() { return compact_cut_bin<kCBlock>(a, q, n, cc.t); };
-        m = cluster_topk<CS, kCBlock>(cluster, keys, n, k, true, sc.x, -sc.x, filt, keep, compact, tmp, tie,
-                                      kCTieCap, out, ss, cc, a.err);
+        out = reinterpret_cast<uint64_t*>(smem_raw) + ((k + 1) & ~1) + kCTieCap;
+        m = cl_general<CS>(a, q, k, n, keys, true, sc.x, -sc.x, reinterpret_cast<uint64_t*>(smem_raw), ss, cc);
         if (m < 0) return;  // not the leader
     } else {
         const int cap = cl_buf_cap(k);
@@ -104,13 +123,15 @@ select_cluster_kernel(SearchArgs a)
         uint64_t* tmp = out + pwk;                               // [k, rounded up to even]
         uint64_t* tie = tmp + ((k + 1) & ~1);                    // [kCTieSmall]
         // 1. the cut: the highest bin with at least min(n, k) keys at or above it
+        constexpr int kPer = kTcBins / 32;  // bins per lane
         if (warp == 0) {
-            const uint4* h = reinterpret_cast<const uint4*>(a.qhist + int64_t(q) * kTcBins);
-            const uint4 x0 = __ldcg(h + 2 * lane), x1 = __ldcg(h + 2 * lane + 1);
-            const uint32_t gv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            const uint4* h = reinterpret_cast<const uint4*>(a.qhist + int64_t(q) * kTcBins) + lane * (kPer / 4);
             uint32_t tot = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) tot += gv[i];
+            for (int i = 0; i < kPer / 4; ++i) {
+                const uint4 x = __ldcg(h + i);
+                tot += x.x + x.y + x.z + x.w;
+            }
             uint32_t incl = tot;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -118,23 +139,30 @@ select_cluster_kernel(SearchArgs a)
                 if (lane + off < 32) incl += o;
             }
             const uint32_t want = n < k ? uint32_t(n) : uint32_t(k);
-            uint32_t run = incl - tot;
+            uint32_t run = incl - tot;  // keys in the bins above this lane's
             int best = -1;
             uint32_t at = 0;
-#pragma unroll
-            for (int i = 7; i >= 0; --i) {
-                run += gv[i];
-                if (best < 0 && run >= want) {
-                    best = 8 * lane + i;
-                    at = run;
+            if (run < want && incl >= want) {  // the cut is in this lane's bins: walk them down
+#pragma unroll 1
+                for (int i = kPer / 4 - 1; i >= 0 && best < 0; --i) {
+                    const uint4 x = __ldcg(h + i);
+                    const uint32_t c4[4] = {x.x, x.y, x.z, x.w};
+                    for (int j = 3; j >= 0; --j) {
+                        run += c4[j];
+                        if (run >= want) {
+                            best = kPer * lane + 4 * i + j;
+                            at = run;
+                            break;
+                        }
+                    }
                 }
             }
-            const int top = __reduce_max_sync(0xffffffffu, best + 1) - 1;
-            if (best == top && top >= 0) {  // the lane holding the cut
-                s_cut = top;
+            if (best >= 0) {  // the lane holding the cut
+                s_cut = best;
                 s_m = at;
             }
-            if (lane == 0 && top < 0) {  // cannot happen: the bins hold all n keys
+            const unsigned found = __ballot_sync(0xffffffffu, best >= 0);
+            if (lane == 0 && found == 0u) {  // cannot happen: the bins hold all n keys
                 s_cut = 0;
                 s_m = 0xFFFFFFFFu;
             }
@@ -145,9 +173,10 @@ select_cluster_kernel(SearchArgs a)
         const int32_t T = sc.x + (cut << sc.y);  // lowest score of the cut bin
         if (mt > uint32_t(cap)) {
             // too many keys at or above the cut (many equal or close scores):
-            // the leader selects over all of them in global memory
-            if (rank != 0) return;
-            m = block_topk_sorted<kCBlock>(keys, n, k, out, tmp, tie, kCTieSmall, true, sc.x, -sc.x, ss, a.err);
+            // the general cluster selection over all of them
+            out = reinterpret_cast<uint64_t*>(smem_raw) + ((k + 1) & ~1) + kCTieCap;
+            m = cl_general<CS>(a, q, k, n, keys, false, T, -sc.x, reinterpret_cast<uint64_t*>(smem_raw), ss, cc);
+            if (m < 0) return;  // not the leader
         } else {
             if (rank == 0 && tid == 0) s_cnt = 0;
             cluster.sync();  // the leader's counter is zero

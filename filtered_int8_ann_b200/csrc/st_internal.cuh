@@ -19,7 +19,7 @@ constexpr int kQMax = 16;                  // queries per work unit
 // scan in units of up to kTcQMax queries (the MMA's N).
 constexpr int kTcQMax = 32;
 constexpr int kTcMinQDefault = 8;
-constexpr int kTcBins = 256;               // per-query score bins of the written candidate keys
+constexpr int kTcBins = 1024;              // per-query score bins of the written candidate keys
 constexpr int kRngThr = 12;                // score_rng word: the query's running score bound (biased)
 
 constexpr int kProbeBlock = 512;
@@ -128,6 +128,7 @@ struct SearchArgs {
     int2* qscale;            // [B] per query {lowest possible score -S, shift of kTcBins bins over
                              // [-S, S]}: S = 128 sum_j |q_j| bounds |<q, x>| for any int8 row x
     uint32_t* qhist;         // [B][kTcBins] candidate keys written by the scans per score bin (zeroed)
+    int32_t count_bins;      // the warp scan counts its keys in qhist (the final top-k reads them)
     uint64_t* cand;          // [B][cap]
     int64_t cap;             // candidate keys per query
     uint32_t* err;           // device error word
@@ -173,6 +174,14 @@ __device__ __forceinline__ int32_t dot16(const int4 a, const int4 b, int32_t acc
 }
 
 __device__ __forceinline__ void set_error(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
+
+// Count one key in bin `bin` of `hist` for every lane of `members` (the lanes
+// that call it, all of them): lanes with the same bin add once together.
+__device__ __forceinline__ void count_bin(uint32_t* hist, int bin, unsigned members)
+{
+    const unsigned same = __match_any_sync(members, bin);
+    if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(hist + bin, uint32_t(__popc(same)));
+}
 
 __device__ __forceinline__ unsigned lanemask_lt()
 {
@@ -803,6 +812,7 @@ cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_scan_tc(const SearchArgs& a, const void* tmap, int num_sms, cudaStream_t s);
 bool scan_tc_supported(int d);
 cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s);
+bool select_reads_bins(int B, int k);  // the final top-k reads the scans' score bins
 cudaError_t launch_merge(const int64_t* ids, const int32_t* scores, int G, int B, int k, int64_t* out_ids,
                          int32_t* out_scores, cudaStream_t s);
 cudaError_t merge_error_word(uint32_t* word, bool clear);
