@@ -122,6 +122,11 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
         out = buf + cap;                                         // [next_pow2(k)]
         uint64_t* tmp = out + pwk;                               // [k, rounded up to even]
         uint64_t* tie = tmp + ((k + 1) & ~1);                    // [kCTieSmall]
+        // the leader's counter starts at zero; the cluster barrier that makes
+        // it (and every CTA's start) visible is awaited only before the
+        // first remote access
+        if (rank == 0 && tid == 0) s_cnt = 0;
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
         // 1. the cut: the highest bin with at least min(n, k) keys at or above it
         constexpr int kPer = kTcBins / 32;  // bins per lane
         if (warp == 0) {
@@ -171,6 +176,7 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
         const int cut = s_cut;
         const uint32_t mt = s_m;
         const int32_t T = sc.x + (cut << sc.y);  // lowest score of the cut bin
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
         if (mt > uint32_t(cap)) {
             // too many keys at or above the cut (many equal or close scores):
             // the general cluster selection over all of them
@@ -178,8 +184,6 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
             m = cl_general<CS>(a, q, k, n, keys, false, T, -sc.x, reinterpret_cast<uint64_t*>(smem_raw), ss, cc);
             if (m < 0) return;  // not the leader
         } else {
-            if (rank == 0 && tid == 0) s_cnt = 0;
-            cluster.sync();  // the leader's counter is zero
             uint32_t* lcnt = cluster.map_shared_rank(&s_cnt, 0);
             uint64_t* lbuf = cluster.map_shared_rank(buf, 0);
             // 2. this CTA's share of the keys; those at or above the cut go to the leader

@@ -73,7 +73,8 @@ __host__ __device__ __forceinline__ int64_t key_id(uint64_t key)
 struct PlanCtl {
     int32_t n_units;       // work units allocated by the plan (clamped to the table by the scan)
     int32_t n_dense;       // dense (tensor-core) units allocated by the plan
-    int32_t pad[2];
+    int32_t probe_done;    // queries whose probe is filed (the last one sizes the unit tables)
+    int32_t pad;
 };
 
 struct SearchArgs {
@@ -134,6 +135,12 @@ struct SearchArgs {
     uint32_t* err;           // device error word
 };
 
+
+// A list's units go to the tensor-core scan when enough queries probe it.
+__device__ __forceinline__ bool dense_list(const SearchArgs& a, int cnt)
+{
+    return a.tc_min_q > 0 && cnt >= a.tc_min_q;
+}
 
 // Programmatic dependent launch: launch_dep() lets a kernel start while its
 // predecessor in the stream drains; every such kernel calls dep_enter() first
@@ -807,6 +814,7 @@ cudaError_t launch_probe_search(const SearchArgs& a, int num_sms, cudaStream_t s
 size_t probe_noalloc_scratch_bytes(int B, int S, int P, int nlist, bool keys_in_smem);
 cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
+
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
 // tmap: the index's item rows as a 2-D tensor map (opaque CUtensorMap, 128 bytes)
 cudaError_t launch_scan_tc(const SearchArgs& a, const void* tmap, int num_sms, cudaStream_t s);
