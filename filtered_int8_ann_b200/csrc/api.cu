@@ -50,7 +50,7 @@ struct st_index {
     int64_t cand_cap_override = 0;
     int64_t id_offset = 0;
     uint32_t* dead = nullptr;        // [ceil(rows_alloc / 32)] deletion bitmap, allocated at the first deletion
-    CUtensorMap tmap;                // the item rows as a 2-D tensor (TMA tile loads of the dense scan)
+    CUtensorMap tmap[2];             // the item rows as a 2-D tensor (TMA tiles of 32 and 128 rows, dense scan)
     bool tmap_ok = false;
     int32_t tc_min_q = st::kTcMinQDefault;  // queries per list from which its units are dense
 };
@@ -142,9 +142,9 @@ st::RowMap row_map(const st_index* idx)
     return m;
 }
 
-// The item rows [rows_alloc][d] as a 2-D uint8 tensor for TMA tile loads of
-// 32 rows x d bytes into the dense scan's swizzled layout (128-byte swizzle for
-// d = 128, 64-byte for d = 64). Other d have no dense scan.
+// The item rows [rows_alloc][d] as 2-D uint8 tensors for TMA tile loads of
+// 32 and of 128 rows x d bytes into the dense scan's swizzled layout (128-byte
+// swizzle for d = 128, 64-byte for d = 64). Other d have no dense scan.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -166,13 +166,17 @@ bool make_items_tmap(st_index* idx)
     }
     const cuuint64_t dims[2] = {cuuint64_t(idx->d), cuuint64_t(idx->rows_alloc)};
     const cuuint64_t strides[1] = {cuuint64_t(idx->d)};
-    const cuuint32_t box[2] = {cuuint32_t(idx->d), 32};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = encode(&idx->tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, idx->items, dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              idx->d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    idx->tmap_ok = (r == CUDA_SUCCESS);
+    bool ok = true;
+    for (int t = 0; t < 2; ++t) {
+        const cuuint32_t box[2] = {cuuint32_t(idx->d), t == 0 ? 32u : 128u};
+        const CUresult r = encode(&idx->tmap[t], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, idx->items, dims, strides, box,
+                                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                  idx->d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        ok = ok && r == CUDA_SUCCESS;
+    }
+    idx->tmap_ok = ok;
     return idx->tmap_ok;
 }
 
@@ -425,7 +429,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     if (e == cudaSuccess) e = st::launch_plan(a, idx->num_sms, stream);
     mark(2);
     if (e == cudaSuccess) e = st::launch_scan(a, idx->num_sms, stream);
-    if (e == cudaSuccess && tc_min_q) e = st::launch_scan_tc(a, &idx->tmap, idx->num_sms, stream);
+    if (e == cudaSuccess && tc_min_q) e = st::launch_scan_tc(a, idx->tmap, idx->num_sms, stream);
     mark(3);
     if (e == cudaSuccess) e = st::launch_select(a, idx->num_sms, stream);
     mark(4);

@@ -15,7 +15,8 @@
 //     signature bit-planes (the union of its queries' mask bits, by cp.async,
 //     two units ahead), the Bloom test (pass words [32-row block][query]),
 //     then the rows: a 32-row block with many survivors (for any of the unit's
-//     queries) is copied whole by a TMA tile load, a block with few has only
+//     queries) is copied whole by a TMA tile load (a 128-row tile when four
+//     neighbouring blocks are), a block with few has only
 //     its survivors' rows gathered by cp.async, a block without survivors is
 //     not read; both land in the canonical 128-byte (d = 128) or 64-byte
 //     (d = 64) swizzled K-major layout of an operand stage, with the unit's
@@ -24,11 +25,11 @@
 //     unit's queries rounded up to 16, K = 32) into int32 accumulators in TMEM
 //     and commits to mbarriers that free the operand stage and hand the
 //     accumulators to an epilogue;
-//   * two epilogue warpgroups, one per TMEM accumulator stage (alternate
-//     units): each thread reads its row's scores (tcgen05.ld), applies the pass
-//     bits, and keeps a key only if its score reaches the query's running
-//     bound (below); kept keys are counted per query, slots are reserved with
-//     one atomic per query, and the keys are written.
+//   * four epilogue warpgroups, one per TMEM accumulator stage (every fourth
+//     unit each): each thread reads its row's scores (tcgen05.ld), applies the
+//     pass bits, and keeps a key only if its score reaches the query's running
+//     bound (below); each warp counts its kept keys per query, reserves their
+//     slots with one atomic per query (all in flight at once) and writes them.
 //
 // Running top-k bound. Intermediate results should stay on chip (Andromeda
 // review, section on why the bottleneck moved from compute to bandwidth), so
@@ -58,12 +59,15 @@ constexpr int kTcPlaneSlots = 48;        // planes one buffer holds
 #endif
 constexpr int kTcDenseBlk = ST_TC_DENSE_BLK;  // survivors of a 32-row block from which the whole block is loaded
 constexpr uint32_t kTcWaitLimit = 1u << 22;
-constexpr int kTcMeta = 8;               // units whose data are held at once
+// Units whose data are held at once: a unit's slot is refilled only after its
+// epilogue, which the producer knows to be done once S + 4 units later have
+// had their operands consumed (operand stages S, epilogue groups 4).
+constexpr int kTcMeta = 12;
 constexpr uint32_t kTcBoundMinKeys = 16; // keys of a query in one unit that make it re-read its bound
-constexpr int kTcEpiWarps = 8;           // two epilogue warpgroups
-constexpr int kTcThreads = 32 * (2 + kTcEpiWarps);
+constexpr int kTcEpiGroups = 4;         // epilogue warpgroups, one per TMEM accumulator stage
+constexpr int kTcThreads = 32 * (2 + 4 * kTcEpiGroups);
 constexpr int kTcAccCols = 4 * kTcQMax;  // TMEM columns of one unit's accumulators (4 row blocks)
-constexpr int kTcTmemCols = 2 * kTcAccCols;
+constexpr int kTcTmemCols = kTcEpiGroups * kTcAccCols;
 
 // operand stages (rows and queries of one unit each)
 template <int D>
@@ -86,8 +90,8 @@ struct TcMeta {                          // one unit, from its slots to its epil
     uint32_t mbmask;                     // 128-row blocks with survivors (MMAs issued for them)
 };
 
-struct TcEpi {                           // one epilogue warpgroup's per-query counters
-    uint32_t cnt[kTcQMax], cur[kTcQMax], gbase[kTcQMax];
+struct TcEpi {                           // one epilogue warpgroup's per-query key counts (two units)
+    uint32_t cnt[2][kTcQMax];
 };
 
 #ifdef ST_TC_PROF
@@ -118,7 +122,7 @@ __host__ __device__ constexpr size_t tc_dyn_smem()
 
 template <int D, int W>
 __global__ void __launch_bounds__(kTcThreads, 1)
-scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
+scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmap128)
 {
     dep_enter();
     const int n_units = a.ctl->n_dense < a.max_units ? a.ctl->n_dense : a.max_units;
@@ -128,7 +132,8 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
     constexpr int NPL = 64 * W;          // planes per chunk
     constexpr int CH = D / 16;           // 16-byte chunks per row
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], acc_full[2], acc_empty[2], meta_full[kTcMeta];
+    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], acc_full[kTcEpiGroups], acc_empty[kTcEpiGroups],
+        meta_full[kTcMeta];
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
@@ -146,7 +151,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
             mbar_init(&full_bar[i], 2);   // the TMA byte count's arrival + the gathers' arrival
             mbar_init(&empty_bar[i], 1);  // the MMAs reading the stage are done
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kTcEpiGroups; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 1);
         }
@@ -159,6 +164,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
         tmem_alloc(&s_tmem, kTcTmemCols);
         tmem_relinquish();
     }
+    for (int i = tid; i < kTcEpiGroups * 2 * kTcQMax; i += kTcThreads) (&epi[0].cnt[0][0])[i] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -317,8 +323,15 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
             if (lane == 0) {
                 mt.mbmask = mb;
                 mbar_arrive_expect_tx(&full_bar[s], bytes);
-                for (int b = 0; b < 16; ++b)
-                    if ((dmask >> b) & 1u) tma_load_2d(A + b * 32 * D, &tmap, 0, e.x + 32 * b, &full_bar[s]);
+                for (int r4 = 0; r4 < 4; ++r4) {
+                    const uint32_t quad = (dmask >> (4 * r4)) & 0xFu;
+                    if (quad == 0xFu) {  // the whole 128-row block in one tile
+                        tma_load_2d(A + r4 * 128 * D, &tmap128, 0, e.x + 128 * r4, &full_bar[s]);
+                        continue;
+                    }
+                    for (int b = 4 * r4; b < 4 * r4 + 4; ++b)
+                        if ((dmask >> b) & 1u) tma_load_2d(A + b * 32 * D, &tmap, 0, e.x + 32 * b, &full_bar[s]);
+                }
             }
             for (int b = 0; b < 16; ++b) {  // the survivors of the other blocks, one lane per row
                 if (((dmask >> b) & 1u) || !((mt.uni[b] >> lane) & 1u)) continue;
@@ -393,11 +406,11 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
     } else if (warp == 1) {
         // ================================ MMA =================================
         for (int j = 0; j < n_iter; ++j) {
-            const int s = j % S, g = j & 1, m = j % kTcMeta;
+            const int s = j % S, g = j % kTcEpiGroups, m = j % kTcMeta;
             TC_T0(t0);
             if (!wait(&full_bar[s], uint32_t(j / S) & 1u)) break;
             TC_T0(t1);
-            if (j >= 2 && !wait(&acc_empty[g], uint32_t(j / 2 - 1) & 1u)) break;
+            if (j >= kTcEpiGroups && !wait(&acc_empty[g], uint32_t(j / kTcEpiGroups - 1) & 1u)) break;
             if (lane == 0) { TC_ACC(8, t0); TC_ACC(9, t1); }
             tc_fence_after();
             if (lane == 0) {
@@ -425,18 +438,21 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
         }
     } else {
         // ============================== epilogue ==============================
-        const int g = (warp - 2) >> 2;             // warpgroup: TMEM stage g, units j = g, g + 2, ...
+        const int g = (warp - 2) >> 2;             // warpgroup: TMEM stage g, units j = g, g + G, ...
         const int gt = tid - 64 - 128 * g;         // thread within the warpgroup
         const int wq = warp & 3;                   // TMEM lane quarter of this warp
         TcEpi& E = epi[g];
         const bool filt = a.dead != nullptr || a.qexclude != nullptr;
         const uint32_t acc_base = tmem + (uint32_t(wq * 32) << 16) + uint32_t(g * kTcAccCols);
-        for (int j = g; j < n_iter; j += 2) {
+        // keys a query must gain in one unit before its bound is re-read
+        const uint32_t bound_min = uint32_t(a.k / 16) > kTcBoundMinKeys ? uint32_t(a.k / 16) : kTcBoundMinKeys;
+        for (int j = g, it = 0; j < n_iter; j += kTcEpiGroups, ++it) {
             const int m = j % kTcMeta;
+            uint32_t* cnt = E.cnt[it & 1];
             TC_T0(e0);
             if (!wait(&meta_full[m], uint32_t(j / kTcMeta) & 1u)) break;
-            if (!wait(&acc_full[g], uint32_t(j / 2) & 1u)) break;
-            if (gt == 0) TC_ACC(10 + g, e0);
+            if (!wait(&acc_full[g], uint32_t(j / kTcEpiGroups) & 1u)) break;
+            if (gt == 0) TC_ACC(10 + (g & 1), e0);
             TC_T0(e1);
             tc_fence_after();
             const TcMeta& mt = meta[m];
@@ -444,14 +460,10 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
             const int4 e = mt.e;
             const int qn = e.w & 0xFFFF;
             if (mbm) {
-                if (gt < qn) {
-                    E.cnt[gt] = 0;
-                    E.cur[gt] = 0;
-                }
-                named_barrier(1 + g, 128);
                 const int nsl = (qn + 15) >> 4;
-                // pass 1: count the keys at or above the bound, per query (one
-                // shared atomic per warp and query)
+                // pass 1: this warp's keys at or above the bound, counted per
+                // query in lane q
+                uint32_t myc = 0;
                 bool anyk = false;
                 for (int mb = 0; mb < 4; ++mb) {
                     if (!((mbm >> mb) & 1u)) continue;
@@ -469,17 +481,19 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                                         (uint32_t(int32_t(v[jj])) ^ 0x80000000u) >= mt.thr[q];
                             if (filt && keep) keep = keep_item(a, mt.qid[q], int64_t(e.x) + r);
                             const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                            if (bal && lane == 0) atomicAdd(&E.cnt[q], uint32_t(__popc(bal)));
+                            if (lane == q) myc += __popc(bal);
                             anyk |= keep;
                         }
                     }
                 }
-                named_barrier(1 + g, 128);
-                if (gt < qn && E.cnt[gt])
-                    E.gbase[gt] = atomicAdd(&a.cand_cnt[int64_t(mt.qid[gt]) * kCntStride], E.cnt[gt]);
-                named_barrier(1 + g, 128);
-                // pass 2: write the same keys into the reserved slots (ranked
-                // within the warp by ballot) and count each in its score bin
+                // this warp's slots: one atomic per query, all in flight at once
+                uint32_t mybase = 0;
+                if (lane < qn && myc) {
+                    mybase = atomicAdd(&a.cand_cnt[int64_t(mt.qid[lane]) * kCntStride], myc);
+                    atomicAdd(&cnt[lane], myc);
+                }
+                // pass 2: write the same keys (ranked within the warp by
+                // ballot) and count each in its score bin
                 if (__any_sync(0xffffffffu, anyk)) {
                     for (int mb = 0; mb < 4; ++mb) {
                         if (!((mbm >> mb) & 1u)) continue;
@@ -501,11 +515,10 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                                 if (filt && keep) keep = keep_item(a, qid, int64_t(id));
                                 const unsigned bal = __ballot_sync(0xffffffffu, keep);
                                 if (!bal) continue;
-                                uint32_t b0 = 0;
-                                if (lane == 0) b0 = atomicAdd(&E.cur[q], uint32_t(__popc(bal)));
-                                b0 = __shfl_sync(0xffffffffu, b0, 0);
+                                const uint32_t b0 = __shfl_sync(0xffffffffu, mybase, q);
+                                if (lane == q) mybase += __popc(bal);
                                 if (keep) {
-                                    const uint32_t pos = E.gbase[q] + b0 + __popc(bal & lanemask_lt());
+                                    const uint32_t pos = b0 + __popc(bal & lanemask_lt());
                                     if (int64_t(pos) < a.cap) a.cand[int64_t(qid) * a.cap + pos] = pack_key(score, id);
                                     count_bin(a.qhist + int64_t(qid) * kTcBins, (score - mt.qbase[q]) >> mt.qsh[q], bal);
                                 }
@@ -513,14 +526,15 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                         }
                     }
                 }
-                // raise the bound of each query that wrote at least
-                // kTcBoundMinKeys keys here: the highest bin edge with at least
-                // k written keys at or above it, from the query's bins at or
+                named_barrier(1 + g, 128);  // the unit's key counts are complete
+                // raise the bound of each query that gained at least
+                // bound_min keys here: the highest bin edge with at least k
+                // written keys at or above it, from the query's bins at or
                 // above its bound's bin (lane l reads bins 32 l .. 32 l + 31;
                 // the warp takes queries wq, wq + 4, ...)
                 constexpr int kPer = kTcBins / 32;
                 for (int q = wq; q < qn; q += 4) {
-                    if (E.cnt[q] < kTcBoundMinKeys) continue;  // warp-uniform
+                    if (cnt[q] < bound_min) continue;  // warp-uniform
                     const uint4* gh = reinterpret_cast<const uint4*>(a.qhist + int64_t(mt.qid[q]) * kTcBins) + lane * (kPer / 4);
                     const int tb = mt.thr[q] ? ((int32_t(mt.thr[q] ^ 0x80000000u) - mt.qbase[q]) >> mt.qsh[q]) : 0;
                     uint32_t gv[kPer], tot = 0;
@@ -554,10 +568,11 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
                     }
                 }
             }
+            if (gt < kTcQMax) E.cnt[(it + 1) & 1][gt] = 0;  // the counts of this group's next unit
             tc_fence_before();
             named_barrier(1 + g, 128);  // every read of TMEM and of meta[m] is done
             if (gt == 0) mbar_arrive(&acc_empty[g]);
-            if (gt == 0) TC_ACC(12 + g, e1);
+            if (gt == 0) TC_ACC(12 + (g & 1), e1);
         }
     }
 
@@ -568,7 +583,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap)
     __syncthreads();
     if (s_abort && tid == 0) {
         for (int i = 0; i < S; ++i) mbar_wait(&full_bar[i], 0, 1u << 12);
-        for (int i = 0; i < 2; ++i) mbar_wait(&acc_full[i], 0, 1u << 12);
+        for (int i = 0; i < kTcEpiGroups; ++i) mbar_wait(&acc_full[i], 0, 1u << 12);
     }
     tc_fence_before();
     __syncthreads();
@@ -593,21 +608,22 @@ namespace st {
 #endif
 
 template <int D, int W>
-static cudaError_t launch_tc(const SearchArgs& a, const void* tmap, int num_sms, cudaStream_t s)
+static cudaError_t launch_tc(const SearchArgs& a, const void* tmaps, int num_sms, cudaStream_t s)
 {
     const size_t smem = tc_dyn_smem<D>();
     const void* fn = reinterpret_cast<const void*>(scan_tc_kernel<D, W>);
     cudaError_t e = ensure_smem_attr(fn, int(smem));
     if (e != cudaSuccess) return e;
-    CUtensorMap map;
-    memcpy(&map, tmap, sizeof(map));
-    return launch_dep(scan_tc_kernel<D, W>, dim3(num_sms), dim3(kTcThreads), smem, s, a, map);
+    CUtensorMap map32, map128;
+    memcpy(&map32, tmaps, sizeof(CUtensorMap));
+    memcpy(&map128, static_cast<const CUtensorMap*>(tmaps) + 1, sizeof(CUtensorMap));
+    return launch_dep(scan_tc_kernel<D, W>, dim3(num_sms), dim3(kTcThreads), smem, s, a, map32, map128);
 }
 
-cudaError_t launch_scan_tc(const SearchArgs& a, const void* tmap, int num_sms, cudaStream_t s)
+cudaError_t launch_scan_tc(const SearchArgs& a, const void* tmaps, int num_sms, cudaStream_t s)
 {
-    if (a.d == 128) return a.W == 2 ? launch_tc<128, 2>(a, tmap, num_sms, s) : launch_tc<128, 1>(a, tmap, num_sms, s);
-    if (a.d == 64) return a.W == 2 ? launch_tc<64, 2>(a, tmap, num_sms, s) : launch_tc<64, 1>(a, tmap, num_sms, s);
+    if (a.d == 128) return a.W == 2 ? launch_tc<128, 2>(a, tmaps, num_sms, s) : launch_tc<128, 1>(a, tmaps, num_sms, s);
+    if (a.d == 64) return a.W == 2 ? launch_tc<64, 2>(a, tmaps, num_sms, s) : launch_tc<64, 1>(a, tmaps, num_sms, s);
     return cudaErrorInvalidValue;
 }
 

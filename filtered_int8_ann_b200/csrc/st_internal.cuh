@@ -816,8 +816,9 @@ cudaError_t launch_probe_noalloc(SearchArgs a, int S, cudaStream_t s);
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s);
 
 cudaError_t launch_scan(const SearchArgs& a, int num_sms, cudaStream_t s);
-// tmap: the index's item rows as a 2-D tensor map (opaque CUtensorMap, 128 bytes)
-cudaError_t launch_scan_tc(const SearchArgs& a, const void* tmap, int num_sms, cudaStream_t s);
+// tmaps: the index's item rows as two 2-D tensor maps (opaque CUtensorMap, 128
+// bytes each): tiles of 32 rows, then of 128 rows
+cudaError_t launch_scan_tc(const SearchArgs& a, const void* tmaps, int num_sms, cudaStream_t s);
 bool scan_tc_supported(int d);
 cudaError_t launch_select(const SearchArgs& a, int num_sms, cudaStream_t s);
 bool select_reads_bins(int B, int k);  // the final top-k reads the scans' score bins
