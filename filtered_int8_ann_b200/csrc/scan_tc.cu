@@ -113,11 +113,26 @@ __device__ __forceinline__ uint32_t swz(int r, int c)
     return uint32_t((r >> 3) * (8 * D) + (r & 7) * D + ((c ^ x) << 4));
 }
 
+// Dynamic shared memory of one CTA, in order: operand stages (rows, then
+// query vectors), two plane buffers, the unit ring, the epilogue counts. The
+// kernel carves its buffers from these offsets and the launch requests
+// tc_dyn_smem() (the end plus the slack for aligning the base to 1024 bytes,
+// which the swizzled operand layouts need).
+template <int D>
+struct TcLayout {
+    static constexpr size_t kA = 0;
+    static constexpr size_t kB = kA + size_t(tc_stages<D>()) * kTcRows * D;
+    static constexpr size_t kP = kB + size_t(tc_stages<D>()) * kTcQMax * D;
+    static constexpr size_t kMeta = kP + size_t(2) * kTcPlaneSlots * 64;
+    static constexpr size_t kEpi = kMeta + size_t(kTcMeta) * sizeof(TcMeta);
+    static constexpr size_t kEnd = kEpi + size_t(kTcEpiGroups) * sizeof(TcEpi);
+    static_assert(kMeta % alignof(TcMeta) == 0 && kEpi % alignof(TcEpi) == 0, "aligned carve-up");
+};
+
 template <int D>
 __host__ __device__ constexpr size_t tc_dyn_smem()
 {
-    return size_t(tc_stages<D>()) * (size_t(kTcRows) * D + size_t(kTcQMax) * D) + size_t(2) * kTcPlaneSlots * 64 +
-           kTcMeta * sizeof(TcMeta) + 2 * sizeof(TcEpi) + 1024;
+    return TcLayout<D>::kEnd + 1024;
 }
 
 template <int D, int W>
@@ -140,11 +155,12 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t raw_sa = smem_u32(smem_raw);
     unsigned char* const base = smem_raw + (((raw_sa + 1023u) & ~1023u) - raw_sa);
-    unsigned char* const Abuf = base;                                     // [S][kTcRows * D]
-    unsigned char* const Bbuf = base + S * kTcRows * D;                   // [S][kTcQMax * D]
-    uint32_t* const Pbuf = reinterpret_cast<uint32_t*>(Bbuf + S * kTcQMax * D);  // [2][kTcPlaneSlots][16]
-    TcMeta* const meta = reinterpret_cast<TcMeta*>(Pbuf + 2 * kTcPlaneSlots * 16);   // [kTcMeta]
-    TcEpi* const epi = reinterpret_cast<TcEpi*>(meta + kTcMeta);                       // [2]
+    using L = TcLayout<D>;
+    unsigned char* const Abuf = base + L::kA;                                 // [S][kTcRows * D]
+    unsigned char* const Bbuf = base + L::kB;                                 // [S][kTcQMax * D]
+    uint32_t* const Pbuf = reinterpret_cast<uint32_t*>(base + L::kP);         // [2][kTcPlaneSlots][16]
+    TcMeta* const meta = reinterpret_cast<TcMeta*>(base + L::kMeta);          // [kTcMeta]
+    TcEpi* const epi = reinterpret_cast<TcEpi*>(base + L::kEpi);              // [kTcEpiGroups]
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
