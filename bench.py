@@ -126,20 +126,25 @@ class Peaks:
                 "dp4a_tops": self.dp4a_tops, "dp4a_kind": "measured (dp4a_peak.cu, 8 chains per thread)"}
 
 
-def roofline(bytes_, ops, ms, pk, compute="dp4a"):
+def roofline(bytes_, ops, ms, pk, dense_frac=0.0):
     """Bound times of one launch (or step) and the fraction of the slower bound
-    achieved. `compute` names the unit the int8 products ran on."""
+    achieved. The int8 products of the dense units (a fraction `dense_frac` of
+    the eligible pairs) ran on the tensor cores, the others on dp4a: the
+    compute bound is the sum of the two parts' times at their peaks."""
     t = ms * 1e-3
     t_hbm = bytes_ / (pk.hbm_gbs * 1e9)
     t_tensor = ops / (pk.int8_tensor_tops * 1e12)
     t_dp4a = ops / (pk.dp4a_tops * 1e12) if pk.dp4a_tops else None
-    t_comp = t_dp4a if (compute == "dp4a" and t_dp4a is not None) else t_tensor
-    bound = "hbm" if t_hbm >= t_comp else ("alu" if compute == "dp4a" else "tensor")
+    t_tc_part = ops * dense_frac / (pk.int8_tensor_tops * 1e12)
+    t_dp_part = (ops * (1.0 - dense_frac) / (pk.dp4a_tops * 1e12)) if pk.dp4a_tops else 0.0
+    t_comp = t_tc_part + t_dp_part
+    bound = "hbm" if t_hbm >= t_comp else ("alu" if t_dp_part >= t_tc_part else "tensor")
     return {"bound": bound, "frac": max(t_hbm, t_comp) / t if t > 0 else None,
             "hbm_frac": t_hbm / t if t > 0 else None, "achieved_gbs": bytes_ / t / 1e9 if t > 0 else None,
             "int8_tensor_frac": t_tensor / t if t > 0 else None,
             "dp4a_frac": (t_dp4a / t) if (t_dp4a is not None and t > 0) else None,
-            "achieved_tops": ops / t / 1e12 if t > 0 else None}
+            "achieved_tops": ops / t / 1e12 if t > 0 else None,
+            "dense_pair_frac": dense_frac, "compute_frac": t_comp / t if t > 0 else None}
 
 
 def scan_traffic(workload):
@@ -312,6 +317,12 @@ def byte_model(data, probe, qmasks, W, d, k, nlist):
     surv = torch.zeros(data.items.shape[0], dtype=torch.bool, device=off.device)
     per_q = sizes[probe.long()].sum(1)
     b0, B = 0, probe.shape[0]
+    # eligible (query, item) pairs in lists the tensor-core scan takes (probed
+    # by at least the dense-unit threshold of queries) and in all lists
+    dmq = 8 if DENSE_MIN_Q is None else DENSE_MIN_Q
+    qcount = torch.bincount(probe.flatten().long(), minlength=nlist)
+    dense_list = (qcount >= dmq) if (dmq > 0 and d in (64, 128)) else torch.zeros_like(qcount, dtype=torch.bool)
+    pairs = pairs_dense = 0
     while b0 < B:
         b1, acc = b0, 0
         while b1 < B and (b1 == b0 or acc + int(per_q[b1]) <= (32 << 20)):
@@ -323,6 +334,9 @@ def byte_model(data, probe, qmasks, W, d, k, nlist):
         m = qmasks[owner]
         ok = torch.all((data.sigs[idx] & m) == m, dim=1)
         surv[idx[ok]] = True
+        lst = torch.repeat_interleave(pl.reshape(-1), sizes[pl.reshape(-1)])
+        pairs += int(ok.sum())
+        pairs_dense += int((ok & dense_list[lst]).sum())
         b0 = b1
     n_surv = int(surv.sum())
     extra = nlist * d + B * (d + 8 * W) + B * k * 12
@@ -331,7 +345,8 @@ def byte_model(data, probe, qmasks, W, d, k, nlist):
     return {"scan_planes": scan_planes, "scan_rowmajor": scan_rowmajor,
             "step_planes": scan_planes + extra, "step_rowmajor": scan_rowmajor + extra,
             "full_scan": (8 * W + d) * scanned, "plane_bytes": plane_bytes,
-            "scanned_items": scanned, "survivor_rows": n_surv, "distinct_lists": int(lists.numel())}
+            "scanned_items": scanned, "survivor_rows": n_surv, "distinct_lists": int(lists.numel()),
+            "dense_pair_frac": pairs_dense / pairs if pairs else 0.0}
 
 
 def bloom_fp(data, probe, q0):
@@ -574,10 +589,10 @@ def measure_config(st, name, B, steps, warmup, flush_reps, flush, pk, pool=4, da
            "candidates_per_query": float(cands.double().mean()),
            "candidate_bytes_per_step": float(cands.sum(1).double().mean()) * 8,
            "bytes": mdl, "int8_ops": {"scan": ops_scan, "step": ops_step},
-           "scan_roofline": {"planes": roofline(mdl["scan_planes"], ops_scan, stg[2], pk),
-                             "rowmajor": roofline(mdl["scan_rowmajor"], ops_scan, stg[2], pk)},
-           "step_roofline": {"planes": roofline(mdl["step_planes"], ops_step, ms, pk),
-                             "rowmajor": roofline(mdl["step_rowmajor"], ops_step, ms, pk)},
+           "scan_roofline": {"planes": roofline(mdl["scan_planes"], ops_scan, stg[2], pk, mdl["dense_pair_frac"]),
+                             "rowmajor": roofline(mdl["scan_rowmajor"], ops_scan, stg[2], pk, mdl["dense_pair_frac"])},
+           "step_roofline": {"planes": roofline(mdl["step_planes"], ops_step, ms, pk, mdl["dense_pair_frac"]),
+                             "rowmajor": roofline(mdl["step_rowmajor"], ops_step, ms, pk, mdl["dense_pair_frac"])},
            "l2": f"steps cycle {pool} query batches; l2_flushed writes {FLUSH_BYTES >> 20} MB between steps"}
     if recall_flat and P < wl.nlist <= 4096:
         # flat filtered search = the same index probed with nprobe = nlist
@@ -905,7 +920,7 @@ def main():
 
     if rank == 0:
         traffic = scan_traffic(wl.name)
-        scan_rf = roofline(mean["scan_planes"], ops_scan, scan_ms, pk)
+        scan_rf = roofline(mean["scan_planes"], ops_scan, scan_ms, pk, mean["dense_pair_frac"])
         line = {
             "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
@@ -930,10 +945,12 @@ def main():
                          "int8_tensor_frac": scan_rf["int8_tensor_frac"], "dp4a_frac": scan_rf["dp4a_frac"],
                          "signature_plane_bytes_per_launch": mean["plane_bytes"],
                          "rowmajor_model_bytes_per_launch": mean["scan_rowmajor"],
-                         "rowmajor_model_frac": roofline(mean["scan_rowmajor"], ops_scan, scan_ms, pk)["hbm_frac"],
+                         "rowmajor_model_frac": roofline(mean["scan_rowmajor"], ops_scan, scan_ms, pk,
+                                                                         mean["dense_pair_frac"])["hbm_frac"],
+                         "dense_pair_frac": mean["dense_pair_frac"],
                          "full_scan_bytes_per_launch": mean["full_scan"]},
-            "step_roofline": {"planes": roofline(mean["step_planes"], ops_step, ms / K, pk),
-                              "rowmajor": roofline(mean["step_rowmajor"], ops_step, ms / K, pk),
+            "step_roofline": {"planes": roofline(mean["step_planes"], ops_step, ms / K, pk, mean["dense_pair_frac"]),
+                              "rowmajor": roofline(mean["step_rowmajor"], ops_step, ms / K, pk, mean["dense_pair_frac"]),
                               "step_bytes_planes": mean["step_planes"], "step_bytes_rowmajor": mean["step_rowmajor"],
                               "int8_ops_per_step": ops_step},
             "peaks": pk.describe(),

@@ -72,3 +72,39 @@ def test_cpu_baseline_reports_parallel_and_single_thread_rates():
     assert cpu["cores"] == oracle.max_threads()
     assert cpu["single_thread"]["value"] > 0 and cpu["single_thread"]["unit"] == "queries/s"
     assert "cpu_model" in cpu
+
+
+class _Peaks:
+    hbm_gbs = 1000.0          # 1 ms per GB
+    int8_tensor_tops = 1000.0  # 1 ms per 10^12 ops
+    dp4a_tops = 100.0          # 10 ms per 10^12 ops
+
+
+def test_roofline_splits_the_int8_products_between_tensor_cores_and_dp4a():
+    # 1 GB and 10^12 products measured in 20 ms: HBM 1 ms; compute 10 ms on
+    # dp4a alone, 1 ms on the tensor cores alone, 0.5 + 5 ms half and half
+    r = bench.roofline(1e9, 1e12, 20.0, _Peaks, 0.0)
+    assert r["bound"] == "alu" and abs(r["frac"] - 0.5) < 1e-12 and abs(r["hbm_frac"] - 0.05) < 1e-12
+    r = bench.roofline(1e9, 1e12, 20.0, _Peaks, 1.0)
+    assert r["bound"] == "hbm" and abs(r["frac"] - 0.05) < 1e-12 and abs(r["compute_frac"] - 0.05) < 1e-12
+    r = bench.roofline(1e9, 1e12, 20.0, _Peaks, 0.5)
+    assert r["bound"] == "alu" and abs(r["compute_frac"] - 5.5 / 20.0) < 1e-12
+    r = bench.roofline(1e8, 4e12, 20.0, _Peaks, 1.0)
+    assert r["bound"] == "tensor" and abs(r["frac"] - 0.2) < 1e-12
+
+
+def test_byte_model_counts_dense_list_pairs():
+    # every query probes every list: with the threshold at B all pairs are in
+    # dense lists (d = 64 has the tensor-core scan), with 0 none are
+    data = small(n=3000, d=64, nlist=4, sig_bits=64, B=9, nprobe=4, k=20, seed=11, mask_flags=1)
+    probe = torch.arange(4, dtype=torch.int32).repeat(9, 1)
+    old = bench.DENSE_MIN_Q
+    try:
+        bench.DENSE_MIN_Q = 9
+        assert bench.byte_model(data, probe, data.masks, 1, 64, 20, 4)["dense_pair_frac"] == 1.0
+        bench.DENSE_MIN_Q = 10
+        assert bench.byte_model(data, probe, data.masks, 1, 64, 20, 4)["dense_pair_frac"] == 0.0
+        bench.DENSE_MIN_Q = 0
+        assert bench.byte_model(data, probe, data.masks, 1, 64, 20, 4)["dense_pair_frac"] == 0.0
+    finally:
+        bench.DENSE_MIN_Q = old
