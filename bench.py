@@ -44,17 +44,17 @@ FLUSH_BYTES = 512 << 20  # written between L2-flushed steps (L2 is 126 MB)
 
 
 def kernels_per_search(k, B, d):
-    """Kernels one search launches: probe score + select (which also sizes the
-    unit tables), units write, the warp scan, the tensor-core scan (when a
-    list can have the dense-unit threshold of queries: B >= that threshold,
-    d = 64 or 128), then the cluster final top-k (k <= 4096, B > 8), hist +
-    scatter + finish (k <= 4096, B <= 8) or hist + scatter + ties + rank
-    (larger k). The memset node is not counted."""
+    """Kernels one search launches: probe score + select, units alloc + write,
+    the warp scan, the tensor-core scan (when a list can have the dense-unit
+    threshold of queries: B >= that threshold, d = 64 or 128), then the
+    cluster final top-k (k <= 4096, B > 8), hist + scatter + finish (k <= 4096,
+    B <= 8) or hist + scatter + ties + rank (larger k). The memset node is not
+    counted."""
     dmq = 8 if DENSE_MIN_Q is None else DENSE_MIN_Q
     tc = 1 if (d in (64, 128) and dmq > 0 and B >= dmq) else 0
     if k > 4096:
-        return 8 + tc
-    return (7 if B <= 8 else 5) + tc
+        return 9 + tc
+    return (8 if B <= 8 else 6) + tc
 
 
 def parse():

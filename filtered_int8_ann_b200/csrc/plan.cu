@@ -8,9 +8,10 @@
 //
 // The probe kernel already filed each query into the slot row of every list it
 // chose (slots L*B .. L*B + count-1), so no scan over lists or scatter of pairs
-// is needed here. The last probe CTA to finish sizes every list's block of
-// the unit tables (size_units, one CTA: a scan of the lists' unit counts), and
-// one small balanced kernel writes the entries:
+// is needed here. Two small balanced kernels:
+//   * units_alloc: one thread per list; a warp-wide scan of the lists' unit
+//     counts and one atomic per warp give every probed list its block of the
+//     unit table (blocks land in completion order, which the scan ignores);
 //   * units_write: one thread per list chunk (the index's chunk table, list by
 //     list: a list's creation chunks, then its append chunks), so a list of
 //     millions of rows is written by thousands of threads: the thread writes
@@ -21,6 +22,50 @@ namespace st {
 
 constexpr int kUnitsBlock = 256;
 
+__global__ void __launch_bounds__(kUnitsBlock)
+units_alloc_kernel(SearchArgs a)
+{
+    dep_enter();
+    const int lane = threadIdx.x & 31;
+    const int L = blockIdx.x * kUnitsBlock + threadIdx.x;
+    uint32_t u = 0;
+    bool dense = false;
+    if (L < a.nlist) {
+        const int cnt = a.list_cnt[L];
+        if (cnt > 0) {
+            dense = dense_list(a, cnt);
+            const int qg = dense ? kTcQMax : kQMax;
+            u = uint32_t(a.chunk_start[L + 1] - a.chunk_start[L]) * uint32_t((cnt + qg - 1) / qg);
+        }
+    }
+    // one warp-wide scan per table (sparse, dense)
+    const uint32_t us = dense ? 0u : u, ud = dense ? u : 0u;
+    uint32_t is = us, id = ud;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t ts = __shfl_up_sync(0xffffffffu, is, off), td = __shfl_up_sync(0xffffffffu, id, off);
+        if (lane >= off) {
+            is += ts;
+            id += td;
+        }
+    }
+    const uint32_t tot_s = __shfl_sync(0xffffffffu, is, 31), tot_d = __shfl_sync(0xffffffffu, id, 31);
+    if (tot_s + tot_d == 0u) return;  // warp-uniform
+    uint32_t bs = 0, bd = 0;
+    if (lane == 31) {
+        if (tot_s) {
+            bs = atomicAdd(reinterpret_cast<unsigned int*>(&a.ctl->n_units), tot_s);
+            if (uint64_t(bs) + tot_s > uint64_t(a.max_units)) set_error(a.err, kErrUnitTable);
+        }
+        if (tot_d) {
+            bd = atomicAdd(reinterpret_cast<unsigned int*>(&a.ctl->n_dense), tot_d);
+            if (uint64_t(bd) + tot_d > uint64_t(a.max_units)) set_error(a.err, kErrUnitTable);
+        }
+    }
+    bs = __shfl_sync(0xffffffffu, bs, 31);
+    bd = __shfl_sync(0xffffffffu, bd, 31);
+    if (u > 0) a.list_ustart[L] = dense ? int32_t(bd + id - ud) : int32_t(bs + is - us);
+}
 
 __global__ void __launch_bounds__(kUnitsBlock)
 units_write_kernel(SearchArgs a)
@@ -65,6 +110,8 @@ units_write_kernel(SearchArgs a)
 cudaError_t launch_plan(const SearchArgs& a, int num_sms, cudaStream_t s)
 {
     (void)num_sms;
+    cudaError_t e = launch_dep(units_alloc_kernel, dim3((a.nlist + kUnitsBlock - 1) / kUnitsBlock), dim3(kUnitsBlock), 0, s, a);
+    if (e != cudaSuccess) return e;
     return launch_dep(units_write_kernel, dim3((a.n_chunks + kUnitsBlock - 1) / kUnitsBlock), dim3(kUnitsBlock), 0, s, a);
 }
 

@@ -15,15 +15,15 @@
 //     thread, and the (score, list id) keys go to a [B][nlist] array that
 //     stays in L2;
 //   * probe_select_cluster_kernel: one thread-block cluster per query (up to
-//     8 CTAs at small batches, so the whole GPU works on the selections). Each
-//     CTA selects the nprobe best keys of its slice of the query's row (a
-//     2048-bin histogram over the slice's score range and its suffix counts
-//     give the bin holding the nprobe-th best score, so only that bin needs an
-//     exact selection) and hands them to the leader CTA through distributed
-//     shared memory; the leader selects the nprobe best of those, sorts them,
-//     writes the probe result and files the query into every chosen list: it
-//     takes the next rank of the list's query counter and writes its id and
-//     mask into the list's slot row, which the plan and the scan read.
+//     8 CTAs at small batches, so the whole GPU works on the selections). The
+//     keys' score range, a 2048-bin histogram over it summed through
+//     distributed shared memory, and the suffix counts give the bin holding
+//     the nprobe-th best score, so only the keys at or above that bin (a few
+//     more than nprobe) reach the leader CTA for the exact selection and the
+//     sort. The leader then writes the probe result and files the query into
+//     every chosen list: it takes the next rank of the list's query counter
+//     and writes its id and mask into the list's slot row, which the plan and
+//     the scan read.
 // The allocation-free probe-only call keeps an older single-kernel form (CTAs
 // over query x centroid slices, last CTA merges), whose scratch is bounded.
 #include <mutex>
@@ -228,73 +228,10 @@ probe_score_kernel(SearchArgs a)
         if (g * kQPer + j < nq) out[int64_t(j) * ld] = pack_key(acc[j], uint32_t(c));
 }
 
-// The plan's first step, folded into the probe (done by the last query's
-// CTA): every list's units (chunks x query groups), an exclusive scan per
-// table over the lists in order, and the totals.
-template <int BLOCK>
-__device__ void size_units(const SearchArgs& a)
-{
-    __shared__ uint32_t part_s[32], part_d[32];
-    const int nlist = a.nlist;
-    const int per = (nlist + BLOCK - 1) / BLOCK;
-    const int l0 = threadIdx.x * per;
-    uint32_t loc_s = 0, loc_d = 0;
-    for (int j = 0; j < per; ++j) {
-        const int L = l0 + j;
-        if (L >= nlist) break;
-        const int cnt = __ldcg(a.list_cnt + L);
-        if (cnt <= 0) continue;
-        const bool dense = dense_list(a, cnt);
-        const int qg = dense ? kTcQMax : kQMax;
-        const uint32_t u = uint32_t(a.chunk_start[L + 1] - a.chunk_start[L]) * uint32_t((cnt + qg - 1) / qg);
-        if (dense) loc_d += u;
-        else loc_s += u;
-    }
-    uint32_t tot_s, tot_d;
-    uint32_t run_s = block_excl_scan<BLOCK>(loc_s, part_s, tot_s);
-    uint32_t run_d = block_excl_scan<BLOCK>(loc_d, part_d, tot_d);
-    for (int j = 0; j < per; ++j) {
-        const int L = l0 + j;
-        if (L >= nlist) break;
-        const int cnt = __ldcg(a.list_cnt + L);
-        if (cnt <= 0) continue;
-        const bool dense = dense_list(a, cnt);
-        const int qg = dense ? kTcQMax : kQMax;
-        const uint32_t u = uint32_t(a.chunk_start[L + 1] - a.chunk_start[L]) * uint32_t((cnt + qg - 1) / qg);
-        if (dense) {
-            a.list_ustart[L] = int32_t(run_d);
-            run_d += u;
-        } else {
-            a.list_ustart[L] = int32_t(run_s);
-            run_s += u;
-        }
-    }
-    if (threadIdx.x == 0) {
-        a.ctl->n_units = int32_t(tot_s);
-        a.ctl->n_dense = int32_t(tot_d);
-        if (uint64_t(tot_s) > uint64_t(a.max_units) || uint64_t(tot_d) > uint64_t(a.max_units))
-            set_error(a.err, kErrUnitTable);
-    }
-}
-// One cluster of CS CTAs per query, in two levels: every CTA selects the
-// nprobe best keys of its slice of the query's row of centroid keys (its own
-// shared memory, block barriers only) and writes them into its slots of the
-// leader's gather buffer (distributed shared memory); after one cluster
-// barrier the leader selects the nprobe best of those CS * nprobe keys, sorts
-// them, and writes the probe result and the filing. The cluster's start is
-// awaited (a split arrive / wait) only just before the first remote write.
+// One cluster of CS CTAs per query: the nprobe best keys of the query's row
+// of centroid keys (cluster_topk.cuh), then its probe result and filing.
 constexpr int kProbeCBlock = 512;
 constexpr int kProbeTieCap = 1024;
-constexpr int kProbeGatherMax = 4096;  // CS * nprobe keys the leader gathers
-
-__device__ __forceinline__ void cluster_arrive_relaxed()
-{
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait()
-{
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-}
 
 template <int CS>
 __global__ void __launch_bounds__(kProbeCBlock)
@@ -302,63 +239,38 @@ probe_select_cluster_kernel(SearchArgs a)
 {
     dep_enter();
     cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
-    const int rank = int(cluster.block_rank());
     const int b = int(blockIdx.x) / CS;
-    const int P = a.P, nlist = a.nlist;
-    const int pw = next_pow2(P), pe = (P + 1) & ~1;
+    const int P = a.P;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ SelectSmem ss;
-    // shared layout: [local best: pw][tmp: P, even][tie: kProbeTieCap][gather: CS * P][out: pw]
-    uint64_t* loc = reinterpret_cast<uint64_t*>(smem_raw);
-    uint64_t* tmp = loc + pw;
-    uint64_t* tie = tmp + pe;
-    uint64_t* gather = tie + kProbeTieCap;
-    uint64_t* out = gather + CS * P;
-    const uint64_t* row = a.probe_keys + int64_t(b) * probe_keys_ld(nlist);
-    if (CS > 1) cluster_arrive_relaxed();
-    const int s0 = int(int64_t(nlist) * rank / CS), s1 = int(int64_t(nlist) * (rank + 1) / CS);
-    const int m_loc = block_topk_sorted<kProbeCBlock>(row + s0, s1 - s0, P, CS > 1 ? loc : out, tmp, tie,
-                                                      kProbeTieCap, false, 0, 0, ss, a.err);
-    int m = m_loc;
-    if (CS > 1) {
-        cluster_wait();  // every CTA of the cluster has started
-        uint64_t* lg = cluster.map_shared_rank(gather, 0) + rank * P;
-        for (int i = threadIdx.x; i < P; i += kProbeCBlock) lg[i] = i < m_loc ? loc[i] : 0ull;
-        cluster.sync();  // the leader holds every CTA's best
-        if (rank != 0) return;
-        // the best P of them (every slice holds at least P keys, so there is
-        // no empty slot)
-        m = block_topk_sorted<kProbeCBlock>(gather, int64_t(CS) * P, P, out, tmp, tie, kProbeTieCap, false, 0, 0, ss,
-                                            a.err);
-    }
+    __shared__ ClusterCut cc;
+    // shared layout: [tmp: P keys, rounded up to even][tie: kProbeTieCap keys][out: next_pow2(P) keys]
+    uint64_t* tmp = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* tie = tmp + ((P + 1) & ~1);
+    uint64_t* out = tie + kProbeTieCap;
+    const uint64_t* row = a.probe_keys + int64_t(b) * probe_keys_ld(a.nlist);
+    auto none = [](uint64_t) { return true; };
+    auto no_compact = []() { return 0; };
+    const int m = cluster_topk<CS, kProbeCBlock>(cluster, row, a.nlist, P, false, 0, 0, false, none, no_compact, tmp,
+                                                 tie, kProbeTieCap, out, ss, cc, a.err);
+    if (m < 0) return;  // not the leader
     if (threadIdx.x == 0 && m != P) set_error(a.err, kErrSelectCount);
     file_query<kProbeCBlock, true>(a, b, out);
-    // the last query to be filed (a counter, no waiting) sizes the unit tables
-    __shared__ int s_last;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&a.ctl->probe_done, 1) == a.B - 1;
-    __syncthreads();
-    if (s_last) {
-        __threadfence();
-        size_units<kProbeCBlock>(a);
-    }
 }
 
-static size_t probe_select_smem(int P, int cs)
+static size_t probe_select_smem(int P)
 {
-    return (size_t(2) * next_pow2(P) + ((P + 1) & ~1) + kProbeTieCap + size_t(cs) * P) * 8;
+    return (size_t((P + 1) & ~1) + kProbeTieCap + size_t(next_pow2(P))) * 8;
 }
 
 template <int CS>
 static cudaError_t launch_probe_select(const SearchArgs& a, cudaStream_t s)
 {
     const void* fn = reinterpret_cast<const void*>(probe_select_cluster_kernel<CS>);
-    // the largest request of this cluster size (the gather bounds nprobe when CS > 1)
-    cudaError_t e = ensure_smem_attr(fn, int(probe_select_smem(CS == 1 ? ST_MAX_NPROBE : kProbeGatherMax / CS, CS)));
+    cudaError_t e = ensure_smem_attr(fn, int(probe_select_smem(ST_MAX_NPROBE)));
     if (e != cudaSuccess) return e;
     return launch_dep_cluster(probe_select_cluster_kernel<CS>, dim3(unsigned(a.B) * CS), dim3(kProbeCBlock),
-                              probe_select_smem(a.P, CS), CS, s, a);
+                              probe_select_smem(a.P), CS, s, a);
 }
 
 cudaError_t launch_probe_search(const SearchArgs& a, int num_sms, cudaStream_t s)
@@ -370,9 +282,7 @@ cudaError_t launch_probe_search(const SearchArgs& a, int num_sms, cudaStream_t s
     probe_score_kernel<<<grid, kScoreBlock, qbytes, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    int cs = cluster_size_for(a.B, num_sms);
-    while (cs > 1 && (cs * a.P > kProbeGatherMax || a.nlist < cs * a.P)) cs >>= 1;  // the gather fits; slices hold P
-    switch (cs) {
+    switch (cluster_size_for(a.B, num_sms)) {
     case 8: return launch_probe_select<8>(a, s);
     case 4: return launch_probe_select<4>(a, s);
     case 2: return launch_probe_select<2>(a, s);

@@ -73,8 +73,7 @@ __host__ __device__ __forceinline__ int64_t key_id(uint64_t key)
 struct PlanCtl {
     int32_t n_units;       // work units allocated by the plan (clamped to the table by the scan)
     int32_t n_dense;       // dense (tensor-core) units allocated by the plan
-    int32_t probe_done;    // queries whose probe is filed (the last one sizes the unit tables)
-    int32_t pad;
+    int32_t pad[2];
 };
 
 struct SearchArgs {
