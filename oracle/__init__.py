@@ -41,6 +41,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_search_ids.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, i32, i32, i32, i32,
                                       P, P, P, P, i32]
     lib.oracle_search_ids.restype = i32
+    lib.oracle_search_or.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, i32, i32, i32, i32, i32,
+                                     P, P, P, P, i32]
+    lib.oracle_search_or.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     return lib
@@ -110,6 +113,40 @@ def search(items, sigs, offsets, centroids, queries, masks, nprobe, k, b0=0, b1=
         rc = lib.oracle_search_ids(_ptr(items), _ptr(sigs), _ptr(offsets), _ptr(row_ids), _ptr(centroids), n,
                                    d, nlist, W, _ptr(queries), _ptr(masks), b0, b1, nprobe, k, _ptr(ids),
                                    _ptr(scores), _ptr(probe_out), _ptr(elig), nthreads)
+    assert rc == 0, "oracle allocation failed"
+    return ids, scores, probe_out, elig
+
+
+def search_or(items, sigs, offsets, centroids, queries, mask_sets, nprobe, k, b0=0, b1=None,
+              nthreads=1, lib=None, row_ids=None):
+    """Search with A alternative masks per query, mask_sets uint64 [B, A, W]:
+    an item is eligible when it passes any of its query's masks. Same outputs
+    as search()."""
+    lib = lib or load()
+    items = np.ascontiguousarray(items, dtype=np.int8)
+    sigs = np.ascontiguousarray(sigs).view(np.uint64)
+    if sigs.ndim == 1:
+        sigs = sigs.reshape(-1, 1)
+    offsets = np.ascontiguousarray(offsets, dtype=np.int64)
+    centroids = np.ascontiguousarray(centroids, dtype=np.int8)
+    queries = np.ascontiguousarray(queries, dtype=np.int8)
+    mask_sets = np.ascontiguousarray(mask_sets).view(np.uint64)
+    n, d = items.shape
+    W = sigs.shape[1]
+    B = queries.shape[0]
+    assert mask_sets.ndim == 3 and mask_sets.shape[0] == B and mask_sets.shape[2] == W
+    A = mask_sets.shape[1]
+    nlist = centroids.shape[0]
+    b1 = B if b1 is None else b1
+    nb = b1 - b0
+    ids = np.empty((nb, k), dtype=np.int64)
+    scores = np.empty((nb, k), dtype=np.int32)
+    probe_out = np.empty((nb, nprobe), dtype=np.int32)
+    elig = np.empty(nb, dtype=np.int64)
+    rid = None if row_ids is None else np.ascontiguousarray(row_ids, dtype=np.int64)
+    rc = lib.oracle_search_or(_ptr(items), _ptr(sigs), _ptr(offsets), None if rid is None else _ptr(rid),
+                              _ptr(centroids), n, d, nlist, W, _ptr(queries), _ptr(mask_sets), A, b0, b1,
+                              nprobe, k, _ptr(ids), _ptr(scores), _ptr(probe_out), _ptr(elig), nthreads)
     assert rc == 0, "oracle allocation failed"
     return ids, scores, probe_out, elig
 

@@ -20,7 +20,9 @@
  *      and one bit operation tests it against the request at serving time --
  *      same page, Bloom index filter paragraph). Only eligible items are
  *      scored: the filter runs inside the chosen clusters and only the items
- *      that pass it are scored.
+ *      that pass it are scored. A query may carry several alternative masks
+ *      (an OR of values, e.g. any of several languages): the item is eligible
+ *      when it passes at least one of them (oracle_search_or).
  *   4. Score = sum_j q[b][j] * x[i][j] in int32 (int8 storage, fused Int8 ANN
  *      paragraph). Order the candidates by score descending, then item id
  *      ascending, and output the first min(k, count); the remaining slots get
@@ -90,11 +92,21 @@ int32_t oracle_probe(const int8_t* q, const int8_t* cent, int32_t nlist, int32_t
     return 0;
 }
 
-/* Steps 3-4 for one query over a given set of lists. Row i is item row_ids[i]
- * (item i when row_ids is NULL). */
+/* 1 when the signature passes at least one of the A masks m[0..A) (W words
+ * each): an OR of alternative masks, each tested as above. */
+static int32_t bloom_pass_any(const uint64_t* sig, const uint64_t* m, int32_t A, int32_t W)
+{
+    for (int32_t a = 0; a < A; ++a)
+        if (oracle_bloom_pass(sig, m + (int64_t)a * W, W)) return 1;
+    return 0;
+}
+
+/* Steps 3-4 for one query over a given set of lists, its A alternative masks
+ * in m[0..A) (A = 1: the plain search). Row i is item row_ids[i] (item i when
+ * row_ids is NULL). */
 static int32_t search_lists(const int8_t* items, const uint64_t* sigs, const int64_t* off,
                             const int64_t* row_ids, int32_t d, int32_t W, const int8_t* q, const uint64_t* m,
-                            const int32_t* lists, int32_t P, int32_t k,
+                            int32_t A, const int32_t* lists, int32_t P, int32_t k,
                             int64_t* out_ids, int32_t* out_scores, int64_t* out_count)
 {
     int64_t cap = 0;
@@ -105,7 +117,7 @@ static int32_t search_lists(const int8_t* items, const uint64_t* sigs, const int
     for (int32_t p = 0; p < P; ++p) {
         int32_t c = lists[p];
         for (int64_t i = off[c]; i < off[c + 1]; ++i) {
-            if (!oracle_bloom_pass(sigs + i * W, m, W)) continue;
+            if (!bloom_pass_any(sigs + i * W, m, A, W)) continue;
             cand[n].score = oracle_dot(q, items + i * d, d);
             cand[n].id = row_ids ? row_ids[i] : i;
             ++n;
@@ -127,19 +139,20 @@ static int32_t search_lists(const int8_t* items, const uint64_t* sigs, const int
 }
 
 /*
- * The whole search for queries [b0, b1). Arrays are row-major:
- * items int8 [n][d], sigs uint64 [n][W], off int64 [nlist+1], row_ids int64
- * [n] or NULL (item id of each row; NULL: the row index), cent int8
- * [nlist][d], queries int8 [B][d], masks uint64 [B][W]; outputs int64/int32
- * [B][k]; out_probe int32 [B][P] and out_eligible int64 [B] may be NULL.
- * nthreads > 1 runs queries in parallel (the result does not depend on it).
- * Returns 0, or -1 when an allocation failed.
+ * The whole search for queries [b0, b1), each with A alternative masks (an
+ * item is eligible when it passes any of them; A = 1 is the plain search).
+ * Arrays are row-major: items int8 [n][d], sigs uint64 [n][W], off int64
+ * [nlist+1], row_ids int64 [n] or NULL (item id of each row; NULL: the row
+ * index), cent int8 [nlist][d], queries int8 [B][d], masks uint64 [B][A][W];
+ * outputs int64/int32 [B][k]; out_probe int32 [B][P] and out_eligible int64
+ * [B] may be NULL. nthreads > 1 runs queries in parallel (the result does not
+ * depend on it). Returns 0, or -1 when an allocation failed.
  */
-int32_t oracle_search_ids(const int8_t* items, const uint64_t* sigs, const int64_t* off,
-                          const int64_t* row_ids, const int8_t* cent, int64_t n, int32_t d, int32_t nlist,
-                          int32_t W, const int8_t* queries, const uint64_t* masks, int32_t b0, int32_t b1,
-                          int32_t P, int32_t k, int64_t* out_ids, int32_t* out_scores,
-                          int32_t* out_probe, int64_t* out_eligible, int32_t nthreads)
+int32_t oracle_search_or(const int8_t* items, const uint64_t* sigs, const int64_t* off,
+                         const int64_t* row_ids, const int8_t* cent, int64_t n, int32_t d, int32_t nlist,
+                         int32_t W, const int8_t* queries, const uint64_t* masks, int32_t A, int32_t b0,
+                         int32_t b1, int32_t P, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                         int32_t* out_probe, int64_t* out_eligible, int32_t nthreads)
 {
     (void)n;
     int32_t err = 0;
@@ -149,11 +162,11 @@ int32_t oracle_search_ids(const int8_t* items, const uint64_t* sigs, const int64
         int32_t* lists = (int32_t*)malloc(sizeof(int32_t) * (size_t)P);
         if (!lists) { err |= 1; continue; }
         const int8_t* q = queries + (int64_t)b * d;
-        const uint64_t* m = masks + (int64_t)b * W;
+        const uint64_t* m = masks + (int64_t)b * A * W;
         if (oracle_probe(q, cent, nlist, d, P, lists) != 0) { err |= 1; free(lists); continue; }
         if (out_probe) memcpy(out_probe + (int64_t)(b - b0) * P, lists, sizeof(int32_t) * (size_t)P);
         int64_t cnt = 0;
-        if (search_lists(items, sigs, off, row_ids, d, W, q, m, lists, P, k,
+        if (search_lists(items, sigs, off, row_ids, d, W, q, m, A, lists, P, k,
                          out_ids + (int64_t)(b - b0) * k, out_scores + (int64_t)(b - b0) * k,
                          &cnt) != 0)
             err |= 1;
@@ -161,6 +174,17 @@ int32_t oracle_search_ids(const int8_t* items, const uint64_t* sigs, const int64
         free(lists);
     }
     return err ? -1 : 0;
+}
+
+/* oracle_search_or with one mask per query (the plain search) */
+int32_t oracle_search_ids(const int8_t* items, const uint64_t* sigs, const int64_t* off,
+                          const int64_t* row_ids, const int8_t* cent, int64_t n, int32_t d, int32_t nlist,
+                          int32_t W, const int8_t* queries, const uint64_t* masks, int32_t b0, int32_t b1,
+                          int32_t P, int32_t k, int64_t* out_ids, int32_t* out_scores,
+                          int32_t* out_probe, int64_t* out_eligible, int32_t nthreads)
+{
+    return oracle_search_or(items, sigs, off, row_ids, cent, n, d, nlist, W, queries, masks, 1, b0, b1, P, k,
+                            out_ids, out_scores, out_probe, out_eligible, nthreads);
 }
 
 /* oracle_search_ids with every item id equal to its row index */

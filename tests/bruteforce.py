@@ -57,3 +57,31 @@ def search(items, sigs, offsets, centroids, queries, masks, nprobe, k, row_ids=N
         ids[b, :o.size] = item[o]
         out[b, :o.size] = s[o]
     return ids, out, probes, elig
+
+
+def search_or(items, sigs, offsets, centroids, queries, mask_sets, nprobe, k, row_ids=None):
+    """search() with mask_sets [B, A, W]: an item is eligible when it passes any
+    of its query's A masks."""
+    B = queries.shape[0]
+    ids = np.full((B, k), -1, dtype=np.int64)
+    out = np.full((B, k), INT32_MIN, dtype=np.int32)
+    probes = np.zeros((B, nprobe), dtype=np.int32)
+    elig = np.zeros(B, dtype=np.int64)
+    for b in range(B):
+        lists = probe(queries[b], centroids, nprobe)
+        probes[b] = lists
+        rows = np.concatenate([np.arange(offsets[c], offsets[c + 1]) for c in lists]) \
+            if len(lists) else np.zeros(0, np.int64)
+        ok = np.zeros(rows.size, dtype=bool)
+        for m in mask_sets[b]:
+            ok |= bloom_pass(sigs[rows], m)
+        rows = rows[ok]
+        elig[b] = rows.size
+        if rows.size == 0:
+            continue
+        s = scores(queries[b][None, :], items[rows])[0]
+        item = rows if row_ids is None else np.asarray(row_ids, dtype=np.int64)[rows]
+        o = order_desc(s, item)[:k]
+        ids[b, :o.size] = item[o]
+        out[b, :o.size] = s[o]
+    return ids, out, probes, elig

@@ -267,4 +267,72 @@ def pin_row_ids_bruteforce(lib):
             assert np.array_equal(g, e), (c, what)
 
 
+# --- step 3 with alternative masks (an OR of values) ---------------------------------
+def pin_or_golden(lib):
+    g = golden("or_masks.json")
+    x, q = _axis_items(g["scores"])
+    n = len(g["scores"])
+    off, cen = _one_list(n, x.shape[1])
+    sigs = np.array(g["sigs"], np.uint64).reshape(n, 1)
+    for order in (1, -1):  # the result does not depend on the order of the alternatives
+        ms = np.array(g["masks"][::order], np.uint64).reshape(1, -1, 1)
+        ids, sc, _, el = oracle.search_or(x, sigs, off, cen, q, ms, 1, g["k"], lib=lib)
+        assert list(ids[0]) == g["expect_ids"] and list(sc[0]) == g["expect_scores"], (ids, sc)
+        assert int(el[0]) == g["expect_eligible"], el
+
+
+def _or_cases():
+    rng = np.random.default_rng(71)
+    out = []
+    for c in (dict(n=1500, d=32, nlist=8, sig_bits=64, hash_bits=2, B=6, nprobe=3, k=60, seed=72, mask_flags=2),
+              dict(n=2000, d=16, nlist=12, sig_bits=128, hash_bits=3, B=5, nprobe=4, k=300, seed=73,
+                   mask_country=True, mask_flags=1),
+              dict(n=800, d=48, nlist=1, sig_bits=128, B=4, nprobe=1, k=900, seed=74, mask_mode="item")):
+        a = _arrays(small(**c))
+        B, W = a["masks"].shape
+        n = a["sigs"].shape[0]
+        # alternatives: the query's own mask, another query's, and the bits of
+        # a random item's signature under a random sub-mask
+        alt = [a["masks"], np.roll(a["masks"], 1, axis=0),
+               a["sigs"][rng.integers(0, n, B)] & rng.integers(0, 2**63, (B, W), dtype=np.uint64)]
+        out.append((c, a, np.ascontiguousarray(np.stack(alt, axis=1))))
+    return out
+
+
+def pin_or_bruteforce(lib):
+    for c, a, ms in _or_cases():
+        P, k = c["nprobe"], c["k"]
+        for A in (1, 2, 3):
+            got = oracle.search_or(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"],
+                                   np.ascontiguousarray(ms[:, :A]), P, k, lib=lib)
+            exp = bruteforce.search_or(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"],
+                                       ms[:, :A], P, k)
+            for g_, e, what in zip(got, exp, ("ids", "scores", "probe", "eligible")):
+                assert np.array_equal(g_, e), (c, A, what)
+
+
+def pin_or_union_of_single_masks(lib):
+    # every item of the union's top-k is in the top-k of each alternative it
+    # passes, so merging the single-mask results (distinct ids, score
+    # descending, id ascending) gives the OR search's ids and scores
+    for c, a, ms in _or_cases():
+        P, k = c["nprobe"], c["k"]
+        A = ms.shape[1]
+        got = oracle.search_or(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"], ms, P, k,
+                               lib=lib)
+        singles = [oracle.search(a["items"], a["sigs"], a["offsets"], a["centroids"], a["queries"],
+                                 np.ascontiguousarray(ms[:, j]), P, k, lib=lib) for j in range(A)]
+        for b in range(a["queries"].shape[0]):
+            pairs = {}
+            for r in singles:
+                for i, s_ in zip(r[0][b], r[1][b]):
+                    if i >= 0:
+                        pairs[int(i)] = int(s_)
+            best = sorted(pairs.items(), key=lambda t: (-t[1], t[0]))[:k]
+            exp_i = [t[0] for t in best] + [-1] * (k - len(best))
+            exp_s = [t[1] for t in best] + [INT32_MIN] * (k - len(best))
+            assert list(got[0][b]) == exp_i and list(got[1][b]) == exp_s, (c, b)
+            assert int(got[3][b]) >= max(int(r[3][b]) for r in singles), (c, b)
+
+
 PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

@@ -1,7 +1,7 @@
 """Plant one plausible mistake at a time in a copy of the oracle and check that
 at least one pin fails for each. This shows the pins constrain every step of
-the oracle: probe order, Bloom test, inner product, list range, top-k order and
-padding. The mutants are built from the oracle source into a temporary folder;
+the oracle: probe order, Bloom test (and its OR over alternative masks), inner
+product, list range, top-k order and padding. The mutants are built from the oracle source into a temporary folder;
 the real oracle is never modified."""
 import os
 import subprocess
@@ -32,7 +32,13 @@ MUTANTS = {
     "item_row_stride": ("oracle_dot(q, items + i * d, d)", "oracle_dot(q, items + i, d)"),
     "pad_id_zero": ("out_ids[r] = -1;", "out_ids[r] = 0;"),
     "pad_score_zero": ("out_scores[r] = INT32_MIN;", "out_scores[r] = 0;"),
-    "filter_after_topk": ("if (!oracle_bloom_pass(sigs + i * W, m, W)) continue;", ""),
+    "filter_after_topk": ("if (!bloom_pass_any(sigs + i * W, m, A, W)) continue;", ""),
+    "or_needs_every_mask": ("if (oracle_bloom_pass(sig, m + (int64_t)a * W, W)) return 1;\n    return 0;",
+                            "if (!oracle_bloom_pass(sig, m + (int64_t)a * W, W)) return 0;\n    return 1;"),
+    "or_first_mask_only": ("for (int32_t a = 0; a < A; ++a)\n        if (oracle_bloom_pass",
+                           "for (int32_t a = 0; a < 1; ++a)\n        if (oracle_bloom_pass"),
+    "or_mask_stride": ("m + (int64_t)a * W, W)", "m + (int64_t)a, W)"),
+    "or_query_stride": ("masks + (int64_t)b * A * W;", "masks + (int64_t)b * W;"),
     "row_ids_ignored": ("cand[n].id = row_ids ? row_ids[i] : i;", "cand[n].id = i;"),
 }
 
