@@ -284,7 +284,7 @@ struct ScratchLayout {
     size_t off_list_cnt, off_cand_cnt, off_elig, off_rng, off_sel_hist, off_sel_cursor, off_ctl, off_tc_hist, zero_bytes;
     size_t off_units_tc, off_qscale;
     size_t off_sel_out, off_sel_tie;
-    size_t off_probe, off_probe_keys, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_units, off_cand;
+    size_t off_probe, off_probe_keys, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_slot_bits, off_units, off_cand;
     size_t add(size_t bytes)
     {
         const size_t o = total;
@@ -352,6 +352,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_qnbits = L.add(size_t(B) * 4);
     L.off_qlist = L.add(slots * 4);
     L.off_qmask = L.add(slots * 16);
+    L.off_slot_bits = L.add(slots * st::kSlotBits);
     L.off_units = L.add(size_t(max_units) * 16);
     L.off_units_tc = L.add(tc_min_q ? size_t(max_units) * 16 : 0);
     L.off_qscale = L.add(size_t(B) * 8);
@@ -403,6 +404,7 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.qnbits = reinterpret_cast<int32_t*>(base + L.off_qnbits);
     a.qlist = reinterpret_cast<int32_t*>(base + L.off_qlist);
     a.qmask_slot = reinterpret_cast<uint64_t*>(base + L.off_qmask);
+    a.slot_bits = reinterpret_cast<uint8_t*>(base + L.off_slot_bits);
     a.units = reinterpret_cast<int4*>(base + L.off_units);
     a.max_units = int32_t(max_units);
     a.tc_min_q = tc_min_q;

@@ -35,8 +35,8 @@ namespace st {
 // Write the probe result of query b from its P best keys, sorted (sorted[p],
 // p < P). kFile: also file the query into its lists (the search): the query's
 // mask bits in increasing order, then for each chosen list the next rank of
-// the list's query counter and the query's id and mask in that slot of the
-// list's slot row. The allocation-free probe-only call writes the result alone.
+// the list's query counter and the query's id, mask and first kSlotBits mask
+// bits in that slot of the list's slot row. The allocation-free probe-only call writes the result alone.
 template <int BLOCK, bool kFile>
 __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
 {
@@ -46,6 +46,7 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
         return;
     }
     const int W = a.W;
+    __shared__ __align__(16) uint8_t s_bits[kSlotBits];
     if (threadIdx.x < 32) {
         const uint64_t m0 = a.qmasks[int64_t(b) * W];
         const uint64_t m1 = W > 1 ? a.qmasks[int64_t(b) * W + 1] : 0ull;
@@ -56,10 +57,15 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
             const uint64_t word = bit < 64 ? m0 : m1;
             const bool on = (word >> (bit & 63)) & 1ull;
             const unsigned bal = __ballot_sync(0xffffffffu, on);
-            if (on) a.qbits[int64_t(b) * kMaskBitsMax + n_before + __popc(bal & lanemask_lt())] = uint8_t(bit);
+            const int j = n_before + __popc(bal & lanemask_lt());
+            if (on) {
+                a.qbits[int64_t(b) * kMaskBitsMax + j] = uint8_t(bit);
+                if (j < kSlotBits) s_bits[j] = uint8_t(bit);
+            }
             n_before += __popc(bal);
         }
         if (lane == 0) a.qnbits[b] = n_before;
+        for (int j = n_before + lane; j < kSlotBits; j += 32) s_bits[j] = 0;
     }
     if (a.qscale != nullptr && threadIdx.x >= 32 && threadIdx.x < 64) {
         // bound of the query's scores, for the score bins of the scans and
@@ -76,6 +82,8 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
             a.qscale[b] = make_int2(-S, sh);
         }
     }
+    __syncthreads();  // s_bits holds the query's first mask bits
+    const uint4 sb0 = reinterpret_cast<const uint4*>(s_bits)[0], sb1 = reinterpret_cast<const uint4*>(s_bits)[1];
     for (int p = threadIdx.x; p < P; p += BLOCK) {
         const int L = int(key_id(sorted[p]));
         a.probe[int64_t(b) * P + p] = L;
@@ -86,6 +94,9 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
             const uint64_t m0 = a.qmasks[int64_t(b) * W];
             const uint64_t m1 = W > 1 ? a.qmasks[int64_t(b) * W + 1] : 0ull;
             reinterpret_cast<ulonglong2*>(a.qmask_slot)[slot] = make_ulonglong2(m0, m1);
+            uint4* sbits = reinterpret_cast<uint4*>(a.slot_bits + slot * kSlotBits);
+            sbits[0] = sb0;
+            sbits[1] = sb1;
         }
     }
 }

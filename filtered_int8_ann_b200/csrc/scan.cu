@@ -45,6 +45,7 @@
 namespace st {
 
 constexpr int kPlaneSlots = 32;                         // planes one buffer holds
+static_assert(kPlaneSlots <= kSlotBits, "a slot carries every bit of a mask whose planes fit the buffer");
 constexpr int kPlaneBytes = kWarpItems / 8;             // 64 bytes per plane
 constexpr int kPlaneBufBytes = kPlaneSlots * kPlaneBytes;
 
@@ -149,32 +150,40 @@ scan_kernel(SearchArgs a)
     if (u >= n_units) return;
 
     // unit entry: {first row, chunk, first query slot, rows << 16 | queries};
-    // lane s < queries holds query s's id and mask
-    auto load_slots = [&](const int4& e, int& qid, uint64_t& m0, uint64_t& m1) {
+    // lane s < queries holds query s's id and mask; for a single-query unit,
+    // lane j also holds the query's j-th mask bit (from its slot, so that no
+    // load waits for the query id)
+    auto load_slots = [&](const int4& e, int& qid, uint64_t& m0, uint64_t& m1, uint32_t& sb) {
         qid = 0;
         m0 = 0;
         m1 = 0;
-        if (lane < (e.w & 0xFFFF)) {
+        sb = 0;
+        const int qn = e.w & 0xFFFF;
+        if (lane < qn) {
             qid = a.qlist[e.z + lane];
             const ulonglong2 m = reinterpret_cast<const ulonglong2*>(a.qmask_slot)[e.z + lane];
             m0 = m.x;
             m1 = m.y;
         }
+        if (qn == 1) sb = a.slot_bits[int64_t(e.z) * kSlotBits + lane];
     };
 
     // Request a unit's planes into the buffer; returns the number of planes it
     // then holds, or -1 when the test must read global planes. A single-query
     // unit needs no union: its planes are the query's mask bits in increasing
-    // order, listed by the probe.
-    auto request_planes = [&](const int4& e, int qid, uint64_t m0, uint64_t m1) -> int {
+    // order, which its slot carries (lane j holds bit j in sb).
+    auto request_planes = [&](const int4& e, uint64_t m0, uint64_t m1, uint32_t sb) -> int {
         if ((e.w & 0xFFFF) == 1) {
-            const int q = __shfl_sync(0xffffffffu, qid, 0);
-            const int nb = __ldg(a.qnbits + q);
+            const uint64_t x = __shfl_sync(0xffffffffu, m0, 0), y = __shfl_sync(0xffffffffu, m1, 0);
+            const int nb = __popcll(x) + (W > 1 ? __popcll(y) : 0);
             if (nb > kPlaneSlots) return -1;
-            const uint8_t* bits = a.qbits + int64_t(q) * kMaskBitsMax;
             const uint32_t* src = a.planes + int64_t(e.y) * NPL * 16 + (lane & 3) * 4;
-            for (int j = lane >> 2; j < nb; j += 8)
-                cp_async16_cg(pbuf + j * 16 + (lane & 3) * 4, src + __ldg(bits + j) * 16);
+#pragma unroll
+            for (int t = 0; t < kPlaneSlots / 8; ++t) {
+                const int j = (lane >> 2) + 8 * t;
+                const int bit = int(__shfl_sync(0xffffffffu, sb, j));
+                if (j < nb) cp_async16_cg(pbuf + j * 16 + (lane & 3) * 4, src + bit * 16);
+            }
             return nb;
         }
         uint64_t x = m0, y = m1;
@@ -196,7 +205,8 @@ scan_kernel(SearchArgs a)
     // Test a unit whose planes are in the buffer (held >= 0) or in global
     // memory: pass words -> pass[s][blk]; returns the OR over queries in `any`
     // and, in lane s, query s's survivor count (general path only).
-    auto test_unit = [&](const int4& e, int qid, int held, uint32_t* pass, uint32_t& any, uint32_t& mycnt) {
+    auto test_unit = [&](const int4& e, int qid, uint64_t m0, uint64_t m1, int held, uint32_t* pass, uint32_t& any,
+                         uint32_t& mycnt) {
         const int len = e.w >> 16;
         const int qn = e.w & 0xFFFF;
         const uint32_t valid = len >= 32 * (blk + 1) ? 0xFFFFFFFFu
@@ -219,10 +229,15 @@ scan_kernel(SearchArgs a)
         }
         const uint32_t* gpl = a.planes + int64_t(e.y) * NPL * 16 + blk;
         for (int s = 0; s < qn; ++s) {
+            // query s's mask bits: from its slot when the buffer holds the
+            // planes (then it has at most kPlaneSlots <= kSlotBits of them),
+            // else from the query's own list
             const int qg = __shfl_sync(0xffffffffu, qid, s);
-            const int nb = __ldg(a.qnbits + qg);
+            const uint64_t x = __shfl_sync(0xffffffffu, m0, s), y = __shfl_sync(0xffffffffu, m1, s);
+            const int nb = __popcll(x) + (W > 1 ? __popcll(y) : 0);
             const int h0 = (nb + 1) >> 1;
-            const uint8_t* bits = a.qbits + int64_t(qg) * kMaskBitsMax;
+            const uint8_t* bits = held >= 0 ? a.slot_bits + int64_t(e.z + s) * kSlotBits
+                                            : a.qbits + int64_t(qg) * kMaskBitsMax;
             const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
             // four independent bit -> slot -> plane chains per step
             uint32_t acc = 0xFFFFFFFFu;
@@ -296,23 +311,25 @@ scan_kernel(SearchArgs a)
     if (u_n2 < n_units) e_n2 = a.units[u_n2];
     int qid_c, qid_n = 0;
     uint64_t m0_n = 0, m1_n = 0;
+    uint32_t sb_n = 0;
     int held;          // planes the buffer holds for the next unit to test (-1: global)
     uint32_t base_c;   // lane s: reservation of query s of the unit being scored
     int nsurv_c;       // survivors of the unit being scored
     bool single_c;     // it took the single-query path
     {
         uint64_t m0_c, m1_c;
-        load_slots(e_cur, qid_c, m0_c, m1_c);
-        if (u_n1 < n_units) load_slots(e_nxt, qid_n, m0_n, m1_n);
-        const int held0 = request_planes(e_cur, qid_c, m0_c, m1_c);
+        uint32_t sb_c;
+        load_slots(e_cur, qid_c, m0_c, m1_c, sb_c);
+        if (u_n1 < n_units) load_slots(e_nxt, qid_n, m0_n, m1_n, sb_n);
+        const int held0 = request_planes(e_cur, m0_c, m1_c, sb_c);
         cp_async_commit();
         cp_async_wait_group<0>();
         __syncwarp();
         uint32_t any, mycnt;
-        test_unit(e_cur, qid_c, held0, pass2, any, mycnt);
+        test_unit(e_cur, qid_c, m0_c, m1_c, held0, pass2, any, mycnt);
         single_c = (e_cur.w & 0xFFFF) == 1 && held0 >= 0;
         __syncwarp();
-        held = u_n1 < n_units ? request_planes(e_nxt, qid_n, m0_n, m1_n) : -1;
+        held = u_n1 < n_units ? request_planes(e_nxt, m0_n, m1_n, sb_n) : -1;
         cp_async_commit();
         nsurv_c = settle_unit(e_cur, qid_c, single_c, any, mycnt, surv2, base_c);
     }
@@ -332,7 +349,8 @@ scan_kernel(SearchArgs a)
         if (has_n3) e_n3 = a.units[u_n3];
         int qid_2 = 0;
         uint64_t m0_2 = 0, m1_2 = 0;
-        if (has_n2) load_slots(e_n2, qid_2, m0_2, m1_2);
+        uint32_t sb_2 = 0;
+        if (has_n2) load_slots(e_n2, qid_2, m0_2, m1_2, sb_2);
 
         // test the next unit: its planes are the older of the (at most two)
         // pending groups [planes(u+1), queries(u)]
@@ -343,10 +361,10 @@ scan_kernel(SearchArgs a)
             cp_async_wait_group<1>();
             __syncwarp();
             uint32_t any, mycnt;
-            test_unit(e_nxt, qid_n, held, pass2 + (cb ^ 1) * kQMax * 16, any, mycnt);
+            test_unit(e_nxt, qid_n, m0_n, m1_n, held, pass2 + (cb ^ 1) * kQMax * 16, any, mycnt);
             single_n = (e_nxt.w & 0xFFFF) == 1 && held >= 0;
             __syncwarp();
-            held = has_n2 ? request_planes(e_n2, qid_2, m0_2, m1_2) : -1;
+            held = has_n2 ? request_planes(e_n2, m0_2, m1_2, sb_2) : -1;
             cp_async_commit();
             nsurv_n = settle_unit(e_nxt, qid_n, single_n, any, mycnt, surv2 + (cb ^ 1) * kWarpItems, base_n);
         } else {

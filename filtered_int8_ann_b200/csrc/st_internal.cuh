@@ -33,6 +33,7 @@ constexpr int kCntStride = 32;             // uint32 words (16 uint64) per query
 // every row starts on a 16-byte boundary for vector copies.
 __host__ __device__ __forceinline__ int64_t probe_keys_ld(int nlist) { return (int64_t(nlist) + 1) & ~int64_t(1); }
 constexpr int kMaskBitsMax = 128;          // signature bits
+constexpr int kSlotBits = 32;              // mask bits a slot carries (the rest: the query's own list)
 constexpr int kSelBits = 11;               // radix digit of the selections
 constexpr int kSelBins = 1 << kSelBits;
 constexpr int kSelTieCap = 4096;           // cut-bin keys the final top-k keeps per query
@@ -119,6 +120,7 @@ struct SearchArgs {
     int32_t* list_ustart;    // [nlist] first unit of each probed list
     int32_t* qlist;          // [nlist][B] slot row of each list: ids of the queries probing it
     uint64_t* qmask_slot;    // [nlist][B][2] that query's mask words (word 1 = 0 when W = 1)
+    uint8_t* slot_bits;      // [nlist][B][kSlotBits] that query's first kSlotBits mask bits, increasing
     uint8_t* qbits;          // [B][kMaskBitsMax] each query's mask bits, in increasing order
     int32_t* qnbits;         // [B] number of mask bits of each query
     int4* units;             // [max_units] {first row, chunk, first slot, rows << 16 | queries}
