@@ -10,15 +10,18 @@
 // (kTcBins bins over its possible range [-S, S]), so the bin holding the k-th
 // best score -- the cut -- is known before any key is read, and so is the
 // number of keys at or above it (k plus at most the cut bin's keys):
-//   1. every CTA reads the bins and finds the cut (no communication);
+//   1. every CTA reads the bins and finds the cut (no communication): a
+//      suffix scan over the lanes' bin sums finds the lane holding it, a
+//      second one over that lane's bins the bin itself;
 //   2. each CTA reads its share of the keys once and sends the keys at or
 //      above the cut straight into the leader's shared memory (distributed
 //      shared memory; one atomic per warp for their positions);
-//   3. the leader selects and orders the k best of those few keys in its own
-//      shared memory and writes the ids and scores.
+//   3. the leader sorts those few keys in its own shared memory (a counting
+//      sort over their own score range) and writes the k best.
 // Two cluster barriers in all. When the keys above the cut would not fit the
 // leader's buffer (many equal or close scores), the general cluster selection
-// (cluster_topk.cuh) runs over the query's keys at or above the cut instead. With deletions or exclude masks the
+// (cluster_topk.cuh) runs over the query's keys at or above the cut instead.
+// With deletions or exclude masks the
 // scans' counts include keys the post-filter drops, so those searches take
 // the general cluster selection (cluster_topk.cuh) with the post-filter
 // applied to every key; a query whose candidates overflowed the scan's buffer
@@ -33,7 +36,6 @@ namespace st {
 
 constexpr int kCBlock = 512;
 constexpr int kCTieCap = 4096;   // cut-bin keys of the general (post-filter) path
-constexpr int kCTieSmall = 1024; // cut-bin keys of the leader's final selection
 
 // Keys at or above the cut the leader can hold.
 __host__ __device__ __forceinline__ int cl_buf_cap(int k)
@@ -45,7 +47,7 @@ __host__ __device__ __forceinline__ int cl_buf_cap(int k)
 __host__ __device__ __forceinline__ size_t select_cluster_smem(int k)
 {
     const size_t ke = size_t((k + 1) & ~1), pw = size_t(next_pow2(k));
-    const size_t fast = size_t(cl_buf_cap(k)) + pw + ke + kCTieSmall;
+    const size_t fast = 2 * size_t(cl_buf_cap(k));  // gathered keys, then the sort's scratch
     const size_t general = ke + kCTieCap + pw;
     return (fast > general ? fast : general) * 8;
 }
@@ -94,7 +96,6 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
     __shared__ int s_cut;
     __shared__ uint32_t s_m, s_cnt;
     const int k = a.k;
-    const int pwk = next_pow2(k);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     const uint32_t cnt = a.cand_cnt[int64_t(q) * kCntStride];
@@ -119,9 +120,7 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
     } else {
         const int cap = cl_buf_cap(k);
         uint64_t* buf = reinterpret_cast<uint64_t*>(smem_raw);   // [cap] keys at or above the cut (leader)
-        out = buf + cap;                                         // [next_pow2(k)]
-        uint64_t* tmp = out + pwk;                               // [k, rounded up to even]
-        uint64_t* tie = tmp + ((k + 1) & ~1);                    // [kCTieSmall]
+        out = buf + cap;                                         // [cap] the leader's sort scratch
         // the leader's counter starts at zero; the cluster barrier that makes
         // it (and every CTA's start) visible is awaited only before the
         // first remote access
@@ -144,32 +143,34 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
                 if (lane + off < 32) incl += o;
             }
             const uint32_t want = n < k ? uint32_t(n) : uint32_t(k);
-            uint32_t run = incl - tot;  // keys in the bins above this lane's
-            int best = -1;
-            uint32_t at = 0;
-            if (run < want && incl >= want) {  // the cut is in this lane's bins: walk them down
-#pragma unroll 1
-                for (int i = kPer / 4 - 1; i >= 0 && best < 0; --i) {
-                    const uint4 x = __ldcg(h + i);
-                    const uint32_t c4[4] = {x.x, x.y, x.z, x.w};
-                    for (int j = 3; j >= 0; --j) {
-                        run += c4[j];
-                        if (run >= want) {
-                            best = kPer * lane + 4 * i + j;
-                            at = run;
-                            break;
-                        }
-                    }
+            const uint32_t above = incl - tot;  // keys in the bins above this lane's
+            const unsigned found = __ballot_sync(0xffffffffu, above < want && incl >= want);
+            if (found == 0u) {  // cannot happen: the bins hold all n keys
+                if (lane == 0) {
+                    s_cut = 0;
+                    s_m = 0xFFFFFFFFu;
                 }
-            }
-            if (best >= 0) {  // the lane holding the cut
-                s_cut = best;
-                s_m = at;
-            }
-            const unsigned found = __ballot_sync(0xffffffffu, best >= 0);
-            if (lane == 0 && found == 0u) {  // cannot happen: the bins hold all n keys
-                s_cut = 0;
-                s_m = 0xFFFFFFFFu;
+            } else {
+                // the lane L holding the cut: the whole warp reads its kPer bins
+                // (one per lane) and finds the highest bin with at least `want`
+                // keys at or above it by a suffix scan
+                static_assert(kPer == 32, "one bin per lane");
+                const int L = __ffs(found) - 1;
+                const uint32_t runL = __shfl_sync(0xffffffffu, above, L);
+                const uint32_t v = __ldcg(a.qhist + int64_t(q) * kTcBins + kPer * L + lane);
+                uint32_t suf = v;  // keys in bins lane .. kPer - 1 of lane L's
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t o = __shfl_down_sync(0xffffffffu, suf, off);
+                    if (lane + off < 32) suf += o;
+                }
+                const unsigned ok = __ballot_sync(0xffffffffu, runL + suf >= want);
+                const int j = 31 - __clz(ok);  // ok != 0: lane 0 sees every key of lane L's bins
+                const uint32_t at = __shfl_sync(0xffffffffu, runL + suf, j);
+                if (lane == 0) {
+                    s_cut = kPer * L + j;
+                    s_m = at;
+                }
             }
         }
         __syncthreads();
@@ -213,8 +214,13 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
             // 3. the leader: the k best of them, sorted
             const uint32_t got = s_cnt;
             if (tid == 0 && got != mt) set_error(a.err, kErrSelectCount);
-            const int64_t nb = got < uint32_t(cap) ? int64_t(got) : int64_t(cap);
-            m = block_topk_sorted<kCBlock>(buf, nb, k, out, tmp, tie, kCTieSmall, true, T, -sc.x, ss, a.err);
+            const int nb = int(got < uint32_t(cap) ? got : uint32_t(cap));
+            // every gathered key is at or above the cut, and there are few of
+            // them: sort them all (counting sort over their own score range;
+            // out[] and what follows it serve as its scratch) and keep the k best
+            block_sort_desc_counting<kCBlock>(buf, nb, out, ss);
+            m = nb < k ? nb : k;
+            out = buf;
         }
     }
     for (int r = tid; r < k; r += kCBlock) {
