@@ -26,6 +26,7 @@ ST_PROBE_NOALLOC_SCRATCH_BYTES = 16 << 20
 ST_INSERT_CHUNK = 512
 ST_MERGE_MAX_KEYS = 16384
 ST_MAX_D, ST_MAX_K, ST_MAX_NPROBE, ST_SMALL_K, ST_MAX_B = 512, 262144, 4096, 4096, 32768
+ST_MAX_OR = 7
 
 # Every symbol include/st.h declares.
 EXPORTS = ("st_index_create", "st_search", "st_search_ex", "st_search_host", "st_search_host_async",
@@ -43,7 +44,7 @@ class StError(RuntimeError):
 class _Extras(ctypes.Structure):
     _fields_ = [("eligible", ctypes.c_void_p), ("probe", ctypes.c_void_p),
                 ("stage_events", ctypes.c_void_p * 5), ("exclude_masks", ctypes.c_void_p),
-                ("candidates", ctypes.c_void_p)]
+                ("candidates", ctypes.c_void_p), ("or_masks", ctypes.c_void_p), ("n_or", ctypes.c_int32)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -136,13 +137,15 @@ def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: i
               out_ids: Optional[torch.Tensor] = None, out_scores: Optional[torch.Tensor] = None,
               stream=None, eligible: Optional[torch.Tensor] = None,
               probe: Optional[torch.Tensor] = None, stage_events=None,
-              exclude: Optional[torch.Tensor] = None, candidates: Optional[torch.Tensor] = None):
+              exclude: Optional[torch.Tensor] = None, candidates: Optional[torch.Tensor] = None,
+              or_masks: Optional[torch.Tensor] = None):
     """Asynchronous search of device-resident queries; returns (ids int64 [B,k],
     scores int32 [B,k]). `eligible` [B] int64 and `probe` [B,nprobe] int32 are
     optional extra outputs, as is `candidates` [B] int64 (keys the scan wrote
     for each query's final top-k); `stage_events` is a list of up to five recorded
     torch.cuda.Event objects marking the stage boundaries; `exclude` [B,W]
-    holds per-query exclude masks (st_search_ex)."""
+    holds per-query exclude masks; `or_masks` [B,A,W] alternative masks (an
+    item passing qmasks[b] or any of or_masks[b] is eligible) (st_search_ex)."""
     qmasks = _as_words(qmasks)
     B = queries.shape[0]
     dev = queries.device
@@ -152,7 +155,20 @@ def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: i
         out_scores = torch.empty((B, k), dtype=torch.int32, device=dev)
     if exclude is not None:
         exclude = _as_words(exclude)
-    if eligible is None and probe is None and not stage_events and exclude is None and candidates is None:
+    n_or = 0
+    if or_masks is not None:
+        if or_masks.dtype == torch.uint64:
+            or_masks = or_masks.view(torch.int64)
+        if or_masks.dtype != torch.int64:
+            raise ValueError("or_masks are 64-bit words")
+        if or_masks.dim() == 2:  # [B, A] of one-word masks
+            or_masks = or_masks.unsqueeze(-1)
+        or_masks = or_masks.contiguous()
+        if or_masks.dim() != 3 or or_masks.shape[0] != B or or_masks.shape[2] != qmasks.shape[-1]:
+            raise ValueError("or_masks must be [B, A, W] with the masks' W")
+        n_or = int(or_masks.shape[1])
+    if eligible is None and probe is None and not stage_events and exclude is None and candidates is None \
+            and n_or == 0:
         st = lib().st_search(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
                              _ptr(out_scores), _stream(stream))
         _check(st, "st_search")
@@ -160,6 +176,8 @@ def st_search(index: int, queries: torch.Tensor, qmasks: torch.Tensor, nprobe: i
         ex = _Extras(_ptr(eligible), _ptr(probe))
         ex.exclude_masks = _ptr(exclude)
         ex.candidates = _ptr(candidates)
+        ex.or_masks = _ptr(or_masks) if n_or else None
+        ex.n_or = n_or
         for i, ev in enumerate(stage_events or ()):
             ex.stage_events[i] = ev.cuda_event if ev is not None else None
         st = lib().st_search_ex(index, _ptr(queries), _ptr(qmasks), B, nprobe, k, _ptr(out_ids),
@@ -279,8 +297,16 @@ class Index:
 
     def search_any(self, queries, mask_sets, nprobe, k, stream=None, **kw):
         """OR of several masks per query: an item is eligible if any of the masks
-        passes. mask_sets [M, B, W] (M alternatives); one search per alternative,
-        then the exact union merge (k <= 4096, M * k <= ST_MERGE_MAX_KEYS)."""
+        passes. mask_sets [M, B, W] (M alternatives, M <= ST_MAX_OR + 1): one
+        search whose scan tests every alternative (st_search_extras.or_masks)."""
+        M = mask_sets.shape[0]
+        alt = mask_sets[1:].permute(1, 0, 2).contiguous() if M > 1 else None
+        return self.search(queries, mask_sets[0].contiguous(), nprobe, k, stream=stream, or_masks=alt, **kw)
+
+    def search_any_merged(self, queries, mask_sets, nprobe, k, stream=None, **kw):
+        """search_any as one search per alternative followed by the exact union
+        merge of their results (st_merge_topk_union; k <= 4096, M * k <=
+        ST_MERGE_MAX_KEYS): the same result, for checking the fused scan."""
         M, B = mask_sets.shape[0], queries.shape[0]
         ids = torch.empty((M, B, k), dtype=torch.int64, device=queries.device)
         sc = torch.empty((M, B, k), dtype=torch.int32, device=queries.device)

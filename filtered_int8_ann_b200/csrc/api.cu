@@ -348,8 +348,9 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_probe = L.add(size_t(B) * nprobe * 4);
     L.off_probe_keys = L.add(size_t(B) * size_t(st::probe_keys_ld(idx->nlist)) * 8);
     L.off_list_ustart = L.add(nl4 * 4);
-    L.off_qbits = L.add(size_t(B) * st::kMaskBitsMax);
-    L.off_qnbits = L.add(size_t(B) * 4);
+    const int n_alt = 1 + (extras ? extras->n_or : 0);  // masks per query
+    L.off_qbits = L.add(size_t(B) * n_alt * st::kMaskBitsMax);
+    L.off_qnbits = L.add(size_t(B) * n_alt * 4);
     L.off_qlist = L.add(slots * 4);
     L.off_qmask = L.add(slots * 16);
     L.off_slot_bits = L.add(slots * st::kSlotBits);
@@ -417,6 +418,8 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.id_offset = idx->id_offset;
     a.dead = idx->dead;
     a.qexclude = extras ? extras->exclude_masks : nullptr;
+    a.n_or = extras ? extras->n_or : 0;
+    a.or_masks = a.n_or > 0 ? extras->or_masks : nullptr;
     a.sel_out = reinterpret_cast<uint64_t*>(base + L.off_sel_out);
     a.sel_tie = reinterpret_cast<uint64_t*>(base + L.off_sel_tie);
     a.err = idx->err;
@@ -595,6 +598,9 @@ st_status st_search_ex(const st_index* idx, const int8_t* queries, const uint64_
             return ST_ERR_INVALID_ARG;
         if (extras->exclude_masks &&
             (!is_device_ptr(extras->exclude_masks, idx->device) || !aligned(extras->exclude_masks, 8)))
+            return ST_ERR_INVALID_ARG;
+        if (extras->n_or < 0 || extras->n_or > ST_MAX_OR ||
+            (extras->n_or > 0 && (!is_device_ptr(extras->or_masks, idx->device) || !aligned(extras->or_masks, 8))))
             return ST_ERR_INVALID_ARG;
     }
     return search_impl(idx, queries, qmasks, B, nprobe, k, out_ids, out_scores, extras, stream);

@@ -16,8 +16,9 @@
 //     stays in L2;
 //   * probe_select_cluster_kernel: one thread-block cluster per query (up to
 //     8 CTAs at small batches, so the whole GPU works on the selections). The
-//     keys' score range, a 2048-bin histogram over it summed through
-//     distributed shared memory, and the suffix counts give the bin holding
+//     keys' a-priori score range [-128 sum|q_j|, 128 sum|q_j|], a 2048-bin
+//     histogram over it summed through distributed shared memory, and the
+//     suffix counts give the bin holding
 //     the nprobe-th best score, so only the keys at or above that bin (a few
 //     more than nprobe) reach the leader CTA for the exact selection and the
 //     sort. The leader then writes the probe result and files the query into
@@ -33,10 +34,11 @@
 namespace st {
 
 // Write the probe result of query b from its P best keys, sorted (sorted[p],
-// p < P). kFile: also file the query into its lists (the search): the query's
-// mask bits in increasing order, then for each chosen list the next rank of
-// the list's query counter and the query's id, mask and first kSlotBits mask
-// bits in that slot of the list's slot row. The allocation-free probe-only call writes the result alone.
+// p < P). kFile: also file the query into its lists (the search): the bits of
+// each of its masks (its mask and its alternatives) in increasing order, then
+// for each chosen list the next rank of the list's query counter and, in that
+// slot of the list's slot row, the query's id, the union of its masks and the
+// first kSlotBits bits of its mask. The allocation-free probe-only call writes the result alone.
 template <int BLOCK, bool kFile>
 __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
 {
@@ -46,26 +48,40 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
         return;
     }
     const int W = a.W;
+    const int n_alt = 1 + a.n_or;  // the query's masks: qmasks[b], then its alternatives
     __shared__ __align__(16) uint8_t s_bits[kSlotBits];
+    __shared__ uint64_t s_union[2];
     if (threadIdx.x < 32) {
-        const uint64_t m0 = a.qmasks[int64_t(b) * W];
-        const uint64_t m1 = W > 1 ? a.qmasks[int64_t(b) * W + 1] : 0ull;
         const int lane = threadIdx.x;
-        int n_before = 0;
-        for (int r = 0; r < 2 * W; ++r) {
-            const int bit = 32 * r + lane;
-            const uint64_t word = bit < 64 ? m0 : m1;
-            const bool on = (word >> (bit & 63)) & 1ull;
-            const unsigned bal = __ballot_sync(0xffffffffu, on);
-            const int j = n_before + __popc(bal & lanemask_lt());
-            if (on) {
-                a.qbits[int64_t(b) * kMaskBitsMax + j] = uint8_t(bit);
-                if (j < kSlotBits) s_bits[j] = uint8_t(bit);
+        uint64_t u0 = 0, u1 = 0;
+        for (int alt = 0; alt < n_alt; ++alt) {
+            const uint64_t* mk = alt == 0 ? a.qmasks + int64_t(b) * W : a.or_masks + (int64_t(b) * a.n_or + alt - 1) * W;
+            const uint64_t m0 = mk[0];
+            const uint64_t m1 = W > 1 ? mk[1] : 0ull;
+            u0 |= m0;
+            u1 |= m1;
+            const int64_t row = int64_t(b) * n_alt + alt;
+            int n_before = 0;
+            for (int r = 0; r < 2 * W; ++r) {
+                const int bit = 32 * r + lane;
+                const uint64_t word = bit < 64 ? m0 : m1;
+                const bool on = (word >> (bit & 63)) & 1ull;
+                const unsigned bal = __ballot_sync(0xffffffffu, on);
+                const int j = n_before + __popc(bal & lanemask_lt());
+                if (on) {
+                    a.qbits[row * kMaskBitsMax + j] = uint8_t(bit);
+                    if (alt == 0 && j < kSlotBits) s_bits[j] = uint8_t(bit);
+                }
+                n_before += __popc(bal);
             }
-            n_before += __popc(bal);
+            if (lane == 0) a.qnbits[row] = n_before;
+            if (alt == 0)
+                for (int j = n_before + lane; j < kSlotBits; j += 32) s_bits[j] = 0;
         }
-        if (lane == 0) a.qnbits[b] = n_before;
-        for (int j = n_before + lane; j < kSlotBits; j += 32) s_bits[j] = 0;
+        if (lane == 0) {
+            s_union[0] = u0;
+            s_union[1] = u1;
+        }
     }
     if (a.qscale != nullptr && threadIdx.x >= 32 && threadIdx.x < 64) {
         // bound of the query's scores, for the score bins of the scans and
@@ -82,7 +98,7 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
             a.qscale[b] = make_int2(-S, sh);
         }
     }
-    __syncthreads();  // s_bits holds the query's first mask bits
+    __syncthreads();  // s_bits holds the query's first mask bits, s_union its masks' union
     const uint4 sb0 = reinterpret_cast<const uint4*>(s_bits)[0], sb1 = reinterpret_cast<const uint4*>(s_bits)[1];
     for (int p = threadIdx.x; p < P; p += BLOCK) {
         const int L = int(key_id(sorted[p]));
@@ -91,9 +107,8 @@ __device__ void file_query(const SearchArgs& a, int b, const uint64_t* sorted)
             const int r = atomicAdd(&a.list_cnt[L], 1);
             const int64_t slot = int64_t(L) * a.B + r;
             a.qlist[slot] = b;
-            const uint64_t m0 = a.qmasks[int64_t(b) * W];
-            const uint64_t m1 = W > 1 ? a.qmasks[int64_t(b) * W + 1] : 0ull;
-            reinterpret_cast<ulonglong2*>(a.qmask_slot)[slot] = make_ulonglong2(m0, m1);
+            // the union of the query's masks: the planes its units need
+            reinterpret_cast<ulonglong2*>(a.qmask_slot)[slot] = make_ulonglong2(s_union[0], s_union[1]);
             uint4* sbits = reinterpret_cast<uint4*>(a.slot_bits + slot * kSlotBits);
             sbits[0] = sb0;
             sbits[1] = sb1;
@@ -260,9 +275,20 @@ probe_select_cluster_kernel(SearchArgs a)
     uint64_t* tie = tmp + ((P + 1) & ~1);
     uint64_t* out = tie + kProbeTieCap;
     const uint64_t* row = a.probe_keys + int64_t(b) * probe_keys_ld(a.nlist);
+    // every centroid score lies in [-Sc, Sc], Sc = 128 sum_j |q_j| (int8
+    // centroids), so the selection needs no pass over the keys for their range
+    __shared__ int32_t s_sc;
+    if (threadIdx.x < 32) {
+        int32_t sum = 0;
+        for (int j = threadIdx.x; j < a.d; j += 32) sum += abs(int32_t(a.queries[int64_t(b) * a.d + j]));
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (threadIdx.x == 0) s_sc = 128 * sum;
+    }
+    __syncthreads();
+    const int32_t sc = s_sc;
     auto none = [](uint64_t) { return true; };
     auto no_compact = []() { return 0; };
-    const int m = cluster_topk<CS, kProbeCBlock>(cluster, row, a.nlist, P, false, 0, 0, false, none, no_compact, tmp,
+    const int m = cluster_topk<CS, kProbeCBlock>(cluster, row, a.nlist, P, true, -sc, sc, false, none, no_compact, tmp,
                                                  tie, kProbeTieCap, out, ss, cc, a.err);
     if (m < 0) return;  // not the leader
     if (threadIdx.x == 0 && m != P) set_error(a.err, kErrSelectCount);

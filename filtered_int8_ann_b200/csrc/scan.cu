@@ -31,15 +31,18 @@
 //     shuffle joins the halves, so 32 rows cost one AND per mask bit;
 //   * filter-before-load: per-query survivor counts reserve candidate slots
 //     (one atomic per unit and query, answered while the previous unit is
-//     scored) and the survivors' rows are prefetched into L2; one iteration
-//     later only those rows are read (16-byte read-only loads) and dotted with
-//     dp4a against the query vectors (staged in shared memory by cp.async); a
+//     scored); the first survivors' rows are copied into the warp's shared
+//     memory by cp.async and the next ones prefetched into L2, so one
+//     iteration later only those rows are read (from shared memory, or by
+//     16-byte read-only loads) and dotted with dp4a against the query vectors
+//     (staged in shared memory by cp.async); a
 //     key's slot is its rank among the unit's survivors of that query, and
 //     the key is counted in the query's score bins (kTcBins bins over the
 //     query's possible range [-S, S]), which guide the final top-k.
 // Every unit commits exactly two cp.async groups (planes of the unit two
-// ahead, then query vectors of the next unit), so fixed wait_group depths find
-// every copy: there is no spin loop and nothing to time out.
+// ahead, then query vectors and staged rows of the next unit), so fixed
+// wait_group depths find every copy: there is no spin loop and nothing to
+// time out.
 #include "st_internal.cuh"
 
 namespace st {
@@ -49,14 +52,20 @@ static_assert(kPlaneSlots <= kSlotBits, "a slot carries every bit of a mask whos
 constexpr int kPlaneBytes = kWarpItems / 8;             // 64 bytes per plane
 constexpr int kPlaneBufBytes = kPlaneSlots * kPlaneBytes;
 
-// Per-warp shared memory: plane buffer | survivor offsets [2][kWarpItems] u16 |
-// pass words [2][kQMax][16] | query vectors [kQMax][d] | bit -> slot table
-// [128] | slot -> bit [kPlaneSlots]
+// Survivor rows a unit stages in shared memory (its first survivors; the
+// others are read from global memory): sized so that the warps the registers
+// allow stay resident (five CTAs per SM for d = 64, four for d = 128).
+__host__ __device__ constexpr int scan_stage_rows(int d) { return d == 64 ? 24 : d == 128 ? 16 : 0; }
+
+// Per-warp shared memory: staged survivor rows [2][scan_stage_rows(d)][d] |
+// plane buffer | survivor offsets [2][kWarpItems] u16 | pass words
+// [2][kQMax][16] | query vectors [kQMax][d] | bit -> slot table [128] | slot
+// -> bit [kPlaneSlots]
 __host__ __device__ inline size_t scan_warp_bytes(int d, int W)
 {
     (void)W;
-    return (kPlaneBufBytes + 2 * kWarpItems * 2 + 2 * kQMax * 16 * 4 + size_t(kQMax) * d + kMaskBitsMax +
-            kPlaneSlots + 127) / 128 * 128;
+    return (size_t(2) * scan_stage_rows(d) * d + kPlaneBufBytes + 2 * kWarpItems * 2 + 2 * kQMax * 16 * 4 +
+            size_t(kQMax) * d + kMaskBitsMax + kPlaneSlots + 127) / 128 * 128;
 }
 
 size_t scan_smem_bytes(int d, int W) { return size_t(kScanBlock / 32) * scan_warp_bytes(d, W); }
@@ -124,7 +133,10 @@ scan_kernel(SearchArgs a)
     const int blk = lane & 15;   // 32-row block of the chunk this lane tests
     const int half = lane >> 4;  // which half of the mask bits it ANDs
 
+    constexpr int R = scan_stage_rows(NP * 16);  // staged rows per unit (0: none)
     unsigned char* wb = smem_raw + size_t(warp) * scan_warp_bytes(d, W);
+    int4* const srow2 = reinterpret_cast<int4*>(wb);  // [2][R][NP]
+    wb += size_t(2) * R * NP * 16;
     uint32_t* const pbuf = reinterpret_cast<uint32_t*>(wb);
     uint16_t* const surv2 = reinterpret_cast<uint16_t*>(wb + kPlaneBufBytes);            // [2][kWarpItems]
     uint32_t* const pass2 = reinterpret_cast<uint32_t*>(surv2 + 2 * kWarpItems);         // [2][kQMax][16]
@@ -173,7 +185,7 @@ scan_kernel(SearchArgs a)
     // unit needs no union: its planes are the query's mask bits in increasing
     // order, which its slot carries (lane j holds bit j in sb).
     auto request_planes = [&](const int4& e, uint64_t m0, uint64_t m1, uint32_t sb) -> int {
-        if ((e.w & 0xFFFF) == 1) {
+        if ((e.w & 0xFFFF) == 1 && a.n_or == 0) {
             const uint64_t x = __shfl_sync(0xffffffffu, m0, 0), y = __shfl_sync(0xffffffffu, m1, 0);
             const int nb = __popcll(x) + (W > 1 ? __popcll(y) : 0);
             if (nb > kPlaneSlots) return -1;
@@ -213,7 +225,7 @@ scan_kernel(SearchArgs a)
                              : (len <= 32 * blk ? 0u : ((1u << (len - 32 * blk)) - 1u));
         any = 0;
         mycnt = 0;
-        if (qn == 1 && held >= 0) {
+        if (qn == 1 && held >= 0 && a.n_or == 0) {
             // the buffer holds exactly the query's planes, in bit order
             const int h0 = (held + 1) >> 1;
             const int j1 = half ? held : h0;
@@ -228,18 +240,9 @@ scan_kernel(SearchArgs a)
             return;
         }
         const uint32_t* gpl = a.planes + int64_t(e.y) * NPL * 16 + blk;
-        for (int s = 0; s < qn; ++s) {
-            // query s's mask bits: from its slot when the buffer holds the
-            // planes (then it has at most kPlaneSlots <= kSlotBits of them),
-            // else from the query's own list
-            const int qg = __shfl_sync(0xffffffffu, qid, s);
-            const uint64_t x = __shfl_sync(0xffffffffu, m0, s), y = __shfl_sync(0xffffffffu, m1, s);
-            const int nb = __popcll(x) + (W > 1 ? __popcll(y) : 0);
-            const int h0 = (nb + 1) >> 1;
-            const uint8_t* bits = held >= 0 ? a.slot_bits + int64_t(e.z + s) * kSlotBits
-                                            : a.qbits + int64_t(qg) * kMaskBitsMax;
-            const int j0 = half ? h0 : 0, j1 = half ? nb : h0;
-            // four independent bit -> slot -> plane chains per step
+        // AND of the planes of bits[j0 .. j1) for this lane's 32-row block:
+        // four independent bit -> slot -> plane chains per step
+        auto and_bits = [&](const uint8_t* bits, int j0, int j1) -> uint32_t {
             uint32_t acc = 0xFFFFFFFFu;
             if (held >= 0) {
                 int j = j0;
@@ -253,7 +256,37 @@ scan_kernel(SearchArgs a)
             } else {
                 for (int j = j0; j < j1; ++j) acc &= __ldg(gpl + __ldg(bits + j) * 16);
             }
-            acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
+            return acc;
+        };
+        for (int s = 0; s < qn; ++s) {
+            const int qg = __shfl_sync(0xffffffffu, qid, s);
+            uint32_t acc;
+            if (a.n_or == 0) {
+                // query s's mask bits: from its slot when the buffer holds the
+                // planes (then it has at most kPlaneSlots <= kSlotBits of them),
+                // else from the query's own list; the two half-warps take the
+                // two halves of them
+                const uint64_t x = __shfl_sync(0xffffffffu, m0, s), y = __shfl_sync(0xffffffffu, m1, s);
+                const int nb = __popcll(x) + (W > 1 ? __popcll(y) : 0);
+                const int h0 = (nb + 1) >> 1;
+                const uint8_t* bits = held >= 0 ? a.slot_bits + int64_t(e.z + s) * kSlotBits
+                                                : a.qbits + int64_t(qg) * kMaskBitsMax;
+                acc = and_bits(bits, half ? h0 : 0, half ? nb : h0);
+                acc &= __shfl_xor_sync(0xffffffffu, acc, 16);
+            } else {
+                // alternative masks: the OR over them of each one's AND (the
+                // slot's mask, the union, chose the planes)
+                const int n_alt = 1 + a.n_or;
+                acc = 0;
+                for (int alt = 0; alt < n_alt; ++alt) {
+                    const int64_t row = int64_t(qg) * n_alt + alt;
+                    const int nb = __ldg(a.qnbits + row);
+                    const int h0 = (nb + 1) >> 1;
+                    uint32_t ac = and_bits(a.qbits + row * kMaskBitsMax, half ? h0 : 0, half ? nb : h0);
+                    ac &= __shfl_xor_sync(0xffffffffu, ac, 16);
+                    acc |= ac;
+                }
+            }
             acc &= valid;
             if (half == 0) pass[s * 16 + blk] = acc;
             any |= acc;
@@ -267,10 +300,11 @@ scan_kernel(SearchArgs a)
     };
 
     // After a unit's test: survivor row offsets -> sv, one reservation per
-    // query (lane s, the reply lands in `base`), L2 prefetch of the first
-    // survivors' rows. Returns the number of survivors.
+    // query (lane s, the reply lands in `base`), the first R survivors' rows
+    // copied into `srow` (cp.async, in the group the caller commits next) and
+    // the next ones prefetched into L2. Returns the number of survivors.
     auto settle_unit = [&](const int4& e, int qid, bool single, uint32_t any, uint32_t mycnt, uint16_t* sv,
-                           uint32_t& base) -> int {
+                           int4* srow, uint32_t& base) -> int {
         const uint32_t mine = half == 0 ? uint32_t(__popc(any)) : 0u;
         uint32_t incl = mine;
 #pragma unroll
@@ -295,8 +329,16 @@ scan_kernel(SearchArgs a)
             atomicAdd(&a.eligible_cnt[int64_t(qid) * (kCntStride / 2)], (unsigned long long)mycnt);
         }
         __syncwarp();
-        const int npf = nsurv < 64 ? nsurv : 64;
-        for (int idx = lane; idx < npf; idx += 32) {
+        if constexpr (R > 0) {
+            constexpr int NPS = NP > 0 ? NP : 1;
+            const int ns = nsurv < R ? nsurv : R;
+            for (int c = lane; c < ns * NPS; c += 32) {
+                const int idx = c / NPS, p = c - idx * NPS;
+                cp_async16_cg(srow + c, a.items + (int64_t(e.x) + sv[idx]) * d + 16 * p);
+            }
+        }
+        const int npf = nsurv < R + 64 ? nsurv : R + 64;
+        for (int idx = R + lane; idx < npf; idx += 32) {
             const int8_t* row = a.items + (int64_t(e.x) + sv[idx]) * d;
             for (int o = 0; o < d; o += 32) prefetch_l2(row + o);
         }
@@ -331,7 +373,7 @@ scan_kernel(SearchArgs a)
         __syncwarp();
         held = u_n1 < n_units ? request_planes(e_nxt, m0_n, m1_n, sb_n) : -1;
         cp_async_commit();
-        nsurv_c = settle_unit(e_cur, qid_c, single_c, any, mycnt, surv2, base_c);
+        nsurv_c = settle_unit(e_cur, qid_c, single_c, any, mycnt, surv2, srow2, base_c);
     }
     stage_queries(e_cur.w & 0xFFFF, qid_c);
     cp_async_commit();
@@ -366,7 +408,8 @@ scan_kernel(SearchArgs a)
             __syncwarp();
             held = has_n2 ? request_planes(e_n2, m0_2, m1_2, sb_2) : -1;
             cp_async_commit();
-            nsurv_n = settle_unit(e_nxt, qid_n, single_n, any, mycnt, surv2 + (cb ^ 1) * kWarpItems, base_n);
+            nsurv_n = settle_unit(e_nxt, qid_n, single_n, any, mycnt, surv2 + (cb ^ 1) * kWarpItems,
+                                  srow2 + (cb ^ 1) * R * NP, base_n);
         } else {
             cp_async_commit();  // two groups per unit, always
         }
@@ -378,6 +421,7 @@ scan_kernel(SearchArgs a)
         const int qn = e_cur.w & 0xFFFF;
         const uint16_t* surv = surv2 + cb * kWarpItems;
         const uint32_t* s_pass = pass2 + cb * kQMax * 16;
+        const int4* srow = srow2 + cb * R * NP;  // the first R survivors' rows
         if (single_c) {
             // every survivor is a key of the one query, in survivor order
             const int qg = __shfl_sync(0xffffffffu, qid_c, 0);
@@ -393,8 +437,13 @@ scan_kernel(SearchArgs a)
                     int32_t acc0 = 0, acc1 = 0;
                     if (NP > 0) {
                         int4 row[NP > 0 ? NP : 1];
+                        if (idx < R) {
 #pragma unroll
-                        for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
+                            for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = srow[idx * NP + p];
+                        } else {
+#pragma unroll
+                            for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
+                        }
 #pragma unroll
                         for (int p = 0; p < (NP > 0 ? NP : 1); p += 2) {
                             acc0 = dot16(row[p], s_q[p], acc0);
@@ -424,8 +473,13 @@ scan_kernel(SearchArgs a)
                     i = ib + off;
                     rp = reinterpret_cast<const int4*>(a.items + i * d);
                     if (NP > 0) {
+                        if (idx < R) {
 #pragma unroll
-                        for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
+                            for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = srow[idx * NP + p];
+                        } else {
+#pragma unroll
+                            for (int p = 0; p < (NP > 0 ? NP : 1); ++p) row[p] = __ldg(rp + p);
+                        }
                     }
                 }
                 const uint32_t* pw = s_pass + (off >= 0 ? (off >> 5) : 0);

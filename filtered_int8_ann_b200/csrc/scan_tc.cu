@@ -281,7 +281,48 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
 #pragma unroll
             for (int w = 0; w < 16; ++w)
                 acc[w] = len >= 32 * (w + 1) ? 0xFFFFFFFFu : (len <= 32 * w ? 0u : ((1u << (len - 32 * w)) - 1u));
-            if (lane < qn) {
+            if (lane < qn && a.n_or > 0) {
+                // alternative masks: for each 16-byte chunk of the pass words,
+                // the OR over the query's masks of each one's AND (the slot's
+                // mask, the union, chose the planes)
+                const uint4* pl = reinterpret_cast<const uint4*>(Pbuf + p * kTcPlaneSlots * 16);
+                const uint4* gpl = reinterpret_cast<const uint4*>(a.planes + int64_t(e.y) * NPL * 16);
+                const int qid = mt.qid[lane], n_alt = 1 + a.n_or;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                    for (int alt = 0; alt < n_alt; ++alt) {
+                        const uint64_t* mk = alt == 0 ? a.qmasks + int64_t(qid) * W
+                                                      : a.or_masks + (int64_t(qid) * a.n_or + alt - 1) * W;
+                        uint4 v = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+                        for (int word = 0; word < W; ++word) {
+                            unsigned long long m = __ldg(mk + word);
+                            while (m) {
+                                const int b = 64 * word + __ffsll(static_cast<long long>(m)) - 1;
+                                m &= m - 1;
+                                const uint4 x = held >= 0 ? pl[mt.tab[b] * 4 + c] : __ldg(gpl + b * 4 + c);
+                                v.x &= x.x;
+                                v.y &= x.y;
+                                v.z &= x.z;
+                                v.w &= x.w;
+                            }
+                        }
+                        o.x |= v.x;
+                        o.y |= v.y;
+                        o.z |= v.z;
+                        o.w |= v.w;
+                    }
+                    // (a dynamic chunk index would put acc[] in local memory)
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        if (cc == c) {
+                            acc[4 * cc] &= o.x;
+                            acc[4 * cc + 1] &= o.y;
+                            acc[4 * cc + 2] &= o.z;
+                            acc[4 * cc + 3] &= o.w;
+                        }
+                }
+            } else if (lane < qn) {
                 const uint4* pl = reinterpret_cast<const uint4*>(Pbuf + p * kTcPlaneSlots * 16);
                 const uint4* gpl = reinterpret_cast<const uint4*>(a.planes + int64_t(e.y) * NPL * 16);
 #pragma unroll

@@ -68,6 +68,10 @@ __device__ int64_t overflow_path(const SearchArgs& a, int q, uint64_t* sortbuf, 
                     const uint64_t* sg = a.sigs + i * W;
                     bool pass = (sg[0] & m0) == m0;
                     if (W > 1) pass = pass && ((sg[1] & m1) == m1);
+                    for (int alt = 0; alt < a.n_or && !pass; ++alt) {  // alternative masks: any one passes
+                        const uint64_t* x = a.or_masks + (int64_t(q) * a.n_or + alt) * W;
+                        pass = (sg[0] & x[0]) == x[0] && (W < 2 || (sg[1] & x[1]) == x[1]);
+                    }
                     pass = pass && keep_item(a, q, i);
                     if (pass) {
                         const int4* rp = reinterpret_cast<const int4*>(a.items + i * d);

@@ -112,6 +112,8 @@ struct SearchArgs {
     int64_t id_offset;       // added to every returned item id
     const uint32_t* dead;    // [ceil(n / 32)] deleted items, or null (none deleted)
     const uint64_t* qexclude;  // [B][W] exclude masks, or null
+    const uint64_t* or_masks;  // [B][n_or][W] alternative masks (an item passing any mask is eligible), or null
+    int32_t n_or;              // alternatives per query besides qmasks (0: none)
     unsigned long long* eligible_cnt;  // [B][kCntStride / 2], word 0 used        (zeroed)
     PlanCtl* ctl;            // unit allocation counter                   (zeroed)
     int32_t* probe;          // [B][P]
@@ -121,8 +123,8 @@ struct SearchArgs {
     int32_t* qlist;          // [nlist][B] slot row of each list: ids of the queries probing it
     uint64_t* qmask_slot;    // [nlist][B][2] that query's mask words (word 1 = 0 when W = 1)
     uint8_t* slot_bits;      // [nlist][B][kSlotBits] that query's first kSlotBits mask bits, increasing
-    uint8_t* qbits;          // [B][kMaskBitsMax] each query's mask bits, in increasing order
-    int32_t* qnbits;         // [B] number of mask bits of each query
+    uint8_t* qbits;          // [B][1 + n_or][kMaskBitsMax] each mask's bits, in increasing order
+    int32_t* qnbits;         // [B][1 + n_or] number of bits of each mask
     int4* units;             // [max_units] {first row, chunk, first slot, rows << 16 | queries}
     int4* units_tc;          // [max_units] dense units, same entries (up to kTcQMax queries)
     int32_t max_units;

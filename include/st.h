@@ -60,6 +60,7 @@ typedef enum {
                                 probed lists (ST_ERR_OOM when it does not fit) */
 #define ST_MAX_NPROBE 4096   /* 1 <= nprobe <= min(nlist, 4096) */
 #define ST_MAX_B 32768       /* 1 <= B <= 32768 queries per call */
+#define ST_MAX_OR 7          /* alternative masks per query (st_search_extras.n_or) */
 /* n < 2^31 items; sig_words is 1 (64-bit signatures) or 2 (128-bit). */
 
 /*
@@ -128,6 +129,15 @@ typedef struct {
        final top-k (at most its eligible count; fewer when the scan dropped
        keys that could no longer enter the top-k). */
     int64_t* candidates;
+    /* device uint64 [B][n_or][sig_words]: alternative masks, an OR of values
+       (for example any of several languages). An item is eligible for query b
+       when its signature passes qmasks[b] or any of query b's n_or
+       alternatives, each tested like the mask itself; the list scan tests
+       them all in the same pass, and eligible counts count an item once.
+       n_or = 0 (or_masks may then be NULL): the plain mask. INVALID_ARG when
+       n_or is outside [0, ST_MAX_OR] or or_masks is not a device pointer. */
+    const uint64_t* or_masks;
+    int32_t n_or;
 } st_search_extras;
 
 /* st_search with optional extra outputs (extras may be NULL). */
