@@ -11,16 +11,17 @@
 //
 // A persistent CTA per SM, warp-specialized, its roles handing units on
 // through mbarriers so that several units are in flight at once:
-//   * producer warp: the unit's query slots (three units ahead), its
+//   * two producer warps, on different SM sub-partitions, taking alternate
+//     units: the unit's query slots (three of the warp's units ahead), its
 //     signature bit-planes (the union of its queries' mask bits, by cp.async,
-//     two units ahead), the Bloom test (pass words [32-row block][query]),
-//     then the rows: a 32-row block with many survivors (for any of the unit's
-//     queries) is copied whole by a TMA tile load (a 128-row tile when four
-//     neighbouring blocks are), a block with few has only
-//     its survivors' rows gathered by cp.async, a block without survivors is
-//     not read; both land in the canonical 128-byte (d = 128) or 64-byte
-//     (d = 64) swizzled K-major layout of an operand stage, with the unit's
-//     query vectors;
+//     two of its units ahead, into the warp's own two plane buffers), the
+//     Bloom test (pass words [32-row block][query]), then the rows: a 32-row
+//     block with many survivors (for any of the unit's queries) is copied
+//     whole by a TMA tile load (a 128-row tile when four neighbouring blocks
+//     are), a block with few has only its survivors' rows gathered by
+//     cp.async, a block without survivors is not read; both land in the
+//     canonical 128-byte (d = 128) or 64-byte (d = 64) swizzled K-major layout
+//     of an operand stage, with the unit's query vectors;
 //   * MMA warp: one thread issues tcgen05.mma kind::i8 (M = 128 rows, N = the
 //     unit's queries rounded up to 16, K = 32) into int32 accumulators in TMEM
 //     and commits to mbarriers that free the operand stage and hand the
@@ -59,13 +60,17 @@ constexpr int kTcPlaneSlots = 48;        // planes one buffer holds
 #endif
 constexpr int kTcDenseBlk = ST_TC_DENSE_BLK;  // survivors of a 32-row block from which the whole block is loaded
 constexpr uint32_t kTcWaitLimit = 1u << 22;
-// Units whose data are held at once: a unit's slot is refilled only after its
-// epilogue, which the producer knows to be done once S + 4 units later have
-// had their operands consumed (operand stages S, epilogue groups 4).
+// Units whose data are held at once. A producer refills the slot of unit
+// j - 8 (with unit j + 4) only after the MMAs of unit j - S (operand stages
+// S = 2 or 4) are done; those of unit j - 4 then are too, and they waited for
+// the epilogue of unit j - 8 (epilogue groups 4) to free its accumulators.
 constexpr int kTcMeta = 12;
 constexpr uint32_t kTcBoundMinKeys = 16; // keys of a query in one unit that make it re-read its bound
 constexpr int kTcEpiGroups = 4;         // epilogue warpgroups, one per TMEM accumulator stage
-constexpr int kTcThreads = 32 * (2 + 4 * kTcEpiGroups);
+constexpr int kTcProducers = 2;         // producer warps (units alternate between them)
+constexpr int kTcProd1Warp = 2 + 4 * kTcEpiGroups;  // the second producer: the last warp
+constexpr int kTcThreads = 32 * (2 + 4 * kTcEpiGroups + 1);
+static_assert(kTcProducers == 2, "warp 0 and the last warp produce");
 constexpr int kTcAccCols = 4 * kTcQMax;  // TMEM columns of one unit's accumulators (4 row blocks)
 constexpr int kTcTmemCols = kTcEpiGroups * kTcAccCols;
 
@@ -123,7 +128,7 @@ struct TcLayout {
     static constexpr size_t kA = 0;
     static constexpr size_t kB = kA + size_t(tc_stages<D>()) * kTcRows * D;
     static constexpr size_t kP = kB + size_t(tc_stages<D>()) * kTcQMax * D;
-    static constexpr size_t kMeta = kP + size_t(2) * kTcPlaneSlots * 64;
+    static constexpr size_t kMeta = kP + size_t(2 * kTcProducers) * kTcPlaneSlots * 64;
     static constexpr size_t kEpi = kMeta + size_t(kTcMeta) * sizeof(TcMeta);
     static constexpr size_t kEnd = kEpi + size_t(kTcEpiGroups) * sizeof(TcEpi);
     static_assert(kMeta % alignof(TcMeta) == 0 && kEpi % alignof(TcEpi) == 0, "aligned carve-up");
@@ -158,7 +163,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
     using L = TcLayout<D>;
     unsigned char* const Abuf = base + L::kA;                                 // [S][kTcRows * D]
     unsigned char* const Bbuf = base + L::kB;                                 // [S][kTcQMax * D]
-    uint32_t* const Pbuf = reinterpret_cast<uint32_t*>(base + L::kP);         // [2][kTcPlaneSlots][16]
+    uint32_t* const Pbuf = reinterpret_cast<uint32_t*>(base + L::kP);  // [2 * kTcProducers][kTcPlaneSlots][16]
     TcMeta* const meta = reinterpret_cast<TcMeta*>(base + L::kMeta);          // [kTcMeta]
     TcEpi* const epi = reinterpret_cast<TcEpi*>(base + L::kEpi);              // [kTcEpiGroups]
 
@@ -195,8 +200,12 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
         return false;
     };
 
-    if (warp == 0) {
-        // ============================== producer ==============================
+    if (warp == 0 || warp == kTcProd1Warp) {
+        // ============================== producers =============================
+        // producer `pid` takes units pid, pid + 2, pid + 4, ... with plane
+        // buffers 2 pid and 2 pid + 1 (alternate units of its own)
+        const int pid = warp == 0 ? 0 : 1;
+        constexpr int P2 = kTcProducers;
         struct Slots {
             int4 e;
             int qid;
@@ -410,48 +419,64 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             if (lane == 0) mbar_arrive(&full_bar[s]);
         };
 
-        // prologue: slots and planes of units 0 and 1, slots of unit 2 in registers
-        Slots r0 = load_slots(0);
-        finish_slots(r0);
-        store_and_request(0, 0, r0);
+        // prologue: slots and planes of this producer's first two units, slots
+        // of its third in registers
+        if (pid < n_iter) {
+            Slots r0 = load_slots(pid);
+            finish_slots(r0);
+            store_and_request(pid % kTcMeta, 2 * pid, r0);
+        }
         cp_async_commit();
-        if (n_iter > 1) {
-            Slots r1 = load_slots(1);
+        if (pid + P2 < n_iter) {
+            Slots r1 = load_slots(pid + P2);
             finish_slots(r1);
-            store_and_request(1, 1, r1);
+            store_and_request((pid + P2) % kTcMeta, 2 * pid + 1, r1);
         }
         cp_async_commit();
         cp_async_commit();
         Slots nxt;
-        if (n_iter > 2) {
-            nxt = load_slots(2);
+        if (pid + 2 * P2 < n_iter) {
+            nxt = load_slots(pid + 2 * P2);
             finish_slots(nxt);
         }
-        for (int j = 0; j < n_iter; ++j) {
-            const int s = j % S, m = j % kTcMeta, p = j & 1;
+        int last = -1;  // this producer's latest unit
+        for (int j = pid, it = 0; j < n_iter; j += P2, ++it) {
+            const int s = j % S, m = j % kTcMeta, p = 2 * pid + (it & 1);
             TC_T0(t0);
+            // the queries' current bounds (they only grow; the ones loaded with
+            // the slots are several units old), stored before the epilogue gets
+            // the unit, so both of its passes see one value per query
+            uint32_t thr_now = 0;
+            const int qn_j = meta[m].e.w & 0xFFFF;
+            if (lane < qn_j) thr_now = __ldcg(a.score_rng + int64_t(meta[m].qid[lane]) * kCntStride + kRngThr);
             cp_async_wait_group<2>();  // planes of unit j
             __syncwarp();
             TC_T0(t1);
             test_unit(m, p);
             TC_T0(t2);
-            if (j >= S && !wait(&empty_bar[s], uint32_t(j / S - 1) & 1u)) break;
+            // the rows of this producer's previous unit (the older of the two
+            // pending groups [rows, planes]) complete its operand stage: this
+            // must not wait for a free stage, which that unit's MMAs may be
+            // the ones to free (two producers, two stages)
+            if (last >= 0) {
+                cp_async_wait_group<1>();
+                gathers_done(last % S);
+            }
             TC_T0(t3);
+            if (j >= S && !wait(&empty_bar[s], uint32_t(j / S - 1) & 1u)) break;
+            TC_T0(t4);
             issue_rows(m, s);
             cp_async_commit();
+            if (lane < qn_j && thr_now > meta[m].thr[lane]) meta[m].thr[lane] = thr_now;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&meta_full[m]);  // slots, pass words and row blocks of unit j
-            TC_T0(t4);
-            if (j >= 1) {
-                cp_async_wait_group<2>();  // rows of unit j - 1
-                gathers_done((j - 1) % S);
-            }
+            if (lane == 0) mbar_arrive(&meta_full[m]);  // slots, pass words, bounds and row blocks of unit j
+            last = j;
             TC_T0(t5);
-            if (j + 2 < n_iter) store_and_request((j + 2) % kTcMeta, p, nxt);
+            if (j + 2 * P2 < n_iter) store_and_request((j + 2 * P2) % kTcMeta, p, nxt);
             cp_async_commit();
             TC_T0(t6);
-            if (j + 3 < n_iter) {
-                nxt = load_slots(j + 3);
+            if (j + 3 * P2 < n_iter) {
+                nxt = load_slots(j + 3 * P2);
                 finish_slots(nxt);
             }
             if (lane == 0) {
@@ -459,7 +484,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             }
         }
         cp_async_wait_all();
-        if (!s_abort && n_iter > 0) gathers_done((n_iter - 1) % S);
+        if (!s_abort && last >= 0) gathers_done(last % S);
     } else if (warp == 1) {
         // ================================ MMA =================================
         for (int j = 0; j < n_iter; ++j) {
