@@ -284,7 +284,7 @@ def _probed_rows(off, sizes, lists):
         int(lens.sum()), device=off.device)
 
 
-def byte_model(data, probe, qmasks, W, d, k, nlist):
+def byte_model(data, probe, qmasks, W, d, k, nlist, alt=None):
     """Algorithmic bytes of one search (probe [B, P] of the batch).
 
     Scan kernel, index layout of the library: every probed list is read once
@@ -296,13 +296,18 @@ def byte_model(data, probe, qmasks, W, d, k, nlist):
     model the method's description implies (`scan_rowmajor`).
     Whole step: the scan plus the centroids (nlist d), the queries and masks
     (B (d + 8W)) and the outputs (B k 12) -- `step_planes`, `step_rowmajor`.
-    Full scan: every row and signature of every distinct probed list."""
+    Full scan: every row and signature of every distinct probed list.
+    alt [B, A, W] (optional): alternative masks of each query (an item passing
+    any of the query's masks is eligible): a list's planes are those of the
+    union of all of them, a row is read when it passes any."""
     off = data.offsets
     sizes = off[1:] - off[:-1]
     lists = torch.unique(probe.flatten().long())
     scanned = int(sizes[lists].sum())
     pr = probe.long().cpu().numpy()
     mk = qmasks.cpu().numpy().view(np.uint64).reshape(qmasks.shape[0], -1)
+    if alt is not None:
+        mk = mk | np.bitwise_or.reduce(alt.cpu().numpy().view(np.uint64), axis=1)
     union = np.zeros((sizes.numel(), mk.shape[1]), dtype=np.uint64)
     for w in range(mk.shape[1]):
         np.bitwise_or.at(union[:, w], pr.reshape(-1), np.repeat(mk[:, w], pr.shape[1]))
@@ -333,6 +338,9 @@ def byte_model(data, probe, qmasks, W, d, k, nlist):
         owner = torch.repeat_interleave(torch.arange(b0, b1, device=off.device), sizes[pl].sum(1))
         m = qmasks[owner]
         ok = torch.all((data.sigs[idx] & m) == m, dim=1)
+        for j in range(alt.shape[1] if alt is not None else 0):
+            ma = alt[owner, j]
+            ok |= torch.all((data.sigs[idx] & ma) == ma, dim=1)
         surv[idx[ok]] = True
         lst = torch.repeat_interleave(pl.reshape(-1), sizes[pl.reshape(-1)])
         pairs += int(ok.sum())
@@ -895,6 +903,40 @@ def main():
             except st.StError as ex:
                 lk[str(kk)] = {"error": str(ex)}
         ext["large_k"] = lk
+        # OR of M masks per query (M - 1 alternatives: other queries' masks of
+        # the batch, i.e. other languages and countries): one fused search
+        # against M single-mask searches merged, with the scan's algorithmic
+        # bytes of each
+        orr = {}
+        for M in (2, 4):
+            alts = [torch.stack([torch.roll(m[b], -j, dims=0) for j in range(1, M)], dim=1).contiguous()
+                    for b in range(pool)]
+            sets = [torch.cat([m[b].unsqueeze(0), alts[b].permute(1, 0, 2)], dim=0).contiguous() for b in range(pool)]
+            for i in range(3):
+                idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores, or_masks=alts[i % pool])
+                idx.search_any_merged(q[i % pool], sets[i % pool], P, k)
+            torch.cuda.synchronize()
+            reps = 20
+            x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            x0.record()
+            for i in range(reps):
+                idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores, or_masks=alts[i % pool])
+            x1.record()
+            torch.cuda.synchronize()
+            t_fused = x0.elapsed_time(x1) / reps
+            x0.record()
+            for i in range(reps):
+                idx.search_any_merged(q[i % pool], sets[i % pool], P, k)
+            x1.record()
+            torch.cuda.synchronize()
+            t_sep = x0.elapsed_time(x1) / reps
+            assert idx.check() == st.ST_OK and st.st_merge_check() == st.ST_OK
+            fused_b = byte_model(data, probe[0], m[0], W, d, k, wl.nlist, alt=alts[0])["scan_planes"]
+            sep_b = sum(byte_model(data, probe[0], sets[0][j], W, d, k, wl.nlist)["scan_planes"] for j in range(M))
+            orr[str(M)] = {"fused_ms_per_step": t_fused, "separate_ms_per_step": t_sep,
+                           "fused_scan_bytes": fused_b, "separate_scan_bytes": sep_b,
+                           "separate": "M single-mask searches, then the exact union merge"}
+        ext["or_masks"] = orr
         # streamed updates, last: they change the headline index
         ext["freshness"] = freshness(st, idx, flat_src[0], flat_src[1], wl.nlist, q, m, P, k)
         del flat_src
@@ -974,7 +1016,7 @@ def main():
                                "bloom_false_negatives": None if fp_stats is None else int(fp_stats[2]),
                                **({"recall_at_k": ext["recall_at_k"]} if "recall_at_k" in ext else {})},
         }
-        for key in ("large_k", "freshness", "per_config"):
+        for key in ("large_k", "or_masks", "freshness", "per_config"):
             if key in ext:
                 line[key] = ext[key]
         print(json.dumps(line), flush=True)
