@@ -735,6 +735,17 @@ def main():
         flat_idx = open_index(st, data.items, data.sigs,
                             torch.tensor([0, data.items.shape[0]], dtype=torch.int64, device=dev),
                             torch.zeros((1, d), dtype=torch.int8, device=dev))
+    # OR of M masks per query (the extras): M - 1 alternatives per query, the
+    # masks of the next queries of the batch (other languages and countries);
+    # the scan's algorithmic bytes of one fused search and of M single searches
+    or_alts, or_bytes = {}, {}
+    if extras:
+        for M in (2, 4):
+            or_alts[M] = [torch.stack([torch.roll(m[b], -j, dims=0) for j in range(1, M)], dim=1).contiguous()
+                          for b in range(pool)]
+            sets0 = [m[0]] + [or_alts[M][0][:, j].contiguous() for j in range(M - 1)]
+            or_bytes[M] = (byte_model(data, probe[0], m[0], W, d, k, wl.nlist, alt=or_alts[M][0])["scan_planes"],
+                           sum(byte_model(data, probe[0], x, W, d, k, wl.nlist)["scan_planes"] for x in sets0))
     del data
     torch.cuda.empty_cache()
 
@@ -909,8 +920,7 @@ def main():
         # bytes of each
         orr = {}
         for M in (2, 4):
-            alts = [torch.stack([torch.roll(m[b], -j, dims=0) for j in range(1, M)], dim=1).contiguous()
-                    for b in range(pool)]
+            alts = or_alts[M]
             sets = [torch.cat([m[b].unsqueeze(0), alts[b].permute(1, 0, 2)], dim=0).contiguous() for b in range(pool)]
             for i in range(3):
                 idx.search(q[i % pool], m[i % pool], P, k, out_ids=ids, out_scores=scores, or_masks=alts[i % pool])
@@ -931,8 +941,7 @@ def main():
             torch.cuda.synchronize()
             t_sep = x0.elapsed_time(x1) / reps
             assert idx.check() == st.ST_OK and st.st_merge_check() == st.ST_OK
-            fused_b = byte_model(data, probe[0], m[0], W, d, k, wl.nlist, alt=alts[0])["scan_planes"]
-            sep_b = sum(byte_model(data, probe[0], sets[0][j], W, d, k, wl.nlist)["scan_planes"] for j in range(M))
+            fused_b, sep_b = or_bytes[M]
             orr[str(M)] = {"fused_ms_per_step": t_fused, "separate_ms_per_step": t_sep,
                            "fused_scan_bytes": fused_b, "separate_scan_bytes": sep_b,
                            "separate": "M single-mask searches, then the exact union merge"}

@@ -339,8 +339,11 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_cand_cnt = L.add(size_t(B) * st::kCntStride * 4);
     L.off_elig = L.add(size_t(B) * st::kCntStride * 4);
     L.off_rng = L.add(size_t(B) * st::kCntStride * 4);
-    L.off_sel_hist = L.add(size_t(B) * st::kSelBins * 4);
-    L.off_sel_cursor = L.add(size_t(B) * st::kSelBins * 4);
+    // the chunked final top-k's per-query histograms (the cluster final top-k
+    // has no use for them, so they are not cleared then)
+    const size_t sel_bytes = st::select_reads_bins(B, k) ? 0 : size_t(B) * st::kSelBins * 4;
+    L.off_sel_hist = L.add(sel_bytes);
+    L.off_sel_cursor = L.add(sel_bytes);
     L.off_ctl = L.add(sizeof(st::PlanCtl));
     const int tc_min_q = (idx->tmap_ok && idx->tc_min_q > 0 && B >= idx->tc_min_q) ? idx->tc_min_q : 0;
     L.off_tc_hist = L.add(size_t(B) * st::kTcBins * 4);

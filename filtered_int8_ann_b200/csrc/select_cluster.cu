@@ -187,27 +187,41 @@ select_cluster_kernel(const __grid_constant__ SearchArgs a)
         } else {
             uint32_t* lcnt = cluster.map_shared_rank(&s_cnt, 0);
             uint64_t* lbuf = cluster.map_shared_rank(buf, 0);
-            // 2. this CTA's share of the keys; those at or above the cut go to the leader
-            const int64_t s0 = n * rank / CS, s1 = n * (rank + 1) / CS;
+            // 2. this CTA's share of the keys; those at or above the cut go to
+            // the leader. Shares start on even keys and are read as 16-byte
+            // pairs, eight pairs in flight per thread (the query's buffer is
+            // 256-byte aligned); an odd last key is read on its own.
+            const int64_t s0 = (n * rank / CS) & ~int64_t(1);
+            const int64_t s1 = rank == CS - 1 ? n : ((n * (rank + 1) / CS) & ~int64_t(1));
+            const ulonglong2* kp = reinterpret_cast<const ulonglong2*>(keys);
+            auto push = [&](bool take, uint64_t key) {
+                const unsigned bal = __ballot_sync(0xffffffffu, take);
+                if (!bal) return;
+                uint32_t p0 = 0;
+                if (lane == 0) p0 = atomicAdd(lcnt, uint32_t(__popc(bal)));
+                p0 = __shfl_sync(0xffffffffu, p0, 0);
+                const uint32_t pos = p0 + __popc(bal & lanemask_lt());
+                if (take && pos < uint32_t(cap)) lbuf[pos] = key;
+            };
             constexpr int U = 8;
-            for (int64_t base = s0; base < s1; base += int64_t(kCBlock) * U) {
-                uint64_t v[U];
+            const int64_t e0 = s0 >> 1, e1 = s1 >> 1;  // whole pairs of the share
+            for (int64_t base = e0; base < e1; base += int64_t(kCBlock) * U) {
+                ulonglong2 v[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const int64_t i = base + int64_t(u) * kCBlock + tid;
-                    v[u] = i < s1 ? keys[i] : 0ull;
+                    const int64_t e = base + int64_t(u) * kCBlock + tid;
+                    v[u] = e < e1 ? kp[e] : make_ulonglong2(0ull, 0ull);
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const bool take = base + int64_t(u) * kCBlock + tid < s1 && key_score(v[u]) >= T;
-                    const unsigned bal = __ballot_sync(0xffffffffu, take);
-                    if (!bal) continue;
-                    uint32_t p0 = 0;
-                    if (lane == 0) p0 = atomicAdd(lcnt, uint32_t(__popc(bal)));
-                    p0 = __shfl_sync(0xffffffffu, p0, 0);
-                    const uint32_t pos = p0 + __popc(bal & lanemask_lt());
-                    if (take && pos < uint32_t(cap)) lbuf[pos] = v[u];
+                    const bool in = base + int64_t(u) * kCBlock + tid < e1;
+                    push(in && key_score(v[u].x) >= T, v[u].x);
+                    push(in && key_score(v[u].y) >= T, v[u].y);
                 }
+            }
+            if (s1 & 1) {  // the odd last key (last CTA only)
+                const uint64_t key = warp == 0 ? keys[s1 - 1] : 0ull;
+                if (warp == 0) push(lane == 0 && key_score(key) >= T, key);
             }
             cluster.sync();  // every key at or above the cut is in the leader's memory
             if (rank != 0) return;
