@@ -27,10 +27,16 @@
 //     and commits to mbarriers that free the operand stage and hand the
 //     accumulators to an epilogue;
 //   * four epilogue warpgroups, one per TMEM accumulator stage (every fourth
-//     unit each): each thread reads its row's scores (tcgen05.ld), applies the
-//     pass bits, and keeps a key only if its score reaches the query's running
-//     bound (below); each warp counts its kept keys per query, reserves their
-//     slots with one atomic per query (all in flight at once) and writes them.
+//     unit each): each thread reads its row's scores (tcgen05.ld) and keeps a
+//     key only if the row passes the query's Bloom test and its score reaches
+//     the query's running bound (below), as one bit per query; a 32 x 32 bit
+//     transpose across the warp turns the pass words into these per-row words
+//     and the kept words into per-query row masks, whose popcounts are the
+//     warp's key counts. Each warp reserves its slots with one atomic per query
+//     (all in flight at once) and writes its keys at the query's base plus the
+//     key's rank in the row mask, counting each in its score bin with one
+//     atomic (the keys of one query in one 32-row block rarely share a bin, so
+//     grouping them first costs more than it saves).
 //
 // Running top-k bound. Intermediate results should stay on chip (Andromeda
 // review, section on why the bottleneck moved from compute to bandwidth), so
@@ -97,7 +103,24 @@ struct TcMeta {                          // one unit, from its slots to its epil
 
 struct TcEpi {                           // one epilogue warpgroup's per-query key counts (two units)
     uint32_t cnt[2][kTcQMax];
+    uint32_t wbase[4][kTcQMax];          // per warp: query q's next key slot in the current row block
+    uint32_t wcol[4][kTcQMax];           // per warp: query q's kept rows of the current row block
 };
+
+// 32 x 32 bit-matrix transpose across a warp: lane i holds row i (bit j =
+// element (i, j)) and gets column i (bit j = element (j, i)), by exchanging
+// ever smaller blocks between lanes
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane)
+{
+    const uint32_t lo[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        const int sft = 16 >> i;
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, x, sft);
+        x = (lane & sft) ? ((x & ~lo[i]) | ((y & ~lo[i]) >> sft)) : ((x & lo[i]) | ((y & lo[i]) << sft));
+    }
+    return x;
+}
 
 #ifdef ST_TC_PROF
 // Per-CTA cycle counters of the pipeline roles (a measuring build only).
@@ -185,7 +208,8 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
         tmem_alloc(&s_tmem, kTcTmemCols);
         tmem_relinquish();
     }
-    for (int i = tid; i < kTcEpiGroups * 2 * kTcQMax; i += kTcThreads) (&epi[0].cnt[0][0])[i] = 0;
+    for (int i = tid; i < kTcEpiGroups * 2 * kTcQMax; i += kTcThreads)
+        epi[i / (2 * kTcQMax)].cnt[(i / kTcQMax) & 1][i % kTcQMax] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -449,19 +473,12 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             uint32_t thr_now = 0;
             const int qn_j = meta[m].e.w & 0xFFFF;
             if (lane < qn_j) thr_now = __ldcg(a.score_rng + int64_t(meta[m].qid[lane]) * kCntStride + kRngThr);
-            cp_async_wait_group<2>();  // planes of unit j
+            cp_async_wait_group<1>();  // planes of unit j, rows of the previous unit
             __syncwarp();
+            if (last >= 0) gathers_done(last % S);
             TC_T0(t1);
             test_unit(m, p);
             TC_T0(t2);
-            // the rows of this producer's previous unit (the older of the two
-            // pending groups [rows, planes]) complete its operand stage: this
-            // must not wait for a free stage, which that unit's MMAs may be
-            // the ones to free (two producers, two stages)
-            if (last >= 0) {
-                cp_async_wait_group<1>();
-                gathers_done(last % S);
-            }
             TC_T0(t3);
             if (j >= S && !wait(&empty_bar[s], uint32_t(j / S - 1) & 1u)) break;
             TC_T0(t4);
@@ -543,68 +560,85 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             const int qn = e.w & 0xFFFF;
             if (mbm) {
                 const int nsl = (qn + 15) >> 4;
-                // pass 1: this warp's keys at or above the bound, counted per
-                // query in lane q
+                // pass 1: this thread's kept pairs of each row block as a word
+                // over the queries (bit q: the row passes query q's Bloom test
+                // and its score reaches q's bound), and, transposed, lane q's
+                // kept rows of query q
                 uint32_t myc = 0;
-                bool anyk = false;
+                uint32_t kw[4] = {0u, 0u, 0u, 0u}, cw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll 1
                 for (int mb = 0; mb < 4; ++mb) {
-                    if (!((mbm >> mb) & 1u)) continue;
+                    if (!((mbm >> mb) & 1u)) continue;  // warp-uniform
                     const int r = mb * 128 + wq * 32 + lane;
                     const int wb = r >> 5;
+                    const uint32_t T = warp_transpose32(lane < qn ? mt.pass[wb][lane] : 0u, lane);
+                    uint32_t K = 0;
                     for (int sl = 0; sl < nsl; ++sl) {
                         uint32_t v[16];
                         tmem_ld16(acc_base + uint32_t(mb * kTcQMax + sl * 16), v);
                         tmem_wait_ld();
+                        uint32_t k16 = 0;
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) {
-                            const int q = sl * 16 + jj;
-                            if (q >= qn) break;  // warp-uniform
-                            bool keep = ((mt.pass[wb][q] >> lane) & 1u) &&
-                                        (uint32_t(int32_t(v[jj])) ^ 0x80000000u) >= mt.thr[q];
-                            if (filt && keep) keep = keep_item(a, mt.qid[q], int64_t(e.x) + r);
-                            const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                            if (lane == q) myc += __popc(bal);
-                            anyk |= keep;
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (int32_t(v[jj]) >= int32_t(mt.thr[sl * 16 + jj] ^ 0x80000000u)) k16 |= 1u << jj;
+                        K |= k16 << (16 * sl);
+                    }
+                    K &= T;
+                    if (filt) {
+                        for (uint32_t kk = K; kk; kk &= kk - 1) {
+                            const int q = __ffs(int(kk)) - 1;
+                            if (!keep_item(a, mt.qid[q], int64_t(e.x) + r)) K &= ~(1u << q);
                         }
                     }
+                    const uint32_t C = warp_transpose32(K, lane);
+                    myc += __popc(C);
+                    kw[0] = mb == 0 ? K : kw[0];
+                    kw[1] = mb == 1 ? K : kw[1];
+                    kw[2] = mb == 2 ? K : kw[2];
+                    kw[3] = mb == 3 ? K : kw[3];
+                    cw[0] = mb == 0 ? C : cw[0];
+                    cw[1] = mb == 1 ? C : cw[1];
+                    cw[2] = mb == 2 ? C : cw[2];
+                    cw[3] = mb == 3 ? C : cw[3];
                 }
                 // this warp's slots: one atomic per query, all in flight at once
-                uint32_t mybase = 0;
+                uint32_t run = 0;
                 if (lane < qn && myc) {
-                    mybase = atomicAdd(&a.cand_cnt[int64_t(mt.qid[lane]) * kCntStride], myc);
+                    run = atomicAdd(&a.cand_cnt[int64_t(mt.qid[lane]) * kCntStride], myc);
                     atomicAdd(&cnt[lane], myc);
                 }
-                // pass 2: write the same keys (ranked within the warp by
-                // ballot) and count each in its score bin
-                if (__any_sync(0xffffffffu, anyk)) {
-                    for (int mb = 0; mb < 4; ++mb) {
-                        if (!((mbm >> mb) & 1u)) continue;
-                        const int r = mb * 128 + wq * 32 + lane;
-                        const int wb = r >> 5;
-                        const uint32_t id = uint32_t(e.x + r);
-                        for (int sl = 0; sl < nsl; ++sl) {
-                            uint32_t v[16];
-                            tmem_ld16(acc_base + uint32_t(mb * kTcQMax + sl * 16), v);
-                            tmem_wait_ld();
+                // pass 2: write the kept keys; a key's slot is its query's
+                // base for the row block plus its rank among the block's kept
+                // rows of that query (both from lane q, through shared memory)
+                uint32_t* const wbase = E.wbase[wq];
+                uint32_t* const wcol = E.wcol[wq];
+#pragma unroll 1
+                for (int mb = 0; mb < 4; ++mb) {
+                    const uint32_t K = mb == 0 ? kw[0] : mb == 1 ? kw[1] : mb == 2 ? kw[2] : kw[3];
+                    const uint32_t C = mb == 0 ? cw[0] : mb == 1 ? cw[1] : mb == 2 ? cw[2] : cw[3];
+                    if (!__any_sync(0xffffffffu, K != 0u)) continue;  // then every C is 0 too
+                    __syncwarp();
+                    wbase[lane] = run;
+                    wcol[lane] = C;
+                    run += __popc(C);
+                    __syncwarp();
+                    const int r = mb * 128 + wq * 32 + lane;
+                    const uint32_t id = uint32_t(e.x + r);
+                    const uint32_t lt = lanemask_lt();
+                    for (int sl = 0; sl < nsl; ++sl) {
+                        uint32_t v[16];
+                        tmem_ld16(acc_base + uint32_t(mb * kTcQMax + sl * 16), v);
+                        tmem_wait_ld();
+                        const uint32_t k16 = K >> (16 * sl);
 #pragma unroll
-                            for (int jj = 0; jj < 16; ++jj) {
-                                const int q = sl * 16 + jj;
-                                if (q >= qn) break;  // warp-uniform
-                                const int32_t score = int32_t(v[jj]);
-                                bool keep = ((mt.pass[wb][q] >> lane) & 1u) &&
-                                            (uint32_t(score) ^ 0x80000000u) >= mt.thr[q];
-                                const int qid = mt.qid[q];
-                                if (filt && keep) keep = keep_item(a, qid, int64_t(id));
-                                const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                                if (!bal) continue;
-                                const uint32_t b0 = __shfl_sync(0xffffffffu, mybase, q);
-                                if (lane == q) mybase += __popc(bal);
-                                if (keep) {
-                                    const uint32_t pos = b0 + __popc(bal & lanemask_lt());
-                                    if (int64_t(pos) < a.cap) a.cand[int64_t(qid) * a.cap + pos] = pack_key(score, id);
-                                    count_bin(a.qhist + int64_t(qid) * kTcBins, (score - mt.qbase[q]) >> mt.qsh[q], bal);
-                                }
-                            }
+                        for (int jj = 0; jj < 16; ++jj) {
+                            if (!((k16 >> jj) & 1u)) continue;
+                            const int q = sl * 16 + jj;
+                            const int32_t score = int32_t(v[jj]);
+                            const uint32_t pos = wbase[q] + __popc(wcol[q] & lt);
+                            const int qid = mt.qid[q];
+                            if (int64_t(pos) < a.cap) a.cand[int64_t(qid) * a.cap + pos] = pack_key(score, id);
+                            atomicAdd(a.qhist + int64_t(qid) * kTcBins + ((score - mt.qbase[q]) >> mt.qsh[q]), 1u);
                         }
                     }
                 }
