@@ -38,7 +38,9 @@
 //     (staged in shared memory by cp.async); a
 //     key's slot is its rank among the unit's survivors of that query, and
 //     the key is counted in the query's score bins (kTcBins bins over the
-//     query's possible range [-S, S]), which guide the final top-k.
+//     query's possible range [-S, S]), which guide the final top-k and the
+//     dense scan's running bound (not with deletions or exclude masks: this
+//     scan writes the keys those drop, and the final top-k filters them).
 // Every unit commits exactly two cp.async groups (planes of the unit two
 // ahead, then query vectors and staged rows of the next unit), so fixed
 // wait_group depths find every copy: there is no spin loop and nothing to
@@ -160,6 +162,11 @@ scan_kernel(SearchArgs a)
     };
     int u = draw();
     if (u >= n_units) return;
+    // keys are counted in the score bins only when every written key is a
+    // result candidate: with deletions or exclude masks the final top-k
+    // filters the keys itself and does not read the bins, and the dense
+    // scan's running bound must not count keys the filter would drop
+    const bool count_keys = a.count_bins && a.dead == nullptr && a.qexclude == nullptr;
 
     // unit entry: {first row, chunk, first query slot, rows << 16 | queries};
     // lane s < queries holds query s's id and mask; for a single-query unit,
@@ -455,7 +462,7 @@ scan_kernel(SearchArgs a)
                     const int32_t score = acc0 + acc1;
                     const uint64_t pos = uint64_t(base0) + uint32_t(idx);
                     if (pos < uint64_t(a.cap)) cand[pos] = pack_key(score, uint32_t(i));
-                    if (a.count_bins) count_bin(qh, (score - sc.x) >> sc.y, __activemask());
+                    if (count_keys) count_bin(qh, (score - sc.x) >> sc.y, __activemask());
                 }
             }
         } else {
@@ -506,7 +513,7 @@ scan_kernel(SearchArgs a)
                         const uint64_t pos = uint64_t(slot0) + __popc(bal & lanemask_lt());
                         const int32_t score = acc0 + acc1;
                         if (pos < uint64_t(a.cap)) a.cand[int64_t(qg) * a.cap + int64_t(pos)] = pack_key(score, uint32_t(i));
-                        if (a.count_bins) count_bin(a.qhist + int64_t(qg) * kTcBins, (score - sc.x) >> sc.y, bal);
+                        if (count_keys) count_bin(a.qhist + int64_t(qg) * kTcBins, (score - sc.x) >> sc.y, bal);
                     }
                     if (lane == s) run += __popc(bal);
                 }

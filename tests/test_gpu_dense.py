@@ -148,3 +148,49 @@ def test_dense_scan_sweep_batch():
         assert float(cands.sum()) < 0.25 * float(elig.sum()), (float(cands.sum()), float(elig.sum()))
     finally:
         idx.close()
+
+
+def test_dense_bound_ignores_deleted_keys_of_the_warp_scan():
+    # one query (X) probes a list of 600 rows that no other query probes (the
+    # warp scan takes it) and a 1M-row list shared with eight other queries
+    # (the tensor cores take it). Every row of the small list is deleted and
+    # scores far above anything live for X; X's best live rows are the last
+    # rows of the large list, which the dense scan reaches after its first
+    # units have raised X's running bound. That bound must count only keys
+    # that can be results: the warp scan leaves deleted items to the final
+    # top-k's post-filter, so it must not count them in the score bins the
+    # dense scan reads, or X's true results are pruned.
+    rng = np.random.default_rng(141)
+    nA, nB, nC, d = 1_000_000, 600, 4096, 64
+    n = nA + nB + nC
+    items = rng.integers(-20, 21, size=(n, d)).astype(np.int8)
+    items[:nA, 0] += 40
+    items[nA - 2048:nA, 1] = 40
+    items[nA:nA + nB, 1] = 100
+    items[nA + nB:, 2] += 40
+    sigs = np.ones((n, 1), dtype=np.uint64)
+    offsets = np.array([0, nA, nA + nB, n], dtype=np.int64)
+    cent = np.zeros((3, d), dtype=np.int8)
+    cent[0, 0] = cent[1, 1] = cent[2, 2] = 100
+    q = np.zeros((9, d), dtype=np.int8)
+    q[:8, 0] = 40
+    q[:8, 2] = 40
+    q[:8, 3:] = rng.integers(-3, 4, size=(8, d - 3))
+    q[8, 0], q[8, 1] = 30, 60
+    masks = np.ones((9, 1), dtype=np.uint64)
+    deleted = np.arange(nA, nA + nB, dtype=np.int64)
+    live = sigs.copy()
+    live[deleted] = 0
+    P, k = 2, 20
+    exp = oracle.search(items, live, offsets, cent, q, masks, P, k, nthreads=oracle.max_threads())
+    assert exp[2][8].tolist() == [1, 0] and all(r == [0, 2] for r in exp[2][:8].tolist())
+    dev = lambda x, dt: torch.from_numpy(np.ascontiguousarray(x).view(dt)).cuda()
+    idx = st.Index(dev(items, np.int8), dev(sigs, np.int64), dev(offsets, np.int64), dev(cent, np.int8))
+    try:
+        idx.delete(torch.from_numpy(deleted).cuda())
+        ids, sc = idx.search(dev(q, np.int8), dev(masks, np.int64), P, k)
+        assert idx.check() == st.ST_OK
+        assert np.array_equal(sc.cpu().numpy(), exp[1]), (sc.cpu().numpy()[8][:4], exp[1][8][:4])
+        assert np.array_equal(ids.cpu().numpy(), exp[0])
+    finally:
+        idx.close()
