@@ -53,6 +53,8 @@ struct st_index {
     CUtensorMap tmap[2];             // the item rows as a 2-D tensor (TMA tiles of 32 and 128 rows, dense scan)
     bool tmap_ok = false;
     int32_t tc_min_q = st::kTcMinQDefault;  // queries per list from which its units are dense
+    uint64_t* sig_sample = nullptr;  // [n_sample][W] signatures of creation rows 0, s, 2s, ... (s = n / kSelSample)
+    int32_t n_sample = 0;
 };
 
 namespace st {
@@ -282,7 +284,7 @@ st_status grow_rows(st_index* idx, int32_t app_cap, cudaStream_t stream)
 struct ScratchLayout {
     size_t total = 0;
     size_t off_list_cnt, off_cand_cnt, off_elig, off_rng, off_sel_hist, off_sel_cursor, off_ctl, off_tc_hist, zero_bytes;
-    size_t off_units_tc, off_qscale;
+    size_t off_units_tc, off_qscale, off_qsel;
     size_t off_sel_out, off_sel_tie;
     size_t off_probe, off_probe_keys, off_list_ustart, off_qbits, off_qnbits, off_qlist, off_qmask, off_slot_bits, off_units, off_cand;
     size_t add(size_t bytes)
@@ -360,6 +362,11 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     L.off_units = L.add(size_t(max_units) * 16);
     L.off_units_tc = L.add(tc_min_q ? size_t(max_units) * 16 : 0);
     L.off_qscale = L.add(size_t(B) * 8);
+    // lists of fewer than tc_min_q queries may go dense by their queries'
+    // selectivity once the batch is large enough to fill the dense pipeline
+    // (tc_min_q = 1 already sends every list there)
+    const bool sel_route = tc_min_q > 1 && idx->n_sample > 0 && int64_t(B) * nprobe >= st::kSelMinProbes;
+    L.off_qsel = L.add(sel_route ? size_t(B) * 2 : 0);
     L.off_cand = L.add(size_t(B) * size_t(cap) * 8);
     L.off_sel_out = L.add(size_t(B) * size_t(k) * 8);
     L.off_sel_tie = L.add(size_t(B) * st::kSelTieCap * 8);
@@ -413,6 +420,11 @@ st_status search_impl(const st_index* idx, const int8_t* queries, const uint64_t
     a.max_units = int32_t(max_units);
     a.tc_min_q = tc_min_q;
     if (tc_min_q) a.units_tc = reinterpret_cast<int4*>(base + L.off_units_tc);
+    if (sel_route) {
+        a.sig_sample = idx->sig_sample;
+        a.n_sample = idx->n_sample;
+        a.qsel = reinterpret_cast<uint16_t*>(base + L.off_qsel);
+    }
     a.qscale = reinterpret_cast<int2*>(base + L.off_qscale);
     a.qhist = reinterpret_cast<uint32_t*>(base + L.off_tc_hist);
     a.count_bins = st::select_reads_bins(B, k) ? 1 : 0;
@@ -554,6 +566,19 @@ st_status st_index_create(const int8_t* items, const uint64_t* sigs, const int64
         }
         e = st::launch_build_planes(idx->sigs, idx->offsets, idx->base_chunk_start, idx->chunk_list,
                                     idx->n_base_chunks, sig_words, idx->planes, stream);
+    }
+    // a fixed sample of the rows' signatures, for each search's selectivity
+    // estimates (they choose between the two scans only; not updated when
+    // rows are inserted, updated or deleted)
+    if (e == cudaSuccess) {
+        const int64_t stride = std::max<int64_t>(1, n / st::kSelSample);
+        idx->n_sample = int32_t(std::min<int64_t>(st::kSelSample, (n + stride - 1) / stride));
+        if (cudaMalloc(&idx->sig_sample, size_t(idx->n_sample) * sig_words * 8) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(ST_ERR_OOM);
+        }
+        e = cudaMemcpy2DAsync(idx->sig_sample, size_t(sig_words) * 8, idx->sigs, size_t(stride) * sig_words * 8,
+                              size_t(sig_words) * 8, size_t(idx->n_sample), cudaMemcpyDeviceToDevice, stream);
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e == cudaSuccess) make_items_tmap(idx);
@@ -916,6 +941,7 @@ void st_index_destroy(st_index* idx)
         cudaFree(idx->planes);
         cudaFree(idx->err);
         cudaFree(idx->dead);
+        cudaFree(idx->sig_sample);
         if (idx->pool) cudaMemPoolDestroy(idx->pool);
         cudaGetLastError();
     }

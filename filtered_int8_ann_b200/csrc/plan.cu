@@ -3,8 +3,9 @@
 // however many queries probe it. One self-contained 16-byte entry per unit:
 // {first row, chunk, first query slot, rows << 16 | queries}. Lists probed by
 // fewer than tc_min_q queries get groups of up to kQMax queries, scanned by
-// one warp each (scan.cu); lists probed by more get groups of up to kTcQMax
-// queries in a second table, scanned as dense tensor-core tiles (scan_tc.cu).
+// one warp each (scan.cu); lists probed by more, or whose queries expect many
+// eligible rows (dense_by_selectivity), get groups of up to kTcQMax queries in
+// a second table, scanned as dense tensor-core tiles (scan_tc.cu).
 //
 // The probe kernel already filed each query into the slot row of every list it
 // chose (slots L*B .. L*B + count-1), so no scan over lists or scatter of pairs
@@ -33,7 +34,7 @@ units_alloc_kernel(SearchArgs a)
     if (L < a.nlist) {
         const int cnt = a.list_cnt[L];
         if (cnt > 0) {
-            dense = dense_list(a, cnt);
+            dense = dense_list(a, cnt) || dense_by_selectivity(a, L, cnt);
             const int qg = dense ? kTcQMax : kQMax;
             u = uint32_t(a.chunk_start[L + 1] - a.chunk_start[L]) * uint32_t((cnt + qg - 1) / qg);
         }
@@ -64,7 +65,9 @@ units_alloc_kernel(SearchArgs a)
     }
     bs = __shfl_sync(0xffffffffu, bs, 31);
     bd = __shfl_sync(0xffffffffu, bd, 31);
-    if (u > 0) a.list_ustart[L] = dense ? int32_t(bd + id - ud) : int32_t(bs + is - us);
+    // a dense list's first unit is stored bit-inverted, so units_write reads
+    // the choice made here instead of repeating it
+    if (u > 0) a.list_ustart[L] = dense ? ~int32_t(bd + id - ud) : int32_t(bs + is - us);
 }
 
 __global__ void __launch_bounds__(kUnitsBlock)
@@ -95,8 +98,9 @@ units_write_kernel(SearchArgs a)
         set_error(a.err, kErrUnitDecode);
         unit = make_int4(0, 0, 0, 0);
     }
-    const int64_t base = a.list_ustart[L];
-    const bool dense = dense_list(a, cnt);
+    const int32_t us = a.list_ustart[L];
+    const bool dense = us < 0;
+    const int64_t base = dense ? int64_t(~us) : int64_t(us);
     const int qg = dense ? kTcQMax : kQMax;
     int4* table = dense ? a.units_tc : a.units;
     const int groups = (cnt + qg - 1) / qg;

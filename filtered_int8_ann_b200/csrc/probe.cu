@@ -278,13 +278,43 @@ probe_select_cluster_kernel(SearchArgs a)
     // every centroid score lies in [-Sc, Sc], Sc = 128 sum_j |q_j| (int8
     // centroids), so the selection needs no pass over the keys for their range
     __shared__ int32_t s_sc;
+    __shared__ uint32_t s_hits[4];
+    // the query's expected selectivity (sample rows passing any of its masks),
+    // counted by the leader CTA's warps 1 to 4 while warp 0 sums |q|
+    const bool count_sel = a.qsel != nullptr && int(blockIdx.x) % CS == 0;
+    static_assert(kSelSample % 128 == 0 && 32 + 128 <= kProbeCBlock, "four warps hold the sample");
     if (threadIdx.x < 32) {
         int32_t sum = 0;
         for (int j = threadIdx.x; j < a.d; j += 32) sum += abs(int32_t(a.queries[int64_t(b) * a.d + j]));
         sum = __reduce_add_sync(0xffffffffu, sum);
         if (threadIdx.x == 0) s_sc = 128 * sum;
+    } else if (count_sel && threadIdx.x < 32 + 128) {
+        constexpr int kRows = kSelSample / 128;  // sample rows per thread
+        const int t = threadIdx.x - 32, W = a.W;
+        uint64_t s0[kRows], s1[kRows];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+            const int i = t + 128 * r;
+            s0[r] = i < a.n_sample ? a.sig_sample[int64_t(i) * W] : 0ull;
+            s1[r] = i < a.n_sample && W > 1 ? a.sig_sample[int64_t(i) * W + 1] : 0ull;
+        }
+        uint32_t pass = 0;  // bit r: row t + 128 r passes one of the masks
+        for (int alt = 0; alt <= a.n_or; ++alt) {
+            const uint64_t* mk = alt == 0 ? a.qmasks + int64_t(b) * W : a.or_masks + (int64_t(b) * a.n_or + alt - 1) * W;
+            const uint64_t m0 = mk[0], m1 = W > 1 ? mk[1] : 0ull;
+#pragma unroll
+            for (int r = 0; r < kRows; ++r)
+                if (t + 128 * r < a.n_sample && (s0[r] & m0) == m0 && (s1[r] & m1) == m1) pass |= 1u << r;
+        }
+        const uint32_t hits = __reduce_add_sync(0xffffffffu, uint32_t(__popc(pass)));
+        if ((threadIdx.x & 31) == 0) s_hits[(threadIdx.x >> 5) - 1] = hits;
     }
     __syncthreads();
+    if (count_sel && threadIdx.x == 0) {
+        const uint32_t h = s_hits[0] + s_hits[1] + s_hits[2] + s_hits[3];
+        a.qsel[b] = uint16_t(h);
+        atomicMax(reinterpret_cast<unsigned int*>(&a.ctl->max_qsel), h);  // lets the plan skip hopeless lists
+    }
     const int32_t sc = s_sc;
     auto none = [](uint64_t) { return true; };
     auto no_compact = []() { return 0; };

@@ -19,6 +19,8 @@ constexpr int kQMax = 16;                  // queries per work unit
 // scan in units of up to kTcQMax queries (the MMA's N).
 constexpr int kTcQMax = 32;
 constexpr int kTcMinQDefault = 8;
+constexpr int kSelSample = 512;             // index rows whose signatures estimate each query's selectivity
+constexpr int kSelMinProbes = 2048;         // (query, list) probes from which selectivity routes lists
 constexpr int kTcBins = 1024;              // per-query score bins of the written candidate keys
 constexpr int kRngThr = 12;                // score_rng word: the query's running score bound (biased)
 
@@ -74,7 +76,8 @@ __host__ __device__ __forceinline__ int64_t key_id(uint64_t key)
 struct PlanCtl {
     int32_t n_units;       // work units allocated by the plan (clamped to the table by the scan)
     int32_t n_dense;       // dense (tensor-core) units allocated by the plan
-    int32_t pad[2];
+    int32_t max_qsel;      // the batch's largest sample count of one query (selectivity routing)
+    int32_t pad;
 };
 
 struct SearchArgs {
@@ -129,6 +132,9 @@ struct SearchArgs {
     int4* units_tc;          // [max_units] dense units, same entries (up to kTcQMax queries)
     int32_t max_units;
     int32_t tc_min_q;        // queries per list from which its units are dense (0: no dense units)
+    const uint64_t* sig_sample;  // [n_sample][W] signatures of evenly spaced rows of the index
+    int32_t n_sample;
+    uint16_t* qsel;          // [B] sample rows passing each query's mask(s), or null (no selectivity routing)
     int2* qscale;            // [B] per query {lowest possible score -S, shift of kTcBins bins over
                              // [-S, S]}: S = 128 sum_j |q_j| bounds |<q, x>| for any int8 row x
     uint32_t* qhist;         // [B][kTcBins] candidate keys written by the scans per score bin (zeroed)
@@ -143,6 +149,22 @@ struct SearchArgs {
 __device__ __forceinline__ bool dense_list(const SearchArgs& a, int cnt)
 {
     return a.tc_min_q > 0 && cnt >= a.tc_min_q;
+}
+
+// A list probed by fewer queries still goes to the tensor cores when they
+// expect together at least 3/4 of an eligible (query, row) pair per row (each
+// query's expectation: the share of a fixed sample of the index's rows that
+// passes its mask). Such a list's tiles waste little, while the warp scan
+// would score and write nearly every row once per query. Only the choice of
+// scan depends on it, never the result.
+__device__ __forceinline__ bool dense_by_selectivity(const SearchArgs& a, int L, int cnt)
+{
+    if (a.qsel == nullptr || a.n_sample <= 0) return false;
+    const uint32_t need = 3u * uint32_t(a.n_sample);
+    if (4u * uint32_t(cnt) * uint32_t(a.ctl->max_qsel) < need) return false;  // not even with cnt of the best query
+    uint32_t s = 0;
+    for (int i = 0; i < cnt && 4u * s < need; ++i) s += a.qsel[a.qlist[int64_t(L) * a.B + i]];
+    return 4u * s >= need;
 }
 
 // Programmatic dependent launch: launch_dep() lets a kernel start while its

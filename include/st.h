@@ -202,10 +202,15 @@ typedef enum {
        UNSUPPORTED when the ids would reach 2^31 (with the id offset). */
     ST_OPT_INSERT_RESERVE = 4,
     /* Lists probed by at least this many queries of a batch are scanned as
-       dense tiles on the tensor cores (int8 x int8 -> int32, up to 64 queries
-       per tile) instead of per-pair dp4a; results are identical. Default 8;
-       1 sends every probed list there; 0 turns the tensor-core scan off. Only
-       d = 64 and d = 128 have the tensor-core scan. At most ST_MAX_B. */
+       dense tiles on the tensor cores (int8 x int8 -> int32, up to 32 queries
+       per tile) instead of per-pair dp4a; results are identical. With a value
+       above 1, a list probed by fewer queries goes there too when the batch
+       has at least 2048 (query, list) probes and its queries expect together
+       at least 0.75 eligible pairs per row (each query's share of a fixed
+       sample of 512 of the index's rows, taken at creation, that passes its
+       masks). Default 8; 1 sends every probed list there; 0 turns the
+       tensor-core scan off. Only d = 64 and d = 128 have the tensor-core
+       scan. At most ST_MAX_B. */
     ST_OPT_DENSE_MIN_QUERIES = 5
 } st_option;
 
