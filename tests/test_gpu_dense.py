@@ -194,3 +194,23 @@ def test_dense_bound_ignores_deleted_keys_of_the_warp_scan():
         assert np.array_equal(ids.cpu().numpy(), exp[0])
     finally:
         idx.close()
+
+
+def test_selectivity_routes_small_lists_to_the_tensor_cores():
+    # 512 lists of ~3.9k rows, 64 queries x 32 probes (2048 probes): lists
+    # are probed by ~4 queries, below the default threshold of 8, but one-flag
+    # masks pass ~90 % of the rows, so the queries' sampled selectivities send
+    # their lists to the tensor cores. The warp scan writes every eligible key,
+    # the dense scan only keys that can still reach the top-k: fewer candidates
+    # than eligible items show which scan ran. Results equal the oracle's.
+    data = small(n=2_000_000, d=128, nlist=512, sig_bits=128, hash_bits=3, B=64, nprobe=32, k=100, seed=151,
+                 mask_flags=1, mask_lang=False)
+    exp = run_oracle(data, 32, 100)
+    got, cands = _run(data, 32, 100, None)
+    assert_parity(got, exp, "selectivity-routed")
+    per_list = np.bincount(got[2].ravel(), minlength=512)
+    assert np.median(per_list[per_list > 0]) < 8, per_list
+    assert cands.sum() < 0.5 * got[3].sum(), (cands.sum(), got[3].sum())
+    got0, cands0 = _run(data, 32, 100, 0)  # tensor cores off: every eligible key written
+    assert_parity(got0, exp, "warp scan only")
+    assert np.array_equal(cands0, got0[3])
