@@ -14,22 +14,23 @@
 //   * two producer warps, on different SM sub-partitions, taking alternate
 //     units: the unit's query slots (three of the warp's units ahead), its
 //     signature bit-planes (the union of its queries' mask bits, by cp.async,
-//     two of its units ahead, into the warp's own two plane buffers), the
-//     Bloom test (pass words [32-row block][query]), then the rows: a 32-row
-//     block with many survivors (for any of the unit's queries) is copied
-//     whole by a TMA tile load (a 128-row tile when four neighbouring blocks
-//     are), a block with few has only its survivors' rows gathered by
-//     cp.async, a block without survivors is not read; both land in the
-//     canonical 128-byte (d = 128) or 64-byte (d = 64) swizzled K-major layout
-//     of an operand stage, with the unit's query vectors;
+//     two of its units ahead, into the unit's slot of the unit ring, where they
+//     stay until its epilogue is done), then its rows, as whole 128-row TMA
+//     tiles in the canonical 128-byte (d = 128) or 64-byte (d = 64) swizzled
+//     K-major layout of an operand stage, and the unit's query vectors. The
+//     lists here have many queries or many eligible rows, so nearly every row
+//     block holds a survivor of some query: testing first to skip row blocks
+//     cost the producers more than the reads it saved;
 //   * MMA warp: one thread issues tcgen05.mma kind::i8 (M = 128 rows, N = the
 //     unit's queries rounded up to 16, K = 32) into int32 accumulators in TMEM
 //     and commits to mbarriers that free the operand stage and hand the
 //     accumulators to an epilogue;
 //   * four epilogue warpgroups, one per TMEM accumulator stage (every fourth
-//     unit each): each thread reads its row's scores (tcgen05.ld) and keeps a
-//     key only if the row passes the query's Bloom test and its score reaches
-//     the query's running bound (below), as one bit per query; a 32 x 32 bit
+//     unit each): lane q of each warp runs the Bloom test of query q on the
+//     warp's four 32-row blocks (the AND of the unit's planes of its mask
+//     bits); each thread reads its row's scores (tcgen05.ld) and keeps a key
+//     only if the row passes the query's test and its score reaches the
+//     query's running bound (below), as one bit per query; a 32 x 32 bit
 //     transpose across the warp turns the pass words into these per-row words
 //     and the kept words into per-query row masks, whose popcounts are the
 //     warp's key counts. Each warp reserves its slots with one atomic per query
@@ -43,14 +44,15 @@
 // keys that can no longer enter a query's top-k are not written at all. Every
 // written key is a real candidate, so if at least k written keys have scores
 // >= T, the query's k-th best score is >= T and any key below T can be
-// dropped. Every written key (of either scan) is counted in the query's 1024
+// dropped. Every written key is counted in the query's 1024
 // bins over its possible score range [-S, S], S = 128 sum_j |q_j| (bin b
 // holds scores in [-S + b 2^sh, -S + (b+1) 2^sh)); when a unit wrote at least
 // kTcBoundMinKeys keys of a query, the bins from the query's bound upward give
 // the highest bin edge with k written keys at or above it, published with
 // atomicMax. The bound only grows and the final top-k is unchanged (exact).
-// With deletions or exclude masks the post-filter is applied before a key is
-// counted, so every counted key is still a result candidate.
+// With deletions or exclude masks this scan applies the post-filter before it
+// counts a key, and the warp scan (which writes its keys unfiltered for the
+// final top-k to filter) counts none, so every counted key is a candidate.
 //
 // Waits are bounded: a wait that runs out sets an error bit and an abort flag;
 // every role then leaves its loop (its own waits are bounded too), and the CTA
@@ -60,11 +62,7 @@
 namespace st {
 
 constexpr int kTcRows = kWarpItems;      // rows per unit
-constexpr int kTcPlaneSlots = 48;        // planes one buffer holds
-#ifndef ST_TC_DENSE_BLK
-#define ST_TC_DENSE_BLK 24
-#endif
-constexpr int kTcDenseBlk = ST_TC_DENSE_BLK;  // survivors of a 32-row block from which the whole block is loaded
+constexpr int kTcPlaneSlots = 24;        // planes a unit's ring slot holds (a wider union reads global planes)
 constexpr uint32_t kTcWaitLimit = 1u << 22;
 // Units whose data are held at once. A producer refills the slot of unit
 // j - 8 (with unit j + 4) only after the MMAs of unit j - S (operand stages
@@ -89,16 +87,15 @@ __host__ __device__ constexpr int tc_stages()
 
 struct TcMeta {                          // one unit, from its slots to its epilogue
     int4 e;                              // {first row, plane block, first slot, rows << 16 | queries}
+    uint32_t planes[kTcPlaneSlots][16];  // the signature bit-planes of the union of its queries' masks
     int32_t qid[kTcQMax];
     unsigned long long qm[kTcQMax][2];   // the queries' masks
     uint32_t thr[kTcQMax];               // the queries' running bounds when the unit was loaded
     int32_t qbase[kTcQMax], qsh[kTcQMax];  // score bins: lowest possible score, bin shift
-    uint32_t pass[16][kTcQMax];          // [32-row block][query] Bloom pass words
     uint8_t tab[kMaskBitsMax];           // signature bit -> plane slot
     uint8_t inv[kTcPlaneSlots];          // plane slot -> signature bit
     int32_t held;                        // planes in the buffer (-1: the test reads global planes)
-    uint32_t uni[16];                    // OR over the queries of the pass words
-    uint32_t mbmask;                     // 128-row blocks with survivors (MMAs issued for them)
+    uint32_t mbmask;                     // 128-row blocks holding rows of the unit (MMAs issued for them)
 };
 
 struct TcEpi {                           // one epilogue warpgroup's per-query key counts (two units)
@@ -150,8 +147,7 @@ template <int D>
 struct TcLayout {
     static constexpr size_t kA = 0;
     static constexpr size_t kB = kA + size_t(tc_stages<D>()) * kTcRows * D;
-    static constexpr size_t kP = kB + size_t(tc_stages<D>()) * kTcQMax * D;
-    static constexpr size_t kMeta = kP + size_t(2 * kTcProducers) * kTcPlaneSlots * 64;
+    static constexpr size_t kMeta = kB + size_t(tc_stages<D>()) * kTcQMax * D;
     static constexpr size_t kEpi = kMeta + size_t(kTcMeta) * sizeof(TcMeta);
     static constexpr size_t kEnd = kEpi + size_t(kTcEpiGroups) * sizeof(TcEpi);
     static_assert(kMeta % alignof(TcMeta) == 0 && kEpi % alignof(TcEpi) == 0, "aligned carve-up");
@@ -186,7 +182,6 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
     using L = TcLayout<D>;
     unsigned char* const Abuf = base + L::kA;                                 // [S][kTcRows * D]
     unsigned char* const Bbuf = base + L::kB;                                 // [S][kTcQMax * D]
-    uint32_t* const Pbuf = reinterpret_cast<uint32_t*>(base + L::kP);  // [2 * kTcProducers][kTcPlaneSlots][16]
     TcMeta* const meta = reinterpret_cast<TcMeta*>(base + L::kMeta);          // [kTcMeta]
     TcEpi* const epi = reinterpret_cast<TcEpi*>(base + L::kEpi);              // [kTcEpiGroups]
 
@@ -259,8 +254,8 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
                 r.sc = a.qscale[r.qid];
             }
         };
-        // slots -> meta[m]; the union's planes -> plane buffer p
-        auto store_and_request = [&](int m, int p, const Slots& r) {
+        // slots -> meta[m]; the union's planes -> meta[m].planes
+        auto store_and_request = [&](int m, const Slots& r) {
             const int qn = r.e.w & 0xFFFF;
             TcMeta& mt = meta[m];
             if (lane == 0) mt.e = r.e;
@@ -297,101 +292,10 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
                 if (on) mt.inv[slot] = uint8_t(b);
             }
             __syncwarp();
-            uint32_t* dst = Pbuf + p * kTcPlaneSlots * 16;
+            uint32_t* dst = &mt.planes[0][0];
             const uint32_t* src = a.planes + int64_t(r.e.y) * NPL * 16;
             for (int item = lane; item < 4 * nb; item += 32)
                 cp_async16_cg(dst + item * 4, src + mt.inv[item >> 2] * 16 + (item & 3) * 4);
-        };
-        // Bloom test of meta[m] with plane buffer p: lane q takes query q and
-        // ANDs, for each of its mask bits, the 16 words (512 rows) of that
-        // bit's plane into its 16 pass words
-        auto test_unit = [&](int m, int p) {
-            TcMeta& mt = meta[m];
-            const int4 e = mt.e;
-            const int qn = e.w & 0xFFFF, len = e.w >> 16;
-            const int held = mt.held;
-            uint32_t acc[16];
-#pragma unroll
-            for (int w = 0; w < 16; ++w)
-                acc[w] = len >= 32 * (w + 1) ? 0xFFFFFFFFu : (len <= 32 * w ? 0u : ((1u << (len - 32 * w)) - 1u));
-            if (lane < qn && a.n_or > 0) {
-                // alternative masks: for each 16-byte chunk of the pass words,
-                // the OR over the query's masks of each one's AND (the slot's
-                // mask, the union, chose the planes)
-                const uint4* pl = reinterpret_cast<const uint4*>(Pbuf + p * kTcPlaneSlots * 16);
-                const uint4* gpl = reinterpret_cast<const uint4*>(a.planes + int64_t(e.y) * NPL * 16);
-                const int qid = mt.qid[lane], n_alt = 1 + a.n_or;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint4 o = make_uint4(0u, 0u, 0u, 0u);
-                    for (int alt = 0; alt < n_alt; ++alt) {
-                        const uint64_t* mk = alt == 0 ? a.qmasks + int64_t(qid) * W
-                                                      : a.or_masks + (int64_t(qid) * a.n_or + alt - 1) * W;
-                        uint4 v = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-                        for (int word = 0; word < W; ++word) {
-                            unsigned long long m = __ldg(mk + word);
-                            while (m) {
-                                const int b = 64 * word + __ffsll(static_cast<long long>(m)) - 1;
-                                m &= m - 1;
-                                const uint4 x = held >= 0 ? pl[mt.tab[b] * 4 + c] : __ldg(gpl + b * 4 + c);
-                                v.x &= x.x;
-                                v.y &= x.y;
-                                v.z &= x.z;
-                                v.w &= x.w;
-                            }
-                        }
-                        o.x |= v.x;
-                        o.y |= v.y;
-                        o.z |= v.z;
-                        o.w |= v.w;
-                    }
-                    // (a dynamic chunk index would put acc[] in local memory)
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-                        if (cc == c) {
-                            acc[4 * cc] &= o.x;
-                            acc[4 * cc + 1] &= o.y;
-                            acc[4 * cc + 2] &= o.z;
-                            acc[4 * cc + 3] &= o.w;
-                        }
-                }
-            } else if (lane < qn) {
-                const uint4* pl = reinterpret_cast<const uint4*>(Pbuf + p * kTcPlaneSlots * 16);
-                const uint4* gpl = reinterpret_cast<const uint4*>(a.planes + int64_t(e.y) * NPL * 16);
-#pragma unroll
-                for (int word = 0; word < W; ++word) {
-                    unsigned long long mk = mt.qm[lane][word];
-                    while (mk) {
-                        const int b = 64 * word + __ffsll(static_cast<long long>(mk)) - 1;
-                        mk &= mk - 1;
-                        const uint4* src = held >= 0 ? pl + mt.tab[b] * 4 : gpl + b * 4;
-                        uint4 v[4];
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) v[c] = held >= 0 ? src[c] : __ldg(src + c);
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            acc[4 * c] &= v[c].x;
-                            acc[4 * c + 1] &= v[c].y;
-                            acc[4 * c + 2] &= v[c].z;
-                            acc[4 * c + 3] &= v[c].w;
-                        }
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int w = 0; w < 16; ++w) acc[w] = 0;
-            }
-            uint32_t c = 0;
-#pragma unroll
-            for (int w = 0; w < 16; ++w) {
-                if (lane < qn) mt.pass[w][lane] = acc[w];
-                c += __popc(acc[w]);
-                const uint32_t u = __reduce_or_sync(0xffffffffu, acc[w]);
-                if (lane == 0) mt.uni[w] = u;
-            }
-            if (lane < qn && c)
-                atomicAdd(&a.eligible_cnt[int64_t(mt.qid[lane]) * (kCntStride / 2)], (unsigned long long)c);
-            __syncwarp();
         };
         // rows and query vectors of meta[m] -> operand stage s
         auto issue_rows = [&](int m, int s) {
@@ -400,35 +304,15 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             const int qn = e.w & 0xFFFF;
             unsigned char* A = Abuf + s * kTcRows * D;
             unsigned char* Bq = Bbuf + s * kTcQMax * D;
-            uint32_t mb = 0, dmask = 0, bytes = 0;
-#pragma unroll
-            for (int b = 0; b < 16; ++b) {
-                const int pc = __popc(mt.uni[b]);
-                if (pc) mb |= 1u << (b >> 2);
-                if (pc >= kTcDenseBlk) {
-                    dmask |= 1u << b;
-                    bytes += 32 * D;
-                }
-            }
+            // every 128-row tile holding rows of the unit, by TMA (rows past
+            // the end of the index read as zeros; rows past the unit's pass
+            // no Bloom test in the epilogue)
+            const int nblk = ((e.w >> 16) + 127) >> 7;
+            const uint32_t mb = nblk > 0 ? (1u << nblk) - 1u : 0u;
             if (lane == 0) {
                 mt.mbmask = mb;
-                mbar_arrive_expect_tx(&full_bar[s], bytes);
-                for (int r4 = 0; r4 < 4; ++r4) {
-                    const uint32_t quad = (dmask >> (4 * r4)) & 0xFu;
-                    if (quad == 0xFu) {  // the whole 128-row block in one tile
-                        tma_load_2d(A + r4 * 128 * D, &tmap128, 0, e.x + 128 * r4, &full_bar[s]);
-                        continue;
-                    }
-                    for (int b = 4 * r4; b < 4 * r4 + 4; ++b)
-                        if ((dmask >> b) & 1u) tma_load_2d(A + b * 32 * D, &tmap, 0, e.x + 32 * b, &full_bar[s]);
-                }
-            }
-            for (int b = 0; b < 16; ++b) {  // the survivors of the other blocks, one lane per row
-                if (((dmask >> b) & 1u) || !((mt.uni[b] >> lane) & 1u)) continue;
-                const int r = 32 * b + lane;
-                const int8_t* src = a.items + (int64_t(e.x) + r) * D;
-#pragma unroll
-                for (int c = 0; c < CH; ++c) cp_async16_cg(A + swz<D>(r, c), src + 16 * c);
+                mbar_arrive_expect_tx(&full_bar[s], uint32_t(nblk) * 128u * D);
+                for (int r4 = 0; r4 < nblk; ++r4) tma_load_2d(A + r4 * 128 * D, &tmap128, 0, e.x + 128 * r4, &full_bar[s]);
             }
             for (int item = lane; item < qn * CH; item += 32) {
                 const int q = item / CH, c = item - q * CH;
@@ -448,13 +332,13 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
         if (pid < n_iter) {
             Slots r0 = load_slots(pid);
             finish_slots(r0);
-            store_and_request(pid % kTcMeta, 2 * pid, r0);
+            store_and_request(pid % kTcMeta, r0);
         }
         cp_async_commit();
         if (pid + P2 < n_iter) {
             Slots r1 = load_slots(pid + P2);
             finish_slots(r1);
-            store_and_request((pid + P2) % kTcMeta, 2 * pid + 1, r1);
+            store_and_request((pid + P2) % kTcMeta, r1);
         }
         cp_async_commit();
         cp_async_commit();
@@ -464,8 +348,8 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             finish_slots(nxt);
         }
         int last = -1;  // this producer's latest unit
-        for (int j = pid, it = 0; j < n_iter; j += P2, ++it) {
-            const int s = j % S, m = j % kTcMeta, p = 2 * pid + (it & 1);
+        for (int j = pid; j < n_iter; j += P2) {
+            const int s = j % S, m = j % kTcMeta;
             TC_T0(t0);
             // the queries' current bounds (they only grow; the ones loaded with
             // the slots are several units old), stored before the epilogue gets
@@ -473,11 +357,11 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             uint32_t thr_now = 0;
             const int qn_j = meta[m].e.w & 0xFFFF;
             if (lane < qn_j) thr_now = __ldcg(a.score_rng + int64_t(meta[m].qid[lane]) * kCntStride + kRngThr);
-            cp_async_wait_group<1>();  // planes of unit j, rows of the previous unit
+            // unit j's planes (its epilogue reads them) and the previous unit's rows
+            cp_async_wait_group<1>();
             __syncwarp();
             if (last >= 0) gathers_done(last % S);
             TC_T0(t1);
-            test_unit(m, p);
             TC_T0(t2);
             TC_T0(t3);
             if (j >= S && !wait(&empty_bar[s], uint32_t(j / S - 1) & 1u)) break;
@@ -486,10 +370,10 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             cp_async_commit();
             if (lane < qn_j && thr_now > meta[m].thr[lane]) meta[m].thr[lane] = thr_now;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&meta_full[m]);  // slots, pass words, bounds and row blocks of unit j
+            if (lane == 0) mbar_arrive(&meta_full[m]);  // slots, planes, bounds and row blocks of unit j
             last = j;
             TC_T0(t5);
-            if (j + 2 * P2 < n_iter) store_and_request((j + 2 * P2) % kTcMeta, p, nxt);
+            if (j + 2 * P2 < n_iter) store_and_request((j + 2 * P2) % kTcMeta, nxt);
             cp_async_commit();
             TC_T0(t6);
             if (j + 3 * P2 < n_iter) {
@@ -560,6 +444,57 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             const int qn = e.w & 0xFFFF;
             if (mbm) {
                 const int nsl = (qn + 15) >> 4;
+                // the Bloom test of this warp's four 32-row blocks (4 mb + wq)
+                // for query `lane`: the AND over its mask's bits of the unit's
+                // planes (for alternative masks, the OR over them of each one's
+                // AND), limited to the unit's rows
+                uint32_t pw0 = 0, pw1 = 0, pw2 = 0, pw3 = 0;
+                if (lane < qn) {
+                    const int len = e.w >> 16, held = mt.held;
+                    const uint32_t* gpl = a.planes + int64_t(e.y) * NPL * 16;
+                    auto plane_word = [&](int b, int wb) -> uint32_t {
+                        return held >= 0 ? mt.planes[mt.tab[b]][wb] : __ldg(gpl + b * 16 + wb);
+                    };
+                    auto and_mask = [&](uint64_t m0, uint64_t m1, uint32_t& v0, uint32_t& v1, uint32_t& v2, uint32_t& v3) {
+                        v0 = v1 = v2 = v3 = 0xFFFFFFFFu;
+                        for (int word = 0; word < W; ++word) {
+                            unsigned long long mk = word == 0 ? m0 : m1;
+                            while (mk) {
+                                const int b = 64 * word + __ffsll(static_cast<long long>(mk)) - 1;
+                                mk &= mk - 1;
+                                v0 &= plane_word(b, wq);
+                                v1 &= plane_word(b, 4 + wq);
+                                v2 &= plane_word(b, 8 + wq);
+                                v3 &= plane_word(b, 12 + wq);
+                            }
+                        }
+                    };
+                    if (a.n_or == 0) {
+                        and_mask(mt.qm[lane][0], mt.qm[lane][1], pw0, pw1, pw2, pw3);
+                    } else {
+                        const int qid = mt.qid[lane];
+                        for (int alt = 0; alt <= a.n_or; ++alt) {
+                            const uint64_t* mk = alt == 0 ? a.qmasks + int64_t(qid) * W
+                                                          : a.or_masks + (int64_t(qid) * a.n_or + alt - 1) * W;
+                            uint32_t v0, v1, v2, v3;
+                            and_mask(__ldg(mk), W > 1 ? __ldg(mk + 1) : 0ull, v0, v1, v2, v3);
+                            pw0 |= v0;
+                            pw1 |= v1;
+                            pw2 |= v2;
+                            pw3 |= v3;
+                        }
+                    }
+                    auto rows_of = [&](int wb) -> uint32_t {
+                        const int r0 = 32 * wb;
+                        return len >= r0 + 32 ? 0xFFFFFFFFu : (len <= r0 ? 0u : ((1u << (len - r0)) - 1u));
+                    };
+                    pw0 &= rows_of(wq);
+                    pw1 &= rows_of(4 + wq);
+                    pw2 &= rows_of(8 + wq);
+                    pw3 &= rows_of(12 + wq);
+                    const uint32_t ne = __popc(pw0) + __popc(pw1) + __popc(pw2) + __popc(pw3);
+                    if (ne) atomicAdd(&a.eligible_cnt[int64_t(mt.qid[lane]) * (kCntStride / 2)], (unsigned long long)ne);
+                }
                 // pass 1: this thread's kept pairs of each row block as a word
                 // over the queries (bit q: the row passes query q's Bloom test
                 // and its score reaches q's bound), and, transposed, lane q's
@@ -570,8 +505,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
                 for (int mb = 0; mb < 4; ++mb) {
                     if (!((mbm >> mb) & 1u)) continue;  // warp-uniform
                     const int r = mb * 128 + wq * 32 + lane;
-                    const int wb = r >> 5;
-                    const uint32_t T = warp_transpose32(lane < qn ? mt.pass[wb][lane] : 0u, lane);
+                    const uint32_t T = warp_transpose32(mb == 0 ? pw0 : mb == 1 ? pw1 : mb == 2 ? pw2 : pw3, lane);
                     uint32_t K = 0;
                     for (int sl = 0; sl < nsl; ++sl) {
                         uint32_t v[16];

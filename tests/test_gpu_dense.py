@@ -3,10 +3,10 @@ every probed list sent to the tensor cores (ST_OPT_DENSE_MIN_QUERIES = 1),
 with none sent there (0) and at the default threshold, and each run must equal
 the CPU oracle bit for bit (ids, int32 scores, probed lists, eligible counts).
 The cases cover d = 64 and 128, 64- and 128-bit signatures, survivor densities
-from a few per cent (rows gathered one by one) to nearly all rows (whole
-32-row blocks by TMA), more than 64 queries on one list (several dense units
-per chunk), ragged list tails, small k (the running top-k bound prunes most
-keys) and k above the eligible count (nothing can be pruned)."""
+from a few per cent to nearly all rows, unions of mask bits wider than a unit's
+plane slots (global planes), more than 32 queries on one list (several dense
+units per chunk), ragged list tails, small k (the running top-k bound prunes
+most keys) and k above the eligible count (nothing can be pruned)."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +19,7 @@ from workloads import WORKLOADS, generate, small, to_numpy
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # nearly every row eligible, many queries per list: whole blocks by TMA
+    # nearly every row eligible, many queries per list
     dict(n=6000, d=128, nlist=4, sig_bits=128, hash_bits=3, B=40, nprobe=3, k=50, seed=101,
          mask_flags=1, mask_lang=False),
     dict(n=6000, d=64, nlist=4, sig_bits=128, hash_bits=3, B=40, nprobe=3, k=50, seed=102,
@@ -28,13 +28,13 @@ CASES = [
          mask_flags=0, mask_lang=False),
     dict(n=5000, d=64, nlist=5, sig_bits=64, hash_bits=2, B=24, nprobe=4, k=7, seed=104,
          mask_flags=0, mask_lang=False),
-    # a few per cent eligible: survivors gathered row by row
+    # a few per cent eligible
     dict(n=9000, d=128, nlist=3, sig_bits=128, hash_bits=3, B=33, nprobe=2, k=100, seed=105, mask_flags=3),
     dict(n=9000, d=64, nlist=3, sig_bits=128, hash_bits=3, B=33, nprobe=2, k=100, seed=106, mask_flags=3),
     # item-mode masks: the unit's mask union exceeds the plane buffer (global planes)
     dict(n=8000, d=64, nlist=3, sig_bits=128, hash_bits=3, B=60, nprobe=3, k=150, seed=107,
          mask_mode="item", mask_country=True, mask_flags=2),
-    # more than 64 queries per list: several dense units per chunk
+    # more than 32 queries per list: several dense units per chunk
     dict(n=7000, d=128, nlist=2, sig_bits=128, hash_bits=3, B=150, nprobe=2, k=64, seed=108,
          mask_flags=1, mask_lang=False),
     dict(n=7000, d=64, nlist=3, sig_bits=64, hash_bits=2, B=130, nprobe=2, k=300, seed=109, mask_flags=2),
