@@ -187,7 +187,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full_bar[i], 2);   // the TMA byte count's arrival + the gathers' arrival
+            mbar_init(&full_bar[i], 2);   // the TMA byte count's arrival + the query vectors' arrival
             mbar_init(&empty_bar[i], 1);  // the MMAs reading the stage are done
         }
         for (int i = 0; i < kTcEpiGroups; ++i) {
@@ -319,8 +319,9 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
                 cp_async16(Bq + swz<D>(q, c), a.queries + int64_t(mt.qid[q]) * D + 16 * c);
             }
         };
-        // the gathers of the unit using stage s have landed: make them visible
-        // to the tensor cores and count the stage's second arrival
+        // the query vectors (cp.async) of the unit using stage s have landed:
+        // make them visible to the tensor cores and count the stage's second
+        // arrival
         auto gathers_done = [&](int s) {
             fence_proxy_async_smem();
             __syncwarp();
