@@ -429,7 +429,7 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
         const bool filt = a.dead != nullptr || a.qexclude != nullptr;
         const uint32_t acc_base = tmem + (uint32_t(wq * 32) << 16) + uint32_t(g * kTcAccCols);
         // keys a query must gain in one unit before its bound is re-read
-        const uint32_t bound_min = uint32_t(a.k / 16) > kTcBoundMinKeys ? uint32_t(a.k / 16) : kTcBoundMinKeys;
+        const uint32_t bound_min = uint32_t(a.k / 8) > kTcBoundMinKeys ? uint32_t(a.k / 8) : kTcBoundMinKeys;
         for (int j = g, it = 0; j < n_iter; j += kTcEpiGroups, ++it) {
             const int m = j % kTcMeta;
             uint32_t* cnt = E.cnt[it & 1];
