@@ -47,7 +47,7 @@
 // dropped. Every written key is counted in the query's 1024
 // bins over its possible score range [-S, S], S = 128 sum_j |q_j| (bin b
 // holds scores in [-S + b 2^sh, -S + (b+1) 2^sh)); when a unit wrote at least
-// kTcBoundMinKeys keys of a query, the bins from the query's bound upward give
+// max(kTcBoundMinKeys, k / 8) keys of a query, the bins from its bound upward give
 // the highest bin edge with k written keys at or above it, published with
 // atomicMax. The bound only grows and the final top-k is unchanged (exact).
 // With deletions or exclude masks this scan applies the post-filter before it
@@ -69,7 +69,7 @@ constexpr uint32_t kTcWaitLimit = 1u << 22;
 // S = 2 or 4) are done; those of unit j - 4 then are too, and they waited for
 // the epilogue of unit j - 8 (epilogue groups 4) to free its accumulators.
 constexpr int kTcMeta = 12;
-constexpr uint32_t kTcBoundMinKeys = 16; // keys of a query in one unit that make it re-read its bound
+constexpr uint32_t kTcBoundMinKeys = 16; // least keys of a query in one unit that make it re-read its bound (else k / 8)
 constexpr int kTcEpiGroups = 4;         // epilogue warpgroups, one per TMEM accumulator stage
 constexpr int kTcProducers = 2;         // producer warps (units alternate between them)
 constexpr int kTcProd1Warp = 2 + 4 * kTcEpiGroups;  // the second producer: the last warp
