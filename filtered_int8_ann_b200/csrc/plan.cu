@@ -26,9 +26,11 @@ constexpr int kUnitsBlock = 256;
 __global__ void __launch_bounds__(kUnitsBlock)
 units_alloc_kernel(SearchArgs a)
 {
-    dep_enter();
     const int lane = threadIdx.x & 31;
     const int L = blockIdx.x * kUnitsBlock + threadIdx.x;
+    // the index's chunk table is read before waiting for the probe
+    const int nch = L < a.nlist ? a.chunk_start[L + 1] - a.chunk_start[L] : 0;
+    dep_enter();
     uint32_t u = 0;
     bool dense = false;
     if (L < a.nlist) {
@@ -36,7 +38,7 @@ units_alloc_kernel(SearchArgs a)
         if (cnt > 0) {
             dense = dense_list(a, cnt) || dense_by_selectivity(a, L, cnt);
             const int qg = dense ? kTcQMax : kQMax;
-            u = uint32_t(a.chunk_start[L + 1] - a.chunk_start[L]) * uint32_t((cnt + qg - 1) / qg);
+            u = uint32_t(nch) * uint32_t((cnt + qg - 1) / qg);
         }
     }
     // one warp-wide scan per table (sparse, dense)
@@ -73,10 +75,19 @@ units_alloc_kernel(SearchArgs a)
 __global__ void __launch_bounds__(kUnitsBlock)
 units_write_kernel(SearchArgs a)
 {
-    dep_enter();
     const int t = blockIdx.x * kUnitsBlock + threadIdx.x;  // chunk table entry
+    // the index's chunk table is read before waiting for the unit blocks
+    int4 c = make_int4(0, 0, 0, -1);  // {first row, plane block, rows, list}
+    int c0 = 0, nch = 0;
+    if (t < a.n_chunks) {
+        c = a.chunk_desc[t];
+        if (c.w >= 0 && c.w < a.nlist) {
+            c0 = a.chunk_start[c.w];
+            nch = a.chunk_start[c.w + 1] - c0;
+        }
+    }
+    dep_enter();
     if (t >= a.n_chunks) return;
-    const int4 c = a.chunk_desc[t];  // {first row, plane block, rows, list}
     const int L = c.w;
     if (L < 0 || L >= a.nlist) {
         set_error(a.err, kErrUnitDecode);
@@ -84,8 +95,6 @@ units_write_kernel(SearchArgs a)
     }
     const int cnt = a.list_cnt[L];
     if (cnt <= 0) return;
-    const int c0 = a.chunk_start[L];
-    const int nch = a.chunk_start[L + 1] - c0;
     const int ci = t - c0;
     if (ci < 0 || ci >= nch) {  // the list's block of units does not cover this entry
         set_error(a.err, kErrUnitDecode);

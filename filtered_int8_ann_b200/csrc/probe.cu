@@ -226,6 +226,8 @@ constexpr int kScoreBlock = kTileC * (kTileQ / kQPer);
 __global__ void __launch_bounds__(kScoreBlock)
 probe_score_kernel(SearchArgs a)
 {
+    // the selection kernel may start its query-only prologue meanwhile
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     int4* sq = reinterpret_cast<int4*>(smem_raw);  // [kTileQ][np]
     const int d = a.d, np = d >> 4, nlist = a.nlist;
@@ -263,7 +265,6 @@ template <int CS>
 __global__ void __launch_bounds__(kProbeCBlock)
 probe_select_cluster_kernel(SearchArgs a)
 {
-    dep_enter();
     cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
     const int b = int(blockIdx.x) / CS;
     const int P = a.P;
@@ -315,6 +316,10 @@ probe_select_cluster_kernel(SearchArgs a)
         a.qsel[b] = uint16_t(h);
         atomicMax(reinterpret_cast<unsigned int*>(&a.ctl->max_qsel), h);  // lets the plan skip hopeless lists
     }
+    // everything above reads the query, its masks and the index only (and
+    // writes scratch the search's memset cleared before the scoring kernel
+    // started), so it ran while the scoring kernel was still working
+    dep_enter();
     const int32_t sc = s_sc;
     auto none = [](uint64_t) { return true; };
     auto no_compact = []() { return 0; };
