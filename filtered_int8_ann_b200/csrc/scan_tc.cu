@@ -443,6 +443,9 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
             const uint32_t mbm = mt.mbmask;
             const int4 e = mt.e;
             const int qn = e.w & 0xFFFF;
+            int bq_id = 0, bq_base = 0, bq_sh = 0;  // this lane's query for the bound update
+            uint32_t bq_thr = 0;
+            bool bq_go = false;
             if (mbm) {
                 const int nsl = (qn + 15) >> 4;
                 // the Bloom test of this warp's four 32-row blocks (4 mb + wq)
@@ -578,51 +581,65 @@ scan_tc_kernel(SearchArgs a, const __grid_constant__ CUtensorMap tmap, const __g
                     }
                 }
                 named_barrier(1 + g, 128);  // the unit's key counts are complete
-                // raise the bound of each query that gained at least
-                // bound_min keys here: the highest bin edge with at least k
-                // written keys at or above it, from the query's bins at or
-                // above its bound's bin (lane l reads bins 32 l .. 32 l + 31;
-                // the warp takes queries wq, wq + 4, ...)
-                constexpr int kPer = kTcBins / 32;
-                for (int q = wq; q < qn; q += 4) {
-                    if (cnt[q] < bound_min) continue;  // warp-uniform
-                    const uint4* gh = reinterpret_cast<const uint4*>(a.qhist + int64_t(mt.qid[q]) * kTcBins) + lane * (kPer / 4);
-                    const int tb = mt.thr[q] ? ((int32_t(mt.thr[q] ^ 0x80000000u) - mt.qbase[q]) >> mt.qsh[q]) : 0;
-                    uint32_t gv[kPer], tot = 0;
-                    const bool mine = kPer * lane + kPer - 1 >= tb;
-#pragma unroll
-                    for (int i = 0; i < kPer / 4; ++i) {
-                        const uint4 x = mine ? __ldcg(gh + i) : make_uint4(0, 0, 0, 0);
-                        gv[4 * i] = x.x;
-                        gv[4 * i + 1] = x.y;
-                        gv[4 * i + 2] = x.z;
-                        gv[4 * i + 3] = x.w;
-                    }
-#pragma unroll
-                    for (int i = 0; i < kPer; ++i) tot += gv[i];
-                    uint32_t incl = tot;  // suffix sum over lanes >= this one
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
-                        if (lane + off < 32) incl += o;
-                    }
-                    uint32_t run = incl - tot, best = 0;  // keys in bins above this lane's
-#pragma unroll
-                    for (int i = kPer - 1; i >= 0; --i) {
-                        run += gv[i];
-                        if (best == 0 && run >= uint32_t(a.k)) best = uint32_t(kPer * lane + i);
-                    }
-                    best = __reduce_max_sync(0xffffffffu, best);
-                    if (lane == 0 && best > 0) {
-                        const int32_t T = mt.qbase[q] + int32_t(best << mt.qsh[q]);
-                        atomicMax(a.score_rng + int64_t(mt.qid[q]) * kCntStride + kRngThr, uint32_t(T) ^ 0x80000000u);
-                    }
+                // the bound update's inputs (below), read before the unit's
+                // TMEM stage and ring slot are released: lane i takes query
+                // wq + 4 i
+                const int q = wq + 4 * lane;
+                if (lane < kTcQMax / 4 && q < qn && cnt[q] >= bound_min) {
+                    bq_go = true;
+                    bq_id = mt.qid[q];
+                    bq_thr = mt.thr[q];
+                    bq_base = mt.qbase[q];
+                    bq_sh = mt.qsh[q];
                 }
             }
             if (gt < kTcQMax) E.cnt[(it + 1) & 1][gt] = 0;  // the counts of this group's next unit
             tc_fence_before();
             named_barrier(1 + g, 128);  // every read of TMEM and of meta[m] is done
             if (gt == 0) mbar_arrive(&acc_empty[g]);
+            // then raise the bound of each query that gained at least
+            // bound_min keys in the unit: the highest bin edge with at least k
+            // written keys at or above it, from the query's bins at or above
+            // its bound's bin (lane l reads bins 32 l .. 32 l + 31)
+            constexpr int kPer = kTcBins / 32;
+            for (unsigned go = __ballot_sync(0xffffffffu, bq_go); go; go &= go - 1) {
+                const int i = __ffs(int(go)) - 1;
+                const int qid = __shfl_sync(0xffffffffu, bq_id, i);
+                const uint32_t thr = __shfl_sync(0xffffffffu, bq_thr, i);
+                const int32_t qbase = __shfl_sync(0xffffffffu, bq_base, i);
+                const int qsh = __shfl_sync(0xffffffffu, bq_sh, i);
+                const uint4* gh = reinterpret_cast<const uint4*>(a.qhist + int64_t(qid) * kTcBins) + lane * (kPer / 4);
+                const int tb = thr ? ((int32_t(thr ^ 0x80000000u) - qbase) >> qsh) : 0;
+                uint32_t gv[kPer], tot = 0;
+                const bool mine = kPer * lane + kPer - 1 >= tb;
+#pragma unroll
+                for (int r = 0; r < kPer / 4; ++r) {
+                    const uint4 x = mine ? __ldcg(gh + r) : make_uint4(0, 0, 0, 0);
+                    gv[4 * r] = x.x;
+                    gv[4 * r + 1] = x.y;
+                    gv[4 * r + 2] = x.z;
+                    gv[4 * r + 3] = x.w;
+                }
+#pragma unroll
+                for (int r = 0; r < kPer; ++r) tot += gv[r];
+                uint32_t incl = tot;  // suffix sum over lanes >= this one
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+                    if (lane + off < 32) incl += o;
+                }
+                uint32_t run = incl - tot, best = 0;  // keys in bins above this lane's
+#pragma unroll
+                for (int r = kPer - 1; r >= 0; --r) {
+                    run += gv[r];
+                    if (best == 0 && run >= uint32_t(a.k)) best = uint32_t(kPer * lane + r);
+                }
+                best = __reduce_max_sync(0xffffffffu, best);
+                if (lane == 0 && best > 0) {
+                    const int32_t T = qbase + int32_t(best << qsh);
+                    atomicMax(a.score_rng + int64_t(qid) * kCntStride + kRngThr, uint32_t(T) ^ 0x80000000u);
+                }
+            }
             if (gt == 0) TC_ACC(12 + (g & 1), e1);
         }
     }
